@@ -1,0 +1,255 @@
+"""fp64 CPU oracle of the smoothed-INT8-QK / FP8-PV attention forward.
+
+TEST INFRASTRUCTURE ONLY: the test-suite, the smoke check and the CPU-baseline
+leg of ``bench.py`` may import this package; the CUDA product path never does.
+It shares no code with the CUDA path.  The arithmetic lives in
+``sage_oracle.c`` (plain C, fp64, OpenMP over rows); this module compiles it
+with gcc, loads it with ctypes and marshals numpy arrays.
+
+Method sources (page title and section):
+  * "SageAttention2: Efficient Attention with Thorough Outlier Smoothing and
+    Per-thread INT4 Quantization" (arXiv 2411.10958), abstract -- Q/K smoothing,
+    fine-grained Q/K quantization, FP8 (P~, V), two-level PV accumulation.
+  * pith.science verdict on arXiv 2505.21136 (SageAttention2++), fields
+    key_machinery and core_discovery -- per-channel delta_V = |max V| / Vr,
+    P range Pr, the Pr x Vr <= 2047/2 bound of the FP16-accumulator variant.
+
+Parity status of each function is stated in its docstring; the pins live in
+``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sage_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libsage_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+TILE = 128
+
+
+def build(force: bool = False) -> str:
+    """Compile sage_oracle.c into oracle/_build/libsage_oracle.so (gcc, OpenMP)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+           "-ffp-contract=off", "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("n_q", ctypes.c_int), ("n_kv", ctypes.c_int), ("d", ctypes.c_int),
+                ("g_q", ctypes.c_int), ("g_k", ctypes.c_int),
+                ("smooth_q", ctypes.c_int), ("smooth_k", ctypes.c_int),
+                ("quant_qk", ctypes.c_int), ("quant_p", ctypes.c_int), ("quant_v", ctypes.c_int),
+                ("p_range", ctypes.c_double), ("v_range", ctypes.c_double),
+                ("sm_scale", ctypes.c_double), ("causal", ctypes.c_int)]
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            lib.oracle_e4m3_from_f32.argtypes = [ctypes.c_float]
+            lib.oracle_e4m3_from_f32.restype = ctypes.c_uint8
+            lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+            lib.oracle_e4m3_to_f64.restype = ctypes.c_double
+            lib.oracle_int8_code.argtypes = [ctypes.c_float, ctypes.c_float]
+            lib.oracle_int8_code.restype = ctypes.c_int8
+            lib.oracle_int8_scale.argtypes = [ctypes.c_float]
+            lib.oracle_int8_scale.restype = ctypes.c_float
+            lib.oracle_prepass.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 15
+            lib.oracle_prepass.restype = ctypes.c_int
+            lib.oracle_attn.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 9 + [ctypes.c_int, P, P, P]
+            lib.oracle_attn.restype = ctypes.c_int
+            lib.oracle_ref_attn.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double, ctypes.c_int, P, P, P, P]
+            lib.oracle_ref_attn.restype = ctypes.c_int
+            lib.oracle_num_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+# ---------------------------------------------------------------------------
+# Codecs
+# ---------------------------------------------------------------------------
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 (e4m3fn) code of each value, rounded to fp32 first; RNE, saturating to +-448.
+
+    Pinned against torch.float8_e4m3fn on every value it does not saturate, and
+    by decoding all 256 codes against the format's definition."""
+    lib = _load()
+    xs = np.asarray(x, dtype=np.float32).ravel()
+    out = np.fromiter((lib.oracle_e4m3_from_f32(float(v)) for v in xs), dtype=np.uint8, count=xs.size)
+    return out.reshape(np.shape(x))
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    lib = _load()
+    cs = np.asarray(codes, dtype=np.uint8).ravel()
+    out = np.fromiter((lib.oracle_e4m3_to_f64(int(c)) for c in cs), dtype=np.float64, count=cs.size)
+    return out.reshape(np.shape(codes))
+
+
+def int8_code(xs, delta) -> np.ndarray:
+    """INT8 code: round-half-even of the fp32 quotient xs / delta, clamped to +-127."""
+    lib = _load()
+    xs = np.asarray(xs, dtype=np.float32).ravel()
+    ds = np.broadcast_to(np.asarray(delta, dtype=np.float32), xs.shape).ravel()
+    return np.fromiter((lib.oracle_int8_code(float(a), float(b)) for a, b in zip(xs, ds)),
+                       dtype=np.int8, count=xs.size)
+
+
+def int8_scale(amax: float) -> float:
+    return float(_load().oracle_int8_scale(float(amax)))
+
+
+# ---------------------------------------------------------------------------
+# Granularities (group sizes in rows of Q / keys of K); any divisor of 128 works.
+# ---------------------------------------------------------------------------
+GRANULARITY = {
+    "per_block": (128, 128),
+    "per_warp": (32, 128),
+    "per_threadgroup": (32, 16),
+}
+
+
+def _cfg(n_q, n_kv, d, g_q, g_k, smooth_q, smooth_k, quant, p_range, v_range, sm_scale, causal):
+    qqk, qp, qv = quant
+    return _Cfg(n_q, n_kv, d, g_q, g_k, int(smooth_q), int(smooth_k), int(qqk), int(qp), int(qv),
+                float(p_range), float(v_range), float(sm_scale), int(causal))
+
+
+def prepass_head(q, k, v, *, g_q=32, g_k=16, smooth_q=True, smooth_k=True,
+                 quant=(1, 1, 1), p_range=448.0, v_range=448.0):
+    """Smoothing + quantization of one head.  q: [Nq, d], k, v: [Nkv, d] (any float dtype,
+    converted to fp64 exactly).  Returns a dict of the pre-pass tensors (see sage_oracle.c)."""
+    lib = _load()
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    nq, d = q.shape
+    nk = k.shape[0]
+    tq = -(-nq // TILE)
+    nq_pad, nk_pad = tq * TILE, -(-nk // TILE) * TILE
+    cfg = _cfg(nq, nk, d, g_q, g_k, smooth_q, smooth_k, quant, p_range, v_range, 1.0, 0)
+    r = dict(
+        qbar=np.zeros((tq, d), np.float32), kbar=np.zeros((d,), np.float32),
+        q_code=np.zeros((nq_pad, d), np.int8), q_hat=np.zeros((nq_pad, d), np.float64),
+        dq_row=np.zeros((nq_pad,), np.float32),
+        k_code=np.zeros((nk_pad, d), np.int8), k_hat=np.zeros((nk_pad, d), np.float64),
+        dk_key=np.zeros((nk_pad,), np.float32), k_s=np.zeros((max(nk, 1), d), np.float64),
+        v_code=np.zeros((max(nk, 1), d), np.uint8), v_hat=np.zeros((max(nk, 1), d), np.float64),
+        dv=np.zeros((d,), np.float32),
+    )
+    rc = lib.oracle_prepass(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v),
+                            _ptr(r["qbar"]), _ptr(r["kbar"]),
+                            _ptr(r["q_code"]), _ptr(r["q_hat"]), _ptr(r["dq_row"]),
+                            _ptr(r["k_code"]), _ptr(r["k_hat"]), _ptr(r["dk_key"]), _ptr(r["k_s"]),
+                            _ptr(r["v_code"]), _ptr(r["v_hat"]), _ptr(r["dv"]))
+    if rc != 0:
+        raise ValueError("oracle_prepass failed with code %d" % rc)
+    r["k_s"] = r["k_s"][:nk]
+    r["v_code"] = r["v_code"][:nk]
+    r["v_hat"] = r["v_hat"][:nk]
+    r["cfg"] = dict(n_q=nq, n_kv=nk, d=d, g_q=g_q, g_k=g_k, smooth_q=smooth_q, smooth_k=smooth_k,
+                    quant=tuple(quant), p_range=p_range, v_range=v_range)
+    return r
+
+
+def delta_s(pre, t: int) -> np.ndarray:
+    """Q-smoothing bias of Q block t over all keys: dS[t, j] = qbar_t . (K[j] - kbar), fp64."""
+    return pre["k_s"] @ pre["qbar"][t].astype(np.float64)
+
+
+def attn_head(pre, *, causal=False, sm_scale=None, qblocks=None, return_stats=False):
+    """Attention of one head from ``prepass_head`` output.  Returns O [Nq, d] fp64; rows of
+    Q blocks not listed in ``qblocks`` are left 0."""
+    lib = _load()
+    c = pre["cfg"]
+    nq, nk, d = c["n_q"], c["n_kv"], c["d"]
+    if sm_scale is None or sm_scale <= 0:
+        sm_scale = 1.0 / np.sqrt(d)
+    tq = -(-nq // TILE)
+    blocks = np.arange(tq, dtype=np.int32) if qblocks is None else np.ascontiguousarray(qblocks, dtype=np.int32)
+    cfg = _cfg(nq, nk, d, c["g_q"], c["g_k"], c["smooth_q"], c["smooth_k"], c["quant"],
+               c["p_range"], c["v_range"], sm_scale, causal)
+    o = np.zeros((max(nq, 1), d), np.float64)
+    rl = np.zeros((max(nq, 1),), np.float64)
+    rm = np.full((max(nq, 1),), -np.inf, np.float64)
+    k_s = np.ascontiguousarray(pre["k_s"]) if nk > 0 else np.zeros((1, d))
+    v_hat = np.ascontiguousarray(pre["v_hat"]) if nk > 0 else np.zeros((1, d))
+    rc = lib.oracle_attn(ctypes.byref(cfg), _ptr(pre["qbar"]), _ptr(pre["q_hat"]), _ptr(pre["dq_row"]),
+                         _ptr(pre["k_hat"]), _ptr(pre["dk_key"]), _ptr(k_s),
+                         _ptr(v_hat), _ptr(pre["dv"]), _ptr(blocks), int(blocks.size),
+                         _ptr(o), _ptr(rl), _ptr(rm))
+    if rc != 0:
+        raise ValueError("oracle_attn failed with code %d" % rc)
+    o, rl, rm = o[:nq], rl[:nq], rm[:nq]
+    if return_stats:
+        return o, rl, rm
+    return o
+
+
+def sage_attention(q, k, v, *, causal=False, sm_scale=None, granularity="per_threadgroup",
+                   smooth_q=True, smooth_k=True, quant=(1, 1, 1), p_range=448.0, v_range=448.0,
+                   heads=None, qblocks=None):
+    """Whole quantized attention forward on [B, H, N, d] arrays (head-major).
+
+    ``heads``: optional list of (b, h) to compute (others stay 0); ``qblocks``: optional
+    list of Q block indices to compute within each head.  Returns O fp64 [B, H, Nq, d]."""
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    B, H, nq, d = q.shape
+    g_q, g_k = GRANULARITY[granularity] if isinstance(granularity, str) else granularity
+    o = np.zeros((B, H, nq, d), np.float64)
+    hs = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    for b, h in hs:
+        pre = prepass_head(q[b, h], k[b, h], v[b, h], g_q=g_q, g_k=g_k, smooth_q=smooth_q,
+                           smooth_k=smooth_k, quant=quant, p_range=p_range, v_range=v_range)
+        o[b, h] = attn_head(pre, causal=causal, sm_scale=sm_scale, qblocks=qblocks)
+    return o
+
+
+def reference_attention(q, k, v, *, causal=False, sm_scale=None, heads=None):
+    """Textbook full-precision attention in fp64 (two-pass softmax), [B, H, N, d]."""
+    lib = _load()
+    q = np.asarray(q)
+    B, H, nq, d = q.shape
+    nk = np.asarray(k).shape[2]
+    if sm_scale is None or sm_scale <= 0:
+        sm_scale = 1.0 / np.sqrt(d)
+    o = np.zeros((B, H, nq, d), np.float64)
+    hs = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    for b, h in hs:
+        qq = np.ascontiguousarray(q[b, h], dtype=np.float64)
+        kk = np.ascontiguousarray(np.asarray(k)[b, h], dtype=np.float64)
+        vv = np.ascontiguousarray(np.asarray(v)[b, h], dtype=np.float64)
+        oo = np.zeros((max(nq, 1), d), np.float64)
+        lib.oracle_ref_attn(nq, nk, d, float(sm_scale), int(causal), _ptr(qq), _ptr(kk), _ptr(vv), _ptr(oo))
+        o[b, h] = oo[:nq]
+    return o
