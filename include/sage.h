@@ -1,0 +1,185 @@
+/*
+ * sage.h -- C ABI of libsage_b200.so: the smoothed-INT8-QK / FP8-PV quantized
+ * attention forward (the SageAttention2 / SageAttention2++ method) on NVIDIA
+ * B200 (sm_100a).
+ *
+ * What is computed (per batch b, head h; Q [N_q, d], K and V [N_kv, d]):
+ *   1. K smoothing: K_s = K - mean over the N_kv valid tokens of K.
+ *      ("SageAttention2" arXiv 2411.10958, abstract: outlier smoothing;
+ *       zhaifeiyue.github.io notes on 2411.10958: fine-grained quantization + smoothing.)
+ *   2. Q smoothing: for each 128-row Q block t, qbar_t = mean of its valid rows,
+ *      Q_s = Q - qbar_t, and the bias dS[t, j] = qbar_t . K[j] is added back to the
+ *      scores.  (2411.10958 abstract: "a method to smooth Q".)  Using K instead of
+ *      K_s in dS changes every score of a row by the same constant, which softmax
+ *      ignores.
+ *   3. INT8 quantization of Q_s and K_s per group (g_q consecutive rows of a Q
+ *      block, g_k consecutive keys of a 128-key tile): delta = amax / 127 (fp32),
+ *      code = clamp(round-half-even(x / delta), -127, 127).
+ *   4. V per channel: delta_V[c] = max_j |V[j, c]| / Vr, V8 = E4M3(V / delta_V).
+ *      (pith.science verdict on arXiv 2505.21136, key_machinery.)
+ *   5. S = delta_Q(i) delta_K(j) (Q_int . K_int) + dS, computed as an exact INT32
+ *      tensor-core product; tiled online softmax over 128-key tiles with an exact
+ *      rescale whenever a row maximum grows; P~ = exp(x - m) scaled by Pr and rounded
+ *      to E4M3 (static scale 1 / Pr, since P~ <= 1); O += P8 . V8 on FP8 tensor cores
+ *      with FP32 accumulation in tensor memory.
+ *   6. O = acc / Pr * delta_V[c] / l, with l the sum of the unquantized P~; a row
+ *      that sees no key is 0.  Rounded to the input dtype (round to nearest even).
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are plain CUDA device addresses; `stream` is a cudaStream_t
+ *     (NULL = legacy default stream).  All work is enqueued on `stream`; nothing
+ *     synchronizes except sage_get_device_status.
+ *   - Tensors: dtype SAGE_DTYPE_F16 / SAGE_DTYPE_BF16; layout SAGE_LAYOUT_HND is a
+ *     contiguous [B, H, N, d] array, SAGE_LAYOUT_NHD a contiguous [B, N, H, d] array.
+ *     Q, K, V and O share dtype and layout.  Base addresses must be 16-byte aligned.
+ *   - d is 64 or 128.  Heads are multi-head (H queries heads = H key/value heads).
+ *   - The caller owns all memory, including the workspace; the library allocates
+ *     nothing and keeps no state between calls.  The workspace must be at least
+ *     sage_workspace_bytes(...) bytes, 1024-byte aligned, and its first 256 bytes
+ *     (the device status block) must be zero before first use.
+ *   - Argument errors return a status synchronously and enqueue nothing.  A launch
+ *     failure returns SAGE_ERR_CUDA.  A device-side wait that runs out (about one
+ *     second) makes the kernel stop early and record SAGE_ERR_TIMEOUT in the status
+ *     block, read with sage_get_device_status.
+ *   - B * H == 0 or N_q == 0 is a no-op returning SAGE_OK.  N_kv == 0 writes O = 0.
+ */
+#ifndef SAGE_B200_H
+#define SAGE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define SAGE_API
+#else
+#define SAGE_API __attribute__((visibility("default")))
+#endif
+
+typedef enum {
+    SAGE_OK = 0,
+    SAGE_ERR_INVALID_ARG = 1,  /* null pointer, bad size or enum                  */
+    SAGE_ERR_UNSUPPORTED = 2,  /* valid but not supported: d, alignment, size cap  */
+    SAGE_ERR_WORKSPACE = 3,    /* workspace smaller than sage_workspace_bytes      */
+    SAGE_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed              */
+    SAGE_ERR_TIMEOUT = 5       /* a device-side bounded wait ran out               */
+} sage_status_t;
+
+typedef enum { SAGE_LAYOUT_HND = 0, SAGE_LAYOUT_NHD = 1 } sage_layout_t;
+typedef enum { SAGE_DTYPE_F16 = 0, SAGE_DTYPE_BF16 = 1 } sage_dtype_t;
+
+/* INT8 group sizes (g_q rows of Q, g_k keys of K).  The pages name the
+ * granularities per block (SageAttention, "INT8 per-block") and per thread
+ * (SageAttention2, thread-level); tcgen05 has no per-thread operand fragments, so
+ * the finest mode groups 32 rows (one tensor-memory lane quadrant) and 16 keys. */
+typedef enum {
+    SAGE_QK_PER_BLOCK = 0,        /* g_q = 128, g_k = 128 */
+    SAGE_QK_PER_WARP = 1,         /* g_q = 32,  g_k = 128 */
+    SAGE_QK_PER_THREADGROUP = 2   /* g_q = 32,  g_k = 16  (default) */
+} sage_qk_gran_t;
+
+typedef struct {
+    int32_t gran;      /* sage_qk_gran_t                                        */
+    int32_t smooth_q;  /* 1: subtract per-block Q mean and add dS back          */
+    int32_t smooth_k;  /* 1: subtract per-head K mean                           */
+    float p_range;     /* Pr, (0, 448]; 448 = full E4M3 range (default)         */
+    float v_range;     /* Vr, (0, 448]; 448 (SageAttention2 default)            */
+} sage_quant_mode_t;
+/* A NULL mode pointer means {SAGE_QK_PER_THREADGROUP, 1, 1, 448, 448}. */
+
+/* Bytes of workspace for one problem size (any dtype/layout).  0 on bad sizes. */
+SAGE_API size_t sage_workspace_bytes(int B, int H, int n_q, int n_kv, int d);
+
+/* Steps 1-3 (and the dS bias) for Q and K into the workspace.
+ * q: [B,H,n_q,d] or [B,n_q,H,d]; k: [B,H,n_kv,d] or [B,n_kv,H,d]. */
+SAGE_API sage_status_t sage_quant_qk(const void *q, const void *k, int dtype, int layout,
+                                     int B, int H, int n_q, int n_kv, int d,
+                                     const sage_quant_mode_t *mode,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/* Step 4 for V into the workspace (n_q only sizes the workspace regions). */
+SAGE_API sage_status_t sage_quant_v(const void *v, int dtype, int layout,
+                                    int B, int H, int n_q, int n_kv, int d,
+                                    const sage_quant_mode_t *mode,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* Steps 5-6 from a workspace filled by sage_quant_qk and sage_quant_v with the same
+ * sizes and mode.  o: output, same dtype/layout as the inputs were.
+ * sm_scale <= 0 means 1/sqrt(d).  causal: key j is visible to query i iff
+ * j <= i + n_kv - n_q (bottom-right aligned). */
+SAGE_API sage_status_t sage_attn_fwd_prequant(void *o, int dtype, int layout,
+                                              int B, int H, int n_q, int n_kv, int d,
+                                              int causal, float sm_scale,
+                                              const sage_quant_mode_t *mode,
+                                              const void *workspace, size_t workspace_bytes,
+                                              void *stream);
+
+/* The whole forward: quant_qk + quant_v + attn_fwd_prequant, enqueued on `stream`. */
+SAGE_API sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *o,
+                                     int dtype, int layout, int B, int H, int n_q, int n_kv,
+                                     int d, int causal, float sm_scale,
+                                     const sage_quant_mode_t *mode,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronizes `stream`, copies the workspace status block to the host and clears
+ * it.  *code receives SAGE_OK or the first device-side error (SAGE_ERR_TIMEOUT);
+ * *site an id of the wait that ran out (0 if none).  Returns SAGE_ERR_CUDA if the
+ * copy fails. */
+SAGE_API sage_status_t sage_get_device_status(void *workspace, void *stream, int *code, int *site);
+
+/* ---- workspace views (for tests and tools; all offsets in bytes) -------------
+ * The workspace holds, per (b, h) = bh in [0, B*H), with Tq = ceil(n_q/128),
+ * Tk = ceil(n_kv/128), nq_pad = 128 Tq, nk_pad = 128 Tk:
+ *   SAGE_WS_Q8    int8  [BH][nq_pad][d]          Q codes (pad rows 0)
+ *   SAGE_WS_K8    int8  [BH][nk_pad][d]          K codes (pad rows 0)
+ *   SAGE_WS_VT8   e4m3  [BH][d][nk_pad]          V codes, transposed (pad 0)
+ *   SAGE_WS_DQ    fp32  [BH][nq_pad]             delta_Q of each row's group
+ *   SAGE_WS_DK    fp32  [BH][nk_pad/16]          delta_K of each 16-key run
+ *   SAGE_WS_DV    fp32  [BH][d]                  delta_V per channel
+ *   SAGE_WS_QBAR  fp32  [BH][Tq][d]              Q block means
+ *   SAGE_WS_KBAR  fp32  [BH][d]                  K token mean
+ *   SAGE_WS_DS    fp32  [BH][Tq][nk_pad]         dS = qbar_t . K[j] (causally
+ *                                                invisible entries left unwritten)
+ */
+enum {
+    SAGE_WS_Q8 = 0, SAGE_WS_K8 = 1, SAGE_WS_VT8 = 2, SAGE_WS_DQ = 3, SAGE_WS_DK = 4,
+    SAGE_WS_DV = 5, SAGE_WS_QBAR = 6, SAGE_WS_KBAR = 7, SAGE_WS_DS = 8, SAGE_WS_NUM_VIEWS = 9
+};
+/* Byte offset of view `which` inside the workspace, or -1 for bad arguments. */
+SAGE_API int64_t sage_workspace_offset(int B, int H, int n_q, int n_kv, int d, int which);
+
+/* ---- diagnostics (no counterpart on the pages' API) ---------------------------
+ * INT32 scores of one (bh, Q tile, KV tile) straight from tensor memory, computed
+ * by the same descriptors and tcgen05.mma kind::i8 issue as the attention kernel,
+ * from a workspace filled by sage_quant_qk.  s_out: device int32 [128][128],
+ * row = query row within the tile, column = key within the tile. */
+SAGE_API sage_status_t sage_debug_qk_tile(const void *workspace, int B, int H, int n_q, int n_kv,
+                                          int d, int bh, int q_tile, int kv_tile,
+                                          int32_t *s_out, void *stream);
+
+/* O = sum over n_tiles of P_t . V_t on the FP8 path of the attention kernel (the
+ * same shared-memory layout, descriptors and tcgen05.mma kind::f8f6f4 issue, one
+ * FP32 tensor-memory accumulator).  p: device E4M3 [n_tiles][128][128] (row,
+ * key); vt: device E4M3 [n_tiles][d][128] (channel, key); o: device fp32
+ * [128][d].  Used to check the accumulation precision of the FP8 tensor core. */
+SAGE_API sage_status_t sage_debug_pv_accumulate(const uint8_t *p, const uint8_t *vt, int n_tiles,
+                                                int d, float *o, void *stream);
+
+/* Runs the attention kernel with one deliberately missing producer signal so that
+ * the consumer's bounded wait must run out; the kernel records SAGE_ERR_TIMEOUT in
+ * the status block and exits without hanging.  Arguments as sage_attn_fwd_prequant. */
+SAGE_API sage_status_t sage_debug_attn_fault_inject(void *o, int dtype, int layout, int B, int H,
+                                                    int n_q, int n_kv, int d, int causal,
+                                                    const void *workspace, size_t workspace_bytes,
+                                                    void *stream);
+
+/* Library build identification string (static storage). */
+SAGE_API const char *sage_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SAGE_B200_H */

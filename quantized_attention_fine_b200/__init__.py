@@ -1,0 +1,297 @@
+"""Smoothed-INT8-QK / FP8-PV quantized attention forward for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libsage_b200.so`` (declared in
+``include/sage.h``).  Every step of the computation runs in the library's CUDA
+kernels; this module only marshals arguments: torch tensors supply device memory
+and the current CUDA stream.  There is no CPU fallback: if the library is missing
+every call raises.
+
+    import torch, quantized_attention_fine_b200 as sage
+    o = sage.attn_fwd(q, k, v, causal=True)          # q, k, v: [B, H, N, d] bf16/fp16
+
+Method: "SageAttention2" (arXiv 2411.10958) with the per-channel FP8 V scaling and
+P range of SageAttention2++ (arXiv 2505.21136); see include/sage.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+__all__ = [
+    "QuantMode", "Workspace", "workspace_bytes", "make_workspace", "quant_qk", "quant_v", "attn_fwd_prequant",
+    "attn_fwd", "get_device_status", "workspace_view", "debug_qk_tile", "debug_pv_accumulate",
+    "debug_fault_inject", "library_path", "load_library", "SageError", "GRANULARITIES",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libsage_b200.so")
+_lock = threading.Lock()
+_lib = None
+
+SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_WORKSPACE, SAGE_ERR_CUDA, SAGE_ERR_TIMEOUT = range(6)
+_ERR_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED", 3: "SAGE_ERR_WORKSPACE",
+              4: "SAGE_ERR_CUDA", 5: "SAGE_ERR_TIMEOUT"}
+GRANULARITIES = {"per_block": 0, "per_warp": 1, "per_threadgroup": 2}
+_LAYOUTS = {"HND": 0, "NHD": 1}
+WS_VIEWS = {"q8": 0, "k8": 1, "vt8": 2, "dq": 3, "dk": 4, "dv": 5, "qbar": 6, "kbar": 7, "ds": 8}
+WS_ALIGN = 1024
+
+
+class SageError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__("%s failed: %s (%d)" % (what, _ERR_NAMES.get(code, "?"), code))
+        self.code = code
+
+
+class QuantMode(ctypes.Structure):
+    """Mirror of sage_quant_mode_t."""
+    _fields_ = [("gran", ctypes.c_int32), ("smooth_q", ctypes.c_int32), ("smooth_k", ctypes.c_int32),
+                ("p_range", ctypes.c_float), ("v_range", ctypes.c_float)]
+
+    @classmethod
+    def make(cls, granularity="per_threadgroup", smooth_q=True, smooth_k=True, p_range=448.0, v_range=448.0):
+        g = GRANULARITIES[granularity] if isinstance(granularity, str) else int(granularity)
+        return cls(g, int(bool(smooth_q)), int(bool(smooth_k)), float(p_range), float(v_range))
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libsage_b200.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError("libsage_b200.so is not built (run `python -m quantized_attention_fine_b200._build`); "
+                               "there is no fallback implementation")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        QM = ctypes.POINTER(QuantMode)
+        lib.sage_workspace_bytes.argtypes = [I] * 5
+        lib.sage_workspace_bytes.restype = S
+        lib.sage_workspace_offset.argtypes = [I] * 6
+        lib.sage_workspace_offset.restype = ctypes.c_int64
+        lib.sage_quant_qk.argtypes = [P, P, I, I, I, I, I, I, I, QM, P, S, P]
+        lib.sage_quant_v.argtypes = [P, I, I, I, I, I, I, I, QM, P, S, P]
+        lib.sage_attn_fwd_prequant.argtypes = [P, I, I, I, I, I, I, I, I, F, QM, P, S, P]
+        lib.sage_attn_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, F, QM, P, S, P]
+        lib.sage_get_device_status.argtypes = [P, P, ctypes.POINTER(I), ctypes.POINTER(I)]
+        lib.sage_debug_qk_tile.argtypes = [P, I, I, I, I, I, I, I, I, P, P]
+        lib.sage_debug_pv_accumulate.argtypes = [P, P, I, I, P, P]
+        lib.sage_debug_attn_fault_inject.argtypes = [P, I, I, I, I, I, I, I, I, P, S, P]
+        lib.sage_version.restype = ctypes.c_char_p
+        for fn in ("sage_quant_qk", "sage_quant_v", "sage_attn_fwd_prequant", "sage_attn_fwd",
+                   "sage_get_device_status", "sage_debug_qk_tile", "sage_debug_pv_accumulate",
+                   "sage_debug_attn_fault_inject"):
+            getattr(lib, fn).restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def _check(code: int, what: str):
+    if code != SAGE_OK:
+        raise SageError(code, what)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return 1
+    if t.dtype == torch.float16:
+        return 0
+    raise TypeError("q, k, v must be bfloat16 or float16, got %s" % t.dtype)
+
+
+def _shape(q, k, layout):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D")
+    if layout == "HND":
+        B, H, n_q, d = q.shape
+        n_kv = k.shape[2]
+        if k.shape[0] != B or k.shape[1] != H or k.shape[3] != d:
+            raise ValueError("k shape %s does not match q %s" % (tuple(k.shape), tuple(q.shape)))
+    elif layout == "NHD":
+        B, n_q, H, d = q.shape
+        n_kv = k.shape[1]
+        if k.shape[0] != B or k.shape[2] != H or k.shape[3] != d:
+            raise ValueError("k shape %s does not match q %s" % (tuple(k.shape), tuple(q.shape)))
+    else:
+        raise ValueError("layout must be 'HND' or 'NHD'")
+    return int(B), int(H), int(n_q), int(n_kv), int(d)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def workspace_bytes(B, H, n_q, n_kv, d) -> int:
+    return int(load_library().sage_workspace_bytes(B, H, n_q, n_kv, d))
+
+
+class Workspace:
+    """Caller-owned device workspace: a zeroed uint8 tensor with a 1024-byte aligned window."""
+
+    def __init__(self, B, H, n_q, n_kv, d, device=None):
+        torch = _torch()
+        self.dims = (int(B), int(H), int(n_q), int(n_kv), int(d))
+        self.nbytes = workspace_bytes(*self.dims)
+        if self.nbytes == 0:
+            raise SageError(SAGE_ERR_UNSUPPORTED, "sage_workspace_bytes")
+        self.tensor = torch.zeros(self.nbytes + WS_ALIGN, dtype=torch.uint8, device=device or "cuda")
+        base = self.tensor.data_ptr()
+        self.offset = (-base) % WS_ALIGN
+        self.ptr = base + self.offset
+
+    def fits(self, B, H, n_q, n_kv, d) -> bool:
+        return self.dims == (int(B), int(H), int(n_q), int(n_kv), int(d))
+
+    def view(self, which: str):
+        """Typed view of a workspace region (see include/sage.h, SAGE_WS_*)."""
+        torch = _torch()
+        B, H, n_q, n_kv, d = self.dims
+        off = int(load_library().sage_workspace_offset(B, H, n_q, n_kv, d, WS_VIEWS[which]))
+        BH, Tq = B * H, -(-n_q // 128)
+        nq_pad, nk_pad = Tq * 128, -(-n_kv // 128) * 128
+        shapes = {"q8": ((BH, nq_pad, d), torch.int8), "k8": ((BH, nk_pad, d), torch.int8),
+                  "vt8": ((BH, d, nk_pad), torch.uint8), "dq": ((BH, nq_pad), torch.float32),
+                  "dk": ((BH, nk_pad // 16), torch.float32), "dv": ((BH, d), torch.float32),
+                  "qbar": ((BH, Tq, d), torch.float32), "kbar": ((BH, d), torch.float32),
+                  "ds": ((BH, Tq, nk_pad), torch.float32)}
+        shp, dt = shapes[which]
+        n = math.prod(shp) * torch.tensor([], dtype=dt).element_size()
+        start = self.offset + off
+        return self.tensor[start:start + n].view(dt).view(shp)
+
+
+def make_workspace(B, H, n_q, n_kv, d, device=None) -> Workspace:
+    return Workspace(B, H, n_q, n_kv, d, device)
+
+
+def _ws_for(ws, B, H, n_q, n_kv, d, device):
+    if ws is None:
+        return Workspace(B, H, n_q, n_kv, d, device)
+    if not ws.fits(B, H, n_q, n_kv, d):
+        raise ValueError("workspace was made for %s, not %s" % (ws.dims, (B, H, n_q, n_kv, d)))
+    return ws
+
+
+def quant_qk(q, k, *, layout="HND", mode=None, workspace=None, stream=None) -> Workspace:
+    B, H, n_q, n_kv, d = _shape(q, k, layout)
+    ws = _ws_for(workspace, B, H, n_q, n_kv, d, q.device)
+    mode = mode or QuantMode.make()
+    _check(load_library().sage_quant_qk(_ptr(q), _ptr(k), _dtype_code(q), _LAYOUTS[layout], B, H, n_q, n_kv, d,
+                                        ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
+                                        _stream_handle(stream)), "sage_quant_qk")
+    return ws
+
+
+def quant_v(v, *, n_q, layout="HND", mode=None, workspace=None, stream=None) -> Workspace:
+    if layout == "HND":
+        B, H, n_kv, d = v.shape
+    else:
+        B, n_kv, H, d = v.shape
+    ws = _ws_for(workspace, B, H, n_q, n_kv, d, v.device)
+    mode = mode or QuantMode.make()
+    _check(load_library().sage_quant_v(_ptr(v), _dtype_code(v), _LAYOUTS[layout], B, H, n_q, n_kv, d,
+                                       ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
+                                       _stream_handle(stream)), "sage_quant_v")
+    return ws
+
+
+def attn_fwd_prequant(workspace: Workspace, *, dtype, layout="HND", causal=False, sm_scale=None, mode=None,
+                      out=None, stream=None):
+    torch = _torch()
+    B, H, n_q, n_kv, d = workspace.dims
+    if out is None:
+        shape = (B, H, n_q, d) if layout == "HND" else (B, n_q, H, d)
+        out = torch.empty(shape, dtype=dtype, device=workspace.tensor.device)
+    mode = mode or QuantMode.make()
+    _check(load_library().sage_attn_fwd_prequant(_ptr(out), _dtype_code(out), _LAYOUTS[layout], B, H, n_q, n_kv, d,
+                                                 int(bool(causal)), float(sm_scale or 0.0), ctypes.byref(mode),
+                                                 ctypes.c_void_p(workspace.ptr), workspace.nbytes,
+                                                 _stream_handle(stream)), "sage_attn_fwd_prequant")
+    return out
+
+
+def attn_fwd(q, k, v, *, causal=False, sm_scale=None, layout="HND", granularity="per_threadgroup",
+             smooth_q=True, smooth_k=True, p_range=448.0, v_range=448.0, out=None, workspace=None, stream=None):
+    """O = quantized attention of q, k, v (pre-pass + fused kernel, enqueued on the current stream)."""
+    torch = _torch()
+    B, H, n_q, n_kv, d = _shape(q, k, layout)
+    if v.shape != k.shape:
+        raise ValueError("v shape %s must equal k shape %s" % (tuple(v.shape), tuple(k.shape)))
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share a dtype")
+    ws = _ws_for(workspace, B, H, n_q, n_kv, d, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    mode = QuantMode.make(granularity, smooth_q, smooth_k, p_range, v_range)
+    _check(load_library().sage_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), _LAYOUTS[layout],
+                                        B, H, n_q, n_kv, d, int(bool(causal)), float(sm_scale or 0.0),
+                                        ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
+                                        _stream_handle(stream)), "sage_attn_fwd")
+    return out
+
+
+def get_device_status(workspace: Workspace, stream=None):
+    """(code, site) of the first device-side error since the last call; clears it."""
+    code, site = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load_library().sage_get_device_status(ctypes.c_void_p(workspace.ptr), _stream_handle(stream),
+                                                 ctypes.byref(code), ctypes.byref(site)), "sage_get_device_status")
+    return code.value, site.value
+
+
+def workspace_view(workspace: Workspace, which: str):
+    return workspace.view(which)
+
+
+def debug_qk_tile(workspace: Workspace, bh: int, q_tile: int, kv_tile: int, stream=None):
+    """INT32 S tile [128, 128] read back from tensor memory (diagnostic)."""
+    torch = _torch()
+    B, H, n_q, n_kv, d = workspace.dims
+    out = torch.empty((128, 128), dtype=torch.int32, device=workspace.tensor.device)
+    _check(load_library().sage_debug_qk_tile(ctypes.c_void_p(workspace.ptr), B, H, n_q, n_kv, d, bh, q_tile,
+                                             kv_tile, _ptr(out), _stream_handle(stream)), "sage_debug_qk_tile")
+    return out
+
+
+def debug_pv_accumulate(p_codes, vt_codes, stream=None):
+    """sum_t P_t . V_t with FP32 tensor-memory accumulation (diagnostic).
+    p_codes: uint8 [T, 128, 128] E4M3; vt_codes: uint8 [T, d, 128] E4M3.  Returns fp32 [128, d]."""
+    torch = _torch()
+    T, d = int(p_codes.shape[0]), int(vt_codes.shape[1])
+    out = torch.empty((128, d), dtype=torch.float32, device=p_codes.device)
+    _check(load_library().sage_debug_pv_accumulate(_ptr(p_codes), _ptr(vt_codes), T, d, _ptr(out),
+                                                   _stream_handle(stream)), "sage_debug_pv_accumulate")
+    return out
+
+
+def debug_fault_inject(workspace: Workspace, out, *, layout="HND", causal=False, stream=None):
+    """Run the attention kernel with one producer signal withheld (the bounded wait must run out)."""
+    B, H, n_q, n_kv, d = workspace.dims
+    _check(load_library().sage_debug_attn_fault_inject(_ptr(out), _dtype_code(out), _LAYOUTS[layout], B, H, n_q,
+                                                       n_kv, d, int(bool(causal)), ctypes.c_void_p(workspace.ptr),
+                                                       workspace.nbytes, _stream_handle(stream)),
+           "sage_debug_attn_fault_inject")

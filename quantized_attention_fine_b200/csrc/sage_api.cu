@@ -1,0 +1,326 @@
+// sage_api.cu -- the C ABI of libsage_b200 (declared in include/sage.h):
+// argument validation, workspace layout, TMA tensor-map encoding and kernel
+// launches on the caller's stream.  No memory is allocated here.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/sage.h"
+#include "sage_internal.h"
+
+using namespace sage;
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode;
+}
+
+struct Mode {
+    int g_q, g_k, smooth_q, smooth_k;
+    float p_range, v_range;
+};
+
+sage_status_t read_mode(const sage_quant_mode_t *m, Mode *out) {
+    sage_quant_mode_t d = {SAGE_QK_PER_THREADGROUP, 1, 1, 448.f, 448.f};
+    if (m) d = *m;
+    switch (d.gran) {
+        case SAGE_QK_PER_BLOCK: out->g_q = 128; out->g_k = 128; break;
+        case SAGE_QK_PER_WARP: out->g_q = 32; out->g_k = 128; break;
+        case SAGE_QK_PER_THREADGROUP: out->g_q = 32; out->g_k = 16; break;
+        default: return SAGE_ERR_INVALID_ARG;
+    }
+    if (!(d.p_range > 0.f && d.p_range <= 448.f) || !(d.v_range > 0.f && d.v_range <= 448.f))
+        return SAGE_ERR_INVALID_ARG;
+    out->smooth_q = d.smooth_q ? 1 : 0;
+    out->smooth_k = d.smooth_k ? 1 : 0;
+    out->p_range = d.p_range;
+    out->v_range = d.v_range;
+    return SAGE_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Sizes shared by all entry points.  Returns SAGE_OK and fills *s, or an error.
+sage_status_t check_sizes(int B, int H, int n_q, int n_kv, int d, Shape *s) {
+    if (B < 0 || H < 0 || n_q < 0 || n_kv < 0) return SAGE_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
+    // TMA coordinates are 32-bit signed: BH * padded length must stay below 2^31.
+    const int64_t bh = (int64_t)B * H;
+    const int64_t nq_pad = ((int64_t)n_q + kTile - 1) / kTile * kTile;
+    const int64_t nk_pad = ((int64_t)n_kv + kTile - 1) / kTile * kTile;
+    if (bh * nq_pad >= (1ll << 31) || bh * nk_pad >= (1ll << 31) || bh * d >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
+    if ((bh * ((nq_pad + kTile - 1) / kTile)) >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
+    *s = make_shape(B, H, n_q, n_kv, d);
+    return SAGE_OK;
+}
+
+sage_status_t check_ws(const Shape &s, const void *ws, size_t ws_bytes) {
+    if (!ws) return SAGE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)) != 0) return SAGE_ERR_UNSUPPORTED;
+    if (ws_bytes < ws_layout(s).total) return SAGE_ERR_WORKSPACE;
+    return SAGE_OK;
+}
+
+bool encode_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+               uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Tensor maps of the Q codes, K codes ([rows][d] bytes, 128-row boxes) and the
+// transposed V codes ([BH*d][nk_pad] bytes, d x 128 boxes).
+bool make_maps(const Shape &s, const uint8_t *ws, CUtensorMap *tq, CUtensorMap *tk, CUtensorMap *tv) {
+    const WsLayout L = ws_layout(s);
+    const CUtensorMapSwizzle swz_qk = (s.d == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const uint64_t d = (uint64_t)s.d;
+    if (tq && !encode_2d(tq, ws + L.q8, d, (uint64_t)s.BH * s.nq_pad, d, (uint32_t)d, kTile, swz_qk)) return false;
+    if (tk && !encode_2d(tk, ws + L.k8, d, (uint64_t)s.BH * s.nk_pad, d, (uint32_t)d, kTile, swz_qk)) return false;
+    if (tv && !encode_2d(tv, ws + L.vt8, (uint64_t)s.nk_pad, (uint64_t)s.BH * d, (uint64_t)s.nk_pad, kTile,
+                         (uint32_t)d, CU_TENSOR_MAP_SWIZZLE_128B))
+        return false;
+    return true;
+}
+
+sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype, int layout, const Shape &s,
+                          const Mode &m, uint8_t *ws, int ds_t_skip, int causal_off, cudaStream_t stream) {
+    PrepassArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.bf16 = (dtype == SAGE_DTYPE_BF16);
+    a.sq = make_strides(layout, s.H, s.n_q, s.d);
+    a.skv = make_strides(layout, s.H, s.n_kv, s.d);
+    a.shape = s;
+    a.g_q = m.g_q;
+    a.g_k = m.g_k;
+    a.smooth_q = m.smooth_q;
+    a.smooth_k = m.smooth_k;
+    a.v_range = m.v_range;
+    a.ws = ws;
+    a.L = ws_layout(s);
+    return launch_prepass(a, ds_t_skip, causal_off, stream) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+sage_status_t run_attention(void *o, int dtype, int layout, const Shape &s, int causal, float sm_scale,
+                            const Mode &m, const uint8_t *ws, int fault_inject, cudaStream_t stream) {
+    CUtensorMap tq, tk, tv;
+    if (!make_maps(s, ws, &tq, &tk, &tv)) return SAGE_ERR_CUDA;
+    const WsLayout L = ws_layout(s);
+    const Strides so = make_strides(layout, s.H, s.n_q, s.d);
+    AttnParams p;
+    p.dq = reinterpret_cast<const float *>(ws + L.dq);
+    p.dk = reinterpret_cast<const float *>(ws + L.dk);
+    p.dv = reinterpret_cast<const float *>(ws + L.dv);
+    p.ds = reinterpret_cast<const float *>(ws + L.ds);
+    p.o = o;
+    p.so_b = so.b;
+    p.so_h = so.h;
+    p.so_n = so.n;
+    p.H = s.H;
+    p.n_q = s.n_q;
+    p.n_kv = s.n_kv;
+    p.Tq = s.Tq;
+    p.Tk = s.Tk;
+    p.nq_pad = s.nq_pad;
+    p.nk_pad = s.nk_pad;
+    p.BH = s.BH;
+    p.causal = causal ? 1 : 0;
+    p.use_ds = m.smooth_q;
+    p.out_bf16 = (dtype == SAGE_DTYPE_BF16);
+    const float scale = (sm_scale > 0.f) ? sm_scale : 1.0f / sqrtf((float)s.d);
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.log2_pr = log2f(m.p_range);
+    p.status = reinterpret_cast<int *>(const_cast<uint8_t *>(ws) + L.status);
+    p.fault_inject = fault_inject;
+    return launch_attention(tq, tk, tv, p, s.d, stream) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+sage_status_t check_common(int dtype, int layout) {
+    if (dtype != SAGE_DTYPE_F16 && dtype != SAGE_DTYPE_BF16) return SAGE_ERR_INVALID_ARG;
+    if (layout != SAGE_LAYOUT_HND && layout != SAGE_LAYOUT_NHD) return SAGE_ERR_INVALID_ARG;
+    return SAGE_OK;
+}
+
+#define SAGE_TRY(expr)                     \
+    do {                                   \
+        sage_status_t _st = (expr);        \
+        if (_st != SAGE_OK) return _st;    \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t sage_workspace_bytes(int B, int H, int n_q, int n_kv, int d) {
+    Shape s;
+    if (check_sizes(B, H, n_q, n_kv, d, &s) != SAGE_OK) return 0;
+    return ws_layout(s).total;
+}
+
+int64_t sage_workspace_offset(int B, int H, int n_q, int n_kv, int d, int which) {
+    Shape s;
+    if (check_sizes(B, H, n_q, n_kv, d, &s) != SAGE_OK) return -1;
+    const WsLayout L = ws_layout(s);
+    switch (which) {
+        case SAGE_WS_Q8: return (int64_t)L.q8;
+        case SAGE_WS_K8: return (int64_t)L.k8;
+        case SAGE_WS_VT8: return (int64_t)L.vt8;
+        case SAGE_WS_DQ: return (int64_t)L.dq;
+        case SAGE_WS_DK: return (int64_t)L.dk;
+        case SAGE_WS_DV: return (int64_t)L.dv;
+        case SAGE_WS_QBAR: return (int64_t)L.qbar;
+        case SAGE_WS_KBAR: return (int64_t)L.kbar;
+        case SAGE_WS_DS: return (int64_t)L.ds;
+        default: return -1;
+    }
+}
+
+sage_status_t sage_quant_qk(const void *q, const void *k, int dtype, int layout, int B, int H, int n_q, int n_kv,
+                            int d, const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+    Shape s;
+    Mode m;
+    SAGE_TRY(check_common(dtype, layout));
+    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    SAGE_TRY(read_mode(mode, &m));
+    if (s.BH == 0 || (n_q == 0 && n_kv == 0)) return SAGE_OK;
+    if ((n_q > 0 && !q) || (n_kv > 0 && !k)) return SAGE_ERR_INVALID_ARG;
+    if ((q && !aligned16(q)) || (k && !aligned16(k))) return SAGE_ERR_UNSUPPORTED;
+    SAGE_TRY(check_ws(s, workspace, workspace_bytes));
+    return run_prepass(n_q > 0 ? q : nullptr, n_kv > 0 ? k : nullptr, nullptr, dtype, layout, s, m,
+                       static_cast<uint8_t *>(workspace), 0, 0, static_cast<cudaStream_t>(stream));
+}
+
+sage_status_t sage_quant_v(const void *v, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
+                           const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes, void *stream) {
+    Shape s;
+    Mode m;
+    SAGE_TRY(check_common(dtype, layout));
+    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    SAGE_TRY(read_mode(mode, &m));
+    if (s.BH == 0 || n_kv == 0) return SAGE_OK;
+    if (!v) return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(v)) return SAGE_ERR_UNSUPPORTED;
+    SAGE_TRY(check_ws(s, workspace, workspace_bytes));
+    return run_prepass(nullptr, nullptr, v, dtype, layout, s, m, static_cast<uint8_t *>(workspace), 0, 0,
+                       static_cast<cudaStream_t>(stream));
+}
+
+sage_status_t sage_attn_fwd_prequant(void *o, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
+                                     int causal, float sm_scale, const sage_quant_mode_t *mode,
+                                     const void *workspace, size_t workspace_bytes, void *stream) {
+    Shape s;
+    Mode m;
+    SAGE_TRY(check_common(dtype, layout));
+    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    SAGE_TRY(read_mode(mode, &m));
+    if (s.BH == 0 || n_q == 0) return SAGE_OK;
+    if (!o) return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(o)) return SAGE_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n_kv == 0)
+        return cudaMemsetAsync(o, 0, (size_t)s.BH * n_q * d * 2, st) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+    SAGE_TRY(check_ws(s, workspace, workspace_bytes));
+    return run_attention(o, dtype, layout, s, causal, sm_scale, m, static_cast<const uint8_t *>(workspace), 0, st);
+}
+
+sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *o, int dtype, int layout, int B,
+                            int H, int n_q, int n_kv, int d, int causal, float sm_scale,
+                            const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes, void *stream) {
+    Shape s;
+    Mode m;
+    SAGE_TRY(check_common(dtype, layout));
+    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    SAGE_TRY(read_mode(mode, &m));
+    if (s.BH == 0 || n_q == 0) return SAGE_OK;
+    if (!q || !o || (n_kv > 0 && (!k || !v))) return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(o) || (k && !aligned16(k)) || (v && !aligned16(v))) return SAGE_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n_kv == 0)
+        return cudaMemsetAsync(o, 0, (size_t)s.BH * n_q * d * 2, st) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+    SAGE_TRY(check_ws(s, workspace, workspace_bytes));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    SAGE_TRY(run_prepass(q, k, v, dtype, layout, s, m, ws, causal ? 1 : 0, n_kv - n_q, st));
+    return run_attention(o, dtype, layout, s, causal, sm_scale, m, ws, 0, st);
+}
+
+sage_status_t sage_get_device_status(void *workspace, void *stream, int *code, int *site) {
+    if (!workspace || !code || !site) return SAGE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int host[2] = {0, 0};
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SAGE_ERR_CUDA;
+    if (cudaMemcpyAsync(host, workspace, sizeof(host), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SAGE_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(host), st) != cudaSuccess) return SAGE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SAGE_ERR_CUDA;
+    *code = host[0];
+    *site = host[1];
+    return SAGE_OK;
+}
+
+sage_status_t sage_debug_qk_tile(const void *workspace, int B, int H, int n_q, int n_kv, int d, int bh, int q_tile,
+                                 int kv_tile, int32_t *s_out, void *stream) {
+    Shape s;
+    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    if (!workspace || !s_out || s.BH == 0 || n_q == 0 || n_kv == 0) return SAGE_ERR_INVALID_ARG;
+    if (bh < 0 || bh >= s.BH || q_tile < 0 || q_tile >= s.Tq || kv_tile < 0 || kv_tile >= s.Tk)
+        return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(s_out)) return SAGE_ERR_UNSUPPORTED;
+    const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+    CUtensorMap tq, tk;
+    if (!make_maps(s, ws, &tq, &tk, nullptr)) return SAGE_ERR_CUDA;
+    int *status = reinterpret_cast<int *>(const_cast<uint8_t *>(ws) + ws_layout(s).status);
+    return launch_debug_qk_tile(tq, tk, d, bh * s.nq_pad + q_tile * kTile, bh * s.nk_pad + kv_tile * kTile, s_out,
+                                status, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SAGE_OK
+               : SAGE_ERR_CUDA;
+}
+
+sage_status_t sage_debug_pv_accumulate(const uint8_t *p, const uint8_t *vt, int n_tiles, int d, float *o,
+                                       void *stream) {
+    if (!p || !vt || !o || n_tiles < 1) return SAGE_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
+    if (!aligned16(p) || !aligned16(vt) || !aligned16(o)) return SAGE_ERR_UNSUPPORTED;
+    return launch_debug_pv(p, vt, n_tiles, d, o, nullptr, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SAGE_OK
+               : SAGE_ERR_CUDA;
+}
+
+sage_status_t sage_debug_attn_fault_inject(void *o, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
+                                           int causal, const void *workspace, size_t workspace_bytes,
+                                           void *stream) {
+    Shape s;
+    Mode m;
+    SAGE_TRY(check_common(dtype, layout));
+    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    SAGE_TRY(read_mode(nullptr, &m));
+    if (!o || s.BH == 0 || n_q == 0 || n_kv == 0) return SAGE_ERR_INVALID_ARG;
+    SAGE_TRY(check_ws(s, workspace, workspace_bytes));
+    return run_attention(o, dtype, layout, s, causal, 0.f, m, static_cast<const uint8_t *>(workspace), 1,
+                         static_cast<cudaStream_t>(stream));
+}
+
+const char *sage_version(void) { return "libsage_b200 1.0 (sm_100a; tcgen05 INT8 QK / FP8 PV)"; }
+
+}  // extern "C"

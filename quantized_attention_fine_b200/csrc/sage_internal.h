@@ -1,0 +1,110 @@
+// sage_internal.h -- host-side shared definitions of libsage_b200: workspace
+// layout, kernel parameter blocks and launcher prototypes.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sage {
+
+constexpr int kTile = 128;        // Q block rows = KV tile keys (part of the numerics)
+constexpr int kKeyRun = 16;       // delta_K is stored once per 16 keys
+constexpr int kStatChunk = 512;   // tokens per CTA of the K-mean / V-amax pass
+constexpr size_t kWsAlign = 1024;
+constexpr size_t kStatusBytes = 256;
+
+struct Shape {
+    int B, H, n_q, n_kv, d;
+    int BH, Tq, Tk, nq_pad, nk_pad, n_chunks;
+};
+
+inline Shape make_shape(int B, int H, int n_q, int n_kv, int d) {
+    Shape s;
+    s.B = B; s.H = H; s.n_q = n_q; s.n_kv = n_kv; s.d = d;
+    s.BH = B * H;
+    s.Tq = (n_q + kTile - 1) / kTile;
+    s.Tk = (n_kv + kTile - 1) / kTile;
+    s.nq_pad = s.Tq * kTile;
+    s.nk_pad = s.Tk * kTile;
+    s.n_chunks = (n_kv + kStatChunk - 1) / kStatChunk;
+    if (s.n_chunks < 1) s.n_chunks = 1;
+    return s;
+}
+
+// Byte offsets of every workspace region.
+struct WsLayout {
+    size_t status, q8, k8, vt8, dq, dk, dv, qbar, kbar, ds, ksum_part, vmax_part, total;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline WsLayout ws_layout(const Shape &s) {
+    WsLayout w;
+    const size_t BH = (size_t)s.BH, d = (size_t)s.d;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, kWsAlign); return o; };
+    w.status = take(kStatusBytes);
+    w.q8 = take(BH * s.nq_pad * d);
+    w.k8 = take(BH * s.nk_pad * d);
+    w.vt8 = take(BH * d * s.nk_pad);
+    w.dq = take(BH * s.nq_pad * 4);
+    w.dk = take(BH * (s.nk_pad / kKeyRun) * 4);
+    w.dv = take(BH * d * 4);
+    w.qbar = take(BH * s.Tq * d * 4);
+    w.kbar = take(BH * d * 4);
+    w.ds = take(BH * s.Tq * (size_t)s.nk_pad * 4);
+    w.ksum_part = take(BH * s.n_chunks * d * 8);
+    w.vmax_part = take(BH * s.n_chunks * d * 4);
+    w.total = off;
+    return w;
+}
+
+// Element strides of a [B, H, N, d] (HND) or [B, N, H, d] (NHD) tensor.
+struct Strides {
+    int64_t b, h, n;
+};
+inline Strides make_strides(int layout, int H, int N, int d) {
+    Strides st;
+    if (layout == 0) { st.b = (int64_t)H * N * d; st.h = (int64_t)N * d; st.n = d; }
+    else { st.b = (int64_t)N * H * d; st.h = d; st.n = (int64_t)H * d; }
+    return st;
+}
+
+struct PrepassArgs {
+    const void *q, *k, *v;   // any may be null: that part is skipped
+    int bf16;
+    Strides sq, skv;
+    Shape shape;
+    int g_q, g_k, smooth_q, smooth_k;
+    float v_range;
+    uint8_t *ws;
+    WsLayout L;
+};
+
+struct AttnParams {
+    const float *dq, *dk, *dv, *ds;
+    void *o;
+    int64_t so_b, so_h, so_n;
+    int H, n_q, n_kv, Tq, Tk, nq_pad, nk_pad, BH;
+    int causal;
+    int use_ds;         // 0: Q smoothing off, dS not read
+    int out_bf16;
+    float scale_log2;   // sm_scale * log2(e)
+    float log2_pr;      // log2(Pr)
+    int *status;
+    int fault_inject;
+};
+
+// ds_t_skip: leave dS entries of Q blocks that can never see a tile unwritten
+// (causal attention, key j visible to query i iff j <= i + causal_off).
+cudaError_t launch_prepass(const PrepassArgs &a, int ds_t_skip, int causal_off, cudaStream_t stream);
+cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                             const AttnParams &p, int d, cudaStream_t stream);
+cudaError_t launch_debug_qk_tile(const CUtensorMap &tq, const CUtensorMap &tk, int d, int q_row0, int k_row0,
+                                 int32_t *s_out, int *status, cudaStream_t stream);
+cudaError_t launch_debug_pv(const uint8_t *p, const uint8_t *vt, int n_tiles, int d, float *o, int *status,
+                            cudaStream_t stream);
+cudaError_t launch_zero_output(void *o, size_t bytes, cudaStream_t stream);
+
+}  // namespace sage

@@ -1,0 +1,110 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+symbol include/sage.h declares, sizes its workspace consistently, and rejects bad
+arguments synchronously (before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import quantized_attention_fine_b200 as sage
+from quantized_attention_fine_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sage.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return sage.load_library()
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SAGE_API\s+[\w\s\*]+?\b(sage_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_symbols()
+    for required in ("sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd",
+                     "sage_attn_fwd_prequant", "sage_get_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in _declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_library_hides_internal_symbols(lib):
+    # only the C ABI is exported (built with -fvisibility=hidden)
+    for internal in ("_ZN4sage14launch_prepassERKNS_11PrepassArgsEiiP11CUstream_st", "launch_prepass"):
+        with pytest.raises(AttributeError):
+            getattr(lib, internal)
+
+
+def test_version_string(lib):
+    assert b"sm_100a" in lib.sage_version()
+
+
+@pytest.mark.parametrize("dims", [(1, 2, 256, 256, 64), (2, 16, 4096, 4096, 128), (1, 32, 32768, 32768, 128),
+                                  (2, 48, 17776, 17776, 64), (1, 1, 1, 1, 64), (3, 5, 200, 333, 128)])
+def test_workspace_layout_regions_are_aligned_and_disjoint(lib, dims):
+    B, H, nq, nk, d = dims
+    total = sage.workspace_bytes(*dims)
+    BH, Tq = B * H, -(-nq // 128)
+    nq_pad, nk_pad = Tq * 128, -(-nk // 128) * 128
+    sizes = {0: BH * nq_pad * d, 1: BH * nk_pad * d, 2: BH * d * nk_pad, 3: BH * nq_pad * 4,
+             4: BH * nk_pad // 16 * 4, 5: BH * d * 4, 6: BH * Tq * d * 4, 7: BH * d * 4, 8: BH * Tq * nk_pad * 4}
+    spans = []
+    for which, size in sizes.items():
+        off = lib.sage_workspace_offset(B, H, nq, nk, d, which)
+        assert off >= 256 and off % 1024 == 0
+        spans.append((off, off + size))
+    spans.sort()
+    for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+        assert a1 <= b0
+    assert spans[-1][1] <= total
+
+
+def test_workspace_bytes_rejects_bad_sizes(lib):
+    assert lib.sage_workspace_bytes(1, 1, 128, 128, 96) == 0      # d must be 64 or 128
+    assert lib.sage_workspace_bytes(-1, 1, 128, 128, 64) == 0
+    assert lib.sage_workspace_bytes(1 << 16, 1 << 10, 1 << 12, 128, 64) == 0   # beyond 32-bit TMA coordinates
+    assert lib.sage_workspace_offset(1, 1, 128, 128, 64, 99) == -1
+
+
+def test_argument_errors_return_synchronously(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced: validation fails first
+    # bad dtype / layout / d / null pointers
+    assert lib.sage_attn_fwd(fake, fake, fake, fake, 7, 0, 1, 1, 128, 128, 64, 0, 0.0, None, fake, 1 << 30, None) == 1
+    assert lib.sage_attn_fwd(fake, fake, fake, fake, 1, 3, 1, 1, 128, 128, 64, 0, 0.0, None, fake, 1 << 30, None) == 1
+    assert lib.sage_attn_fwd(fake, fake, fake, fake, 1, 0, 1, 1, 128, 128, 80, 0, 0.0, None, fake, 1 << 30, None) == 2
+    assert lib.sage_attn_fwd(None, fake, fake, fake, 1, 0, 1, 1, 128, 128, 64, 0, 0.0, None, fake, 1 << 30, None) == 1
+    # misaligned input
+    assert lib.sage_attn_fwd(P((1 << 20) + 2), fake, fake, fake, 1, 0, 1, 1, 128, 128, 64, 0, 0.0, None, fake,
+                             1 << 30, None) == 2
+    # workspace too small / misaligned
+    assert lib.sage_attn_fwd(fake, fake, fake, fake, 1, 0, 1, 1, 128, 128, 64, 0, 0.0, None, fake, 16, None) == 3
+    assert lib.sage_attn_fwd(fake, fake, fake, fake, 1, 0, 1, 1, 128, 128, 64, 0, 0.0, None, P((1 << 20) + 512),
+                             1 << 30, None) == 2
+    # bad quant modes
+    bad = sage.QuantMode(9, 1, 1, 448.0, 448.0)
+    assert lib.sage_quant_qk(fake, fake, 1, 0, 1, 1, 128, 128, 64, ctypes.byref(bad), fake, 1 << 30, None) == 1
+    bad = sage.QuantMode(2, 1, 1, 500.0, 448.0)
+    assert lib.sage_quant_v(fake, 1, 0, 1, 1, 128, 128, 64, ctypes.byref(bad), fake, 1 << 30, None) == 1
+    # empty problems are a successful no-op
+    assert lib.sage_attn_fwd(fake, fake, fake, fake, 1, 0, 0, 4, 128, 128, 64, 0, 0.0, None, None, 0, None) == 0
+    assert lib.sage_attn_fwd(fake, fake, fake, fake, 1, 0, 1, 4, 0, 128, 64, 0, 0.0, None, None, 0, None) == 0
+    # diagnostics validate their indices
+    assert lib.sage_debug_qk_tile(fake, 1, 1, 128, 128, 64, 1, 0, 0, fake, None) == 1
+    assert lib.sage_debug_pv_accumulate(fake, fake, 0, 64, fake, None) == 1
+
+
+def test_python_binding_has_no_fallback(monkeypatch, tmp_path):
+    monkeypatch.setattr(sage, "_LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(sage, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        sage.load_library()

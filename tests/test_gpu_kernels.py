@@ -1,0 +1,265 @@
+"""GPU parity of the CUDA path against the fp64 oracle, through the C ABI.
+
+Pre-pass: codes and scales bit-exact (the code decisions are IEEE fp32 on both
+sides).  INT32 QK^T tiles: bit-exact against int64 products of the GPU's own codes.
+FP8 PV: accumulation checked against exact sums.  Attention output: max-abs and
+cosine against the oracle, cosine against full-precision attention, on inputs that
+span several tiles with ragged tails, both head dims, dtypes and layouts.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_attention_fine_b200 as sage
+from quantized_attention_fine_b200 import workloads as wl
+
+from helpers import (O_COS_FULL, GRAN_OF, assert_close_to_oracle, cos, head_slices, oracle_head, to_np64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from quantized_attention_fine_b200 import _build
+    _build.build()
+    sage.load_library()
+
+
+def _inputs(name, B, H, nq, nk, d, causal, dtype=torch.bfloat16, recipe="image_dit", layout="HND", seed=None):
+    w = wl.custom(name, B, H, nq, nk, d, causal, dtype=dtype, recipe=recipe,
+                  seed=seed if seed is not None else (hash((B, H, nq, nk, d)) & 0xFFFF) + 5000)
+    q, k, v = wl.generate(w)
+    if layout == "NHD":
+        q, k, v = wl.to_nhd(q), wl.to_nhd(k), wl.to_nhd(v)
+    return w, q, k, v
+
+
+# ---------------------------------------------------------------------------
+# Pre-pass
+# ---------------------------------------------------------------------------
+PREPASS_CASES = [
+    # B, H, nq, nk, d, dtype, layout, granularity
+    (1, 2, 256, 256, 64, torch.float16, "HND", "per_threadgroup"),
+    (2, 3, 300, 520, 128, torch.bfloat16, "HND", "per_threadgroup"),
+    (1, 2, 520, 300, 64, torch.bfloat16, "NHD", "per_warp"),
+    (1, 1, 200, 130, 128, torch.float16, "NHD", "per_block"),
+]
+
+
+@pytest.mark.parametrize("B,H,nq,nk,d,dtype,layout,gran", PREPASS_CASES)
+def test_prepass_bit_exact(B, H, nq, nk, d, dtype, layout, gran):
+    _, q, k, v = _inputs("prepass", B, H, nq, nk, d, False, dtype=dtype, layout=layout)
+    mode = sage.QuantMode.make(gran)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    ws = sage.quant_qk(qd, kd, layout=layout, mode=mode)
+    sage.quant_v(vd, n_q=nq, layout=layout, mode=mode, workspace=ws)
+    torch.cuda.synchronize()
+    views = {n: ws.view(n).cpu() for n in sage.WS_VIEWS}
+    g_q, g_k = GRAN_OF[gran]
+    for b in range(B):
+        for h in range(H):
+            bh = b * H + h
+            qh, kh, vh = head_slices(q, k, v, b, h, layout)
+            pre = oracle.prepass_head(to_np64(qh), to_np64(kh), to_np64(vh), g_q=g_q, g_k=g_k)
+            assert np.array_equal(views["qbar"][bh].numpy(), pre["qbar"]), "qbar"
+            assert np.array_equal(views["kbar"][bh].numpy(), pre["kbar"]), "kbar"
+            assert np.array_equal(views["dq"][bh].numpy(), pre["dq_row"]), "delta_Q"
+            assert np.array_equal(views["dk"][bh].numpy(), pre["dk_key"][::16]), "delta_K"
+            assert np.array_equal(views["dv"][bh].numpy(), pre["dv"]), "delta_V"
+            assert np.array_equal(views["q8"][bh].numpy(), pre["q_code"]), "Q codes"
+            assert np.array_equal(views["k8"][bh].numpy(), pre["k_code"]), "K codes"
+            vt = views["vt8"][bh].numpy()
+            assert np.array_equal(vt[:, :nk].T, pre["v_code"]), "V codes"
+            assert not vt[:, nk:].any(), "V pad"
+            # dS = qbar_t . K[j] (raw K; differs from the oracle's qbar_t . K_s by a per-block constant)
+            ds = views["ds"][bh].numpy()[:, :nk].astype(np.float64)
+            ref = pre["qbar"].astype(np.float64) @ to_np64(kh).T
+            scale = np.abs(pre["qbar"]).astype(np.float64) @ np.abs(to_np64(kh)).T + 1e-30
+            assert np.max(np.abs(ds - ref) / scale) < 1e-5, "dS"
+            # the two dS readings differ by qbar_t . kbar for every key
+            diff = ref - np.stack([oracle.delta_s(pre, t) for t in range(ref.shape[0])])
+            assert np.max(np.abs(diff - diff[:, :1])) < 1e-9
+
+
+# ---------------------------------------------------------------------------
+# Tensor-core stages
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("d", [64, 128])
+def test_qk_tiles_bit_exact_int32(d):
+    B, H, nq, nk = 1, 2, 300, 400
+    _, q, k, v = _inputs("qk", B, H, nq, nk, d, False)
+    ws = sage.quant_qk(q.cuda(), k.cuda())
+    q8 = ws.view("q8").cpu().to(torch.int64)
+    k8 = ws.view("k8").cpu().to(torch.int64)
+    for bh, qt, kt in [(0, 0, 0), (1, 2, 3), (0, 1, 2), (1, 0, 1)]:
+        s = sage.debug_qk_tile(ws, bh, qt, kt).cpu().to(torch.int64)
+        ref = q8[bh, qt * 128:(qt + 1) * 128] @ k8[bh, kt * 128:(kt + 1) * 128].T
+        assert torch.equal(s, ref), "S tile (%d,%d,%d) differs in %d entries" % (bh, qt, kt, (s != ref).sum())
+    code, site = sage.get_device_status(ws)
+    assert code == 0
+
+
+def _e4m3(x):
+    return torch.as_tensor(x, dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp8_pv_random_tiles_match_exact_sum(d):
+    g = torch.Generator().manual_seed(d)
+    T = 3
+    p = torch.rand((T, 128, 128), generator=g) * 448
+    v = torch.randn((T, d, 128), generator=g) * 4
+    pc, vc = _e4m3(p), _e4m3(v)
+    pf = pc.view(torch.float8_e4m3fn).double()
+    vf = vc.view(torch.float8_e4m3fn).double()
+    exact = sum(pf[t] @ vf[t].T for t in range(T))
+    o = sage.debug_pv_accumulate(pc.cuda(), vc.cuda()).cpu().double()
+    bound = sum(pf[t].abs() @ vf[t].abs().T for t in range(T)) * (2.0 ** -22)
+    assert torch.all((o - exact).abs() <= bound + 1e-30)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp8_pv_accumulates_in_full_fp32(d):
+    """One product of 448 plus 127 products of 2^-8 per tile: exact in FP32 (needs 17
+    significant bits), lost by an accumulator with a 13-bit mantissa."""
+    T = 2
+    p = torch.zeros((T, 128, 128))
+    v = torch.zeros((T, d, 128))
+    p[:, :, 0] = 448.0
+    v[:, :, 0] = 1.0
+    p[:, :, 1:] = 2.0 ** -4
+    v[:, :, 1:] = 2.0 ** -4
+    o = sage.debug_pv_accumulate(_e4m3(p).cuda(), _e4m3(v).cuda()).cpu().double()
+    expect = T * (448.0 + 127 * 2.0 ** -8)
+    assert torch.all(o == expect), "accumulated %r, exact %r" % (o[0, 0].item(), expect)
+
+
+# ---------------------------------------------------------------------------
+# Attention output
+# ---------------------------------------------------------------------------
+ATTN_CASES = [
+    # name, B, H, nq, nk, d, causal, dtype, layout, granularity, recipe
+    ("tiny", 1, 2, 256, 256, 64, False, torch.float16, "HND", "per_threadgroup", "tiny"),
+    ("ragged_causal_d128", 1, 2, 600, 600, 128, True, torch.bfloat16, "HND", "per_threadgroup", "llm"),
+    ("kv_longer_d64_nhd", 2, 1, 300, 520, 64, False, torch.bfloat16, "NHD", "per_threadgroup", "video_dit"),
+    ("q_longer_causal_fp16", 1, 2, 520, 300, 128, True, torch.float16, "HND", "per_threadgroup", "image_dit"),
+    ("per_block", 1, 2, 384, 384, 128, False, torch.bfloat16, "HND", "per_block", "image_dit"),
+    ("per_warp_causal_d64", 1, 2, 333, 333, 64, True, torch.bfloat16, "NHD", "per_warp", "sweep"),
+    ("single_row", 1, 1, 1, 700, 128, False, torch.bfloat16, "HND", "per_threadgroup", "image_dit"),
+    ("single_key_causal", 1, 1, 130, 1, 64, True, torch.bfloat16, "HND", "per_threadgroup", "image_dit"),
+]
+
+
+@pytest.mark.parametrize("name,B,H,nq,nk,d,causal,dtype,layout,gran,recipe", ATTN_CASES, ids=[c[0] for c in ATTN_CASES])
+def test_attention_matches_oracle(name, B, H, nq, nk, d, causal, dtype, layout, gran, recipe):
+    if name == "tiny":
+        q, k, v = wl.generate(wl.TINY)
+    else:
+        _, q, k, v = _inputs(name, B, H, nq, nk, d, causal, dtype=dtype, recipe=recipe, layout=layout)
+    o = sage.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, layout=layout, granularity=gran).cpu()
+    assert o.dtype == dtype and o.shape == q.shape
+    for b in range(B):
+        for h in range(H):
+            qh, kh, vh = head_slices(q, k, v, b, h, layout)
+            og = head_slices(o, o, o, b, h, layout)[0]
+            _, oo = oracle_head(qh, kh, vh, causal=causal, granularity=gran)
+            assert_close_to_oracle(to_np64(og), oo, "%s b%d h%d" % (name, b, h))
+            ref = oracle.reference_attention(to_np64(qh)[None, None], to_np64(kh)[None, None],
+                                             to_np64(vh)[None, None], causal=causal)[0, 0]
+            if np.abs(ref).sum() > 0:
+                assert cos(to_np64(og), ref) >= O_COS_FULL
+
+
+def test_smoothing_off_and_sa2pp_ranges():
+    _, q, k, v = _inputs("modes", 1, 2, 300, 300, 128, False, recipe="image_dit")
+    for kw in (dict(smooth_q=False, smooth_k=False), dict(p_range=224.0, v_range=4.5), dict(smooth_q=False)):
+        o = sage.attn_fwd(q.cuda(), k.cuda(), v.cuda(), **kw).cpu()
+        for h in range(2):
+            _, oo = oracle_head(q[0, h], k[0, h], v[0, h], causal=False, **kw)
+            assert_close_to_oracle(to_np64(o[0, h]), oo, str(kw))
+
+
+def test_explicit_sm_scale():
+    _, q, k, v = _inputs("scale", 1, 1, 256, 256, 64, False)
+    o = sage.attn_fwd(q.cuda(), k.cuda(), v.cuda(), sm_scale=0.05).cpu()
+    _, oo = oracle_head(q[0, 0], k[0, 0], v[0, 0], causal=False, sm_scale=0.05)
+    assert_close_to_oracle(to_np64(o[0, 0]), oo, "sm_scale=0.05")
+
+
+def test_causal_rows_ignore_future_keys_bit_exact():
+    B, H, n, d, cut = 1, 2, 500, 128, 260
+    _, q, k, v = _inputs("causal", B, H, n, n, d, True, recipe="llm")
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    ws = sage.quant_qk(qd, kd)
+    sage.quant_v(vd, n_q=n, workspace=ws)
+    o1 = sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=True).clone()
+    g = torch.Generator(device="cuda").manual_seed(3)
+    k8, vt8 = ws.view("k8"), ws.view("vt8")
+    k8[:, cut:n] = torch.randint(-127, 128, k8[:, cut:n].shape, generator=g, device="cuda", dtype=torch.int8)
+    vt8[:, :, cut:n] = torch.randint(0, 0x7F, vt8[:, :, cut:n].shape, generator=g, device="cuda").to(torch.uint8)
+    o2 = sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1[:, :, :cut], o2[:, :, :cut])
+    assert not torch.equal(o1[:, :, cut:], o2[:, :, cut:])
+
+
+def test_prequant_path_equals_fused_call():
+    _, q, k, v = _inputs("prequant", 2, 2, 333, 333, 64, True, recipe="video_dit")
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o_full = sage.attn_fwd(qd, kd, vd, causal=True)
+    ws = sage.quant_qk(qd, kd)
+    sage.quant_v(vd, n_q=333, workspace=ws)
+    o_pre = sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o_full, o_pre)
+
+
+def test_repeated_calls_deterministic():
+    _, q, k, v = _inputs("det", 1, 4, 700, 700, 128, True, recipe="llm")
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    ws = sage.make_workspace(1, 4, 700, 700, 128)
+    a = sage.attn_fwd(qd, kd, vd, causal=True, workspace=ws).clone()
+    b = sage.attn_fwd(qd, kd, vd, causal=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_empty_and_keyless_inputs():
+    d = 64
+    q = torch.randn(1, 2, 100, d, dtype=torch.bfloat16, device="cuda")
+    k = torch.randn(1, 2, 0, d, dtype=torch.bfloat16, device="cuda")
+    o = torch.full_like(q, 7.0)
+    lib = sage.load_library()
+    ws = sage.make_workspace(1, 2, 100, 1, d)
+    rc = lib.sage_attn_fwd(ctypes.c_void_p(q.data_ptr()), None, None, ctypes.c_void_p(o.data_ptr()), 1, 0, 1, 2, 100,
+                           0, d, 0, 0.0, None, ctypes.c_void_p(ws.ptr), ws.nbytes,
+                           ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert rc == 0 and not o.float().abs().sum().item()
+    # B*H = 0 and N_q = 0: no-op
+    e = torch.empty(0, 2, 128, d, dtype=torch.bfloat16, device="cuda")
+    rc = lib.sage_attn_fwd(ctypes.c_void_p(e.data_ptr()), ctypes.c_void_p(e.data_ptr()), ctypes.c_void_p(e.data_ptr()),
+                           ctypes.c_void_p(e.data_ptr()), 1, 0, 0, 2, 128, 128, d, 0, 0.0, None, None, 0, None)
+    assert rc == 0
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    _, q, k, v = _inputs("fault", 1, 1, 128, 256, 64, False)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    ws = sage.quant_qk(qd, kd)
+    sage.quant_v(vd, n_q=128, workspace=ws)
+    assert sage.get_device_status(ws) == (0, 0)
+    out = torch.zeros_like(qd)
+    sage.debug_fault_inject(ws, out)
+    code, site = sage.get_device_status(ws)
+    assert code == sage.SAGE_ERR_TIMEOUT and site != 0
+    assert sage.get_device_status(ws) == (0, 0)        # read-and-clear
+    # the context is still usable and the normal path still matches the oracle
+    o = sage.attn_fwd_prequant(ws, dtype=q.dtype).cpu()
+    _, oo = oracle_head(q[0, 0], k[0, 0], v[0, 0], causal=False)
+    assert_close_to_oracle(to_np64(o[0, 0]), oo, "after timeout")
