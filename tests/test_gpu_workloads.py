@@ -1,0 +1,78 @@
+"""Parity at the full workload sizes, in the launch configuration bench.py times
+(sage_quant_qk + sage_quant_v + sage_attn_fwd_prequant on one workspace).
+
+The oracle cannot redo a whole 32K-token workload, so it recomputes sampled heads
+completely (pre-pass, bit-exact) and sampled Q blocks of them over the full KV range
+(attention output within tolerance); full-precision attention is evaluated on the
+same rows in numpy fp64.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_attention_fine_b200 as sage
+from quantized_attention_fine_b200 import workloads as wl
+
+from helpers import O_COS_FULL, assert_close_to_oracle, cos, rows_of_blocks, to_np64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from quantized_attention_fine_b200 import _build
+    _build.build()
+    sage.load_library()
+
+
+def _full_precision_rows(qh, kh, vh, rows, causal):
+    q = qh[rows]
+    x = (q @ kh.T) / np.sqrt(qh.shape[1])
+    if causal:
+        off = kh.shape[0] - qh.shape[0]
+        j = np.arange(kh.shape[0])[None, :]
+        x = np.where(j <= rows[:, None] + off, x, -np.inf)
+    m = x.max(1, keepdims=True)
+    p = np.exp(x - m)
+    return (p @ vh) / p.sum(1, keepdims=True)
+
+
+@pytest.mark.parametrize("name", ["image_dit", "llm_prefill", "video_dit"])
+def test_full_size_workload_sampled(name):
+    w = wl.WORKLOADS[name]
+    q, k, v = wl.generate(w)
+    dev = torch.device("cuda", 0)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    mode = sage.QuantMode.make()
+    ws = sage.make_workspace(w.B, w.H, w.N_q, w.N_kv, w.d, device=dev)
+    sage.quant_qk(qd, kd, mode=mode, workspace=ws)
+    sage.quant_v(vd, n_q=w.N_q, mode=mode, workspace=ws)
+    o = sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode)
+    assert sage.get_device_status(ws) == (0, 0)
+    tq = -(-w.N_q // 128)
+    heads = [(0, 0), (w.B - 1, w.H - 1)]
+    blocks = sorted({0, tq // 2, tq - 1})
+    views = {n: ws.view(n) for n in ("q8", "k8", "vt8", "dq", "dk", "dv", "qbar", "kbar")}
+    for b, h in heads:
+        bh = b * w.H + h
+        qh, kh, vh = to_np64(q[b, h]), to_np64(k[b, h]), to_np64(v[b, h])
+        pre = oracle.prepass_head(qh, kh, vh)
+        # the pre-pass of the sampled head, bit-exact
+        assert np.array_equal(views["qbar"][bh].cpu().numpy(), pre["qbar"])
+        assert np.array_equal(views["kbar"][bh].cpu().numpy(), pre["kbar"])
+        assert np.array_equal(views["dq"][bh].cpu().numpy(), pre["dq_row"])
+        assert np.array_equal(views["dk"][bh].cpu().numpy(), pre["dk_key"][::16])
+        assert np.array_equal(views["dv"][bh].cpu().numpy(), pre["dv"])
+        assert np.array_equal(views["q8"][bh].cpu().numpy(), pre["q_code"])
+        assert np.array_equal(views["k8"][bh].cpu().numpy(), pre["k_code"])
+        assert np.array_equal(views["vt8"][bh].cpu().numpy()[:, :w.N_kv].T, pre["v_code"])
+        # attention rows of the sampled Q blocks over the full KV range
+        oo = oracle.attn_head(pre, causal=w.causal, qblocks=blocks)
+        rows = rows_of_blocks(w.N_q, blocks)
+        og = to_np64(o[b, h].cpu())[rows]
+        assert_close_to_oracle(og, oo[rows], "%s head (%d,%d)" % (name, b, h))
+        ref = _full_precision_rows(qh, kh, vh, rows, w.causal)
+        assert cos(og, ref) >= O_COS_FULL, "%s: cos vs full precision %.5f" % (name, cos(og, ref))
