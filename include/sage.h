@@ -124,6 +124,27 @@ SAGE_API sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v
                                      const sage_quant_mode_t *mode,
                                      void *workspace, size_t workspace_bytes, void *stream);
 
+/* The whole forward, exactly as sage_attn_fwd, for callers that must not allocate
+ * device memory (for example a plugin whose host application owns every device
+ * allocation, or a serving loop where a cudaMalloc, which can synchronize the
+ * device, is not acceptable) and so cannot provide a workspace.  The pages have no
+ * counterpart of this entry point.
+ *   - Scratch: one 64 MiB device array inside the library, reserved on every GPU
+ *     the library is loaded on and held until the process exits.  Problems whose
+ *     sage_workspace_bytes(...) exceeds 64 MiB - 1 KiB are refused with
+ *     SAGE_ERR_WORKSPACE before anything is enqueued.
+ *   - Allocates nothing: no cudaMalloc / cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's device address; make that
+ *     first call before any stream capture.
+ *   - All calls on a device share the array, which keeps the previous call's
+ *     contents (the status block is cleared at the start of each call).  Calls
+ *     that overlap on the GPU (other streams, other host threads) race with each
+ *     other: serialize them.
+ *   - Arguments, layouts and errors otherwise as sage_attn_fwd. */
+SAGE_API sage_status_t sage_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *o, int dtype,
+                                             int layout, int B, int H, int n_q, int n_kv, int d, int causal,
+                                             float sm_scale, const sage_quant_mode_t *mode, void *stream);
+
 /* Synchronizes `stream`, copies the workspace status block to the host and clears
  * it.  *code receives SAGE_OK or the first device-side error (SAGE_ERR_TIMEOUT);
  * *site an id of the wait that ran out (0 if none).  Returns SAGE_ERR_CUDA if the

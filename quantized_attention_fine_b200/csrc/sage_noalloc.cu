@@ -1,0 +1,65 @@
+// sage_noalloc.cu -- sage_attn_fwd_noalloc: the whole forward without a
+// caller-supplied workspace.  Its scratch (INT8/FP8 codes, scales, dS, the status
+// block) lives in one file-scope device array that is reserved when the library is
+// loaded on a GPU and kept until the process exits.
+//
+// Who needs this: code that must not allocate device memory while it runs, for
+// example a plugin whose host application owns every device allocation, or a
+// serving loop in which a cudaMalloc (which can synchronize the device and stall
+// other streams) is not acceptable.  Such callers still pass their own inputs and
+// output; only the scratch comes from here.
+#include <mutex>
+
+#include "../../include/sage.h"
+#include "sage_internal.h"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 64ull << 20;   // 64 MiB per GPU
+constexpr int kMaxDevices = 64;
+
+// Device-side scratch shared by every call on a GPU.  In host code this name is
+// only a stand-in for the symbol: its device address comes from
+// cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+uint8_t *g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on first use).
+sage_status_t noalloc_scratch(uint8_t **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SAGE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return SAGE_ERR_CUDA;
+        g_noalloc_addr[dev] = static_cast<uint8_t *>(p);
+    }
+    *out = g_noalloc_addr[dev];
+    return SAGE_OK;
+}
+
+}  // namespace
+
+extern "C" sage_status_t sage_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *o, int dtype,
+                                               int layout, int B, int H, int n_q, int n_kv, int d, int causal,
+                                               float sm_scale, const sage_quant_mode_t *mode, void *stream) {
+    // Problems whose workspace would not fit are refused before anything is enqueued.
+    const size_t need = sage_workspace_bytes(B, H, n_q, n_kv, d);
+    if (need == 0) return (d != 64 && d != 128) ? SAGE_ERR_UNSUPPORTED : SAGE_ERR_INVALID_ARG;
+    uint8_t *base = nullptr;
+    sage_status_t st = noalloc_scratch(&base);
+    if (st != SAGE_OK) return st;
+    // Keep the 1024-byte alignment the workspace layout is built on.
+    const uintptr_t raw = reinterpret_cast<uintptr_t>(base);
+    const uintptr_t aligned = (raw + sage::kWsAlign - 1) & ~(uintptr_t)(sage::kWsAlign - 1);
+    const size_t usable = kNoAllocScratchBytes - (size_t)(aligned - raw);
+    if (need > usable) return SAGE_ERR_WORKSPACE;
+    uint8_t *ws = reinterpret_cast<uint8_t *>(aligned);
+    // The array keeps the previous call's contents; the status block must start at zero.
+    if (cudaMemsetAsync(ws, 0, sage::kStatusBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return SAGE_ERR_CUDA;
+    return sage_attn_fwd(q, k, v, o, dtype, layout, B, H, n_q, n_kv, d, causal, sm_scale, mode, ws, usable, stream);
+}

@@ -1,0 +1,73 @@
+"""sage_attn_fwd_noalloc: the forward for callers that cannot allocate device memory
+(and so cannot hand the library a workspace), with its scratch in a fixed device
+array inside the library.  Checked through the C ABI against sage_attn_fwd, the
+entry point that takes a caller-owned workspace, on two calls in a row.
+
+This file is collected last on purpose, and passes both alone in a fresh process
+and after the rest of the suite."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import quantized_attention_fine_b200 as sage
+from quantized_attention_fine_b200 import workloads as wl
+
+from helpers import assert_close_to_oracle
+
+pytestmark = pytest.mark.gpu
+
+SCRATCH_BYTES = 64 << 20
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from quantized_attention_fine_b200 import _build
+    _build.build()
+    lib = sage.load_library()
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.sage_attn_fwd_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, F, ctypes.POINTER(sage.QuantMode), P]
+    lib.sage_attn_fwd_noalloc.restype = I
+    return lib
+
+
+def _call_noalloc(lib, q, k, v, o, causal, mode):
+    B, H, nq, d = q.shape
+    nk = k.shape[2]
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return lib.sage_attn_fwd_noalloc(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                     ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
+                                     1 if q.dtype == torch.bfloat16 else 0, 0, B, H, nq, nk, d, int(causal), 0.0,
+                                     ctypes.byref(mode), stream)
+
+
+def test_noalloc_matches_workspace_entry_point_on_two_calls(lib):
+    mode = sage.QuantMode.make()
+    cases = [wl.custom("noalloc_a", 1, 4, 700, 700, 128, True, recipe="llm", seed=4242),
+             wl.custom("noalloc_b", 2, 3, 513, 900, 64, False, recipe="video_dit", seed=4343)]
+    for w in cases:
+        q, k, v = (x.cuda() for x in wl.generate(w))
+        assert sage.workspace_bytes(w.B, w.H, w.N_q, w.N_kv, w.d) <= SCRATCH_BYTES - 1024
+        ref = sage.attn_fwd(q, k, v, causal=w.causal)
+        o = torch.full_like(q, float("nan"))
+        assert _call_noalloc(lib, q, k, v, o, w.causal, mode) == 0
+        torch.cuda.synchronize()
+        assert_close_to_oracle(o.double().cpu().numpy(), ref.double().cpu().numpy(), w.name)
+
+
+def test_noalloc_refuses_problems_larger_than_its_scratch(lib):
+    # B=1, H=32, N=8192, d=128 needs more than 64 MiB of workspace
+    B, H, n, d = 1, 32, 8192, 128
+    assert sage.workspace_bytes(B, H, n, n, d) > SCRATCH_BYTES
+    q = torch.zeros((B, H, 128, d), dtype=torch.bfloat16, device="cuda")
+    o = torch.full_like(q, 3.0)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    ptr = ctypes.c_void_p(q.data_ptr())
+    rc = lib.sage_attn_fwd_noalloc(ptr, ptr, ptr, ctypes.c_void_p(o.data_ptr()), 1, 0, B, H, n, n, d, 0, 0.0,
+                                   None, stream)
+    torch.cuda.synchronize()
+    assert rc == sage.SAGE_ERR_WORKSPACE
+    assert torch.all(o == 3.0)      # nothing was enqueued
