@@ -8,14 +8,19 @@
 // Pr and rounded to E4M3; O += P8 . V8 on the FP8 tensor core, FP32 accumulation
 // in tensor memory; O = acc * delta_V / (Pr l).
 //
-// One CTA computes one 128-row Q tile of one head (192 threads):
-//   warps 0-3  softmax + epilogue; thread i owns query row i = tensor-memory lane i
-//   warp 4     TMA producer: Q tile once, then K / V^T tiles, dS and delta_K runs
-//              through a 3-stage shared-memory ring
-//   warp 5     tensor-memory allocation and single-thread tcgen05.mma issue
-// Tensor memory (512 columns): S double buffer (int32, columns 0-127 and 128-255),
-// O accumulator (fp32, columns 256 .. 256 + d).  QK^T of tile j + 1 runs on the
-// tensor core while the softmax warps work on tile j.
+// One CTA computes two 128-row Q tiles (A = 2u, B = 2u + 1) of one head, sharing
+// every K / V^T tile between them (384 threads, 12 warps):
+//   warps 0-3   softmax + epilogue of tile A (thread i owns row i = TMEM lane i)
+//   warps 4-7   softmax + epilogue of tile B
+//   warp 8      TMA producer: Q tiles once, then K, V^T, dS (per tile) and
+//               delta_K runs through a shared-memory ring
+//   warp 9      tensor-memory allocation and single-thread tcgen05.mma issue
+//   warps 10-11 idle (they only give the producer warpgroup its register share)
+// Tensor memory (512 columns): S_A 0-127, S_B 128-255 (int32), O_A 256.., O_B
+// 256 + d.. (fp32).  A softmax warpgroup releases its S buffer as soon as the
+// scores are in registers, so QK^T of the next key tile runs on the tensor core
+// while the current one is being exponentiated, and the two warpgroups alternate
+// on the tensor core (QK_A, QK_B, PV_A, PV_B per key tile).
 // Every wait is bounded: a wait that runs out records SAGE_ERR_TIMEOUT in the
 // status block, raises a CTA-wide abort flag that makes every role leave its loop,
 // drains the copies in flight, frees tensor memory and exits.
@@ -27,24 +32,34 @@
 
 namespace sage {
 
-constexpr int kStages = 3;
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;
 constexpr uint64_t kDrainNs = 50ull * 1000ull * 1000ull;
+// Register split (setmaxnreg): 384 threads launch with 168 registers each; the
+// producer warpgroup gives back to 40 so the two softmax warpgroups can hold 232:
+// 128 * 40 + 256 * 232 = 384 * 168.
+constexpr uint32_t kRegsProducer = 40;
+constexpr uint32_t kRegsSoftmax = 232;
 
 // Wait-site ids recorded with a timeout.
-enum { kSiteQ = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteS = 4, kSiteP = 5, kSiteO = 6, kSiteDebug = 9 };
+enum { kSiteQ = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteS = 4, kSiteP = 5, kSiteO = 6, kSiteSfree = 7, kSiteDebug = 9 };
+
+template <int D>
+struct AttnCfg {
+    static constexpr int kStages = (D == 128) ? 3 : 4;
+};
 
 template <int D>
 struct __align__(1024) AttnSmem {
-    uint8_t q[kTile * D];
-    uint8_t k[kStages][kTile * D];
-    uint8_t v[kStages][D * kTile];
-    uint8_t p[kTile * kTile];
-    float ds[kStages][kTile];
-    float dk[kStages][kTile / kKeyRun];
-    uint64_t bar_q, bar_full[kStages], bar_empty[kStages], bar_s[2], bar_p, bar_o, bar_drain;
+    static constexpr int ST = AttnCfg<D>::kStages;
+    uint8_t q[2][kTile * D];
+    uint8_t k[ST][kTile * D];
+    uint8_t v[ST][D * kTile];
+    uint8_t p[2][kTile * kTile];
+    float ds[ST][2][kTile];
+    float dk[ST][kTile / kKeyRun];
+    uint64_t bar_q, bar_full[ST], bar_empty[ST], bar_s[2], bar_sfree[2], bar_p[2], bar_o[2], bar_drain;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -109,52 +124,235 @@ __device__ __forceinline__ void store_row_chunk(void *dst, const float (&y)[32],
     for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Number of key tiles Q tile t sees (causal: key j visible to row i iff j <= i + off).
+__device__ __forceinline__ int kv_tiles_of(int t, int Tq, int Tk, int n_q, int off, int causal) {
+    if (t >= Tq) return 0;
+    if (!causal) return Tk;
+    const int last_key = min(t * kTile + kTile - 1, n_q - 1) + off;
+    return last_key < 0 ? 0 : min(Tk, last_key / kTile + 1);
+}
+
+// ---------------------------------------------------------------------------
+// Softmax + epilogue of one Q tile (128 threads, one query row each).
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &p, uint32_t tmem, int X, int t,
+                                             int n_tiles, int bh, int64_t o_base, volatile int *abort_flag) {
+    constexpr int ST = AttnCfg<D>::kStages;
+    const int wq = (threadIdx.x >> 5) & 3;
+    const int lane = threadIdx.x & 31;
+    const int r = wq * 32 + lane;
+    const int row = t * kTile + r;
+    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+    const uint32_t s_tmem = tmem + lane_base + (uint32_t)X * 128u;
+    const uint32_t o_tmem = tmem + lane_base + kTmemO + (uint32_t)X * D;
+    const int off = p.n_kv - p.n_q;
+    uint16_t *orow = static_cast<uint16_t *>(p.o) + o_base + (int64_t)row * p.so_n;
+
+    if (n_tiles == 0) {  // this tile's rows see no key: O = 0
+        if (row < p.n_q) {
+            uint4 *dst = reinterpret_cast<uint4 *>(orow);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+        }
+        return;
+    }
+
+    const float dq = p.dq[(size_t)bh * p.nq_pad + row];
+    const float c = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % ST;
+        if (!warp_wait(&sm.bar_s[X], it & 1, abort_flag, p.status, kSiteS)) { ok = false; break; }
+        if (!warp_wait(&sm.bar_full[s], (it / ST) & 1, abort_flag, p.status, kSiteFull)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sv[4][32];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(s_tmem + q4 * 32, sv[q4]);
+        tmem_wait_ld_regs(sv[0]);
+        reg_fence(sv[1]);
+        reg_fence(sv[2]);
+        reg_fence(sv[3]);
+        // scores are in registers: the S buffer may take the next QK^T
+        tc_fence_before();
+        mbar_arrive(&sm.bar_sfree[X]);
+
+        const float *ds = sm.ds[s][X];
+        const bool masked = (it * kTile + kTile > p.n_kv) || (p.causal && it * kTile + kTile - 1 > t * kTile + off);
+        // s = S * dQ dK + dS, in place over the score registers
+#pragma unroll
+        for (int g = 0; g < kTile / kKeyRun; ++g) {
+            const float a = dq * sm.dk[s][g];
+            const float2 a2 = make_float2(a, a);
+#pragma unroll
+            for (int j = g * kKeyRun; j < (g + 1) * kKeyRun; j += 4) {
+                uint32_t *w = &sv[j / 32][j % 32];
+                const float4 d4 = p.use_ds ? *reinterpret_cast<const float4 *>(ds + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float2 y01 = __ffma2_rn(make_float2((float)(int)w[0], (float)(int)w[1]), a2, make_float2(d4.x, d4.y));
+                const float2 y23 = __ffma2_rn(make_float2((float)(int)w[2], (float)(int)w[3]), a2, make_float2(d4.z, d4.w));
+                w[0] = __float_as_uint(y01.x);
+                w[1] = __float_as_uint(y01.y);
+                w[2] = __float_as_uint(y23.x);
+                w[3] = __float_as_uint(y23.y);
+            }
+        }
+#define SV(j) __uint_as_float(sv[(j) / 32][(j) % 32])
+        if (masked) {
+#pragma unroll
+            for (int j = 0; j < kTile; ++j) {
+                const int key = it * kTile + j;
+                const bool vis = key < p.n_kv && (!p.causal || key <= row + off);
+                if (!vis) sv[j / 32][j % 32] = __float_as_uint(-INFINITY);
+            }
+        }
+        float mx[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int b0 = 16 * u;
+            const float a0 = max3f(SV(b0), SV(b0 + 1), SV(b0 + 2));
+            const float a1 = max3f(SV(b0 + 3), SV(b0 + 4), SV(b0 + 5));
+            const float a2 = max3f(SV(b0 + 6), SV(b0 + 7), SV(b0 + 8));
+            const float a3 = max3f(SV(b0 + 9), SV(b0 + 10), SV(b0 + 11));
+            const float a4 = max3f(SV(b0 + 12), SV(b0 + 13), SV(b0 + 14));
+            mx[u] = max3f(max3f(a0, a1, a2), a3, max3f(a4, SV(b0 + 15), -INFINITY));
+        }
+        const float tmax = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+        const float m_new = fmaxf(m, tmax);
+        float alpha, bias;
+        if (m_new == -INFINITY) {
+            alpha = 1.f;
+            bias = 0.f;
+        } else {
+            alpha = ex2_approx((m - m_new) * c);
+            bias = p.log2_pr - m_new * c;
+        }
+        const float2 c2 = make_float2(c, c), b2 = make_float2(bias, bias);
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        uint32_t pk[kTile / 4];
+#pragma unroll
+        for (int j = 0; j < kTile; j += 4) {
+            const float2 e01 = __ffma2_rn(make_float2(SV(j), SV(j + 1)), c2, b2);
+            const float2 e23 = __ffma2_rn(make_float2(SV(j + 2), SV(j + 3)), c2, b2);
+            const float2 p01 = make_float2(ex2_approx(e01.x), ex2_approx(e01.y));
+            const float2 p23 = make_float2(ex2_approx(e23.x), ex2_approx(e23.y));
+            acc0 = __fadd2_rn(acc0, p01);
+            acc1 = __fadd2_rn(acc1, p23);
+            pk[j / 4] = pack_e4m3x4(p01.x, p01.y, p23.x, p23.y);
+        }
+#undef SV
+        const float2 acc = __fadd2_rn(acc0, acc1);
+        l = l * alpha + (acc.x + acc.y);
+        const bool rescale = (it > 0) && (alpha != 1.f);
+        m = m_new;
+
+        if (it > 0) {  // PV of the previous tile must be done before P and O are touched
+            if (!warp_wait(&sm.bar_o[X], (it - 1) & 1, abort_flag, p.status, kSiteO)) { ok = false; break; }
+            tc_fence_after();
+        }
+        uint8_t *pbuf = sm.p[X];
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16)
+            *reinterpret_cast<uint4 *>(pbuf + sw128_offset(r, c16)) =
+                make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
+        if (__any_sync(0xFFFFFFFFu, rescale)) {
+            const float2 al2 = make_float2(alpha, alpha);
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t ov[32];
+                tmem_ld32(o_tmem + c0, ov);
+                tmem_wait_ld_regs(ov);
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const float2 v2 = __fmul2_rn(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])), al2);
+                    ov[i] = __float_as_uint(v2.x);
+                    ov[i + 1] = __float_as_uint(v2.y);
+                }
+                tmem_st32(o_tmem + c0, ov);
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sm.bar_p[X]);
+    }
+    if (ok) ok = warp_wait(&sm.bar_o[X], (n_tiles - 1) & 1, abort_flag, p.status, kSiteO);
+    if (ok) {
+        tc_fence_after();
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const float *dv = p.dv + (size_t)bh * D;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld32(o_tmem + c0, ov);
+            tmem_wait_ld_regs(ov);
+            float y[32];
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                const float4 s4 = __ldg(reinterpret_cast<const float4 *>(dv + c0 + i));
+                y[i] = __uint_as_float(ov[i]) * s4.x * inv_l;
+                y[i + 1] = __uint_as_float(ov[i + 1]) * s4.y * inv_l;
+                y[i + 2] = __uint_as_float(ov[i + 2]) * s4.z * inv_l;
+                y[i + 3] = __uint_as_float(ov[i + 3]) * s4.w * inv_l;
+            }
+            if (row < p.n_q) store_row_chunk(orow + c0, y, p.out_bf16);
+        }
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
+    constexpr int ST = AttnCfg<D>::kStages;
     extern __shared__ uint8_t smem_raw[];
     AttnSmem<D> &sm =
         *reinterpret_cast<AttnSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // Work item: longest Q tiles first when causal.
-    const int t_idx = blockIdx.x / p.BH;
+    // Work item: a pair of Q tiles of one head; longest pairs first when causal.
+    const int n_pairs = (p.Tq + 1) / 2;
+    const int pair_idx = blockIdx.x / p.BH;
     const int bh = blockIdx.x % p.BH;
-    const int t = p.causal ? (p.Tq - 1 - t_idx) : t_idx;
+    const int u = p.causal ? (n_pairs - 1 - pair_idx) : pair_idx;
+    const int tA = 2 * u, tB = 2 * u + 1;
     const int b = bh / p.H, h = bh % p.H;
     const int off = p.n_kv - p.n_q;
-    int n_tiles = p.Tk;
-    if (p.causal) {
-        const int last_key = min(t * kTile + kTile - 1, p.n_q - 1) + off;
-        n_tiles = last_key < 0 ? 0 : min(p.Tk, last_key / kTile + 1);
-    }
+    const int nA = kv_tiles_of(tA, p.Tq, p.Tk, p.n_q, off, p.causal);
+    const int nB = kv_tiles_of(tB, p.Tq, p.Tk, p.n_q, off, p.causal);
+    const int n_tiles = max(nA, nB);
+    const bool hasB = tB < p.Tq;
     const int64_t o_base = (int64_t)b * p.so_b + (int64_t)h * p.so_h;
-
-    if (n_tiles == 0) {  // no row of this tile sees any key: O = 0
-        if (warp < 4) {
-            const int row = t * kTile + warp * 32 + lane;
-            if (row < p.n_q) {
-                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) + o_base + (int64_t)row * p.so_n);
-#pragma unroll
-                for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
-            }
-        }
-        return;
-    }
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_q, 1);
-        for (int s = 0; s < kStages; ++s) { mbar_init(&sm.bar_full[s], 1); mbar_init(&sm.bar_empty[s], 1); }
-        mbar_init(&sm.bar_s[0], 1);
-        mbar_init(&sm.bar_s[1], 1);
-        mbar_init(&sm.bar_p, 128);
-        mbar_init(&sm.bar_o, 1);
+        for (int s = 0; s < ST; ++s) { mbar_init(&sm.bar_full[s], 1); mbar_init(&sm.bar_empty[s], 1); }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&sm.bar_s[x], 1);
+            mbar_init(&sm.bar_sfree[x], 128);
+            mbar_init(&sm.bar_p[x], 128);
+            mbar_init(&sm.bar_o[x], 1);
+        }
         mbar_init(&sm.bar_drain, 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9 && n_tiles > 0) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -164,183 +362,102 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort_flag = &sm.abort_flag;
 
-    if (warp == 4) {
-        // ------------------------------ TMA producer ------------------------------
-        if (lane == 0) {
+    if (warp >= 8) {
+        setmaxnreg_dec<kRegsProducer>();
+        if (warp == 8 && lane == 0 && n_tiles > 0) {
+            // ------------------------------ TMA producer ------------------------------
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            mbar_arrive_expect_tx(&sm.bar_q, kTile * D);
-            tma_load_2d(sm.q, &tm_q, &sm.bar_q, 0, bh * p.nq_pad + t * kTile);
-            const uint32_t stage_bytes = kTile * D * 2 + (p.use_ds ? kTile * 4 : 0) + (kTile / kKeyRun) * 4;
-            const float *ds_row = p.ds + ((size_t)bh * p.Tq + t) * p.nk_pad;
+            mbar_arrive_expect_tx(&sm.bar_q, (hasB ? 2 : 1) * kTile * D);
+            tma_load_2d(sm.q[0], &tm_q, &sm.bar_q, 0, bh * p.nq_pad + tA * kTile);
+            if (hasB) tma_load_2d(sm.q[1], &tm_q, &sm.bar_q, 0, bh * p.nq_pad + tB * kTile);
+            const float *ds_a = p.ds + ((size_t)bh * p.Tq + tA) * p.nk_pad;
+            const float *ds_b = p.ds + ((size_t)bh * p.Tq + tB) * p.nk_pad;
             const float *dk_row = p.dk + (size_t)bh * (p.nk_pad / kKeyRun);
             int issued = 0;
             for (int it = 0; it < n_tiles; ++it) {
-                const int s = it % kStages;
-                if (it >= kStages && !mbar_wait(&sm.bar_empty[s], ((it / kStages) & 1) ^ 1, abort_flag, p.status, kSiteEmpty))
+                const int s = it % ST;
+                if (it >= ST && !mbar_wait(&sm.bar_empty[s], ((it / ST) & 1) ^ 1, abort_flag, p.status, kSiteEmpty))
                     break;
                 issued = it + 1;
                 if (p.fault_inject && it == 0) continue;  // diagnostic: leave stage 0 unsignalled
-                mbar_arrive_expect_tx(&sm.bar_full[s], stage_bytes);
+                const bool dsA = p.use_ds && it < nA, dsB = p.use_ds && it < nB;
+                const uint32_t bytes = kTile * D * 2 + (dsA ? kTile * 4 : 0) + (dsB ? kTile * 4 : 0) + (kTile / kKeyRun) * 4;
+                mbar_arrive_expect_tx(&sm.bar_full[s], bytes);
                 tma_load_2d(sm.k[s], &tm_k, &sm.bar_full[s], 0, bh * p.nk_pad + it * kTile);
                 tma_load_2d(sm.v[s], &tm_v, &sm.bar_full[s], it * kTile, bh * D);
-                if (p.use_ds) bulk_load(sm.ds[s], ds_row + it * kTile, kTile * 4, &sm.bar_full[s]);
+                if (dsA) bulk_load(sm.ds[s][0], ds_a + it * kTile, kTile * 4, &sm.bar_full[s]);
+                if (dsB) bulk_load(sm.ds[s][1], ds_b + it * kTile, kTile * 4, &sm.bar_full[s]);
                 bulk_load(sm.dk[s], dk_row + it * (kTile / kKeyRun), (kTile / kKeyRun) * 4, &sm.bar_full[s]);
             }
             if (*abort_flag) {  // let the copies in flight land before the CTA exits
                 mbar_wait_quiet(&sm.bar_q, 0, kDrainNs);
-                for (int it = max(0, issued - kStages); it < issued; ++it) {
+                for (int it = max(0, issued - ST); it < issued; ++it) {
                     if (p.fault_inject && it == 0) continue;
-                    mbar_wait_quiet(&sm.bar_full[it % kStages], (it / kStages) & 1, kDrainNs);
+                    mbar_wait_quiet(&sm.bar_full[it % ST], (it / ST) & 1, kDrainNs);
                 }
             }
-        }
-    } else if (warp == 5) {
-        // ------------------------------ MMA issuer ------------------------------
-        if (lane == 0) {
-            const uint32_t q_s = smem_u32(sm.q), p_s = smem_u32(sm.p);
+        } else if (warp == 9 && lane == 0 && n_tiles > 0) {
+            // ------------------------------ MMA issuer ------------------------------
+            const uint32_t q_s[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
+            const uint32_t p_s[2] = {smem_u32(sm.p[0]), smem_u32(sm.p[1])};
+            const int nX[2] = {nA, nB};
             bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, p.status, kSiteQ);
-            auto qk = [&](int i) -> bool {
-                const int s = i % kStages;
-                if (!mbar_wait(&sm.bar_full[s], (i / kStages) & 1, abort_flag, p.status, kSiteFull)) return false;
+            if (ok) ok = mbar_wait(&sm.bar_full[0], 0, abort_flag, p.status, kSiteFull);
+            if (ok) {
                 tc_fence_after();
-                issue_qk<D>(tmem + (uint32_t)(i & 1) * 128u, q_s, smem_u32(sm.k[s]));
-                mma_commit(&sm.bar_s[i & 1]);
-                return true;
-            };
-            if (ok) ok = qk(0);
+                for (int x = 0; x < 2; ++x)
+                    if (nX[x] > 0) {
+                        issue_qk<D>(tmem + (uint32_t)x * 128u, q_s[x], smem_u32(sm.k[0]));
+                        mma_commit(&sm.bar_s[x]);
+                    }
+            }
             for (int it = 0; ok && it < n_tiles; ++it) {
-                if (it + 1 < n_tiles && !qk(it + 1)) break;
-                if (!mbar_wait(&sm.bar_p, it & 1, abort_flag, p.status, kSiteP)) break;
-                tc_fence_after();
-                const int s = it % kStages;
-                issue_pv<D>(tmem + kTmemO, p_s, smem_u32(sm.v[s]), it > 0);
-                mma_commit(&sm.bar_o);
+                const int s = it % ST;
+                if (it + 1 < n_tiles) {
+                    const int s1 = (it + 1) % ST;
+                    if (!mbar_wait(&sm.bar_full[s1], ((it + 1) / ST) & 1, abort_flag, p.status, kSiteFull)) break;
+                    bool brk = false;
+                    for (int x = 0; x < 2; ++x) {
+                        if (it + 1 >= nX[x]) continue;
+                        if (!mbar_wait(&sm.bar_sfree[x], it & 1, abort_flag, p.status, kSiteSfree)) { brk = true; break; }
+                        tc_fence_after();
+                        issue_qk<D>(tmem + (uint32_t)x * 128u, q_s[x], smem_u32(sm.k[s1]));
+                        mma_commit(&sm.bar_s[x]);
+                    }
+                    if (brk) break;
+                }
+                bool brk = false;
+                for (int x = 0; x < 2; ++x) {
+                    if (it >= nX[x]) continue;
+                    if (!mbar_wait(&sm.bar_p[x], it & 1, abort_flag, p.status, kSiteP)) { brk = true; break; }
+                    tc_fence_after();
+                    issue_pv<D>(tmem + kTmemO + (uint32_t)x * D, p_s[x], smem_u32(sm.v[s]), it > 0);
+                    mma_commit(&sm.bar_o[x]);
+                }
+                if (brk) break;
                 mma_commit(&sm.bar_empty[s]);
             }
             mma_commit(&sm.bar_drain);
             mbar_wait_quiet(&sm.bar_drain, 0, kDrainNs);
         }
-    } else {
-        // ------------------------- softmax (warps 0-3) -------------------------
-        const int r = warp * 32 + lane;
-        const int row = t * kTile + r;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const float dq = p.dq[(size_t)bh * p.nq_pad + row];
-        const float c = p.scale_log2;
-        float m = -INFINITY, l = 0.f;
-        bool ok = true;
-        for (int it = 0; it < n_tiles; ++it) {
-            const int s = it % kStages;
-            if (!warp_wait(&sm.bar_s[it & 1], (it >> 1) & 1, abort_flag, p.status, kSiteS)) { ok = false; break; }
-            if (!warp_wait(&sm.bar_full[s], (it / kStages) & 1, abort_flag, p.status, kSiteFull)) { ok = false; break; }
+        // all roles meet here before tensor memory is released
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 9 && n_tiles > 0) {
+            __syncwarp();
             tc_fence_after();
-            uint32_t sv[4][32];
-            const uint32_t s_addr = tmem + lane_base + (uint32_t)(it & 1) * 128u;
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(s_addr + q4 * 32, sv[q4]);
-            tmem_wait_ld_regs(sv[0]);
-            reg_fence(sv[1]);
-            reg_fence(sv[2]);
-            reg_fence(sv[3]);
-
-            float a[kTile / kKeyRun];
-#pragma unroll
-            for (int g = 0; g < kTile / kKeyRun; ++g) a[g] = dq * sm.dk[s][g];
-            const bool masked = (it * kTile + kTile > p.n_kv) || (p.causal && it * kTile + kTile - 1 > t * kTile + off);
-            float tmax = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < kTile; ++j) {
-                const float ds = p.use_ds ? sm.ds[s][j] : 0.f;
-                float x = fmaf((float)(int)sv[j / 32][j % 32], a[j / kKeyRun], ds);
-                if (masked) {
-                    const int key = it * kTile + j;
-                    const bool vis = key < p.n_kv && (!p.causal || key <= row + off);
-                    x = vis ? x : -INFINITY;
-                }
-                sv[j / 32][j % 32] = __float_as_uint(x);
-                tmax = fmaxf(tmax, x);
-            }
-            const float m_new = fmaxf(m, tmax);
-            float alpha, bias;
-            if (m_new == -INFINITY) {
-                alpha = 1.f;
-                bias = 0.f;
-            } else {
-                alpha = ex2_approx((m - m_new) * c);
-                bias = p.log2_pr - m_new * c;
-            }
-            float sum = 0.f;
-            uint32_t pk[kTile / 4];
-#pragma unroll
-            for (int j = 0; j < kTile; j += 4) {
-                float e[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) e[u] = ex2_approx(fmaf(__uint_as_float(sv[(j + u) / 32][(j + u) % 32]), c, bias));
-                sum += (e[0] + e[1]) + (e[2] + e[3]);
-                pk[j / 4] = pack_e4m3x4(e[0], e[1], e[2], e[3]);
-            }
-            l = l * alpha + sum;
-            const bool rescale = (it > 0) && (alpha != 1.f);
-            m = m_new;
-
-            if (it > 0) {  // PV of the previous tile must be done before P and O are touched
-                if (!warp_wait(&sm.bar_o, (it - 1) & 1, abort_flag, p.status, kSiteO)) { ok = false; break; }
-                tc_fence_after();
-            }
-#pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16)
-                *reinterpret_cast<uint4 *>(sm.p + sw128_offset(r, c16)) =
-                    make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
-            if (__any_sync(0xFFFFFFFFu, rescale)) {
-#pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t ov[32];
-                    tmem_ld32(tmem + lane_base + kTmemO + c0, ov);
-                    tmem_wait_ld_regs(ov);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                    tmem_st32(tmem + lane_base + kTmemO + c0, ov);
-                }
-                tmem_wait_st();
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&sm.bar_p);
+            tmem_dealloc(tmem, kTmemCols);
         }
-        if (ok) ok = warp_wait(&sm.bar_o, (n_tiles - 1) & 1, abort_flag, p.status, kSiteO);
-        if (ok) {
-            tc_fence_after();
-            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-            const float *dv = p.dv + (size_t)bh * D;
-            uint16_t *orow = static_cast<uint16_t *>(p.o) + o_base + (int64_t)row * p.so_n;
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t ov[32];
-                tmem_ld32(tmem + lane_base + kTmemO + c0, ov);
-                tmem_wait_ld_regs(ov);
-                float y[32];
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const float4 s4 = __ldg(reinterpret_cast<const float4 *>(dv + c0 + i));
-                    y[i] = __uint_as_float(ov[i]) * s4.x * inv_l;
-                    y[i + 1] = __uint_as_float(ov[i + 1]) * s4.y * inv_l;
-                    y[i + 2] = __uint_as_float(ov[i + 2]) * s4.z * inv_l;
-                    y[i + 3] = __uint_as_float(ov[i + 3]) * s4.w * inv_l;
-                }
-                if (row < p.n_q) store_row_chunk(orow + c0, y, p.out_bf16);
-            }
-        }
+        return;
     }
-
+    setmaxnreg_inc<kRegsSoftmax>();
+    const int X = warp >> 2;
+    if (X == 0) softmax_role<D>(sm, p, tmem, 0, tA, nA, bh, o_base, abort_flag);
+    else if (hasB) softmax_role<D>(sm, p, tmem, 1, tB, nB, bh, o_base, abort_flag);
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
-    }
 }
 
 template <int D>
@@ -349,7 +466,7 @@ static cudaError_t launch_attention_d(const CUtensorMap &tq, const CUtensorMap &
     const size_t smem = sizeof(AttnSmem<D>) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)p.Tq * (unsigned)p.BH;
+    const unsigned grid = (unsigned)((p.Tq + 1) / 2) * (unsigned)p.BH;
     attn_fwd_kernel<D><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }

@@ -62,8 +62,8 @@ __device__ __forceinline__ void record_error(int *status, int code, int site) {
 // Wait until the phase with `parity` of `bar` has completed.  Gives up (returns
 // false) when the CTA-wide abort flag is raised or after kWaitLimitNs, in which
 // case it records SAGE_ERR_TIMEOUT with `site` and raises the abort flag.
-static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                       int *status, int site) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          int *status, int site) {
     const uint32_t a = smem_u32(bar);
     if (mbar_test(a, parity)) return true;
     const uint64_t t0 = globaltimer();
@@ -81,7 +81,7 @@ static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, vo
 }
 
 // Same, without recording anything: used to drain in-flight copies on the abort path.
-static __device__ __noinline__ void mbar_wait_quiet(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+__device__ __forceinline__ void mbar_wait_quiet(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     const uint32_t a = smem_u32(bar);
     const uint64_t t0 = globaltimer();
     while (!mbar_test(a, parity)) {
