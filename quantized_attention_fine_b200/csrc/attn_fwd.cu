@@ -214,12 +214,12 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
         }
 #define SV(j) __uint_as_float(sv[(j) / 32][(j) % 32])
         if (masked) {
+            // key it*128 + j is visible iff j <= lim (the key-count tail and the causal diagonal)
+            int lim = p.n_kv - 1 - it * kTile;
+            if (p.causal) lim = min(lim, row + off - it * kTile);
 #pragma unroll
-            for (int j = 0; j < kTile; ++j) {
-                const int key = it * kTile + j;
-                const bool vis = key < p.n_kv && (!p.causal || key <= row + off);
-                if (!vis) sv[j / 32][j % 32] = __float_as_uint(-INFINITY);
-            }
+            for (int j = 0; j < kTile; ++j)
+                if (j > lim) sv[j / 32][j % 32] = __float_as_uint(-INFINITY);
         }
         float mx[8];
 #pragma unroll
@@ -453,9 +453,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         return;
     }
     setmaxnreg_inc<kRegsSoftmax>();
+    // one copy of the softmax code serves both warpgroups (instruction-cache footprint)
     const int X = warp >> 2;
-    if (X == 0) softmax_role<D>(sm, p, tmem, 0, tA, nA, bh, o_base, abort_flag);
-    else if (hasB) softmax_role<D>(sm, p, tmem, 1, tB, nB, bh, o_base, abort_flag);
+    if (X == 0 || hasB) softmax_role<D>(sm, p, tmem, X, X ? tB : tA, X ? nB : nA, bh, o_base, abort_flag);
     tc_fence_before();
     __syncthreads();
 }

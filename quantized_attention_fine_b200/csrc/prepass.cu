@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(256) quant_q_kernel(const PrepassArgs a) {
 template <int D>
 struct QuantKvSmem {
     float kt[D][kTile + 1];        // raw K of the tile, transposed (for dS)
-    float qbar[32][D];             // a chunk of Q block means
+    float qbt[D][36];              // a chunk of 32 Q block means, transposed ([channel][block])
     uint8_t vt[D][kTile + 16];     // E4M3 V codes of the tile, transposed
     float ramax[kTile];
     float delta[kTile];
@@ -326,6 +326,8 @@ __global__ void __launch_bounds__(256, 1) quant_kv_kernel(const PrepassArgs a, i
     }
 
     if (need_ds) {
+        // dS[t][j] = qbar_t . K[j] for this tile's keys: thread (j, half) keeps K[j] in
+        // registers and accumulates 8 Q blocks at a time (independent FMA chains).
         __syncthreads();
         const int j = threadIdx.x & (kTile - 1), half = threadIdx.x >> 7;
         float kr[D];
@@ -341,20 +343,32 @@ __global__ void __launch_bounds__(256, 1) quant_kv_kernel(const PrepassArgs a, i
         float *ds = reinterpret_cast<float *>(a.ws + a.L.ds) + (size_t)bh * S.Tq * S.nk_pad + j0 + j;
         for (int tc = t_lo; tc < S.Tq; tc += 32) {
             const int nt = min(32, S.Tq - tc);
-            for (int idx = threadIdx.x; idx < nt * D; idx += blockDim.x)
-                sm.qbar[idx / D][idx % D] = qbar[(size_t)tc * D + idx];
+            for (int idx = threadIdx.x; idx < 32 * D; idx += blockDim.x) {
+                const int tt = idx / D, c = idx % D;
+                sm.qbt[c][tt] = (tt < nt) ? qbar[(size_t)(tc + tt) * D + c] : 0.f;
+            }
             __syncthreads();
-            for (int tt = half; tt < nt; tt += 2) {
-                float acc = 0.f;
+#pragma unroll 1
+            for (int tt0 = half * 16; tt0 < half * 16 + 16 && tt0 < nt; tt0 += 8) {
+                float acc[8];
 #pragma unroll
-                for (int c = 0; c < D; c += 4) {
-                    const float4 qv = *reinterpret_cast<const float4 *>(&sm.qbar[tt][c]);
-                    acc = fmaf(qv.x, kr[c], acc);
-                    acc = fmaf(qv.y, kr[c + 1], acc);
-                    acc = fmaf(qv.z, kr[c + 2], acc);
-                    acc = fmaf(qv.w, kr[c + 3], acc);
+                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+                for (int c = 0; c < D; ++c) {
+                    const float4 qa = *reinterpret_cast<const float4 *>(&sm.qbt[c][tt0]);
+                    const float4 qb = *reinterpret_cast<const float4 *>(&sm.qbt[c][tt0 + 4]);
+                    acc[0] = fmaf(qa.x, kr[c], acc[0]);
+                    acc[1] = fmaf(qa.y, kr[c], acc[1]);
+                    acc[2] = fmaf(qa.z, kr[c], acc[2]);
+                    acc[3] = fmaf(qa.w, kr[c], acc[3]);
+                    acc[4] = fmaf(qb.x, kr[c], acc[4]);
+                    acc[5] = fmaf(qb.y, kr[c], acc[5]);
+                    acc[6] = fmaf(qb.z, kr[c], acc[6]);
+                    acc[7] = fmaf(qb.w, kr[c], acc[7]);
                 }
-                ds[(size_t)(tc + tt) * S.nk_pad] = acc;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (tt0 + i < nt) ds[(size_t)(tc + tt0 + i) * S.nk_pad] = acc[i];
             }
             __syncthreads();
         }
