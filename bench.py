@@ -31,6 +31,9 @@ METRIC = "attention TOPS (4*B*H*Nq*Nkv*d/t, causal /2) and % of B200 dense INT8/
 UNIT = "TOPS"
 SPEC_INT8_TOPS = 4500.0          # B200 dense INT8 / FP8 datasheet figure
 FALLBACK_BF16_TFLOPS = 1590.0    # pool measurement used when MEASURED_PEAKS.json is absent
+# library kernels per step: quant_qk (kv_stats, kv_finalize, quant_q, quant_k, ds_gemm),
+# quant_v (kv_stats, kv_finalize, quant_v), attention (attn_fwd_kernel)
+LAUNCHES_PER_STEP = 9
 KERNEL_SOURCES = ["quantized_attention_fine_b200/csrc/attn_fwd.cu", "quantized_attention_fine_b200/csrc/sage_device.cuh"]
 
 
@@ -337,7 +340,7 @@ def main():
                      "peak_source": "%s bf16 burst %.1f x 2 (dense int8/fp8 = 2x bf16)" % (peak_src, bf16_burst),
                      "kernel": "attn_fwd_kernel<%d>" % d},
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-        "gpu_launches": args.steps * 8,
+        "gpu_launches": args.steps * LAUNCHES_PER_STEP,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -3,18 +3,20 @@
 // fine-grained Q/K quantization, FP8 V; per-channel V scale from the
 // pith.science verdict on arXiv 2505.21136, key_machinery).
 //
-// Four kernels, all bandwidth-bound except the dS product:
+// Bandwidth-bound kernels (the dS product is in ds_gemm.cu):
 //   kv_stats     per (head, 512-token chunk): fp64 partial sums of K per channel
 //                and per-channel max |V|.
 //   kv_finalize  per head: kbar = fp32(sum / n_kv); delta_V = max|V| / Vr.
 //   quant_q      per (head, 128-row block): qbar (fp64 mean of the valid rows,
 //                rounded to fp32), Q_s = Q - qbar in fp32, group amax, INT8 codes.
-//   quant_kv     per (head, 128-key tile): K_s = K - kbar, INT8 codes per group,
-//                delta_K per 16-key run; V / delta_V -> E4M3, written transposed
-//                ([channel][key]); dS[t][j] = qbar_t . K[j] for the Q blocks t
-//                that can see the tile.
-// Every code decision (INT8 rounding, E4M3 rounding) is an IEEE fp32 quotient
-// (__fdiv_rn) rounded half to even, so that it is reproducible on the host.
+//   quant_k      per (head, 128-key tile): K_s = K - kbar, INT8 codes per group,
+//                delta_K per 16-key run.
+//   quant_v      per (head, 128-key tile): V / delta_V -> E4M3, written transposed
+//                ([channel][key]).
+// Every code decision (INT8 rounding, E4M3 rounding) is made on the IEEE fp32
+// quotient x / delta, rounded to nearest even, so that it is reproducible on the
+// host.  The quotient is formed as x * (1 / delta) when that product provably
+// rounds to the same code, and by IEEE division otherwise (see fast_quotient_*).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -50,14 +52,30 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-__device__ __forceinline__ int8_t int8_code(float xs, float delta) {
-    float r = rintf(__fdiv_rn(xs, delta));
+// INT8 code: round-half-even of the IEEE fp32 quotient xs / delta, clamped to +-127.
+// For |xs / delta| <= 128, t = RN(xs * RN(1 / delta)) lies within 2.3e-5 of the
+// correctly rounded quotient, so when t is at least 2^-15 (3.05e-5) away from a
+// half-integer both round to the same integer; only the rare near-tie takes the
+// IEEE division.
+__device__ __forceinline__ int8_t int8_code(float xs, float delta, float inv_delta) {
+    const float t = xs * inv_delta;
+    float r;
+    if (fabsf(t - floorf(t) - 0.5f) >= 0x1p-15f) r = rintf(t);
+    else r = rintf(__fdiv_rn(xs, delta));
     r = fminf(fmaxf(r, -127.f), 127.f);
     return (int8_t)(int)r;
 }
 
-__device__ __forceinline__ uint8_t e4m3_code(float x) {
-    return (uint8_t)(pack_e4m3x4(x, 0.f, 0.f, 0.f) & 0xFFu);
+// The IEEE fp32 quotient x / delta as far as its E4M3 rounding is concerned.
+// t = RN(x * RN(1 / delta)) is within about 1.5 fp32 ulp of the correctly rounded
+// quotient; E4M3 rounds at bit 19 of the fp32 mantissa (normal range), so unless the
+// 20 low bits of t are within 4 of the tie pattern 0x80000 both round alike.  The
+// subnormal E4M3 range (|t| < 2^-6) and near-ties use the IEEE division.
+__device__ __forceinline__ float e4m3_quotient(float x, float delta, float inv_delta) {
+    const float t = x * inv_delta;
+    const int dist = (int)(__float_as_uint(t) & 0xFFFFFu) - 0x80000;
+    if (fabsf(t) < 0x1p-6f || (dist >= -4 && dist <= 4)) return __fdiv_rn(x, delta);
+    return t;
 }
 
 template <int VEC>
@@ -218,184 +236,138 @@ __global__ void __launch_bounds__(256) quant_q_kernel(const PrepassArgs a) {
     for (int i = 0; i < RPW; ++i) {
         const int r = warp * RPW + i;
         const float dl = s_delta[r];
+        const float inv = 1.0f / dl;
         int8_t c[VEC];
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) c[v] = int8_code(x[i][v], dl);
+        for (int v = 0; v < VEC; ++v) c[v] = int8_code(x[i][v], dl, inv);
         store_codes<VEC>(q8 + (size_t)r * D, c);
     }
 }
 
 // ---------------------------------------------------------------------------
 template <int D>
-struct QuantKvSmem {
-    float kt[D][kTile + 1];        // raw K of the tile, transposed (for dS)
-    float qbt[D][36];              // a chunk of 32 Q block means, transposed ([channel][block])
-    uint8_t vt[D][kTile + 16];     // E4M3 V codes of the tile, transposed
-    float ramax[kTile];
-    float delta[kTile];
-};
-
-template <int D>
-__global__ void __launch_bounds__(256, 1) quant_kv_kernel(const PrepassArgs a, int ds_t_skip, int causal_off) {
+__global__ void __launch_bounds__(256) quant_k_kernel(const PrepassArgs a) {
     constexpr int VEC = D / 32, RPW = 16;
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    QuantKvSmem<D> &sm = *reinterpret_cast<QuantKvSmem<D> *>(smem_raw);
+    __shared__ float s_ramax[kTile];
+    __shared__ float s_delta[kTile];
     const Shape &S = a.shape;
     const int jt = blockIdx.x, bh = blockIdx.y;
     const int b = bh / S.H, h = bh % S.H;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int j0 = jt * kTile;
     const int nvalid = min(kTile, S.n_kv - j0);
-    const bool need_ds = a.k != nullptr && a.smooth_q;
-
-    if (a.k) {
-        const uint16_t *kp = static_cast<const uint16_t *>(a.k) + b * a.skv.b + h * a.skv.h + lane * VEC;
-        float kb[VEC];
+    const uint16_t *kp = static_cast<const uint16_t *>(a.k) + b * a.skv.b + h * a.skv.h + lane * VEC;
+    float kb[VEC];
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) kb[v] = reinterpret_cast<const float *>(a.ws + a.L.kbar)[(size_t)bh * D + lane * VEC + v];
-        float x[RPW][VEC];
+    for (int v = 0; v < VEC; ++v) kb[v] = reinterpret_cast<const float *>(a.ws + a.L.kbar)[(size_t)bh * D + lane * VEC + v];
+    float x[RPW][VEC];
 #pragma unroll
-        for (int i = 0; i < RPW; ++i) {
-            const int r = warp * RPW + i;
-            if (r < nvalid) {
-                load_row_slice<VEC>(kp + (int64_t)(j0 + r) * a.skv.n, a.bf16, x[i]);
-            } else {
+    for (int i = 0; i < RPW; ++i) {
+        const int r = warp * RPW + i;
+        if (r < nvalid) {
+            load_row_slice<VEC>(kp + (int64_t)(j0 + r) * a.skv.n, a.bf16, x[i]);
+        } else {
 #pragma unroll
-                for (int v = 0; v < VEC; ++v) x[i][v] = 0.f;
-            }
-            float am = 0.f;
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) {
-                if (need_ds) sm.kt[lane * VEC + v][r] = x[i][v];
-                const float xs = (r < nvalid) ? __fsub_rn(x[i][v], kb[v]) : 0.f;
-                x[i][v] = xs;
-                am = fmaxf(am, fabsf(xs));
-            }
-            am = warp_max(am);
-            if (lane == 0) sm.ramax[r] = am;
-        }
-        __syncthreads();
-        if (threadIdx.x < kTile) {
-            const int r = threadIdx.x;
-            const int g0 = (r / a.g_k) * a.g_k;
-            float am = 0.f;
-            for (int rr = g0; rr < g0 + a.g_k; ++rr) am = fmaxf(am, sm.ramax[rr]);
-            const float dl = (am == 0.f) ? 1.f : __fdiv_rn(am, 127.f);
-            sm.delta[r] = dl;
-            if ((r % kKeyRun) == 0)
-                reinterpret_cast<float *>(a.ws + a.L.dk)[(size_t)bh * (S.nk_pad / kKeyRun) + (j0 + r) / kKeyRun] = dl;
-        }
-        __syncthreads();
-        int8_t *k8 = reinterpret_cast<int8_t *>(a.ws + a.L.k8) + ((size_t)bh * S.nk_pad + j0) * D + lane * VEC;
-#pragma unroll
-        for (int i = 0; i < RPW; ++i) {
-            const int r = warp * RPW + i;
-            const float dl = sm.delta[r];
-            int8_t c[VEC];
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) c[v] = int8_code(x[i][v], dl);
-            store_codes<VEC>(k8 + (size_t)r * D, c);
+            for (int v = 0; v < VEC; ++v) x[i][v] = 0.f;
         }
     }
-
-    if (a.v) {
-        const uint16_t *vp = static_cast<const uint16_t *>(a.v) + b * a.skv.b + h * a.skv.h + lane * VEC;
-        float dv[VEC];
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) dv[v] = reinterpret_cast<const float *>(a.ws + a.L.dv)[(size_t)bh * D + lane * VEC + v];
-#pragma unroll 4
-        for (int i = 0; i < RPW; ++i) {
-            const int r = warp * RPW + i;
-            float x[VEC];
-            if (r < nvalid) {
-                load_row_slice<VEC>(vp + (int64_t)(j0 + r) * a.skv.n, a.bf16, x);
-            } else {
+    for (int i = 0; i < RPW; ++i) {
+        const int r = warp * RPW + i;
+        float am = 0.f;
 #pragma unroll
-                for (int v = 0; v < VEC; ++v) x[v] = 0.f;
-            }
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) sm.vt[lane * VEC + v][r] = e4m3_code(__fdiv_rn(x[v], dv[v]));
+        for (int v = 0; v < VEC; ++v) {
+            const float xs = (r < nvalid) ? __fsub_rn(x[i][v], kb[v]) : 0.f;
+            x[i][v] = xs;
+            am = fmaxf(am, fabsf(xs));
         }
-        __syncthreads();
-        uint8_t *vt8 = a.ws + a.L.vt8;
-        for (int idx = threadIdx.x; idx < D * (kTile / 16); idx += blockDim.x) {
-            const int c = idx / (kTile / 16), ch = idx % (kTile / 16);
-            const uint4 val = *reinterpret_cast<const uint4 *>(&sm.vt[c][ch * 16]);
-            *reinterpret_cast<uint4 *>(vt8 + ((size_t)bh * D + c) * S.nk_pad + j0 + ch * 16) = val;
+        am = warp_max(am);
+        if (lane == 0) s_ramax[r] = am;
+    }
+    __syncthreads();
+    if (threadIdx.x < kTile) {
+        const int r = threadIdx.x;
+        const int g0 = (r / a.g_k) * a.g_k;
+        float am = 0.f;
+        for (int rr = g0; rr < g0 + a.g_k; ++rr) am = fmaxf(am, s_ramax[rr]);
+        const float dl = (am == 0.f) ? 1.f : __fdiv_rn(am, 127.f);
+        s_delta[r] = dl;
+        if ((r % kKeyRun) == 0)
+            reinterpret_cast<float *>(a.ws + a.L.dk)[(size_t)bh * (S.nk_pad / kKeyRun) + (j0 + r) / kKeyRun] = dl;
+    }
+    __syncthreads();
+    int8_t *k8 = reinterpret_cast<int8_t *>(a.ws + a.L.k8) + ((size_t)bh * S.nk_pad + j0) * D + lane * VEC;
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+        const int r = warp * RPW + i;
+        const float dl = s_delta[r];
+        const float inv = 1.0f / dl;
+        int8_t c[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) c[v] = int8_code(x[i][v], dl, inv);
+        store_codes<VEC>(k8 + (size_t)r * D, c);
+    }
+}
+
+// V codes of one 128-key tile, written transposed: each lane holds 16 consecutive
+// keys of VEC channels and stores them as one 16-byte piece of each channel's row of
+// V^T ([channel][key]).
+template <int D>
+__global__ void __launch_bounds__(256) quant_v_kernel(const PrepassArgs a) {
+    constexpr int VEC = D / 32, RPW = 16;
+    const Shape &S = a.shape;
+    const int jt = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / S.H, h = bh % S.H;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j0 = jt * kTile;
+    const int nvalid = min(kTile, S.n_kv - j0);
+    const uint16_t *vp = static_cast<const uint16_t *>(a.v) + b * a.skv.b + h * a.skv.h + lane * VEC;
+    float dv[VEC], inv[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+        dv[v] = reinterpret_cast<const float *>(a.ws + a.L.dv)[(size_t)bh * D + lane * VEC + v];
+        inv[v] = 1.0f / dv[v];
+    }
+    float x[RPW][VEC];
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+        const int r = warp * RPW + i;
+        if (r < nvalid) {
+            load_row_slice<VEC>(vp + (int64_t)(j0 + r) * a.skv.n, a.bf16, x[i]);
+        } else {
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) x[i][v] = 0.f;
         }
     }
-
-    if (need_ds) {
-        // dS[t][j] = qbar_t . K[j] for this tile's keys: thread (j, half) keeps K[j] in
-        // registers and accumulates 8 Q blocks at a time (independent FMA chains).
-        __syncthreads();
-        const int j = threadIdx.x & (kTile - 1), half = threadIdx.x >> 7;
-        float kr[D];
+    uint8_t *vt8 = a.ws + a.L.vt8 + ((size_t)bh * D + lane * VEC) * S.nk_pad + j0 + warp * RPW;
 #pragma unroll
-        for (int c = 0; c < D; ++c) kr[c] = sm.kt[c][j];
-        int t_lo = 0;
-        if (ds_t_skip) {
-            const int num = j0 - causal_off - (kTile - 1);
-            t_lo = num <= 0 ? 0 : (num + kTile - 1) / kTile;
-            if (t_lo > S.Tq - 1) t_lo = S.Tq - 1;
-        }
-        const float *qbar = reinterpret_cast<const float *>(a.ws + a.L.qbar) + (size_t)bh * S.Tq * D;
-        float *ds = reinterpret_cast<float *>(a.ws + a.L.ds) + (size_t)bh * S.Tq * S.nk_pad + j0 + j;
-        for (int tc = t_lo; tc < S.Tq; tc += 32) {
-            const int nt = min(32, S.Tq - tc);
-            for (int idx = threadIdx.x; idx < 32 * D; idx += blockDim.x) {
-                const int tt = idx / D, c = idx % D;
-                sm.qbt[c][tt] = (tt < nt) ? qbar[(size_t)(tc + tt) * D + c] : 0.f;
-            }
-            __syncthreads();
-#pragma unroll 1
-            for (int tt0 = half * 16; tt0 < half * 16 + 16 && tt0 < nt; tt0 += 8) {
-                float acc[8];
+    for (int v = 0; v < VEC; ++v) {
+        uint32_t w[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll
-                for (int c = 0; c < D; ++c) {
-                    const float4 qa = *reinterpret_cast<const float4 *>(&sm.qbt[c][tt0]);
-                    const float4 qb = *reinterpret_cast<const float4 *>(&sm.qbt[c][tt0 + 4]);
-                    acc[0] = fmaf(qa.x, kr[c], acc[0]);
-                    acc[1] = fmaf(qa.y, kr[c], acc[1]);
-                    acc[2] = fmaf(qa.z, kr[c], acc[2]);
-                    acc[3] = fmaf(qa.w, kr[c], acc[3]);
-                    acc[4] = fmaf(qb.x, kr[c], acc[4]);
-                    acc[5] = fmaf(qb.y, kr[c], acc[5]);
-                    acc[6] = fmaf(qb.z, kr[c], acc[6]);
-                    acc[7] = fmaf(qb.w, kr[c], acc[7]);
-                }
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    if (tt0 + i < nt) ds[(size_t)(tc + tt0 + i) * S.nk_pad] = acc[i];
-            }
-            __syncthreads();
-        }
+        for (int q = 0; q < 4; ++q)
+            w[q] = pack_e4m3x4(e4m3_quotient(x[4 * q][v], dv[v], inv[v]), e4m3_quotient(x[4 * q + 1][v], dv[v], inv[v]),
+                               e4m3_quotient(x[4 * q + 2][v], dv[v], inv[v]), e4m3_quotient(x[4 * q + 3][v], dv[v], inv[v]));
+        *reinterpret_cast<uint4 *>(vt8 + (size_t)v * S.nk_pad) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
 // ---------------------------------------------------------------------------
 template <int D>
-static cudaError_t launch_prepass_d(const PrepassArgs &a, int ds_t_skip, int causal_off, cudaStream_t stream) {
+static cudaError_t launch_prepass_d(const PrepassArgs &a, cudaStream_t stream) {
     const Shape &S = a.shape;
     if (a.k || a.v) {
         kv_stats_kernel<D><<<dim3(S.n_chunks, S.BH), 256, 0, stream>>>(a);
         kv_finalize_kernel<D><<<S.BH, D, 0, stream>>>(a);
     }
     if (a.q) quant_q_kernel<D><<<dim3(S.Tq, S.BH), 256, 0, stream>>>(a);
-    if (a.k || a.v) {
-        const size_t smem = sizeof(QuantKvSmem<D>);
-        cudaError_t e = cudaFuncSetAttribute(quant_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        quant_kv_kernel<D><<<dim3(S.Tk, S.BH), 256, smem, stream>>>(a, ds_t_skip, causal_off);
-    }
+    if (a.k) quant_k_kernel<D><<<dim3(S.Tk, S.BH), 256, 0, stream>>>(a);
+    if (a.v) quant_v_kernel<D><<<dim3(S.Tk, S.BH), 256, 0, stream>>>(a);
     return cudaGetLastError();
 }
 
-cudaError_t launch_prepass(const PrepassArgs &a, int ds_t_skip, int causal_off, cudaStream_t stream) {
-    if (a.shape.d == 128) return launch_prepass_d<128>(a, ds_t_skip, causal_off, stream);
-    return launch_prepass_d<64>(a, ds_t_skip, causal_off, stream);
+cudaError_t launch_prepass(const PrepassArgs &a, cudaStream_t stream) {
+    if (a.shape.d == 128) return launch_prepass_d<128>(a, stream);
+    return launch_prepass_d<64>(a, stream);
 }
 
 }  // namespace sage

@@ -103,6 +103,34 @@ bool make_maps(const Shape &s, const uint8_t *ws, CUtensorMap *tq, CUtensorMap *
     return true;
 }
 
+// Tensor map of the caller's 16-bit K for the dS product: [BH][n_kv][d] (head-major)
+// or [B][n_kv][H][d] (token-major), 64-element x 128-key boxes, 128-byte swizzle.
+// Keys past n_kv read as zero.
+bool make_k16_map(CUtensorMap *map, const void *k, int dtype, int layout, const Shape &s) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const CUtensorMapDataType dt =
+        (dtype == SAGE_DTYPE_BF16) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const uint64_t d = (uint64_t)s.d;
+    CUresult r;
+    if (layout == SAGE_LAYOUT_HND) {
+        cuuint64_t dims[3] = {d, (uint64_t)s.n_kv, (uint64_t)s.BH};
+        cuuint64_t strides[2] = {d * 2, (uint64_t)s.n_kv * d * 2};
+        cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        r = enc(map, dt, 3, const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        cuuint64_t dims[4] = {d, (uint64_t)s.H, (uint64_t)s.n_kv, (uint64_t)s.B};
+        cuuint64_t strides[3] = {d * 2, (uint64_t)s.H * d * 2, (uint64_t)s.n_kv * s.H * d * 2};
+        cuuint32_t box[4] = {64, 1, (cuuint32_t)kTile, 1};
+        cuuint32_t estr[4] = {1, 1, 1, 1};
+        r = enc(map, dt, 4, const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
+    return r == CUDA_SUCCESS;
+}
+
 sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype, int layout, const Shape &s,
                           const Mode &m, uint8_t *ws, int ds_t_skip, int causal_off, cudaStream_t stream) {
     PrepassArgs a;
@@ -120,7 +148,16 @@ sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype
     a.v_range = m.v_range;
     a.ws = ws;
     a.L = ws_layout(s);
-    return launch_prepass(a, ds_t_skip, causal_off, stream) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+    if (launch_prepass(a, stream) != cudaSuccess) return SAGE_ERR_CUDA;
+    if (k && m.smooth_q) {
+        CUtensorMap tmk;
+        if (!make_k16_map(&tmk, k, dtype, layout, s)) return SAGE_ERR_CUDA;
+        if (launch_ds_gemm(tmk, reinterpret_cast<const float *>(ws + a.L.qbar), reinterpret_cast<float *>(ws + a.L.ds),
+                           s, layout == SAGE_LAYOUT_NHD, dtype == SAGE_DTYPE_BF16, ds_t_skip, causal_off,
+                           reinterpret_cast<int *>(ws + a.L.status), stream) != cudaSuccess)
+            return SAGE_ERR_CUDA;
+    }
+    return SAGE_OK;
 }
 
 sage_status_t run_attention(void *o, int dtype, int layout, const Shape &s, int causal, float sm_scale,
