@@ -10,7 +10,8 @@
 // accumulated in fp32 tensor memory carries qbar to about 2^-17 relative for bf16
 // and 2^-22 for fp16.  tcgen05.mma kind::f16, M = 128 keys, N = up to 256 Q
 // blocks, K = 16 channels per instruction; D[key][block] in tensor memory, read
-// back by four warps and written as dS[block][key] (coalesced along keys).
+// back by eight warps (lane quadrant = warp % 4, alternate 32-column chunks by
+// warp / 4) and written as dS[block][key] (coalesced along keys).
 // Entries of Q blocks that can never see a key tile (causal) are not written.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -20,7 +21,7 @@
 
 namespace sage {
 
-constexpr int kDsThreads = 128;
+constexpr int kDsThreads = 256;
 constexpr int kDsTilesPerCta = 8;
 constexpr int kDsMaxN = 256;
 constexpr uint64_t kDsDrainNs = 50ull * 1000ull * 1000ull;
@@ -158,11 +159,12 @@ __global__ void __launch_bounds__(kDsThreads, 1)
                 t_lo = num <= 0 ? 0 : (num + kTile - 1) / kTile;
                 if (t_lo > Tq - 1) t_lo = Tq - 1;
             }
-            const int key = jt * kTile + warp * 32 + lane;
+            const int wq = warp & 3;
+            const int key = jt * kTile + wq * 32 + lane;
             float *dst = ds + (size_t)bh * Tq * nk_pad + key;
-            for (int c0 = 0; c0 < N; c0 += 32) {
+            for (int c0 = (warp >> 2) * 32; c0 < N; c0 += 64) {
                 uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
+                tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + c0, v);
                 tmem_wait_ld_regs(v);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {

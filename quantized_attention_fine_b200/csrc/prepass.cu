@@ -92,6 +92,11 @@ __device__ __forceinline__ void store_codes(int8_t *dst, const int8_t (&c)[VEC])
 
 }  // namespace
 
+// Quantization kernels: 16 warps per 128-row (or 128-key) tile, 8 rows per warp.
+constexpr int kQuantThreads = 512;
+constexpr int kQuantWarps = kQuantThreads / 32;
+constexpr int kRowsPerWarp = kTile / kQuantWarps;
+
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) kv_stats_kernel(const PrepassArgs a) {
@@ -161,9 +166,9 @@ __global__ void kv_finalize_kernel(const PrepassArgs a) {
 
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) quant_q_kernel(const PrepassArgs a) {
-    constexpr int VEC = D / 32, RPW = 16;
-    __shared__ double s_sum[8][D];
+__global__ void __launch_bounds__(kQuantThreads) quant_q_kernel(const PrepassArgs a) {
+    constexpr int VEC = D / 32, RPW = kRowsPerWarp;
+    __shared__ double s_sum[kQuantWarps][D];
     __shared__ float s_qbar[D];
     __shared__ float s_ramax[kTile];
     __shared__ float s_delta[kTile];
@@ -198,7 +203,7 @@ __global__ void __launch_bounds__(256) quant_q_kernel(const PrepassArgs a) {
         const int c = threadIdx.x;
         double s = 0.0;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) s = __dadd_rn(s, s_sum[w][c]);
+        for (int w = 0; w < kQuantWarps; ++w) s = __dadd_rn(s, s_sum[w][c]);
         const float qb = a.smooth_q ? (float)__ddiv_rn(s, (double)nvalid) : 0.f;
         s_qbar[c] = qb;
         reinterpret_cast<float *>(a.ws + a.L.qbar)[((size_t)bh * S.Tq + t) * D + c] = qb;
@@ -246,8 +251,8 @@ __global__ void __launch_bounds__(256) quant_q_kernel(const PrepassArgs a) {
 
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) quant_k_kernel(const PrepassArgs a) {
-    constexpr int VEC = D / 32, RPW = 16;
+__global__ void __launch_bounds__(kQuantThreads) quant_k_kernel(const PrepassArgs a) {
+    constexpr int VEC = D / 32, RPW = kRowsPerWarp;
     __shared__ float s_ramax[kTile];
     __shared__ float s_delta[kTile];
     const Shape &S = a.shape;
@@ -309,12 +314,12 @@ __global__ void __launch_bounds__(256) quant_k_kernel(const PrepassArgs a) {
     }
 }
 
-// V codes of one 128-key tile, written transposed: each lane holds 16 consecutive
-// keys of VEC channels and stores them as one 16-byte piece of each channel's row of
+// V codes of one 128-key tile, written transposed: each lane holds 8 consecutive
+// keys of VEC channels and stores them as one 8-byte piece of each channel's row of
 // V^T ([channel][key]).
 template <int D>
-__global__ void __launch_bounds__(256) quant_v_kernel(const PrepassArgs a) {
-    constexpr int VEC = D / 32, RPW = 16;
+__global__ void __launch_bounds__(kQuantThreads) quant_v_kernel(const PrepassArgs a) {
+    constexpr int VEC = D / 32, RPW = kRowsPerWarp;
     const Shape &S = a.shape;
     const int jt = blockIdx.x, bh = blockIdx.y;
     const int b = bh / S.H, h = bh % S.H;
@@ -340,14 +345,15 @@ __global__ void __launch_bounds__(256) quant_v_kernel(const PrepassArgs a) {
         }
     }
     uint8_t *vt8 = a.ws + a.L.vt8 + ((size_t)bh * D + lane * VEC) * S.nk_pad + j0 + warp * RPW;
+    static_assert(RPW == 8, "each lane stores 8 keys of a channel as one 8-byte piece");
 #pragma unroll
     for (int v = 0; v < VEC; ++v) {
-        uint32_t w[4];
+        uint32_t w[2];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 2; ++q)
             w[q] = pack_e4m3x4(e4m3_quotient(x[4 * q][v], dv[v], inv[v]), e4m3_quotient(x[4 * q + 1][v], dv[v], inv[v]),
                                e4m3_quotient(x[4 * q + 2][v], dv[v], inv[v]), e4m3_quotient(x[4 * q + 3][v], dv[v], inv[v]));
-        *reinterpret_cast<uint4 *>(vt8 + (size_t)v * S.nk_pad) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint2 *>(vt8 + (size_t)v * S.nk_pad) = make_uint2(w[0], w[1]);
     }
 }
 
@@ -359,9 +365,9 @@ static cudaError_t launch_prepass_d(const PrepassArgs &a, cudaStream_t stream) {
         kv_stats_kernel<D><<<dim3(S.n_chunks, S.BH), 256, 0, stream>>>(a);
         kv_finalize_kernel<D><<<S.BH, D, 0, stream>>>(a);
     }
-    if (a.q) quant_q_kernel<D><<<dim3(S.Tq, S.BH), 256, 0, stream>>>(a);
-    if (a.k) quant_k_kernel<D><<<dim3(S.Tk, S.BH), 256, 0, stream>>>(a);
-    if (a.v) quant_v_kernel<D><<<dim3(S.Tk, S.BH), 256, 0, stream>>>(a);
+    if (a.q) quant_q_kernel<D><<<dim3(S.Tq, S.BH), kQuantThreads, 0, stream>>>(a);
+    if (a.k) quant_k_kernel<D><<<dim3(S.Tk, S.BH), kQuantThreads, 0, stream>>>(a);
+    if (a.v) quant_v_kernel<D><<<dim3(S.Tk, S.BH), kQuantThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 
