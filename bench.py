@@ -202,9 +202,10 @@ def recorded_traffic(workload: str):
 def main():
     args = parse_args()
     from quantized_attention_fine_b200 import workloads as wl
-    if args.workload not in wl.WORKLOADS:
-        raise SystemExit("unknown workload %r (choices: %s)" % (args.workload, ", ".join(wl.WORKLOADS)))
-    w = wl.WORKLOADS[args.workload]
+    try:
+        w = wl.by_name(args.workload)
+    except KeyError as e:
+        raise SystemExit("%s (choices: %s, or sweep_n<N>_d<64|128>_<causal|full>)" % (e, ", ".join(wl.WORKLOADS)))
     if args.impl == "reference":
         return reference_arm(args, w)
 

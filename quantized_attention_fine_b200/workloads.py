@@ -60,6 +60,18 @@ def sweep_point(n: int, d: int, causal: bool) -> Workload:
                     torch.bfloat16, SEED_BASE + 4 + 1000 * (idx + 1), "sweep")
 
 
+def by_name(name: str) -> Workload:
+    """A named workload: one of WORKLOADS, or a sweep point 'sweep_n<N>_d<d>_<causal|full>'."""
+    if name in WORKLOADS:
+        return WORKLOADS[name]
+    if name.startswith("sweep_"):
+        parts = name.split("_")
+        n, d, kind = int(parts[1][1:]), int(parts[2][1:]), parts[3]
+        if n in SWEEP_N and d in (64, 128) and kind in ("causal", "full"):
+            return sweep_point(n, d, kind == "causal")
+    raise KeyError("unknown workload %r" % name)
+
+
 def custom(name, B, H, N_q, N_kv, d, causal, dtype=torch.bfloat16, seed=SEED_BASE + 99, recipe="image_dit"):
     """A workload with the value recipe of one of the families but other sizes (tests)."""
     return Workload(name, B, H, N_q, N_kv, d, causal, dtype, seed, recipe)
