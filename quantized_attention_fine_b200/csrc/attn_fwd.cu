@@ -56,7 +56,7 @@ struct __align__(1024) AttnSmem {
     uint8_t q[2][kTile * D];
     uint8_t k[ST][kTile * D];
     uint8_t v[ST][D * kTile];
-    uint8_t p[2][kTile * kTile];
+    uint8_t p[2][2][kTile * kTile];  // [Q tile][key tile parity]
     float ds[ST][2][kTile];
     float dk[ST][kTile / kKeyRun];
     uint64_t bar_q, bar_full[ST], bar_empty[ST], bar_s[2], bar_sfree[2], bar_p[2], bar_o[2], bar_drain;
@@ -149,7 +149,81 @@ __device__ __forceinline__ int kv_tiles_of(int t, int Tq, int Tk, int n_q, int o
 
 // ---------------------------------------------------------------------------
 // Softmax + epilogue of one Q tile (128 threads, one query row each).
+//
+// The row's work is software-pipelined across key tiles: while the exponentials
+// of tile `it` are taken (a 32-column chunk at a time), the scores of tile it + 1
+// are read from tensor memory and dequantized chunk by chunk, so the exponent
+// unit and the ALU / FMA pipes are fed from one instruction stream.  Chunk q of
+// the register array `sv` first holds tile it's dequantized scores, which the
+// exponentials consume, and is then refilled with tile it + 1's raw scores.
 // ---------------------------------------------------------------------------
+
+// s = S * dQ dK + dS over one 32-key chunk, in place (S int32 -> fp32 bits);
+// returns the chunk maximum.  Keys of a chunk form two runs of kKeyRun = 16 keys,
+// each with its own delta_K.
+__device__ __forceinline__ float dequant_chunk(uint32_t (&w)[32], float dq, float dk0, float dk1,
+                                               const float *ds) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float a = dq * (h ? dk1 : dk0);
+        const float2 a2 = make_float2(a, a);
+#pragma unroll
+        for (int j = 16 * h; j < 16 * h + 16; j += 4) {
+            const float4 d4 = *reinterpret_cast<const float4 *>(ds + j);
+            const float2 y01 = __ffma2_rn(make_float2((float)(int)w[j], (float)(int)w[j + 1]), a2, make_float2(d4.x, d4.y));
+            const float2 y23 =
+                __ffma2_rn(make_float2((float)(int)w[j + 2], (float)(int)w[j + 3]), a2, make_float2(d4.z, d4.w));
+            w[j] = __float_as_uint(y01.x);
+            w[j + 1] = __float_as_uint(y01.y);
+            w[j + 2] = __float_as_uint(y23.x);
+            w[j + 3] = __float_as_uint(y23.y);
+        }
+    }
+#define WV(j) __uint_as_float(w[j])
+    float t[10];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) t[i] = max3f(WV(3 * i), WV(3 * i + 1), WV(3 * i + 2));
+    const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]), u2 = max3f(t[6], t[7], t[8]);
+    const float u3 = max3f(t[9], WV(30), WV(31));
+#undef WV
+    return fmaxf(max3f(u0, u1, u2), u3);
+}
+
+// p = 2^(s c + bias) (bias = log2 Pr - m c) over one 32-key chunk: accumulates the
+// unquantized p into the row sum and packs Pr-scaled E4M3 codes, 4 per word.
+__device__ __forceinline__ void exp_chunk(const uint32_t (&w)[32], float2 c2, float2 b2, float2 &acc0, float2 &acc1,
+                                          uint32_t *pk) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+        const float2 e01 = __ffma2_rn(make_float2(__uint_as_float(w[j]), __uint_as_float(w[j + 1])), c2, b2);
+        const float2 e23 = __ffma2_rn(make_float2(__uint_as_float(w[j + 2]), __uint_as_float(w[j + 3])), c2, b2);
+        const float2 p01 = make_float2(ex2_approx(e01.x), ex2_approx(e01.y));
+        const float2 p23 = make_float2(ex2_approx(e23.x), ex2_approx(e23.y));
+        acc0 = __fadd2_rn(acc0, p01);
+        acc1 = __fadd2_rn(acc1, p23);
+        pk[j / 4] = pack_e4m3x4(p01.x, p01.y, p23.x, p23.y);
+    }
+}
+
+// Key tile `kt` has invisible keys in this row block: the key-count tail, or the
+// causal diagonal (key j visible to row i iff j <= i + off).
+__device__ __forceinline__ bool tile_masked(int kt, int t, int n_kv, int off, int causal) {
+    return (kt * kTile + kTile > n_kv) || (causal && kt * kTile + kTile - 1 > t * kTile + off);
+}
+
+// Sets the invisible keys of key tile kt to -inf and returns the new row maximum.
+__device__ __forceinline__ float mask_tile(uint32_t (&sv)[4][32], int kt, int row, int n_kv, int off, int causal) {
+    int lim = n_kv - 1 - kt * kTile;
+    if (causal) lim = min(lim, row + off - kt * kTile);
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kTile; ++j) {
+        if (j > lim) sv[j / 32][j % 32] = __float_as_uint(-INFINITY);
+        mx = fmaxf(mx, __uint_as_float(sv[j / 32][j % 32]));
+    }
+    return mx;
+}
+
 template <int D>
 __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &p, uint32_t tmem, int X, int t,
                                              int n_tiles, int bh, int64_t o_base, volatile int *abort_flag) {
@@ -175,101 +249,71 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
 
     const float dq = p.dq[(size_t)bh * p.nq_pad + row];
     const float c = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int it = 0; it < n_tiles; ++it) {
-        const int s = it % ST;
-        if (!warp_wait(&sm.bar_s[X], it & 1, abort_flag, p.status, kSiteS)) { ok = false; break; }
-        if (!warp_wait(&sm.bar_full[s], (it / ST) & 1, abort_flag, p.status, kSiteFull)) { ok = false; break; }
+    const float2 c2 = make_float2(c, c);
+    float m, l = 0.f, alpha = 1.f, bias;
+    uint32_t sv[4][32];
+
+    // prologue: scores of key tile 0
+    bool ok = warp_wait(&sm.bar_s[X], 0, abort_flag, p.status, kSiteS) &&
+              warp_wait(&sm.bar_full[0], 0, abort_flag, p.status, kSiteFull);
+    if (ok) {
         tc_fence_after();
-        uint32_t sv[4][32];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(s_tmem + q4 * 32, sv[q4]);
         tmem_wait_ld_regs(sv[0]);
         reg_fence(sv[1]);
         reg_fence(sv[2]);
         reg_fence(sv[3]);
-        // scores are in registers: the S buffer may take the next QK^T
         tc_fence_before();
         mbar_arrive(&sm.bar_sfree[X]);
+        float mx[4];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+            mx[q4] = dequant_chunk(sv[q4], dq, sm.dk[0][2 * q4], sm.dk[0][2 * q4 + 1], sm.ds[0][X] + 32 * q4);
+        m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        if (tile_masked(0, t, p.n_kv, off, p.causal)) m = mask_tile(sv, 0, row, p.n_kv, off, p.causal);
+        bias = (m == -INFINITY) ? 0.f : p.log2_pr - m * c;
+    }
 
-        const float *ds = sm.ds[s][X];
-        const bool masked = (it * kTile + kTile > p.n_kv) || (p.causal && it * kTile + kTile - 1 > t * kTile + off);
-        // s = S * dQ dK + dS, in place over the score registers
-#pragma unroll
-        for (int g = 0; g < kTile / kKeyRun; ++g) {
-            const float a = dq * sm.dk[s][g];
-            const float2 a2 = make_float2(a, a);
-#pragma unroll
-            for (int j = g * kKeyRun; j < (g + 1) * kKeyRun; j += 4) {
-                uint32_t *w = &sv[j / 32][j % 32];
-                const float4 d4 = p.use_ds ? *reinterpret_cast<const float4 *>(ds + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-                const float2 y01 = __ffma2_rn(make_float2((float)(int)w[0], (float)(int)w[1]), a2, make_float2(d4.x, d4.y));
-                const float2 y23 = __ffma2_rn(make_float2((float)(int)w[2], (float)(int)w[3]), a2, make_float2(d4.z, d4.w));
-                w[0] = __float_as_uint(y01.x);
-                w[1] = __float_as_uint(y01.y);
-                w[2] = __float_as_uint(y23.x);
-                w[3] = __float_as_uint(y23.y);
-            }
+    for (int it = 0; ok && it < n_tiles; ++it) {
+        const bool has_next = it + 1 < n_tiles;
+        const int sn = (it + 1) % ST;
+        if (has_next) {
+            if (!warp_wait(&sm.bar_s[X], (it + 1) & 1, abort_flag, p.status, kSiteS)) { ok = false; break; }
+            if (!warp_wait(&sm.bar_full[sn], ((it + 1) / ST) & 1, abort_flag, p.status, kSiteFull)) { ok = false; break; }
+            tc_fence_after();
         }
-#define SV(j) __uint_as_float(sv[(j) / 32][(j) % 32])
-        if (masked) {
-            // key it*128 + j is visible iff j <= lim (the key-count tail and the causal diagonal)
-            int lim = p.n_kv - 1 - it * kTile;
-            if (p.causal) lim = min(lim, row + off - it * kTile);
-#pragma unroll
-            for (int j = 0; j < kTile; ++j)
-                if (j > lim) sv[j / 32][j % 32] = __float_as_uint(-INFINITY);
-        }
-        float mx[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int b0 = 16 * u;
-            const float a0 = max3f(SV(b0), SV(b0 + 1), SV(b0 + 2));
-            const float a1 = max3f(SV(b0 + 3), SV(b0 + 4), SV(b0 + 5));
-            const float a2 = max3f(SV(b0 + 6), SV(b0 + 7), SV(b0 + 8));
-            const float a3 = max3f(SV(b0 + 9), SV(b0 + 10), SV(b0 + 11));
-            const float a4 = max3f(SV(b0 + 12), SV(b0 + 13), SV(b0 + 14));
-            mx[u] = max3f(max3f(a0, a1, a2), a3, max3f(a4, SV(b0 + 15), -INFINITY));
-        }
-        const float tmax = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-        const float m_new = fmaxf(m, tmax);
-        float alpha, bias;
-        if (m_new == -INFINITY) {
-            alpha = 1.f;
-            bias = 0.f;
-        } else {
-            alpha = ex2_approx((m - m_new) * c);
-            bias = p.log2_pr - m_new * c;
-        }
-        const float2 c2 = make_float2(c, c), b2 = make_float2(bias, bias);
+        // exponentials of tile it, interleaved with the scores of tile it + 1 (on the
+        // last tile the reads only see stale, unused values of this warp's own lanes)
+        const float2 b2 = make_float2(bias, bias);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-        uint32_t pk[kTile / 4];
+        float mx[4];
+        const float *dsn = sm.ds[sn][X];
+        const float *dkn = sm.dk[sn];
+        // P(it) goes to the buffer PV(it - 2) read; that PV was waited for before P(it - 1)
+        uint8_t *pbuf = sm.p[X][it & 1];
 #pragma unroll
-        for (int j = 0; j < kTile; j += 4) {
-            const float2 e01 = __ffma2_rn(make_float2(SV(j), SV(j + 1)), c2, b2);
-            const float2 e23 = __ffma2_rn(make_float2(SV(j + 2), SV(j + 3)), c2, b2);
-            const float2 p01 = make_float2(ex2_approx(e01.x), ex2_approx(e01.y));
-            const float2 p23 = make_float2(ex2_approx(e23.x), ex2_approx(e23.y));
-            acc0 = __fadd2_rn(acc0, p01);
-            acc1 = __fadd2_rn(acc1, p23);
-            pk[j / 4] = pack_e4m3x4(p01.x, p01.y, p23.x, p23.y);
+        for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t pk[8];
+            exp_chunk(sv[q4], c2, b2, acc0, acc1, pk);
+            *reinterpret_cast<uint4 *>(pbuf + sw128_offset(r, 2 * q4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4 *>(pbuf + sw128_offset(r, 2 * q4 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            tmem_ld32(s_tmem + q4 * 32, sv[q4]);
+            tmem_wait_ld_regs(sv[q4]);
+            mx[q4] = dequant_chunk(sv[q4], dq, dkn[2 * q4], dkn[2 * q4 + 1], dsn + 32 * q4);
         }
-#undef SV
+        if (has_next) {  // tile it + 1's scores are in registers: its S buffer may take the next QK^T
+            tc_fence_before();
+            mbar_arrive(&sm.bar_sfree[X]);
+        }
         const float2 acc = __fadd2_rn(acc0, acc1);
         l = l * alpha + (acc.x + acc.y);
         const bool rescale = (it > 0) && (alpha != 1.f);
-        m = m_new;
 
-        if (it > 0) {  // PV of the previous tile must be done before P and O are touched
+        if (it > 0) {  // PV of the previous tile must be done before O is rescaled
             if (!warp_wait(&sm.bar_o[X], (it - 1) & 1, abort_flag, p.status, kSiteO)) { ok = false; break; }
             tc_fence_after();
         }
-        uint8_t *pbuf = sm.p[X];
-#pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16)
-            *reinterpret_cast<uint4 *>(pbuf + sw128_offset(r, c16)) =
-                make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
         if (__any_sync(0xFFFFFFFFu, rescale)) {
             const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
@@ -290,6 +334,20 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sm.bar_p[X]);
+
+        if (has_next) {  // running maximum with tile it + 1
+            float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            if (tile_masked(it + 1, t, p.n_kv, off, p.causal)) tmax = mask_tile(sv, it + 1, row, p.n_kv, off, p.causal);
+            const float m_new = fmaxf(m, tmax);
+            if (m_new == -INFINITY) {
+                alpha = 1.f;
+                bias = 0.f;
+            } else {
+                alpha = ex2_approx((m - m_new) * c);
+                bias = p.log2_pr - m_new * c;
+            }
+            m = m_new;
+        }
     }
     if (ok) ok = warp_wait(&sm.bar_o[X], (n_tiles - 1) & 1, abort_flag, p.status, kSiteO);
     if (ok) {
@@ -352,6 +410,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         sm.abort_flag = 0;
         fence_mbar_init();
     }
+    if (!p.use_ds) {  // without Q smoothing the dS rows stay zero
+        float *z = &sm.ds[0][0][0];
+        for (int i = threadIdx.x; i < ST * 2 * kTile; i += kAttnThreads) z[i] = 0.f;
+    }
     if (warp == 9 && n_tiles > 0) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
@@ -400,41 +462,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
         } else if (warp == 9 && lane == 0 && n_tiles > 0) {
             // ------------------------------ MMA issuer ------------------------------
-            const uint32_t q_s[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
-            const uint32_t p_s[2] = {smem_u32(sm.p[0]), smem_u32(sm.p[1])};
-            const int nX[2] = {nA, nB};
+            // Q tile x at q_s + x * kTile * D; P buffer (x, parity) at p_s + (2 x + parity) * kTile^2
+            const uint32_t q_s = smem_u32(sm.q[0]), p_s = smem_u32(sm.p[0][0]);
             bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, p.status, kSiteQ);
             if (ok) ok = mbar_wait(&sm.bar_full[0], 0, abort_flag, p.status, kSiteFull);
             if (ok) {
                 tc_fence_after();
                 for (int x = 0; x < 2; ++x)
-                    if (nX[x] > 0) {
-                        issue_qk<D>(tmem + (uint32_t)x * 128u, q_s[x], smem_u32(sm.k[0]));
+                    if ((x ? nB : nA) > 0) {
+                        issue_qk<D>(tmem + (uint32_t)x * 128u, q_s + (uint32_t)x * (kTile * D), smem_u32(sm.k[0]));
                         mma_commit(&sm.bar_s[x]);
                     }
             }
-            for (int it = 0; ok && it < n_tiles; ++it) {
-                const int s = it % ST;
-                if (it + 1 < n_tiles) {
-                    const int s1 = (it + 1) % ST;
-                    if (!mbar_wait(&sm.bar_full[s1], ((it + 1) / ST) & 1, abort_flag, p.status, kSiteFull)) break;
-                    bool brk = false;
-                    for (int x = 0; x < 2; ++x) {
-                        if (it + 1 >= nX[x]) continue;
-                        if (!mbar_wait(&sm.bar_sfree[x], it & 1, abort_flag, p.status, kSiteSfree)) { brk = true; break; }
+            // QK^T of key tile 1 as soon as a warpgroup holds tile 0's scores
+            if (ok && n_tiles > 1) {
+                ok = mbar_wait(&sm.bar_full[1 % ST], (1 / ST) & 1, abort_flag, p.status, kSiteFull);
+                for (int x = 0; ok && x < 2; ++x)
+                    if ((x ? nB : nA) > 1) {
+                        ok = mbar_wait(&sm.bar_sfree[x], 0, abort_flag, p.status, kSiteSfree);
+                        if (!ok) break;
                         tc_fence_after();
-                        issue_qk<D>(tmem + (uint32_t)x * 128u, q_s[x], smem_u32(sm.k[s1]));
+                        issue_qk<D>(tmem + (uint32_t)x * 128u, q_s + (uint32_t)x * (kTile * D), smem_u32(sm.k[1 % ST]));
                         mma_commit(&sm.bar_s[x]);
                     }
-                    if (brk) break;
-                }
+            }
+            // Steady state, per key tile it and Q tile x: QK^T of tile it + 2 once x's
+            // warpgroup holds tile it + 1's scores, then PV of tile it once its P is in
+            // shared memory (a warpgroup releases the two close together).
+            for (int it = 0; ok && it < n_tiles; ++it) {
+                const int s = it % ST, s2 = (it + 2) % ST;
+                if (it + 2 < n_tiles && !mbar_wait(&sm.bar_full[s2], ((it + 2) / ST) & 1, abort_flag, p.status, kSiteFull))
+                    break;
                 bool brk = false;
                 for (int x = 0; x < 2; ++x) {
-                    if (it >= nX[x]) continue;
-                    if (!mbar_wait(&sm.bar_p[x], it & 1, abort_flag, p.status, kSiteP)) { brk = true; break; }
-                    tc_fence_after();
-                    issue_pv<D>(tmem + kTmemO + (uint32_t)x * D, p_s[x], smem_u32(sm.v[s]), it > 0);
-                    mma_commit(&sm.bar_o[x]);
+                    if (it + 2 < (x ? nB : nA)) {
+                        if (!mbar_wait(&sm.bar_sfree[x], (it + 1) & 1, abort_flag, p.status, kSiteSfree)) { brk = true; break; }
+                        tc_fence_after();
+                        issue_qk<D>(tmem + (uint32_t)x * 128u, q_s + (uint32_t)x * (kTile * D), smem_u32(sm.k[s2]));
+                        mma_commit(&sm.bar_s[x]);
+                    }
+                    if (it < (x ? nB : nA)) {
+                        if (!mbar_wait(&sm.bar_p[x], it & 1, abort_flag, p.status, kSiteP)) { brk = true; break; }
+                        tc_fence_after();
+                        issue_pv<D>(tmem + kTmemO + (uint32_t)x * D, p_s + (uint32_t)(2 * x + (it & 1)) * (kTile * kTile), smem_u32(sm.v[s]), it > 0);
+                        mma_commit(&sm.bar_o[x]);
+                    }
                 }
                 if (brk) break;
                 mma_commit(&sm.bar_empty[s]);
