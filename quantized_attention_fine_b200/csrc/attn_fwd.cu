@@ -158,6 +158,17 @@ __device__ __forceinline__ int kv_tiles_of(int t, int Tq, int Tk, int n_q, int o
 // exponentials consume, and is then refilled with tile it + 1's raw scores.
 // ---------------------------------------------------------------------------
 
+// dS read from shared memory as inline asm, so the compiler keeps it behind the
+// tensor-memory wait of its chunk instead of hoisting a whole tile's dS into
+// registers (which would not fit beside the 128 score registers).
+__device__ __forceinline__ float4 lds_f32x4(const float *ptr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(smem_u32(ptr)));
+    return v;
+}
+
 // s = S * dQ dK + dS over one 32-key chunk, in place (S int32 -> fp32 bits);
 // returns the chunk maximum.  Keys of a chunk form two runs of kKeyRun = 16 keys,
 // each with its own delta_K.
@@ -169,7 +180,7 @@ __device__ __forceinline__ float dequant_chunk(uint32_t (&w)[32], float dq, floa
         const float2 a2 = make_float2(a, a);
 #pragma unroll
         for (int j = 16 * h; j < 16 * h + 16; j += 4) {
-            const float4 d4 = *reinterpret_cast<const float4 *>(ds + j);
+            const float4 d4 = lds_f32x4(ds + j);
             const float2 y01 = __ffma2_rn(make_float2((float)(int)w[j], (float)(int)w[j + 1]), a2, make_float2(d4.x, d4.y));
             const float2 y23 =
                 __ffma2_rn(make_float2((float)(int)w[j + 2], (float)(int)w[j + 3]), a2, make_float2(d4.z, d4.w));
@@ -317,17 +328,17 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
         if (__any_sync(0xFFFFFFFFu, rescale)) {
             const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t ov[32];
-                tmem_ld32(o_tmem + c0, ov);
-                tmem_wait_ld_regs(ov);
+            for (int c0 = 0; c0 < D; c0 += 16) {  // 16 columns at a time: the next tile's scores stay live
+                uint32_t ov[16];
+                tmem_ld16(o_tmem + c0, ov);
+                tmem_wait_ld_regs16(ov);
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
+                for (int i = 0; i < 16; i += 2) {
                     const float2 v2 = __fmul2_rn(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])), al2);
                     ov[i] = __float_as_uint(v2.x);
                     ov[i + 1] = __float_as_uint(v2.y);
                 }
-                tmem_st32(o_tmem + c0, ov);
+                tmem_st16(o_tmem + c0, ov);
             }
             tmem_wait_st();
         }
