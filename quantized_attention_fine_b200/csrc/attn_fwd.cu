@@ -12,15 +12,17 @@
 // every K / V^T tile between them (384 threads, 12 warps):
 //   warps 0-3   softmax + epilogue of tile A (thread i owns row i = TMEM lane i)
 //   warps 4-7   softmax + epilogue of tile B
-//   warp 8      TMA producer: Q tiles once, then K, V^T, dS (per tile) and
-//               delta_K runs through a shared-memory ring
+//   warp 8      TMA producer: Q tiles once, then K tiles with their dS rows and
+//               delta_K runs through one shared-memory ring
 //   warp 9      tensor-memory allocation and single-thread tcgen05.mma issue
-//   warps 10-11 idle (they only give the producer warpgroup its register share)
+//   warp 10     TMA producer of the V^T ring
+//   warp 11     idle (it only completes the producer warpgroup)
 // Tensor memory (512 columns): S_A 0-127, S_B 128-255 (int32), O_A 256.., O_B
 // 256 + d.. (fp32).  A softmax warpgroup releases its S buffer as soon as the
-// scores are in registers, so QK^T of the next key tile runs on the tensor core
-// while the current one is being exponentiated, and the two warpgroups alternate
-// on the tensor core (QK_A, QK_B, PV_A, PV_B per key tile).
+// scores of key tile i + 1 are in registers (it reads them while exponentiating
+// tile i), so QK^T of tile i + 2 runs on the tensor core during the softmax of
+// tile i + 1; the MMA issuer serves the warpgroups in turn with the pair
+// (QK^T of tile i + 2, PV of tile i).  P is double-buffered per warpgroup.
 // Every wait is bounded: a wait that runs out records SAGE_ERR_TIMEOUT in the
 // status block, raises a CTA-wide abort flag that makes every role leave its loop,
 // drains the copies in flight, frees tensor memory and exits.
@@ -45,21 +47,27 @@ constexpr uint32_t kRegsSoftmax = 232;
 // Wait-site ids recorded with a timeout.
 enum { kSiteQ = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteS = 4, kSiteP = 5, kSiteO = 6, kSiteSfree = 7, kSiteDebug = 9 };
 
+// K tiles (with their dS rows and delta_K runs) and V^T tiles travel in separate
+// rings: a K slot is free once QK^T has read it and both warpgroups have
+// dequantized with its dS / delta_K, long before PV is done with the V^T tile of
+// the same key tile, so the K ring can run further ahead.
 template <int D>
 struct AttnCfg {
-    static constexpr int kStages = (D == 128) ? 3 : 4;
+    static constexpr int kKStages = 4;
+    static constexpr int kVStages = (D == 128) ? 3 : 4;
 };
 
 template <int D>
 struct __align__(1024) AttnSmem {
-    static constexpr int ST = AttnCfg<D>::kStages;
+    static constexpr int KS = AttnCfg<D>::kKStages, VS = AttnCfg<D>::kVStages;
     uint8_t q[2][kTile * D];
-    uint8_t k[ST][kTile * D];
-    uint8_t v[ST][D * kTile];
+    uint8_t k[KS][kTile * D];
+    uint8_t v[VS][D * kTile];
     uint8_t p[2][2][kTile * kTile];  // [Q tile][key tile parity]
-    float ds[ST][2][kTile];
-    float dk[ST][kTile / kKeyRun];
-    uint64_t bar_q, bar_full[ST], bar_empty[ST], bar_s[2], bar_sfree[2], bar_p[2], bar_o[2], bar_drain;
+    float ds[KS][2][kTile];
+    float dk[KS][kTile / kKeyRun];
+    uint64_t bar_q, bar_kfull[KS], bar_kempty[KS], bar_vfull[VS], bar_vempty[VS];
+    uint64_t bar_s[2], bar_sfree[2], bar_p[2], bar_o[2], bar_drain;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -238,7 +246,7 @@ __device__ __forceinline__ float mask_tile(uint32_t (&sv)[4][32], int kt, int ro
 template <int D>
 __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &p, uint32_t tmem, int X, int t,
                                              int n_tiles, int bh, int64_t o_base, volatile int *abort_flag) {
-    constexpr int ST = AttnCfg<D>::kStages;
+    constexpr int KS = AttnCfg<D>::kKStages;
     const int wq = (threadIdx.x >> 5) & 3;
     const int lane = threadIdx.x & 31;
     const int r = wq * 32 + lane;
@@ -266,7 +274,7 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
 
     // prologue: scores of key tile 0
     bool ok = warp_wait(&sm.bar_s[X], 0, abort_flag, p.status, kSiteS) &&
-              warp_wait(&sm.bar_full[0], 0, abort_flag, p.status, kSiteFull);
+              warp_wait(&sm.bar_kfull[0], 0, abort_flag, p.status, kSiteFull);
     if (ok) {
         tc_fence_after();
 #pragma unroll
@@ -288,10 +296,10 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
 
     for (int it = 0; ok && it < n_tiles; ++it) {
         const bool has_next = it + 1 < n_tiles;
-        const int sn = (it + 1) % ST;
+        const int sn = (it + 1) % KS;
         if (has_next) {
             if (!warp_wait(&sm.bar_s[X], (it + 1) & 1, abort_flag, p.status, kSiteS)) { ok = false; break; }
-            if (!warp_wait(&sm.bar_full[sn], ((it + 1) / ST) & 1, abort_flag, p.status, kSiteFull)) { ok = false; break; }
+            if (!warp_wait(&sm.bar_kfull[sn], ((it + 1) / KS) & 1, abort_flag, p.status, kSiteFull)) { ok = false; break; }
             tc_fence_after();
         }
         // exponentials of tile it, interleaved with the scores of tile it + 1 (on the
@@ -388,7 +396,7 @@ template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
-    constexpr int ST = AttnCfg<D>::kStages;
+    constexpr int KS = AttnCfg<D>::kKStages, VS = AttnCfg<D>::kVStages;
     extern __shared__ uint8_t smem_raw[];
     AttnSmem<D> &sm =
         *reinterpret_cast<AttnSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -410,7 +418,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_q, 1);
-        for (int s = 0; s < ST; ++s) { mbar_init(&sm.bar_full[s], 1); mbar_init(&sm.bar_empty[s], 1); }
+        for (int s = 0; s < KS; ++s) { mbar_init(&sm.bar_kfull[s], 1); mbar_init(&sm.bar_kempty[s], 1); }
+        for (int s = 0; s < VS; ++s) { mbar_init(&sm.bar_vfull[s], 1); mbar_init(&sm.bar_vempty[s], 1); }
         for (int x = 0; x < 2; ++x) {
             mbar_init(&sm.bar_s[x], 1);
             mbar_init(&sm.bar_sfree[x], 128);
@@ -423,7 +432,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     if (!p.use_ds) {  // without Q smoothing the dS rows stay zero
         float *z = &sm.ds[0][0][0];
-        for (int i = threadIdx.x; i < ST * 2 * kTile; i += kAttnThreads) z[i] = 0.f;
+        for (int i = threadIdx.x; i < KS * 2 * kTile; i += kAttnThreads) z[i] = 0.f;
     }
     if (warp == 9 && n_tiles > 0) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -438,10 +447,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (warp >= 8) {
         setmaxnreg_dec<kRegsProducer>();
         if (warp == 8 && lane == 0 && n_tiles > 0) {
-            // ------------------------------ TMA producer ------------------------------
+            // ---------------- TMA producer: Q tiles, then the K / dS / delta_K ring ----------------
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
             mbar_arrive_expect_tx(&sm.bar_q, (hasB ? 2 : 1) * kTile * D);
             tma_load_2d(sm.q[0], &tm_q, &sm.bar_q, 0, bh * p.nq_pad + tA * kTile);
             if (hasB) tma_load_2d(sm.q[1], &tm_q, &sm.bar_q, 0, bh * p.nq_pad + tB * kTile);
@@ -450,33 +458,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float *dk_row = p.dk + (size_t)bh * (p.nk_pad / kKeyRun);
             int issued = 0;
             for (int it = 0; it < n_tiles; ++it) {
-                const int s = it % ST;
-                if (it >= ST && !mbar_wait(&sm.bar_empty[s], ((it / ST) & 1) ^ 1, abort_flag, p.status, kSiteEmpty))
+                const int s = it % KS;
+                if (it >= KS && !mbar_wait(&sm.bar_kempty[s], ((it / KS) & 1) ^ 1, abort_flag, p.status, kSiteEmpty))
                     break;
                 issued = it + 1;
-                if (p.fault_inject && it == 0) continue;  // diagnostic: leave stage 0 unsignalled
+                if (p.fault_inject && it == 0) continue;  // diagnostic: leave slot 0 unsignalled
                 const bool dsA = p.use_ds && it < nA, dsB = p.use_ds && it < nB;
-                const uint32_t bytes = kTile * D * 2 + (dsA ? kTile * 4 : 0) + (dsB ? kTile * 4 : 0) + (kTile / kKeyRun) * 4;
-                mbar_arrive_expect_tx(&sm.bar_full[s], bytes);
-                tma_load_2d(sm.k[s], &tm_k, &sm.bar_full[s], 0, bh * p.nk_pad + it * kTile);
-                tma_load_2d(sm.v[s], &tm_v, &sm.bar_full[s], it * kTile, bh * D);
-                if (dsA) bulk_load(sm.ds[s][0], ds_a + it * kTile, kTile * 4, &sm.bar_full[s]);
-                if (dsB) bulk_load(sm.ds[s][1], ds_b + it * kTile, kTile * 4, &sm.bar_full[s]);
-                bulk_load(sm.dk[s], dk_row + it * (kTile / kKeyRun), (kTile / kKeyRun) * 4, &sm.bar_full[s]);
+                const uint32_t bytes = kTile * D + (dsA ? kTile * 4 : 0) + (dsB ? kTile * 4 : 0) + (kTile / kKeyRun) * 4;
+                mbar_arrive_expect_tx(&sm.bar_kfull[s], bytes);
+                tma_load_2d(sm.k[s], &tm_k, &sm.bar_kfull[s], 0, bh * p.nk_pad + it * kTile);
+                if (dsA) bulk_load(sm.ds[s][0], ds_a + it * kTile, kTile * 4, &sm.bar_kfull[s]);
+                if (dsB) bulk_load(sm.ds[s][1], ds_b + it * kTile, kTile * 4, &sm.bar_kfull[s]);
+                bulk_load(sm.dk[s], dk_row + it * (kTile / kKeyRun), (kTile / kKeyRun) * 4, &sm.bar_kfull[s]);
             }
             if (*abort_flag) {  // let the copies in flight land before the CTA exits
                 mbar_wait_quiet(&sm.bar_q, 0, kDrainNs);
-                for (int it = max(0, issued - ST); it < issued; ++it) {
+                for (int it = max(0, issued - KS); it < issued; ++it) {
                     if (p.fault_inject && it == 0) continue;
-                    mbar_wait_quiet(&sm.bar_full[it % ST], (it / ST) & 1, kDrainNs);
+                    mbar_wait_quiet(&sm.bar_kfull[it % KS], (it / KS) & 1, kDrainNs);
                 }
             }
+        } else if (warp == 10 && lane == 0 && n_tiles > 0) {
+            // ---------------- TMA producer: the V^T ring ----------------
+            prefetch_tmap(&tm_v);
+            int issued = 0;
+            for (int it = 0; it < n_tiles; ++it) {
+                const int s = it % VS;
+                if (it >= VS && !mbar_wait(&sm.bar_vempty[s], ((it / VS) & 1) ^ 1, abort_flag, p.status, kSiteEmpty))
+                    break;
+                issued = it + 1;
+                mbar_arrive_expect_tx(&sm.bar_vfull[s], kTile * D);
+                tma_load_2d(sm.v[s], &tm_v, &sm.bar_vfull[s], it * kTile, bh * D);
+            }
+            if (*abort_flag)
+                for (int it = max(0, issued - VS); it < issued; ++it)
+                    mbar_wait_quiet(&sm.bar_vfull[it % VS], (it / VS) & 1, kDrainNs);
         } else if (warp == 9 && lane == 0 && n_tiles > 0) {
             // ------------------------------ MMA issuer ------------------------------
             // Q tile x at q_s + x * kTile * D; P buffer (x, parity) at p_s + (2 x + parity) * kTile^2
             const uint32_t q_s = smem_u32(sm.q[0]), p_s = smem_u32(sm.p[0][0]);
             bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, p.status, kSiteQ);
-            if (ok) ok = mbar_wait(&sm.bar_full[0], 0, abort_flag, p.status, kSiteFull);
+            if (ok) ok = mbar_wait(&sm.bar_kfull[0], 0, abort_flag, p.status, kSiteFull);
             if (ok) {
                 tc_fence_after();
                 for (int x = 0; x < 2; ++x)
@@ -485,42 +507,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         mma_commit(&sm.bar_s[x]);
                     }
             }
-            // QK^T of key tile 1 as soon as a warpgroup holds tile 0's scores
-            if (ok && n_tiles > 1) {
-                ok = mbar_wait(&sm.bar_full[1 % ST], (1 / ST) & 1, abort_flag, p.status, kSiteFull);
-                for (int x = 0; ok && x < 2; ++x)
-                    if ((x ? nB : nA) > 1) {
-                        ok = mbar_wait(&sm.bar_sfree[x], 0, abort_flag, p.status, kSiteSfree);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_qk<D>(tmem + (uint32_t)x * 128u, q_s + (uint32_t)x * (kTile * D), smem_u32(sm.k[1 % ST]));
-                        mma_commit(&sm.bar_s[x]);
-                    }
+            // QK^T of key tile 1 as soon as a warpgroup holds tile 0's scores; K slot 0
+            // is released once both warpgroups have dequantized tile 0
+            if (ok && n_tiles > 1) ok = mbar_wait(&sm.bar_kfull[1 % KS], (1 / KS) & 1, abort_flag, p.status, kSiteFull);
+            for (int x = 0; ok && x < 2; ++x) {
+                const int nx = x ? nB : nA;
+                if (nx <= 0) continue;
+                ok = mbar_wait(&sm.bar_sfree[x], 0, abort_flag, p.status, kSiteSfree);
+                if (ok && nx > 1) {
+                    tc_fence_after();
+                    issue_qk<D>(tmem + (uint32_t)x * 128u, q_s + (uint32_t)x * (kTile * D), smem_u32(sm.k[1 % KS]));
+                    mma_commit(&sm.bar_s[x]);
+                }
             }
+            if (ok) mma_commit(&sm.bar_kempty[0]);
             // Steady state, per key tile it and Q tile x: QK^T of tile it + 2 once x's
             // warpgroup holds tile it + 1's scores, then PV of tile it once its P is in
             // shared memory (a warpgroup releases the two close together).
             for (int it = 0; ok && it < n_tiles; ++it) {
-                const int s = it % ST, s2 = (it + 2) % ST;
-                if (it + 2 < n_tiles && !mbar_wait(&sm.bar_full[s2], ((it + 2) / ST) & 1, abort_flag, p.status, kSiteFull))
+                const int k1 = (it + 1) % KS, k2 = (it + 2) % KS, sv = it % VS;
+                if (it + 2 < n_tiles && !mbar_wait(&sm.bar_kfull[k2], ((it + 2) / KS) & 1, abort_flag, p.status, kSiteFull))
                     break;
-                bool brk = false;
+                bool brk = false, v_ready = false;
                 for (int x = 0; x < 2; ++x) {
-                    if (it + 2 < (x ? nB : nA)) {
+                    const int nx = x ? nB : nA;
+                    if (it + 1 < nx) {
                         if (!mbar_wait(&sm.bar_sfree[x], (it + 1) & 1, abort_flag, p.status, kSiteSfree)) { brk = true; break; }
-                        tc_fence_after();
-                        issue_qk<D>(tmem + (uint32_t)x * 128u, q_s + (uint32_t)x * (kTile * D), smem_u32(sm.k[s2]));
-                        mma_commit(&sm.bar_s[x]);
+                        if (it + 2 < nx) {
+                            tc_fence_after();
+                            issue_qk<D>(tmem + (uint32_t)x * 128u, q_s + (uint32_t)x * (kTile * D), smem_u32(sm.k[k2]));
+                            mma_commit(&sm.bar_s[x]);
+                        }
                     }
-                    if (it < (x ? nB : nA)) {
+                    if (it < nx) {
+                        if (!v_ready) {
+                            if (!mbar_wait(&sm.bar_vfull[sv], (it / VS) & 1, abort_flag, p.status, kSiteFull)) { brk = true; break; }
+                            v_ready = true;
+                        }
                         if (!mbar_wait(&sm.bar_p[x], it & 1, abort_flag, p.status, kSiteP)) { brk = true; break; }
                         tc_fence_after();
-                        issue_pv<D>(tmem + kTmemO + (uint32_t)x * D, p_s + (uint32_t)(2 * x + (it & 1)) * (kTile * kTile), smem_u32(sm.v[s]), it > 0);
+                        issue_pv<D>(tmem + kTmemO + (uint32_t)x * D, p_s + (uint32_t)(2 * x + (it & 1)) * (kTile * kTile),
+                                    smem_u32(sm.v[sv]), it > 0);
                         mma_commit(&sm.bar_o[x]);
                     }
                 }
                 if (brk) break;
-                mma_commit(&sm.bar_empty[s]);
+                if (it + 1 < n_tiles) mma_commit(&sm.bar_kempty[k1]);  // tile it + 1 dequantized by both warpgroups
+                mma_commit(&sm.bar_vempty[sv]);                         // once PV(it) has read V^T(it)
             }
             mma_commit(&sm.bar_drain);
             mbar_wait_quiet(&sm.bar_drain, 0, kDrainNs);
