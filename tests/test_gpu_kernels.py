@@ -232,6 +232,28 @@ def test_repeated_calls_deterministic():
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("nq,d,causal,H", [(8192, 128, True, 8), (4096, 64, False, 16)])
+def test_long_sequences_deterministic(nq, d, causal, H):
+    """Many key tiles per CTA and every SM busy: a synchronization race between the
+    kernel's roles (a buffer reused before its reader is done) would show up as
+    run-to-run differences, since the outcome would depend on timing."""
+    w = wl.custom("det_long", 1, H, nq, nq, d, causal, recipe="llm" if causal else "image_dit")
+    q, k, v = (x.cuda() for x in wl.generate(w))
+    mode = sage.QuantMode.make()
+    ws = sage.make_workspace(1, H, nq, nq, d)
+    sage.quant_qk(q, k, mode=mode, workspace=ws)
+    sage.quant_v(v, n_q=nq, mode=mode, workspace=ws)
+    outs = []
+    for _ in range(4):
+        o = torch.empty_like(q)
+        sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=causal, mode=mode, out=o)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert sage.get_device_status(ws) == (0, 0)
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+
+
 def test_empty_and_keyless_inputs():
     d = 64
     q = torch.randn(1, 2, 100, d, dtype=torch.bfloat16, device="cuda")
