@@ -9,10 +9,11 @@
 //     dS = K . hi^T + K . lo^T
 // accumulated in fp32 tensor memory carries qbar to about 2^-17 relative for bf16
 // and 2^-22 for fp16.  tcgen05.mma kind::f16, M = 128 keys, N = up to 256 Q
-// blocks, K = 16 channels per instruction; D[key][block] in tensor memory, read
-// back by eight warps (lane quadrant = warp % 4, alternate 32-column chunks by
-// warp / 4) and written as dS[block][key] (coalesced along keys).
-// Entries of Q blocks that can never see a key tile (causal) are not written.
+// blocks, K = 16 channels per instruction; D[key][block] in tensor memory (two
+// accumulators, so the product of one key tile overlaps the write-out of the
+// previous one), transposed through shared memory and written as dS[block][key]
+// by TMA stores.  32-block chunks whose blocks can never see a key tile (causal)
+// are not written.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -22,17 +23,26 @@
 namespace sage {
 
 constexpr int kDsThreads = 256;
-constexpr int kDsTilesPerCta = 8;
+constexpr int kDsTilesPerCta = 16;
 constexpr int kDsMaxN = 256;
+constexpr int kDsChunk = 32;   // Q blocks per epilogue store box
 constexpr uint64_t kDsDrainNs = 50ull * 1000ull * 1000ull;
 
+// Roles (256 threads): warp 0 loads K tiles (TMA, two buffers); warp 1 issues the
+// MMAs into one of two 256-column tensor-memory accumulators, so the product of
+// key tile i + 1 overlaps the epilogue of tile i; warps 4-7 (one per lane
+// quadrant) move each 32-block chunk of D[key][block] through shared memory,
+// transposed to [block][key], and write it with a TMA store.  All 256 threads
+// stage qbar.
 template <int D>
 struct __align__(1024) DsSmem {
     static constexpr int KA = D / 64;              // 128-byte (64-element) atoms along d
     uint8_t qhi[KA][kDsMaxN * 128];
     uint8_t qlo[KA][kDsMaxN * 128];
     uint8_t k[2][KA][kTile * 128];
-    uint64_t bar_k[2], bar_mma;
+    float stage[2][kDsChunk][kTile];
+    uint64_t bar_kfull[2], bar_kempty[2], bar_afull[2], bar_aempty[2];
+    uint64_t bar_stage_full[2], bar_stage_free[2];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -51,8 +61,8 @@ __device__ __forceinline__ float round16(float a, bool bf16) {
 
 template <int D>
 __global__ void __launch_bounds__(kDsThreads, 1)
-    ds_gemm_kernel(const __grid_constant__ CUtensorMap tm_k, const float *__restrict__ qbar, float *__restrict__ ds,
-                   int BH, int H, int Tq, int Tk, int n_q, int n_kv, int nk_pad, int nhd, int bf16, int causal_skip,
+    ds_gemm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ds,
+                   const float *__restrict__ qbar, int H, int Tq, int Tk, int nhd, int bf16, int causal_skip,
                    int causal_off, int *status) {
     constexpr int KA = D / 64;
     extern __shared__ uint8_t smem_raw[];
@@ -64,13 +74,18 @@ __global__ void __launch_bounds__(kDsThreads, 1)
     const bool is_bf16 = bf16 != 0;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sm.bar_k[0], 1);
-        mbar_init(&sm.bar_k[1], 1);
-        mbar_init(&sm.bar_mma, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.bar_kfull[i], 1);
+            mbar_init(&sm.bar_kempty[i], 1);
+            mbar_init(&sm.bar_afull[i], 1);
+            mbar_init(&sm.bar_aempty[i], 128);
+            mbar_init(&sm.bar_stage_full[i], 128);
+            mbar_init(&sm.bar_stage_free[i], 1);
+        }
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0) { tmem_alloc(&sm.tmem_base, 256); tmem_relinquish(); }
+    if (warp == 0) { tmem_alloc(&sm.tmem_base, 512); tmem_relinquish(); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -78,28 +93,20 @@ __global__ void __launch_bounds__(kDsThreads, 1)
     volatile int *abort_flag = &sm.abort_flag;
     const int b = bh / H, h = bh % H;
 
-    auto load_k = [&](int i, int buf) {
-        const int j0 = (jt0 + i) * kTile;
-        mbar_arrive_expect_tx(&sm.bar_k[buf], KA * kTile * 128);
-        for (int a = 0; a < KA; ++a) {
-            if (nhd) tma_load_4d(sm.k[buf][a], &tm_k, &sm.bar_k[buf], a * 64, h, j0, b);
-            else tma_load_3d(sm.k[buf][a], &tm_k, &sm.bar_k[buf], a * 64, j0, bh);
-        }
-    };
-
-    uint32_t k_phase[2] = {0, 0}, mma_phase = 0;
-    bool ok = true;
-    for (int tc = 0; tc < Tq && ok; tc += kDsMaxN) {
+    int g = 0;              // key tiles of earlier block chunks (buffer phases run on across chunks)
+    uint32_t n_chunks = 0;  // epilogue store boxes issued (staging buffer parity)
+    for (int tc = 0; tc < Tq; tc += kDsMaxN) {
         const int nt = min(kDsMaxN, Tq - tc);
         const int N = (nt + 15) / 16 * 16;
         // --- stage qbar[tc .. tc + N) as hi / lo 16-bit K-major operands (128-byte swizzle)
         const float *qsrc = qbar + ((size_t)bh * Tq + tc) * D;
+#pragma unroll 4
         for (int idx = threadIdx.x; idx < N * (D / 8); idx += kDsThreads) {
             const int n = idx / (D / 8), c8 = idx % (D / 8);
             float v[8];
             if (n < nt) {
-                const float4 x0 = *reinterpret_cast<const float4 *>(qsrc + (size_t)n * D + c8 * 8);
-                const float4 x1 = *reinterpret_cast<const float4 *>(qsrc + (size_t)n * D + c8 * 8 + 4);
+                const float4 x0 = __ldg(reinterpret_cast<const float4 *>(qsrc + (size_t)n * D + c8 * 8));
+                const float4 x1 = __ldg(reinterpret_cast<const float4 *>(qsrc + (size_t)n * D + c8 * 8 + 4));
                 v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w; v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
             } else {
 #pragma unroll
@@ -119,88 +126,128 @@ __global__ void __launch_bounds__(kDsThreads, 1)
         }
         fence_proxy_async_smem();
         __syncthreads();
-        if (threadIdx.x == 0) {
-            load_k(0, 0);
-            if (n_kt > 1) load_k(1, 1);
-        }
-        const uint32_t idesc = idesc_f16_f32(128, N, is_bf16);
-        for (int i = 0; i < n_kt; ++i) {
-            const int buf = i & 1;
-            if (threadIdx.x == 0) {
-                if (mbar_wait(&sm.bar_k[buf], k_phase[buf], abort_flag, status, 21)) {
-                    tc_fence_after();
-                    int step = 0;
+
+        if (warp == 0 && lane == 0) {
+            // ------------------------------ K producer ------------------------------
+            int issued = 0;
+            for (int i = 0; i < n_kt; ++i) {
+                const int gi = g + i, buf = gi & 1;
+                if (gi >= 2 && !mbar_wait(&sm.bar_kempty[buf], ((gi >> 1) & 1) ^ 1, abort_flag, status, 23)) break;
+                const int j0 = (jt0 + i) * kTile;
+                mbar_arrive_expect_tx(&sm.bar_kfull[buf], KA * kTile * 128);
+                for (int a = 0; a < KA; ++a) {
+                    if (nhd) tma_load_4d(sm.k[buf][a], &tm_k, &sm.bar_kfull[buf], a * 64, h, j0, b);
+                    else tma_load_3d(sm.k[buf][a], &tm_k, &sm.bar_kfull[buf], a * 64, j0, bh);
+                }
+                issued = i + 1;
+            }
+            if (*abort_flag)  // let the copies in flight land before the CTA exits
+                for (int i = max(0, issued - 2); i < issued; ++i)
+                    mbar_wait_quiet(&sm.bar_kfull[(g + i) & 1], ((g + i) >> 1) & 1, kDsDrainNs);
+        } else if (warp == 1 && lane == 0) {
+            // ------------------------------ MMA issuer ------------------------------
+            const uint32_t idesc = idesc_f16_f32(128, N, is_bf16);
+            for (int i = 0; i < n_kt; ++i) {
+                const int gi = g + i, buf = gi & 1;
+                if (!mbar_wait(&sm.bar_kfull[buf], (gi >> 1) & 1, abort_flag, status, 21)) break;
+                if (gi >= 2 && !mbar_wait(&sm.bar_aempty[buf], ((gi >> 1) & 1) ^ 1, abort_flag, status, 24)) break;
+                tc_fence_after();
+                const uint32_t acc = tmem + (uint32_t)buf * 256u;
+                int step = 0;
 #pragma unroll
-                    for (int a = 0; a < KA; ++a) {
+                for (int a = 0; a < KA; ++a) {
+                    const uint64_t ad = smem_desc(smem_u32(sm.k[buf][a]), 1024u, 2u);
+                    const uint64_t bh_d = smem_desc(smem_u32(sm.qhi[a]), 1024u, 2u);
+                    const uint64_t bl_d = smem_desc(smem_u32(sm.qlo[a]), 1024u, 2u);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk, ++step) {
-                            const uint64_t ad = smem_desc(smem_u32(sm.k[buf][a]) + kk * 32, 1024u, 2u);
-                            const uint64_t bh_d = smem_desc(smem_u32(sm.qhi[a]) + kk * 32, 1024u, 2u);
-                            const uint64_t bl_d = smem_desc(smem_u32(sm.qlo[a]) + kk * 32, 1024u, 2u);
-                            mma_f16_ss(tmem, ad, bh_d, idesc, step > 0 ? 1u : 0u);
-                            mma_f16_ss(tmem, ad, bl_d, idesc, 1u);
-                        }
+                    for (int kk = 0; kk < 4; ++kk, ++step) {
+                        mma_f16_ss(acc, ad + 2 * kk, bh_d + 2 * kk, idesc, step > 0 ? 1u : 0u);
+                        mma_f16_ss(acc, ad + 2 * kk, bl_d + 2 * kk, idesc, 1u);
                     }
                 }
-                mma_commit(&sm.bar_mma);
+                mma_commit(&sm.bar_kempty[buf]);
+                mma_commit(&sm.bar_afull[buf]);
             }
-            k_phase[buf] ^= 1;
-            __syncwarp();
-            mbar_wait(&sm.bar_mma, mma_phase, abort_flag, status, 22);
-            mma_phase ^= 1;
-            tc_fence_after();
-            __syncthreads();
-            if (*abort_flag) { ok = false; break; }
-            // --- epilogue: D[key][block] -> dS[block][key]
-            const int jt = jt0 + i;
-            int t_lo = 0;
-            if (causal_skip) {
-                const int num = jt * kTile - causal_off - (kTile - 1);
-                t_lo = num <= 0 ? 0 : (num + kTile - 1) / kTile;
-                if (t_lo > Tq - 1) t_lo = Tq - 1;
-            }
-            const int wq = warp & 3;
-            const int key = jt * kTile + wq * 32 + lane;
-            float *dst = ds + (size_t)bh * Tq * nk_pad + key;
-            for (int c0 = (warp >> 2) * 32; c0 < N; c0 += 64) {
-                uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + c0, v);
-                tmem_wait_ld_regs(v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int t = tc + c0 + e;
-                    if (c0 + e < nt && t >= t_lo) dst[(size_t)t * nk_pad] = __uint_as_float(v[e]);
+        } else if (warp >= 4) {
+            // ------------------------------ epilogue ------------------------------
+            // Store box n goes through staging buffer n & 1: its 128 writers arrive on
+            // stage_full, thread 0 then issues the TMA store and, once the store before
+            // it has finished reading shared memory, frees that buffer (stage_free).
+            const int wq = warp & 3, et = threadIdx.x - 128;
+            bool ok = true;
+            for (int i = 0; ok && i < n_kt; ++i) {
+                const int gi = g + i, buf = gi & 1;
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.bar_afull[buf], (gi >> 1) & 1, abort_flag, status, 22));
+                if (!ok) break;
+                tc_fence_after();
+                const int jt = jt0 + i;
+                int t_lo = 0;  // Q blocks below t_lo never see key tile jt (causal)
+                if (causal_skip) {
+                    const int num = jt * kTile - causal_off - (kTile - 1);
+                    t_lo = num <= 0 ? 0 : (num + kTile - 1) / kTile;
                 }
+                const uint32_t acc = tmem + (uint32_t)buf * 256u + ((uint32_t)(wq * 32) << 16);
+                for (int c0 = 0; c0 < N; c0 += kDsChunk) {
+                    if (tc + c0 + kDsChunk - 1 < t_lo) continue;
+                    const uint32_t n = n_chunks++, sb = n & 1u;
+                    uint32_t v[32];
+                    tmem_ld32(acc + c0, v);
+                    tmem_wait_ld_regs(v);
+                    if (n >= 2) {
+                        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.bar_stage_free[sb], ((n >> 1) - 1) & 1, abort_flag,
+                                                               status, 25));
+                        if (!ok) break;
+                    }
+                    float *col = &sm.stage[sb][0][wq * 32 + lane];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) col[e * kTile] = __uint_as_float(v[e]);
+                    fence_proxy_async_smem();
+                    mbar_arrive(&sm.bar_stage_full[sb]);
+                    if (et == 0) {
+                        if (!mbar_wait(&sm.bar_stage_full[sb], (n >> 1) & 1, abort_flag, status, 26)) { ok = false; }
+                        else {
+                            tma_store_3d(&tm_ds, sm.stage[sb], jt * kTile, tc + c0, bh);
+                            bulk_commit_group();
+                            if (n >= 1) {  // box n - 1 has been read out of stage[sb ^ 1]
+                                bulk_wait_group_read<1>();
+                                mbar_arrive(&sm.bar_stage_free[sb ^ 1u]);
+                            }
+                        }
+                    }
+                    ok = __all_sync(0xFFFFFFFFu, ok);
+                    if (!ok) break;
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.bar_aempty[buf]);
             }
-            tc_fence_before();
-            __syncthreads();   // TMEM read and K buffer consumed
-            if (threadIdx.x == 0 && i + 2 < n_kt) load_k(i + 2, buf);
+            if (et == 0) bulk_wait_group<0>();
         }
-        if (!ok && threadIdx.x == 0) {   // let the copies in flight land before the CTA exits
-            for (int i2 = 0; i2 < 2; ++i2) mbar_wait_quiet(&sm.bar_k[i2], k_phase[i2], kDsDrainNs);
-        }
-        __syncthreads();
+        g += n_kt;
+        tc_fence_before();
+        __syncthreads();  // every role is done with this block chunk before qbar is restaged
+        tc_fence_after();
+        if (*abort_flag) break;
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) { __syncwarp(); tc_fence_after(); tmem_dealloc(tmem, 256); }
+    if (warp == 0) { __syncwarp(); tc_fence_after(); tmem_dealloc(tmem, 512); }
 }
 
-cudaError_t launch_ds_gemm(const CUtensorMap &tm_k, const float *qbar, float *ds, const Shape &s, int nhd, int bf16,
-                           int causal_skip, int causal_off, int *status, cudaStream_t stream) {
+cudaError_t launch_ds_gemm(const CUtensorMap &tm_k, const CUtensorMap &tm_ds, const float *qbar, const Shape &s,
+                           int nhd, int bf16, int causal_skip, int causal_off, int *status, cudaStream_t stream) {
     dim3 grid((s.Tk + kDsTilesPerCta - 1) / kDsTilesPerCta, s.BH);
     if (s.d == 128) {
         const size_t smem = sizeof(DsSmem<128>) + 1024;
         cudaError_t e = cudaFuncSetAttribute(ds_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        ds_gemm_kernel<128><<<grid, kDsThreads, smem, stream>>>(tm_k, qbar, ds, s.BH, s.H, s.Tq, s.Tk, s.n_q, s.n_kv,
-                                                                 s.nk_pad, nhd, bf16, causal_skip, causal_off, status);
+        ds_gemm_kernel<128><<<grid, kDsThreads, smem, stream>>>(tm_k, tm_ds, qbar, s.H, s.Tq, s.Tk, nhd, bf16,
+                                                                 causal_skip, causal_off, status);
     } else {
         const size_t smem = sizeof(DsSmem<64>) + 1024;
         cudaError_t e = cudaFuncSetAttribute(ds_gemm_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        ds_gemm_kernel<64><<<grid, kDsThreads, smem, stream>>>(tm_k, qbar, ds, s.BH, s.H, s.Tq, s.Tk, s.n_q, s.n_kv,
-                                                                s.nk_pad, nhd, bf16, causal_skip, causal_off, status);
+        ds_gemm_kernel<64><<<grid, kDsThreads, smem, stream>>>(tm_k, tm_ds, qbar, s.H, s.Tq, s.Tk, nhd, bf16,
+                                                                causal_skip, causal_off, status);
     }
     return cudaGetLastError();
 }

@@ -101,8 +101,8 @@ cudaError_t launch_prepass(const PrepassArgs &a, cudaStream_t stream);
 // (3-D [BH][n_kv][d] for head-major, 4-D [B][n_kv][H][d] for token-major, 64 x 128
 // boxes, 128-byte swizzle).  causal_skip: leave entries of Q blocks that can never
 // see a key tile unwritten (key j visible to query i iff j <= i + causal_off).
-cudaError_t launch_ds_gemm(const CUtensorMap &tm_k, const float *qbar, float *ds, const Shape &s, int nhd, int bf16,
-                           int causal_skip, int causal_off, int *status, cudaStream_t stream);
+cudaError_t launch_ds_gemm(const CUtensorMap &tm_k, const CUtensorMap &tm_ds, const float *qbar, const Shape &s,
+                           int nhd, int bf16, int causal_skip, int causal_off, int *status, cudaStream_t stream);
 cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                              const AttnParams &p, int d, cudaStream_t stream);
 cudaError_t launch_debug_qk_tile(const CUtensorMap &tq, const CUtensorMap &tk, int d, int q_row0, int k_row0,
