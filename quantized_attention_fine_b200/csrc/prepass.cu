@@ -3,7 +3,8 @@
 // fine-grained Q/K quantization, FP8 V; per-channel V scale from the
 // pith.science verdict on arXiv 2505.21136, key_machinery).
 //
-// Bandwidth-bound kernels (the dS product is in ds_gemm.cu):
+// Bandwidth-bound kernels (the dS product is in ds_gemm.cu); the three quantization
+// kernels stream their input through TMA rings (see below):
 //   kv_stats     per (head, 512-token chunk): fp64 partial sums of K per channel
 //                and per-channel max |V|.
 //   kv_finalize  per head: kbar = fp32(sum / n_kv); delta_V = max|V| / Vr.
@@ -92,10 +93,90 @@ __device__ __forceinline__ void store_codes(int8_t *dst, const int8_t (&c)[VEC])
 
 }  // namespace
 
-// Quantization kernels: 16 warps per 128-row (or 128-key) tile, 8 rows per warp.
-constexpr int kQuantThreads = 512;
+// Quantization kernels: persistent CTAs of 8 warps stream 128-row tiles (one
+// head's rows or keys) through a ring of shared-memory stages filled by TMA, so the
+// loads of the next tiles are in flight while a tile is reduced and quantized.
+// Warp w owns rows 16w .. 16w + 15 of a tile; lane l owns channels l*VEC ...
+constexpr int kQuantThreads = 256;
 constexpr int kQuantWarps = kQuantThreads / 32;
-constexpr int kRowsPerWarp = kTile / kQuantWarps;
+constexpr int kRowsPerWarp = kTile / kQuantWarps;   // 16 = one delta_K run
+constexpr int kSitePrepass = 31;
+constexpr uint64_t kPrepassDrainNs = 50ull * 1000ull * 1000ull;
+
+template <int D>
+struct QuantRing {
+    static constexpr int kStages = (D == 128) ? 3 : 4;
+    static constexpr uint32_t kTileBytes = kTile * D * 2;
+    static constexpr size_t kSmemBytes = kStages * kTileBytes + 128;
+};
+
+// TMA load of work unit u (row tile t = u % T of head bh = u / T) of a 16-bit
+// [BH][n][d] (head-major) or [B][n][H][d] (token-major) tensor; rows past n read 0.
+__device__ __forceinline__ void load_rows_tile(const CUtensorMap *tm, int nhd, int H, int T, int u, void *dst,
+                                               uint64_t *bar, uint32_t bytes) {
+    const int bh = u / T, t = u % T;
+    mbar_arrive_expect_tx(bar, bytes);
+    if (nhd) tma_load_4d(dst, tm, bar, 0, bh % H, t * kTile, bh / H);
+    else tma_load_3d(dst, tm, bar, 0, t * kTile, bh);
+}
+
+// Ring bookkeeping shared by the three kernels: thread 0 primes kStages loads; the
+// k-th unit of this CTA sits in stage k % kStages.
+template <int D>
+struct RingCtl {
+    uint16_t *ring;
+    uint64_t *full;
+    int n_units, T, H, nhd;
+    const CUtensorMap *tm;
+    __device__ __forceinline__ uint16_t *stage(int k) const { return ring + (size_t)(k % QuantRing<D>::kStages) * kTile * D; }
+    __device__ __forceinline__ void issue(int k) const {  // load this CTA's k-th unit, if any
+        const int u = blockIdx.x + k * gridDim.x;
+        if (u < n_units)
+            load_rows_tile(tm, nhd, H, T, u, stage(k), &full[k % QuantRing<D>::kStages], QuantRing<D>::kTileBytes);
+    }
+    __device__ __forceinline__ bool wait(int k, volatile int *abort_flag, int *status) const {
+        return __all_sync(0xFFFFFFFFu, mbar_wait(&full[k % QuantRing<D>::kStages], (k / QuantRing<D>::kStages) & 1,
+                                                  abort_flag, status, kSitePrepass));
+    }
+    // on the abort path: let the loads still in flight land before the CTA exits
+    __device__ __forceinline__ void drain(int k_next) const {
+        for (int k = k_next; k < k_next + QuantRing<D>::kStages; ++k)
+            if ((int)(blockIdx.x + k * gridDim.x) < n_units)
+                mbar_wait_quiet(&full[k % QuantRing<D>::kStages], (k / QuantRing<D>::kStages) & 1, kPrepassDrainNs);
+    }
+};
+
+template <int D>
+__device__ __forceinline__ RingCtl<D> ring_setup(const CUtensorMap *tm, int nhd, int H, int T, int BH, uint64_t *full,
+                                                 volatile int *abort_flag) {
+    extern __shared__ uint8_t smem_raw[];
+    RingCtl<D> rc;
+    rc.ring = reinterpret_cast<uint16_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    rc.full = full;
+    rc.n_units = BH * T;
+    rc.T = T;
+    rc.H = H;
+    rc.nhd = nhd;
+    rc.tm = tm;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < QuantRing<D>::kStages; ++s) mbar_init(&full[s], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        prefetch_tmap(tm);
+        for (int k = 0; k < QuantRing<D>::kStages; ++k) rc.issue(k);
+    }
+    return rc;
+}
+
+// Largest |x| over the 16-row groups of warps [w0, w0 + n) of this tile.
+__device__ __forceinline__ float group_amax(const float *wmax, int w0, int n) {
+    float am = 0.f;
+    for (int w = w0; w < w0 + n; ++w) am = fmaxf(am, wmax[w]);
+    return am;
+}
 
 // ---------------------------------------------------------------------------
 template <int D>
@@ -166,195 +247,190 @@ __global__ void kv_finalize_kernel(const PrepassArgs a) {
 
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(kQuantThreads) quant_q_kernel(const PrepassArgs a) {
+__global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_constant__ PrepassArgs a) {
     constexpr int VEC = D / 32, RPW = kRowsPerWarp;
+    __shared__ uint64_t s_full[QuantRing<D>::kStages];
     __shared__ double s_sum[kQuantWarps][D];
     __shared__ float s_qbar[D];
-    __shared__ float s_ramax[kTile];
-    __shared__ float s_delta[kTile];
+    __shared__ float s_wmax[kQuantWarps];
+    __shared__ int s_abort;
     const Shape &S = a.shape;
-    const int t = blockIdx.x, bh = blockIdx.y;
-    const int b = bh / S.H, h = bh % S.H;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r0 = t * kTile;
-    const int nvalid = min(kTile, S.n_q - r0);
-    const uint16_t *qp = static_cast<const uint16_t *>(a.q) + b * a.sq.b + h * a.sq.h + lane * VEC;
-
-    float x[RPW][VEC];
-    double ps[VEC];
+    int *status = reinterpret_cast<int *>(a.ws + a.L.status);
+    const RingCtl<D> rc = ring_setup<D>(&a.tm_q, a.nhd, S.H, S.Tq, S.BH, s_full, &s_abort);
+    int k = 0;
+    for (;; ++k) {
+        const int u = blockIdx.x + k * gridDim.x;
+        if (u >= rc.n_units) break;
+        if (!rc.wait(k, &s_abort, status)) break;
+        const int bh = u / S.Tq, t = u % S.Tq;
+        const int r0 = t * kTile, nvalid = min(kTile, S.n_q - r0);
+        const uint16_t *tile = rc.stage(k) + lane * VEC;
+        float x[RPW][VEC];
+        double ps[VEC];
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) ps[v] = 0.0;
+        for (int v = 0; v < VEC; ++v) ps[v] = 0.0;
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-        const int r = warp * RPW + i;
-        if (r < nvalid) {
-            load_row_slice<VEC>(qp + (int64_t)(r0 + r) * a.sq.n, a.bf16, x[i]);
+        for (int i = 0; i < RPW; ++i) {
+            const int r = warp * RPW + i;
+            load_row_slice<VEC>(tile + r * D, a.bf16, x[i]);
+            if (r < nvalid) {
 #pragma unroll
-            for (int v = 0; v < VEC; ++v) ps[v] = __dadd_rn(ps[v], (double)x[i][v]);
-        } else {
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) x[i][v] = 0.f;
+                for (int v = 0; v < VEC; ++v) ps[v] = __dadd_rn(ps[v], (double)x[i][v]);
+            }
         }
-    }
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) s_sum[warp][lane * VEC + v] = ps[v];
-    __syncthreads();
-    if (threadIdx.x < D) {
-        const int c = threadIdx.x;
-        double s = 0.0;
+        for (int v = 0; v < VEC; ++v) s_sum[warp][lane * VEC + v] = ps[v];
+        __syncthreads();  // the stage is in registers: refill it
+        if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
+        if (threadIdx.x < D) {  // qbar: fp64 mean of the valid rows, rounded to fp32
+            const int c = threadIdx.x;
+            double sum = 0.0;
 #pragma unroll
-        for (int w = 0; w < kQuantWarps; ++w) s = __dadd_rn(s, s_sum[w][c]);
-        const float qb = a.smooth_q ? (float)__ddiv_rn(s, (double)nvalid) : 0.f;
-        s_qbar[c] = qb;
-        reinterpret_cast<float *>(a.ws + a.L.qbar)[((size_t)bh * S.Tq + t) * D + c] = qb;
-    }
-    __syncthreads();
-    float qb[VEC];
+            for (int w = 0; w < kQuantWarps; ++w) sum = __dadd_rn(sum, s_sum[w][c]);
+            const float qb = a.smooth_q ? (float)__ddiv_rn(sum, (double)nvalid) : 0.f;
+            s_qbar[c] = qb;
+            reinterpret_cast<float *>(a.ws + a.L.qbar)[((size_t)bh * S.Tq + t) * D + c] = qb;
+        }
+        __syncthreads();
+        float qb[VEC];
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) qb[v] = s_qbar[lane * VEC + v];
-#pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-        const int r = warp * RPW + i;
+        for (int v = 0; v < VEC; ++v) qb[v] = s_qbar[lane * VEC + v];
         float am = 0.f;
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) {
-            const float xs = (r < nvalid) ? __fsub_rn(x[i][v], qb[v]) : 0.f;
-            x[i][v] = xs;
-            am = fmaxf(am, fabsf(xs));
+        for (int i = 0; i < RPW; ++i) {
+            const int r = warp * RPW + i;
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                const float xs = (r < nvalid) ? __fsub_rn(x[i][v], qb[v]) : 0.f;
+                x[i][v] = xs;
+                am = fmaxf(am, fabsf(xs));
+            }
         }
         am = warp_max(am);
-        if (lane == 0) s_ramax[r] = am;
-    }
-    __syncthreads();
-    if (threadIdx.x < kTile) {
-        const int r = threadIdx.x;
-        const int g0 = (r / a.g_q) * a.g_q;
-        float am = 0.f;
-        for (int rr = g0; rr < g0 + a.g_q; ++rr) am = fmaxf(am, s_ramax[rr]);
-        const float dl = (am == 0.f) ? 1.f : __fdiv_rn(am, 127.f);
-        s_delta[r] = dl;
-        reinterpret_cast<float *>(a.ws + a.L.dq)[(size_t)bh * S.nq_pad + r0 + r] = dl;
-    }
-    __syncthreads();
-    int8_t *q8 = reinterpret_cast<int8_t *>(a.ws + a.L.q8) + ((size_t)bh * S.nq_pad + r0) * D + lane * VEC;
-#pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-        const int r = warp * RPW + i;
-        const float dl = s_delta[r];
+        if (lane == 0) s_wmax[warp] = am;
+        __syncthreads();
+        const int gw = a.g_q / RPW;  // warps per quantization group (g_q = 32 or 128)
+        const float gam = group_amax(s_wmax, (warp / gw) * gw, gw);
+        const float dl = (gam == 0.f) ? 1.f : __fdiv_rn(gam, 127.f);
+        if (lane < RPW) reinterpret_cast<float *>(a.ws + a.L.dq)[(size_t)bh * S.nq_pad + r0 + warp * RPW + lane] = dl;
         const float inv = 1.0f / dl;
-        int8_t c[VEC];
+        int8_t *q8 = reinterpret_cast<int8_t *>(a.ws + a.L.q8) + ((size_t)bh * S.nq_pad + r0 + warp * RPW) * D + lane * VEC;
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) c[v] = int8_code(x[i][v], dl, inv);
-        store_codes<VEC>(q8 + (size_t)r * D, c);
+        for (int i = 0; i < RPW; ++i) {
+            int8_t c[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) c[v] = int8_code(x[i][v], dl, inv);
+            store_codes<VEC>(q8 + (size_t)i * D, c);
+        }
     }
+    if (s_abort && threadIdx.x == 0) rc.drain(k);
 }
 
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(kQuantThreads) quant_k_kernel(const PrepassArgs a) {
+__global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_constant__ PrepassArgs a) {
     constexpr int VEC = D / 32, RPW = kRowsPerWarp;
-    __shared__ float s_ramax[kTile];
-    __shared__ float s_delta[kTile];
+    __shared__ uint64_t s_full[QuantRing<D>::kStages];
+    __shared__ float s_wmax[2][kQuantWarps];
+    __shared__ int s_abort;
     const Shape &S = a.shape;
-    const int jt = blockIdx.x, bh = blockIdx.y;
-    const int b = bh / S.H, h = bh % S.H;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int j0 = jt * kTile;
-    const int nvalid = min(kTile, S.n_kv - j0);
-    const uint16_t *kp = static_cast<const uint16_t *>(a.k) + b * a.skv.b + h * a.skv.h + lane * VEC;
-    float kb[VEC];
+    int *status = reinterpret_cast<int *>(a.ws + a.L.status);
+    const RingCtl<D> rc = ring_setup<D>(&a.tm_k, a.nhd, S.H, S.Tk, S.BH, s_full, &s_abort);
+    int k = 0;
+    for (;; ++k) {
+        const int u = blockIdx.x + k * gridDim.x;
+        if (u >= rc.n_units) break;
+        if (!rc.wait(k, &s_abort, status)) break;
+        const int bh = u / S.Tk, jt = u % S.Tk;
+        const int j0 = jt * kTile, nvalid = min(kTile, S.n_kv - j0);
+        const uint16_t *tile = rc.stage(k) + lane * VEC;
+        float kb[VEC];
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) kb[v] = reinterpret_cast<const float *>(a.ws + a.L.kbar)[(size_t)bh * D + lane * VEC + v];
-    float x[RPW][VEC];
-#pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-        const int r = warp * RPW + i;
-        if (r < nvalid) {
-            load_row_slice<VEC>(kp + (int64_t)(j0 + r) * a.skv.n, a.bf16, x[i]);
-        } else {
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) x[i][v] = 0.f;
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-        const int r = warp * RPW + i;
+        for (int v = 0; v < VEC; ++v) kb[v] = reinterpret_cast<const float *>(a.ws + a.L.kbar)[(size_t)bh * D + lane * VEC + v];
+        float x[RPW][VEC];
         float am = 0.f;
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) {
-            const float xs = (r < nvalid) ? __fsub_rn(x[i][v], kb[v]) : 0.f;
-            x[i][v] = xs;
-            am = fmaxf(am, fabsf(xs));
+        for (int i = 0; i < RPW; ++i) {
+            const int r = warp * RPW + i;
+            load_row_slice<VEC>(tile + r * D, a.bf16, x[i]);
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                const float xs = (r < nvalid) ? __fsub_rn(x[i][v], kb[v]) : 0.f;
+                x[i][v] = xs;
+                am = fmaxf(am, fabsf(xs));
+            }
         }
         am = warp_max(am);
-        if (lane == 0) s_ramax[r] = am;
-    }
-    __syncthreads();
-    if (threadIdx.x < kTile) {
-        const int r = threadIdx.x;
-        const int g0 = (r / a.g_k) * a.g_k;
-        float am = 0.f;
-        for (int rr = g0; rr < g0 + a.g_k; ++rr) am = fmaxf(am, s_ramax[rr]);
-        const float dl = (am == 0.f) ? 1.f : __fdiv_rn(am, 127.f);
-        s_delta[r] = dl;
-        if ((r % kKeyRun) == 0)
-            reinterpret_cast<float *>(a.ws + a.L.dk)[(size_t)bh * (S.nk_pad / kKeyRun) + (j0 + r) / kKeyRun] = dl;
-    }
-    __syncthreads();
-    int8_t *k8 = reinterpret_cast<int8_t *>(a.ws + a.L.k8) + ((size_t)bh * S.nk_pad + j0) * D + lane * VEC;
-#pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-        const int r = warp * RPW + i;
-        const float dl = s_delta[r];
+        if (lane == 0) s_wmax[k & 1][warp] = am;
+        __syncthreads();  // the stage is in registers: refill it
+        if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
+        const int gw = a.g_k / RPW;  // warps per quantization group (g_k = 16 or 128)
+        const float gam = group_amax(s_wmax[k & 1], (warp / gw) * gw, gw);
+        const float dl = (gam == 0.f) ? 1.f : __fdiv_rn(gam, 127.f);
+        if (lane == 0)  // one delta_K per 16-key run = this warp's rows
+            reinterpret_cast<float *>(a.ws + a.L.dk)[(size_t)bh * (S.nk_pad / kKeyRun) + (j0 + warp * RPW) / kKeyRun] = dl;
         const float inv = 1.0f / dl;
-        int8_t c[VEC];
+        int8_t *k8 = reinterpret_cast<int8_t *>(a.ws + a.L.k8) + ((size_t)bh * S.nk_pad + j0 + warp * RPW) * D + lane * VEC;
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) c[v] = int8_code(x[i][v], dl, inv);
-        store_codes<VEC>(k8 + (size_t)r * D, c);
-    }
-}
-
-// V codes of one 128-key tile, written transposed: each lane holds 8 consecutive
-// keys of VEC channels and stores them as one 8-byte piece of each channel's row of
-// V^T ([channel][key]).
-template <int D>
-__global__ void __launch_bounds__(kQuantThreads) quant_v_kernel(const PrepassArgs a) {
-    constexpr int VEC = D / 32, RPW = kRowsPerWarp;
-    const Shape &S = a.shape;
-    const int jt = blockIdx.x, bh = blockIdx.y;
-    const int b = bh / S.H, h = bh % S.H;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int j0 = jt * kTile;
-    const int nvalid = min(kTile, S.n_kv - j0);
-    const uint16_t *vp = static_cast<const uint16_t *>(a.v) + b * a.skv.b + h * a.skv.h + lane * VEC;
-    float dv[VEC], inv[VEC];
+        for (int i = 0; i < RPW; ++i) {
+            int8_t c[VEC];
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) {
-        dv[v] = reinterpret_cast<const float *>(a.ws + a.L.dv)[(size_t)bh * D + lane * VEC + v];
-        inv[v] = 1.0f / dv[v];
-    }
-    float x[RPW][VEC];
-#pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-        const int r = warp * RPW + i;
-        if (r < nvalid) {
-            load_row_slice<VEC>(vp + (int64_t)(j0 + r) * a.skv.n, a.bf16, x[i]);
-        } else {
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) x[i][v] = 0.f;
+            for (int v = 0; v < VEC; ++v) c[v] = int8_code(x[i][v], dl, inv);
+            store_codes<VEC>(k8 + (size_t)i * D, c);
         }
     }
-    uint8_t *vt8 = a.ws + a.L.vt8 + ((size_t)bh * D + lane * VEC) * S.nk_pad + j0 + warp * RPW;
-    static_assert(RPW == 8, "each lane stores 8 keys of a channel as one 8-byte piece");
+    if (s_abort && threadIdx.x == 0) rc.drain(k);
+}
+
+// V codes of a 128-key tile, written transposed ([channel][key]): lane l holds the
+// 16 keys of its warp for channels l*VEC .., and stores each channel's 16 codes as
+// one 16-byte piece of that channel's row of V^T.
+template <int D>
+__global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_constant__ PrepassArgs a) {
+    constexpr int VEC = D / 32, RPW = kRowsPerWarp;
+    static_assert(RPW == 16, "a lane stores 16 keys of a channel as one 16-byte piece");
+    __shared__ uint64_t s_full[QuantRing<D>::kStages];
+    __shared__ int s_abort;
+    const Shape &S = a.shape;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int *status = reinterpret_cast<int *>(a.ws + a.L.status);
+    const RingCtl<D> rc = ring_setup<D>(&a.tm_v, a.nhd, S.H, S.Tk, S.BH, s_full, &s_abort);
+    int k = 0;
+    for (;; ++k) {
+        const int u = blockIdx.x + k * gridDim.x;
+        if (u >= rc.n_units) break;
+        if (!rc.wait(k, &s_abort, status)) break;
+        const int bh = u / S.Tk, jt = u % S.Tk;
+        const int j0 = jt * kTile, nvalid = min(kTile, S.n_kv - j0);
+        const uint16_t *tile = rc.stage(k) + lane * VEC;
+        float x[RPW][VEC];
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) {
-        uint32_t w[2];
+        for (int i = 0; i < RPW; ++i) {
+            const int r = warp * RPW + i;
+            load_row_slice<VEC>(tile + r * D, a.bf16, x[i]);
+            if (r >= nvalid) {
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
-            w[q] = pack_e4m3x4(e4m3_quotient(x[4 * q][v], dv[v], inv[v]), e4m3_quotient(x[4 * q + 1][v], dv[v], inv[v]),
-                               e4m3_quotient(x[4 * q + 2][v], dv[v], inv[v]), e4m3_quotient(x[4 * q + 3][v], dv[v], inv[v]));
-        *reinterpret_cast<uint2 *>(vt8 + (size_t)v * S.nk_pad) = make_uint2(w[0], w[1]);
+                for (int v = 0; v < VEC; ++v) x[i][v] = 0.f;
+            }
+        }
+        __syncthreads();  // the stage is in registers: refill it
+        if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
+        uint8_t *vt8 = a.ws + a.L.vt8 + ((size_t)bh * D + lane * VEC) * S.nk_pad + j0 + warp * RPW;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+            const float dv = reinterpret_cast<const float *>(a.ws + a.L.dv)[(size_t)bh * D + lane * VEC + v];
+            const float inv = 1.0f / dv;
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                w[q] = pack_e4m3x4(e4m3_quotient(x[4 * q][v], dv, inv), e4m3_quotient(x[4 * q + 1][v], dv, inv),
+                                   e4m3_quotient(x[4 * q + 2][v], dv, inv), e4m3_quotient(x[4 * q + 3][v], dv, inv));
+            *reinterpret_cast<uint4 *>(vt8 + (size_t)v * S.nk_pad) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
     }
+    if (s_abort && threadIdx.x == 0) rc.drain(k);
 }
 
 // ---------------------------------------------------------------------------
@@ -365,9 +441,23 @@ static cudaError_t launch_prepass_d(const PrepassArgs &a, cudaStream_t stream) {
         kv_stats_kernel<D><<<dim3(S.n_chunks, S.BH), 256, 0, stream>>>(a);
         kv_finalize_kernel<D><<<S.BH, D, 0, stream>>>(a);
     }
-    if (a.q) quant_q_kernel<D><<<dim3(S.Tq, S.BH), kQuantThreads, 0, stream>>>(a);
-    if (a.k) quant_k_kernel<D><<<dim3(S.Tk, S.BH), kQuantThreads, 0, stream>>>(a);
-    if (a.v) quant_v_kernel<D><<<dim3(S.Tk, S.BH), kQuantThreads, 0, stream>>>(a);
+    // persistent grids: two CTAs per SM, or one per work unit if fewer
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const size_t smem = QuantRing<D>::kSmemBytes;
+    auto grid_of = [&](int units) { return (unsigned)(units < 2 * sms ? units : 2 * sms); };
+    if (a.q) {
+        cudaFuncSetAttribute(quant_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        quant_q_kernel<D><<<grid_of(S.BH * S.Tq), kQuantThreads, smem, stream>>>(a);
+    }
+    if (a.k) {
+        cudaFuncSetAttribute(quant_k_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        quant_k_kernel<D><<<grid_of(S.BH * S.Tk), kQuantThreads, smem, stream>>>(a);
+    }
+    if (a.v) {
+        cudaFuncSetAttribute(quant_v_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        quant_v_kernel<D><<<grid_of(S.BH * S.Tk), kQuantThreads, smem, stream>>>(a);
+    }
     return cudaGetLastError();
 }
 

@@ -131,6 +131,32 @@ bool make_k16_map(CUtensorMap *map, const void *k, int dtype, int layout, const 
     return r == CUDA_SUCCESS;
 }
 
+// Load map of a caller's 16-bit Q, K or V (n rows per head): d x 128-row boxes, no
+// swizzle; rows past n read as zero.
+bool make_rows16_map(CUtensorMap *map, const void *x, int dtype, int layout, const Shape &s, int n) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const CUtensorMapDataType dt =
+        (dtype == SAGE_DTYPE_BF16) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const uint64_t d = (uint64_t)s.d;
+    if (layout == SAGE_LAYOUT_HND) {
+        cuuint64_t dims[3] = {d, (uint64_t)n, (uint64_t)s.BH};
+        cuuint64_t strides[2] = {d * 2, (uint64_t)n * d * 2};
+        cuuint32_t box[3] = {(cuuint32_t)d, (cuuint32_t)kTile, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        return enc(map, dt, 3, const_cast<void *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
+    cuuint64_t dims[4] = {d, (uint64_t)s.H, (uint64_t)n, (uint64_t)s.B};
+    cuuint64_t strides[3] = {d * 2, (uint64_t)s.H * d * 2, (uint64_t)n * s.H * d * 2};
+    cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)kTile, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, dt, 4, const_cast<void *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 // Store map of the dS array [BH][Tq][nk_pad] fp32: 128-key x 32-block boxes, no
 // swizzle; rows past Tq are clipped by the copy engine.
 bool make_ds_map(CUtensorMap *map, float *ds, const Shape &s) {
@@ -152,6 +178,10 @@ sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype
     a.k = k;
     a.v = v;
     a.bf16 = (dtype == SAGE_DTYPE_BF16);
+    a.nhd = (layout == SAGE_LAYOUT_NHD);
+    if (q && !make_rows16_map(&a.tm_q, q, dtype, layout, s, s.n_q)) return SAGE_ERR_CUDA;
+    if (k && !make_rows16_map(&a.tm_k, k, dtype, layout, s, s.n_kv)) return SAGE_ERR_CUDA;
+    if (v && !make_rows16_map(&a.tm_v, v, dtype, layout, s, s.n_kv)) return SAGE_ERR_CUDA;
     a.sq = make_strides(layout, s.H, s.n_q, s.d);
     a.skv = make_strides(layout, s.H, s.n_kv, s.d);
     a.shape = s;

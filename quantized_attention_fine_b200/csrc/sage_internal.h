@@ -72,8 +72,11 @@ inline Strides make_strides(int layout, int H, int N, int d) {
 }
 
 struct PrepassArgs {
+    // tensor maps of the caller's 16-bit Q, K, V ([BH][n][d] or [B][n][H][d]; d x 128-row
+    // boxes, no swizzle), valid where the pointer below is not null
+    CUtensorMap tm_q, tm_k, tm_v;
     const void *q, *k, *v;   // any may be null: that part is skipped
-    int bf16;
+    int bf16, nhd;
     Strides sq, skv;
     Shape shape;
     int g_q, g_k, smooth_q, smooth_k;
