@@ -5,9 +5,10 @@
     python bench.py --impl reference ...        # the fp64 CPU oracle on the host cores
 
 One step = one pass of the whole hot path over one batch of synthetic input
-already resident in HBM: the smoothing/quantization pre-pass of Q, K and V
-(sage_quant_qk, sage_quant_v) and the fused attention kernel
-(sage_attn_fwd_prequant), all through the C ABI.  Metric: attention TOPS
+already resident in HBM, through the public C-ABI call sage_attn_fwd: the
+smoothing/quantization pre-pass of Q, K and V, the dS product, and the fused
+attention kernel.  A second timed loop runs the attention kernel alone
+(sage_attn_fwd_prequant on the same workspace) for its roofline figure.  Metric: attention TOPS
 = 4 B H N_q N_kv d / t (halved when causal), summed over all ranks.  With N > 1
 every rank runs the full workload on its own seeded inputs (heads are independent,
 so the path shards with no collective): weak scaling.  Rank 0 prints one JSON line.
@@ -31,9 +32,9 @@ METRIC = "attention TOPS (4*B*H*Nq*Nkv*d/t, causal /2) and % of B200 dense INT8/
 UNIT = "TOPS"
 SPEC_INT8_TOPS = 4500.0          # B200 dense INT8 / FP8 datasheet figure
 FALLBACK_BF16_TFLOPS = 1590.0    # pool measurement used when MEASURED_PEAKS.json is absent
-# library kernels per step: quant_qk (kv_stats, kv_finalize, quant_q, quant_k, ds_gemm),
-# quant_v (kv_stats, kv_finalize, quant_v), attention (attn_fwd_kernel)
-LAUNCHES_PER_STEP = 9
+# library kernels per step of sage_attn_fwd: kv_stats, kv_finalize, quant_q, quant_k,
+# quant_v, ds_gemm, attn_fwd_kernel
+LAUNCHES_PER_STEP = 7
 KERNEL_SOURCES = ["quantized_attention_fine_b200/csrc/attn_fwd.cu", "quantized_attention_fine_b200/csrc/sage_device.cuh"]
 
 
@@ -57,8 +58,36 @@ def dist_env():
 
 
 # ---------------------------------------------------------------------------
+# Multi-rank host logic (weak scaling: every rank runs the whole workload on its own
+# seeded inputs; no data-path collective).  Tested with gloo ranks on the CPU.
+# ---------------------------------------------------------------------------
+def rank_workload(w, rank: int):
+    """The workload with rank's own seed (the inputs differ per rank, the shapes do not)."""
+    from quantized_attention_fine_b200 import workloads as wl
+    return wl.Workload(w.name, w.B, w.H, w.N_q, w.N_kv, w.d, w.causal, w.dtype, w.seed + 7919 * rank, w.recipe)
+
+
+def max_over_ranks(values, device="cpu"):
+    """Element-wise max of per-rank timings (ms) over the process group, if any."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], device=device, dtype=torch.float64)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tops(world: int, ops_per_rank_step: float, ms_per_step: float) -> float:
+    """Aggregate throughput: the units every rank processed over the slowest rank's time."""
+    return world * ops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle sample (baseline arm and cpu_baseline key)
 # ---------------------------------------------------------------------------
+_HEAD_CACHE = {}
+
+
 def oracle_sample(w, seconds: float):
     """Time the fp64 oracle on a bounded sample of workload w: head (0, 0) of the seeded
     inputs, its pre-pass, then Q blocks in a seeded order until `seconds` have passed.
@@ -66,9 +95,11 @@ def oracle_sample(w, seconds: float):
     import numpy as np
     import oracle
     from quantized_attention_fine_b200 import workloads as wl
-    q, k, v = wl.generate(w)
-    qh, kh, vh = (x[0, 0].double().numpy() for x in (q, k, v))
-    del q, k, v
+    if w.name not in _HEAD_CACHE:  # the seeded inputs are drawn once per process
+        q, k, v = wl.generate(w)
+        _HEAD_CACHE[w.name] = tuple(x[0, 0].double().numpy() for x in (q, k, v))
+        del q, k, v
+    qh, kh, vh = _HEAD_CACHE[w.name]
     t0 = time.perf_counter()
     pre = oracle.prepass_head(qh, kh, vh)
     t_pre = time.perf_counter() - t0
@@ -222,7 +253,7 @@ def main():
     sage.load_library()
 
     # seeded inputs: each rank draws its own batch (weak scaling)
-    wr = wl.Workload(w.name, w.B, w.H, w.N_q, w.N_kv, w.d, w.causal, w.dtype, w.seed + 7919 * rank, w.recipe)
+    wr = rank_workload(w, rank)
     q_cpu, k_cpu, v_cpu = wl.generate(wr)
     q, k, v = q_cpu.to(dev), k_cpu.to(dev), v_cpu.to(dev)
     B, H, nq, nk, d = w.B, w.H, w.N_q, w.N_kv, w.d
@@ -232,17 +263,19 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        sage.quant_qk(q, k, mode=mode, workspace=ws)
-        sage.quant_v(v, n_q=nq, mode=mode, workspace=ws)
+        sage.attn_fwd(q, k, v, causal=w.causal, out=out, workspace=ws)
+
+    def attn_only():
+        sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode, out=out)
 
     for _ in range(args.warmup):
         step()
-        sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode, out=out)
+        attn_only()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     clocks = ClockSampler(local, enabled=not args.no_clocks)
     if clocks.proc is not None:
         time.sleep(0.3)
@@ -253,28 +286,28 @@ def main():
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(args.steps):
-        ev[i][0].record(stream)
         step()
-        ev[i][1].record(stream)
-        sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode, out=out)
-        ev[i][2].record(stream)
     t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    # the attention kernel alone, each launch bracketed by events on its stream
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        attn_only()
+        ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
 
     total_ms = t_start.elapsed_time(t_end)
-    attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
-    pre_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    t_tensor = torch.tensor([total_ms, statistics.mean(attn_ms), statistics.mean(pre_ms)], device=dev,
-                            dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t_tensor, op=dist.ReduceOp.MAX)
-    total_ms, attn_avg_ms, pre_avg_ms = (float(x) for x in t_tensor.tolist())
+    attn_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    total_ms, attn_avg_ms = max_over_ranks([total_ms, statistics.mean(attn_ms)], device=dev)
     ms_per_step = total_ms / args.steps
+    pre_avg_ms = ms_per_step - attn_avg_ms
     ops_step = w.ops()
-    value = world * ops_step / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tops(world, ops_step, ms_per_step)
     attn_tops = ops_step / (attn_avg_ms * 1e-3) / 1e12
 
     # end to end through the public call with host buffers: H2D of Q, K, V from pinned memory,
@@ -302,12 +335,9 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], device=dev, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e_ms = float(e_ms.item())
+        e_ms = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], device=dev)[0]
         nbytes = q.numel() * q.element_size()
-        e2e = {"value": world * ops_step / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+        e2e = {"value": whole_job_tops(world, ops_step, e_ms), "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
                "call": "sage_attn_fwd with pinned-host Q/K/V copied in and O copied out each step"}
 
@@ -335,6 +365,7 @@ def main():
                        l2="inputs (%.0f MiB) larger than L2 (126 MB); no flush" % (4 * q.numel() * 2 / 2 ** 20),
                        granularity="per_threadgroup (g_q=32, g_k=16)", pr=448, vr=448),
         "attn_kernel_tops": attn_tops, "attn_kernel_ms": attn_avg_ms, "prepass_ms": pre_avg_ms,
+        "step_call": "sage_attn_fwd (pre-pass + dS + attention); prepass_ms = ms_per_step - attn_kernel_ms",
         "attn_frac_of_spec_4500": attn_tops / SPEC_INT8_TOPS,
         "roofline": {"bound": "tensor", "achieved": attn_tops, "peak": peak, "unit": "TFLOP/s",
                      "frac": attn_tops / peak, "traffic": recorded_traffic(w.name),
