@@ -283,12 +283,14 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
         reg_fence(sv[1]);
         reg_fence(sv[2]);
         reg_fence(sv[3]);
-        tc_fence_before();
-        mbar_arrive(&sm.bar_sfree[X]);
         float mx[4];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4)
             mx[q4] = dequant_chunk(sv[q4], dq, sm.dk[0][2 * q4], sm.dk[0][2 * q4 + 1], sm.ds[0][X] + 32 * q4);
+        // S may take the next QK^T, and K slot 0 may be refilled: both are read now (the
+        // arrival must follow the dS / delta_K reads above, since it also frees the slot)
+        tc_fence_before();
+        mbar_arrive(&sm.bar_sfree[X]);
         m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         if (tile_masked(0, t, p.n_kv, off, p.causal)) m = mask_tile(sv, 0, row, p.n_kv, off, p.causal);
         bias = (m == -INFINITY) ? 0.f : p.log2_pr - m * c;
