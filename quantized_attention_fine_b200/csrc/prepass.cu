@@ -53,18 +53,36 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-// INT8 code: round-half-even of the IEEE fp32 quotient xs / delta, clamped to +-127.
-// For |xs / delta| <= 128, t = RN(xs * RN(1 / delta)) lies within 2.3e-5 of the
-// correctly rounded quotient, so when t is at least 2^-15 (3.05e-5) away from a
-// half-integer both round to the same integer; only the rare near-tie takes the
-// IEEE division.
-__device__ __forceinline__ int8_t int8_code(float xs, float delta, float inv_delta) {
-    const float t = xs * inv_delta;
-    float r;
-    if (fabsf(t - floorf(t) - 0.5f) >= 0x1p-15f) r = rintf(t);
-    else r = rintf(__fdiv_rn(xs, delta));
-    r = fminf(fmaxf(r, -127.f), 127.f);
-    return (int8_t)(int)r;
+// INT8 codes of VEC values, round-half-even of the IEEE fp32 quotient xs / delta,
+// packed little-endian.
+// - For |xs / delta| <= 128, t = RN(xs * RN(1 / delta)) lies within 2.3e-5 of the
+//   correctly rounded quotient, so when t is at least 2^-15 (3.05e-5) away from a
+//   half-integer both round to the same integer; only the rare near-tie takes the
+//   IEEE division.
+// - Rounding is done on the FMA pipe: m = RN(t + 1.5 * 2^23) holds round-half-even(t)
+//   in its low mantissa bits, so its low byte is the two's-complement code, and
+//   m - 1.5 * 2^23 is that integer exactly.
+// - delta = amax / 127 bounds |t| by 127 (1 + 3 * 2^-24) < 127.5, so the codes never
+//   leave [-127, 127] and the clamp of the definition never binds.
+template <int VEC>
+__device__ __forceinline__ uint32_t int8_codes(const float (&xs)[VEC], float delta, float inv_delta) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    uint32_t m[4] = {0, 0, 0, 0};
+    bool near_tie = false;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+        const float t = xs[v] * inv_delta;
+        const float tm = t + kMagic;
+        near_tie |= fabsf(t - (tm - kMagic)) > 0.5f - 0x1p-15f;
+        m[v] = __float_as_uint(tm);
+    }
+    if (near_tie) {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) m[v] = __float_as_uint(__fdiv_rn(xs[v], delta) + kMagic);
+    }
+    const uint32_t lo = __byte_perm(m[0], m[1], 0x0040);
+    if constexpr (VEC == 4) return __byte_perm(lo, __byte_perm(m[2], m[3], 0x0040), 0x5410);
+    return lo & 0xFFFFu;
 }
 
 // The IEEE fp32 quotient x / delta as far as its E4M3 rounding is concerned.
@@ -80,15 +98,9 @@ __device__ __forceinline__ float e4m3_quotient(float x, float delta, float inv_d
 }
 
 template <int VEC>
-__device__ __forceinline__ void store_codes(int8_t *dst, const int8_t (&c)[VEC]) {
-    if constexpr (VEC == 4) {
-        uint32_t w = (uint32_t)(uint8_t)c[0] | ((uint32_t)(uint8_t)c[1] << 8) | ((uint32_t)(uint8_t)c[2] << 16) |
-                     ((uint32_t)(uint8_t)c[3] << 24);
-        *reinterpret_cast<uint32_t *>(dst) = w;
-    } else {
-        uint16_t w = (uint16_t)((uint32_t)(uint8_t)c[0] | ((uint32_t)(uint8_t)c[1] << 8));
-        *reinterpret_cast<uint16_t *>(dst) = w;
-    }
+__device__ __forceinline__ void store_codes(int8_t *dst, uint32_t packed) {
+    if constexpr (VEC == 4) *reinterpret_cast<uint32_t *>(dst) = packed;
+    else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)packed;
 }
 
 }  // namespace
@@ -317,12 +329,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
         const float inv = 1.0f / dl;
         int8_t *q8 = reinterpret_cast<int8_t *>(a.ws + a.L.q8) + ((size_t)bh * S.nq_pad + r0 + warp * RPW) * D + lane * VEC;
 #pragma unroll
-        for (int i = 0; i < RPW; ++i) {
-            int8_t c[VEC];
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) c[v] = int8_code(x[i][v], dl, inv);
-            store_codes<VEC>(q8 + (size_t)i * D, c);
-        }
+        for (int i = 0; i < RPW; ++i) store_codes<VEC>(q8 + (size_t)i * D, int8_codes<VEC>(x[i], dl, inv));
     }
     if (s_abort && threadIdx.x == 0) rc.drain(k);
 }
@@ -374,12 +381,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_
         const float inv = 1.0f / dl;
         int8_t *k8 = reinterpret_cast<int8_t *>(a.ws + a.L.k8) + ((size_t)bh * S.nk_pad + j0 + warp * RPW) * D + lane * VEC;
 #pragma unroll
-        for (int i = 0; i < RPW; ++i) {
-            int8_t c[VEC];
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) c[v] = int8_code(x[i][v], dl, inv);
-            store_codes<VEC>(k8 + (size_t)i * D, c);
-        }
+        for (int i = 0; i < RPW; ++i) store_codes<VEC>(k8 + (size_t)i * D, int8_codes<VEC>(x[i], dl, inv));
     }
     if (s_abort && threadIdx.x == 0) rc.drain(k);
 }
