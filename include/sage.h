@@ -164,6 +164,10 @@ SAGE_API sage_status_t sage_get_device_status(void *workspace, void *stream, int
  *   SAGE_WS_KBAR  fp32  [BH][d]                  K token mean
  *   SAGE_WS_DS    fp32  [BH][Tq][nk_pad]         dS = qbar_t . K[j] (causally
  *                                                invisible entries left unwritten)
+ * Along the key axis of VT8 and DS, each 128-key tile is stored in the order
+ * (even keys, odd keys): key j of the tile starting at j0 is at position
+ * j0 + (j & 1) * 64 + (j >> 1).  The attention kernel's threads hold the even and
+ * the odd keys of a row, and PV does not depend on the order of keys.
  */
 enum {
     SAGE_WS_Q8 = 0, SAGE_WS_K8 = 1, SAGE_WS_VT8 = 2, SAGE_WS_DQ = 3, SAGE_WS_DK = 4,

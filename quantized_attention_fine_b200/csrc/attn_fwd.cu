@@ -9,20 +9,26 @@
 // in tensor memory; O = acc * delta_V / (Pr l).
 //
 // One CTA computes two 128-row Q tiles (A = 2u, B = 2u + 1) of one head, sharing
-// every K / V^T tile between them (384 threads, 12 warps):
-//   warps 0-3   softmax + epilogue of tile A (thread i owns row i = TMEM lane i)
-//   warps 4-7   softmax + epilogue of tile B
-//   warp 8      TMA producer: Q tiles once, then K tiles with their dS rows and
+// every K / V^T tile between them (640 threads, 20 warps):
+//   warps 0-7   softmax + epilogue of tile A
+//   warps 8-15  softmax + epilogue of tile B
+//   warp 16     TMA producer: Q tiles once, then K tiles with their dS rows and
 //               delta_K runs through one shared-memory ring
-//   warp 9      tensor-memory allocation and single-thread tcgen05.mma issue
-//   warp 10     TMA producer of the V^T ring
-//   warp 11     idle (it only completes the producer warpgroup)
+//   warp 17     tensor-memory allocation and single-thread tcgen05.mma issue
+//   warp 18     TMA producer of the V^T ring
+//   warp 19     idle (it only completes the producer warpgroup)
+// Half rows: each row of a tile is held by two threads of one warp, one with its
+// even and one with its odd keys (the tcgen05.ld 16x64b shape), so each scheduler
+// runs four softmax warps.  Keys are stored in every 128-key tile in the order
+// (even keys, odd keys) -- in P here, and in V^T and dS by the pre-pass -- so each
+// thread's 64 keys are contiguous; PV is a sum over keys and does not depend on
+// their order.
 // Tensor memory (512 columns): S_A 0-127, S_B 128-255 (int32), O_A 256.., O_B
 // 256 + d.. (fp32).  A softmax warpgroup releases its S buffer as soon as the
 // scores of key tile i + 1 are in registers (it reads them while exponentiating
 // tile i), so QK^T of tile i + 2 runs on the tensor core during the softmax of
-// tile i + 1; the MMA issuer serves the warpgroups in turn with the pair
-// (QK^T of tile i + 2, PV of tile i).  P is double-buffered per warpgroup.
+// tile i + 1; the MMA issuer serves the tiles in turn with the pair (QK^T of tile
+// i + 2, PV of tile i).  P is double-buffered per tile.
 // Every wait is bounded: a wait that runs out records SAGE_ERR_TIMEOUT in the
 // status block, raises a CTA-wide abort flag that makes every role leave its loop,
 // drains the copies in flight, frees tensor memory and exits.
@@ -34,21 +40,23 @@
 
 namespace sage {
 
-constexpr int kAttnThreads = 384;
+constexpr int kAttnThreads = 640;
+constexpr int kSoftmaxWarps = 16;
+constexpr int kWarpK = 16, kWarpMma = 17, kWarpV = 18;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;
 constexpr uint64_t kDrainNs = 50ull * 1000ull * 1000ull;
-// Register split (setmaxnreg): 384 threads launch with 168 registers each; the
-// producer warpgroup gives back to 40 so the two softmax warpgroups can hold 232:
-// 128 * 40 + 256 * 232 = 384 * 168.
-constexpr uint32_t kRegsProducer = 40;
-constexpr uint32_t kRegsSoftmax = 232;
+// Register split (setmaxnreg): 640 threads launch with 96 registers each; the
+// producer warpgroup gives back to 32 so the four softmax warpgroups can hold 112:
+// 128 * 32 + 512 * 112 = 640 * 96.
+constexpr uint32_t kRegsProducer = 32;
+constexpr uint32_t kRegsSoftmax = 112;
 
 // Wait-site ids recorded with a timeout.
 enum { kSiteQ = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteS = 4, kSiteP = 5, kSiteO = 6, kSiteSfree = 7, kSiteDebug = 9 };
 
 // K tiles (with their dS rows and delta_K runs) and V^T tiles travel in separate
-// rings: a K slot is free once QK^T has read it and both warpgroups have
+// rings: a K slot is free once QK^T has read it and both tiles' warps have
 // dequantized with its dS / delta_K, long before PV is done with the V^T tile of
 // the same key tile, so the K ring can run further ahead.
 template <int D>
@@ -63,8 +71,8 @@ struct __align__(1024) AttnSmem {
     uint8_t q[2][kTile * D];
     uint8_t k[KS][kTile * D];
     uint8_t v[VS][D * kTile];
-    uint8_t p[2][2][kTile * kTile];  // [Q tile][key tile parity]
-    float ds[KS][2][kTile];
+    uint8_t p[2][2][kTile * kTile];  // [Q tile][key tile parity], keys in storage order
+    float ds[KS][2][kTile];          // keys in storage order
     float dk[KS][kTile / kKeyRun];
     uint64_t bar_q, bar_kfull[KS], bar_kempty[KS], bar_vfull[VS], bar_vempty[VS];
     uint64_t bar_s[2], bar_sfree[2], bar_p[2], bar_o[2], bar_drain;
@@ -115,23 +123,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
-__device__ __forceinline__ void store_row_chunk(void *dst, const float (&y)[32], int out_bf16) {
-    uint32_t w[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        if (out_bf16) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
-            w[i] = *reinterpret_cast<uint32_t *>(&h);
-        } else {
-            __half2 h = __floats2half2_rn(y[2 * i], y[2 * i + 1]);
-            w[i] = *reinterpret_cast<uint32_t *>(&h);
-        }
-    }
-    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-}
-
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -155,20 +146,20 @@ __device__ __forceinline__ int kv_tiles_of(int t, int Tq, int Tk, int n_q, int o
     return last_key < 0 ? 0 : min(Tk, last_key / kTile + 1);
 }
 
+
 // ---------------------------------------------------------------------------
-// Softmax + epilogue of one Q tile (128 threads, one query row each).
+// Softmax + epilogue of one Q tile: 8 warps, each row held by a pair of threads
+// (t, t ^ 2) of one warp, one with the row's even keys and one with its odd keys.
 //
 // The row's work is software-pipelined across key tiles: while the exponentials
-// of tile `it` are taken (a 32-column chunk at a time), the scores of tile it + 1
-// are read from tensor memory and dequantized chunk by chunk, so the exponent
-// unit and the ALU / FMA pipes are fed from one instruction stream.  Chunk q of
-// the register array `sv` first holds tile it's dequantized scores, which the
-// exponentials consume, and is then refilled with tile it + 1's raw scores.
+// of tile `it` are taken (16 of the thread's keys at a time), the scores of tile
+// it + 1 are read from tensor memory and dequantized, so the exponent unit and the
+// ALU / FMA pipes are fed from one instruction stream.
 // ---------------------------------------------------------------------------
 
 // dS read from shared memory as inline asm, so the compiler keeps it behind the
 // tensor-memory wait of its chunk instead of hoisting a whole tile's dS into
-// registers (which would not fit beside the 128 score registers).
+// registers.
 __device__ __forceinline__ float4 lds_f32x4(const float *ptr) {
     float4 v;
     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -177,43 +168,37 @@ __device__ __forceinline__ float4 lds_f32x4(const float *ptr) {
     return v;
 }
 
-// s = S * dQ dK + dS over one 32-key chunk, in place (S int32 -> fp32 bits);
-// returns the chunk maximum.  Keys of a chunk form two runs of kKeyRun = 16 keys,
-// each with its own delta_K.
-__device__ __forceinline__ float dequant_chunk(uint32_t (&w)[32], float dq, float dk0, float dk1,
-                                               const float *ds) {
+// s = S * dQ dK + dS over 16 of a thread's keys (keys 2k + parity of a 32-key
+// chunk), in place (S int32 -> fp32 bits); ds holds their dS contiguously (storage
+// order); a_lo / a_hi scale the keys of the chunk's first / second 16-key run
+// (k < 8 / k >= 8).  Returns the maximum.
+__device__ __forceinline__ float dequant16(uint32_t (&w)[16], float a_lo, float a_hi, const float *ds) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const float a = dq * (h ? dk1 : dk0);
+    for (int j = 0; j < 16; j += 4) {
+        const float a = j < 8 ? a_lo : a_hi;
         const float2 a2 = make_float2(a, a);
-#pragma unroll
-        for (int j = 16 * h; j < 16 * h + 16; j += 4) {
-            const float4 d4 = lds_f32x4(ds + j);
-            const float2 y01 = __ffma2_rn(make_float2((float)(int)w[j], (float)(int)w[j + 1]), a2, make_float2(d4.x, d4.y));
-            const float2 y23 =
-                __ffma2_rn(make_float2((float)(int)w[j + 2], (float)(int)w[j + 3]), a2, make_float2(d4.z, d4.w));
-            w[j] = __float_as_uint(y01.x);
-            w[j + 1] = __float_as_uint(y01.y);
-            w[j + 2] = __float_as_uint(y23.x);
-            w[j + 3] = __float_as_uint(y23.y);
-        }
+        const float4 d4 = lds_f32x4(ds + j);
+        const float2 y01 = __ffma2_rn(make_float2((float)(int)w[j], (float)(int)w[j + 1]), a2, make_float2(d4.x, d4.y));
+        const float2 y23 = __ffma2_rn(make_float2((float)(int)w[j + 2], (float)(int)w[j + 3]), a2, make_float2(d4.z, d4.w));
+        w[j] = __float_as_uint(y01.x);
+        w[j + 1] = __float_as_uint(y01.y);
+        w[j + 2] = __float_as_uint(y23.x);
+        w[j + 3] = __float_as_uint(y23.y);
     }
 #define WV(j) __uint_as_float(w[j])
-    float t[10];
-#pragma unroll
-    for (int i = 0; i < 10; ++i) t[i] = max3f(WV(3 * i), WV(3 * i + 1), WV(3 * i + 2));
-    const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]), u2 = max3f(t[6], t[7], t[8]);
-    const float u3 = max3f(t[9], WV(30), WV(31));
+    const float t0 = max3f(WV(0), WV(1), WV(2)), t1 = max3f(WV(3), WV(4), WV(5)), t2 = max3f(WV(6), WV(7), WV(8));
+    const float t3 = max3f(WV(9), WV(10), WV(11)), t4 = max3f(WV(12), WV(13), WV(14));
+    return fmaxf(max3f(t0, t1, t2), max3f(t3, t4, WV(15)));
 #undef WV
-    return fmaxf(max3f(u0, u1, u2), u3);
 }
 
-// p = 2^(s c + bias) (bias = log2 Pr - m c) over one 32-key chunk: accumulates the
-// unquantized p into the row sum and packs Pr-scaled E4M3 codes, 4 per word.
-__device__ __forceinline__ void exp_chunk(const uint32_t (&w)[32], float2 c2, float2 b2, float2 &acc0, float2 &acc1,
-                                          uint32_t *pk) {
+// p = 2^(s c + bias) (bias = log2 Pr - m c) over 16 keys: accumulates the
+// unquantized p into the thread's part of the row sum and packs Pr-scaled E4M3
+// codes, 4 per word.
+__device__ __forceinline__ void exp16(const uint32_t (&w)[16], float2 c2, float2 b2, float2 &acc0, float2 &acc1,
+                                      uint32_t (&pk)[4]) {
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
+    for (int j = 0; j < 16; j += 4) {
         const float2 e01 = __ffma2_rn(make_float2(__uint_as_float(w[j]), __uint_as_float(w[j + 1])), c2, b2);
         const float2 e23 = __ffma2_rn(make_float2(__uint_as_float(w[j + 2]), __uint_as_float(w[j + 3])), c2, b2);
         const float2 p01 = make_float2(ex2_approx(e01.x), ex2_approx(e01.y));
@@ -230,38 +215,58 @@ __device__ __forceinline__ bool tile_masked(int kt, int t, int n_kv, int off, in
     return (kt * kTile + kTile > n_kv) || (causal && kt * kTile + kTile - 1 > t * kTile + off);
 }
 
-// Sets the invisible keys of key tile kt to -inf and returns the new row maximum.
-__device__ __forceinline__ float mask_tile(uint32_t (&sv)[4][32], int kt, int row, int n_kv, int off, int causal) {
+// Sets this thread's invisible keys of key tile kt to -inf (its keys are
+// 32 q + 2 k + par) and returns the maximum of its remaining scores.
+__device__ __forceinline__ float mask_tile(uint32_t (&sv)[4][16], int kt, int row, int par, int n_kv, int off,
+                                           int causal) {
     int lim = n_kv - 1 - kt * kTile;
     if (causal) lim = min(lim, row + off - kt * kTile);
     float mx = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < kTile; ++j) {
-        if (j > lim) sv[j / 32][j % 32] = __float_as_uint(-INFINITY);
-        mx = fmaxf(mx, __uint_as_float(sv[j / 32][j % 32]));
-    }
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            if (32 * q + 2 * k + par > lim) sv[q][k] = __float_as_uint(-INFINITY);
+            mx = fmaxf(mx, __uint_as_float(sv[q][k]));
+        }
     return mx;
+}
+
+// Row maximum of the two threads of a row pair.
+__device__ __forceinline__ float pair_max(float v) { return fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, 2)); }
+
+__device__ __forceinline__ uint32_t pack16x2(float lo, float hi, int out_bf16) {
+    if (out_bf16) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t *>(&h);
+    }
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
 }
 
 template <int D>
 __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &p, uint32_t tmem, int X, int t,
                                              int n_tiles, int bh, int64_t o_base, volatile int *abort_flag) {
     constexpr int KS = AttnCfg<D>::kKStages;
-    const int wq = (threadIdx.x >> 5) & 3;
+    const int w8 = (threadIdx.x >> 5) & 7;  // warp within the tile's eight
+    const int quad = w8 & 3, half = w8 >> 2;
     const int lane = threadIdx.x & 31;
-    const int r = wq * 32 + lane;
+    const int par = (lane >> 1) & 1;        // this thread's key parity (tcgen05.ld 16x64b layout)
+    const int r = 32 * quad + 16 * half + 8 * (lane & 1) + (lane >> 2);  // tile row = TMEM lane
     const int row = t * kTile + r;
-    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(32 * quad + 16 * half) << 16;
     const uint32_t s_tmem = tmem + lane_base + (uint32_t)X * 128u;
     const uint32_t o_tmem = tmem + lane_base + kTmemO + (uint32_t)X * D;
     const int off = p.n_kv - p.n_q;
-    uint16_t *orow = static_cast<uint16_t *>(p.o) + o_base + (int64_t)row * p.so_n;
+    const int pos0 = par * (kTile / 2);  // storage position of this thread's first key of a tile
+    // this thread writes output columns [par * D / 2, par * D / 2 + D / 2) of its row
+    uint16_t *orow = static_cast<uint16_t *>(p.o) + o_base + (int64_t)row * p.so_n + par * (D / 2);
 
     if (n_tiles == 0) {  // this tile's rows see no key: O = 0
         if (row < p.n_q) {
             uint4 *dst = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
-            for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < D / 16; ++i) dst[i] = make_uint4(0, 0, 0, 0);
         }
         return;
     }
@@ -270,29 +275,27 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
     const float c = p.scale_log2;
     const float2 c2 = make_float2(c, c);
     float m, l = 0.f, alpha = 1.f, bias;
-    uint32_t sv[4][32];
+    uint32_t sv[4][16];  // 32-key chunks of the tile, 16 of this thread's keys each
 
     // prologue: scores of key tile 0
     bool ok = warp_wait(&sm.bar_s[X], 0, abort_flag, p.status, kSiteS) &&
               warp_wait(&sm.bar_kfull[0], 0, abort_flag, p.status, kSiteFull);
     if (ok) {
         tc_fence_after();
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(s_tmem + q4 * 32, sv[q4]);
-        tmem_wait_ld_regs(sv[0]);
-        reg_fence(sv[1]);
-        reg_fence(sv[2]);
-        reg_fence(sv[3]);
         float mx[4];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-            mx[q4] = dequant_chunk(sv[q4], dq, sm.dk[0][2 * q4], sm.dk[0][2 * q4 + 1], sm.ds[0][X] + 32 * q4);
+        for (int q = 0; q < 4; ++q) {
+            tmem_ld16x64b_x16(s_tmem + q * 32, sv[q]);
+            tmem_wait_ld_regs16(sv[q]);
+            mx[q] = dequant16(sv[q], dq * sm.dk[0][2 * q], dq * sm.dk[0][2 * q + 1], sm.ds[0][X] + pos0 + 16 * q);
+        }
         // S may take the next QK^T, and K slot 0 may be refilled: both are read now (the
         // arrival must follow the dS / delta_K reads above, since it also frees the slot)
         tc_fence_before();
         mbar_arrive(&sm.bar_sfree[X]);
         m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        if (tile_masked(0, t, p.n_kv, off, p.causal)) m = mask_tile(sv, 0, row, p.n_kv, off, p.causal);
+        if (tile_masked(0, t, p.n_kv, off, p.causal)) m = mask_tile(sv, 0, row, par, p.n_kv, off, p.causal);
+        m = pair_max(m);
         bias = (m == -INFINITY) ? 0.f : p.log2_pr - m * c;
     }
 
@@ -309,38 +312,37 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
         const float2 b2 = make_float2(bias, bias);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         float mx[4];
-        const float *dsn = sm.ds[sn][X];
+        const float *dsn = sm.ds[sn][X] + pos0;
         const float *dkn = sm.dk[sn];
         // P(it) goes to the buffer PV(it - 2) read; that PV was waited for before P(it - 1)
         uint8_t *pbuf = sm.p[X][it & 1];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t pk[8];
-            exp_chunk(sv[q4], c2, b2, acc0, acc1, pk);
-            *reinterpret_cast<uint4 *>(pbuf + sw128_offset(r, 2 * q4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            *reinterpret_cast<uint4 *>(pbuf + sw128_offset(r, 2 * q4 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            tmem_ld32(s_tmem + q4 * 32, sv[q4]);
-            tmem_wait_ld_regs(sv[q4]);
-            mx[q4] = dequant_chunk(sv[q4], dq, dkn[2 * q4], dkn[2 * q4 + 1], dsn + 32 * q4);
+        for (int q = 0; q < 4; ++q) {
+            uint32_t pk[4];
+            exp16(sv[q], c2, b2, acc0, acc1, pk);
+            *reinterpret_cast<uint4 *>(pbuf + sw128_offset(r, par * 4 + q)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            tmem_ld16x64b_x16(s_tmem + q * 32, sv[q]);
+            tmem_wait_ld_regs16(sv[q]);
+            mx[q] = dequant16(sv[q], dq * dkn[2 * q], dq * dkn[2 * q + 1], dsn + 16 * q);
         }
         if (has_next) {  // tile it + 1's scores are in registers: its S buffer may take the next QK^T
             tc_fence_before();
             mbar_arrive(&sm.bar_sfree[X]);
         }
         const float2 acc = __fadd2_rn(acc0, acc1);
-        l = l * alpha + (acc.x + acc.y);
+        l = l * alpha + (acc.x + acc.y);  // this thread's half of the row sum
         const bool rescale = (it > 0) && (alpha != 1.f);
 
         if (it > 0) {  // PV of the previous tile must be done before O is rescaled
             if (!warp_wait(&sm.bar_o[X], (it - 1) & 1, abort_flag, p.status, kSiteO)) { ok = false; break; }
             tc_fence_after();
         }
-        if (__any_sync(0xFFFFFFFFu, rescale)) {
+        if (__any_sync(0xFFFFFFFFu, rescale)) {  // this thread's half of the row's O columns
             const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 16) {  // 16 columns at a time: the next tile's scores stay live
+            for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t ov[16];
-                tmem_ld16(o_tmem + c0, ov);
+                tmem_ld16x64b_x16(o_tmem + c0, ov);
                 tmem_wait_ld_regs16(ov);
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
@@ -348,7 +350,7 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
                     ov[i] = __float_as_uint(v2.x);
                     ov[i + 1] = __float_as_uint(v2.y);
                 }
-                tmem_st16(o_tmem + c0, ov);
+                tmem_st16x64b_x16(o_tmem + c0, ov);
             }
             tmem_wait_st();
         }
@@ -358,8 +360,9 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
 
         if (has_next) {  // running maximum with tile it + 1
             float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            if (tile_masked(it + 1, t, p.n_kv, off, p.causal)) tmax = mask_tile(sv, it + 1, row, p.n_kv, off, p.causal);
-            const float m_new = fmaxf(m, tmax);
+            if (tile_masked(it + 1, t, p.n_kv, off, p.causal))
+                tmax = mask_tile(sv, it + 1, row, par, p.n_kv, off, p.causal);
+            const float m_new = fmaxf(m, pair_max(tmax));
             if (m_new == -INFINITY) {
                 alpha = 1.f;
                 bias = 0.f;
@@ -373,23 +376,33 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
     if (ok) ok = warp_wait(&sm.bar_o[X], (n_tiles - 1) & 1, abort_flag, p.status, kSiteO);
     if (ok) {
         tc_fence_after();
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const float l_row = l + __shfl_xor_sync(0xFFFFFFFFu, l, 2);
+        const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
         const float *dv = p.dv + (size_t)bh * D;
+        // The thread holds O columns 2v + par (v < D / 2).  Output word i of the even
+        // thread is columns (2i, 2i + 1), i < D / 4; of the odd thread, columns
+        // (D / 2 + 2i, D / 2 + 2i + 1): each thread swaps half its values with its pair.
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t ov[32];
-            tmem_ld32(o_tmem + c0, ov);
-            tmem_wait_ld_regs(ov);
-            float y[32];
+        for (int cb = 0; cb < D / 64; ++cb) {
+            uint32_t lo[16], hi[16];  // values v = 16 cb + k and v = D / 4 + 16 cb + k
+            tmem_ld16x64b_x16(o_tmem + 32 * cb, lo);
+            tmem_ld16x64b_x16(o_tmem + D / 2 + 32 * cb, hi);
+            tmem_wait_ld_regs16(lo);
+            tmem_wait_ld_regs16(hi);
+            uint32_t out[16];  // output words for columns 32 cb + 2k (+ D / 2 on the odd thread)
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-                const float4 s4 = __ldg(reinterpret_cast<const float4 *>(dv + c0 + i));
-                y[i] = __uint_as_float(ov[i]) * s4.x * inv_l;
-                y[i + 1] = __uint_as_float(ov[i + 1]) * s4.y * inv_l;
-                y[i + 2] = __uint_as_float(ov[i + 2]) * s4.z * inv_l;
-                y[i + 3] = __uint_as_float(ov[i + 3]) * s4.w * inv_l;
+            for (int k = 0; k < 16; ++k) {
+                const int v_lo = 16 * cb + k, v_hi = D / 4 + 16 * cb + k;
+                const float y_lo = __uint_as_float(lo[k]) * __ldg(dv + 2 * v_lo + par) * inv_l;
+                const float y_hi = __uint_as_float(hi[k]) * __ldg(dv + 2 * v_hi + par) * inv_l;
+                const float got = __shfl_xor_sync(0xFFFFFFFFu, par ? y_lo : y_hi, 2);
+                out[k] = par ? pack16x2(got, y_hi, p.out_bf16) : pack16x2(y_lo, got, p.out_bf16);
             }
-            if (row < p.n_q) store_row_chunk(orow + c0, y, p.out_bf16);
+            if (row < p.n_q) {
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * cb);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+            }
         }
     }
 }
@@ -424,8 +437,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int s = 0; s < VS; ++s) { mbar_init(&sm.bar_vfull[s], 1); mbar_init(&sm.bar_vempty[s], 1); }
         for (int x = 0; x < 2; ++x) {
             mbar_init(&sm.bar_s[x], 1);
-            mbar_init(&sm.bar_sfree[x], 128);
-            mbar_init(&sm.bar_p[x], 128);
+            mbar_init(&sm.bar_sfree[x], 256);  // the 8 warps of the tile
+            mbar_init(&sm.bar_p[x], 256);
             mbar_init(&sm.bar_o[x], 1);
         }
         mbar_init(&sm.bar_drain, 1);
@@ -436,7 +449,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float *z = &sm.ds[0][0][0];
         for (int i = threadIdx.x; i < KS * 2 * kTile; i += kAttnThreads) z[i] = 0.f;
     }
-    if (warp == 9 && n_tiles > 0) {
+    if (warp == kWarpMma && n_tiles > 0) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -446,9 +459,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort_flag = &sm.abort_flag;
 
-    if (warp >= 8) {
+    if (warp >= kSoftmaxWarps) {
         setmaxnreg_dec<kRegsProducer>();
-        if (warp == 8 && lane == 0 && n_tiles > 0) {
+        if (warp == kWarpK && lane == 0 && n_tiles > 0) {
             // ---------------- TMA producer: Q tiles, then the K / dS / delta_K ring ----------------
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
@@ -480,7 +493,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     mbar_wait_quiet(&sm.bar_kfull[it % KS], (it / KS) & 1, kDrainNs);
                 }
             }
-        } else if (warp == 10 && lane == 0 && n_tiles > 0) {
+        } else if (warp == kWarpV && lane == 0 && n_tiles > 0) {
             // ---------------- TMA producer: the V^T ring ----------------
             prefetch_tmap(&tm_v);
             int issued = 0;
@@ -495,7 +508,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (*abort_flag)
                 for (int it = max(0, issued - VS); it < issued; ++it)
                     mbar_wait_quiet(&sm.bar_vfull[it % VS], (it / VS) & 1, kDrainNs);
-        } else if (warp == 9 && lane == 0 && n_tiles > 0) {
+        } else if (warp == kWarpMma && lane == 0 && n_tiles > 0) {
             // ------------------------------ MMA issuer ------------------------------
             // Q tile x at q_s + x * kTile * D; P buffer (x, parity) at p_s + (2 x + parity) * kTile^2
             const uint32_t q_s = smem_u32(sm.q[0]), p_s = smem_u32(sm.p[0][0]);
@@ -563,7 +576,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // all roles meet here before tensor memory is released
         tc_fence_before();
         __syncthreads();
-        if (warp == 9 && n_tiles > 0) {
+        if (warp == kWarpMma && n_tiles > 0) {
             __syncwarp();
             tc_fence_after();
             tmem_dealloc(tmem, kTmemCols);
@@ -571,8 +584,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         return;
     }
     setmaxnreg_inc<kRegsSoftmax>();
-    // one copy of the softmax code serves both warpgroups (instruction-cache footprint)
-    const int X = warp >> 2;
+    // one copy of the softmax code serves both tiles (instruction-cache footprint)
+    const int X = warp >> 3;
     if (X == 0 || hasB) softmax_role<D>(sm, p, tmem, X, X ? tB : tA, X ? nB : nA, bh, o_base, abort_flag);
     tc_fence_before();
     __syncthreads();

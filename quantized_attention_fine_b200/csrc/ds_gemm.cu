@@ -11,9 +11,9 @@
 // and 2^-22 for fp16.  tcgen05.mma kind::f16, M = 128 keys, N = up to 256 Q
 // blocks, K = 16 channels per instruction; D[key][block] in tensor memory (two
 // accumulators, so the product of one key tile overlaps the write-out of the
-// previous one), transposed through shared memory and written as dS[block][key]
-// by TMA stores.  32-block chunks whose blocks can never see a key tile (causal)
-// are not written.
+// previous one), transposed through shared memory and written as dS[block][position]
+// by TMA stores, keys of each 128-key tile in the storage order (even, then odd).
+// 32-block chunks whose blocks can never see a key tile (causal) are not written.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -198,7 +198,9 @@ __global__ void __launch_bounds__(kDsThreads, 1)
                                                                status, 25));
                         if (!ok) break;
                     }
-                    float *col = &sm.stage[sb][0][wq * 32 + lane];
+                    // key k = 32 wq + lane of the tile goes to its storage position
+                    const int key = wq * 32 + lane;
+                    float *col = &sm.stage[sb][0][(key & 1) * (kTile / 2) + (key >> 1)];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) col[e * kTile] = __uint_as_float(v[e]);
                     fence_proxy_async_smem();

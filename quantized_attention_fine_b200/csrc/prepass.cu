@@ -13,7 +13,7 @@
 //   quant_k      per (head, 128-key tile): K_s = K - kbar, INT8 codes per group,
 //                delta_K per 16-key run.
 //   quant_v      per (head, 128-key tile): V / delta_V -> E4M3, written transposed
-//                ([channel][key]).
+//                ([channel][position], keys in the tile storage order: even, then odd).
 // Every code decision (INT8 rounding, E4M3 rounding) is made on the IEEE fp32
 // quotient x / delta, rounded to nearest even, so that it is reproducible on the
 // host.  The quotient is formed as x * (1 / delta) when that product provably
@@ -386,9 +386,11 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_
     if (s_abort && threadIdx.x == 0) rc.drain(k);
 }
 
-// V codes of a 128-key tile, written transposed ([channel][key]): lane l holds the
-// 16 keys of its warp for channels l*VEC .., and stores each channel's 16 codes as
-// one 16-byte piece of that channel's row of V^T.
+// V codes of a 128-key tile, written transposed ([channel][position]) in the tile's
+// storage order: key j of a tile sits at position (j & 1) * 64 + (j >> 1) (even keys
+// first, then odd keys), the order in which the attention kernel's threads hold P.
+// Lane l holds the 16 keys of its warp for channels l*VEC ..; their 8 even and 8 odd
+// codes per channel are two 8-byte pieces of that channel's row of V^T.
 template <int D>
 __global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_constant__ PrepassArgs a) {
     constexpr int VEC = D / 32, RPW = kRowsPerWarp;
@@ -419,17 +421,23 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_
         }
         __syncthreads();  // the stage is in registers: refill it
         if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
-        uint8_t *vt8 = a.ws + a.L.vt8 + ((size_t)bh * D + lane * VEC) * S.nk_pad + j0 + warp * RPW;
+        // keys j0 + 16w + i: even i at position 8w + i/2, odd i at 64 + 8w + i/2
+        uint8_t *vt8 = a.ws + a.L.vt8 + ((size_t)bh * D + lane * VEC) * S.nk_pad + j0 + warp * (RPW / 2);
 #pragma unroll
         for (int v = 0; v < VEC; ++v) {
             const float dv = reinterpret_cast<const float *>(a.ws + a.L.dv)[(size_t)bh * D + lane * VEC + v];
             const float inv = 1.0f / dv;
-            uint32_t w[4];
+            uint32_t w[2][2];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                w[q] = pack_e4m3x4(e4m3_quotient(x[4 * q][v], dv, inv), e4m3_quotient(x[4 * q + 1][v], dv, inv),
-                                   e4m3_quotient(x[4 * q + 2][v], dv, inv), e4m3_quotient(x[4 * q + 3][v], dv, inv));
-            *reinterpret_cast<uint4 *>(vt8 + (size_t)v * S.nk_pad) = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int par = 0; par < 2; ++par)
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+                    w[par][q] = pack_e4m3x4(e4m3_quotient(x[8 * q + par][v], dv, inv),
+                                            e4m3_quotient(x[8 * q + 2 + par][v], dv, inv),
+                                            e4m3_quotient(x[8 * q + 4 + par][v], dv, inv),
+                                            e4m3_quotient(x[8 * q + 6 + par][v], dv, inv));
+            *reinterpret_cast<uint2 *>(vt8 + (size_t)v * S.nk_pad) = make_uint2(w[0][0], w[0][1]);
+            *reinterpret_cast<uint2 *>(vt8 + (size_t)v * S.nk_pad + kTile / 2) = make_uint2(w[1][0], w[1][1]);
         }
     }
     if (s_abort && threadIdx.x == 0) rc.drain(k);

@@ -58,3 +58,17 @@ def assert_close_to_oracle(o_gpu, o_orc, what=""):
     assert err <= O_MAX_ABS, "%s: max |O_gpu - O_oracle| = %.3e > %.0e" % (what, err, O_MAX_ABS)
     assert c >= O_COS_ORACLE, "%s: cos(O_gpu, O_oracle) = %.6f < %.4f" % (what, c, O_COS_ORACLE)
     return err, c
+
+
+def storage_positions(n_pad: int) -> np.ndarray:
+    """Position of key j in the workspace's key-ordered arrays (V^T codes, dS): inside
+    each 128-key tile the tile's even keys come first, then its odd keys."""
+    j = np.arange(n_pad)
+    k = j % 128
+    return (j - k) + (k & 1) * 64 + (k >> 1)
+
+
+def natural_key_order(x: np.ndarray) -> np.ndarray:
+    """An array whose last axis is in the workspace's key storage order -> natural key order."""
+    return x[..., storage_positions(x.shape[-1])]
+

@@ -16,7 +16,8 @@ import oracle
 import quantized_attention_fine_b200 as sage
 from quantized_attention_fine_b200 import workloads as wl
 
-from helpers import (O_COS_FULL, GRAN_OF, assert_close_to_oracle, cos, head_slices, oracle_head, to_np64)
+from helpers import (O_COS_FULL, GRAN_OF, assert_close_to_oracle, cos, head_slices, natural_key_order, oracle_head,
+                     storage_positions, to_np64)
 
 pytestmark = pytest.mark.gpu
 
@@ -73,11 +74,11 @@ def test_prepass_bit_exact(B, H, nq, nk, d, dtype, layout, gran):
             assert np.array_equal(views["dv"][bh].numpy(), pre["dv"]), "delta_V"
             assert np.array_equal(views["q8"][bh].numpy(), pre["q_code"]), "Q codes"
             assert np.array_equal(views["k8"][bh].numpy(), pre["k_code"]), "K codes"
-            vt = views["vt8"][bh].numpy()
+            vt = natural_key_order(views["vt8"][bh].numpy())
             assert np.array_equal(vt[:, :nk].T, pre["v_code"]), "V codes"
             assert not vt[:, nk:].any(), "V pad"
             # dS = qbar_t . K[j] (raw K; differs from the oracle's qbar_t . K_s by a per-block constant)
-            ds = views["ds"][bh].numpy()[:, :nk].astype(np.float64)
+            ds = natural_key_order(views["ds"][bh].numpy())[:, :nk].astype(np.float64)
             ref = pre["qbar"].astype(np.float64) @ to_np64(kh).T
             scale = np.abs(pre["qbar"]).astype(np.float64) @ np.abs(to_np64(kh)).T + 1e-30
             assert np.max(np.abs(ds - ref) / scale) < 1e-5, "dS"
@@ -204,7 +205,8 @@ def test_causal_rows_ignore_future_keys_bit_exact():
     g = torch.Generator(device="cuda").manual_seed(3)
     k8, vt8 = ws.view("k8"), ws.view("vt8")
     k8[:, cut:n] = torch.randint(-127, 128, k8[:, cut:n].shape, generator=g, device="cuda", dtype=torch.int8)
-    vt8[:, :, cut:n] = torch.randint(0, 0x7F, vt8[:, :, cut:n].shape, generator=g, device="cuda").to(torch.uint8)
+    pos = torch.as_tensor(storage_positions(vt8.shape[-1])[cut:n], device="cuda")  # where keys cut.. are stored
+    vt8[:, :, pos] = torch.randint(0, 0x7F, (vt8.shape[0], vt8.shape[1], n - cut), generator=g, device="cuda").to(torch.uint8)
     o2 = sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=True)
     torch.cuda.synchronize()
     assert torch.equal(o1[:, :, :cut], o2[:, :, :cut])
