@@ -64,7 +64,8 @@ def dist_env():
 def rank_workload(w, rank: int):
     """The workload with rank's own seed (the inputs differ per rank, the shapes do not)."""
     from quantized_attention_fine_b200 import workloads as wl
-    return wl.Workload(w.name, w.B, w.H, w.N_q, w.N_kv, w.d, w.causal, w.dtype, w.seed + 7919 * rank, w.recipe)
+    return wl.Workload(w.name, w.B, w.H, w.N_q, w.N_kv, w.d, w.causal, w.dtype, w.seed + 7919 * rank, w.recipe,
+                       H_kv=w.H_kv)
 
 
 def max_over_ranks(values, device="cpu"):
@@ -257,7 +258,7 @@ def main():
     q_cpu, k_cpu, v_cpu = wl.generate(wr)
     q, k, v = q_cpu.to(dev), k_cpu.to(dev), v_cpu.to(dev)
     B, H, nq, nk, d = w.B, w.H, w.N_q, w.N_kv, w.d
-    ws = sage.make_workspace(B, H, nq, nk, d, device=dev)
+    ws = sage.make_workspace(B, H, nq, nk, d, device=dev, H_kv=w.Hk)
     out = torch.empty_like(q)
     mode = sage.QuantMode.make()
     stream = torch.cuda.current_stream(dev)
@@ -356,9 +357,9 @@ def main():
         if world > 1:
             dist.barrier()
         e_ms = max_over_ranks([e2e_run(args.e2e_steps) / args.e2e_steps], device=dev)[0]
-        nbytes = q.numel() * q.element_size()
+        qbytes, kvbytes = q.numel() * q.element_size(), k.numel() * k.element_size()
         e2e = {"value": whole_job_tops(world, ops_step, e_ms), "unit": UNIT, "ms_per_step": e_ms,
-               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+               "h2d_bytes_per_step": qbytes + 2 * kvbytes, "d2h_bytes_per_step": qbytes,
                "call": "sage_attn_fwd with pinned-host Q/K/V copied in and O copied out each step; "
                        "copies and compute of neighbouring steps overlap on three streams"}
 
@@ -383,7 +384,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8+e4m3", "data": "synthetic",
         "config": dict(w.describe(), parallelism="heads sharded: each of %d rank(s) runs the full workload" % world,
-                       l2="inputs (%.0f MiB) larger than L2 (126 MB); no flush" % (4 * q.numel() * 2 / 2 ** 20),
+                       l2="inputs (%.0f MiB) larger than L2 (126 MB); no flush" % ((2 * q.numel() + 2 * k.numel()) * 2 / 2 ** 20),
                        granularity="per_threadgroup (g_q=32, g_k=16)", pr=448, vr=448),
         "attn_kernel_tops": attn_tops, "attn_kernel_ms": attn_avg_ms, "prepass_ms": pre_avg_ms,
         "step_call": "sage_attn_fwd (pre-pass + dS + attention); prepass_ms = ms_per_step - attn_kernel_ms",

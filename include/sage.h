@@ -32,7 +32,16 @@
  *   - Tensors: dtype SAGE_DTYPE_F16 / SAGE_DTYPE_BF16; layout SAGE_LAYOUT_HND is a
  *     contiguous [B, H, N, d] array, SAGE_LAYOUT_NHD a contiguous [B, N, H, d] array.
  *     Q, K, V and O share dtype and layout.  Base addresses must be 16-byte aligned.
- *   - d is 64 or 128.  Heads are multi-head (H queries heads = H key/value heads).
+ *   - d is 64 or 128.  The entry points without a suffix are multi-head (H query
+ *     heads, H key/value heads).  The `_gqa` entry points take H query heads and
+ *     H_kv key/value heads (H_kv divides H, grouped-query attention): query head h
+ *     of batch b attends to key/value head h / (H / H_kv) of batch b.  K and V are
+ *     then [B, H_kv, N_kv, d] (HND) or [B, N_kv, H_kv, d] (NHD); Q and O keep H.
+ *     K smoothing and delta_V are properties of one key/value head and are shared
+ *     by its query heads; Q smoothing and dS stay per query head.  (The pages
+ *     validate the method on multi-head attention only and name grouped-query
+ *     attention as a variant an attention backend must serve: notes on 2505.21136,
+ *     the comparison with SGLang and the list of unvalidated variants.)
  *   - The caller owns all memory, including the workspace; the library allocates
  *     nothing and keeps no state between calls.  The workspace must be at least
  *     sage_workspace_bytes(...) bytes, 1024-byte aligned, and its first 256 bytes
@@ -92,6 +101,7 @@ typedef struct {
 
 /* Bytes of workspace for one problem size (any dtype/layout).  0 on bad sizes. */
 SAGE_API size_t sage_workspace_bytes(int B, int H, int n_q, int n_kv, int d);
+SAGE_API size_t sage_workspace_bytes_gqa(int B, int H, int H_kv, int n_q, int n_kv, int d);
 
 /* Steps 1-3 (and the dS bias) for Q and K into the workspace.
  * q: [B,H,n_q,d] or [B,n_q,H,d]; k: [B,H,n_kv,d] or [B,n_kv,H,d]. */
@@ -99,12 +109,20 @@ SAGE_API sage_status_t sage_quant_qk(const void *q, const void *k, int dtype, in
                                      int B, int H, int n_q, int n_kv, int d,
                                      const sage_quant_mode_t *mode,
                                      void *workspace, size_t workspace_bytes, void *stream);
+SAGE_API sage_status_t sage_quant_qk_gqa(const void *q, const void *k, int dtype, int layout,
+                                         int B, int H, int H_kv, int n_q, int n_kv, int d,
+                                         const sage_quant_mode_t *mode,
+                                         void *workspace, size_t workspace_bytes, void *stream);
 
 /* Step 4 for V into the workspace (n_q only sizes the workspace regions). */
 SAGE_API sage_status_t sage_quant_v(const void *v, int dtype, int layout,
                                     int B, int H, int n_q, int n_kv, int d,
                                     const sage_quant_mode_t *mode,
                                     void *workspace, size_t workspace_bytes, void *stream);
+SAGE_API sage_status_t sage_quant_v_gqa(const void *v, int dtype, int layout,
+                                        int B, int H, int H_kv, int n_q, int n_kv, int d,
+                                        const sage_quant_mode_t *mode,
+                                        void *workspace, size_t workspace_bytes, void *stream);
 
 /* Steps 5-6 from a workspace filled by sage_quant_qk and sage_quant_v with the same
  * sizes and mode.  o: output, same dtype/layout as the inputs were.
@@ -116,6 +134,12 @@ SAGE_API sage_status_t sage_attn_fwd_prequant(void *o, int dtype, int layout,
                                               const sage_quant_mode_t *mode,
                                               const void *workspace, size_t workspace_bytes,
                                               void *stream);
+SAGE_API sage_status_t sage_attn_fwd_prequant_gqa(void *o, int dtype, int layout,
+                                                  int B, int H, int H_kv, int n_q, int n_kv, int d,
+                                                  int causal, float sm_scale,
+                                                  const sage_quant_mode_t *mode,
+                                                  const void *workspace, size_t workspace_bytes,
+                                                  void *stream);
 
 /* The whole forward: quant_qk + quant_v + attn_fwd_prequant, enqueued on `stream`. */
 SAGE_API sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *o,
@@ -123,6 +147,11 @@ SAGE_API sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v
                                      int d, int causal, float sm_scale,
                                      const sage_quant_mode_t *mode,
                                      void *workspace, size_t workspace_bytes, void *stream);
+SAGE_API sage_status_t sage_attn_fwd_gqa(const void *q, const void *k, const void *v, void *o,
+                                         int dtype, int layout, int B, int H, int H_kv, int n_q,
+                                         int n_kv, int d, int causal, float sm_scale,
+                                         const sage_quant_mode_t *mode,
+                                         void *workspace, size_t workspace_bytes, void *stream);
 
 /* The whole forward, exactly as sage_attn_fwd, for callers that must not allocate
  * device memory (for example a plugin whose host application owns every device
@@ -152,16 +181,17 @@ SAGE_API sage_status_t sage_attn_fwd_noalloc(const void *q, const void *k, const
 SAGE_API sage_status_t sage_get_device_status(void *workspace, void *stream, int *code, int *site);
 
 /* ---- workspace views (for tests and tools; all offsets in bytes) -------------
- * The workspace holds, per (b, h) = bh in [0, B*H), with Tq = ceil(n_q/128),
- * Tk = ceil(n_kv/128), nq_pad = 128 Tq, nk_pad = 128 Tk:
+ * The workspace holds, per query head bh = b*H + h in [0, BH = B*H) and per
+ * key/value head bk = b*H_kv + h_kv in [0, BHk = B*H_kv) (BHk = BH without _gqa),
+ * with Tq = ceil(n_q/128), Tk = ceil(n_kv/128), nq_pad = 128 Tq, nk_pad = 128 Tk:
  *   SAGE_WS_Q8    int8  [BH][nq_pad][d]          Q codes (pad rows 0)
- *   SAGE_WS_K8    int8  [BH][nk_pad][d]          K codes (pad rows 0)
- *   SAGE_WS_VT8   e4m3  [BH][d][nk_pad]          V codes, transposed (pad 0)
+ *   SAGE_WS_K8    int8  [BHk][nk_pad][d]         K codes (pad rows 0)
+ *   SAGE_WS_VT8   e4m3  [BHk][d][nk_pad]         V codes, transposed (pad 0)
  *   SAGE_WS_DQ    fp32  [BH][nq_pad]             delta_Q of each row's group
- *   SAGE_WS_DK    fp32  [BH][nk_pad/16]          delta_K of each 16-key run
- *   SAGE_WS_DV    fp32  [BH][d]                  delta_V per channel
+ *   SAGE_WS_DK    fp32  [BHk][nk_pad/16]         delta_K of each 16-key run
+ *   SAGE_WS_DV    fp32  [BHk][d]                 delta_V per channel
  *   SAGE_WS_QBAR  fp32  [BH][Tq][d]              Q block means
- *   SAGE_WS_KBAR  fp32  [BH][d]                  K token mean
+ *   SAGE_WS_KBAR  fp32  [BHk][d]                 K token mean
  *   SAGE_WS_DS    fp32  [BH][Tq][nk_pad]         dS = qbar_t . K[j] (causally
  *                                                invisible entries left unwritten)
  * Along the key axis of VT8 and DS, each 128-key tile is stored in the order
@@ -175,6 +205,7 @@ enum {
 };
 /* Byte offset of view `which` inside the workspace, or -1 for bad arguments. */
 SAGE_API int64_t sage_workspace_offset(int B, int H, int n_q, int n_kv, int d, int which);
+SAGE_API int64_t sage_workspace_offset_gqa(int B, int H, int H_kv, int n_q, int n_kv, int d, int which);
 
 /* ---- diagnostics (no counterpart on the pages' API) ---------------------------
  * INT32 scores of one (bh, Q tile, KV tile) straight from tensor memory, computed

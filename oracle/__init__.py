@@ -214,41 +214,54 @@ def attn_head(pre, *, causal=False, sm_scale=None, qblocks=None, return_stats=Fa
     return o
 
 
+def _group(H: int, H_kv: int) -> int:
+    """Query heads per key/value head."""
+    if H_kv < 1 or H % H_kv != 0:
+        raise ValueError("key/value heads (%d) must divide query heads (%d)" % (H_kv, H))
+    return H // H_kv
+
+
 def sage_attention(q, k, v, *, causal=False, sm_scale=None, granularity="per_threadgroup",
                    smooth_q=True, smooth_k=True, quant=(1, 1, 1), p_range=448.0, v_range=448.0,
                    heads=None, qblocks=None):
     """Whole quantized attention forward on [B, H, N, d] arrays (head-major).
 
-    ``heads``: optional list of (b, h) to compute (others stay 0); ``qblocks``: optional
-    list of Q block indices to compute within each head.  Returns O fp64 [B, H, Nq, d]."""
+    k and v may hold H_kv heads, H_kv dividing H (grouped-query attention): query head
+    h reads key/value head h // (H // H_kv), and the method runs on that pair as on a
+    multi-head pair.  ``heads``: optional list of (b, h) to compute (others stay 0);
+    ``qblocks``: optional list of Q block indices to compute within each head.
+    Returns O fp64 [B, H, Nq, d]."""
     q = np.asarray(q)
     k = np.asarray(k)
     v = np.asarray(v)
     B, H, nq, d = q.shape
+    group = _group(H, k.shape[1])
     g_q, g_k = GRANULARITY[granularity] if isinstance(granularity, str) else granularity
     o = np.zeros((B, H, nq, d), np.float64)
     hs = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
     for b, h in hs:
-        pre = prepass_head(q[b, h], k[b, h], v[b, h], g_q=g_q, g_k=g_k, smooth_q=smooth_q,
+        pre = prepass_head(q[b, h], k[b, h // group], v[b, h // group], g_q=g_q, g_k=g_k, smooth_q=smooth_q,
                            smooth_k=smooth_k, quant=quant, p_range=p_range, v_range=v_range)
         o[b, h] = attn_head(pre, causal=causal, sm_scale=sm_scale, qblocks=qblocks)
     return o
 
 
 def reference_attention(q, k, v, *, causal=False, sm_scale=None, heads=None):
-    """Textbook full-precision attention in fp64 (two-pass softmax), [B, H, N, d]."""
+    """Textbook full-precision attention in fp64 (two-pass softmax), [B, H, N, d].
+    k and v may hold fewer heads than q, as in sage_attention."""
     lib = _load()
     q = np.asarray(q)
     B, H, nq, d = q.shape
     nk = np.asarray(k).shape[2]
+    group = _group(H, np.asarray(k).shape[1])
     if sm_scale is None or sm_scale <= 0:
         sm_scale = 1.0 / np.sqrt(d)
     o = np.zeros((B, H, nq, d), np.float64)
     hs = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
     for b, h in hs:
         qq = np.ascontiguousarray(q[b, h], dtype=np.float64)
-        kk = np.ascontiguousarray(np.asarray(k)[b, h], dtype=np.float64)
-        vv = np.ascontiguousarray(np.asarray(v)[b, h], dtype=np.float64)
+        kk = np.ascontiguousarray(np.asarray(k)[b, h // group], dtype=np.float64)
+        vv = np.ascontiguousarray(np.asarray(v)[b, h // group], dtype=np.float64)
         oo = np.zeros((max(nq, 1), d), np.float64)
         lib.oracle_ref_attn(nq, nk, d, float(sm_scale), int(causal), _ptr(qq), _ptr(kk), _ptr(vv), _ptr(oo))
         o[b, h] = oo[:nq]

@@ -80,12 +80,21 @@ def load_library():
         lib.sage_quant_v.argtypes = [P, I, I, I, I, I, I, I, QM, P, S, P]
         lib.sage_attn_fwd_prequant.argtypes = [P, I, I, I, I, I, I, I, I, F, QM, P, S, P]
         lib.sage_attn_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, F, QM, P, S, P]
+        lib.sage_workspace_bytes_gqa.argtypes = [I] * 6
+        lib.sage_workspace_bytes_gqa.restype = S
+        lib.sage_workspace_offset_gqa.argtypes = [I] * 7
+        lib.sage_workspace_offset_gqa.restype = ctypes.c_int64
+        lib.sage_quant_qk_gqa.argtypes = [P, P, I, I, I, I, I, I, I, I, QM, P, S, P]
+        lib.sage_quant_v_gqa.argtypes = [P, I, I, I, I, I, I, I, I, QM, P, S, P]
+        lib.sage_attn_fwd_prequant_gqa.argtypes = [P, I, I, I, I, I, I, I, I, I, F, QM, P, S, P]
+        lib.sage_attn_fwd_gqa.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, F, QM, P, S, P]
         lib.sage_get_device_status.argtypes = [P, P, ctypes.POINTER(I), ctypes.POINTER(I)]
         lib.sage_debug_qk_tile.argtypes = [P, I, I, I, I, I, I, I, I, P, P]
         lib.sage_debug_pv_accumulate.argtypes = [P, P, I, I, P, P]
         lib.sage_debug_attn_fault_inject.argtypes = [P, I, I, I, I, I, I, I, I, P, S, P]
         lib.sage_version.restype = ctypes.c_char_p
         for fn in ("sage_quant_qk", "sage_quant_v", "sage_attn_fwd_prequant", "sage_attn_fwd",
+                   "sage_quant_qk_gqa", "sage_quant_v_gqa", "sage_attn_fwd_prequant_gqa", "sage_attn_fwd_gqa",
                    "sage_get_device_status", "sage_debug_qk_tile", "sage_debug_pv_accumulate",
                    "sage_debug_attn_fault_inject"):
             getattr(lib, fn).restype = ctypes.c_int
@@ -119,21 +128,20 @@ def _dtype_code(t) -> int:
 
 
 def _shape(q, k, layout):
+    """(B, H, H_kv, n_q, n_kv, d) of q and k; k may have fewer heads than q (H_kv divides H)."""
     if q.dim() != 4 or k.dim() != 4:
         raise ValueError("q, k, v must be 4-D")
     if layout == "HND":
         B, H, n_q, d = q.shape
-        n_kv = k.shape[2]
-        if k.shape[0] != B or k.shape[1] != H or k.shape[3] != d:
-            raise ValueError("k shape %s does not match q %s" % (tuple(k.shape), tuple(q.shape)))
+        H_kv, n_kv = k.shape[1], k.shape[2]
     elif layout == "NHD":
         B, n_q, H, d = q.shape
-        n_kv = k.shape[1]
-        if k.shape[0] != B or k.shape[2] != H or k.shape[3] != d:
-            raise ValueError("k shape %s does not match q %s" % (tuple(k.shape), tuple(q.shape)))
+        n_kv, H_kv = k.shape[1], k.shape[2]
     else:
         raise ValueError("layout must be 'HND' or 'NHD'")
-    return int(B), int(H), int(n_q), int(n_kv), int(d)
+    if k.shape[0] != B or k.shape[3] != d or H_kv < 1 or H % H_kv != 0:
+        raise ValueError("k shape %s does not match q %s" % (tuple(k.shape), tuple(q.shape)))
+    return int(B), int(H), int(H_kv), int(n_q), int(n_kv), int(d)
 
 
 def _ptr(t):
@@ -146,17 +154,22 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def workspace_bytes(B, H, n_q, n_kv, d) -> int:
-    return int(load_library().sage_workspace_bytes(B, H, n_q, n_kv, d))
+def workspace_bytes(B, H, n_q, n_kv, d, H_kv=None) -> int:
+    H_kv = H if H_kv is None else H_kv
+    return int(load_library().sage_workspace_bytes_gqa(B, H, H_kv, n_q, n_kv, d))
 
 
 class Workspace:
-    """Caller-owned device workspace: a zeroed uint8 tensor with a 1024-byte aligned window."""
+    """Caller-owned device workspace: a zeroed uint8 tensor with a 1024-byte aligned window.
 
-    def __init__(self, B, H, n_q, n_kv, d, device=None):
+    dims = (B, H, n_q, n_kv, d) with H query heads; H_kv key/value heads (H_kv = H
+    for multi-head attention)."""
+
+    def __init__(self, B, H, n_q, n_kv, d, device=None, H_kv=None):
         torch = _torch()
         self.dims = (int(B), int(H), int(n_q), int(n_kv), int(d))
-        self.nbytes = workspace_bytes(*self.dims)
+        self.H_kv = int(H if H_kv is None else H_kv)
+        self.nbytes = workspace_bytes(*self.dims, H_kv=self.H_kv)
         if self.nbytes == 0:
             raise SageError(SAGE_ERR_UNSUPPORTED, "sage_workspace_bytes")
         self.tensor = torch.zeros(self.nbytes + WS_ALIGN, dtype=torch.uint8, device=device or "cuda")
@@ -164,20 +177,22 @@ class Workspace:
         self.offset = (-base) % WS_ALIGN
         self.ptr = base + self.offset
 
-    def fits(self, B, H, n_q, n_kv, d) -> bool:
-        return self.dims == (int(B), int(H), int(n_q), int(n_kv), int(d))
+    def fits(self, B, H, n_q, n_kv, d, H_kv=None) -> bool:
+        H_kv = H if H_kv is None else H_kv
+        return self.dims == (int(B), int(H), int(n_q), int(n_kv), int(d)) and self.H_kv == int(H_kv)
 
     def view(self, which: str):
-        """Typed view of a workspace region (see include/sage.h, SAGE_WS_*)."""
+        """Typed view of a workspace region (see include/sage.h, SAGE_WS_*): per query
+        head for q8, dq, qbar, ds; per key/value head for k8, vt8, dk, dv, kbar."""
         torch = _torch()
         B, H, n_q, n_kv, d = self.dims
-        off = int(load_library().sage_workspace_offset(B, H, n_q, n_kv, d, WS_VIEWS[which]))
-        BH, Tq = B * H, -(-n_q // 128)
+        off = int(load_library().sage_workspace_offset_gqa(B, H, self.H_kv, n_q, n_kv, d, WS_VIEWS[which]))
+        BH, BHk, Tq = B * H, B * self.H_kv, -(-n_q // 128)
         nq_pad, nk_pad = Tq * 128, -(-n_kv // 128) * 128
-        shapes = {"q8": ((BH, nq_pad, d), torch.int8), "k8": ((BH, nk_pad, d), torch.int8),
-                  "vt8": ((BH, d, nk_pad), torch.uint8), "dq": ((BH, nq_pad), torch.float32),
-                  "dk": ((BH, nk_pad // 16), torch.float32), "dv": ((BH, d), torch.float32),
-                  "qbar": ((BH, Tq, d), torch.float32), "kbar": ((BH, d), torch.float32),
+        shapes = {"q8": ((BH, nq_pad, d), torch.int8), "k8": ((BHk, nk_pad, d), torch.int8),
+                  "vt8": ((BHk, d, nk_pad), torch.uint8), "dq": ((BH, nq_pad), torch.float32),
+                  "dk": ((BHk, nk_pad // 16), torch.float32), "dv": ((BHk, d), torch.float32),
+                  "qbar": ((BH, Tq, d), torch.float32), "kbar": ((BHk, d), torch.float32),
                   "ds": ((BH, Tq, nk_pad), torch.float32)}
         shp, dt = shapes[which]
         n = math.prod(shp) * torch.tensor([], dtype=dt).element_size()
@@ -185,38 +200,44 @@ class Workspace:
         return self.tensor[start:start + n].view(dt).view(shp)
 
 
-def make_workspace(B, H, n_q, n_kv, d, device=None) -> Workspace:
-    return Workspace(B, H, n_q, n_kv, d, device)
+def make_workspace(B, H, n_q, n_kv, d, device=None, H_kv=None) -> Workspace:
+    return Workspace(B, H, n_q, n_kv, d, device, H_kv=H_kv)
 
 
-def _ws_for(ws, B, H, n_q, n_kv, d, device):
+def _ws_for(ws, B, H, H_kv, n_q, n_kv, d, device):
     if ws is None:
-        return Workspace(B, H, n_q, n_kv, d, device)
-    if not ws.fits(B, H, n_q, n_kv, d):
-        raise ValueError("workspace was made for %s, not %s" % (ws.dims, (B, H, n_q, n_kv, d)))
+        return Workspace(B, H, n_q, n_kv, d, device, H_kv=H_kv)
+    if not ws.fits(B, H, n_q, n_kv, d, H_kv):
+        raise ValueError("workspace was made for %s (H_kv %d), not %s (H_kv %d)"
+                         % (ws.dims, ws.H_kv, (B, H, n_q, n_kv, d), H_kv))
     return ws
 
 
 def quant_qk(q, k, *, layout="HND", mode=None, workspace=None, stream=None) -> Workspace:
-    B, H, n_q, n_kv, d = _shape(q, k, layout)
-    ws = _ws_for(workspace, B, H, n_q, n_kv, d, q.device)
+    B, H, H_kv, n_q, n_kv, d = _shape(q, k, layout)
+    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, q.device)
     mode = mode or QuantMode.make()
-    _check(load_library().sage_quant_qk(_ptr(q), _ptr(k), _dtype_code(q), _LAYOUTS[layout], B, H, n_q, n_kv, d,
-                                        ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
-                                        _stream_handle(stream)), "sage_quant_qk")
+    _check(load_library().sage_quant_qk_gqa(_ptr(q), _ptr(k), _dtype_code(q), _LAYOUTS[layout], B, H, H_kv, n_q,
+                                            n_kv, d, ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
+                                            _stream_handle(stream)), "sage_quant_qk_gqa")
     return ws
 
 
-def quant_v(v, *, n_q, layout="HND", mode=None, workspace=None, stream=None) -> Workspace:
+def quant_v(v, *, n_q, H=None, layout="HND", mode=None, workspace=None, stream=None) -> Workspace:
+    """V codes and scales into the workspace.  H: query heads (default: those of
+    `workspace`, else the heads of v)."""
     if layout == "HND":
-        B, H, n_kv, d = v.shape
+        B, H_kv, n_kv, d = v.shape
     else:
-        B, n_kv, H, d = v.shape
-    ws = _ws_for(workspace, B, H, n_q, n_kv, d, v.device)
+        B, n_kv, H_kv, d = v.shape
+    if H is None:
+        H = workspace.dims[1] if workspace is not None else H_kv
+    B, H, H_kv, n_kv, d = int(B), int(H), int(H_kv), int(n_kv), int(d)
+    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, v.device)
     mode = mode or QuantMode.make()
-    _check(load_library().sage_quant_v(_ptr(v), _dtype_code(v), _LAYOUTS[layout], B, H, n_q, n_kv, d,
-                                       ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
-                                       _stream_handle(stream)), "sage_quant_v")
+    _check(load_library().sage_quant_v_gqa(_ptr(v), _dtype_code(v), _LAYOUTS[layout], B, H, H_kv, n_q, n_kv, d,
+                                           ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
+                                           _stream_handle(stream)), "sage_quant_v_gqa")
     return ws
 
 
@@ -228,30 +249,34 @@ def attn_fwd_prequant(workspace: Workspace, *, dtype, layout="HND", causal=False
         shape = (B, H, n_q, d) if layout == "HND" else (B, n_q, H, d)
         out = torch.empty(shape, dtype=dtype, device=workspace.tensor.device)
     mode = mode or QuantMode.make()
-    _check(load_library().sage_attn_fwd_prequant(_ptr(out), _dtype_code(out), _LAYOUTS[layout], B, H, n_q, n_kv, d,
-                                                 int(bool(causal)), float(sm_scale or 0.0), ctypes.byref(mode),
-                                                 ctypes.c_void_p(workspace.ptr), workspace.nbytes,
-                                                 _stream_handle(stream)), "sage_attn_fwd_prequant")
+    _check(load_library().sage_attn_fwd_prequant_gqa(_ptr(out), _dtype_code(out), _LAYOUTS[layout], B, H,
+                                                     workspace.H_kv, n_q, n_kv, d, int(bool(causal)),
+                                                     float(sm_scale or 0.0), ctypes.byref(mode),
+                                                     ctypes.c_void_p(workspace.ptr), workspace.nbytes,
+                                                     _stream_handle(stream)), "sage_attn_fwd_prequant_gqa")
     return out
 
 
 def attn_fwd(q, k, v, *, causal=False, sm_scale=None, layout="HND", granularity="per_threadgroup",
              smooth_q=True, smooth_k=True, p_range=448.0, v_range=448.0, out=None, workspace=None, stream=None):
-    """O = quantized attention of q, k, v (pre-pass + fused kernel, enqueued on the current stream)."""
+    """O = quantized attention of q, k, v (pre-pass + fused kernel, enqueued on the current stream).
+
+    k and v may have fewer heads than q (grouped-query attention): query head h
+    reads key/value head h // (H // H_kv)."""
     torch = _torch()
-    B, H, n_q, n_kv, d = _shape(q, k, layout)
+    B, H, H_kv, n_q, n_kv, d = _shape(q, k, layout)
     if v.shape != k.shape:
         raise ValueError("v shape %s must equal k shape %s" % (tuple(v.shape), tuple(k.shape)))
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share a dtype")
-    ws = _ws_for(workspace, B, H, n_q, n_kv, d, q.device)
+    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, q.device)
     if out is None:
         out = torch.empty_like(q)
     mode = QuantMode.make(granularity, smooth_q, smooth_k, p_range, v_range)
-    _check(load_library().sage_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), _LAYOUTS[layout],
-                                        B, H, n_q, n_kv, d, int(bool(causal)), float(sm_scale or 0.0),
-                                        ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
-                                        _stream_handle(stream)), "sage_attn_fwd")
+    _check(load_library().sage_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q),
+                                            _LAYOUTS[layout], B, H, H_kv, n_q, n_kv, d, int(bool(causal)),
+                                            float(sm_scale or 0.0), ctypes.byref(mode), ctypes.c_void_p(ws.ptr),
+                                            ws.nbytes, _stream_handle(stream)), "sage_attn_fwd_gqa")
     return out
 
 
@@ -271,6 +296,8 @@ def debug_qk_tile(workspace: Workspace, bh: int, q_tile: int, kv_tile: int, stre
     """INT32 S tile [128, 128] read back from tensor memory (diagnostic)."""
     torch = _torch()
     B, H, n_q, n_kv, d = workspace.dims
+    if workspace.H_kv != H:
+        raise ValueError("debug_qk_tile takes a multi-head workspace")
     out = torch.empty((128, 128), dtype=torch.int32, device=workspace.tensor.device)
     _check(load_library().sage_debug_qk_tile(ctypes.c_void_p(workspace.ptr), B, H, n_q, n_kv, d, bh, q_tile,
                                              kv_tile, _ptr(out), _stream_handle(stream)), "sage_debug_qk_tile")
@@ -291,6 +318,8 @@ def debug_pv_accumulate(p_codes, vt_codes, stream=None):
 def debug_fault_inject(workspace: Workspace, out, *, layout="HND", causal=False, stream=None):
     """Run the attention kernel with one producer signal withheld (the bounded wait must run out)."""
     B, H, n_q, n_kv, d = workspace.dims
+    if workspace.H_kv != H:
+        raise ValueError("debug_fault_inject takes a multi-head workspace")
     _check(load_library().sage_debug_attn_fault_inject(_ptr(out), _dtype_code(out), _LAYOUTS[layout], B, H, n_q,
                                                        n_kv, d, int(bool(causal)), ctypes.c_void_p(workspace.ptr),
                                                        workspace.nbytes, _stream_handle(stream)),

@@ -78,6 +78,7 @@ struct __align__(1024) AttnSmem {
     uint64_t bar_s[2], bar_sfree[2], bar_p[2], bar_o[2], bar_drain;
     uint32_t tmem_base;
     int abort_flag;
+    int bh_kv;  // key/value head of this CTA's query head (read by the epilogue)
 };
 
 // K-major operand layout of a Q or K tile: rows of d bytes; d = 128 uses the
@@ -378,7 +379,7 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
         tc_fence_after();
         const float l_row = l + __shfl_xor_sync(0xFFFFFFFFu, l, 2);
         const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
-        const float *dv = p.dv + (size_t)bh * D;
+        const float *dv = p.dv + (size_t)sm.bh_kv * D;
         // The thread holds O columns 2v + par (v < D / 2).  Output word i of the even
         // thread is columns (2i, 2i + 1), i < D / 4; of the odd thread, columns
         // (D / 2 + 2i, D / 2 + 2i + 1): each thread swaps half its values with its pair.
@@ -424,6 +425,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int u = p.causal ? (n_pairs - 1 - pair_idx) : pair_idx;
     const int tA = 2 * u, tB = 2 * u + 1;
     const int b = bh / p.H, h = bh % p.H;
+    const int bh_kv = b * p.H_kv + h / p.group;  // key/value head of query head h
     const int off = p.n_kv - p.n_q;
     const int nA = kv_tiles_of(tA, p.Tq, p.Tk, p.n_q, off, p.causal);
     const int nB = kv_tiles_of(tB, p.Tq, p.Tk, p.n_q, off, p.causal);
@@ -443,6 +445,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         mbar_init(&sm.bar_drain, 1);
         sm.abort_flag = 0;
+        sm.bh_kv = bh_kv;
         fence_mbar_init();
     }
     if (!p.use_ds) {  // without Q smoothing the dS rows stay zero
@@ -470,7 +473,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (hasB) tma_load_2d(sm.q[1], &tm_q, &sm.bar_q, 0, bh * p.nq_pad + tB * kTile);
             const float *ds_a = p.ds + ((size_t)bh * p.Tq + tA) * p.nk_pad;
             const float *ds_b = p.ds + ((size_t)bh * p.Tq + tB) * p.nk_pad;
-            const float *dk_row = p.dk + (size_t)bh * (p.nk_pad / kKeyRun);
+            const float *dk_row = p.dk + (size_t)bh_kv * (p.nk_pad / kKeyRun);
             int issued = 0;
             for (int it = 0; it < n_tiles; ++it) {
                 const int s = it % KS;
@@ -481,7 +484,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const bool dsA = p.use_ds && it < nA, dsB = p.use_ds && it < nB;
                 const uint32_t bytes = kTile * D + (dsA ? kTile * 4 : 0) + (dsB ? kTile * 4 : 0) + (kTile / kKeyRun) * 4;
                 mbar_arrive_expect_tx(&sm.bar_kfull[s], bytes);
-                tma_load_2d(sm.k[s], &tm_k, &sm.bar_kfull[s], 0, bh * p.nk_pad + it * kTile);
+                tma_load_2d(sm.k[s], &tm_k, &sm.bar_kfull[s], 0, bh_kv * p.nk_pad + it * kTile);
                 if (dsA) bulk_load(sm.ds[s][0], ds_a + it * kTile, kTile * 4, &sm.bar_kfull[s]);
                 if (dsB) bulk_load(sm.ds[s][1], ds_b + it * kTile, kTile * 4, &sm.bar_kfull[s]);
                 bulk_load(sm.dk[s], dk_row + it * (kTile / kKeyRun), (kTile / kKeyRun) * 4, &sm.bar_kfull[s]);
@@ -503,7 +506,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     break;
                 issued = it + 1;
                 mbar_arrive_expect_tx(&sm.bar_vfull[s], kTile * D);
-                tma_load_2d(sm.v[s], &tm_v, &sm.bar_vfull[s], it * kTile, bh * D);
+                tma_load_2d(sm.v[s], &tm_v, &sm.bar_vfull[s], it * kTile, bh_kv * D);
             }
             if (*abort_flag)
                 for (int it = max(0, issued - VS); it < issued; ++it)
@@ -709,7 +712,7 @@ __global__ void __launch_bounds__(128, 1)
     extern __shared__ uint8_t smem_raw[];
     PvDebugSmem<D> &sm =
         *reinterpret_cast<PvDebugSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     const int r = threadIdx.x;
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_mma, 1);

@@ -62,13 +62,13 @@ __device__ __forceinline__ float round16(float a, bool bf16) {
 template <int D>
 __global__ void __launch_bounds__(kDsThreads, 1)
     ds_gemm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ds,
-                   const float *__restrict__ qbar, int H, int Tq, int Tk, int nhd, int bf16, int causal_skip,
+                   const float *__restrict__ qbar, int H, int H_kv, int Tq, int Tk, int nhd, int bf16, int causal_skip,
                    int causal_off, int *status) {
     constexpr int KA = D / 64;
     extern __shared__ uint8_t smem_raw[];
     DsSmem<D> &sm = *reinterpret_cast<DsSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.y;
+    const int bh = blockIdx.y;  // query head
     const int jt0 = blockIdx.x * kDsTilesPerCta;
     const int n_kt = min(kDsTilesPerCta, Tk - jt0);
     const bool is_bf16 = bf16 != 0;
@@ -91,7 +91,8 @@ __global__ void __launch_bounds__(kDsThreads, 1)
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort_flag = &sm.abort_flag;
-    const int b = bh / H, h = bh % H;
+    // key/value head read by query head bh: h_kv = h / (H / H_kv)
+    const int b = bh / H, h_kv = (bh % H) / (H / H_kv), bh_kv = b * H_kv + h_kv;
 
     int g = 0;              // key tiles of earlier block chunks (buffer phases run on across chunks)
     uint32_t n_chunks = 0;  // epilogue store boxes issued (staging buffer parity)
@@ -136,8 +137,8 @@ __global__ void __launch_bounds__(kDsThreads, 1)
                 const int j0 = (jt0 + i) * kTile;
                 mbar_arrive_expect_tx(&sm.bar_kfull[buf], KA * kTile * 128);
                 for (int a = 0; a < KA; ++a) {
-                    if (nhd) tma_load_4d(sm.k[buf][a], &tm_k, &sm.bar_kfull[buf], a * 64, h, j0, b);
-                    else tma_load_3d(sm.k[buf][a], &tm_k, &sm.bar_kfull[buf], a * 64, j0, bh);
+                    if (nhd) tma_load_4d(sm.k[buf][a], &tm_k, &sm.bar_kfull[buf], a * 64, h_kv, j0, b);
+                    else tma_load_3d(sm.k[buf][a], &tm_k, &sm.bar_kfull[buf], a * 64, j0, bh_kv);
                 }
                 issued = i + 1;
             }
@@ -242,13 +243,13 @@ cudaError_t launch_ds_gemm(const CUtensorMap &tm_k, const CUtensorMap &tm_ds, co
         const size_t smem = sizeof(DsSmem<128>) + 1024;
         cudaError_t e = cudaFuncSetAttribute(ds_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        ds_gemm_kernel<128><<<grid, kDsThreads, smem, stream>>>(tm_k, tm_ds, qbar, s.H, s.Tq, s.Tk, nhd, bf16,
+        ds_gemm_kernel<128><<<grid, kDsThreads, smem, stream>>>(tm_k, tm_ds, qbar, s.H, s.H_kv, s.Tq, s.Tk, nhd, bf16,
                                                                  causal_skip, causal_off, status);
     } else {
         const size_t smem = sizeof(DsSmem<64>) + 1024;
         cudaError_t e = cudaFuncSetAttribute(ds_gemm_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        ds_gemm_kernel<64><<<grid, kDsThreads, smem, stream>>>(tm_k, tm_ds, qbar, s.H, s.Tq, s.Tk, nhd, bf16,
+        ds_gemm_kernel<64><<<grid, kDsThreads, smem, stream>>>(tm_k, tm_ds, qbar, s.H, s.H_kv, s.Tq, s.Tk, nhd, bf16,
                                                                 causal_skip, causal_off, status);
     }
     return cudaGetLastError();

@@ -5,9 +5,9 @@
 //
 // Bandwidth-bound kernels (the dS product is in ds_gemm.cu); the three quantization
 // kernels stream their input through TMA rings (see below):
-//   kv_stats     per (head, 512-token chunk): fp64 partial sums of K per channel
-//                and per-channel max |V|.
-//   kv_finalize  per head: kbar = fp32(sum / n_kv); delta_V = max|V| / Vr.
+//   kv_stats     per (key/value head, 512-token chunk): fp64 partial sums of K per
+//                channel and per-channel max |V|.
+//   kv_finalize  per key/value head: kbar = fp32(sum / n_kv); delta_V = max|V| / Vr.
 //   quant_q      per (head, 128-row block): qbar (fp64 mean of the valid rows,
 //                rounded to fp32), Q_s = Q - qbar in fp32, group amax, INT8 codes.
 //   quant_k      per (head, 128-key tile): K_s = K - kbar, INT8 codes per group,
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(256) kv_stats_kernel(const PrepassArgs a) {
     __shared__ double s_sum[8][D];
     __shared__ float s_max[8][D];
     const int chunk = blockIdx.x, bh = blockIdx.y;
-    const int b = bh / a.shape.H, h = bh % a.shape.H;
+    const int b = bh / a.shape.H_kv, h = bh % a.shape.H_kv;  // key/value head
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int j0 = chunk * kStatChunk;
     const int j1 = min(j0 + kStatChunk, a.shape.n_kv);
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_
     const Shape &S = a.shape;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *status = reinterpret_cast<int *>(a.ws + a.L.status);
-    const RingCtl<D> rc = ring_setup<D>(&a.tm_k, a.nhd, S.H, S.Tk, S.BH, s_full, &s_abort);
+    const RingCtl<D> rc = ring_setup<D>(&a.tm_k, a.nhd, S.H_kv, S.Tk, S.BH_kv, s_full, &s_abort);
     int k = 0;
     for (;; ++k) {
         const int u = blockIdx.x + k * gridDim.x;
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_
     const Shape &S = a.shape;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *status = reinterpret_cast<int *>(a.ws + a.L.status);
-    const RingCtl<D> rc = ring_setup<D>(&a.tm_v, a.nhd, S.H, S.Tk, S.BH, s_full, &s_abort);
+    const RingCtl<D> rc = ring_setup<D>(&a.tm_v, a.nhd, S.H_kv, S.Tk, S.BH_kv, s_full, &s_abort);
     int k = 0;
     for (;; ++k) {
         const int u = blockIdx.x + k * gridDim.x;
@@ -448,8 +448,8 @@ template <int D>
 static cudaError_t launch_prepass_d(const PrepassArgs &a, cudaStream_t stream) {
     const Shape &S = a.shape;
     if (a.k || a.v) {
-        kv_stats_kernel<D><<<dim3(S.n_chunks, S.BH), 256, 0, stream>>>(a);
-        kv_finalize_kernel<D><<<S.BH, D, 0, stream>>>(a);
+        kv_stats_kernel<D><<<dim3(S.n_chunks, S.BH_kv), 256, 0, stream>>>(a);
+        kv_finalize_kernel<D><<<S.BH_kv, D, 0, stream>>>(a);
     }
     // persistent grids: two CTAs per SM, or one per work unit if fewer
     int dev = 0, sms = 148;
@@ -462,11 +462,11 @@ static cudaError_t launch_prepass_d(const PrepassArgs &a, cudaStream_t stream) {
     }
     if (a.k) {
         cudaFuncSetAttribute(quant_k_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        quant_k_kernel<D><<<grid_of(S.BH * S.Tk), kQuantThreads, smem, stream>>>(a);
+        quant_k_kernel<D><<<grid_of(S.BH_kv * S.Tk), kQuantThreads, smem, stream>>>(a);
     }
     if (a.v) {
         cudaFuncSetAttribute(quant_v_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        quant_v_kernel<D><<<grid_of(S.BH * S.Tk), kQuantThreads, smem, stream>>>(a);
+        quant_v_kernel<D><<<grid_of(S.BH_kv * S.Tk), kQuantThreads, smem, stream>>>(a);
     }
     return cudaGetLastError();
 }

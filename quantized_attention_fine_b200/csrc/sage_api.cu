@@ -55,8 +55,10 @@ sage_status_t read_mode(const sage_quant_mode_t *m, Mode *out) {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Sizes shared by all entry points.  Returns SAGE_OK and fills *s, or an error.
-sage_status_t check_sizes(int B, int H, int n_q, int n_kv, int d, Shape *s) {
+// H query heads, H_kv key/value heads (H_kv divides H).
+sage_status_t check_sizes(int B, int H, int H_kv, int n_q, int n_kv, int d, Shape *s) {
     if (B < 0 || H < 0 || n_q < 0 || n_kv < 0) return SAGE_ERR_INVALID_ARG;
+    if (H_kv < 0 || (H > 0 && (H_kv == 0 || H % H_kv != 0)) || (H == 0 && H_kv != 0)) return SAGE_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
     // TMA coordinates are 32-bit signed: BH * padded length must stay below 2^31.
     const int64_t bh = (int64_t)B * H;
@@ -64,7 +66,7 @@ sage_status_t check_sizes(int B, int H, int n_q, int n_kv, int d, Shape *s) {
     const int64_t nk_pad = ((int64_t)n_kv + kTile - 1) / kTile * kTile;
     if (bh * nq_pad >= (1ll << 31) || bh * nk_pad >= (1ll << 31) || bh * d >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
     if ((bh * ((nq_pad + kTile - 1) / kTile)) >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
-    *s = make_shape(B, H, n_q, n_kv, d);
+    *s = make_shape(B, H, H_kv, n_q, n_kv, d);
     return SAGE_OK;
 }
 
@@ -96,8 +98,8 @@ bool make_maps(const Shape &s, const uint8_t *ws, CUtensorMap *tq, CUtensorMap *
     const CUtensorMapSwizzle swz_qk = (s.d == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     const uint64_t d = (uint64_t)s.d;
     if (tq && !encode_2d(tq, ws + L.q8, d, (uint64_t)s.BH * s.nq_pad, d, (uint32_t)d, kTile, swz_qk)) return false;
-    if (tk && !encode_2d(tk, ws + L.k8, d, (uint64_t)s.BH * s.nk_pad, d, (uint32_t)d, kTile, swz_qk)) return false;
-    if (tv && !encode_2d(tv, ws + L.vt8, (uint64_t)s.nk_pad, (uint64_t)s.BH * d, (uint64_t)s.nk_pad, kTile,
+    if (tk && !encode_2d(tk, ws + L.k8, d, (uint64_t)s.BH_kv * s.nk_pad, d, (uint32_t)d, kTile, swz_qk)) return false;
+    if (tv && !encode_2d(tv, ws + L.vt8, (uint64_t)s.nk_pad, (uint64_t)s.BH_kv * d, (uint64_t)s.nk_pad, kTile,
                          (uint32_t)d, CU_TENSOR_MAP_SWIZZLE_128B))
         return false;
     return true;
@@ -114,15 +116,15 @@ bool make_k16_map(CUtensorMap *map, const void *k, int dtype, int layout, const 
     const uint64_t d = (uint64_t)s.d;
     CUresult r;
     if (layout == SAGE_LAYOUT_HND) {
-        cuuint64_t dims[3] = {d, (uint64_t)s.n_kv, (uint64_t)s.BH};
+        cuuint64_t dims[3] = {d, (uint64_t)s.n_kv, (uint64_t)s.BH_kv};
         cuuint64_t strides[2] = {d * 2, (uint64_t)s.n_kv * d * 2};
         cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
         cuuint32_t estr[3] = {1, 1, 1};
         r = enc(map, dt, 3, const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     } else {
-        cuuint64_t dims[4] = {d, (uint64_t)s.H, (uint64_t)s.n_kv, (uint64_t)s.B};
-        cuuint64_t strides[3] = {d * 2, (uint64_t)s.H * d * 2, (uint64_t)s.n_kv * s.H * d * 2};
+        cuuint64_t dims[4] = {d, (uint64_t)s.H_kv, (uint64_t)s.n_kv, (uint64_t)s.B};
+        cuuint64_t strides[3] = {d * 2, (uint64_t)s.H_kv * d * 2, (uint64_t)s.n_kv * s.H_kv * d * 2};
         cuuint32_t box[4] = {64, 1, (cuuint32_t)kTile, 1};
         cuuint32_t estr[4] = {1, 1, 1, 1};
         r = enc(map, dt, 4, const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -133,14 +135,14 @@ bool make_k16_map(CUtensorMap *map, const void *k, int dtype, int layout, const 
 
 // Load map of a caller's 16-bit Q, K or V (n rows per head): d x 128-row boxes, no
 // swizzle; rows past n read as zero.
-bool make_rows16_map(CUtensorMap *map, const void *x, int dtype, int layout, const Shape &s, int n) {
+bool make_rows16_map(CUtensorMap *map, const void *x, int dtype, int layout, const Shape &s, int n, int heads) {
     auto enc = get_encode();
     if (!enc) return false;
     const CUtensorMapDataType dt =
         (dtype == SAGE_DTYPE_BF16) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const uint64_t d = (uint64_t)s.d;
     if (layout == SAGE_LAYOUT_HND) {
-        cuuint64_t dims[3] = {d, (uint64_t)n, (uint64_t)s.BH};
+        cuuint64_t dims[3] = {d, (uint64_t)n, (uint64_t)s.B * heads};
         cuuint64_t strides[2] = {d * 2, (uint64_t)n * d * 2};
         cuuint32_t box[3] = {(cuuint32_t)d, (cuuint32_t)kTile, 1};
         cuuint32_t estr[3] = {1, 1, 1};
@@ -148,8 +150,8 @@ bool make_rows16_map(CUtensorMap *map, const void *x, int dtype, int layout, con
                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     }
-    cuuint64_t dims[4] = {d, (uint64_t)s.H, (uint64_t)n, (uint64_t)s.B};
-    cuuint64_t strides[3] = {d * 2, (uint64_t)s.H * d * 2, (uint64_t)n * s.H * d * 2};
+    cuuint64_t dims[4] = {d, (uint64_t)heads, (uint64_t)n, (uint64_t)s.B};
+    cuuint64_t strides[3] = {d * 2, (uint64_t)heads * d * 2, (uint64_t)n * heads * d * 2};
     cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)kTile, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(map, dt, 4, const_cast<void *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -179,11 +181,11 @@ sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype
     a.v = v;
     a.bf16 = (dtype == SAGE_DTYPE_BF16);
     a.nhd = (layout == SAGE_LAYOUT_NHD);
-    if (q && !make_rows16_map(&a.tm_q, q, dtype, layout, s, s.n_q)) return SAGE_ERR_CUDA;
-    if (k && !make_rows16_map(&a.tm_k, k, dtype, layout, s, s.n_kv)) return SAGE_ERR_CUDA;
-    if (v && !make_rows16_map(&a.tm_v, v, dtype, layout, s, s.n_kv)) return SAGE_ERR_CUDA;
+    if (q && !make_rows16_map(&a.tm_q, q, dtype, layout, s, s.n_q, s.H)) return SAGE_ERR_CUDA;
+    if (k && !make_rows16_map(&a.tm_k, k, dtype, layout, s, s.n_kv, s.H_kv)) return SAGE_ERR_CUDA;
+    if (v && !make_rows16_map(&a.tm_v, v, dtype, layout, s, s.n_kv, s.H_kv)) return SAGE_ERR_CUDA;
     a.sq = make_strides(layout, s.H, s.n_q, s.d);
-    a.skv = make_strides(layout, s.H, s.n_kv, s.d);
+    a.skv = make_strides(layout, s.H_kv, s.n_kv, s.d);
     a.shape = s;
     a.g_q = m.g_q;
     a.g_k = m.g_k;
@@ -221,6 +223,8 @@ sage_status_t run_attention(void *o, int dtype, int layout, const Shape &s, int 
     p.so_h = so.h;
     p.so_n = so.n;
     p.H = s.H;
+    p.H_kv = s.H_kv;
+    p.group = s.H / s.H_kv;
     p.n_q = s.n_q;
     p.n_kv = s.n_kv;
     p.Tq = s.Tq;
@@ -255,15 +259,19 @@ sage_status_t check_common(int dtype, int layout) {
 
 extern "C" {
 
-size_t sage_workspace_bytes(int B, int H, int n_q, int n_kv, int d) {
+size_t sage_workspace_bytes_gqa(int B, int H, int H_kv, int n_q, int n_kv, int d) {
     Shape s;
-    if (check_sizes(B, H, n_q, n_kv, d, &s) != SAGE_OK) return 0;
+    if (check_sizes(B, H, H_kv, n_q, n_kv, d, &s) != SAGE_OK) return 0;
     return ws_layout(s).total;
 }
 
-int64_t sage_workspace_offset(int B, int H, int n_q, int n_kv, int d, int which) {
+size_t sage_workspace_bytes(int B, int H, int n_q, int n_kv, int d) {
+    return sage_workspace_bytes_gqa(B, H, H, n_q, n_kv, d);
+}
+
+int64_t sage_workspace_offset_gqa(int B, int H, int H_kv, int n_q, int n_kv, int d, int which) {
     Shape s;
-    if (check_sizes(B, H, n_q, n_kv, d, &s) != SAGE_OK) return -1;
+    if (check_sizes(B, H, H_kv, n_q, n_kv, d, &s) != SAGE_OK) return -1;
     const WsLayout L = ws_layout(s);
     switch (which) {
         case SAGE_WS_Q8: return (int64_t)L.q8;
@@ -279,13 +287,17 @@ int64_t sage_workspace_offset(int B, int H, int n_q, int n_kv, int d, int which)
     }
 }
 
-sage_status_t sage_quant_qk(const void *q, const void *k, int dtype, int layout, int B, int H, int n_q, int n_kv,
-                            int d, const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes,
-                            void *stream) {
+int64_t sage_workspace_offset(int B, int H, int n_q, int n_kv, int d, int which) {
+    return sage_workspace_offset_gqa(B, H, H, n_q, n_kv, d, which);
+}
+
+sage_status_t sage_quant_qk_gqa(const void *q, const void *k, int dtype, int layout, int B, int H, int H_kv, int n_q,
+                                int n_kv, int d, const sage_quant_mode_t *mode, void *workspace,
+                                size_t workspace_bytes, void *stream) {
     Shape s;
     Mode m;
     SAGE_TRY(check_common(dtype, layout));
-    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
     if (s.BH == 0 || (n_q == 0 && n_kv == 0)) return SAGE_OK;
     if ((n_q > 0 && !q) || (n_kv > 0 && !k)) return SAGE_ERR_INVALID_ARG;
@@ -295,12 +307,19 @@ sage_status_t sage_quant_qk(const void *q, const void *k, int dtype, int layout,
                        static_cast<uint8_t *>(workspace), 0, 0, static_cast<cudaStream_t>(stream));
 }
 
-sage_status_t sage_quant_v(const void *v, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
-                           const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes, void *stream) {
+sage_status_t sage_quant_qk(const void *q, const void *k, int dtype, int layout, int B, int H, int n_q, int n_kv,
+                            int d, const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+    return sage_quant_qk_gqa(q, k, dtype, layout, B, H, H, n_q, n_kv, d, mode, workspace, workspace_bytes, stream);
+}
+
+sage_status_t sage_quant_v_gqa(const void *v, int dtype, int layout, int B, int H, int H_kv, int n_q, int n_kv,
+                               int d, const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes,
+                               void *stream) {
     Shape s;
     Mode m;
     SAGE_TRY(check_common(dtype, layout));
-    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
     if (s.BH == 0 || n_kv == 0) return SAGE_OK;
     if (!v) return SAGE_ERR_INVALID_ARG;
@@ -310,13 +329,19 @@ sage_status_t sage_quant_v(const void *v, int dtype, int layout, int B, int H, i
                        static_cast<cudaStream_t>(stream));
 }
 
-sage_status_t sage_attn_fwd_prequant(void *o, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
-                                     int causal, float sm_scale, const sage_quant_mode_t *mode,
-                                     const void *workspace, size_t workspace_bytes, void *stream) {
+sage_status_t sage_quant_v(const void *v, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
+                           const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes, void *stream) {
+    return sage_quant_v_gqa(v, dtype, layout, B, H, H, n_q, n_kv, d, mode, workspace, workspace_bytes, stream);
+}
+
+sage_status_t sage_attn_fwd_prequant_gqa(void *o, int dtype, int layout, int B, int H, int H_kv, int n_q,
+                                         int n_kv, int d, int causal, float sm_scale,
+                                         const sage_quant_mode_t *mode, const void *workspace,
+                                         size_t workspace_bytes, void *stream) {
     Shape s;
     Mode m;
     SAGE_TRY(check_common(dtype, layout));
-    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
     if (s.BH == 0 || n_q == 0) return SAGE_OK;
     if (!o) return SAGE_ERR_INVALID_ARG;
@@ -328,13 +353,21 @@ sage_status_t sage_attn_fwd_prequant(void *o, int dtype, int layout, int B, int 
     return run_attention(o, dtype, layout, s, causal, sm_scale, m, static_cast<const uint8_t *>(workspace), 0, st);
 }
 
-sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *o, int dtype, int layout, int B,
-                            int H, int n_q, int n_kv, int d, int causal, float sm_scale,
-                            const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes, void *stream) {
+sage_status_t sage_attn_fwd_prequant(void *o, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
+                                     int causal, float sm_scale, const sage_quant_mode_t *mode,
+                                     const void *workspace, size_t workspace_bytes, void *stream) {
+    return sage_attn_fwd_prequant_gqa(o, dtype, layout, B, H, H, n_q, n_kv, d, causal, sm_scale, mode, workspace,
+                                      workspace_bytes, stream);
+}
+
+sage_status_t sage_attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, int dtype, int layout, int B,
+                                int H, int H_kv, int n_q, int n_kv, int d, int causal, float sm_scale,
+                                const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes,
+                                void *stream) {
     Shape s;
     Mode m;
     SAGE_TRY(check_common(dtype, layout));
-    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
     if (s.BH == 0 || n_q == 0) return SAGE_OK;
     if (!q || !o || (n_kv > 0 && (!k || !v))) return SAGE_ERR_INVALID_ARG;
@@ -346,6 +379,13 @@ sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *o
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     SAGE_TRY(run_prepass(q, k, v, dtype, layout, s, m, ws, causal ? 1 : 0, n_kv - n_q, st));
     return run_attention(o, dtype, layout, s, causal, sm_scale, m, ws, 0, st);
+}
+
+sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *o, int dtype, int layout, int B,
+                            int H, int n_q, int n_kv, int d, int causal, float sm_scale,
+                            const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes, void *stream) {
+    return sage_attn_fwd_gqa(q, k, v, o, dtype, layout, B, H, H, n_q, n_kv, d, causal, sm_scale, mode, workspace,
+                             workspace_bytes, stream);
 }
 
 sage_status_t sage_get_device_status(void *workspace, void *stream, int *code, int *site) {
@@ -364,7 +404,7 @@ sage_status_t sage_get_device_status(void *workspace, void *stream, int *code, i
 sage_status_t sage_debug_qk_tile(const void *workspace, int B, int H, int n_q, int n_kv, int d, int bh, int q_tile,
                                  int kv_tile, int32_t *s_out, void *stream) {
     Shape s;
-    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    SAGE_TRY(check_sizes(B, H, H, n_q, n_kv, d, &s));
     if (!workspace || !s_out || s.BH == 0 || n_q == 0 || n_kv == 0) return SAGE_ERR_INVALID_ARG;
     if (bh < 0 || bh >= s.BH || q_tile < 0 || q_tile >= s.Tq || kv_tile < 0 || kv_tile >= s.Tk)
         return SAGE_ERR_INVALID_ARG;
@@ -395,7 +435,7 @@ sage_status_t sage_debug_attn_fault_inject(void *o, int dtype, int layout, int B
     Shape s;
     Mode m;
     SAGE_TRY(check_common(dtype, layout));
-    SAGE_TRY(check_sizes(B, H, n_q, n_kv, d, &s));
+    SAGE_TRY(check_sizes(B, H, H, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(nullptr, &m));
     if (!o || s.BH == 0 || n_q == 0 || n_kv == 0) return SAGE_ERR_INVALID_ARG;
     SAGE_TRY(check_ws(s, workspace, workspace_bytes));

@@ -14,15 +14,18 @@ constexpr int kStatChunk = 512;   // tokens per CTA of the K-mean / V-amax pass
 constexpr size_t kWsAlign = 1024;
 constexpr size_t kStatusBytes = 256;
 
+// H query heads share H_kv key/value heads (H_kv divides H; H_kv = H is multi-head
+// attention): query head h reads key/value head h / (H / H_kv).
 struct Shape {
-    int B, H, n_q, n_kv, d;
-    int BH, Tq, Tk, nq_pad, nk_pad, n_chunks;
+    int B, H, H_kv, n_q, n_kv, d;
+    int BH, BH_kv, Tq, Tk, nq_pad, nk_pad, n_chunks;
 };
 
-inline Shape make_shape(int B, int H, int n_q, int n_kv, int d) {
+inline Shape make_shape(int B, int H, int H_kv, int n_q, int n_kv, int d) {
     Shape s;
-    s.B = B; s.H = H; s.n_q = n_q; s.n_kv = n_kv; s.d = d;
+    s.B = B; s.H = H; s.H_kv = H_kv; s.n_q = n_q; s.n_kv = n_kv; s.d = d;
     s.BH = B * H;
+    s.BH_kv = B * H_kv;
     s.Tq = (n_q + kTile - 1) / kTile;
     s.Tk = (n_kv + kTile - 1) / kTile;
     s.nq_pad = s.Tq * kTile;
@@ -41,21 +44,21 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline WsLayout ws_layout(const Shape &s) {
     WsLayout w;
-    const size_t BH = (size_t)s.BH, d = (size_t)s.d;
+    const size_t BH = (size_t)s.BH, BHk = (size_t)s.BH_kv, d = (size_t)s.d;
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, kWsAlign); return o; };
     w.status = take(kStatusBytes);
     w.q8 = take(BH * s.nq_pad * d);
-    w.k8 = take(BH * s.nk_pad * d);
-    w.vt8 = take(BH * d * s.nk_pad);
+    w.k8 = take(BHk * s.nk_pad * d);
+    w.vt8 = take(BHk * d * s.nk_pad);
     w.dq = take(BH * s.nq_pad * 4);
-    w.dk = take(BH * (s.nk_pad / kKeyRun) * 4);
-    w.dv = take(BH * d * 4);
+    w.dk = take(BHk * (s.nk_pad / kKeyRun) * 4);
+    w.dv = take(BHk * d * 4);
     w.qbar = take(BH * s.Tq * d * 4);
-    w.kbar = take(BH * d * 4);
+    w.kbar = take(BHk * d * 4);
     w.ds = take(BH * s.Tq * (size_t)s.nk_pad * 4);
-    w.ksum_part = take(BH * s.n_chunks * d * 8);
-    w.vmax_part = take(BH * s.n_chunks * d * 4);
+    w.ksum_part = take(BHk * s.n_chunks * d * 8);
+    w.vmax_part = take(BHk * s.n_chunks * d * 4);
     w.total = off;
     return w;
 }
@@ -90,6 +93,8 @@ struct AttnParams {
     void *o;
     int64_t so_b, so_h, so_n;
     int H, n_q, n_kv, Tq, Tk, nq_pad, nk_pad, BH;
+    int group;          // query heads per key/value head (H / H_kv)
+    int H_kv;
     int causal;
     int use_ds;         // 0: Q smoothing off, dS not read
     int out_bf16;

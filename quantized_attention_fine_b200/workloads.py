@@ -30,7 +30,12 @@ class Workload:
     dtype: torch.dtype
     seed: int
     recipe: str
+    H_kv: int = 0   # key/value heads (grouped-query attention); 0 means H (multi-head)
     extra: dict = field(default_factory=dict, compare=False, hash=False)
+
+    @property
+    def Hk(self) -> int:
+        return self.H_kv or self.H
 
     def ops(self) -> float:
         """Algorithmic tensor ops 4 B H Nq Nkv d (QK^T and PV, 2 ops per MAC), halved if causal."""
@@ -38,8 +43,8 @@ class Workload:
         return o / 2.0 if self.causal else o
 
     def describe(self) -> dict:
-        return {"workload": self.name, "B": self.B, "H": self.H, "N_q": self.N_q, "N_kv": self.N_kv,
-                "d": self.d, "causal": self.causal, "dtype": str(self.dtype).replace("torch.", ""),
+        return {"workload": self.name, "B": self.B, "H": self.H, "H_kv": self.Hk, "N_q": self.N_q,
+                "N_kv": self.N_kv, "d": self.d, "causal": self.causal, "dtype": str(self.dtype).replace("torch.", ""),
                 "seed": self.seed, "recipe": self.recipe}
 
 
@@ -48,8 +53,11 @@ TINY = Workload("tiny", 1, 2, 256, 256, 64, False, torch.float16, SEED_BASE + 0,
 IMAGE_DIT = Workload("image_dit", 2, 16, 4096, 4096, 128, False, torch.bfloat16, SEED_BASE + 1, "image_dit")
 LLM_PREFILL = Workload("llm_prefill", 1, 32, 32768, 32768, 128, True, torch.bfloat16, SEED_BASE + 2, "llm")
 VIDEO_DIT = Workload("video_dit", 2, 48, 17776, 17776, 64, False, torch.bfloat16, SEED_BASE + 3, "video_dit")
+# LLM prefill with grouped-query attention: 32 query heads over 8 key/value heads
+LLM_PREFILL_GQA = Workload("llm_prefill_gqa", 1, 32, 32768, 32768, 128, True, torch.bfloat16, SEED_BASE + 5, "llm",
+                           H_kv=8)
 
-WORKLOADS = {w.name: w for w in (TINY, IMAGE_DIT, LLM_PREFILL, VIDEO_DIT)}
+WORKLOADS = {w.name: w for w in (TINY, IMAGE_DIT, LLM_PREFILL, VIDEO_DIT, LLM_PREFILL_GQA)}
 
 SWEEP_N = (1024, 2048, 4096, 8192, 16384, 32768, 65536)
 
@@ -72,9 +80,9 @@ def by_name(name: str) -> Workload:
     raise KeyError("unknown workload %r" % name)
 
 
-def custom(name, B, H, N_q, N_kv, d, causal, dtype=torch.bfloat16, seed=SEED_BASE + 99, recipe="image_dit"):
+def custom(name, B, H, N_q, N_kv, d, causal, dtype=torch.bfloat16, seed=SEED_BASE + 99, recipe="image_dit", H_kv=0):
     """A workload with the value recipe of one of the families but other sizes (tests)."""
-    return Workload(name, B, H, N_q, N_kv, d, causal, dtype, seed, recipe)
+    return Workload(name, B, H, N_q, N_kv, d, causal, dtype, seed, recipe, H_kv=H_kv)
 
 
 def _rope(x: torch.Tensor, base: float = 10000.0) -> torch.Tensor:
@@ -89,29 +97,29 @@ def _rope(x: torch.Tensor, base: float = 10000.0) -> torch.Tensor:
 
 
 def generate(w: Workload):
-    """Q [B,H,Nq,d], K, V [B,H,Nkv,d] on the CPU, head-major, in the workload dtype."""
+    """Q [B,H,Nq,d], K, V [B,H_kv,Nkv,d] on the CPU, head-major, in the workload dtype."""
     g = torch.Generator().manual_seed(w.seed)
-    B, H, nq, nk, d = w.B, w.H, w.N_q, w.N_kv, w.d
+    B, H, Hk, nq, nk, d = w.B, w.H, w.Hk, w.N_q, w.N_kv, w.d
     q = torch.randn((B, H, nq, d), generator=g, dtype=torch.float32)
-    k = torch.randn((B, H, nk, d), generator=g, dtype=torch.float32)
-    v = torch.randn((B, H, nk, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, Hk, nk, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, Hk, nk, d), generator=g, dtype=torch.float32)
     if w.recipe == "tiny":
         # per-channel K offset, variance 4, shared across tokens
-        k += math.sqrt(4.0) * torch.randn((B, H, 1, d), generator=g)
+        k += math.sqrt(4.0) * torch.randn((B, Hk, 1, d), generator=g)
     elif w.recipe == "image_dit":
-        k += math.sqrt(8.0) * torch.randn((B, H, 1, d), generator=g)
+        k += math.sqrt(8.0) * torch.randn((B, Hk, 1, d), generator=g)
         mask = torch.rand((B, H, nq, d), generator=g) < 0.01
         q = torch.where(mask, q * 20.0, q)
     elif w.recipe == "llm":
-        k += math.sqrt(5.0) * torch.randn((B, H, 1, d), generator=g)
+        k += math.sqrt(5.0) * torch.randn((B, Hk, 1, d), generator=g)
         q = _rope(q)
         k = _rope(k)
     elif w.recipe == "video_dit":
-        k += math.sqrt(10.0) * torch.randn((B, H, 1, d), generator=g)
-        log_std = torch.rand((B, H, 1, d), generator=g) * 3.0 - 2.0     # U(-2, 1)
+        k += math.sqrt(10.0) * torch.randn((B, Hk, 1, d), generator=g)
+        log_std = torch.rand((B, Hk, 1, d), generator=g) * 3.0 - 2.0     # U(-2, 1)
         v = v * torch.pow(10.0, log_std)
     elif w.recipe == "sweep":
-        k += math.sqrt(5.0) * torch.randn((B, H, 1, d), generator=g)
+        k += math.sqrt(5.0) * torch.randn((B, Hk, 1, d), generator=g)
         mask = torch.rand((B, H, nq, d), generator=g) < 0.01
         q = torch.where(mask, q * 20.0, q)
     else:

@@ -68,6 +68,39 @@ def test_workspace_layout_regions_are_aligned_and_disjoint(lib, dims):
     assert spans[-1][1] <= total
 
 
+@pytest.mark.parametrize("dims", [(1, 8, 2, 256, 300, 64), (2, 32, 8, 4096, 4096, 128), (1, 6, 1, 1, 129, 128)])
+def test_gqa_workspace_regions_sized_per_kv_head(lib, dims):
+    """Per-query-head regions take B*H rows, per-key/value-head regions B*H_kv."""
+    B, H, Hk, nq, nk, d = dims
+    total = sage.workspace_bytes(B, H, nq, nk, d, H_kv=Hk)
+    assert 0 < total < sage.workspace_bytes(B, H, nq, nk, d)
+    BH, BHk, Tq = B * H, B * Hk, -(-nq // 128)
+    nq_pad, nk_pad = Tq * 128, -(-nk // 128) * 128
+    sizes = {0: BH * nq_pad * d, 1: BHk * nk_pad * d, 2: BHk * d * nk_pad, 3: BH * nq_pad * 4,
+             4: BHk * nk_pad // 16 * 4, 5: BHk * d * 4, 6: BH * Tq * d * 4, 7: BHk * d * 4, 8: BH * Tq * nk_pad * 4}
+    spans = []
+    for which, size in sizes.items():
+        off = lib.sage_workspace_offset_gqa(B, H, Hk, nq, nk, d, which)
+        assert off >= 256 and off % 1024 == 0
+        spans.append((off, off + size))
+    spans.sort()
+    for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+        assert a1 <= b0
+    assert spans[-1][1] <= total
+    # the multi-head entry points are the H_kv = H case
+    assert lib.sage_workspace_bytes_gqa(B, H, H, nq, nk, d) == lib.sage_workspace_bytes(B, H, nq, nk, d)
+
+
+def test_gqa_head_counts_validated(lib):
+    assert lib.sage_workspace_bytes_gqa(1, 6, 4, 128, 128, 64) == 0    # 4 does not divide 6
+    assert lib.sage_workspace_bytes_gqa(1, 6, 0, 128, 128, 64) == 0
+    assert lib.sage_workspace_bytes_gqa(1, 2, 4, 128, 128, 64) == 0    # more key/value heads than query heads
+    assert lib.sage_workspace_bytes_gqa(1, 6, 3, 128, 128, 64) > 0
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.sage_attn_fwd_gqa(fake, fake, fake, fake, 1, 0, 1, 6, 4, 128, 128, 64, 0, 0.0, None, fake, 1 << 30,
+                                 None) == 1
+
+
 def test_workspace_bytes_rejects_bad_sizes(lib):
     assert lib.sage_workspace_bytes(1, 1, 128, 128, 96) == 0      # d must be 64 or 128
     assert lib.sage_workspace_bytes(-1, 1, 128, 128, 64) == 0

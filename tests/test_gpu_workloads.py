@@ -40,35 +40,36 @@ def _full_precision_rows(qh, kh, vh, rows, causal):
     return (p @ vh) / p.sum(1, keepdims=True)
 
 
-@pytest.mark.parametrize("name", ["image_dit", "llm_prefill", "video_dit"])
+@pytest.mark.parametrize("name", ["image_dit", "llm_prefill", "video_dit", "llm_prefill_gqa"])
 def test_full_size_workload_sampled(name):
     w = wl.WORKLOADS[name]
     q, k, v = wl.generate(w)
     dev = torch.device("cuda", 0)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     mode = sage.QuantMode.make()
-    ws = sage.make_workspace(w.B, w.H, w.N_q, w.N_kv, w.d, device=dev)
+    ws = sage.make_workspace(w.B, w.H, w.N_q, w.N_kv, w.d, device=dev, H_kv=w.Hk)
     sage.quant_qk(qd, kd, mode=mode, workspace=ws)
     sage.quant_v(vd, n_q=w.N_q, mode=mode, workspace=ws)
     o = sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode)
     assert sage.get_device_status(ws) == (0, 0)
     tq = -(-w.N_q // 128)
     heads = [(0, 0), (w.B - 1, w.H - 1)]
+    group = w.H // w.Hk
     blocks = sorted({0, tq // 2, tq - 1})
     views = {n: ws.view(n) for n in ("q8", "k8", "vt8", "dq", "dk", "dv", "qbar", "kbar")}
     for b, h in heads:
-        bh = b * w.H + h
-        qh, kh, vh = to_np64(q[b, h]), to_np64(k[b, h]), to_np64(v[b, h])
+        bh, bk = b * w.H + h, b * w.Hk + h // group   # query head, its key/value head
+        qh, kh, vh = to_np64(q[b, h]), to_np64(k[b, h // group]), to_np64(v[b, h // group])
         pre = oracle.prepass_head(qh, kh, vh)
         # the pre-pass of the sampled head, bit-exact
         assert np.array_equal(views["qbar"][bh].cpu().numpy(), pre["qbar"])
-        assert np.array_equal(views["kbar"][bh].cpu().numpy(), pre["kbar"])
+        assert np.array_equal(views["kbar"][bk].cpu().numpy(), pre["kbar"])
         assert np.array_equal(views["dq"][bh].cpu().numpy(), pre["dq_row"])
-        assert np.array_equal(views["dk"][bh].cpu().numpy(), pre["dk_key"][::16])
-        assert np.array_equal(views["dv"][bh].cpu().numpy(), pre["dv"])
+        assert np.array_equal(views["dk"][bk].cpu().numpy(), pre["dk_key"][::16])
+        assert np.array_equal(views["dv"][bk].cpu().numpy(), pre["dv"])
         assert np.array_equal(views["q8"][bh].cpu().numpy(), pre["q_code"])
-        assert np.array_equal(views["k8"][bh].cpu().numpy(), pre["k_code"])
-        assert np.array_equal(natural_key_order(views["vt8"][bh].cpu().numpy())[:, :w.N_kv].T, pre["v_code"])
+        assert np.array_equal(views["k8"][bk].cpu().numpy(), pre["k_code"])
+        assert np.array_equal(natural_key_order(views["vt8"][bk].cpu().numpy())[:, :w.N_kv].T, pre["v_code"])
         # attention rows of the sampled Q blocks over the full KV range
         oo = oracle.attn_head(pre, causal=w.causal, qblocks=blocks)
         rows = rows_of_blocks(w.N_q, blocks)

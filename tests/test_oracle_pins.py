@@ -375,3 +375,54 @@ def test_empty_and_degenerate_heads():
     o = oracle.attn_head(pre)
     vdeq = (pre["v_hat"] * pre["dv"]).mean(0)
     assert np.max(np.abs(o - vdeq[None, :])) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Grouped-query attention (H_kv key/value heads shared by H query heads)
+# ---------------------------------------------------------------------------
+def _gqa_inputs(B, H, H_kv, nq, nk, d, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, H, nq, d, generator=g).to(torch.bfloat16).double()
+    k = (torch.randn(B, H_kv, nk, d, generator=g) + 3 * torch.randn(B, H_kv, 1, d, generator=g)).to(torch.bfloat16)
+    v = torch.randn(B, H_kv, nk, d, generator=g).to(torch.bfloat16)
+    return q, k.double(), v.double()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_unquantized_equals_torch_sdpa_enable_gqa(causal):
+    """With the quantizers off, the oracle's grouped-query forward is torch's own
+    grouped-query attention (scaled_dot_product_attention with enable_gqa), whose
+    head grouping is the library's definition."""
+    B, H, H_kv, nq, nk, d = 2, 6, 2, 150, 150, 64
+    q, k, v = _gqa_inputs(B, H, H_kv, nq, nk, d, seed=5)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=causal, enable_gqa=True).numpy()
+    o = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), causal=causal, quant=(0, 0, 0))
+    assert np.max(np.abs(o - ref)) < 1e-12
+    r = oracle.reference_attention(q.numpy(), k.numpy(), v.numpy(), causal=causal)
+    assert np.max(np.abs(r - ref)) < 1e-12
+
+
+def test_gqa_equals_multi_head_on_repeated_kv_heads():
+    """The quantized grouped-query forward equals the multi-head forward on K and V
+    whose heads are repeated group-size times (torch.repeat_interleave), bit for bit:
+    smoothing and delta_V depend on the key/value head alone."""
+    B, H, H_kv, nq, nk, d = 1, 4, 2, 200, 260, 64
+    q, k, v = _gqa_inputs(B, H, H_kv, nq, nk, d, seed=9)
+    o = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), causal=True)
+    rep = H // H_kv
+    o_mha = oracle.sage_attention(q.numpy(), k.repeat_interleave(rep, dim=1).numpy(),
+                                  v.repeat_interleave(rep, dim=1).numpy(), causal=True)
+    assert np.array_equal(o, o_mha)
+    # tiling the heads instead (head h -> h % H_kv) is a different, wrong grouping
+    o_tile = oracle.sage_attention(q.numpy(), k.repeat(1, rep, 1, 1).numpy(), v.repeat(1, rep, 1, 1).numpy(),
+                                   causal=True)
+    assert not np.array_equal(o[0, 1], o_tile[0, 1])
+
+
+def test_gqa_bad_head_counts_rejected():
+    q = np.zeros((1, 3, 4, 64))
+    k = np.zeros((1, 2, 4, 64))
+    with pytest.raises(ValueError):
+        oracle.sage_attention(q, k, k)
+    with pytest.raises(ValueError):
+        oracle.reference_attention(q, k, k)
