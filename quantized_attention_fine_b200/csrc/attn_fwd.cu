@@ -46,6 +46,9 @@ constexpr int kWarpK = 16, kWarpMma = 17, kWarpV = 18;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;
 constexpr uint64_t kDrainNs = 50ull * 1000ull * 1000ull;
+// K codes + V^T codes of the heads whose CTAs run together stay within this many
+// bytes, a part of the 126 MB L2 (the rest holds the streaming Q codes, dS and O).
+constexpr size_t kKvL2Budget = 48ull << 20;
 // Register split (setmaxnreg): 640 threads launch with 96 registers each; the
 // producer warpgroup gives back to 32 so the four softmax warpgroups can hold 112:
 // 128 * 32 + 512 * 112 = 640 * 96.
@@ -418,10 +421,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         *reinterpret_cast<AttnSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // Work item: a pair of Q tiles of one head; longest pairs first when causal.
+    // Work item: a pair of Q tiles of one head.  The CTAs are ordered in blocks of
+    // p.head_block heads and, within a block, pair-major (the pairs of rank 0 of every
+    // head first; longest pairs first when causal): the CTAs in flight read the K and
+    // V^T tiles of a block's heads, which stay in L2, and the long causal pairs of a
+    // block start early.  The last block may hold fewer heads.
     const int n_pairs = (p.Tq + 1) / 2;
-    const int pair_idx = blockIdx.x / p.BH;
-    const int bh = blockIdx.x % p.BH;
+    const int blk = blockIdx.x / (n_pairs * p.head_block);
+    const int r = blockIdx.x - blk * (n_pairs * p.head_block);
+    const int nb = min(p.head_block, p.BH - blk * p.head_block);
+    const int pair_idx = r / nb;
+    const int bh = blk * p.head_block + r % nb;
     const int u = p.causal ? (n_pairs - 1 - pair_idx) : pair_idx;
     const int tA = 2 * u, tB = 2 * u + 1;
     const int b = bh / p.H, h = bh % p.H;
@@ -601,7 +611,15 @@ static cudaError_t launch_attention_d(const CUtensorMap &tq, const CUtensorMap &
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((p.Tq + 1) / 2) * (unsigned)p.BH;
-    attn_fwd_kernel<D><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, p);
+    // Heads per block of the CTA order: as many key/value heads as fit kKvL2Budget
+    // bytes of K codes + V^T codes, times the query heads that share each.
+    AttnParams pp = p;
+    const size_t kv_head_bytes = 2ull * (size_t)p.nk_pad * D;
+    const size_t kv_heads = kv_head_bytes ? kKvL2Budget / kv_head_bytes : 0;
+    const size_t hb = (kv_heads < 1 ? 1 : kv_heads) * (size_t)p.group;
+    pp.head_block = (int)(hb < (size_t)p.BH ? hb : (size_t)p.BH);
+    if (pp.head_block < 1) pp.head_block = 1;
+    attn_fwd_kernel<D><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, pp);
     return cudaGetLastError();
 }
 

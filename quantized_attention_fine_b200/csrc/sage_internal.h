@@ -95,6 +95,7 @@ struct AttnParams {
     int H, n_q, n_kv, Tq, Tk, nq_pad, nk_pad, BH;
     int group;          // query heads per key/value head (H / H_kv)
     int H_kv;
+    int head_block;     // query heads per block of the CTA order (set by launch_attention)
     int causal;
     int use_ds;         // 0: Q smoothing off, dS not read
     int out_bf16;
