@@ -177,6 +177,7 @@ def prepass_head(q, k, v, *, g_q=32, g_k=16, smooth_q=True, smooth_k=True,
     r["v_hat"] = r["v_hat"][:nk]
     r["cfg"] = dict(n_q=nq, n_kv=nk, d=d, g_q=g_q, g_k=g_k, smooth_q=smooth_q, smooth_k=smooth_k,
                     quant=tuple(quant), p_range=p_range, v_range=v_range)
+    r["q"] = q
     return r
 
 
@@ -212,6 +213,30 @@ def attn_head(pre, *, causal=False, sm_scale=None, qblocks=None, return_stats=Fa
     if return_stats:
         return o, rl, rm
     return o
+
+
+def lse_head(pre, *, causal=False, sm_scale=None, qblocks=None):
+    """Log-sum-exp (natural log) of each row's attention logits, as the method computes
+    them, referred back to the unsmoothed logits sm_scale * q_i . k_j.
+
+    The method's logits are x_ij = sm_scale * S_ij with S = dQ dK S_int + qbar_t . K_s
+    (steps of ``attn_head``).  K smoothing shifts every logit of row i by the same
+    -sm_scale * q_i . kbar (q . K_s = q . K - q . kbar), which softmax ignores but the
+    log-sum-exp does not; it is added back here so that the value approximates
+    log sum_j exp(sm_scale q_i . k_j), the quantity that merges partial results over
+    key ranges.  lse_i = m_i + log(l_i) + sm_scale q_i . kbar, with m, l the running max
+    and sum of the online softmax; -inf for a row that sees no key.  Rows of Q blocks not
+    in ``qblocks`` are -inf."""
+    c = pre["cfg"]
+    d = c["d"]
+    if sm_scale is None or sm_scale <= 0:
+        sm_scale = 1.0 / np.sqrt(d)
+    _, rl, rm = attn_head(pre, causal=causal, sm_scale=sm_scale, qblocks=qblocks, return_stats=True)
+    shift = sm_scale * (pre["q"] @ pre["kbar"].astype(np.float64))
+    out = np.full(rl.shape, -np.inf)
+    ok = rl > 0
+    out[ok] = rm[ok] + np.log(rl[ok]) + shift[ok]
+    return out
 
 
 def _group(H: int, H_kv: int) -> int:

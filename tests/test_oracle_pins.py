@@ -426,3 +426,56 @@ def test_gqa_bad_head_counts_rejected():
         oracle.sage_attention(q, k, k)
     with pytest.raises(ValueError):
         oracle.reference_attention(q, k, k)
+
+
+# ---------------------------------------------------------------------------
+# Log-sum-exp of the rows
+# ---------------------------------------------------------------------------
+def _torch_lse(q, k, causal, scale):
+    x = torch.from_numpy(q @ k.T) * scale
+    if causal:
+        nq, nk = q.shape[0], k.shape[0]
+        vis = torch.arange(nk)[None, :] <= torch.arange(nq)[:, None] + (nk - nq)
+        x = torch.where(vis, x, torch.tensor(-float("inf"), dtype=x.dtype))
+    return torch.logsumexp(x, dim=1).numpy()
+
+
+@pytest.mark.parametrize("smooth_q,smooth_k", [(True, True), (False, True), (True, False), (False, False)])
+@pytest.mark.parametrize("causal,nq,nk", [(False, 200, 333), (True, 333, 200), (True, 256, 256)])
+def test_lse_unquantized_equals_torch_logsumexp(smooth_q, smooth_k, causal, nq, nk):
+    """With the quantizers off the method's row log-sum-exp, referred back to the
+    unsmoothed logits, is torch.logsumexp of sm_scale * q . k (the K bias of these
+    inputs shifts the smoothed logits by several units, so a missing correction fails)."""
+    q, k, v = _rand_head(nq, nk, 64, seed=nq + nk, kbias=3.0, qbias=1.0)
+    pre = oracle.prepass_head(q, k, v, quant=(0, 0, 0), smooth_q=smooth_q, smooth_k=smooth_k)
+    lse = oracle.lse_head(pre, causal=causal)
+    ref = _torch_lse(q, k, causal, 1 / 8)
+    fin = np.isfinite(ref)
+    assert np.array_equal(fin, np.isfinite(lse))
+    assert np.max(np.abs(lse[fin] - ref[fin])) < 1e-11
+    if causal and nq > nk:
+        assert np.all(lse[:nq - nk] == -np.inf)
+
+
+@pytest.mark.parametrize("gran", ["per_block", "per_threadgroup"])
+def test_lse_quantized_within_logit_error_bound(gran):
+    """Log-sum-exp is 1-Lipschitz in the largest logit change, and the row sum uses the
+    unquantized P~, so each row's LSE lies within sm_scale times its largest INT8 score
+    error bound, sum_c (dQ/2 |K_s| + dK/2 |Q_s| + dQ dK/4), of the exact value."""
+    nq, nk, d = 300, 400, 128
+    q, k, v = _rand_head(nq, nk, d, seed=77, kbias=3.0)
+    g_q, g_k = oracle.GRANULARITY[gran]
+    pre = oracle.prepass_head(q, k, v, g_q=g_q, g_k=g_k)
+    lse = oracle.lse_head(pre, causal=True)
+    scale = 1 / math.sqrt(d)
+    ref = _torch_lse(q, k, True, scale)
+    qs = q - np.repeat(pre["qbar"].astype(np.float64), 128, axis=0)[:nq]
+    ks = pre["k_s"]
+    dq = pre["dq_row"][:nq].astype(np.float64)[:, None]
+    dk = pre["dk_key"][:nk].astype(np.float64)[None, :]
+    bound = (dq / 2) * np.abs(ks).sum(1)[None, :] + (dk / 2) * np.abs(qs).sum(1)[:, None] + d * dq * dk / 4
+    vis = np.arange(nk)[None, :] <= np.arange(nq)[:, None] + (nk - nq)
+    row_bound = scale * np.where(vis, bound, 0.0).max(1)
+    err = np.abs(lse - ref)
+    assert np.all(err <= row_bound + 1e-9)
+    assert err.max() > 0   # the quantizers did act
