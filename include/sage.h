@@ -194,6 +194,17 @@ SAGE_API sage_status_t sage_get_device_status(void *workspace, void *stream, int
  *   SAGE_WS_KBAR  fp32  [BHk][d]                 K token mean
  *   SAGE_WS_DS    fp32  [BH][Tq][nk_pad]         dS = qbar_t . K[j] (causally
  *                                                invisible entries left unwritten)
+ *   SAGE_WS_QS_KBAR fp32 [BH][nq_pad]            (q_i - qbar_t) . kbar per row: the
+ *                                                shift K smoothing gives the row's logits
+ *   SAGE_WS_LSE   fp32  [BH][nq_pad]             per row, written by the attention
+ *                                                step: log-sum-exp (natural log) of the
+ *                                                row's logits sm_scale q_i . k_j over its
+ *                                                visible keys, as the method computes
+ *                                                them (quantized scores, dS), with the K
+ *                                                smoothing shift added back; -inf for a
+ *                                                row that sees no key; rows >= n_q are
+ *                                                not written.  It merges partial outputs
+ *                                                over key ranges.
  * Along the key axis of VT8 and DS, each 128-key tile is stored in the order
  * (even keys, odd keys): key j of the tile starting at j0 is at position
  * j0 + (j & 1) * 64 + (j >> 1).  The attention kernel's threads hold the even and
@@ -201,7 +212,8 @@ SAGE_API sage_status_t sage_get_device_status(void *workspace, void *stream, int
  */
 enum {
     SAGE_WS_Q8 = 0, SAGE_WS_K8 = 1, SAGE_WS_VT8 = 2, SAGE_WS_DQ = 3, SAGE_WS_DK = 4,
-    SAGE_WS_DV = 5, SAGE_WS_QBAR = 6, SAGE_WS_KBAR = 7, SAGE_WS_DS = 8, SAGE_WS_NUM_VIEWS = 9
+    SAGE_WS_DV = 5, SAGE_WS_QBAR = 6, SAGE_WS_KBAR = 7, SAGE_WS_DS = 8, SAGE_WS_QS_KBAR = 9,
+    SAGE_WS_LSE = 10, SAGE_WS_NUM_VIEWS = 11
 };
 /* Byte offset of view `which` inside the workspace, or -1 for bad arguments. */
 SAGE_API int64_t sage_workspace_offset(int B, int H, int n_q, int n_kv, int d, int which);

@@ -35,7 +35,8 @@ _ERR_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED"
               4: "SAGE_ERR_CUDA", 5: "SAGE_ERR_TIMEOUT"}
 GRANULARITIES = {"per_block": 0, "per_warp": 1, "per_threadgroup": 2}
 _LAYOUTS = {"HND": 0, "NHD": 1}
-WS_VIEWS = {"q8": 0, "k8": 1, "vt8": 2, "dq": 3, "dk": 4, "dv": 5, "qbar": 6, "kbar": 7, "ds": 8}
+WS_VIEWS = {"q8": 0, "k8": 1, "vt8": 2, "dq": 3, "dk": 4, "dv": 5, "qbar": 6, "kbar": 7, "ds": 8, "qs_kbar": 9,
+            "lse": 10}
 WS_ALIGN = 1024
 
 
@@ -181,6 +182,12 @@ class Workspace:
         H_kv = H if H_kv is None else H_kv
         return self.dims == (int(B), int(H), int(n_q), int(n_kv), int(d)) and self.H_kv == int(H_kv)
 
+    def lse(self):
+        """Row log-sum-exp [B, H, n_q] (fp32, natural log) of the last attention call on
+        this workspace; a view into the workspace, overwritten by the next call."""
+        B, H, n_q, _, _ = self.dims
+        return self.view("lse").view(B, H, -1)[:, :, :n_q]
+
     def view(self, which: str):
         """Typed view of a workspace region (see include/sage.h, SAGE_WS_*): per query
         head for q8, dq, qbar, ds; per key/value head for k8, vt8, dk, dv, kbar."""
@@ -193,7 +200,8 @@ class Workspace:
                   "vt8": ((BHk, d, nk_pad), torch.uint8), "dq": ((BH, nq_pad), torch.float32),
                   "dk": ((BHk, nk_pad // 16), torch.float32), "dv": ((BHk, d), torch.float32),
                   "qbar": ((BH, Tq, d), torch.float32), "kbar": ((BHk, d), torch.float32),
-                  "ds": ((BH, Tq, nk_pad), torch.float32)}
+                  "ds": ((BH, Tq, nk_pad), torch.float32), "qs_kbar": ((BH, nq_pad), torch.float32),
+                  "lse": ((BH, nq_pad), torch.float32)}
         shp, dt = shapes[which]
         n = math.prod(shp) * torch.tensor([], dtype=dt).element_size()
         start = self.offset + off
@@ -242,7 +250,9 @@ def quant_v(v, *, n_q, H=None, layout="HND", mode=None, workspace=None, stream=N
 
 
 def attn_fwd_prequant(workspace: Workspace, *, dtype, layout="HND", causal=False, sm_scale=None, mode=None,
-                      out=None, stream=None):
+                      out=None, stream=None, return_lse=False):
+    """Attention from a workspace filled by quant_qk and quant_v.  With return_lse, also
+    the rows' log-sum-exp [B, H, n_q] (a view into the workspace, see Workspace.lse)."""
     torch = _torch()
     B, H, n_q, n_kv, d = workspace.dims
     if out is None:
@@ -254,15 +264,17 @@ def attn_fwd_prequant(workspace: Workspace, *, dtype, layout="HND", causal=False
                                                      float(sm_scale or 0.0), ctypes.byref(mode),
                                                      ctypes.c_void_p(workspace.ptr), workspace.nbytes,
                                                      _stream_handle(stream)), "sage_attn_fwd_prequant_gqa")
-    return out
+    return (out, workspace.lse()) if return_lse else out
 
 
 def attn_fwd(q, k, v, *, causal=False, sm_scale=None, layout="HND", granularity="per_threadgroup",
-             smooth_q=True, smooth_k=True, p_range=448.0, v_range=448.0, out=None, workspace=None, stream=None):
+             smooth_q=True, smooth_k=True, p_range=448.0, v_range=448.0, out=None, workspace=None, stream=None,
+             return_lse=False):
     """O = quantized attention of q, k, v (pre-pass + fused kernel, enqueued on the current stream).
 
     k and v may have fewer heads than q (grouped-query attention): query head h
-    reads key/value head h // (H // H_kv)."""
+    reads key/value head h // (H // H_kv).  With return_lse, returns (O, LSE), LSE the
+    rows' log-sum-exp [B, H, n_q] fp32 (a view into the workspace)."""
     torch = _torch()
     B, H, H_kv, n_q, n_kv, d = _shape(q, k, layout)
     if v.shape != k.shape:
@@ -277,7 +289,7 @@ def attn_fwd(q, k, v, *, causal=False, sm_scale=None, layout="HND", granularity=
                                             _LAYOUTS[layout], B, H, H_kv, n_q, n_kv, d, int(bool(causal)),
                                             float(sm_scale or 0.0), ctypes.byref(mode), ctypes.c_void_p(ws.ptr),
                                             ws.nbytes, _stream_handle(stream)), "sage_attn_fwd_gqa")
-    return out
+    return (out, ws.lse()) if return_lse else out
 
 
 def get_device_status(workspace: Workspace, stream=None):

@@ -266,11 +266,12 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
     // this thread writes output columns [par * D / 2, par * D / 2 + D / 2) of its row
     uint16_t *orow = static_cast<uint16_t *>(p.o) + o_base + (int64_t)row * p.so_n + par * (D / 2);
 
-    if (n_tiles == 0) {  // this tile's rows see no key: O = 0
+    if (n_tiles == 0) {  // this tile's rows see no key: O = 0, LSE = -inf
         if (row < p.n_q) {
             uint4 *dst = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
             for (int i = 0; i < D / 16; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+            if (par == 0) p.lse[(size_t)bh * p.nq_pad + row] = -INFINITY;
         }
         return;
     }
@@ -382,6 +383,14 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
         tc_fence_after();
         const float l_row = l + __shfl_xor_sync(0xFFFFFFFFu, l, 2);
         const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
+        if (par == 0 && row < p.n_q) {
+            // l carries the factor Pr and m is in score units: the logits' log-sum-exp is
+            // ln 2 (c (m + Q_s . kbar) + log2(l / Pr)), the Q_s . kbar term undoing the
+            // shift that K smoothing applied to the whole row
+            const size_t ri = (size_t)bh * p.nq_pad + row;
+            p.lse[ri] = (l_row > 0.f) ? 0.6931471805599453f * (c * (m + p.qs_kbar[ri]) + log2f(l_row) - p.log2_pr)
+                                      : -INFINITY;
+        }
         const float *dv = p.dv + (size_t)sm.bh_kv * D;
         // The thread holds O columns 2v + par (v < D / 2).  Output word i of the even
         // thread is columns (2i, 2i + 1), i < D / 4; of the odd thread, columns

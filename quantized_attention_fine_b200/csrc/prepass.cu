@@ -9,7 +9,8 @@
 //                channel and per-channel max |V|.
 //   kv_finalize  per key/value head: kbar = fp32(sum / n_kv); delta_V = max|V| / Vr.
 //   quant_q      per (head, 128-row block): qbar (fp64 mean of the valid rows,
-//                rounded to fp32), Q_s = Q - qbar in fp32, group amax, INT8 codes.
+//                rounded to fp32), Q_s = Q - qbar in fp32, group amax, INT8 codes, and
+//                per row Q_s . kbar (the logit shift of K smoothing, for the row LSE).
 //   quant_k      per (head, 128-key tile): K_s = K - kbar, INT8 codes per group,
 //                delta_K per 16-key run.
 //   quant_v      per (head, 128-key tile): V / delta_V -> E4M3, written transposed
@@ -51,6 +52,24 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
     return v;
+}
+
+// Sums each of 16 per-lane values over the warp's 32 lanes (a reduce-scatter: every
+// exchange halves the values a lane still holds, 16 shuffles in all).  Returns, in
+// lane l, the total of value l >> 1.
+__device__ __forceinline__ float warp_sum16_scatter(float (&v)[16]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1) {  // exchange with the lane 2 w away: keep half
+        const bool up = (lane & (2 * w)) != 0;
+#pragma unroll
+        for (int k = 0; k < w; ++k) {
+            const float send = up ? v[k] : v[k + w];
+            const float keep = up ? v[k + w] : v[k];
+            v[k] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 2 * w);
+        }
+    }
+    return v[0] + __shfl_xor_sync(0xFFFFFFFFu, v[0], 1);
 }
 
 // INT8 codes of VEC values, round-half-even of the IEEE fp32 quotient xs / delta,
@@ -305,20 +324,33 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
             reinterpret_cast<float *>(a.ws + a.L.qbar)[((size_t)bh * S.Tq + t) * D + c] = qb;
         }
         __syncthreads();
-        float qb[VEC];
+        float qb[VEC], kb[VEC];
+        // kbar of this query head's key/value head (0 without K, i.e. no keys)
+        const int bh_kv = (bh / S.H) * S.H_kv + (bh % S.H) / (S.H / S.H_kv);
+        const float *kbar = reinterpret_cast<const float *>(a.ws + a.L.kbar) + (size_t)bh_kv * D + lane * VEC;
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) qb[v] = s_qbar[lane * VEC + v];
+        for (int v = 0; v < VEC; ++v) {
+            qb[v] = s_qbar[lane * VEC + v];
+            kb[v] = a.k ? kbar[v] : 0.f;
+        }
         float am = 0.f;
+        float shift[RPW];  // this lane's part of Q_s . kbar for each of the warp's rows
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
             const int r = warp * RPW + i;
+            shift[i] = 0.f;
 #pragma unroll
             for (int v = 0; v < VEC; ++v) {
                 const float xs = (r < nvalid) ? __fsub_rn(x[i][v], qb[v]) : 0.f;
                 x[i][v] = xs;
                 am = fmaxf(am, fabsf(xs));
+                shift[i] = fmaf(xs, kb[v], shift[i]);
             }
         }
+        static_assert(RPW == 16, "one shift value per row of the warp's 16");
+        const float row_shift = warp_sum16_scatter(shift);  // row warp * RPW + (lane >> 1)
+        if ((lane & 1) == 0)
+            reinterpret_cast<float *>(a.ws + a.L.qs_kbar)[(size_t)bh * S.nq_pad + r0 + warp * RPW + (lane >> 1)] = row_shift;
         am = warp_max(am);
         if (lane == 0) s_wmax[warp] = am;
         __syncthreads();

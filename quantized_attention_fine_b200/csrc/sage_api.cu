@@ -218,6 +218,8 @@ sage_status_t run_attention(void *o, int dtype, int layout, const Shape &s, int 
     p.dk = reinterpret_cast<const float *>(ws + L.dk);
     p.dv = reinterpret_cast<const float *>(ws + L.dv);
     p.ds = reinterpret_cast<const float *>(ws + L.ds);
+    p.qs_kbar = reinterpret_cast<const float *>(ws + L.qs_kbar);
+    p.lse = reinterpret_cast<float *>(const_cast<uint8_t *>(ws) + L.lse);
     p.o = o;
     p.so_b = so.b;
     p.so_h = so.h;
@@ -283,6 +285,8 @@ int64_t sage_workspace_offset_gqa(int B, int H, int H_kv, int n_q, int n_kv, int
         case SAGE_WS_QBAR: return (int64_t)L.qbar;
         case SAGE_WS_KBAR: return (int64_t)L.kbar;
         case SAGE_WS_DS: return (int64_t)L.ds;
+        case SAGE_WS_QS_KBAR: return (int64_t)L.qs_kbar;
+        case SAGE_WS_LSE: return (int64_t)L.lse;
         default: return -1;
     }
 }

@@ -37,7 +37,7 @@ inline Shape make_shape(int B, int H, int H_kv, int n_q, int n_kv, int d) {
 
 // Byte offsets of every workspace region.
 struct WsLayout {
-    size_t status, q8, k8, vt8, dq, dk, dv, qbar, kbar, ds, ksum_part, vmax_part, total;
+    size_t status, q8, k8, vt8, dq, dk, dv, qbar, kbar, ds, qs_kbar, lse, ksum_part, vmax_part, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -57,6 +57,8 @@ inline WsLayout ws_layout(const Shape &s) {
     w.qbar = take(BH * s.Tq * d * 4);
     w.kbar = take(BHk * d * 4);
     w.ds = take(BH * s.Tq * (size_t)s.nk_pad * 4);
+    w.qs_kbar = take(BH * s.nq_pad * 4);
+    w.lse = take(BH * s.nq_pad * 4);
     w.ksum_part = take(BHk * s.n_chunks * d * 8);
     w.vmax_part = take(BHk * s.n_chunks * d * 4);
     w.total = off;
@@ -90,6 +92,8 @@ struct PrepassArgs {
 
 struct AttnParams {
     const float *dq, *dk, *dv, *ds;
+    const float *qs_kbar;   // per row: (q_i - qbar_t) . kbar, the logit shift of K smoothing
+    float *lse;             // per row: log-sum-exp of the logits (natural log)
     void *o;
     int64_t so_b, so_h, so_n;
     int H, n_q, n_kv, Tq, Tk, nq_pad, nk_pad, BH;

@@ -56,7 +56,8 @@ def test_workspace_layout_regions_are_aligned_and_disjoint(lib, dims):
     BH, Tq = B * H, -(-nq // 128)
     nq_pad, nk_pad = Tq * 128, -(-nk // 128) * 128
     sizes = {0: BH * nq_pad * d, 1: BH * nk_pad * d, 2: BH * d * nk_pad, 3: BH * nq_pad * 4,
-             4: BH * nk_pad // 16 * 4, 5: BH * d * 4, 6: BH * Tq * d * 4, 7: BH * d * 4, 8: BH * Tq * nk_pad * 4}
+             4: BH * nk_pad // 16 * 4, 5: BH * d * 4, 6: BH * Tq * d * 4, 7: BH * d * 4, 8: BH * Tq * nk_pad * 4,
+             9: BH * nq_pad * 4, 10: BH * nq_pad * 4}
     spans = []
     for which, size in sizes.items():
         off = lib.sage_workspace_offset(B, H, nq, nk, d, which)
@@ -77,7 +78,8 @@ def test_gqa_workspace_regions_sized_per_kv_head(lib, dims):
     BH, BHk, Tq = B * H, B * Hk, -(-nq // 128)
     nq_pad, nk_pad = Tq * 128, -(-nk // 128) * 128
     sizes = {0: BH * nq_pad * d, 1: BHk * nk_pad * d, 2: BHk * d * nk_pad, 3: BH * nq_pad * 4,
-             4: BHk * nk_pad // 16 * 4, 5: BHk * d * 4, 6: BH * Tq * d * 4, 7: BHk * d * 4, 8: BH * Tq * nk_pad * 4}
+             4: BHk * nk_pad // 16 * 4, 5: BHk * d * 4, 6: BH * Tq * d * 4, 7: BHk * d * 4, 8: BH * Tq * nk_pad * 4,
+             9: BH * nq_pad * 4, 10: BH * nq_pad * 4}
     spans = []
     for which, size in sizes.items():
         off = lib.sage_workspace_offset_gqa(B, H, Hk, nq, nk, d, which)
