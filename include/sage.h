@@ -153,6 +153,32 @@ SAGE_API sage_status_t sage_attn_fwd_gqa(const void *q, const void *k, const voi
                                          const sage_quant_mode_t *mode,
                                          void *workspace, size_t workspace_bytes, void *stream);
 
+/* ---- variable-length (packed) batches -------------------------------------------
+ * B sequences of different lengths packed token-major, as in the pages' varlen
+ * kernels (the deployment guide's "dynamic sequence length" tip: a per-block causal
+ * varlen attention):
+ *   q, o : [total_q,  H,    d], sequence b holding tokens [cu_seqlens_q[b], cu_seqlens_q[b+1])
+ *   k, v : [total_kv, H_kv, d], sequence b holding tokens [cu_seqlens_kv[b], cu_seqlens_kv[b+1])
+ * cu_seqlens_q / cu_seqlens_kv: DEVICE int32 arrays of B + 1 nondecreasing offsets
+ * starting at 0 and ending at most at total_q / total_kv.  Each sequence is attended on
+ * its own, with the method's steps per sequence and head (K mean, delta_V, Q blocks of
+ * 128 rows, causal bottom-right aligned per sequence: key j visible to query i iff
+ * j <= i + n_kv,b - n_q,b).  max_seqlen_q / max_seqlen_kv must be at least every
+ * sequence's length (longer sequences are cut to them); the workspace is sized by them
+ * (sage_workspace_bytes_varlen), its per-sequence arrays padded to these lengths and
+ * indexed as for a dense batch of B sequences (the SAGE_WS_* views below, with
+ * n_q = max_seqlen_q, n_kv = max_seqlen_kv).  Work scales with the actual lengths:
+ * tiles past a sequence's end are skipped.  Offsets outside [0, total] are clamped;
+ * tokens of o that no sequence covers are not written.  total_kv == 0 writes o = 0.
+ * Other arguments and errors as sage_attn_fwd_gqa. */
+SAGE_API size_t sage_workspace_bytes_varlen(int B, int H, int H_kv, int max_seqlen_q, int max_seqlen_kv, int d);
+SAGE_API sage_status_t sage_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, int dtype,
+                                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_kv,
+                                            int B, int H, int H_kv, int total_q, int total_kv,
+                                            int max_seqlen_q, int max_seqlen_kv, int d, int causal,
+                                            float sm_scale, const sage_quant_mode_t *mode,
+                                            void *workspace, size_t workspace_bytes, void *stream);
+
 /* The whole forward, exactly as sage_attn_fwd, for callers that must not allocate
  * device memory (for example a plugin whose host application owns every device
  * allocation, or a serving loop where a cudaMalloc, which can synchronize the

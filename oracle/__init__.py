@@ -271,6 +271,34 @@ def sage_attention(q, k, v, *, causal=False, sm_scale=None, granularity="per_thr
     return o
 
 
+def sage_attention_varlen(q, k, v, cu_q, cu_kv, *, causal=False, sm_scale=None, return_lse=False, **kw):
+    """Quantized attention of a packed batch: q [total_q, H, d], k, v [total_kv, H_kv, d]
+    (token-major), sequence b holding tokens [cu_q[b], cu_q[b+1]) of q and
+    [cu_kv[b], cu_kv[b+1]) of k and v.  Each sequence is attended on its own: the method
+    runs on (q, k, v) of that sequence as on a batch of one (``sage_attention``
+    arguments in ``kw``); causal is bottom-right aligned per sequence.  Returns O
+    [total_q, H, d] fp64 (tokens no sequence covers stay 0) and, with return_lse, the
+    rows' log-sum-exp [total_q, H] (``lse_head``)."""
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    total_q, H, d = q.shape
+    group = _group(H, k.shape[1])
+    g_q, g_k = GRANULARITY[kw.pop("granularity", "per_threadgroup")]
+    o = np.zeros((total_q, H, d), np.float64)
+    lse = np.full((total_q, H), -np.inf)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_kv[b]), int(cu_kv[b + 1])
+        if q1 <= q0:
+            continue
+        for h in range(H):
+            pre = prepass_head(q[q0:q1, h], k[k0:k1, h // group], v[k0:k1, h // group], g_q=g_q, g_k=g_k, **kw)
+            o[q0:q1, h] = attn_head(pre, causal=causal, sm_scale=sm_scale)
+            if return_lse:
+                lse[q0:q1, h] = lse_head(pre, causal=causal, sm_scale=sm_scale)
+    return (o, lse) if return_lse else o
+
+
 def reference_attention(q, k, v, *, causal=False, sm_scale=None, heads=None):
     """Textbook full-precision attention in fp64 (two-pass softmax), [B, H, N, d].
     k and v may hold fewer heads than q, as in sage_attention."""

@@ -21,7 +21,7 @@ import threading
 
 __all__ = [
     "QuantMode", "Workspace", "workspace_bytes", "make_workspace", "quant_qk", "quant_v", "attn_fwd_prequant",
-    "attn_fwd", "get_device_status", "workspace_view", "debug_qk_tile", "debug_pv_accumulate",
+    "attn_fwd", "attn_fwd_varlen", "get_device_status", "workspace_view", "debug_qk_tile", "debug_pv_accumulate",
     "debug_fault_inject", "library_path", "load_library", "SageError", "GRANULARITIES",
 ]
 
@@ -89,6 +89,9 @@ def load_library():
         lib.sage_quant_v_gqa.argtypes = [P, I, I, I, I, I, I, I, I, QM, P, S, P]
         lib.sage_attn_fwd_prequant_gqa.argtypes = [P, I, I, I, I, I, I, I, I, I, F, QM, P, S, P]
         lib.sage_attn_fwd_gqa.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, F, QM, P, S, P]
+        lib.sage_workspace_bytes_varlen.argtypes = [I] * 6
+        lib.sage_workspace_bytes_varlen.restype = S
+        lib.sage_attn_fwd_varlen.argtypes = [P, P, P, P, I, P, P] + [I] * 9 + [F, QM, P, S, P]
         lib.sage_get_device_status.argtypes = [P, P, ctypes.POINTER(I), ctypes.POINTER(I)]
         lib.sage_debug_qk_tile.argtypes = [P, I, I, I, I, I, I, I, I, P, P]
         lib.sage_debug_pv_accumulate.argtypes = [P, P, I, I, P, P]
@@ -96,6 +99,7 @@ def load_library():
         lib.sage_version.restype = ctypes.c_char_p
         for fn in ("sage_quant_qk", "sage_quant_v", "sage_attn_fwd_prequant", "sage_attn_fwd",
                    "sage_quant_qk_gqa", "sage_quant_v_gqa", "sage_attn_fwd_prequant_gqa", "sage_attn_fwd_gqa",
+                   "sage_attn_fwd_varlen",
                    "sage_get_device_status", "sage_debug_qk_tile", "sage_debug_pv_accumulate",
                    "sage_debug_attn_fault_inject"):
             getattr(lib, fn).restype = ctypes.c_int
@@ -290,6 +294,49 @@ def attn_fwd(q, k, v, *, causal=False, sm_scale=None, layout="HND", granularity=
                                             float(sm_scale or 0.0), ctypes.byref(mode), ctypes.c_void_p(ws.ptr),
                                             ws.nbytes, _stream_handle(stream)), "sage_attn_fwd_gqa")
     return (out, ws.lse()) if return_lse else out
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, max_seqlen_q=None, max_seqlen_kv=None, causal=False,
+                    sm_scale=None, granularity="per_threadgroup", smooth_q=True, smooth_k=True, p_range=448.0,
+                    v_range=448.0, out=None, workspace=None, stream=None, return_lse=False):
+    """Quantized attention of a packed batch of variable-length sequences.
+
+    q: [total_q, H, d]; k, v: [total_kv, H_kv, d] (H_kv divides H); cu_seqlens_q,
+    cu_seqlens_kv: int32 CUDA tensors of B + 1 offsets.  Sequence b is attended on its
+    own.  max_seqlen_*: the longest lengths (read from the offsets, which synchronizes,
+    when not given).  With return_lse, also the rows' log-sum-exp as a [B, H,
+    max_seqlen_q] view into the workspace (row i of sequence b at [b, h, i])."""
+    torch = _torch()
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
+        raise ValueError("q must be [total_q, H, d] and k, v [total_kv, H_kv, d]")
+    total_q, H, d = (int(x) for x in q.shape)
+    total_kv, H_kv = int(k.shape[0]), int(k.shape[1])
+    if int(k.shape[2]) != d or H_kv < 1 or H % H_kv != 0:
+        raise ValueError("k shape %s does not match q %s" % (tuple(k.shape), tuple(q.shape)))
+    for cu in (cu_seqlens_q, cu_seqlens_kv):
+        if cu.dtype != torch.int32 or cu.dim() != 1 or not cu.is_cuda:
+            raise ValueError("cu_seqlens must be 1-D int32 CUDA tensors")
+    B = int(cu_seqlens_q.numel()) - 1
+    if B < 0 or int(cu_seqlens_kv.numel()) != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_kv must both hold B + 1 offsets")
+    if max_seqlen_q is None:
+        max_seqlen_q = int((cu_seqlens_q[1:] - cu_seqlens_q[:-1]).max().item()) if B > 0 else 0
+    if max_seqlen_kv is None:
+        max_seqlen_kv = int((cu_seqlens_kv[1:] - cu_seqlens_kv[:-1]).max().item()) if B > 0 else 0
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share a dtype")
+    ws = _ws_for(workspace, B, H, H_kv, max_seqlen_q, max_seqlen_kv, d, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    mode = QuantMode.make(granularity, smooth_q, smooth_k, p_range, v_range)
+    _check(load_library().sage_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q),
+                                               _ptr(cu_seqlens_q), _ptr(cu_seqlens_kv), B, H, H_kv, total_q, total_kv,
+                                               int(max_seqlen_q), int(max_seqlen_kv), d, int(bool(causal)),
+                                               float(sm_scale or 0.0), ctypes.byref(mode), ctypes.c_void_p(ws.ptr),
+                                               ws.nbytes, _stream_handle(stream)), "sage_attn_fwd_varlen")
+    if return_lse:
+        return out, ws.view("lse").view(B, H, -1)[:, :, :max_seqlen_q]
+    return out
 
 
 def get_device_status(workspace: Workspace, stream=None):

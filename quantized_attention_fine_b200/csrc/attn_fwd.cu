@@ -250,7 +250,8 @@ __device__ __forceinline__ uint32_t pack16x2(float lo, float hi, int out_bf16) {
 
 template <int D>
 __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &p, uint32_t tmem, int X, int t,
-                                             int n_tiles, int bh, int64_t o_base, volatile int *abort_flag) {
+                                             int n_tiles, int bh, int64_t o_base, int n_q, int n_kv,
+                                             volatile int *abort_flag) {
     constexpr int KS = AttnCfg<D>::kKStages;
     const int w8 = (threadIdx.x >> 5) & 7;  // warp within the tile's eight
     const int quad = w8 & 3, half = w8 >> 2;
@@ -261,13 +262,13 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
     const uint32_t lane_base = (uint32_t)(32 * quad + 16 * half) << 16;
     const uint32_t s_tmem = tmem + lane_base + (uint32_t)X * 128u;
     const uint32_t o_tmem = tmem + lane_base + kTmemO + (uint32_t)X * D;
-    const int off = p.n_kv - p.n_q;
+    const int off = n_kv - n_q;
     const int pos0 = par * (kTile / 2);  // storage position of this thread's first key of a tile
     // this thread writes output columns [par * D / 2, par * D / 2 + D / 2) of its row
     uint16_t *orow = static_cast<uint16_t *>(p.o) + o_base + (int64_t)row * p.so_n + par * (D / 2);
 
     if (n_tiles == 0) {  // this tile's rows see no key: O = 0, LSE = -inf
-        if (row < p.n_q) {
+        if (row < n_q) {
             uint4 *dst = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
             for (int i = 0; i < D / 16; ++i) dst[i] = make_uint4(0, 0, 0, 0);
@@ -299,7 +300,7 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
         tc_fence_before();
         mbar_arrive(&sm.bar_sfree[X]);
         m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        if (tile_masked(0, t, p.n_kv, off, p.causal)) m = mask_tile(sv, 0, row, par, p.n_kv, off, p.causal);
+        if (tile_masked(0, t, n_kv, off, p.causal)) m = mask_tile(sv, 0, row, par, n_kv, off, p.causal);
         m = pair_max(m);
         bias = (m == -INFINITY) ? 0.f : p.log2_pr - m * c;
     }
@@ -365,8 +366,8 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
 
         if (has_next) {  // running maximum with tile it + 1
             float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            if (tile_masked(it + 1, t, p.n_kv, off, p.causal))
-                tmax = mask_tile(sv, it + 1, row, par, p.n_kv, off, p.causal);
+            if (tile_masked(it + 1, t, n_kv, off, p.causal))
+                tmax = mask_tile(sv, it + 1, row, par, n_kv, off, p.causal);
             const float m_new = fmaxf(m, pair_max(tmax));
             if (m_new == -INFINITY) {
                 alpha = 1.f;
@@ -383,7 +384,7 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
         tc_fence_after();
         const float l_row = l + __shfl_xor_sync(0xFFFFFFFFu, l, 2);
         const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
-        if (par == 0 && row < p.n_q) {
+        if (par == 0 && row < n_q) {
             // l carries the factor Pr and m is in score units: the logits' log-sum-exp is
             // ln 2 (c (m + Q_s . kbar) + log2(l / Pr)), the Q_s . kbar term undoing the
             // shift that K smoothing applied to the whole row
@@ -411,7 +412,7 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
                 const float got = __shfl_xor_sync(0xFFFFFFFFu, par ? y_lo : y_hi, 2);
                 out[k] = par ? pack16x2(got, y_hi, p.out_bf16) : pack16x2(y_lo, got, p.out_bf16);
             }
-            if (row < p.n_q) {
+            if (row < n_q) {
                 uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * cb);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) dst[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
@@ -420,7 +421,11 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
     }
 }
 
-template <int D>
+// RT: sequence lengths decided at run time (a packed batch when p.cu_q is set, else
+// the dense lengths); without RT the kernel serves dense batches only and reads the
+// lengths straight from the parameters.  The two compile to different register
+// allocations: d = 128 dense runs faster without RT, d = 64 dense with it (measured).
+template <int D, bool RT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
@@ -445,12 +450,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int tA = 2 * u, tB = 2 * u + 1;
     const int b = bh / p.H, h = bh % p.H;
     const int bh_kv = b * p.H_kv + h / p.group;  // key/value head of query head h
-    const int off = p.n_kv - p.n_q;
-    const int nA = kv_tiles_of(tA, p.Tq, p.Tk, p.n_q, off, p.causal);
-    const int nB = kv_tiles_of(tB, p.Tq, p.Tk, p.n_q, off, p.causal);
+    // Lengths of this head's sequence: a packed batch gives each sequence its own (the
+    // workspace rows stay padded to the longest, p.n_q / p.n_kv)
+    int n_q = p.n_q, n_kv = p.n_kv;
+    int64_t o_base = (int64_t)b * p.so_b + (int64_t)h * p.so_h;
+    if (RT && p.cu_q) {
+        const SeqRange sq = seq_range(p.cu_q, b, p.n_q, p.total_q), sk = seq_range(p.cu_kv, b, p.n_kv, p.total_kv);
+        n_q = sq.n;
+        n_kv = sk.n;
+        o_base = (int64_t)sq.off * p.so_n + (int64_t)h * p.so_h;
+    }
+    const int Tq = (n_q + kTile - 1) / kTile, Tk = (n_kv + kTile - 1) / kTile;
+    if (tA >= Tq) return;  // a pair past the end of a shorter packed sequence (the whole CTA)
+    const int off = n_kv - n_q;
+    const int nA = kv_tiles_of(tA, Tq, Tk, n_q, off, p.causal);
+    const int nB = kv_tiles_of(tB, Tq, Tk, n_q, off, p.causal);
     const int n_tiles = max(nA, nB);
-    const bool hasB = tB < p.Tq;
-    const int64_t o_base = (int64_t)b * p.so_b + (int64_t)h * p.so_h;
+    const bool hasB = tB < Tq;
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_q, 1);
@@ -608,16 +624,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     setmaxnreg_inc<kRegsSoftmax>();
     // one copy of the softmax code serves both tiles (instruction-cache footprint)
     const int X = warp >> 3;
-    if (X == 0 || hasB) softmax_role<D>(sm, p, tmem, X, X ? tB : tA, X ? nB : nA, bh, o_base, abort_flag);
+    if (X == 0 || hasB)
+        softmax_role<D>(sm, p, tmem, X, X ? tB : tA, X ? nB : nA, bh, o_base, n_q, n_kv, abort_flag);
     tc_fence_before();
     __syncthreads();
 }
 
-template <int D>
+template <int D, bool RT>
 static cudaError_t launch_attention_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                       const AttnParams &p, cudaStream_t stream) {
     const size_t smem = sizeof(AttnSmem<D>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(attn_fwd_kernel<D, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((p.Tq + 1) / 2) * (unsigned)p.BH;
     // Heads per block of the CTA order: as many key/value heads as fit kKvL2Budget
@@ -628,14 +646,17 @@ static cudaError_t launch_attention_d(const CUtensorMap &tq, const CUtensorMap &
     const size_t hb = (kv_heads < 1 ? 1 : kv_heads) * (size_t)p.group;
     pp.head_block = (int)(hb < (size_t)p.BH ? hb : (size_t)p.BH);
     if (pp.head_block < 1) pp.head_block = 1;
-    attn_fwd_kernel<D><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, pp);
+    attn_fwd_kernel<D, RT><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, pp);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                              const AttnParams &p, int d, cudaStream_t stream) {
-    if (d == 128) return launch_attention_d<128>(tq, tk, tv, p, stream);
-    return launch_attention_d<64>(tq, tk, tv, p, stream);
+    if (d == 128) {
+        if (p.cu_q) return launch_attention_d<128, true>(tq, tk, tv, p, stream);
+        return launch_attention_d<128, false>(tq, tk, tv, p, stream);
+    }
+    return launch_attention_d<64, true>(tq, tk, tv, p, stream);
 }
 
 // ---------------------------------------------------------------------------

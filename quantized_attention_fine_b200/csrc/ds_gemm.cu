@@ -63,14 +63,24 @@ template <int D>
 __global__ void __launch_bounds__(kDsThreads, 1)
     ds_gemm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ds,
                    const float *__restrict__ qbar, int H, int H_kv, int Tq, int Tk, int nhd, int bf16, int causal_skip,
-                   int causal_off, int *status) {
+                   int causal_off, const int *__restrict__ cu_q, const int *__restrict__ cu_kv, int n_q_max,
+                   int n_kv_max, int total_q, int total_kv, int *status) {
     constexpr int KA = D / 64;
     extern __shared__ uint8_t smem_raw[];
     DsSmem<D> &sm = *reinterpret_cast<DsSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y;  // query head
+    // key/value head read by query head bh: h_kv = h / (H / H_kv)
+    const int b = bh / H, h_kv = (bh % H) / (H / H_kv), bh_kv = b * H_kv + h_kv;
+    // Q blocks and key tiles of this sequence (a packed batch has its own per sequence;
+    // Tq stays the row stride of qbar and dS)
+    const SeqRange sq = seq_range(cu_q, b, n_q_max, total_q), sk = seq_range(cu_kv, b, n_kv_max, total_kv);
+    const int Tq_s = cu_q ? (sq.n + kTile - 1) / kTile : Tq;
+    const int Tk_s = cu_kv ? (sk.n + kTile - 1) / kTile : Tk;
+    if (cu_q) causal_off = sk.n - sq.n;
     const int jt0 = blockIdx.x * kDsTilesPerCta;
-    const int n_kt = min(kDsTilesPerCta, Tk - jt0);
+    const int n_kt = min(kDsTilesPerCta, Tk_s - jt0);
+    if (n_kt <= 0 || Tq_s <= 0) return;  // past the end of a shorter packed sequence
     const bool is_bf16 = bf16 != 0;
 
     if (threadIdx.x == 0) {
@@ -91,13 +101,11 @@ __global__ void __launch_bounds__(kDsThreads, 1)
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort_flag = &sm.abort_flag;
-    // key/value head read by query head bh: h_kv = h / (H / H_kv)
-    const int b = bh / H, h_kv = (bh % H) / (H / H_kv), bh_kv = b * H_kv + h_kv;
 
     int g = 0;              // key tiles of earlier block chunks (buffer phases run on across chunks)
     uint32_t n_chunks = 0;  // epilogue store boxes issued (staging buffer parity)
-    for (int tc = 0; tc < Tq; tc += kDsMaxN) {
-        const int nt = min(kDsMaxN, Tq - tc);
+    for (int tc = 0; tc < Tq_s; tc += kDsMaxN) {
+        const int nt = min(kDsMaxN, Tq_s - tc);
         const int N = (nt + 15) / 16 * 16;
         // --- stage qbar[tc .. tc + N) as hi / lo 16-bit K-major operands (128-byte swizzle)
         const float *qsrc = qbar + ((size_t)bh * Tq + tc) * D;
@@ -137,7 +145,8 @@ __global__ void __launch_bounds__(kDsThreads, 1)
                 const int j0 = (jt0 + i) * kTile;
                 mbar_arrive_expect_tx(&sm.bar_kfull[buf], KA * kTile * 128);
                 for (int a = 0; a < KA; ++a) {
-                    if (nhd) tma_load_4d(sm.k[buf][a], &tm_k, &sm.bar_kfull[buf], a * 64, h_kv, j0, b);
+                    if (cu_kv) tma_load_4d(sm.k[buf][a], &tm_k, &sm.bar_kfull[buf], a * 64, h_kv, sk.off + j0, 0);
+                    else if (nhd) tma_load_4d(sm.k[buf][a], &tm_k, &sm.bar_kfull[buf], a * 64, h_kv, j0, b);
                     else tma_load_3d(sm.k[buf][a], &tm_k, &sm.bar_kfull[buf], a * 64, j0, bh_kv);
                 }
                 issued = i + 1;
@@ -237,20 +246,23 @@ __global__ void __launch_bounds__(kDsThreads, 1)
 }
 
 cudaError_t launch_ds_gemm(const CUtensorMap &tm_k, const CUtensorMap &tm_ds, const float *qbar, const Shape &s,
-                           int nhd, int bf16, int causal_skip, int causal_off, int *status, cudaStream_t stream) {
+                           int nhd, int bf16, int causal_skip, int causal_off, const int *cu_q, const int *cu_kv,
+                           int *status, cudaStream_t stream) {
     dim3 grid((s.Tk + kDsTilesPerCta - 1) / kDsTilesPerCta, s.BH);
     if (s.d == 128) {
         const size_t smem = sizeof(DsSmem<128>) + 1024;
         cudaError_t e = cudaFuncSetAttribute(ds_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         ds_gemm_kernel<128><<<grid, kDsThreads, smem, stream>>>(tm_k, tm_ds, qbar, s.H, s.H_kv, s.Tq, s.Tk, nhd, bf16,
-                                                                 causal_skip, causal_off, status);
+                                                                 causal_skip, causal_off, cu_q, cu_kv, s.n_q, s.n_kv,
+                                                                 s.total_q, s.total_kv, status);
     } else {
         const size_t smem = sizeof(DsSmem<64>) + 1024;
         cudaError_t e = cudaFuncSetAttribute(ds_gemm_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         ds_gemm_kernel<64><<<grid, kDsThreads, smem, stream>>>(tm_k, tm_ds, qbar, s.H, s.H_kv, s.Tq, s.Tk, nhd, bf16,
-                                                                causal_skip, causal_off, status);
+                                                                causal_skip, causal_off, cu_q, cu_kv, s.n_q, s.n_kv,
+                                                                s.total_q, s.total_kv, status);
     }
     return cudaGetLastError();
 }

@@ -143,11 +143,15 @@ struct QuantRing {
 
 // TMA load of work unit u (row tile t = u % T of head bh = u / T) of a 16-bit
 // [BH][n][d] (head-major) or [B][n][H][d] (token-major) tensor; rows past n read 0.
+// A packed batch (cu not null) is token-major [1][total][H][d]: tile t of sequence b
+// starts at token cu[b] + 128 t (its rows past the sequence belong to the next one and
+// are masked by the consumer).
 __device__ __forceinline__ void load_rows_tile(const CUtensorMap *tm, int nhd, int H, int T, int u, void *dst,
-                                               uint64_t *bar, uint32_t bytes) {
+                                               uint64_t *bar, uint32_t bytes, const int *cu, int n_max, int total) {
     const int bh = u / T, t = u % T;
     mbar_arrive_expect_tx(bar, bytes);
-    if (nhd) tma_load_4d(dst, tm, bar, 0, bh % H, t * kTile, bh / H);
+    if (cu) tma_load_4d(dst, tm, bar, 0, bh % H, seq_range(cu, bh / H, n_max, total).off + t * kTile, 0);
+    else if (nhd) tma_load_4d(dst, tm, bar, 0, bh % H, t * kTile, bh / H);
     else tma_load_3d(dst, tm, bar, 0, t * kTile, bh);
 }
 
@@ -159,11 +163,14 @@ struct RingCtl {
     uint64_t *full;
     int n_units, T, H, nhd;
     const CUtensorMap *tm;
+    const int *cu;   // packed batch offsets, or null
+    int n_max, total;
     __device__ __forceinline__ uint16_t *stage(int k) const { return ring + (size_t)(k % QuantRing<D>::kStages) * kTile * D; }
     __device__ __forceinline__ void issue(int k) const {  // load this CTA's k-th unit, if any
         const int u = blockIdx.x + k * gridDim.x;
         if (u < n_units)
-            load_rows_tile(tm, nhd, H, T, u, stage(k), &full[k % QuantRing<D>::kStages], QuantRing<D>::kTileBytes);
+            load_rows_tile(tm, nhd, H, T, u, stage(k), &full[k % QuantRing<D>::kStages], QuantRing<D>::kTileBytes,
+                           cu, n_max, total);
     }
     __device__ __forceinline__ bool wait(int k, volatile int *abort_flag, int *status) const {
         return __all_sync(0xFFFFFFFFu, mbar_wait(&full[k % QuantRing<D>::kStages], (k / QuantRing<D>::kStages) & 1,
@@ -179,7 +186,7 @@ struct RingCtl {
 
 template <int D>
 __device__ __forceinline__ RingCtl<D> ring_setup(const CUtensorMap *tm, int nhd, int H, int T, int BH, uint64_t *full,
-                                                 volatile int *abort_flag) {
+                                                 volatile int *abort_flag, const int *cu, int n_max, int total) {
     extern __shared__ uint8_t smem_raw[];
     RingCtl<D> rc;
     rc.ring = reinterpret_cast<uint16_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -189,6 +196,9 @@ __device__ __forceinline__ RingCtl<D> ring_setup(const CUtensorMap *tm, int nhd,
     rc.H = H;
     rc.nhd = nhd;
     rc.tm = tm;
+    rc.cu = cu;
+    rc.n_max = n_max;
+    rc.total = total;
     if (threadIdx.x == 0) {
         for (int s = 0; s < QuantRing<D>::kStages; ++s) mbar_init(&full[s], 1);
         *abort_flag = 0;
@@ -218,14 +228,16 @@ __global__ void __launch_bounds__(256) kv_stats_kernel(const PrepassArgs a) {
     const int chunk = blockIdx.x, bh = blockIdx.y;
     const int b = bh / a.shape.H_kv, h = bh % a.shape.H_kv;  // key/value head
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const SeqRange sr = seq_range(a.cu_kv, b, a.shape.n_kv, a.shape.total_kv);
+    const int64_t base = a.cu_kv ? (int64_t)sr.off * a.skv.n + h * a.skv.h : b * a.skv.b + h * a.skv.h;
     const int j0 = chunk * kStatChunk;
-    const int j1 = min(j0 + kStatChunk, a.shape.n_kv);
+    const int j1 = min(j0 + kStatChunk, sr.n);
     double ks[VEC];
     float vm[VEC];
 #pragma unroll
     for (int v = 0; v < VEC; ++v) { ks[v] = 0.0; vm[v] = 0.f; }
-    const uint16_t *kp = a.k ? static_cast<const uint16_t *>(a.k) + b * a.skv.b + h * a.skv.h + lane * VEC : nullptr;
-    const uint16_t *vp = a.v ? static_cast<const uint16_t *>(a.v) + b * a.skv.b + h * a.skv.h + lane * VEC : nullptr;
+    const uint16_t *kp = a.k ? static_cast<const uint16_t *>(a.k) + base + lane * VEC : nullptr;
+    const uint16_t *vp = a.v ? static_cast<const uint16_t *>(a.v) + base + lane * VEC : nullptr;
     for (int j = j0 + warp; j < j1; j += 8) {
         float x[VEC];
         if (kp) {
@@ -261,11 +273,12 @@ template <int D>
 __global__ void kv_finalize_kernel(const PrepassArgs a) {
     const int bh = blockIdx.x, c = threadIdx.x;
     const int nc = a.shape.n_chunks;
+    const int n_kv = seq_range(a.cu_kv, bh / a.shape.H_kv, a.shape.n_kv, a.shape.total_kv).n;
     if (a.k) {
         const double *part = reinterpret_cast<const double *>(a.ws + a.L.ksum_part) + (size_t)bh * nc * D + c;
         double s = 0.0;
         for (int ch = 0; ch < nc; ++ch) s = __dadd_rn(s, part[(size_t)ch * D]);
-        const float kb = (a.smooth_k && a.shape.n_kv > 0) ? (float)__ddiv_rn(s, (double)a.shape.n_kv) : 0.f;
+        const float kb = (a.smooth_k && n_kv > 0) ? (float)__ddiv_rn(s, (double)n_kv) : 0.f;
         reinterpret_cast<float *>(a.ws + a.L.kbar)[(size_t)bh * D + c] = kb;
     }
     if (a.v) {
@@ -288,14 +301,19 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
     const Shape &S = a.shape;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *status = reinterpret_cast<int *>(a.ws + a.L.status);
-    const RingCtl<D> rc = ring_setup<D>(&a.tm_q, a.nhd, S.H, S.Tq, S.BH, s_full, &s_abort);
+    const RingCtl<D> rc = ring_setup<D>(&a.tm_q, a.nhd, S.H, S.Tq, S.BH, s_full, &s_abort, a.cu_q, S.n_q, S.total_q);
     int k = 0;
     for (;; ++k) {
         const int u = blockIdx.x + k * gridDim.x;
         if (u >= rc.n_units) break;
         if (!rc.wait(k, &s_abort, status)) break;
         const int bh = u / S.Tq, t = u % S.Tq;
-        const int r0 = t * kTile, nvalid = min(kTile, S.n_q - r0);
+        const int r0 = t * kTile, nvalid = min(kTile, seq_range(a.cu_q, bh / S.H, S.n_q, S.total_q).n - r0);
+        if (nvalid <= 0) {  // a tile past the end of a shorter packed sequence: nothing to do
+            __syncthreads();
+            if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
+            continue;
+        }
         const uint16_t *tile = rc.stage(k) + lane * VEC;
         float x[RPW][VEC];
         double ps[VEC];
@@ -376,14 +394,20 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_
     const Shape &S = a.shape;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *status = reinterpret_cast<int *>(a.ws + a.L.status);
-    const RingCtl<D> rc = ring_setup<D>(&a.tm_k, a.nhd, S.H_kv, S.Tk, S.BH_kv, s_full, &s_abort);
+    const RingCtl<D> rc =
+        ring_setup<D>(&a.tm_k, a.nhd, S.H_kv, S.Tk, S.BH_kv, s_full, &s_abort, a.cu_kv, S.n_kv, S.total_kv);
     int k = 0;
     for (;; ++k) {
         const int u = blockIdx.x + k * gridDim.x;
         if (u >= rc.n_units) break;
         if (!rc.wait(k, &s_abort, status)) break;
         const int bh = u / S.Tk, jt = u % S.Tk;
-        const int j0 = jt * kTile, nvalid = min(kTile, S.n_kv - j0);
+        const int j0 = jt * kTile, nvalid = min(kTile, seq_range(a.cu_kv, bh / S.H_kv, S.n_kv, S.total_kv).n - j0);
+        if (nvalid <= 0) {  // a tile past the end of a shorter packed sequence
+            __syncthreads();
+            if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
+            continue;
+        }
         const uint16_t *tile = rc.stage(k) + lane * VEC;
         float kb[VEC];
 #pragma unroll
@@ -432,14 +456,20 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_
     const Shape &S = a.shape;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *status = reinterpret_cast<int *>(a.ws + a.L.status);
-    const RingCtl<D> rc = ring_setup<D>(&a.tm_v, a.nhd, S.H_kv, S.Tk, S.BH_kv, s_full, &s_abort);
+    const RingCtl<D> rc =
+        ring_setup<D>(&a.tm_v, a.nhd, S.H_kv, S.Tk, S.BH_kv, s_full, &s_abort, a.cu_kv, S.n_kv, S.total_kv);
     int k = 0;
     for (;; ++k) {
         const int u = blockIdx.x + k * gridDim.x;
         if (u >= rc.n_units) break;
         if (!rc.wait(k, &s_abort, status)) break;
         const int bh = u / S.Tk, jt = u % S.Tk;
-        const int j0 = jt * kTile, nvalid = min(kTile, S.n_kv - j0);
+        const int j0 = jt * kTile, nvalid = min(kTile, seq_range(a.cu_kv, bh / S.H_kv, S.n_kv, S.total_kv).n - j0);
+        if (nvalid <= 0) {  // a tile past the end of a shorter packed sequence
+            __syncthreads();
+            if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
+            continue;
+        }
         const uint16_t *tile = rc.stage(k) + lane * VEC;
         float x[RPW][VEC];
 #pragma unroll

@@ -115,7 +115,7 @@ bool make_k16_map(CUtensorMap *map, const void *k, int dtype, int layout, const 
         (dtype == SAGE_DTYPE_BF16) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const uint64_t d = (uint64_t)s.d;
     CUresult r;
-    if (layout == SAGE_LAYOUT_HND) {
+    if (layout == SAGE_LAYOUT_HND && !s.varlen) {
         cuuint64_t dims[3] = {d, (uint64_t)s.n_kv, (uint64_t)s.BH_kv};
         cuuint64_t strides[2] = {d * 2, (uint64_t)s.n_kv * d * 2};
         cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
@@ -123,8 +123,11 @@ bool make_k16_map(CUtensorMap *map, const void *k, int dtype, int layout, const 
         r = enc(map, dt, 3, const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     } else {
-        cuuint64_t dims[4] = {d, (uint64_t)s.H_kv, (uint64_t)s.n_kv, (uint64_t)s.B};
-        cuuint64_t strides[3] = {d * 2, (uint64_t)s.H_kv * d * 2, (uint64_t)s.n_kv * s.H_kv * d * 2};
+        // token-major; a packed batch is one "batch" of total_kv tokens
+        const uint64_t n = s.varlen ? (uint64_t)s.total_kv : (uint64_t)s.n_kv;
+        const uint64_t nb = s.varlen ? 1 : (uint64_t)s.B;
+        cuuint64_t dims[4] = {d, (uint64_t)s.H_kv, n, nb};
+        cuuint64_t strides[3] = {d * 2, (uint64_t)s.H_kv * d * 2, n * s.H_kv * d * 2};
         cuuint32_t box[4] = {64, 1, (cuuint32_t)kTile, 1};
         cuuint32_t estr[4] = {1, 1, 1, 1};
         r = enc(map, dt, 4, const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -133,16 +136,17 @@ bool make_k16_map(CUtensorMap *map, const void *k, int dtype, int layout, const 
     return r == CUDA_SUCCESS;
 }
 
-// Load map of a caller's 16-bit Q, K or V (n rows per head): d x 128-row boxes, no
-// swizzle; rows past n read as zero.
-bool make_rows16_map(CUtensorMap *map, const void *x, int dtype, int layout, const Shape &s, int n, int heads) {
+// Load map of a caller's 16-bit Q, K or V (n rows per head, `batches` batches): d x
+// 128-row boxes, no swizzle; rows past n read as zero.
+bool make_rows16_map(CUtensorMap *map, const void *x, int dtype, int layout, const Shape &s, int n, int heads,
+                     int batches) {
     auto enc = get_encode();
     if (!enc) return false;
     const CUtensorMapDataType dt =
         (dtype == SAGE_DTYPE_BF16) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const uint64_t d = (uint64_t)s.d;
     if (layout == SAGE_LAYOUT_HND) {
-        cuuint64_t dims[3] = {d, (uint64_t)n, (uint64_t)s.B * heads};
+        cuuint64_t dims[3] = {d, (uint64_t)n, (uint64_t)batches * heads};
         cuuint64_t strides[2] = {d * 2, (uint64_t)n * d * 2};
         cuuint32_t box[3] = {(cuuint32_t)d, (cuuint32_t)kTile, 1};
         cuuint32_t estr[3] = {1, 1, 1};
@@ -150,7 +154,7 @@ bool make_rows16_map(CUtensorMap *map, const void *x, int dtype, int layout, con
                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     }
-    cuuint64_t dims[4] = {d, (uint64_t)heads, (uint64_t)n, (uint64_t)s.B};
+    cuuint64_t dims[4] = {d, (uint64_t)heads, (uint64_t)n, (uint64_t)batches};
     cuuint64_t strides[3] = {d * 2, (uint64_t)heads * d * 2, (uint64_t)n * heads * d * 2};
     cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)kTile, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
@@ -173,19 +177,26 @@ bool make_ds_map(CUtensorMap *map, float *ds, const Shape &s) {
            CUDA_SUCCESS;
 }
 
+// Pre-pass of a dense batch (cu_q = cu_kv = null) or of a packed one (token-major
+// [total][heads][d] tensors, per-sequence offsets cu_q, cu_kv on the device).
 sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype, int layout, const Shape &s,
-                          const Mode &m, uint8_t *ws, int ds_t_skip, int causal_off, cudaStream_t stream) {
+                          const Mode &m, uint8_t *ws, int ds_t_skip, int causal_off, const int *cu_q,
+                          const int *cu_kv, cudaStream_t stream) {
     PrepassArgs a;
     a.q = q;
     a.k = k;
     a.v = v;
     a.bf16 = (dtype == SAGE_DTYPE_BF16);
     a.nhd = (layout == SAGE_LAYOUT_NHD);
-    if (q && !make_rows16_map(&a.tm_q, q, dtype, layout, s, s.n_q, s.H)) return SAGE_ERR_CUDA;
-    if (k && !make_rows16_map(&a.tm_k, k, dtype, layout, s, s.n_kv, s.H_kv)) return SAGE_ERR_CUDA;
-    if (v && !make_rows16_map(&a.tm_v, v, dtype, layout, s, s.n_kv, s.H_kv)) return SAGE_ERR_CUDA;
-    a.sq = make_strides(layout, s.H, s.n_q, s.d);
-    a.skv = make_strides(layout, s.H_kv, s.n_kv, s.d);
+    a.cu_q = cu_q;
+    a.cu_kv = cu_kv;
+    const int nq_rows = s.varlen ? s.total_q : s.n_q, nkv_rows = s.varlen ? s.total_kv : s.n_kv;
+    const int batches = s.varlen ? 1 : s.B;
+    if (q && !make_rows16_map(&a.tm_q, q, dtype, layout, s, nq_rows, s.H, batches)) return SAGE_ERR_CUDA;
+    if (k && !make_rows16_map(&a.tm_k, k, dtype, layout, s, nkv_rows, s.H_kv, batches)) return SAGE_ERR_CUDA;
+    if (v && !make_rows16_map(&a.tm_v, v, dtype, layout, s, nkv_rows, s.H_kv, batches)) return SAGE_ERR_CUDA;
+    a.sq = make_strides(layout, s.H, nq_rows, s.d);
+    a.skv = make_strides(layout, s.H_kv, nkv_rows, s.d);
     a.shape = s;
     a.g_q = m.g_q;
     a.g_k = m.g_k;
@@ -200,19 +211,20 @@ sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype
         if (!make_k16_map(&tmk, k, dtype, layout, s)) return SAGE_ERR_CUDA;
         if (!make_ds_map(&tmds, reinterpret_cast<float *>(ws + a.L.ds), s)) return SAGE_ERR_CUDA;
         if (launch_ds_gemm(tmk, tmds, reinterpret_cast<const float *>(ws + a.L.qbar), s, layout == SAGE_LAYOUT_NHD,
-                           dtype == SAGE_DTYPE_BF16, ds_t_skip, causal_off, reinterpret_cast<int *>(ws + a.L.status),
-                           stream) != cudaSuccess)
+                           dtype == SAGE_DTYPE_BF16, ds_t_skip, causal_off, cu_q, cu_kv,
+                           reinterpret_cast<int *>(ws + a.L.status), stream) != cudaSuccess)
             return SAGE_ERR_CUDA;
     }
     return SAGE_OK;
 }
 
 sage_status_t run_attention(void *o, int dtype, int layout, const Shape &s, int causal, float sm_scale,
-                            const Mode &m, const uint8_t *ws, int fault_inject, cudaStream_t stream) {
+                            const Mode &m, const uint8_t *ws, int fault_inject, const int *cu_q, const int *cu_kv,
+                            cudaStream_t stream) {
     CUtensorMap tq, tk, tv;
     if (!make_maps(s, ws, &tq, &tk, &tv)) return SAGE_ERR_CUDA;
     const WsLayout L = ws_layout(s);
-    const Strides so = make_strides(layout, s.H, s.n_q, s.d);
+    const Strides so = make_strides(layout, s.H, s.varlen ? s.total_q : s.n_q, s.d);
     AttnParams p;
     p.dq = reinterpret_cast<const float *>(ws + L.dq);
     p.dk = reinterpret_cast<const float *>(ws + L.dk);
@@ -234,6 +246,10 @@ sage_status_t run_attention(void *o, int dtype, int layout, const Shape &s, int 
     p.nq_pad = s.nq_pad;
     p.nk_pad = s.nk_pad;
     p.BH = s.BH;
+    p.cu_q = cu_q;
+    p.cu_kv = cu_kv;
+    p.total_q = s.total_q;
+    p.total_kv = s.total_kv;
     p.causal = causal ? 1 : 0;
     p.use_ds = m.smooth_q;
     p.out_bf16 = (dtype == SAGE_DTYPE_BF16);
@@ -308,7 +324,7 @@ sage_status_t sage_quant_qk_gqa(const void *q, const void *k, int dtype, int lay
     if ((q && !aligned16(q)) || (k && !aligned16(k))) return SAGE_ERR_UNSUPPORTED;
     SAGE_TRY(check_ws(s, workspace, workspace_bytes));
     return run_prepass(n_q > 0 ? q : nullptr, n_kv > 0 ? k : nullptr, nullptr, dtype, layout, s, m,
-                       static_cast<uint8_t *>(workspace), 0, 0, static_cast<cudaStream_t>(stream));
+                       static_cast<uint8_t *>(workspace), 0, 0, nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_quant_qk(const void *q, const void *k, int dtype, int layout, int B, int H, int n_q, int n_kv,
@@ -329,8 +345,8 @@ sage_status_t sage_quant_v_gqa(const void *v, int dtype, int layout, int B, int 
     if (!v) return SAGE_ERR_INVALID_ARG;
     if (!aligned16(v)) return SAGE_ERR_UNSUPPORTED;
     SAGE_TRY(check_ws(s, workspace, workspace_bytes));
-    return run_prepass(nullptr, nullptr, v, dtype, layout, s, m, static_cast<uint8_t *>(workspace), 0, 0,
-                       static_cast<cudaStream_t>(stream));
+    return run_prepass(nullptr, nullptr, v, dtype, layout, s, m, static_cast<uint8_t *>(workspace), 0, 0, nullptr,
+                       nullptr, static_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_quant_v(const void *v, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
@@ -354,7 +370,8 @@ sage_status_t sage_attn_fwd_prequant_gqa(void *o, int dtype, int layout, int B, 
     if (n_kv == 0)
         return cudaMemsetAsync(o, 0, (size_t)s.BH * n_q * d * 2, st) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
     SAGE_TRY(check_ws(s, workspace, workspace_bytes));
-    return run_attention(o, dtype, layout, s, causal, sm_scale, m, static_cast<const uint8_t *>(workspace), 0, st);
+    return run_attention(o, dtype, layout, s, causal, sm_scale, m, static_cast<const uint8_t *>(workspace), 0, nullptr,
+                         nullptr, st);
 }
 
 sage_status_t sage_attn_fwd_prequant(void *o, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
@@ -381,8 +398,8 @@ sage_status_t sage_attn_fwd_gqa(const void *q, const void *k, const void *v, voi
         return cudaMemsetAsync(o, 0, (size_t)s.BH * n_q * d * 2, st) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
     SAGE_TRY(check_ws(s, workspace, workspace_bytes));
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    SAGE_TRY(run_prepass(q, k, v, dtype, layout, s, m, ws, causal ? 1 : 0, n_kv - n_q, st));
-    return run_attention(o, dtype, layout, s, causal, sm_scale, m, ws, 0, st);
+    SAGE_TRY(run_prepass(q, k, v, dtype, layout, s, m, ws, causal ? 1 : 0, n_kv - n_q, nullptr, nullptr, st));
+    return run_attention(o, dtype, layout, s, causal, sm_scale, m, ws, 0, nullptr, nullptr, st);
 }
 
 sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *o, int dtype, int layout, int B,
@@ -390,6 +407,39 @@ sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *o
                             const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes, void *stream) {
     return sage_attn_fwd_gqa(q, k, v, o, dtype, layout, B, H, H, n_q, n_kv, d, causal, sm_scale, mode, workspace,
                              workspace_bytes, stream);
+}
+
+size_t sage_workspace_bytes_varlen(int B, int H, int H_kv, int max_seqlen_q, int max_seqlen_kv, int d) {
+    return sage_workspace_bytes_gqa(B, H, H_kv, max_seqlen_q, max_seqlen_kv, d);
+}
+
+sage_status_t sage_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, int dtype,
+                                   const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_kv, int B, int H, int H_kv,
+                                   int total_q, int total_kv, int max_seqlen_q, int max_seqlen_kv, int d, int causal,
+                                   float sm_scale, const sage_quant_mode_t *mode, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    Shape s;
+    Mode m;
+    SAGE_TRY(check_common(dtype, SAGE_LAYOUT_NHD));
+    if (total_q < 0 || total_kv < 0 || total_q > (1 << 30) || total_kv > (1 << 30)) return SAGE_ERR_INVALID_ARG;
+    SAGE_TRY(check_sizes(B, H, H_kv, max_seqlen_q, max_seqlen_kv, d, &s));
+    SAGE_TRY(read_mode(mode, &m));
+    s.varlen = 1;
+    s.total_q = total_q;
+    s.total_kv = total_kv;
+    if (s.BH == 0 || total_q == 0 || max_seqlen_q == 0) return SAGE_OK;
+    if (!q || !o || !cu_seqlens_q || !cu_seqlens_kv) return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(o)) return SAGE_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (total_kv == 0 || max_seqlen_kv == 0)
+        return cudaMemsetAsync(o, 0, (size_t)total_q * H * d * 2, st) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+    if (!k || !v) return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v)) return SAGE_ERR_UNSUPPORTED;
+    SAGE_TRY(check_ws(s, workspace, workspace_bytes));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    SAGE_TRY(run_prepass(q, k, v, dtype, SAGE_LAYOUT_NHD, s, m, ws, causal ? 1 : 0, 0, cu_seqlens_q, cu_seqlens_kv,
+                         st));
+    return run_attention(o, dtype, SAGE_LAYOUT_NHD, s, causal, sm_scale, m, ws, 0, cu_seqlens_q, cu_seqlens_kv, st);
 }
 
 sage_status_t sage_get_device_status(void *workspace, void *stream, int *code, int *site) {
@@ -443,8 +493,8 @@ sage_status_t sage_debug_attn_fault_inject(void *o, int dtype, int layout, int B
     SAGE_TRY(read_mode(nullptr, &m));
     if (!o || s.BH == 0 || n_q == 0 || n_kv == 0) return SAGE_ERR_INVALID_ARG;
     SAGE_TRY(check_ws(s, workspace, workspace_bytes));
-    return run_attention(o, dtype, layout, s, causal, 0.f, m, static_cast<const uint8_t *>(workspace), 1,
-                         static_cast<cudaStream_t>(stream));
+    return run_attention(o, dtype, layout, s, causal, 0.f, m, static_cast<const uint8_t *>(workspace), 1, nullptr,
+                         nullptr, static_cast<cudaStream_t>(stream));
 }
 
 const char *sage_version(void) { return "libsage_b200 1.0 (sm_100a; tcgen05 INT8 QK / FP8 PV)"; }

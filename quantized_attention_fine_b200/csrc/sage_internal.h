@@ -16,14 +16,19 @@ constexpr size_t kStatusBytes = 256;
 
 // H query heads share H_kv key/value heads (H_kv divides H; H_kv = H is multi-head
 // attention): query head h reads key/value head h / (H / H_kv).
+// Variable-length batches (varlen = 1): B sequences packed token-major, sequence b
+// holding tokens [cu[b], cu[b + 1]) of [total][heads][d] tensors; n_q and n_kv are then
+// the longest lengths, and every per-sequence workspace array is padded to them.
 struct Shape {
     int B, H, H_kv, n_q, n_kv, d;
     int BH, BH_kv, Tq, Tk, nq_pad, nk_pad, n_chunks;
+    int varlen, total_q, total_kv;
 };
 
 inline Shape make_shape(int B, int H, int H_kv, int n_q, int n_kv, int d) {
     Shape s;
     s.B = B; s.H = H; s.H_kv = H_kv; s.n_q = n_q; s.n_kv = n_kv; s.d = d;
+    s.varlen = 0; s.total_q = 0; s.total_kv = 0;
     s.BH = B * H;
     s.BH_kv = B * H_kv;
     s.Tq = (n_q + kTile - 1) / kTile;
@@ -65,6 +70,21 @@ inline WsLayout ws_layout(const Shape &s) {
     return w;
 }
 
+// Token offset and length of sequence b of a packed batch (cu: B + 1 offsets), clamped
+// so that the range lies inside [0, total) and is no longer than n_max.  Without cu
+// (a dense batch) every sequence has length n_max and the offset is unused.
+struct SeqRange {
+    int off, n;
+};
+__host__ __device__ __forceinline__ SeqRange seq_range(const int *cu, int b, int n_max, int total) {
+    if (!cu) return SeqRange{0, n_max};
+    int a0 = cu[b], a1 = cu[b + 1];
+    a0 = a0 < 0 ? 0 : (a0 > total ? total : a0);
+    a1 = a1 < a0 ? a0 : (a1 > total ? total : a1);
+    const int n = a1 - a0;
+    return SeqRange{a0, n < n_max ? n : n_max};
+}
+
 // Element strides of a [B, H, N, d] (HND) or [B, N, H, d] (NHD) tensor.
 struct Strides {
     int64_t b, h, n;
@@ -82,6 +102,7 @@ struct PrepassArgs {
     CUtensorMap tm_q, tm_k, tm_v;
     const void *q, *k, *v;   // any may be null: that part is skipped
     int bf16, nhd;
+    const int *cu_q, *cu_kv;  // packed batch offsets (device), or null for a dense batch
     Strides sq, skv;
     Shape shape;
     int g_q, g_k, smooth_q, smooth_k;
@@ -97,6 +118,8 @@ struct AttnParams {
     void *o;
     int64_t so_b, so_h, so_n;
     int H, n_q, n_kv, Tq, Tk, nq_pad, nk_pad, BH;
+    const int *cu_q, *cu_kv;  // packed batch offsets (device), or null for a dense batch
+    int total_q, total_kv;
     int group;          // query heads per key/value head (H / H_kv)
     int H_kv;
     int head_block;     // query heads per block of the CTA order (set by launch_attention)
@@ -112,10 +135,14 @@ struct AttnParams {
 cudaError_t launch_prepass(const PrepassArgs &a, cudaStream_t stream);
 // dS = qbar . K^T on the tensor core.  tm_k: tensor map of the caller's 16-bit K
 // (3-D [BH][n_kv][d] for head-major, 4-D [B][n_kv][H][d] for token-major, 64 x 128
-// boxes, 128-byte swizzle).  causal_skip: leave entries of Q blocks that can never
-// see a key tile unwritten (key j visible to query i iff j <= i + causal_off).
+// boxes, 128-byte swizzle; for a packed batch 4-D [1][total_kv][H_kv][d]).
+// causal_skip: leave entries of Q blocks that can never see a key tile unwritten (key
+// j visible to query i iff j <= i + causal_off; for a packed batch the offset is each
+// sequence's n_kv - n_q and causal_off is unused).  cu_q, cu_kv: packed batch offsets
+// or null.
 cudaError_t launch_ds_gemm(const CUtensorMap &tm_k, const CUtensorMap &tm_ds, const float *qbar, const Shape &s,
-                           int nhd, int bf16, int causal_skip, int causal_off, int *status, cudaStream_t stream);
+                           int nhd, int bf16, int causal_skip, int causal_off, const int *cu_q, const int *cu_kv,
+                           int *status, cudaStream_t stream);
 cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                              const AttnParams &p, int d, cudaStream_t stream);
 cudaError_t launch_debug_qk_tile(const CUtensorMap &tq, const CUtensorMap &tk, int d, int q_row0, int k_row0,

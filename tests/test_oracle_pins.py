@@ -479,3 +479,37 @@ def test_lse_quantized_within_logit_error_bound(gran):
     err = np.abs(lse - ref)
     assert np.all(err <= row_bound + 1e-9)
     assert err.max() > 0   # the quantizers did act
+
+
+# ---------------------------------------------------------------------------
+# Packed variable-length batches
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_unquantized_equals_block_diagonal_masked_sdpa(causal):
+    """With the quantizers off the packed-batch forward is attention over the whole
+    packed token axis under a block-diagonal mask (each token sees only its own
+    sequence; causal bottom-right aligned inside each block), computed by torch's
+    scaled_dot_product_attention with an explicit boolean mask."""
+    g = torch.Generator().manual_seed(12)
+    lq, lk = [70, 1, 200, 129], [90, 5, 200, 60]
+    cu_q, cu_kv = np.concatenate([[0], np.cumsum(lq)]), np.concatenate([[0], np.cumsum(lk)])
+    H, H_kv, d = 4, 2, 64
+    q = torch.randn(cu_q[-1], H, d, generator=g, dtype=torch.float64)
+    k = torch.randn(cu_kv[-1], H_kv, d, generator=g, dtype=torch.float64) + 2.0
+    v = torch.randn(cu_kv[-1], H_kv, d, generator=g, dtype=torch.float64)
+    o = oracle.sage_attention_varlen(q.numpy(), k.numpy(), v.numpy(), cu_q, cu_kv, causal=causal, quant=(0, 0, 0))
+    seq_q = np.repeat(np.arange(len(lq)), lq)
+    seq_k = np.repeat(np.arange(len(lk)), lk)
+    pos_q = np.arange(cu_q[-1]) - cu_q[seq_q]
+    pos_k = np.arange(cu_kv[-1]) - cu_kv[seq_k]
+    mask = seq_q[:, None] == seq_k[None, :]
+    if causal:
+        off = (np.asarray(lk) - np.asarray(lq))[seq_q]
+        mask &= pos_k[None, :] <= pos_q[:, None] + off[:, None]
+    m = torch.from_numpy(mask)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.permute(1, 0, 2)[None], k.permute(1, 0, 2)[None], v.permute(1, 0, 2)[None], attn_mask=m,
+        enable_gqa=True)[0].permute(1, 0, 2).numpy()
+    seen = mask.any(1)   # rows with no visible key: SDPA gives NaN, the method 0
+    assert np.max(np.abs(o[seen] - ref[seen])) < 1e-12
+    assert np.all(o[~seen] == 0)
