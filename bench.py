@@ -35,7 +35,8 @@ FALLBACK_BF16_TFLOPS = 1590.0    # pool measurement used when MEASURED_PEAKS.jso
 # library kernels per step of sage_attn_fwd: kv_stats, kv_finalize, quant_q, quant_k,
 # quant_v, ds_gemm, attn_fwd_kernel
 LAUNCHES_PER_STEP = 7
-KERNEL_SOURCES = ["quantized_attention_fine_b200/csrc/attn_fwd.cu", "quantized_attention_fine_b200/csrc/sage_device.cuh"]
+KERNEL_SOURCES = ["quantized_attention_fine_b200/csrc/attn_fwd.cu", "quantized_attention_fine_b200/csrc/attn_mma.cuh",
+                  "quantized_attention_fine_b200/csrc/sage_device.cuh"]
 
 
 def parse_args():
@@ -50,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--mma-rates", action="store_true",
+                    help="print the tensor-core rate of each tcgen05.mma form (diagnostic) and exit")
     return ap.parse_args()
 
 
@@ -240,6 +243,12 @@ def main():
         raise SystemExit("%s (choices: %s, or sweep_n<N>_d<64|128>_<causal|full>)" % (e, ", ".join(wl.WORKLOADS)))
     if args.impl == "reference":
         return reference_arm(args, w)
+    if args.mma_rates:
+        import quantized_attention_fine_b200 as sage
+        rates = {k: sage.debug_mma_rate(k) for k in sage.MMA_KINDS}
+        print(json.dumps({"mma_rates": rates, "unit": "TFLOP/s (TOPS for s8_s32)", "shape": "M128 N256, one CTA per SM"}),
+              flush=True)
+        return 0
 
     import torch
     import torch.distributed as dist

@@ -262,6 +262,25 @@ SAGE_API sage_status_t sage_debug_qk_tile(const void *workspace, int B, int H, i
 SAGE_API sage_status_t sage_debug_pv_accumulate(const uint8_t *p, const uint8_t *vt, int n_tiles,
                                                 int d, float *o, void *stream);
 
+/* The same P . V sum with an FP16 accumulator (tcgen05.mma kind::f8f6f4, D format
+ * f16): the instruction SageAttention2++ moves PV to ("SageAttention2++" verdict,
+ * key_machinery), whose range narrowing Pr * Vr <= 2047/2 keeps the FP16 sums finite.
+ * o_raw: device uint32 [128][d], the raw 32-bit tensor-memory word of each
+ * accumulator element as read by tcgen05.ld (the FP16 value's position in the word
+ * is what the test establishes). */
+SAGE_API sage_status_t sage_debug_pv_accumulate_f16acc(const uint8_t *p, const uint8_t *vt, int n_tiles,
+                                                       int d, uint32_t *o_raw, void *stream);
+
+/* Tensor-core throughput probe: n_ctas CTAs (one per SM) each issue n_iter
+ * tcgen05.mma of M = 128, N = 256 and one 32-byte K step (K = 32 for 8-bit
+ * operands, 16 for 16-bit) from zeroed shared-memory tiles into one tensor-memory
+ * accumulator and wait for them.  kind: 0 E4M3 -> FP32, 1 E4M3 -> FP16, 2 S8 -> S32,
+ * 3 BF16 -> FP32.  The caller times the launch on `stream`: the rate is
+ * n_ctas * n_iter * 2 * 128 * 256 * K / t.  status_block: device buffer of at least
+ * 256 zeroed bytes, read with sage_get_device_status (a wait that runs out records
+ * SAGE_ERR_TIMEOUT).  n_iter <= 2^20, n_ctas <= 4096. */
+SAGE_API sage_status_t sage_debug_mma_rate(int kind, int n_iter, int n_ctas, void *status_block, void *stream);
+
 /* Runs the attention kernel with one deliberately missing producer signal so that
  * the consumer's bounded wait must run out; the kernel records SAGE_ERR_TIMEOUT in
  * the status block and exits without hanging.  Arguments as sage_attn_fwd_prequant. */

@@ -22,7 +22,7 @@ import threading
 __all__ = [
     "QuantMode", "Workspace", "workspace_bytes", "make_workspace", "quant_qk", "quant_v", "attn_fwd_prequant",
     "attn_fwd", "attn_fwd_varlen", "get_device_status", "workspace_view", "debug_qk_tile", "debug_pv_accumulate",
-    "debug_fault_inject", "library_path", "load_library", "SageError", "GRANULARITIES",
+    "debug_fault_inject", "debug_pv_accumulate_f16acc", "debug_mma_rate", "library_path", "load_library", "SageError", "GRANULARITIES",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -95,12 +95,15 @@ def load_library():
         lib.sage_get_device_status.argtypes = [P, P, ctypes.POINTER(I), ctypes.POINTER(I)]
         lib.sage_debug_qk_tile.argtypes = [P, I, I, I, I, I, I, I, I, P, P]
         lib.sage_debug_pv_accumulate.argtypes = [P, P, I, I, P, P]
+        lib.sage_debug_pv_accumulate_f16acc.argtypes = [P, P, I, I, P, P]
+        lib.sage_debug_mma_rate.argtypes = [I, I, I, P, P]
         lib.sage_debug_attn_fault_inject.argtypes = [P, I, I, I, I, I, I, I, I, P, S, P]
         lib.sage_version.restype = ctypes.c_char_p
         for fn in ("sage_quant_qk", "sage_quant_v", "sage_attn_fwd_prequant", "sage_attn_fwd",
                    "sage_quant_qk_gqa", "sage_quant_v_gqa", "sage_attn_fwd_prequant_gqa", "sage_attn_fwd_gqa",
                    "sage_attn_fwd_varlen",
                    "sage_get_device_status", "sage_debug_qk_tile", "sage_debug_pv_accumulate",
+                   "sage_debug_pv_accumulate_f16acc", "sage_debug_mma_rate",
                    "sage_debug_attn_fault_inject"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
@@ -372,6 +375,47 @@ def debug_pv_accumulate(p_codes, vt_codes, stream=None):
     _check(load_library().sage_debug_pv_accumulate(_ptr(p_codes), _ptr(vt_codes), T, d, _ptr(out),
                                                    _stream_handle(stream)), "sage_debug_pv_accumulate")
     return out
+
+
+def debug_pv_accumulate_f16acc(p_codes, vt_codes, stream=None):
+    """sum_t P_t . V_t on the FP8 tensor core with an FP16 accumulator (diagnostic).
+    Returns the raw 32-bit tensor-memory words, int32 [128, d]."""
+    torch = _torch()
+    T, d = int(p_codes.shape[0]), int(vt_codes.shape[1])
+    out = torch.empty((128, d), dtype=torch.int32, device=p_codes.device)
+    _check(load_library().sage_debug_pv_accumulate_f16acc(_ptr(p_codes), _ptr(vt_codes), T, d, _ptr(out),
+                                                          _stream_handle(stream)), "sage_debug_pv_accumulate_f16acc")
+    return out
+
+
+MMA_KINDS = {"e4m3_f32": (0, 32), "e4m3_f16": (1, 32), "s8_s32": (2, 32), "bf16_f32": (3, 16)}
+
+
+def debug_mma_rate(kind: str, n_iter: int = 8192, n_ctas=None, repeats: int = 5, stream=None):
+    """Tensor-core rate of one tcgen05.mma form (M = 128, N = 256; see MMA_KINDS), in
+    dense TFLOP/s (TOPS for S8): best of `repeats` timed launches after one warm-up."""
+    torch = _torch()
+    code, k = MMA_KINDS[kind]
+    dev = torch.cuda.current_device()
+    if n_ctas is None:
+        n_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+    status = torch.zeros(64, dtype=torch.int32, device="cuda")
+    s = stream if stream is not None else torch.cuda.current_stream()
+    lib = load_library()
+    best = float("inf")
+    for i in range(repeats + 1):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        _check(lib.sage_debug_mma_rate(code, n_iter, n_ctas, ctypes.c_void_p(status.data_ptr()),
+                                       ctypes.c_void_p(s.cuda_stream)), "sage_debug_mma_rate")
+        e1.record(s)
+        s.synchronize()
+        if i > 0:
+            best = min(best, e0.elapsed_time(e1))
+    if int(status[0].item()) != 0:
+        raise SageError(int(status[0].item()), "sage_debug_mma_rate (device wait)")
+    flops = n_ctas * n_iter * 2.0 * 128 * 256 * k
+    return flops / (best * 1e-3) / 1e12
 
 
 def debug_fault_inject(workspace: Workspace, out, *, layout="HND", causal=False, stream=None):

@@ -1,5 +1,6 @@
 // attn_fwd.cu -- fused sm_100a attention kernel of the smoothed-INT8-QK / FP8-PV
-// forward, plus two diagnostic kernels that reuse its MMA issue code.
+// forward (its MMA issue sequences are in attn_mma.cuh, shared with the diagnostic
+// kernels of debug_kernels.cu).
 //
 // Method (SageAttention2, arXiv 2411.10958, abstract; SageAttention2++ verdict on
 // pith.science, key_machinery): S = dQ(i) dK(j) (Q_int . K_int) + dS[t, j] on the
@@ -35,6 +36,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "attn_mma.cuh"
 #include "sage_device.cuh"
 #include "sage_internal.h"
 
@@ -56,7 +58,7 @@ constexpr uint32_t kRegsProducer = 32;
 constexpr uint32_t kRegsSoftmax = 112;
 
 // Wait-site ids recorded with a timeout.
-enum { kSiteQ = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteS = 4, kSiteP = 5, kSiteO = 6, kSiteSfree = 7, kSiteDebug = 9 };
+enum { kSiteQ = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteS = 4, kSiteP = 5, kSiteO = 6, kSiteSfree = 7 };
 
 // K tiles (with their dS rows and delta_K runs) and V^T tiles travel in separate
 // rings: a K slot is free once QK^T has read it and both tiles' warps have
@@ -83,41 +85,6 @@ struct __align__(1024) AttnSmem {
     int abort_flag;
     int bh_kv;  // key/value head of this CTA's query head (read by the epilogue)
 };
-
-// K-major operand layout of a Q or K tile: rows of d bytes; d = 128 uses the
-// 128-byte swizzle (8-row groups 1024 bytes apart), d = 64 the 64-byte swizzle.
-template <int D>
-struct QkLayout {
-    static constexpr uint32_t layout = (D == 128) ? 2u : 4u;
-    static constexpr uint32_t sbo = (D == 128) ? 1024u : 512u;
-};
-
-// S[d_tmem] = Q_tile . K_tile^T: d / 32 tcgen05.mma kind::i8 (M = 128, N = 128,
-// K = 32 each), the descriptor start advancing 32 bytes along the swizzled row.
-template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_saddr, uint32_t k_saddr) {
-    constexpr uint32_t idesc = idesc_s8_s32(128, 128);
-#pragma unroll
-    for (int kk = 0; kk < D / 32; ++kk) {
-        const uint64_t a = smem_desc(q_saddr + kk * 32, QkLayout<D>::sbo, QkLayout<D>::layout);
-        const uint64_t b = smem_desc(k_saddr + kk * 32, QkLayout<D>::sbo, QkLayout<D>::layout);
-        mma_s8_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
-    }
-}
-
-// O[d_tmem] (+)= P_tile . V_tile: P is 128 rows x 128 keys (E4M3, 128-byte rows,
-// 128-byte swizzle), V^T is d rows x 128 keys (same layout); 4 tcgen05.mma
-// kind::f8f6f4 with M = 128, N = d, K = 32.
-template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_saddr, uint32_t v_saddr, bool accumulate) {
-    constexpr uint32_t idesc = idesc_e4m3_f32(128, D);
-#pragma unroll
-    for (int kk = 0; kk < kTile / 32; ++kk) {
-        const uint64_t a = smem_desc(p_saddr + kk * 32, 1024u, 2u);
-        const uint64_t b = smem_desc(v_saddr + kk * 32, 1024u, 2u);
-        mma_e4m3_ss(d_tmem, a, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
-    }
-}
 
 // A bounded wait whose outcome is the same for all 32 lanes (so that the warp
 // leaves its loop together and its .sync.aligned instructions stay converged).
@@ -657,175 +624,6 @@ cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const
         return launch_attention_d<128, false>(tq, tk, tv, p, stream);
     }
     return launch_attention_d<64, true>(tq, tk, tv, p, stream);
-}
-
-// ---------------------------------------------------------------------------
-// Diagnostic: one S tile straight from tensor memory.
-// ---------------------------------------------------------------------------
-template <int D>
-struct __align__(1024) QkDebugSmem {
-    uint8_t q[kTile * D];
-    uint8_t k[kTile * D];
-    uint64_t bar_ld, bar_mma;
-    uint32_t tmem_base;
-    int abort_flag;
-};
-
-template <int D>
-__global__ void __launch_bounds__(128, 1)
-    debug_qk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int q_row0,
-                    int k_row0, int32_t *out, int *status) {
-    extern __shared__ uint8_t smem_raw[];
-    QkDebugSmem<D> &sm =
-        *reinterpret_cast<QkDebugSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        mbar_init(&sm.bar_ld, 1);
-        mbar_init(&sm.bar_mma, 1);
-        sm.abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0) { tmem_alloc(&sm.tmem_base, 128); tmem_relinquish(); }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = sm.tmem_base;
-    volatile int *abort_flag = &sm.abort_flag;
-    if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(&sm.bar_ld, 2 * kTile * D);
-        tma_load_2d(sm.q, &tm_q, &sm.bar_ld, 0, q_row0);
-        tma_load_2d(sm.k, &tm_k, &sm.bar_ld, 0, k_row0);
-        if (mbar_wait(&sm.bar_ld, 0, abort_flag, status, kSiteDebug)) {
-            tc_fence_after();
-            issue_qk<D>(tmem, smem_u32(sm.q), smem_u32(sm.k));
-        } else {
-            mbar_wait_quiet(&sm.bar_ld, 0, kDrainNs);
-        }
-        mma_commit(&sm.bar_mma);
-    }
-    __syncwarp();
-    mbar_wait(&sm.bar_mma, 0, abort_flag, status, kSiteDebug);
-    tc_fence_after();
-    __syncthreads();
-    if (*abort_flag == 0) {
-        const int r = warp * 32 + lane;
-#pragma unroll
-        for (int c0 = 0; c0 < kTile; c0 += 32) {
-            uint32_t v[32];
-            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
-            tmem_wait_ld_regs(v);
-            int4 *dst = reinterpret_cast<int4 *>(out + (size_t)r * kTile + c0);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_int4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) { __syncwarp(); tc_fence_after(); tmem_dealloc(tmem, 128); }
-}
-
-cudaError_t launch_debug_qk_tile(const CUtensorMap &tq, const CUtensorMap &tk, int d, int q_row0, int k_row0,
-                                 int32_t *s_out, int *status, cudaStream_t stream) {
-    if (d == 128) {
-        const size_t smem = sizeof(QkDebugSmem<128>) + 1024;
-        cudaError_t e = cudaFuncSetAttribute(debug_qk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        debug_qk_kernel<128><<<1, 128, smem, stream>>>(tq, tk, q_row0, k_row0, s_out, status);
-    } else {
-        const size_t smem = sizeof(QkDebugSmem<64>) + 1024;
-        cudaError_t e = cudaFuncSetAttribute(debug_qk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        debug_qk_kernel<64><<<1, 128, smem, stream>>>(tq, tk, q_row0, k_row0, s_out, status);
-    }
-    return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// Diagnostic: sum over tiles of P . V on the FP8 path, one FP32 accumulator.
-// P and V^T tiles are copied row by row into the 128-byte-swizzled layout the
-// attention kernel uses for P.
-// ---------------------------------------------------------------------------
-template <int D>
-struct __align__(1024) PvDebugSmem {
-    uint8_t p[kTile * kTile];
-    uint8_t v[D * kTile];
-    uint64_t bar_mma;
-    uint32_t tmem_base;
-    int abort_flag;
-};
-
-template <int D>
-__global__ void __launch_bounds__(128, 1)
-    debug_pv_kernel(const uint8_t *p, const uint8_t *vt, int n_tiles, float *out, int *status) {
-    extern __shared__ uint8_t smem_raw[];
-    PvDebugSmem<D> &sm =
-        *reinterpret_cast<PvDebugSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int warp = threadIdx.x >> 5;
-    const int r = threadIdx.x;
-    if (threadIdx.x == 0) {
-        mbar_init(&sm.bar_mma, 1);
-        sm.abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0) { tmem_alloc(&sm.tmem_base, 256); tmem_relinquish(); }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = sm.tmem_base;
-    volatile int *abort_flag = &sm.abort_flag;
-    bool ok = true;
-    for (int tile = 0; tile < n_tiles && ok; ++tile) {
-        const uint4 *src_p = reinterpret_cast<const uint4 *>(p + ((size_t)tile * kTile + r) * kTile);
-#pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) *reinterpret_cast<uint4 *>(sm.p + sw128_offset(r, c16)) = src_p[c16];
-        if (r < D) {
-            const uint4 *src_v = reinterpret_cast<const uint4 *>(vt + ((size_t)tile * D + r) * kTile);
-#pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16) *reinterpret_cast<uint4 *>(sm.v + sw128_offset(r, c16)) = src_v[c16];
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            tc_fence_after();
-            issue_pv<D>(tmem, smem_u32(sm.p), smem_u32(sm.v), tile > 0);
-            mma_commit(&sm.bar_mma);
-        }
-        __syncwarp();
-        mbar_wait(&sm.bar_mma, tile & 1, abort_flag, status, kSiteDebug);
-        tc_fence_after();
-        __syncthreads();
-        ok = (*abort_flag == 0);
-    }
-    if (ok && n_tiles > 0) {
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t v[32];
-            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
-            tmem_wait_ld_regs(v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) out[(size_t)r * D + c0 + i] = __uint_as_float(v[i]);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) { __syncwarp(); tc_fence_after(); tmem_dealloc(tmem, 256); }
-}
-
-cudaError_t launch_debug_pv(const uint8_t *p, const uint8_t *vt, int n_tiles, int d, float *o, int *status,
-                            cudaStream_t stream) {
-    if (d == 128) {
-        const size_t smem = sizeof(PvDebugSmem<128>) + 1024;
-        cudaError_t e = cudaFuncSetAttribute(debug_pv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        debug_pv_kernel<128><<<1, 128, smem, stream>>>(p, vt, n_tiles, o, status);
-    } else {
-        const size_t smem = sizeof(PvDebugSmem<64>) + 1024;
-        cudaError_t e = cudaFuncSetAttribute(debug_pv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        debug_pv_kernel<64><<<1, 128, smem, stream>>>(p, vt, n_tiles, o, status);
-    }
-    return cudaGetLastError();
 }
 
 }  // namespace sage

@@ -1,0 +1,281 @@
+// debug_kernels.cu -- diagnostic kernels: one QK^T tile and a PV sum through the
+// attention kernel's own MMA issue sequences (attn_mma.cuh), and the throughput of
+// the tcgen05.mma forms the forward uses, and of the FP8 form with an FP16 accumulator that SageAttention2++ builds
+// on ("SageAttention2++" verdict on arXiv 2505.21136, key_machinery: the
+// FP16-accumulator FP8 instruction, taken as twice as fast on RTX4090 / RTX5090).
+//
+// Each CTA (one per SM) zeroes an A tile (128 rows) and a B tile (256 rows) of
+// 128-byte K-major rows in shared memory, and one thread issues n_iter MMAs of
+// M = 128, N = 256 and one 32-byte K step each into a tensor-memory accumulator,
+// then waits (bounded) for their completion.  The host times the launch; the MMA
+// count and shape give the rate.  Kinds:
+//   0  kind::f8f6f4, E4M3 x E4M3, FP32 accumulator   (the forward's PV)
+//   1  kind::f8f6f4, E4M3 x E4M3, FP16 accumulator   (SageAttention2++ PV)
+//   2  kind::i8, S8 x S8, S32 accumulator            (the forward's QK^T)
+//   3  kind::f16, BF16 x BF16, FP32 accumulator      (dS)
+#include "attn_mma.cuh"
+#include "sage_device.cuh"
+#include "sage_internal.h"
+
+namespace sage {
+
+namespace {
+
+constexpr int kSiteDebug = 9;
+constexpr uint64_t kDrainNs = 50ull * 1000ull * 1000ull;
+
+struct __align__(1024) MmaRateSmem {
+    uint8_t a[128 * 128];
+    uint8_t b[256 * 128];
+    uint64_t bar;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+constexpr int kSiteRate = 41;
+// Dynamic shared memory requested per CTA: large enough that one CTA runs per SM.
+constexpr size_t kRateSmem = 160u * 1024u;
+
+}  // namespace
+
+template <int KIND>
+__global__ void __launch_bounds__(128, 1) debug_mma_rate_kernel(int n_iter, int *status) {
+    extern __shared__ uint8_t smem_raw[];
+    MmaRateSmem &sm =
+        *reinterpret_cast<MmaRateSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    uint4 *z = reinterpret_cast<uint4 *>(sm.a);
+    for (int i = threadIdx.x; i < (int)((sizeof(sm.a) + sizeof(sm.b)) / 16); i += 128) z[i] = make_uint4(0, 0, 0, 0);
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.bar, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) { tmem_alloc(&sm.tmem_base, 256); tmem_relinquish(); }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    if (threadIdx.x == 0) {
+        const uint32_t sa = smem_u32(sm.a), sb = smem_u32(sm.b);
+        for (int i = 0; i < n_iter; ++i) {
+            const uint32_t kk = (uint32_t)(i & 3) * 32u;
+            const uint64_t ad = smem_desc(sa + kk, 1024u, 2u), bd = smem_desc(sb + kk, 1024u, 2u);
+            const uint32_t acc = i > 0 ? 1u : 0u;
+            if constexpr (KIND == 0) mma_e4m3_ss(tmem, ad, bd, idesc_e4m3_f32(128, 256), acc);
+            else if constexpr (KIND == 1) mma_e4m3_ss(tmem, ad, bd, idesc_e4m3_f32(128, 256) & ~(3u << 4), acc);
+            else if constexpr (KIND == 2) mma_s8_ss(tmem, ad, bd, idesc_s8_s32(128, 256), acc);
+            else mma_f16_ss(tmem, ad, bd, idesc_f16_f32(128, 256, true), acc);
+        }
+        mma_commit(&sm.bar);
+    }
+    __syncwarp();
+    mbar_wait(&sm.bar, 0, &sm.abort_flag, status, kSiteRate);
+    tc_fence_after();
+    __syncthreads();
+    if (warp == 0) { __syncwarp(); tc_fence_after(); tmem_dealloc(tmem, 256); }
+}
+
+template <int KIND>
+static cudaError_t launch_rate(int n_iter, int n_ctas, int *status, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(debug_mma_rate_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kRateSmem);
+    if (e != cudaSuccess) return e;
+    debug_mma_rate_kernel<KIND><<<n_ctas, 128, kRateSmem, stream>>>(n_iter, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_debug_mma_rate(int kind, int n_iter, int n_ctas, int *status, cudaStream_t stream) {
+    static_assert(sizeof(MmaRateSmem) + 1024 <= kRateSmem, "operands fit the requested shared memory");
+    switch (kind) {
+        case 0: return launch_rate<0>(n_iter, n_ctas, status, stream);
+        case 1: return launch_rate<1>(n_iter, n_ctas, status, stream);
+        case 2: return launch_rate<2>(n_iter, n_ctas, status, stream);
+        default: return launch_rate<3>(n_iter, n_ctas, status, stream);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Diagnostic: one S tile straight from tensor memory.
+// ---------------------------------------------------------------------------
+template <int D>
+struct __align__(1024) QkDebugSmem {
+    uint8_t q[kTile * D];
+    uint8_t k[kTile * D];
+    uint64_t bar_ld, bar_mma;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+    debug_qk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int q_row0,
+                    int k_row0, int32_t *out, int *status) {
+    extern __shared__ uint8_t smem_raw[];
+    QkDebugSmem<D> &sm =
+        *reinterpret_cast<QkDebugSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.bar_ld, 1);
+        mbar_init(&sm.bar_mma, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) { tmem_alloc(&sm.tmem_base, 128); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int *abort_flag = &sm.abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(&sm.bar_ld, 2 * kTile * D);
+        tma_load_2d(sm.q, &tm_q, &sm.bar_ld, 0, q_row0);
+        tma_load_2d(sm.k, &tm_k, &sm.bar_ld, 0, k_row0);
+        if (mbar_wait(&sm.bar_ld, 0, abort_flag, status, kSiteDebug)) {
+            tc_fence_after();
+            issue_qk<D>(tmem, smem_u32(sm.q), smem_u32(sm.k));
+        } else {
+            mbar_wait_quiet(&sm.bar_ld, 0, kDrainNs);
+        }
+        mma_commit(&sm.bar_mma);
+    }
+    __syncwarp();
+    mbar_wait(&sm.bar_mma, 0, abort_flag, status, kSiteDebug);
+    tc_fence_after();
+    __syncthreads();
+    if (*abort_flag == 0) {
+        const int r = warp * 32 + lane;
+#pragma unroll
+        for (int c0 = 0; c0 < kTile; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
+            tmem_wait_ld_regs(v);
+            int4 *dst = reinterpret_cast<int4 *>(out + (size_t)r * kTile + c0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_int4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) { __syncwarp(); tc_fence_after(); tmem_dealloc(tmem, 128); }
+}
+
+cudaError_t launch_debug_qk_tile(const CUtensorMap &tq, const CUtensorMap &tk, int d, int q_row0, int k_row0,
+                                 int32_t *s_out, int *status, cudaStream_t stream) {
+    if (d == 128) {
+        const size_t smem = sizeof(QkDebugSmem<128>) + 1024;
+        cudaError_t e = cudaFuncSetAttribute(debug_qk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        debug_qk_kernel<128><<<1, 128, smem, stream>>>(tq, tk, q_row0, k_row0, s_out, status);
+    } else {
+        const size_t smem = sizeof(QkDebugSmem<64>) + 1024;
+        cudaError_t e = cudaFuncSetAttribute(debug_qk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        debug_qk_kernel<64><<<1, 128, smem, stream>>>(tq, tk, q_row0, k_row0, s_out, status);
+    }
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Diagnostic: sum over tiles of P . V on the FP8 path, one FP32 accumulator
+// (ACC16: an FP16 accumulator instead, the SageAttention2++ variant; the raw
+// 32-bit tensor-memory words are written out).  P and V^T tiles are copied row by
+// row into the 128-byte-swizzled layout the attention kernel uses for P.
+// ---------------------------------------------------------------------------
+template <int D>
+struct __align__(1024) PvDebugSmem {
+    uint8_t p[kTile * kTile];
+    uint8_t v[D * kTile];
+    uint64_t bar_mma;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+template <int D, bool ACC16>
+__global__ void __launch_bounds__(128, 1)
+    debug_pv_kernel(const uint8_t *p, const uint8_t *vt, int n_tiles, float *out, int *status) {
+    extern __shared__ uint8_t smem_raw[];
+    PvDebugSmem<D> &sm =
+        *reinterpret_cast<PvDebugSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    const int r = threadIdx.x;
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.bar_mma, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) { tmem_alloc(&sm.tmem_base, 256); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int *abort_flag = &sm.abort_flag;
+    bool ok = true;
+    for (int tile = 0; tile < n_tiles && ok; ++tile) {
+        const uint4 *src_p = reinterpret_cast<const uint4 *>(p + ((size_t)tile * kTile + r) * kTile);
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) *reinterpret_cast<uint4 *>(sm.p + sw128_offset(r, c16)) = src_p[c16];
+        if (r < D) {
+            const uint4 *src_v = reinterpret_cast<const uint4 *>(vt + ((size_t)tile * D + r) * kTile);
+#pragma unroll
+            for (int c16 = 0; c16 < 8; ++c16) *reinterpret_cast<uint4 *>(sm.v + sw128_offset(r, c16)) = src_v[c16];
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            tc_fence_after();
+            if constexpr (ACC16) {
+                constexpr uint32_t idesc = idesc_e4m3_f32(128, D) & ~(3u << 4);  // D format 0: f16
+#pragma unroll
+                for (int kk = 0; kk < kTile / 32; ++kk)
+                    mma_e4m3_ss(tmem, smem_desc(smem_u32(sm.p) + kk * 32, 1024u, 2u),
+                                smem_desc(smem_u32(sm.v) + kk * 32, 1024u, 2u), idesc, (tile > 0 || kk > 0) ? 1u : 0u);
+            } else {
+                issue_pv<D>(tmem, smem_u32(sm.p), smem_u32(sm.v), tile > 0);
+            }
+            mma_commit(&sm.bar_mma);
+        }
+        __syncwarp();
+        mbar_wait(&sm.bar_mma, tile & 1, abort_flag, status, kSiteDebug);
+        tc_fence_after();
+        __syncthreads();
+        ok = (*abort_flag == 0);
+    }
+    if (ok && n_tiles > 0) {
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
+            tmem_wait_ld_regs(v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) out[(size_t)r * D + c0 + i] = __uint_as_float(v[i]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) { __syncwarp(); tc_fence_after(); tmem_dealloc(tmem, 256); }
+}
+
+template <int D, bool ACC16>
+static cudaError_t launch_debug_pv_d(const uint8_t *p, const uint8_t *vt, int n_tiles, float *o, int *status,
+                                     cudaStream_t stream) {
+    const size_t smem = sizeof(PvDebugSmem<D>) + 1024;
+    cudaError_t e =
+        cudaFuncSetAttribute(debug_pv_kernel<D, ACC16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    debug_pv_kernel<D, ACC16><<<1, 128, smem, stream>>>(p, vt, n_tiles, o, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_debug_pv(const uint8_t *p, const uint8_t *vt, int n_tiles, int d, float *o, int *status,
+                            cudaStream_t stream, int acc_f16) {
+    if (d == 128)
+        return acc_f16 ? launch_debug_pv_d<128, true>(p, vt, n_tiles, o, status, stream)
+                       : launch_debug_pv_d<128, false>(p, vt, n_tiles, o, status, stream);
+    return acc_f16 ? launch_debug_pv_d<64, true>(p, vt, n_tiles, o, status, stream)
+                   : launch_debug_pv_d<64, false>(p, vt, n_tiles, o, status, stream);
+}
+
+}  // namespace sage

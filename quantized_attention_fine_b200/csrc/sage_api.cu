@@ -478,7 +478,27 @@ sage_status_t sage_debug_pv_accumulate(const uint8_t *p, const uint8_t *vt, int 
     if (!p || !vt || !o || n_tiles < 1) return SAGE_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
     if (!aligned16(p) || !aligned16(vt) || !aligned16(o)) return SAGE_ERR_UNSUPPORTED;
-    return launch_debug_pv(p, vt, n_tiles, d, o, nullptr, static_cast<cudaStream_t>(stream)) == cudaSuccess
+    return launch_debug_pv(p, vt, n_tiles, d, o, nullptr, static_cast<cudaStream_t>(stream), 0) == cudaSuccess
+               ? SAGE_OK
+               : SAGE_ERR_CUDA;
+}
+
+sage_status_t sage_debug_pv_accumulate_f16acc(const uint8_t *p, const uint8_t *vt, int n_tiles, int d,
+                                              uint32_t *o_raw, void *stream) {
+    if (!p || !vt || !o_raw || n_tiles < 1) return SAGE_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
+    if (!aligned16(p) || !aligned16(vt) || !aligned16(o_raw)) return SAGE_ERR_UNSUPPORTED;
+    return launch_debug_pv(p, vt, n_tiles, d, reinterpret_cast<float *>(o_raw), nullptr,
+                           static_cast<cudaStream_t>(stream), 1) == cudaSuccess
+               ? SAGE_OK
+               : SAGE_ERR_CUDA;
+}
+
+sage_status_t sage_debug_mma_rate(int kind, int n_iter, int n_ctas, void *status_block, void *stream) {
+    if (kind < 0 || kind > 3 || n_iter < 1 || n_iter > (1 << 20) || n_ctas < 1 || n_ctas > 4096 || !status_block)
+        return SAGE_ERR_INVALID_ARG;
+    return launch_debug_mma_rate(kind, n_iter, n_ctas, static_cast<int *>(status_block),
+                                 static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SAGE_OK
                : SAGE_ERR_CUDA;
 }

@@ -148,7 +148,10 @@ cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const
 cudaError_t launch_debug_qk_tile(const CUtensorMap &tq, const CUtensorMap &tk, int d, int q_row0, int k_row0,
                                  int32_t *s_out, int *status, cudaStream_t stream);
 cudaError_t launch_debug_pv(const uint8_t *p, const uint8_t *vt, int n_tiles, int d, float *o, int *status,
-                            cudaStream_t stream);
+                            cudaStream_t stream, int acc_f16);
+// n_ctas CTAs each issue n_iter tcgen05.mma of one kind (M = 128, N = 256) from
+// shared memory into one tensor-memory accumulator; see sage_debug_mma_rate.
+cudaError_t launch_debug_mma_rate(int kind, int n_iter, int n_ctas, int *status, cudaStream_t stream);
 cudaError_t launch_zero_output(void *o, size_t bytes, cudaStream_t stream);
 
 }  // namespace sage
