@@ -73,6 +73,8 @@ def _load():
             lib.oracle_int8_code.restype = ctypes.c_int8
             lib.oracle_int8_scale.argtypes = [ctypes.c_float]
             lib.oracle_int8_scale.restype = ctypes.c_float
+            lib.oracle_f16_round.argtypes = [ctypes.c_float]
+            lib.oracle_f16_round.restype = ctypes.c_double
             lib.oracle_prepass.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 15
             lib.oracle_prepass.restype = ctypes.c_int
             lib.oracle_attn.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 9 + [ctypes.c_int, P, P, P]
@@ -141,6 +143,19 @@ def _cfg(n_q, n_kv, d, g_q, g_k, smooth_q, smooth_k, quant, p_range, v_range, sm
     qqk, qp, qv = quant
     return _Cfg(n_q, n_kv, d, g_q, g_k, int(smooth_q), int(smooth_k), int(qqk), int(qp), int(qv),
                 float(p_range), float(v_range), float(sm_scale), int(causal))
+
+
+# quant = (QK, P, V): 1 = the method's INT8 / E4M3 / E4M3, 0 = exact.  PV_FP16 is the
+# "qk_int8_pv_fp16" mode of the SageAttention deployment guide: P~ and V rounded to
+# IEEE fp16 (P unscaled, V without per-channel scale), the PV product in fp16 x fp16.
+PV_FP8 = (1, 1, 1)
+PV_FP16 = (1, 2, 2)
+
+
+def f16_round(x):
+    """IEEE fp16 rounding (ties to even) of fp32 values, as fp64 (the oracle's codec)."""
+    lib = _load()
+    return np.array([lib.oracle_f16_round(float(v)) for v in np.asarray(x, np.float32).ravel()]).reshape(np.shape(x))
 
 
 def prepass_head(q, k, v, *, g_q=32, g_k=16, smooth_q=True, smooth_k=True,

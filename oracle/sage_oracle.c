@@ -61,8 +61,8 @@ typedef struct {
     int g_q, g_k;         /* INT8 group sizes (rows of a Q block, keys of a KV tile) */
     int smooth_q, smooth_k;
     int quant_qk;         /* 1: INT8 codes as in the method; 0: exact (identity) */
-    int quant_p;          /* 1: E4M3 P; 0: exact P~ * Pr                          */
-    int quant_v;          /* 1: E4M3 V; 0: exact V / delta_V                      */
+    int quant_p;          /* 1: E4M3 P; 0: exact P~ * Pr; 2: FP16 P~ (no Pr scale)  */
+    int quant_v;          /* 1: E4M3 V; 0: exact V / delta_V; 2: FP16 V (no scale)  */
     double p_range, v_range;
     double sm_scale;
     int causal;           /* bottom-right aligned: key j visible to row i iff j <= i + n_kv - n_q */
@@ -111,6 +111,25 @@ double oracle_e4m3_to_f64(uint8_t c)
     if (e == 0) v = ldexp((double)m, -9);
     else v = ldexp(1.0 + m / 8.0, e - 7);
     return s ? -v : v;
+}
+
+/* IEEE binary16 rounding of an fp32 value, returned as its exact fp64 value:
+ * 11 significant bits for |x| >= 2^-14, a fixed spacing of 2^-24 below (the
+ * subnormals), round to nearest with ties to even, and +-inf from 65520 on (the
+ * halfway point above the largest finite value 65504).  Used by the FP16 P / V mode
+ * (the "qk_int8_pv_fp16" quantization mode of the SageAttention deployment guide). */
+double oracle_f16_round(float xf)
+{
+    double x = (double)xf;
+    if (x == 0.0 || isnan(x)) return x;
+    double a = fabs(x);
+    if (a >= 65520.0) return copysign(INFINITY, x);
+    int e;
+    frexp(a, &e);                 /* a in [2^(e-1), 2^e) */
+    int q = e - 11;               /* spacing of 11 significant bits */
+    if (q < -24) q = -24;         /* subnormal spacing */
+    double step = ldexp(1.0, q);
+    return copysign(nearbyint(a / step) * step, x);
 }
 
 /* INT8 code of an fp32 value for a given fp32 scale: round half to even of the
@@ -253,12 +272,15 @@ int oracle_prepass(const oracle_cfg_t *cfg, const double *q, const double *k, co
             float a = fabsf((float)v[(size_t)j * d + c]);
             if (a > amax) amax = a;
         }
-        dv[c] = (amax == 0.0f) ? 1.0f : amax / vr;
+        dv[c] = (amax == 0.0f || cfg->quant_v == 2) ? 1.0f : amax / vr;
     }
     for (int j = 0; j < nk; ++j)
         for (int c = 0; c < d; ++c) {
             size_t o = (size_t)j * d + c;
-            if (cfg->quant_v) {
+            if (cfg->quant_v == 2) {  /* FP16 V, unscaled */
+                v_code[o] = 0;
+                v_hat[o] = oracle_f16_round((float)v[o]);
+            } else if (cfg->quant_v) {
                 float qv = (float)v[o] / dv[c];
                 v_code[o] = oracle_e4m3_from_f32(qv);
                 v_hat[o] = oracle_e4m3_to_f64(v_code[o]);
@@ -279,7 +301,8 @@ int oracle_prepass(const oracle_cfg_t *cfg, const double *q, const double *k, co
 /*   tiled online softmax over 128-key tiles in increasing j ([online-softmax]):*/
 /*     m' = max(m, max_j x), alpha = exp(m - m'), P~ = exp(x - m'),            */
 /*     l  = alpha l + sum P~,  acc = alpha acc + sum_j P8_j v_hat[j],          */
-/*     P8 = E4M3(fp32(P~ Pr)) (or P~ Pr exactly when quant_p = 0);            */
+/*     P8 = E4M3(fp32(P~ Pr)) (or P~ Pr exactly when quant_p = 0; FP16(fp32(P~)) */
+/*     with Pr = 1 when quant_p = 2);                                          */
 /*   O[i,c] = acc[c] / Pr * dv[c] / l   (0 for a row that sees no key).       */
 /* With integer codes the dot product q_hat . k_hat is a sum of at most d     */
 /* products of magnitude <= 127^2, exact in fp64, i.e. the exact integer      */
@@ -294,7 +317,7 @@ int oracle_attn(const oracle_cfg_t *cfg, const float *qbar, const double *q_hat,
     const int nq = cfg->n_q, nk = cfg->n_kv, d = cfg->d;
     const int tq = ceil_div(nq, ORACLE_TILE), tk = ceil_div(nk, ORACLE_TILE);
     const long off = (long)nk - (long)nq;
-    const double pr = cfg->p_range;
+    const double pr = (cfg->quant_p == 2) ? 1.0 : cfg->p_range;  /* FP16 P~ is not scaled */
     for (int b = 0; b < n_qblocks; ++b)
         if (qblocks[b] < 0 || qblocks[b] >= tq) return 1;
 
@@ -340,7 +363,8 @@ int oracle_attn(const oracle_cfg_t *cfg, const float *qbar, const double *q_hat,
                     if (!vis[j - j0]) continue;
                     double p = exp(x[j - j0] - mn);
                     l += p;
-                    double p8 = cfg->quant_p ? oracle_e4m3_to_f64(oracle_e4m3_from_f32((float)(p * pr))) : p * pr;
+                    double p8 = cfg->quant_p == 2 ? oracle_f16_round((float)p)
+                                : cfg->quant_p ? oracle_e4m3_to_f64(oracle_e4m3_from_f32((float)(p * pr))) : p * pr;
                     if (p8 == 0.0) continue;
                     for (int c = 0; c < d; ++c) acc[c] += p8 * v_hat[(size_t)j * d + c];
                 }

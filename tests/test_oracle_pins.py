@@ -513,3 +513,57 @@ def test_varlen_unquantized_equals_block_diagonal_masked_sdpa(causal):
     seen = mask.any(1)   # rows with no visible key: SDPA gives NaN, the method 0
     assert np.max(np.abs(o[seen] - ref[seen])) < 1e-12
     assert np.all(o[~seen] == 0)
+
+
+# ---------------------------------------------------------------------------
+# FP16 P / V mode ("qk_int8_pv_fp16")
+# ---------------------------------------------------------------------------
+def test_f16_codec_matches_numpy():
+    """The oracle's fp16 rounding against numpy's float32 -> float16 conversion (IEEE,
+    ties to even) on random values spanning the subnormals, the normals, the largest
+    finite value and overflow."""
+    rng = np.random.default_rng(3)
+    x = np.concatenate([
+        rng.standard_normal(4000).astype(np.float32) * np.float32(2.0) ** rng.integers(-30, 17, 4000),
+        np.float32([0.0, -0.0, 65504.0, 65519.0, 65520.0, -65520.0, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26,
+                    2.0 ** -14, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11])]).astype(np.float32)
+    got = oracle.f16_round(x)
+    with np.errstate(over="ignore"):   # 65520 and beyond overflow to inf, as IEEE rounding does
+        ref = x.astype(np.float16).astype(np.float64)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_pv_fp16_with_exact_qk_equals_attention_with_fp16_operands(causal):
+    """With exact QK^T, one key tile (so the online softmax is the two-pass one) and
+    FP16 P / V, the oracle equals softmax attention whose P~ = exp(x - m) and V are
+    rounded to fp16 (numpy's float16) before the PV product, divided by the unrounded
+    row sum."""
+    nq, nk, d = 200, 128, 64
+    q, k, v = _rand_head(nq, nk, d, seed=404, kbias=2.0, outliers=False)
+    pre = oracle.prepass_head(q, k, v, quant=(0, 2, 2))
+    o = oracle.attn_head(pre, causal=causal)
+    x = (q @ k.T) / 8.0
+    if causal:
+        x = np.where(np.arange(nk)[None, :] <= np.arange(nq)[:, None] + (nk - nq), x, -np.inf)
+    seen = np.isfinite(x).any(1)
+    m = np.where(seen, x.max(1), 0.0)[:, None]
+    p = np.exp(x - m)
+    p16 = p.astype(np.float32).astype(np.float16).astype(np.float64)
+    v16 = v.astype(np.float32).astype(np.float16).astype(np.float64)
+    ref = np.zeros_like(o)
+    ref[seen] = (p16[seen] @ v16) / p[seen].sum(1, keepdims=True)
+    assert np.max(np.abs(o - ref)) < 1e-12
+    assert np.all(pre["dv"] == 1.0)
+    assert np.any(p16 != p)   # the rounding acted
+
+
+def test_pv_fp16_more_accurate_than_fp8():
+    """The FP16 P / V mode is closer to full-precision attention than FP8 P / V."""
+    q, k, v = wl.generate(wl.TINY)
+    qn, kn, vn = (x.double().numpy() for x in (q, k, v))
+    ref = oracle.reference_attention(qn, kn, vn)
+    o8 = oracle.sage_attention(qn, kn, vn, quant=oracle.PV_FP8)
+    o16 = oracle.sage_attention(qn, kn, vn, quant=oracle.PV_FP16)
+    e8, e16 = np.abs(o8 - ref).max(), np.abs(o16 - ref).max()
+    assert e16 < e8
