@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--pv", default="fp8", choices=["fp8", "fp16"],
+                    help="PV precision: fp8 (the method's default) or fp16 (the qk_int8_pv_fp16 mode)")
     ap.add_argument("--mma-rates", action="store_true",
                     help="print the tensor-core rate of each tcgen05.mma form (diagnostic) and exit")
     return ap.parse_args()
@@ -267,13 +269,14 @@ def main():
     q_cpu, k_cpu, v_cpu = wl.generate(wr)
     q, k, v = q_cpu.to(dev), k_cpu.to(dev), v_cpu.to(dev)
     B, H, nq, nk, d = w.B, w.H, w.N_q, w.N_kv, w.d
-    ws = sage.make_workspace(B, H, nq, nk, d, device=dev, H_kv=w.Hk)
+    pv16 = args.pv == "fp16"
+    ws = sage.make_workspace(B, H, nq, nk, d, device=dev, H_kv=w.Hk, pv_fp16=pv16)
     out = torch.empty_like(q)
-    mode = sage.QuantMode.make()
+    mode = sage.QuantMode.make(pv=args.pv)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        sage.attn_fwd(q, k, v, causal=w.causal, out=out, workspace=ws)
+        sage.attn_fwd(q, k, v, causal=w.causal, out=out, workspace=ws, pv=args.pv)
 
     def attn_only():
         sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode, out=out)
@@ -352,7 +355,7 @@ def main():
                 stream.wait_event(ev_in[i])
                 if i >= 2:
                     stream.wait_event(ev_out[i - 2])     # and its output has been copied out
-                sage.attn_fwd(qd, kd, vd, causal=w.causal, out=od, workspace=ws, stream=stream)
+                sage.attn_fwd(qd, kd, vd, causal=w.causal, out=od, workspace=ws, stream=stream, pv=args.pv)
                 ev_comp[i].record(stream)
                 s_out.wait_event(ev_comp[i])
                 with torch.cuda.stream(s_out):
@@ -384,6 +387,11 @@ def main():
 
     bf16_burst, bf16_sust, peak_src = measured_peaks()
     peak = 2.0 * bf16_burst   # dense INT8 / FP8 = 2x dense BF16 (nominal 4.5 vs 2.25 PFLOP/s)
+    peak_note = "%s bf16 burst %.1f x 2 (dense int8/fp8 = 2x bf16)" % (peak_src, bf16_burst)
+    if pv16:  # half the work at the INT8 rate, half at the FP16 rate: the harmonic mean
+        peak = 2.0 / (1.0 / (2.0 * bf16_burst) + 1.0 / bf16_burst)
+        peak_note = ("%s bf16 burst %.1f: INT8 QK at 2x, FP16 PV at 1x, equal work: harmonic mean"
+                     % (peak_src, bf16_burst))
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         ops_s, secs, desc, threads = oracle_sample(w, args.cpu_seconds)
@@ -391,16 +399,17 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8+e4m3", "data": "synthetic",
+        "vs_baseline": None, "dtype": "int8+fp16" if pv16 else "int8+e4m3", "data": "synthetic",
         "config": dict(w.describe(), parallelism="heads sharded: each of %d rank(s) runs the full workload" % world,
                        l2="inputs (%.0f MiB) larger than L2 (126 MB); no flush" % ((2 * q.numel() + 2 * k.numel()) * 2 / 2 ** 20),
-                       granularity="per_threadgroup (g_q=32, g_k=16)", pr=448, vr=448),
+                       granularity="per_threadgroup (g_q=32, g_k=16)",
+                       **({"pv": "fp16 (qk_int8_pv_fp16)"} if pv16 else {"pv": "fp8", "pr": 448, "vr": 448})),
         "attn_kernel_tops": attn_tops, "attn_kernel_ms": attn_avg_ms, "prepass_ms": pre_avg_ms,
         "step_call": "sage_attn_fwd (pre-pass + dS + attention); prepass_ms = ms_per_step - attn_kernel_ms",
         "attn_frac_of_spec_4500": attn_tops / SPEC_INT8_TOPS,
         "roofline": {"bound": "tensor", "achieved": attn_tops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": attn_tops / peak, "traffic": recorded_traffic(w.name),
-                     "peak_source": "%s bf16 burst %.1f x 2 (dense int8/fp8 = 2x bf16)" % (peak_src, bf16_burst),
+                     "frac": attn_tops / peak, "traffic": None if pv16 else recorded_traffic(w.name),
+                     "peak_source": peak_note,
                      "kernel": "attn_fwd_kernel<%d>" % d},
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         "gpu_launches": args.steps * LAUNCHES_PER_STEP,

@@ -96,12 +96,22 @@ typedef struct {
     int32_t smooth_k;  /* 1: subtract per-head K mean                           */
     float p_range;     /* Pr, (0, 448]; 448 = full E4M3 range (default)         */
     float v_range;     /* Vr, (0, 448]; 448 (SageAttention2 default)            */
+    int32_t pv_fp16;   /* 0: E4M3 P (x Pr) and per-channel E4M3 V, FP8 PV (default);
+                        * 1: FP16 P~ (unscaled) and FP16 V (no per-channel scale),
+                        *    FP16 PV with FP32 accumulation: the deployment guide's
+                        *    "qk_int8_pv_fp16" high-fidelity mode; p_range and v_range
+                        *    are unused.  The workspace of this mode is larger
+                        *    (sage_workspace_bytes_mode). */
 } sage_quant_mode_t;
-/* A NULL mode pointer means {SAGE_QK_PER_THREADGROUP, 1, 1, 448, 448}. */
+/* A NULL mode pointer means {SAGE_QK_PER_THREADGROUP, 1, 1, 448, 448, 0}. */
 
 /* Bytes of workspace for one problem size (any dtype/layout).  0 on bad sizes. */
 SAGE_API size_t sage_workspace_bytes(int B, int H, int n_q, int n_kv, int d);
 SAGE_API size_t sage_workspace_bytes_gqa(int B, int H, int H_kv, int n_q, int n_kv, int d);
+/* Bytes of workspace for a mode (NULL = default): the FP16 P / V mode needs 2 bytes per
+ * V element instead of 1; every other mode field leaves the size unchanged. */
+SAGE_API size_t sage_workspace_bytes_mode(int B, int H, int H_kv, int n_q, int n_kv, int d,
+                                          const sage_quant_mode_t *mode);
 
 /* Steps 1-3 (and the dS bias) for Q and K into the workspace.
  * q: [B,H,n_q,d] or [B,n_q,H,d]; k: [B,H,n_kv,d] or [B,n_kv,H,d]. */
@@ -212,7 +222,8 @@ SAGE_API sage_status_t sage_get_device_status(void *workspace, void *stream, int
  * with Tq = ceil(n_q/128), Tk = ceil(n_kv/128), nq_pad = 128 Tq, nk_pad = 128 Tk:
  *   SAGE_WS_Q8    int8  [BH][nq_pad][d]          Q codes (pad rows 0)
  *   SAGE_WS_K8    int8  [BHk][nk_pad][d]         K codes (pad rows 0)
- *   SAGE_WS_VT8   e4m3  [BHk][d][nk_pad]         V codes, transposed (pad 0)
+ *   SAGE_WS_VT8   e4m3  [BHk][d][nk_pad]         V codes, transposed (pad 0); in the
+ *                                                FP16 P / V mode fp16 V, same shape
  *   SAGE_WS_DQ    fp32  [BH][nq_pad]             delta_Q of each row's group
  *   SAGE_WS_DK    fp32  [BHk][nk_pad/16]         delta_K of each 16-key run
  *   SAGE_WS_DV    fp32  [BHk][d]                 delta_V per channel
@@ -244,6 +255,8 @@ enum {
 /* Byte offset of view `which` inside the workspace, or -1 for bad arguments. */
 SAGE_API int64_t sage_workspace_offset(int B, int H, int n_q, int n_kv, int d, int which);
 SAGE_API int64_t sage_workspace_offset_gqa(int B, int H, int H_kv, int n_q, int n_kv, int d, int which);
+SAGE_API int64_t sage_workspace_offset_mode(int B, int H, int H_kv, int n_q, int n_kv, int d,
+                                            const sage_quant_mode_t *mode, int which);
 
 /* ---- diagnostics (no counterpart on the pages' API) ---------------------------
  * INT32 scores of one (bh, Q tile, KV tile) straight from tensor memory, computed

@@ -49,12 +49,17 @@ class SageError(RuntimeError):
 class QuantMode(ctypes.Structure):
     """Mirror of sage_quant_mode_t."""
     _fields_ = [("gran", ctypes.c_int32), ("smooth_q", ctypes.c_int32), ("smooth_k", ctypes.c_int32),
-                ("p_range", ctypes.c_float), ("v_range", ctypes.c_float)]
+                ("p_range", ctypes.c_float), ("v_range", ctypes.c_float), ("pv_fp16", ctypes.c_int32)]
 
     @classmethod
-    def make(cls, granularity="per_threadgroup", smooth_q=True, smooth_k=True, p_range=448.0, v_range=448.0):
+    def make(cls, granularity="per_threadgroup", smooth_q=True, smooth_k=True, p_range=448.0, v_range=448.0,
+             pv="fp8"):
+        """pv: "fp8" (E4M3 P and per-channel E4M3 V, the default) or "fp16" (FP16 P~ and V,
+        the "qk_int8_pv_fp16" high-fidelity mode)."""
         g = GRANULARITIES[granularity] if isinstance(granularity, str) else int(granularity)
-        return cls(g, int(bool(smooth_q)), int(bool(smooth_k)), float(p_range), float(v_range))
+        if pv not in ("fp8", "fp16"):
+            raise ValueError("pv must be 'fp8' or 'fp16'")
+        return cls(g, int(bool(smooth_q)), int(bool(smooth_k)), float(p_range), float(v_range), int(pv == "fp16"))
 
 
 def library_path() -> str:
@@ -83,6 +88,10 @@ def load_library():
         lib.sage_attn_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, F, QM, P, S, P]
         lib.sage_workspace_bytes_gqa.argtypes = [I] * 6
         lib.sage_workspace_bytes_gqa.restype = S
+        lib.sage_workspace_bytes_mode.argtypes = [I] * 6 + [QM]
+        lib.sage_workspace_bytes_mode.restype = S
+        lib.sage_workspace_offset_mode.argtypes = [I] * 6 + [QM, I]
+        lib.sage_workspace_offset_mode.restype = ctypes.c_int64
         lib.sage_workspace_offset_gqa.argtypes = [I] * 7
         lib.sage_workspace_offset_gqa.restype = ctypes.c_int64
         lib.sage_quant_qk_gqa.argtypes = [P, P, I, I, I, I, I, I, I, I, QM, P, S, P]
@@ -162,22 +171,24 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def workspace_bytes(B, H, n_q, n_kv, d, H_kv=None) -> int:
+def workspace_bytes(B, H, n_q, n_kv, d, H_kv=None, pv_fp16=False) -> int:
     H_kv = H if H_kv is None else H_kv
-    return int(load_library().sage_workspace_bytes_gqa(B, H, H_kv, n_q, n_kv, d))
+    mode = QuantMode.make(pv="fp16" if pv_fp16 else "fp8")
+    return int(load_library().sage_workspace_bytes_mode(B, H, H_kv, n_q, n_kv, d, ctypes.byref(mode)))
 
 
 class Workspace:
     """Caller-owned device workspace: a zeroed uint8 tensor with a 1024-byte aligned window.
 
     dims = (B, H, n_q, n_kv, d) with H query heads; H_kv key/value heads (H_kv = H
-    for multi-head attention)."""
+    for multi-head attention); pv_fp16: laid out for the FP16 P / V mode."""
 
-    def __init__(self, B, H, n_q, n_kv, d, device=None, H_kv=None):
+    def __init__(self, B, H, n_q, n_kv, d, device=None, H_kv=None, pv_fp16=False):
         torch = _torch()
         self.dims = (int(B), int(H), int(n_q), int(n_kv), int(d))
         self.H_kv = int(H if H_kv is None else H_kv)
-        self.nbytes = workspace_bytes(*self.dims, H_kv=self.H_kv)
+        self.pv_fp16 = bool(pv_fp16)
+        self.nbytes = workspace_bytes(*self.dims, H_kv=self.H_kv, pv_fp16=self.pv_fp16)
         if self.nbytes == 0:
             raise SageError(SAGE_ERR_UNSUPPORTED, "sage_workspace_bytes")
         self.tensor = torch.zeros(self.nbytes + WS_ALIGN, dtype=torch.uint8, device=device or "cuda")
@@ -185,9 +196,10 @@ class Workspace:
         self.offset = (-base) % WS_ALIGN
         self.ptr = base + self.offset
 
-    def fits(self, B, H, n_q, n_kv, d, H_kv=None) -> bool:
+    def fits(self, B, H, n_q, n_kv, d, H_kv=None, pv_fp16=False) -> bool:
         H_kv = H if H_kv is None else H_kv
-        return self.dims == (int(B), int(H), int(n_q), int(n_kv), int(d)) and self.H_kv == int(H_kv)
+        return (self.dims == (int(B), int(H), int(n_q), int(n_kv), int(d)) and self.H_kv == int(H_kv)
+                and self.pv_fp16 == bool(pv_fp16))
 
     def lse(self):
         """Row log-sum-exp [B, H, n_q] (fp32, natural log) of the last attention call on
@@ -200,11 +212,13 @@ class Workspace:
         head for q8, dq, qbar, ds; per key/value head for k8, vt8, dk, dv, kbar."""
         torch = _torch()
         B, H, n_q, n_kv, d = self.dims
-        off = int(load_library().sage_workspace_offset_gqa(B, H, self.H_kv, n_q, n_kv, d, WS_VIEWS[which]))
+        mode = QuantMode.make(pv="fp16" if self.pv_fp16 else "fp8")
+        off = int(load_library().sage_workspace_offset_mode(B, H, self.H_kv, n_q, n_kv, d, ctypes.byref(mode),
+                                                            WS_VIEWS[which]))
         BH, BHk, Tq = B * H, B * self.H_kv, -(-n_q // 128)
         nq_pad, nk_pad = Tq * 128, -(-n_kv // 128) * 128
         shapes = {"q8": ((BH, nq_pad, d), torch.int8), "k8": ((BHk, nk_pad, d), torch.int8),
-                  "vt8": ((BHk, d, nk_pad), torch.uint8), "dq": ((BH, nq_pad), torch.float32),
+                  "vt8": ((BHk, d, nk_pad), torch.float16 if self.pv_fp16 else torch.uint8), "dq": ((BH, nq_pad), torch.float32),
                   "dk": ((BHk, nk_pad // 16), torch.float32), "dv": ((BHk, d), torch.float32),
                   "qbar": ((BH, Tq, d), torch.float32), "kbar": ((BHk, d), torch.float32),
                   "ds": ((BH, Tq, nk_pad), torch.float32), "qs_kbar": ((BH, nq_pad), torch.float32),
@@ -215,23 +229,23 @@ class Workspace:
         return self.tensor[start:start + n].view(dt).view(shp)
 
 
-def make_workspace(B, H, n_q, n_kv, d, device=None, H_kv=None) -> Workspace:
-    return Workspace(B, H, n_q, n_kv, d, device, H_kv=H_kv)
+def make_workspace(B, H, n_q, n_kv, d, device=None, H_kv=None, pv_fp16=False) -> Workspace:
+    return Workspace(B, H, n_q, n_kv, d, device, H_kv=H_kv, pv_fp16=pv_fp16)
 
 
-def _ws_for(ws, B, H, H_kv, n_q, n_kv, d, device):
+def _ws_for(ws, B, H, H_kv, n_q, n_kv, d, device, pv_fp16=False):
     if ws is None:
-        return Workspace(B, H, n_q, n_kv, d, device, H_kv=H_kv)
-    if not ws.fits(B, H, n_q, n_kv, d, H_kv):
-        raise ValueError("workspace was made for %s (H_kv %d), not %s (H_kv %d)"
-                         % (ws.dims, ws.H_kv, (B, H, n_q, n_kv, d), H_kv))
+        return Workspace(B, H, n_q, n_kv, d, device, H_kv=H_kv, pv_fp16=pv_fp16)
+    if not ws.fits(B, H, n_q, n_kv, d, H_kv, pv_fp16):
+        raise ValueError("workspace was made for %s (H_kv %d, pv_fp16 %s), not %s (H_kv %d, pv_fp16 %s)"
+                         % (ws.dims, ws.H_kv, ws.pv_fp16, (B, H, n_q, n_kv, d), H_kv, bool(pv_fp16)))
     return ws
 
 
 def quant_qk(q, k, *, layout="HND", mode=None, workspace=None, stream=None) -> Workspace:
     B, H, H_kv, n_q, n_kv, d = _shape(q, k, layout)
-    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, q.device)
     mode = mode or QuantMode.make()
+    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, q.device, mode.pv_fp16)
     _check(load_library().sage_quant_qk_gqa(_ptr(q), _ptr(k), _dtype_code(q), _LAYOUTS[layout], B, H, H_kv, n_q,
                                             n_kv, d, ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
                                             _stream_handle(stream)), "sage_quant_qk_gqa")
@@ -248,8 +262,8 @@ def quant_v(v, *, n_q, H=None, layout="HND", mode=None, workspace=None, stream=N
     if H is None:
         H = workspace.dims[1] if workspace is not None else H_kv
     B, H, H_kv, n_kv, d = int(B), int(H), int(H_kv), int(n_kv), int(d)
-    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, v.device)
     mode = mode or QuantMode.make()
+    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, v.device, mode.pv_fp16)
     _check(load_library().sage_quant_v_gqa(_ptr(v), _dtype_code(v), _LAYOUTS[layout], B, H, H_kv, n_q, n_kv, d,
                                            ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
                                            _stream_handle(stream)), "sage_quant_v_gqa")
@@ -266,6 +280,8 @@ def attn_fwd_prequant(workspace: Workspace, *, dtype, layout="HND", causal=False
         shape = (B, H, n_q, d) if layout == "HND" else (B, n_q, H, d)
         out = torch.empty(shape, dtype=dtype, device=workspace.tensor.device)
     mode = mode or QuantMode.make()
+    if bool(mode.pv_fp16) != workspace.pv_fp16:
+        raise ValueError("the mode's pv setting does not match the workspace")
     _check(load_library().sage_attn_fwd_prequant_gqa(_ptr(out), _dtype_code(out), _LAYOUTS[layout], B, H,
                                                      workspace.H_kv, n_q, n_kv, d, int(bool(causal)),
                                                      float(sm_scale or 0.0), ctypes.byref(mode),
@@ -275,8 +291,8 @@ def attn_fwd_prequant(workspace: Workspace, *, dtype, layout="HND", causal=False
 
 
 def attn_fwd(q, k, v, *, causal=False, sm_scale=None, layout="HND", granularity="per_threadgroup",
-             smooth_q=True, smooth_k=True, p_range=448.0, v_range=448.0, out=None, workspace=None, stream=None,
-             return_lse=False):
+             smooth_q=True, smooth_k=True, p_range=448.0, v_range=448.0, pv="fp8", out=None, workspace=None,
+             stream=None, return_lse=False):
     """O = quantized attention of q, k, v (pre-pass + fused kernel, enqueued on the current stream).
 
     k and v may have fewer heads than q (grouped-query attention): query head h
@@ -288,10 +304,10 @@ def attn_fwd(q, k, v, *, causal=False, sm_scale=None, layout="HND", granularity=
         raise ValueError("v shape %s must equal k shape %s" % (tuple(v.shape), tuple(k.shape)))
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share a dtype")
-    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, q.device)
+    mode = QuantMode.make(granularity, smooth_q, smooth_k, p_range, v_range, pv)
+    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, q.device, mode.pv_fp16)
     if out is None:
         out = torch.empty_like(q)
-    mode = QuantMode.make(granularity, smooth_q, smooth_k, p_range, v_range)
     _check(load_library().sage_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q),
                                             _LAYOUTS[layout], B, H, H_kv, n_q, n_kv, d, int(bool(causal)),
                                             float(sm_scale or 0.0), ctypes.byref(mode), ctypes.c_void_p(ws.ptr),
@@ -301,7 +317,7 @@ def attn_fwd(q, k, v, *, causal=False, sm_scale=None, layout="HND", granularity=
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, max_seqlen_q=None, max_seqlen_kv=None, causal=False,
                     sm_scale=None, granularity="per_threadgroup", smooth_q=True, smooth_k=True, p_range=448.0,
-                    v_range=448.0, out=None, workspace=None, stream=None, return_lse=False):
+                    v_range=448.0, pv="fp8", out=None, workspace=None, stream=None, return_lse=False):
     """Quantized attention of a packed batch of variable-length sequences.
 
     q: [total_q, H, d]; k, v: [total_kv, H_kv, d] (H_kv divides H); cu_seqlens_q,
@@ -328,10 +344,10 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, max_seqlen_q=None, 
         max_seqlen_kv = int((cu_seqlens_kv[1:] - cu_seqlens_kv[:-1]).max().item()) if B > 0 else 0
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share a dtype")
-    ws = _ws_for(workspace, B, H, H_kv, max_seqlen_q, max_seqlen_kv, d, q.device)
+    mode = QuantMode.make(granularity, smooth_q, smooth_k, p_range, v_range, pv)
+    ws = _ws_for(workspace, B, H, H_kv, max_seqlen_q, max_seqlen_kv, d, q.device, mode.pv_fp16)
     if out is None:
         out = torch.empty_like(q)
-    mode = QuantMode.make(granularity, smooth_q, smooth_k, p_range, v_range)
     _check(load_library().sage_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q),
                                                _ptr(cu_seqlens_q), _ptr(cu_seqlens_kv), B, H, H_kv, total_q, total_kv,
                                                int(max_seqlen_q), int(max_seqlen_kv), d, int(bool(causal)),

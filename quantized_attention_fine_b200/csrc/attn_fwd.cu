@@ -64,19 +64,26 @@ enum { kSiteQ = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteS = 4, kSiteP = 5, kSiteO
 // rings: a K slot is free once QK^T has read it and both tiles' warps have
 // dequantized with its dS / delta_K, long before PV is done with the V^T tile of
 // the same key tile, so the K ring can run further ahead.
-template <int D>
+// PV16 (the FP16 P / V mode): P~ and V^T are fp16, two 64-key 128-byte swizzle spans
+// per row; the larger tiles leave room for one P buffer per Q tile (a tile's
+// warpgroup writes P(i) once PV(i - 1) has read it) and shorter rings at d = 128.
+template <int D, bool PV16>
 struct AttnCfg {
-    static constexpr int kKStages = 4;
-    static constexpr int kVStages = (D == 128) ? 3 : 4;
+    static constexpr int kKStages = (PV16 && D == 128) ? 3 : 4;
+    static constexpr int kVStages = PV16 ? (D == 128 ? 2 : 3) : (D == 128 ? 3 : 4);
+    static constexpr int kPBufs = PV16 ? 1 : 2;                     // P buffers per Q tile
+    static constexpr int kPBytes = kTile * kTile * (PV16 ? 2 : 1);  // one P tile
+    static constexpr int kVBytes = D * kTile * (PV16 ? 2 : 1);      // one V^T tile
 };
 
-template <int D>
+template <int D, bool PV16>
 struct __align__(1024) AttnSmem {
-    static constexpr int KS = AttnCfg<D>::kKStages, VS = AttnCfg<D>::kVStages;
+    static constexpr int KS = AttnCfg<D, PV16>::kKStages, VS = AttnCfg<D, PV16>::kVStages;
     uint8_t q[2][kTile * D];
     uint8_t k[KS][kTile * D];
-    uint8_t v[VS][D * kTile];
-    uint8_t p[2][2][kTile * kTile];  // [Q tile][key tile parity], keys in storage order
+    uint8_t v[VS][AttnCfg<D, PV16>::kVBytes];
+    // [Q tile][key tile parity (FP8) or 0 (FP16)], keys in storage order
+    uint8_t p[2][AttnCfg<D, PV16>::kPBufs][AttnCfg<D, PV16>::kPBytes];
     float ds[KS][2][kTile];          // keys in storage order
     float dk[KS][kTile / kKeyRun];
     uint64_t bar_q, bar_kfull[KS], bar_kempty[KS], bar_vfull[VS], bar_vempty[VS];
@@ -180,6 +187,24 @@ __device__ __forceinline__ void exp16(const uint32_t (&w)[16], float2 c2, float2
     }
 }
 
+// The same exponentials kept as fp16 (round to nearest even, no Pr scale: bias is
+// -m c), two per word, for the FP16 P / V mode.
+__device__ __forceinline__ void exp16_f16(const uint32_t (&w)[16], float2 c2, float2 b2, float2 &acc0,
+                                          float2 &acc1, uint32_t (&ph)[8]) {
+#pragma unroll
+    for (int j = 0; j < 16; j += 4) {
+        const float2 e01 = __ffma2_rn(make_float2(__uint_as_float(w[j]), __uint_as_float(w[j + 1])), c2, b2);
+        const float2 e23 = __ffma2_rn(make_float2(__uint_as_float(w[j + 2]), __uint_as_float(w[j + 3])), c2, b2);
+        const float2 p01 = make_float2(ex2_approx(e01.x), ex2_approx(e01.y));
+        const float2 p23 = make_float2(ex2_approx(e23.x), ex2_approx(e23.y));
+        acc0 = __fadd2_rn(acc0, p01);
+        acc1 = __fadd2_rn(acc1, p23);
+        const __half2 h01 = __floats2half2_rn(p01.x, p01.y), h23 = __floats2half2_rn(p23.x, p23.y);
+        ph[j / 2] = *reinterpret_cast<const uint32_t *>(&h01);
+        ph[j / 2 + 1] = *reinterpret_cast<const uint32_t *>(&h23);
+    }
+}
+
 // Key tile `kt` has invisible keys in this row block: the key-count tail, or the
 // causal diagonal (key j visible to row i iff j <= i + off).
 __device__ __forceinline__ bool tile_masked(int kt, int t, int n_kv, int off, int causal) {
@@ -215,11 +240,11 @@ __device__ __forceinline__ uint32_t pack16x2(float lo, float hi, int out_bf16) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-template <int D>
-__device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &p, uint32_t tmem, int X, int t,
+template <int D, bool PV16>
+__device__ __forceinline__ void softmax_role(AttnSmem<D, PV16> &sm, const AttnParams &p, uint32_t tmem, int X, int t,
                                              int n_tiles, int bh, int64_t o_base, int n_q, int n_kv,
                                              volatile int *abort_flag) {
-    constexpr int KS = AttnCfg<D>::kKStages;
+    constexpr int KS = AttnCfg<D, PV16>::kKStages;
     const int w8 = (threadIdx.x >> 5) & 7;  // warp within the tile's eight
     const int quad = w8 & 3, half = w8 >> 2;
     const int lane = threadIdx.x & 31;
@@ -287,13 +312,27 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
         float mx[4];
         const float *dsn = sm.ds[sn][X] + pos0;
         const float *dkn = sm.dk[sn];
-        // P(it) goes to the buffer PV(it - 2) read; that PV was waited for before P(it - 1)
-        uint8_t *pbuf = sm.p[X][it & 1];
+        // FP8: P(it) goes to the buffer PV(it - 2) read; that PV was waited for before
+        // P(it - 1).  FP16: the one buffer PV(it - 1) reads; wait for that PV first.
+        uint8_t *pbuf = sm.p[X][PV16 ? 0 : (it & 1)];
+        if constexpr (PV16) {
+            if (it > 0 && !warp_wait(&sm.bar_o[X], (it - 1) & 1, abort_flag, p.status, kSiteO)) { ok = false; break; }
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            uint32_t pk[4];
-            exp16(sv[q], c2, b2, acc0, acc1, pk);
-            *reinterpret_cast<uint4 *>(pbuf + sw128_offset(r, par * 4 + q)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            if constexpr (PV16) {
+                // keys 16 q .. 16 q + 15 of this thread's 64-key span (its parity's half of
+                // the row): two 16-byte chunks of the span's 128-byte row
+                uint32_t ph[8];
+                exp16_f16(sv[q], c2, b2, acc0, acc1, ph);
+                uint8_t *span = pbuf + par * (kTile * 128);
+                *reinterpret_cast<uint4 *>(span + sw128_offset(r, 2 * q)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+                *reinterpret_cast<uint4 *>(span + sw128_offset(r, 2 * q + 1)) = make_uint4(ph[4], ph[5], ph[6], ph[7]);
+            } else {
+                uint32_t pk[4];
+                exp16(sv[q], c2, b2, acc0, acc1, pk);
+                *reinterpret_cast<uint4 *>(pbuf + sw128_offset(r, par * 4 + q)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
             tmem_ld16x64b_x16(s_tmem + q * 32, sv[q]);
             tmem_wait_ld_regs16(sv[q]);
             mx[q] = dequant16(sv[q], dq * dkn[2 * q], dq * dkn[2 * q + 1], dsn + 16 * q);
@@ -392,14 +431,15 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D> &sm, const AttnParams &
 // the dense lengths); without RT the kernel serves dense batches only and reads the
 // lengths straight from the parameters.  The two compile to different register
 // allocations: d = 128 dense runs faster without RT, d = 64 dense with it (measured).
-template <int D, bool RT>
+template <int D, bool RT, bool PV16>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
-    constexpr int KS = AttnCfg<D>::kKStages, VS = AttnCfg<D>::kVStages;
+    constexpr int KS = AttnCfg<D, PV16>::kKStages, VS = AttnCfg<D, PV16>::kVStages;
+    constexpr int kPBufs = AttnCfg<D, PV16>::kPBufs, kPBytes = AttnCfg<D, PV16>::kPBytes;
     extern __shared__ uint8_t smem_raw[];
-    AttnSmem<D> &sm =
-        *reinterpret_cast<AttnSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    AttnSmem<D, PV16> &sm =
+        *reinterpret_cast<AttnSmem<D, PV16> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // Work item: a pair of Q tiles of one head.  The CTAs are ordered in blocks of
@@ -507,15 +547,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (it >= VS && !mbar_wait(&sm.bar_vempty[s], ((it / VS) & 1) ^ 1, abort_flag, p.status, kSiteEmpty))
                     break;
                 issued = it + 1;
-                mbar_arrive_expect_tx(&sm.bar_vfull[s], kTile * D);
-                tma_load_2d(sm.v[s], &tm_v, &sm.bar_vfull[s], it * kTile, bh_kv * D);
+                mbar_arrive_expect_tx(&sm.bar_vfull[s], AttnCfg<D, PV16>::kVBytes);
+                if constexpr (PV16) {  // two 64-key spans of fp16
+                    tma_load_2d(sm.v[s], &tm_v, &sm.bar_vfull[s], it * kTile, bh_kv * D);
+                    tma_load_2d(sm.v[s] + D * 128, &tm_v, &sm.bar_vfull[s], it * kTile + 64, bh_kv * D);
+                } else {
+                    tma_load_2d(sm.v[s], &tm_v, &sm.bar_vfull[s], it * kTile, bh_kv * D);
+                }
             }
             if (*abort_flag)
                 for (int it = max(0, issued - VS); it < issued; ++it)
                     mbar_wait_quiet(&sm.bar_vfull[it % VS], (it / VS) & 1, kDrainNs);
         } else if (warp == kWarpMma && lane == 0 && n_tiles > 0) {
             // ------------------------------ MMA issuer ------------------------------
-            // Q tile x at q_s + x * kTile * D; P buffer (x, parity) at p_s + (2 x + parity) * kTile^2
+            // Q tile x at q_s + x * kTile * D; P buffer (x, b) at p_s + (x * kPBufs + b) * kPBytes
             const uint32_t q_s = smem_u32(sm.q[0]), p_s = smem_u32(sm.p[0][0]);
             bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, p.status, kSiteQ);
             if (ok) ok = mbar_wait(&sm.bar_kfull[0], 0, abort_flag, p.status, kSiteFull);
@@ -566,8 +611,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         }
                         if (!mbar_wait(&sm.bar_p[x], it & 1, abort_flag, p.status, kSiteP)) { brk = true; break; }
                         tc_fence_after();
-                        issue_pv<D>(tmem + kTmemO + (uint32_t)x * D, p_s + (uint32_t)(2 * x + (it & 1)) * (kTile * kTile),
-                                    smem_u32(sm.v[sv]), it > 0);
+                        const uint32_t pb = p_s + (uint32_t)(x * kPBufs + (PV16 ? 0 : (it & 1))) * kPBytes;
+                        if constexpr (PV16) issue_pv16<D>(tmem + kTmemO + (uint32_t)x * D, pb, smem_u32(sm.v[sv]), it > 0);
+                        else issue_pv<D>(tmem + kTmemO + (uint32_t)x * D, pb, smem_u32(sm.v[sv]), it > 0);
                         mma_commit(&sm.bar_o[x]);
                     }
                 }
@@ -592,38 +638,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // one copy of the softmax code serves both tiles (instruction-cache footprint)
     const int X = warp >> 3;
     if (X == 0 || hasB)
-        softmax_role<D>(sm, p, tmem, X, X ? tB : tA, X ? nB : nA, bh, o_base, n_q, n_kv, abort_flag);
+        softmax_role<D, PV16>(sm, p, tmem, X, X ? tB : tA, X ? nB : nA, bh, o_base, n_q, n_kv, abort_flag);
     tc_fence_before();
     __syncthreads();
 }
 
-template <int D, bool RT>
+template <int D, bool RT, bool PV16>
 static cudaError_t launch_attention_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                       const AttnParams &p, cudaStream_t stream) {
-    const size_t smem = sizeof(AttnSmem<D>) + 1024;
+    const size_t smem = sizeof(AttnSmem<D, PV16>) + 1024;
+    static_assert(sizeof(AttnSmem<D, PV16>) + 1024 <= 227 * 1024, "shared memory of one CTA");
     cudaError_t e =
-        cudaFuncSetAttribute(attn_fwd_kernel<D, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(attn_fwd_kernel<D, RT, PV16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((p.Tq + 1) / 2) * (unsigned)p.BH;
     // Heads per block of the CTA order: as many key/value heads as fit kKvL2Budget
     // bytes of K codes + V^T codes, times the query heads that share each.
     AttnParams pp = p;
-    const size_t kv_head_bytes = 2ull * (size_t)p.nk_pad * D;
+    const size_t kv_head_bytes = (PV16 ? 3ull : 2ull) * (size_t)p.nk_pad * D;
     const size_t kv_heads = kv_head_bytes ? kKvL2Budget / kv_head_bytes : 0;
     const size_t hb = (kv_heads < 1 ? 1 : kv_heads) * (size_t)p.group;
     pp.head_block = (int)(hb < (size_t)p.BH ? hb : (size_t)p.BH);
     if (pp.head_block < 1) pp.head_block = 1;
-    attn_fwd_kernel<D, RT><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, pp);
+    attn_fwd_kernel<D, RT, PV16><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, pp);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                              const AttnParams &p, int d, cudaStream_t stream) {
-    if (d == 128) {
-        if (p.cu_q) return launch_attention_d<128, true>(tq, tk, tv, p, stream);
-        return launch_attention_d<128, false>(tq, tk, tv, p, stream);
+    if (p.pv16) {
+        if (d == 128) return launch_attention_d<128, true, true>(tq, tk, tv, p, stream);
+        return launch_attention_d<64, true, true>(tq, tk, tv, p, stream);
     }
-    return launch_attention_d<64, true>(tq, tk, tv, p, stream);
+    if (d == 128) {
+        if (p.cu_q) return launch_attention_d<128, true, false>(tq, tk, tv, p, stream);
+        return launch_attention_d<128, false, false>(tq, tk, tv, p, stream);
+    }
+    return launch_attention_d<64, true, false>(tq, tk, tv, p, stream);
 }
 
 }  // namespace sage

@@ -44,4 +44,21 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_saddr, uint
     }
 }
 
+// O[d_tmem] (+)= P_tile . V_tile in the FP16 P / V mode: P is 128 rows x 128 keys
+// of fp16 and V^T d rows x 128 keys of fp16, each stored as two 64-key spans of
+// 128-byte rows (128-byte swizzle; span 1 follows span 0); 8 tcgen05.mma kind::f16
+// (f16 x f16, FP32 accumulator) with M = 128, N = d, K = 16.
+template <int D>
+__device__ __forceinline__ void issue_pv16(uint32_t d_tmem, uint32_t p_saddr, uint32_t v_saddr, bool accumulate) {
+    constexpr uint32_t idesc = idesc_f16_f32(128, D, false);
+#pragma unroll
+    for (int span = 0; span < 2; ++span)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t a = smem_desc(p_saddr + span * (kTile * 128) + kk * 32, 1024u, 2u);
+            const uint64_t b = smem_desc(v_saddr + span * (D * 128) + kk * 32, 1024u, 2u);
+            mma_f16_ss(d_tmem, a, b, idesc, (accumulate || span > 0 || kk > 0) ? 1u : 0u);
+        }
+}
+
 }  // namespace sage

@@ -14,7 +14,8 @@
 //   quant_k      per (head, 128-key tile): K_s = K - kbar, INT8 codes per group,
 //                delta_K per 16-key run.
 //   quant_v      per (head, 128-key tile): V / delta_V -> E4M3, written transposed
-//                ([channel][position], keys in the tile storage order: even, then odd).
+//                ([channel][position], keys in the tile storage order: even, then odd);
+//                in the FP16 P / V mode V -> fp16 (round to nearest even), same layout.
 // Every code decision (INT8 rounding, E4M3 rounding) is made on the IEEE fp32
 // quotient x / delta, rounded to nearest even, so that it is reproducible on the
 // host.  The quotient is formed as x * (1 / delta) when that product provably
@@ -285,7 +286,8 @@ __global__ void kv_finalize_kernel(const PrepassArgs a) {
         const float *part = reinterpret_cast<const float *>(a.ws + a.L.vmax_part) + (size_t)bh * nc * D + c;
         float m = 0.f;
         for (int ch = 0; ch < nc; ++ch) m = fmaxf(m, part[(size_t)ch * D]);
-        reinterpret_cast<float *>(a.ws + a.L.dv)[(size_t)bh * D + c] = (m == 0.f) ? 1.f : __fdiv_rn(m, a.v_range);
+        reinterpret_cast<float *>(a.ws + a.L.dv)[(size_t)bh * D + c] =
+            (m == 0.f || a.pv16) ? 1.f : __fdiv_rn(m, a.v_range);  // FP16 V carries no scale
     }
 }
 
@@ -483,6 +485,26 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_
         }
         __syncthreads();  // the stage is in registers: refill it
         if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
+        if (a.pv16) {
+            // FP16 V^T, same key order: per channel, the 8 even keys (16 bytes) at 8w and
+            // the 8 odd keys at 64 + 8w
+            __half *vt16 = reinterpret_cast<__half *>(a.ws + a.L.vt8) + ((size_t)bh * D + lane * VEC) * S.nk_pad + j0 +
+                           warp * (RPW / 2);
+#pragma unroll
+            for (int v = 0; v < VEC; ++v)
+#pragma unroll
+                for (int par = 0; par < 2; ++par) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __half2 h2 = __floats2half2_rn(x[4 * e + par][v], x[4 * e + 2 + par][v]);
+                        w4[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                    }
+                    *reinterpret_cast<uint4 *>(vt16 + (size_t)v * S.nk_pad + par * (kTile / 2)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            continue;
+        }
         // keys j0 + 16w + i: even i at position 8w + i/2, odd i at 64 + 8w + i/2
         uint8_t *vt8 = a.ws + a.L.vt8 + ((size_t)bh * D + lane * VEC) * S.nk_pad + j0 + warp * (RPW / 2);
 #pragma unroll

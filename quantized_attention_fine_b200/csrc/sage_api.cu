@@ -32,10 +32,11 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 struct Mode {
     int g_q, g_k, smooth_q, smooth_k;
     float p_range, v_range;
+    int pv16;
 };
 
 sage_status_t read_mode(const sage_quant_mode_t *m, Mode *out) {
-    sage_quant_mode_t d = {SAGE_QK_PER_THREADGROUP, 1, 1, 448.f, 448.f};
+    sage_quant_mode_t d = {SAGE_QK_PER_THREADGROUP, 1, 1, 448.f, 448.f, 0};
     if (m) d = *m;
     switch (d.gran) {
         case SAGE_QK_PER_BLOCK: out->g_q = 128; out->g_k = 128; break;
@@ -49,6 +50,8 @@ sage_status_t read_mode(const sage_quant_mode_t *m, Mode *out) {
     out->smooth_k = d.smooth_k ? 1 : 0;
     out->p_range = d.p_range;
     out->v_range = d.v_range;
+    if (d.pv_fp16 != 0 && d.pv_fp16 != 1) return SAGE_ERR_INVALID_ARG;
+    out->pv16 = d.pv_fp16;
     return SAGE_OK;
 }
 
@@ -91,6 +94,21 @@ bool encode_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t oute
     return r == CUDA_SUCCESS;
 }
 
+// 2-D map of 16-bit elements (inner extent and box in elements, row pitch in bytes).
+bool encode_2d16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                 uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Tensor maps of the Q codes, K codes ([rows][d] bytes, 128-row boxes) and the
 // transposed V codes ([BH*d][nk_pad] bytes, d x 128 boxes).
 bool make_maps(const Shape &s, const uint8_t *ws, CUtensorMap *tq, CUtensorMap *tk, CUtensorMap *tv) {
@@ -99,8 +117,14 @@ bool make_maps(const Shape &s, const uint8_t *ws, CUtensorMap *tq, CUtensorMap *
     const uint64_t d = (uint64_t)s.d;
     if (tq && !encode_2d(tq, ws + L.q8, d, (uint64_t)s.BH * s.nq_pad, d, (uint32_t)d, kTile, swz_qk)) return false;
     if (tk && !encode_2d(tk, ws + L.k8, d, (uint64_t)s.BH_kv * s.nk_pad, d, (uint32_t)d, kTile, swz_qk)) return false;
-    if (tv && !encode_2d(tv, ws + L.vt8, (uint64_t)s.nk_pad, (uint64_t)s.BH_kv * d, (uint64_t)s.nk_pad, kTile,
-                         (uint32_t)d, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (tv && !s.pv16 &&
+        !encode_2d(tv, ws + L.vt8, (uint64_t)s.nk_pad, (uint64_t)s.BH_kv * d, (uint64_t)s.nk_pad, kTile, (uint32_t)d,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return false;
+    // FP16 V^T: 16-bit elements, boxes of 64 keys (one 128-byte swizzle span) x d channels
+    if (tv && s.pv16 &&
+        !encode_2d16(tv, ws + L.vt8, (uint64_t)s.nk_pad, (uint64_t)s.BH_kv * d, (uint64_t)s.nk_pad * 2, 64,
+                     (uint32_t)d, CU_TENSOR_MAP_SWIZZLE_128B))
         return false;
     return true;
 }
@@ -203,6 +227,7 @@ sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype
     a.smooth_q = m.smooth_q;
     a.smooth_k = m.smooth_k;
     a.v_range = m.v_range;
+    a.pv16 = m.pv16;
     a.ws = ws;
     a.L = ws_layout(s);
     if (launch_prepass(a, stream) != cudaSuccess) return SAGE_ERR_CUDA;
@@ -255,7 +280,8 @@ sage_status_t run_attention(void *o, int dtype, int layout, const Shape &s, int 
     p.out_bf16 = (dtype == SAGE_DTYPE_BF16);
     const float scale = (sm_scale > 0.f) ? sm_scale : 1.0f / sqrtf((float)s.d);
     p.scale_log2 = scale * 1.4426950408889634f;
-    p.log2_pr = log2f(m.p_range);
+    p.pv16 = m.pv16;
+    p.log2_pr = m.pv16 ? 0.f : log2f(m.p_range);  // FP16 P~ is not scaled (Pr = 1)
     p.status = reinterpret_cast<int *>(const_cast<uint8_t *>(ws) + L.status);
     p.fault_inject = fault_inject;
     return launch_attention(tq, tk, tv, p, s.d, stream) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
@@ -283,13 +309,24 @@ size_t sage_workspace_bytes_gqa(int B, int H, int H_kv, int n_q, int n_kv, int d
     return ws_layout(s).total;
 }
 
+size_t sage_workspace_bytes_mode(int B, int H, int H_kv, int n_q, int n_kv, int d, const sage_quant_mode_t *mode) {
+    Shape s;
+    Mode m;
+    if (check_sizes(B, H, H_kv, n_q, n_kv, d, &s) != SAGE_OK || read_mode(mode, &m) != SAGE_OK) return 0;
+    s.pv16 = m.pv16;
+    return ws_layout(s).total;
+}
+
 size_t sage_workspace_bytes(int B, int H, int n_q, int n_kv, int d) {
     return sage_workspace_bytes_gqa(B, H, H, n_q, n_kv, d);
 }
 
-int64_t sage_workspace_offset_gqa(int B, int H, int H_kv, int n_q, int n_kv, int d, int which) {
+int64_t sage_workspace_offset_mode(int B, int H, int H_kv, int n_q, int n_kv, int d, const sage_quant_mode_t *mode,
+                                   int which) {
     Shape s;
-    if (check_sizes(B, H, H_kv, n_q, n_kv, d, &s) != SAGE_OK) return -1;
+    Mode m;
+    if (check_sizes(B, H, H_kv, n_q, n_kv, d, &s) != SAGE_OK || read_mode(mode, &m) != SAGE_OK) return -1;
+    s.pv16 = m.pv16;
     const WsLayout L = ws_layout(s);
     switch (which) {
         case SAGE_WS_Q8: return (int64_t)L.q8;
@@ -307,6 +344,10 @@ int64_t sage_workspace_offset_gqa(int B, int H, int H_kv, int n_q, int n_kv, int
     }
 }
 
+int64_t sage_workspace_offset_gqa(int B, int H, int H_kv, int n_q, int n_kv, int d, int which) {
+    return sage_workspace_offset_mode(B, H, H_kv, n_q, n_kv, d, nullptr, which);
+}
+
 int64_t sage_workspace_offset(int B, int H, int n_q, int n_kv, int d, int which) {
     return sage_workspace_offset_gqa(B, H, H, n_q, n_kv, d, which);
 }
@@ -319,6 +360,7 @@ sage_status_t sage_quant_qk_gqa(const void *q, const void *k, int dtype, int lay
     SAGE_TRY(check_common(dtype, layout));
     SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
+    s.pv16 = m.pv16;
     if (s.BH == 0 || (n_q == 0 && n_kv == 0)) return SAGE_OK;
     if ((n_q > 0 && !q) || (n_kv > 0 && !k)) return SAGE_ERR_INVALID_ARG;
     if ((q && !aligned16(q)) || (k && !aligned16(k))) return SAGE_ERR_UNSUPPORTED;
@@ -341,6 +383,7 @@ sage_status_t sage_quant_v_gqa(const void *v, int dtype, int layout, int B, int 
     SAGE_TRY(check_common(dtype, layout));
     SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
+    s.pv16 = m.pv16;
     if (s.BH == 0 || n_kv == 0) return SAGE_OK;
     if (!v) return SAGE_ERR_INVALID_ARG;
     if (!aligned16(v)) return SAGE_ERR_UNSUPPORTED;
@@ -363,6 +406,7 @@ sage_status_t sage_attn_fwd_prequant_gqa(void *o, int dtype, int layout, int B, 
     SAGE_TRY(check_common(dtype, layout));
     SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
+    s.pv16 = m.pv16;
     if (s.BH == 0 || n_q == 0) return SAGE_OK;
     if (!o) return SAGE_ERR_INVALID_ARG;
     if (!aligned16(o)) return SAGE_ERR_UNSUPPORTED;
@@ -390,6 +434,7 @@ sage_status_t sage_attn_fwd_gqa(const void *q, const void *k, const void *v, voi
     SAGE_TRY(check_common(dtype, layout));
     SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
+    s.pv16 = m.pv16;
     if (s.BH == 0 || n_q == 0) return SAGE_OK;
     if (!q || !o || (n_kv > 0 && (!k || !v))) return SAGE_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(o) || (k && !aligned16(k)) || (v && !aligned16(v))) return SAGE_ERR_UNSUPPORTED;
@@ -424,6 +469,7 @@ sage_status_t sage_attn_fwd_varlen(const void *q, const void *k, const void *v, 
     if (total_q < 0 || total_kv < 0 || total_q > (1 << 30) || total_kv > (1 << 30)) return SAGE_ERR_INVALID_ARG;
     SAGE_TRY(check_sizes(B, H, H_kv, max_seqlen_q, max_seqlen_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
+    s.pv16 = m.pv16;
     s.varlen = 1;
     s.total_q = total_q;
     s.total_kv = total_kv;

@@ -23,12 +23,13 @@ struct Shape {
     int B, H, H_kv, n_q, n_kv, d;
     int BH, BH_kv, Tq, Tk, nq_pad, nk_pad, n_chunks;
     int varlen, total_q, total_kv;
+    int pv16;   // FP16 P / V mode: the transposed V holds 2 bytes per element
 };
 
 inline Shape make_shape(int B, int H, int H_kv, int n_q, int n_kv, int d) {
     Shape s;
     s.B = B; s.H = H; s.H_kv = H_kv; s.n_q = n_q; s.n_kv = n_kv; s.d = d;
-    s.varlen = 0; s.total_q = 0; s.total_kv = 0;
+    s.varlen = 0; s.total_q = 0; s.total_kv = 0; s.pv16 = 0;
     s.BH = B * H;
     s.BH_kv = B * H_kv;
     s.Tq = (n_q + kTile - 1) / kTile;
@@ -55,7 +56,7 @@ inline WsLayout ws_layout(const Shape &s) {
     w.status = take(kStatusBytes);
     w.q8 = take(BH * s.nq_pad * d);
     w.k8 = take(BHk * s.nk_pad * d);
-    w.vt8 = take(BHk * d * s.nk_pad);
+    w.vt8 = take(BHk * d * s.nk_pad * (s.pv16 ? 2 : 1));
     w.dq = take(BH * s.nq_pad * 4);
     w.dk = take(BHk * (s.nk_pad / kKeyRun) * 4);
     w.dv = take(BHk * d * 4);
@@ -107,6 +108,7 @@ struct PrepassArgs {
     Shape shape;
     int g_q, g_k, smooth_q, smooth_k;
     float v_range;
+    int pv16;   // FP16 V (no per-channel scale: delta_V = 1) instead of E4M3 codes
     uint8_t *ws;
     WsLayout L;
 };
@@ -125,6 +127,7 @@ struct AttnParams {
     int head_block;     // query heads per block of the CTA order (set by launch_attention)
     int causal;
     int use_ds;         // 0: Q smoothing off, dS not read
+    int pv16;           // FP16 P~ and V, kind::f16 PV (log2_pr is then 0)
     int out_bf16;
     float scale_log2;   // sm_scale * log2(e)
     float log2_pr;      // log2(Pr)

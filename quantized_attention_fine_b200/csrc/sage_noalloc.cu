@@ -47,7 +47,7 @@ extern "C" sage_status_t sage_attn_fwd_noalloc(const void *q, const void *k, con
                                                int layout, int B, int H, int n_q, int n_kv, int d, int causal,
                                                float sm_scale, const sage_quant_mode_t *mode, void *stream) {
     // Problems whose workspace would not fit are refused before anything is enqueued.
-    const size_t need = sage_workspace_bytes(B, H, n_q, n_kv, d);
+    const size_t need = sage_workspace_bytes_mode(B, H, H, n_q, n_kv, d, mode);
     if (need == 0) return (d != 64 && d != 128) ? SAGE_ERR_UNSUPPORTED : SAGE_ERR_INVALID_ARG;
     uint8_t *base = nullptr;
     sage_status_t st = noalloc_scratch(&base);

@@ -103,6 +103,27 @@ def test_gqa_head_counts_validated(lib):
                                  None) == 1
 
 
+def test_fp16_pv_mode_workspace(lib):
+    """The FP16 P / V mode keeps 2 bytes per transposed V element; the other regions move
+    up accordingly.  A bad pv_fp16 value is refused."""
+    B, H, Hk, nq, nk, d = 1, 4, 2, 300, 520, 128
+    m8, m16 = sage.QuantMode.make(), sage.QuantMode.make(pv="fp16")
+    b8 = lib.sage_workspace_bytes_mode(B, H, Hk, nq, nk, d, ctypes.byref(m8))
+    b16 = lib.sage_workspace_bytes_mode(B, H, Hk, nq, nk, d, ctypes.byref(m16))
+    assert b8 == lib.sage_workspace_bytes_gqa(B, H, Hk, nq, nk, d)
+    nk_pad = -(-nk // 128) * 128
+    assert b16 >= b8 + B * Hk * d * nk_pad - 1024
+    o8 = lib.sage_workspace_offset_mode(B, H, Hk, nq, nk, d, ctypes.byref(m8), 2)
+    o16 = lib.sage_workspace_offset_mode(B, H, Hk, nq, nk, d, ctypes.byref(m16), 2)
+    assert o8 == o16   # V^T itself starts at the same place
+    ds8 = lib.sage_workspace_offset_mode(B, H, Hk, nq, nk, d, ctypes.byref(m8), 8)
+    ds16 = lib.sage_workspace_offset_mode(B, H, Hk, nq, nk, d, ctypes.byref(m16), 8)
+    assert ds16 - ds8 >= B * Hk * d * nk_pad - 1024
+    bad = sage.QuantMode.make()
+    bad.pv_fp16 = 2
+    assert lib.sage_workspace_bytes_mode(B, H, Hk, nq, nk, d, ctypes.byref(bad)) == 0
+
+
 def test_workspace_bytes_rejects_bad_sizes(lib):
     assert lib.sage_workspace_bytes(1, 1, 128, 128, 96) == 0      # d must be 64 or 128
     assert lib.sage_workspace_bytes(-1, 1, 128, 128, 64) == 0
