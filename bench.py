@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--pv", default="fp8", choices=["fp8", "fp16"],
                     help="PV precision: fp8 (the method's default) or fp16 (the qk_int8_pv_fp16 mode)")
+    ap.add_argument("--graph", action="store_true",
+                    help="time the step as a replay of a CUDA graph that captured one sage_attn_fwd call")
     ap.add_argument("--mma-rates", action="store_true",
                     help="print the tensor-core rate of each tcgen05.mma form (diagnostic) and exit")
     return ap.parse_args()
@@ -275,8 +277,18 @@ def main():
     mode = sage.QuantMode.make(pv=args.pv)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def step_eager():
         sage.attn_fwd(q, k, v, causal=w.causal, out=out, workspace=ws, pv=args.pv)
+
+    step = step_eager
+    graph = None
+    if args.graph:  # one captured call, replayed each step (no host launch cost)
+        step_eager()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step_eager()
+        step = graph.replay
 
     def attn_only():
         sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode, out=out)
@@ -378,6 +390,8 @@ def main():
     code, site = sage.get_device_status(ws)
     if code != 0:
         raise SystemExit("device status %d at site %d" % (code, site))
+    if graph is not None:
+        del graph
 
     if world > 1:
         dist.barrier()
@@ -405,7 +419,8 @@ def main():
                        granularity="per_threadgroup (g_q=32, g_k=16)",
                        **({"pv": "fp16 (qk_int8_pv_fp16)"} if pv16 else {"pv": "fp8", "pr": 448, "vr": 448})),
         "attn_kernel_tops": attn_tops, "attn_kernel_ms": attn_avg_ms, "prepass_ms": pre_avg_ms,
-        "step_call": "sage_attn_fwd (pre-pass + dS + attention); prepass_ms = ms_per_step - attn_kernel_ms",
+        "step_call": ("sage_attn_fwd (pre-pass + dS + attention)" + (", replayed from a CUDA graph" if args.graph else "")
+                      + "; prepass_ms = ms_per_step - attn_kernel_ms"),
         "attn_frac_of_spec_4500": attn_tops / SPEC_INT8_TOPS,
         "roofline": {"bound": "tensor", "achieved": attn_tops, "peak": peak, "unit": "TFLOP/s",
                      "frac": attn_tops / peak, "traffic": None if pv16 else recorded_traffic(w.name),
