@@ -290,3 +290,24 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     o = sage.attn_fwd_prequant(ws, dtype=q.dtype).cpu()
     _, oo = oracle_head(q[0, 0], k[0, 0], v[0, 0], causal=False)
     assert_close_to_oracle(to_np64(o[0, 0]), oo, "after timeout")
+
+
+def test_suffix_prefill_over_cached_prefix():
+    """Incremental prefill: a 300-token suffix attends causally to a 2048-token prefix
+    plus itself (N_q = 300 < N_kv = 2348, bottom-right aligned), the KV-cache append
+    pattern.  The method's K mean and delta_V cover the whole key range, so the pre-pass
+    runs over all keys; the output matches the oracle and the last 300 rows of a full
+    prefill over all 2348 tokens to the oracle's tolerance."""
+    n_pre, n_suf, d, H = 2048, 300, 128, 2
+    _, q, k, v = _inputs("suffix", 1, H, n_pre + n_suf, n_pre + n_suf, d, True, recipe="llm")
+    qs = q[:, :, n_pre:].contiguous()
+    o = sage.attn_fwd(qs.cuda(), k.cuda(), v.cuda(), causal=True).cpu()
+    o_full = sage.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True).cpu()
+    for h in range(H):
+        _, oo = oracle_head(qs[0, h], k[0, h], v[0, h], causal=True)
+        assert_close_to_oracle(to_np64(o[0, h]), oo, "suffix head %d" % h)
+        ref = oracle.reference_attention(to_np64(qs[0, h])[None, None], to_np64(k[0, h])[None, None],
+                                         to_np64(v[0, h])[None, None], causal=True)[0, 0]
+        assert cos(to_np64(o[0, h]), ref) >= O_COS_FULL
+        # the suffix rows of the full prefill see the same keys; Q smoothing blocks differ
+        assert cos(to_np64(o[0, h]), to_np64(o_full[0, h, n_pre:])) >= 0.999
