@@ -22,6 +22,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -172,8 +173,15 @@ class ClockSampler:
         if not enabled:
             return
         try:
-            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-            self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % device_index)
+            # the raw samples go to a temporary file (or to $SAGE_BENCH_LOG_DIR, kept)
+            log_dir = os.environ.get("SAGE_BENCH_LOG_DIR")
+            if log_dir:
+                os.makedirs(log_dir, exist_ok=True)
+                self.path, self.keep = os.path.join(log_dir, "clocks_rank%d.csv" % device_index), True
+            else:
+                fd, self.path = tempfile.mkstemp(prefix="sage_clocks_rank%d_" % device_index, suffix=".csv")
+                os.close(fd)
+                self.keep = False
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(device_index), "--query-gpu=" + self.FIELDS,
                                           "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
@@ -204,6 +212,8 @@ class ClockSampler:
             for name, val in zip(names, parts[5:9]):
                 if val.lower() == "active":
                     reasons.add(name)
+        if not self.keep:
+            os.remove(self.path)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
