@@ -24,6 +24,9 @@
  *      with FP32 accumulation in tensor memory.
  *   6. O = acc / Pr * delta_V[c] / l, with l the sum of the unquantized P~; a row
  *      that sees no key is 0.  Rounded to the input dtype (round to nearest even).
+ *   7. The row log-sum-exp of the logits, written to the workspace (SAGE_WS_LSE).
+ * The FP16 P / V mode (sage_quant_mode_t.pv_fp16) replaces steps 4-6's E4M3 P and V
+ * by fp16 P~ and V (no Pr, no delta_V) and the FP8 PV product by an FP16 one.
  *
  * Conventions for every entry point:
  *   - Device pointers are plain CUDA device addresses; `stream` is a cudaStream_t
@@ -44,8 +47,11 @@
  *     the comparison with SGLang and the list of unvalidated variants.)
  *   - The caller owns all memory, including the workspace; the library allocates
  *     nothing and keeps no state between calls.  The workspace must be at least
- *     sage_workspace_bytes(...) bytes, 1024-byte aligned, and its first 256 bytes
- *     (the device status block) must be zero before first use.
+ *     sage_workspace_bytes_mode(...) bytes for the mode used (sage_workspace_bytes
+ *     for the default mode), 1024-byte aligned, and its first 256 bytes (the
+ *     device status block) must be zero before first use.  Each entry point
+ *     enqueues its launches on `stream` only and takes its parameters by value, so
+ *     a call may be captured in a CUDA graph and replayed.
  *   - Argument errors return a status synchronously and enqueue nothing.  A launch
  *     failure returns SAGE_ERR_CUDA.  A device-side wait that runs out (about one
  *     second) makes the kernel stop early and record SAGE_ERR_TIMEOUT in the status
