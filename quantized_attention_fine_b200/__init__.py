@@ -21,7 +21,7 @@ import threading
 
 __all__ = [
     "QuantMode", "Workspace", "workspace_bytes", "make_workspace", "quant_qk", "quant_v", "attn_fwd_prequant",
-    "attn_fwd", "attn_fwd_varlen", "get_device_status", "workspace_view", "debug_qk_tile", "debug_pv_accumulate",
+    "attn_fwd", "attn_fwd_varlen", "SageAttention", "scaled_dot_product_attention", "QUANT_MODES", "get_device_status", "workspace_view", "debug_qk_tile", "debug_pv_accumulate",
     "debug_fault_inject", "debug_pv_accumulate_f16acc", "debug_mma_rate", "library_path", "load_library", "SageError", "GRANULARITIES",
 ]
 
@@ -356,6 +356,70 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, max_seqlen_q=None, 
     if return_lse:
         return out, ws.view("lse").view(B, H, -1)[:, :, :max_seqlen_q]
     return out
+
+
+# The quantization modes the SageAttention deployment guide names (its usage section):
+# INT8 Q / K with FP8 or FP16 P and V.
+QUANT_MODES = {"qk_int8_pv_fp8": "fp8", "qk_int8_pv_fp16": "fp16"}
+
+
+class SageAttention:
+    """Callable drop-in for a model's attention function, configured once the way the
+    SageAttention deployment guide shows (head_dim, is_causal, quant_mode):
+
+        attn = SageAttention(head_dim=128, is_causal=True, quant_mode="qk_int8_pv_fp16")
+        o = attn(q, k, v)          # q [B, H, N_q, d], k / v [B, H_kv, N_kv, d]
+
+    tensor_layout "HND" ([B, H, N, d]) or "NHD" ([B, N, H, d]).  The workspace of the
+    last shape is kept and reused (one in-flight call per instance)."""
+
+    def __init__(self, head_dim=128, is_causal=False, quant_mode="qk_int8_pv_fp8", tensor_layout="HND",
+                 sm_scale=None, granularity="per_threadgroup", smooth_q=True, smooth_k=True):
+        if head_dim not in (64, 128):
+            raise ValueError("head_dim must be 64 or 128")
+        if quant_mode not in QUANT_MODES:
+            raise ValueError("quant_mode must be one of %s" % sorted(QUANT_MODES))
+        if tensor_layout not in _LAYOUTS:
+            raise ValueError("tensor_layout must be 'HND' or 'NHD'")
+        if granularity not in GRANULARITIES:
+            raise ValueError("granularity must be one of %s" % sorted(GRANULARITIES))
+        self.head_dim, self.is_causal, self.quant_mode = head_dim, bool(is_causal), quant_mode
+        self.tensor_layout, self.sm_scale, self.granularity = tensor_layout, sm_scale, granularity
+        self.smooth_q, self.smooth_k = smooth_q, smooth_k
+        self._ws = None
+
+    def __call__(self, q, k, v, return_lse=False):
+        if int(q.shape[-1]) != self.head_dim:
+            raise ValueError("head dim %d, configured %d" % (int(q.shape[-1]), self.head_dim))
+        B, H, H_kv, n_q, n_kv, d = _shape(q, k, self.tensor_layout)
+        pv = QUANT_MODES[self.quant_mode]
+        if self._ws is None or not self._ws.fits(B, H, n_q, n_kv, d, H_kv, pv == "fp16") or \
+                self._ws.tensor.device != q.device:
+            self._ws = Workspace(B, H, n_q, n_kv, d, q.device, H_kv=H_kv, pv_fp16=(pv == "fp16"))
+        return attn_fwd(q, k, v, causal=self.is_causal, sm_scale=self.sm_scale, layout=self.tensor_layout,
+                        granularity=self.granularity, smooth_q=self.smooth_q, smooth_k=self.smooth_k, pv=pv,
+                        workspace=self._ws, return_lse=return_lse)
+
+
+def scaled_dot_product_attention(query, key, value, attn_mask=None, dropout_p=0.0, is_causal=False, scale=None,
+                                 enable_gqa=False, quant_mode="qk_int8_pv_fp8"):
+    """The quantized forward behind torch.nn.functional.scaled_dot_product_attention's
+    signature ([B, H, N, d] tensors, head-major).  Explicit masks and dropout are not
+    part of the method and are refused; is_causal is bottom-right aligned when N_q !=
+    N_kv (torch aligns top-left there).  K and V may have fewer heads than Q only with
+    enable_gqa, as in torch."""
+    if attn_mask is not None:
+        raise NotImplementedError("explicit attention masks are not supported (use is_causal)")
+    if dropout_p != 0.0:
+        raise NotImplementedError("dropout is not supported")
+    if quant_mode not in QUANT_MODES:
+        raise ValueError("quant_mode must be one of %s" % sorted(QUANT_MODES))
+    if query.dim() != 4 or key.dim() != 4:
+        raise ValueError("query, key, value must be [B, H, N, d]")
+    if int(key.shape[1]) != int(query.shape[1]) and not enable_gqa:
+        raise ValueError("key has %d heads and query %d: pass enable_gqa=True" % (int(key.shape[1]),
+                                                                                  int(query.shape[1])))
+    return attn_fwd(query, key, value, causal=is_causal, sm_scale=scale, layout="HND", pv=QUANT_MODES[quant_mode])
 
 
 def get_device_status(workspace: Workspace, stream=None):

@@ -149,3 +149,17 @@ def test_gqa_bad_head_counts_rejected_before_launch():
     rc = lib.sage_attn_fwd_gqa(p(q.data_ptr()), p(k.data_ptr()), p(k.data_ptr()), p(o.data_ptr()), 1, 0, 1, 6, 4,
                                128, 128, 64, 0, 0.0, None, p(ws.ptr), ws.nbytes, None)
     assert rc == sage.SAGE_ERR_INVALID_ARG
+
+
+def test_drop_in_interfaces_equal_attn_fwd():
+    """SageAttention(...) and scaled_dot_product_attention(...) only marshal arguments:
+    their outputs equal the attn_fwd call they stand for."""
+    q, k, v = (x.cuda() for x in _inputs(1, 8, 2, 300, 300, 128, True))
+    ref = sage.attn_fwd(q, k, v, causal=True)
+    a = sage.SageAttention(head_dim=128, is_causal=True)
+    assert torch.equal(a(q, k, v), ref)
+    assert torch.equal(a(q, k, v), ref)   # the kept workspace is reused
+    assert torch.equal(sage.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True), ref)
+    a16 = sage.SageAttention(head_dim=128, is_causal=True, quant_mode="qk_int8_pv_fp16", tensor_layout="NHD")
+    qn, kn, vn = (x.transpose(1, 2).contiguous() for x in (q, k, v))
+    assert torch.equal(a16(qn, kn, vn), sage.attn_fwd(qn, kn, vn, causal=True, layout="NHD", pv="fp16"))
