@@ -75,7 +75,11 @@ def _load():
             lib.oracle_int8_scale.restype = ctypes.c_float
             lib.oracle_f16_round.argtypes = [ctypes.c_float]
             lib.oracle_f16_round.restype = ctypes.c_double
-            lib.oracle_prepass.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 15
+            lib.oracle_prepass.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 17
+            lib.oracle_e2m1_from_f32.argtypes = [ctypes.c_float]
+            lib.oracle_e2m1_from_f32.restype = ctypes.c_uint8
+            lib.oracle_e2m1_to_f64.argtypes = [ctypes.c_uint8]
+            lib.oracle_e2m1_to_f64.restype = ctypes.c_double
             lib.oracle_prepass.restype = ctypes.c_int
             lib.oracle_attn.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 9 + [ctypes.c_int, P, P, P]
             lib.oracle_attn.restype = ctypes.c_int
@@ -150,6 +154,22 @@ def _cfg(n_q, n_kv, d, g_q, g_k, smooth_q, smooth_k, quant, p_range, v_range, sm
 # IEEE fp16 (P unscaled, V without per-channel scale), the PV product in fp16 x fp16.
 PV_FP8 = (1, 1, 1)
 PV_FP16 = (1, 2, 2)
+# FP4 Q / K ("4+8": 4-bit QK^T, FP8 PV), in the microscaling form B200's tensor cores
+# take: E2M1 codes, an E4M3 scale per 16 channels of each row and an fp32 scale per
+# 128-row Q block / 128-key K tile (q_sf / k_sf hold the E4M3 scale codes).
+QK_FP4_PV_FP8 = (2, 1, 1)
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """E2M1 codes (round to nearest, ties to even mantissa, saturating at +-6)."""
+    lib = _load()
+    return np.array([lib.oracle_e2m1_from_f32(float(v)) for v in np.asarray(x, np.float32).ravel()],
+                    np.uint8).reshape(np.shape(x))
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    lib = _load()
+    return np.array([lib.oracle_e2m1_to_f64(int(c)) for c in np.asarray(codes).ravel()]).reshape(np.shape(codes))
 
 
 def f16_round(x):
@@ -179,12 +199,13 @@ def prepass_head(q, k, v, *, g_q=32, g_k=16, smooth_q=True, smooth_k=True,
         dk_key=np.zeros((nk_pad,), np.float32), k_s=np.zeros((max(nk, 1), d), np.float64),
         v_code=np.zeros((max(nk, 1), d), np.uint8), v_hat=np.zeros((max(nk, 1), d), np.float64),
         dv=np.zeros((d,), np.float32),
+        q_sf=np.zeros((nq_pad, max(d // 16, 1)), np.uint8), k_sf=np.zeros((nk_pad, max(d // 16, 1)), np.uint8),
     )
     rc = lib.oracle_prepass(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v),
                             _ptr(r["qbar"]), _ptr(r["kbar"]),
                             _ptr(r["q_code"]), _ptr(r["q_hat"]), _ptr(r["dq_row"]),
                             _ptr(r["k_code"]), _ptr(r["k_hat"]), _ptr(r["dk_key"]), _ptr(r["k_s"]),
-                            _ptr(r["v_code"]), _ptr(r["v_hat"]), _ptr(r["dv"]))
+                            _ptr(r["v_code"]), _ptr(r["v_hat"]), _ptr(r["dv"]), _ptr(r["q_sf"]), _ptr(r["k_sf"]))
     if rc != 0:
         raise ValueError("oracle_prepass failed with code %d" % rc)
     r["k_s"] = r["k_s"][:nk]

@@ -60,7 +60,8 @@ typedef struct {
     int n_q, n_kv, d;
     int g_q, g_k;         /* INT8 group sizes (rows of a Q block, keys of a KV tile) */
     int smooth_q, smooth_k;
-    int quant_qk;         /* 1: INT8 codes as in the method; 0: exact (identity) */
+    int quant_qk;         /* 1: INT8 codes as in the method; 0: exact (identity);  */
+                          /* 2: FP4 (E2M1) codes with two-level scales (see below)  */
     int quant_p;          /* 1: E4M3 P; 0: exact P~ * Pr; 2: FP16 P~ (no Pr scale)  */
     int quant_v;          /* 1: E4M3 V; 0: exact V / delta_V; 2: FP16 V (no scale)  */
     double p_range, v_range;
@@ -132,6 +133,74 @@ double oracle_f16_round(float xf)
     return copysign(nearbyint(a / step) * step, x);
 }
 
+/* E2M1 (4-bit: 1 sign, 2 exponent bits with bias 1, 1 mantissa bit; magnitudes
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6; no infinities or NaN).  Encoding rounds to nearest
+ * with ties to the even mantissa and saturates to +-6. */
+static const double oracle_e2m1_mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double oracle_e2m1_to_f64(uint8_t c)
+{
+    double v = oracle_e2m1_mag[c & 7];
+    return (c & 8) ? -v : v;
+}
+
+uint8_t oracle_e2m1_from_f32(float xf)
+{
+    double x = (double)xf;
+    uint8_t sign = (x < 0.0 || (x == 0.0 && signbit(x))) ? 8 : 0;
+    double a = fabs(x);
+    if (isnan(x) || a >= 6.0) return (uint8_t)(sign | 7);
+    int best = 0;
+    for (int i = 1; i < 8; ++i) {
+        double di = fabs(a - oracle_e2m1_mag[i]), db = fabs(a - oracle_e2m1_mag[best]);
+        if (di < db || (di == db && (i & 1) == 0)) best = i;  /* ties: even mantissa */
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* Two-level FP4 scales of one 128-row tile of smoothed values (fp32, [128][d], rows
+ * past `valid` are 0), the microscaling form of 4-bit Q / K on B200 (block-scaled
+ * tcgen05.mma kind::mxf4nvf4; "SageAttention3: Microscaling FP4 Attention", listed
+ * among the notes' related papers):
+ *   g        = amax over the tile / (6 * 448)          (fp32; 1 if amax = 0)
+ *   sf[r][b] = E4M3(fp32(amax of row r, channels 16b..16b+15 / g) / 6)
+ *              (1 if that amax is 0; the smallest subnormal 2^-9 if it rounds to 0)
+ *   code     = E2M1(fp32(x / fp32(g * sf)))
+ * so x ~ g * sf * code.  Writes codes (4-bit values in int8), hat = sf * code (exact),
+ * the sf codes, and returns g. */
+static float oracle_fp4_tile(const float *xs, int d, int8_t *code, double *hat, uint8_t *sf_code)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < ORACLE_TILE * d; ++i) {
+        float a = fabsf(xs[i]);
+        if (a > amax) amax = a;
+    }
+    const float g = (amax == 0.0f) ? 1.0f : amax / 2688.0f;
+    for (int r = 0; r < ORACLE_TILE; ++r)
+        for (int b0 = 0; b0 < d; b0 += 16) {
+            float am = 0.0f;
+            for (int c = b0; c < b0 + 16; ++c) {
+                float a = fabsf(xs[(size_t)r * d + c]);
+                if (a > am) am = a;
+            }
+            uint8_t sc = 0x38;  /* 1.0 */
+            if (am != 0.0f) {
+                sc = oracle_e4m3_from_f32((am / g) / 6.0f);
+                if ((sc & 0x7F) == 0) sc = 0x01;
+            }
+            sf_code[(size_t)r * (d / 16) + b0 / 16] = sc;
+            const double sfv = oracle_e4m3_to_f64(sc);
+            const float delta = g * (float)sfv;
+            for (int c = b0; c < b0 + 16; ++c) {
+                size_t o = (size_t)r * d + c;
+                uint8_t e = oracle_e2m1_from_f32(xs[o] / delta);
+                code[o] = (int8_t)e;
+                hat[o] = sfv * oracle_e2m1_to_f64(e);
+            }
+        }
+    return g;
+}
+
 /* INT8 code of an fp32 value for a given fp32 scale: round half to even of the
  * correctly rounded fp32 quotient, then clamp to the symmetric range +-127. */
 int8_t oracle_int8_code(float xs, float delta)
@@ -169,7 +238,8 @@ int oracle_prepass(const oracle_cfg_t *cfg, const double *q, const double *k, co
                    float *qbar, float *kbar,
                    int8_t *q_code, double *q_hat, float *dq_row,
                    int8_t *k_code, double *k_hat, float *dk_key, double *k_s,
-                   uint8_t *v_code, double *v_hat, float *dv)
+                   uint8_t *v_code, double *v_hat, float *dv,
+                   uint8_t *q_sf, uint8_t *k_sf)
 {
     const int nq = cfg->n_q, nk = cfg->n_kv, d = cfg->d;
     if (nq < 0 || nk < 0 || d <= 0) return 1;
@@ -198,6 +268,12 @@ int oracle_prepass(const oracle_cfg_t *cfg, const double *q, const double *k, co
             int i = t * ORACLE_TILE + r;
             for (int c = 0; c < d; ++c)
                 xs[(size_t)r * d + c] = (i < nq) ? ((float)q[(size_t)i * d + c] - qb[c]) : 0.0f;
+        }
+        if (cfg->quant_qk == 2) {  /* FP4 codes with two-level scales */
+            size_t o0 = (size_t)t * ORACLE_TILE * d;
+            const float g = oracle_fp4_tile(xs, d, q_code + o0, q_hat + o0, q_sf + (size_t)t * ORACLE_TILE * (d / 16));
+            for (int r = 0; r < ORACLE_TILE; ++r) dq_row[t * ORACLE_TILE + r] = g;
+            continue;
         }
         for (int g0 = 0; g0 < ORACLE_TILE; g0 += cfg->g_q) {
             float amax = 0.0f;
@@ -238,8 +314,24 @@ int oracle_prepass(const oracle_cfg_t *cfg, const double *q, const double *k, co
     for (int j = 0; j < nk; ++j)
         for (int c = 0; c < d; ++c)
             k_s[(size_t)j * d + c] = k[(size_t)j * d + c] - (double)kbar[c];
+    /* --- K: FP4 codes with two-level scales per 128-key tile --- */
+    if (cfg->quant_qk == 2) {
+        float *ks = (float *)malloc(sizeof(float) * (size_t)ORACLE_TILE * d);
+        if (!ks) return 3;
+        for (int t = 0; t < tk; ++t) {
+            for (int r = 0; r < ORACLE_TILE; ++r) {
+                int j = t * ORACLE_TILE + r;
+                for (int c = 0; c < d; ++c)
+                    ks[(size_t)r * d + c] = (j < nk) ? ((float)k[(size_t)j * d + c] - kbar[c]) : 0.0f;
+            }
+            size_t o0 = (size_t)t * ORACLE_TILE * d;
+            const float g = oracle_fp4_tile(ks, d, k_code + o0, k_hat + o0, k_sf + (size_t)t * ORACLE_TILE * (d / 16));
+            for (int r = 0; r < ORACLE_TILE; ++r) dk_key[t * ORACLE_TILE + r] = g;
+        }
+        free(ks);
+    }
     /* --- K: INT8 codes per group of g_k keys inside each 128-key tile --- */
-    for (int g0 = 0; g0 < nk_pad; g0 += cfg->g_k) {
+    for (int g0 = 0; cfg->quant_qk != 2 && g0 < nk_pad; g0 += cfg->g_k) {
         float amax = 0.0f;
         for (int j = g0; j < g0 + cfg->g_k && j < nk; ++j)
             for (int c = 0; c < d; ++c) {

@@ -567,3 +567,104 @@ def test_pv_fp16_more_accurate_than_fp8():
     o16 = oracle.sage_attention(qn, kn, vn, quant=oracle.PV_FP16)
     e8, e16 = np.abs(o8 - ref).max(), np.abs(o16 - ref).max()
     assert e16 < e8
+
+
+# ---------------------------------------------------------------------------
+# FP4 (E2M1) Q / K with two-level scales
+# ---------------------------------------------------------------------------
+def _e2m1_value(code):
+    """E2M1 from its definition: sign bit 3, exponent bits 2-1 (bias 1), mantissa bit 0."""
+    s, e, m = (code >> 3) & 1, (code >> 1) & 3, code & 1
+    v = m * 0.5 if e == 0 else 2.0 ** (e - 1) * (1 + m / 2)
+    return -v if s else v
+
+
+def test_e2m1_codec_against_definition_and_brute_force():
+    assert [oracle.e2m1_decode(c) for c in range(16)] == [_e2m1_value(c) for c in range(16)]
+    finite = sorted({_e2m1_value(c) for c in range(16)})
+    rng = np.random.default_rng(8)
+    mids = [(a + b) / 2 for a, b in zip(finite, finite[1:])]
+    xs = np.concatenate([rng.uniform(-7, 7, 3000), mids, [0.0, 6.0, -6.0, 6.5, -100.0, 5.999]]).astype(np.float32)
+    codes = oracle.e2m1_encode(xs)
+    for x, c in zip(xs, codes):
+        if abs(x) >= 6:
+            assert oracle.e2m1_decode(c) == np.sign(x) * 6
+            continue
+        dist = [abs(float(x) - f) for f in finite]
+        best = min(dist)
+        cands = [finite[i] for i, dd in enumerate(dist) if dd == best]
+        if len(cands) == 1:
+            assert oracle.e2m1_decode(c) == cands[0]
+        else:  # a tie goes to the value with an even mantissa bit
+            even = [f for f in cands if int(oracle.e2m1_encode(np.float32([f]))[0]) & 1 == 0]
+            assert oracle.e2m1_decode(c) == even[0]
+
+
+def test_fp4_block_scales_reconstruct_within_half_a_code_step():
+    """x ~ g * sf * code per 16-channel block: the reconstruction error of every
+    element is at most half the E2M1 spacing at its code (saturated elements excepted),
+    every block's largest element codes to 4 or 6, and q_hat is sf * code."""
+    q, k, v = _rand_head(200, 300, 128, seed=55, kbias=3.0, qbias=1.0)
+    pre = oracle.prepass_head(q, k, v, quant=oracle.QK_FP4_PV_FP8)
+    qs = (q - np.repeat(pre["qbar"].astype(np.float64), 128, axis=0)[:200]).astype(np.float32)
+    g = pre["dq_row"][:200].astype(np.float64)
+    sf = np.array([[oracle.e4m3_decode(c) for c in row] for row in pre["q_sf"][:200]])
+    codes = pre["q_code"][:200].astype(np.uint8)
+    a = oracle.e2m1_decode(codes)
+    delta = np.repeat(sf, 16, axis=1) * g[:, None]
+    assert np.array_equal(pre["q_hat"][:200], np.repeat(sf, 16, axis=1) * a)
+    spacing = np.where(np.abs(a) < 2, 0.5, np.where(np.abs(a) < 4, 1.0, 2.0))
+    err = np.abs(qs - delta * a)
+    ok = (err <= delta * spacing / 2 * (1 + 1e-6)) | (np.abs(a) == 6)
+    assert ok.all()
+    blk_max = np.abs(a).reshape(200, 8, 16).max(2)
+    xs_max = np.abs(qs).reshape(200, 8, 16).max(2)
+    assert np.all((blk_max >= 4) | (xs_max == 0))
+
+
+def test_fp4_scores_equal_attention_on_dequantized_q_k():
+    """With FP4 Q / K and exact P / V, the oracle is textbook attention on the
+    dequantized smoothed operands plus the Q-smoothing bias (numpy, from the pre-pass
+    codes and scales)."""
+    nq, nk, d = 150, 260, 64
+    q, k, v = _rand_head(nq, nk, d, seed=66, kbias=3.0, qbias=1.0)
+    pre = oracle.prepass_head(q, k, v, quant=(2, 0, 0))
+    o = oracle.attn_head(pre, causal=True)
+    qh = pre["q_hat"][:nq] * pre["dq_row"][:nq, None].astype(np.float64)
+    kh = pre["k_hat"][:nk] * pre["dk_key"][:nk, None].astype(np.float64)
+    tq = -(-nq // 128)
+    ds = np.stack([oracle.delta_s(pre, t) for t in range(tq)])
+    s = qh @ kh.T + ds[np.arange(nq) // 128]
+    ref = _textbook_from_scores(s / 8.0, v, causal=True)
+    assert np.max(np.abs(o - ref)) < 1e-12
+
+
+def _textbook_from_scores(x, v, causal):
+    nq, nk = x.shape
+    if causal:
+        x = np.where(np.arange(nk)[None, :] <= np.arange(nq)[:, None] + (nk - nq), x, -np.inf)
+    m = x.max(1, keepdims=True)
+    p = np.exp(x - m)
+    return (p @ v) / p.sum(1, keepdims=True)
+
+
+def test_fp4_qk_accuracy_and_smoothing():
+    """FP4 Q / K is lossier than INT8 but close to full precision on the tiny workload
+    (cosine >= 0.985 against 0.999 for INT8), and without K smoothing a large K bias
+    ruins it (inputs with a per-channel K bias of std 8)."""
+    q, k, v = wl.generate(wl.TINY)
+    qn, kn, vn = (x.double().numpy() for x in (q, k, v))
+    ref = oracle.reference_attention(qn, kn, vn)
+    o4 = oracle.sage_attention(qn, kn, vn, quant=oracle.QK_FP4_PV_FP8)
+    o8 = oracle.sage_attention(qn, kn, vn, quant=oracle.PV_FP8)
+    assert 0.985 <= cos_np(o4, ref) < cos_np(o8, ref)
+    qb, kb, vb = _rand_head(256, 256, 64, seed=77, kbias=8.0)
+    r = oracle.reference_attention(qb[None, None], kb[None, None], vb[None, None])[0, 0]
+    on = oracle.attn_head(oracle.prepass_head(qb, kb, vb, quant=oracle.QK_FP4_PV_FP8, smooth_k=False))
+    os_ = oracle.attn_head(oracle.prepass_head(qb, kb, vb, quant=oracle.QK_FP4_PV_FP8))
+    assert cos_np(os_, r) > 0.9 > 0.7 > cos_np(on, r)
+
+
+def cos_np(a, b):
+    a, b = np.ravel(a), np.ravel(b)
+    return float(a @ b / math.sqrt((a @ a) * (b @ b)))
