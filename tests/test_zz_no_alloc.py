@@ -71,3 +71,17 @@ def test_noalloc_refuses_problems_larger_than_its_scratch(lib):
     torch.cuda.synchronize()
     assert rc == sage.SAGE_ERR_WORKSPACE
     assert torch.all(o == 3.0)      # nothing was enqueued
+
+
+def test_noalloc_fp16_pv_mode(lib):
+    """The FP16 P / V mode sizes its scratch with its own (larger) workspace and matches
+    the workspace entry point."""
+    w = wl.custom("noalloc_pv16", 1, 4, 600, 600, 128, True, recipe="llm", seed=4444)
+    q, k, v = (x.cuda() for x in wl.generate(w))
+    mode = sage.QuantMode.make(pv="fp16")
+    assert sage.workspace_bytes(1, 4, 600, 600, 128, pv_fp16=True) > sage.workspace_bytes(1, 4, 600, 600, 128)
+    ref = sage.attn_fwd(q, k, v, causal=True, pv="fp16")
+    o = torch.full_like(q, float("nan"))
+    assert _call_noalloc(lib, q, k, v, o, True, mode) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref)
