@@ -300,6 +300,20 @@ SAGE_API sage_status_t sage_debug_pv_accumulate_f16acc(const uint8_t *p, const u
  * SAGE_ERR_TIMEOUT).  n_iter <= 2^20, n_ctas <= 4096. */
 SAGE_API sage_status_t sage_debug_mma_rate(int kind, int n_iter, int n_ctas, void *status_block, void *stream);
 
+/* FP4 quantization of smoothed rows, the building block of the 4-bit Q / K path
+ * (block-scaled E2M1 operands of tcgen05.mma kind::mxf4nvf4): per 128-row tile an fp32
+ * scale g = amax / 2688 (1 if amax = 0), per row and 16 channels an E4M3 scale
+ * sf = E4M3(amax / g / 6) (1.0 if amax = 0; 2^-9 if it rounds to 0), per element the
+ * E2M1 code of x / (g * sf) (round to nearest even, saturating at +-6), every
+ * quotient rounded to fp32.
+ *   xs    : device fp32 [n_rows][d] (16-byte aligned), rows past n_rows read as 0
+ *   codes : device uint8 [n_pad][d/2], two codes per byte, channel 2i in the low nibble
+ *   sf    : device uint8 [n_pad][d/16], E4M3 codes
+ *   g     : device fp32 [n_pad/128]
+ * with n_pad = ceil(n_rows / 128) * 128. */
+SAGE_API sage_status_t sage_debug_quant_fp4(const float *xs, int n_rows, int d, uint8_t *codes, uint8_t *sf,
+                                            float *g, void *stream);
+
 /* Runs the attention kernel with one deliberately missing producer signal so that
  * the consumer's bounded wait must run out; the kernel records SAGE_ERR_TIMEOUT in
  * the status block and exits without hanging.  Arguments as sage_attn_fwd_prequant. */

@@ -22,7 +22,7 @@ import threading
 __all__ = [
     "QuantMode", "Workspace", "workspace_bytes", "make_workspace", "quant_qk", "quant_v", "attn_fwd_prequant",
     "attn_fwd", "attn_fwd_varlen", "SageAttention", "scaled_dot_product_attention", "QUANT_MODES", "get_device_status", "workspace_view", "debug_qk_tile", "debug_pv_accumulate",
-    "debug_fault_inject", "debug_pv_accumulate_f16acc", "debug_mma_rate", "library_path", "load_library", "SageError", "GRANULARITIES",
+    "debug_fault_inject", "debug_pv_accumulate_f16acc", "debug_mma_rate", "debug_quant_fp4", "library_path", "load_library", "SageError", "GRANULARITIES",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -106,13 +106,14 @@ def load_library():
         lib.sage_debug_pv_accumulate.argtypes = [P, P, I, I, P, P]
         lib.sage_debug_pv_accumulate_f16acc.argtypes = [P, P, I, I, P, P]
         lib.sage_debug_mma_rate.argtypes = [I, I, I, P, P]
+        lib.sage_debug_quant_fp4.argtypes = [P, I, I, P, P, P, P]
         lib.sage_debug_attn_fault_inject.argtypes = [P, I, I, I, I, I, I, I, I, P, S, P]
         lib.sage_version.restype = ctypes.c_char_p
         for fn in ("sage_quant_qk", "sage_quant_v", "sage_attn_fwd_prequant", "sage_attn_fwd",
                    "sage_quant_qk_gqa", "sage_quant_v_gqa", "sage_attn_fwd_prequant_gqa", "sage_attn_fwd_gqa",
                    "sage_attn_fwd_varlen",
                    "sage_get_device_status", "sage_debug_qk_tile", "sage_debug_pv_accumulate",
-                   "sage_debug_pv_accumulate_f16acc", "sage_debug_mma_rate",
+                   "sage_debug_pv_accumulate_f16acc", "sage_debug_mma_rate", "sage_debug_quant_fp4",
                    "sage_debug_attn_fault_inject"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
@@ -496,6 +497,21 @@ def debug_mma_rate(kind: str, n_iter: int = 8192, n_ctas=None, repeats: int = 5,
         raise SageError(int(status[0].item()), "sage_debug_mma_rate (device wait)")
     flops = n_ctas * n_iter * 2.0 * 128 * 256 * k
     return flops / (best * 1e-3) / 1e12
+
+
+def debug_quant_fp4(xs, stream=None):
+    """FP4 (E2M1) codes with two-level scales of fp32 rows xs [n, d] (diagnostic).
+    Returns (codes uint8 [n_pad, d/2], two per byte; sf uint8 [n_pad, d/16] E4M3 codes;
+    g fp32 [n_pad/128])."""
+    torch = _torch()
+    n, d = int(xs.shape[0]), int(xs.shape[1])
+    n_pad = -(-n // 128) * 128
+    codes = torch.empty((n_pad, d // 2), dtype=torch.uint8, device=xs.device)
+    sf = torch.empty((n_pad, d // 16), dtype=torch.uint8, device=xs.device)
+    g = torch.empty((n_pad // 128,), dtype=torch.float32, device=xs.device)
+    _check(load_library().sage_debug_quant_fp4(_ptr(xs), n, d, _ptr(codes), _ptr(sf), _ptr(g),
+                                               _stream_handle(stream)), "sage_debug_quant_fp4")
+    return codes, sf, g
 
 
 def debug_fault_inject(workspace: Workspace, out, *, layout="HND", causal=False, stream=None):

@@ -13,6 +13,8 @@
 //   1  kind::f8f6f4, E4M3 x E4M3, FP16 accumulator   (SageAttention2++ PV)
 //   2  kind::i8, S8 x S8, S32 accumulator            (the forward's QK^T)
 //   3  kind::f16, BF16 x BF16, FP32 accumulator      (dS)
+#include <cuda_fp16.h>
+
 #include "attn_mma.cuh"
 #include "sage_device.cuh"
 #include "sage_internal.h"
@@ -37,6 +39,92 @@ constexpr int kSiteRate = 41;
 constexpr size_t kRateSmem = 160u * 1024u;
 
 }  // namespace
+
+// ---------------------------------------------------------------------------
+// FP4 quantization of smoothed rows, the two-level microscaling form of 4-bit Q / K
+// on B200 (block-scaled tcgen05.mma kind::mxf4nvf4; "SageAttention3: Microscaling
+// FP4 Attention", listed among the notes' related papers): per 128-row tile
+//   g = amax / (6 * 448)  (1 if amax = 0),
+// per row and 16 channels
+//   sf = E4M3(fp32(amax / g) / 6)  (1 if amax = 0; 2^-9 if it rounds to 0),
+// per element
+//   code = E2M1(fp32(x / fp32(g * sf)))  (round to nearest even, saturating at 6).
+// One CTA per tile, 8 warps of 16 rows, lane l holding channels l*VEC ..; a 16-channel
+// block spans 16 / VEC lanes.  Output: codes packed two per byte (channel 2i in the
+// low nibble), [n_pad][d / 2]; E4M3 scale codes [n_pad][d / 16]; g per tile.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float e4m3_value(uint8_t code) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h2) : "r"((uint32_t)code));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+__device__ __forceinline__ uint32_t e2m1x2(float hi, float lo) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\tcvt.u32.u8 %0, b;\n\t}" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) debug_quant_fp4_kernel(const float *__restrict__ xs, int n_rows,
+                                                              uint8_t *__restrict__ codes, uint8_t *__restrict__ sf,
+                                                              float *__restrict__ g_out) {
+    constexpr int VEC = D / 32, LPB = 16 / VEC;  // lanes per 16-channel block
+    __shared__ float s_max[8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r0 = blockIdx.x * kTile + warp * 16;
+    float x[16][VEC];
+    float am = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int r = r0 + i;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+            x[i][v] = (r < n_rows) ? xs[(size_t)r * D + lane * VEC + v] : 0.f;
+            am = fmaxf(am, fabsf(x[i][v]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+    if (lane == 0) s_max[warp] = am;
+    __syncthreads();
+    float tile_max = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tile_max = fmaxf(tile_max, s_max[w]);
+    const float g = (tile_max == 0.f) ? 1.f : __fdiv_rn(tile_max, 2688.f);
+    if (threadIdx.x == 0) g_out[blockIdx.x] = g;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float bm = 0.f;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) bm = fmaxf(bm, fabsf(x[i][v]));
+#pragma unroll
+        for (int o = 1; o < LPB; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, o));
+        uint8_t sc = 0x38;
+        if (bm != 0.f) {
+            sc = (uint8_t)(pack_e4m3x4(__fdiv_rn(__fdiv_rn(bm, g), 6.f), 0.f, 0.f, 0.f) & 0xFFu);
+            if ((sc & 0x7F) == 0) sc = 0x01;
+        }
+        const float delta = __fmul_rn(g, e4m3_value(sc));
+        const size_t row = (size_t)(r0 + i);
+        if (lane % LPB == 0) sf[row * (D / 16) + lane / LPB] = sc;
+        uint32_t packed = 0;  // VEC codes, 4 bits each, channel lane*VEC + v at bits 4v
+#pragma unroll
+        for (int v = 0; v < VEC; v += 2)
+            packed |= e2m1x2(__fdiv_rn(x[i][v + 1], delta), __fdiv_rn(x[i][v], delta)) << (4 * v);
+        uint8_t *dst = codes + row * (D / 2) + lane * (VEC / 2);
+        if constexpr (VEC == 4) *reinterpret_cast<uint16_t *>(dst) = (uint16_t)packed;
+        else *dst = (uint8_t)packed;
+    }
+}
+
+cudaError_t launch_debug_quant_fp4(const float *xs, int n_rows, int d, uint8_t *codes, uint8_t *sf, float *g,
+                                   cudaStream_t stream) {
+    const int tiles = (n_rows + kTile - 1) / kTile;
+    if (d == 128) debug_quant_fp4_kernel<128><<<tiles, 256, 0, stream>>>(xs, n_rows, codes, sf, g);
+    else debug_quant_fp4_kernel<64><<<tiles, 256, 0, stream>>>(xs, n_rows, codes, sf, g);
+    return cudaGetLastError();
+}
 
 template <int KIND>
 __global__ void __launch_bounds__(128, 1) debug_mma_rate_kernel(int n_iter, int *status) {

@@ -549,6 +549,16 @@ sage_status_t sage_debug_mma_rate(int kind, int n_iter, int n_ctas, void *status
                : SAGE_ERR_CUDA;
 }
 
+sage_status_t sage_debug_quant_fp4(const float *xs, int n_rows, int d, uint8_t *codes, uint8_t *sf, float *g,
+                                   void *stream) {
+    if (!xs || !codes || !sf || !g || n_rows < 1 || n_rows > (1 << 24)) return SAGE_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
+    if (!aligned16(xs)) return SAGE_ERR_UNSUPPORTED;
+    return launch_debug_quant_fp4(xs, n_rows, d, codes, sf, g, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SAGE_OK
+               : SAGE_ERR_CUDA;
+}
+
 sage_status_t sage_debug_attn_fault_inject(void *o, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
                                            int causal, const void *workspace, size_t workspace_bytes,
                                            void *stream) {
