@@ -8,6 +8,16 @@ every call raises.
 
     import torch, quantized_attention_fine_b200 as sage
     o = sage.attn_fwd(q, k, v, causal=True)          # q, k, v: [B, H, N, d] bf16/fp16
+    o = sage.attn_fwd(q, k, v, layout="NHD")         # [B, N, H, d]
+    o = sage.attn_fwd(q, k_gqa, v_gqa)               # k, v with H_kv heads, H_kv | H
+    o, lse = sage.attn_fwd(q, k, v, return_lse=True) # row log-sum-exp [B, H, N_q]
+    o = sage.attn_fwd(q, k, v, pv="fp16")            # the qk_int8_pv_fp16 mode
+    o = sage.attn_fwd_varlen(q_packed, k_packed, v_packed, cu_q, cu_kv, causal=True)
+    attn = sage.SageAttention(head_dim=128, is_causal=True, quant_mode="qk_int8_pv_fp8")
+    o = attn(q, k, v)                                # drop-in for a model's attention call
+
+Workspaces (sage.make_workspace) can be kept across calls; a whole call can be
+captured in a CUDA graph.
 
 Method: "SageAttention2" (arXiv 2411.10958) with the per-channel FP8 V scaling and
 P range of SageAttention2++ (arXiv 2505.21136); see include/sage.h.
