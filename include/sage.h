@@ -202,8 +202,8 @@ SAGE_API sage_status_t sage_attn_fwd_varlen(const void *q, const void *k, const 
  * counterpart of this entry point.
  *   - Scratch: one 64 MiB device array inside the library, reserved on every GPU
  *     the library is loaded on and held until the process exits.  Problems whose
- *     sage_workspace_bytes(...) exceeds 64 MiB - 1 KiB are refused with
- *     SAGE_ERR_WORKSPACE before anything is enqueued.
+ *     sage_workspace_bytes_mode(B, H, H, n_q, n_kv, d, mode) exceeds 64 MiB - 1 KiB
+ *     are refused with SAGE_ERR_WORKSPACE before anything is enqueued.
  *   - Allocates nothing: no cudaMalloc / cudaFree or allocating library call.
  *   - The first call on a device looks up the array's device address; make that
  *     first call before any stream capture.
