@@ -311,3 +311,26 @@ def test_suffix_prefill_over_cached_prefix():
         assert cos(to_np64(o[0, h]), ref) >= O_COS_FULL
         # the suffix rows of the full prefill see the same keys; Q smoothing blocks differ
         assert cos(to_np64(o[0, h]), to_np64(o_full[0, h, n_pre:])) >= 0.999
+
+
+def test_head_blocks_with_a_partial_last_block():
+    """H = 20 heads of N = 16384 (d = 128): K / V^T codes of 4 MB per head put 12 heads in
+    a block of the CTA order, so the order has a full block of 12 and a last block of 8.
+    Heads on both sides of the boundary match the oracle on sampled Q blocks, and the
+    launch is deterministic."""
+    H, n, d = 20, 16384, 128
+    w = wl.custom("head_blocks", 1, H, n, n, d, True, recipe="llm", seed=9950)
+    q, k, v = wl.generate(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o1 = sage.attn_fwd(qd, kd, vd, causal=True)
+    o2 = sage.attn_fwd(qd, kd, vd, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+    o = o1.cpu()
+    tq = n // 128
+    for h in (0, 11, 12, 19):
+        pre = oracle.prepass_head(to_np64(q[0, h]), to_np64(k[0, h]), to_np64(v[0, h]))
+        blocks = [0, tq // 2, tq - 1]
+        oo = oracle.attn_head(pre, causal=True, qblocks=blocks)
+        rows = np.concatenate([np.arange(t * 128, t * 128 + 128) for t in blocks])
+        assert_close_to_oracle(to_np64(o[0, h])[rows], oo[rows], "head %d" % h)

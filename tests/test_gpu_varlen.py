@@ -126,3 +126,19 @@ def test_varlen_uncovered_tokens_untouched_and_long_batch_deterministic():
             oo = oracle.attn_head(pre, causal=True, qblocks=[tq - 1])
             rows = np.arange((tq - 1) * 128, n)
             assert_close_to_oracle(o[q0 + rows, h], oo[rows], "seq %d head %d" % (b, h))
+
+
+def test_varlen_fp16_inputs_d64():
+    lq = [129, 1, 640, 77]
+    lk = [300, 64, 640, 77]
+    H, Hk, d = 4, 4, 64
+    q, k, v, cu_q, cu_k = _packed(lq, lk, H, Hk, d, seed=9960, dtype=torch.float16)
+    o = sage.attn_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(cu_q).cuda(),
+                             torch.from_numpy(cu_k).cuda(), causal=True)
+    assert o.dtype == torch.float16
+    o = to_np64(o)
+    oo = oracle.sage_attention_varlen(to_np64(q), to_np64(k), to_np64(v), cu_q, cu_k, causal=True)
+    for b in range(len(lq)):
+        q0, q1 = cu_q[b], cu_q[b + 1]
+        for h in range(H):
+            assert_close_to_oracle(o[q0:q1, h], oo[q0:q1, h], "seq %d head %d" % (b, h))
