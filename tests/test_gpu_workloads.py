@@ -77,3 +77,28 @@ def test_full_size_workload_sampled(name):
         assert_close_to_oracle(og, oo[rows], "%s head (%d,%d)" % (name, b, h))
         ref = _full_precision_rows(qh, kh, vh, rows, w.causal)
         assert cos(og, ref) >= O_COS_FULL, "%s: cos vs full precision %.5f" % (name, cos(og, ref))
+        # the rows' log-sum-exp of the same blocks
+        ll = oracle.lse_head(pre, causal=w.causal, qblocks=blocks)
+        lg = ws.lse()[b, h].cpu().double().numpy()[rows]
+        assert np.max(np.abs(lg - ll[rows])) <= 1e-3, "%s: LSE" % name
+
+
+def test_full_size_fp16_pv_mode_sampled():
+    """The FP16 P / V mode at the llm_prefill size, in the launch configuration of
+    `bench.py --pv fp16`: sampled heads and Q blocks against the oracle's PV_FP16 mode."""
+    w = wl.LLM_PREFILL
+    q, k, v = wl.generate(w)
+    dev = torch.device("cuda", 0)
+    ws = sage.make_workspace(w.B, w.H, w.N_q, w.N_kv, w.d, device=dev, pv_fp16=True)
+    o = sage.attn_fwd(q.to(dev), k.to(dev), v.to(dev), causal=True, pv="fp16", workspace=ws)
+    assert sage.get_device_status(ws) == (0, 0)
+    tq = w.N_q // 128
+    blocks = [0, tq // 2, tq - 1]
+    rows = rows_of_blocks(w.N_q, blocks)
+    for h in (0, w.H - 1):
+        qh, kh, vh = to_np64(q[0, h]), to_np64(k[0, h]), to_np64(v[0, h])
+        pre = oracle.prepass_head(qh, kh, vh, quant=oracle.PV_FP16)
+        oo = oracle.attn_head(pre, causal=True, qblocks=blocks)
+        og = to_np64(o[0, h].cpu())[rows]
+        assert_close_to_oracle(og, oo[rows], "pv16 head %d" % h)
+        assert cos(og, _full_precision_rows(qh, kh, vh, rows, True)) >= O_COS_FULL
