@@ -15,10 +15,13 @@ Method sources (page title and section):
     P range Pr, the Pr x Vr <= 2047/2 bound of the FP16-accumulator variant.
 
 Parity status of each function is stated in its docstring; the pins live in
-``tests/test_oracle_pins.py``.
+``tests/test_oracle_pins.py``.  ``tests/test_oracle_mutations.py`` plants mistakes in
+the C code (built with ORACLE_MUTATION = k, selected by the environment variable
+SAGE_ORACLE_MUTATION, which nothing else sets) and checks that the pins reject each.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
@@ -36,18 +39,21 @@ _lib = None
 TILE = 128
 
 
-def build(force: bool = False) -> str:
-    """Compile sage_oracle.c into oracle/_build/libsage_oracle.so (gcc, OpenMP)."""
+def build(force: bool = False, mutation: int = 0) -> str:
+    """Compile sage_oracle.c into oracle/_build/libsage_oracle.so (gcc, OpenMP).
+    mutation > 0 builds, beside it, the oracle with planted mistake `mutation` (see
+    ORACLE_MUTATION in sage_oracle.c); only the pins' own tests use those builds."""
     os.makedirs(_BUILD, exist_ok=True)
-    if (not force and os.path.exists(_LIB_PATH)
-            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
-        return _LIB_PATH
-    tmp = _LIB_PATH + ".tmp%d" % os.getpid()
+    path = _LIB_PATH if mutation == 0 else os.path.join(_BUILD, "libsage_oracle_mut%d.so" % mutation)
+    if (not force and os.path.exists(path)
+            and os.path.getmtime(path) >= os.path.getmtime(_SRC)):
+        return path
+    tmp = path + ".tmp%d" % os.getpid()
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
-           "-ffp-contract=off", "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+           "-ffp-contract=off", "-fno-fast-math", "-DORACLE_MUTATION=%d" % mutation, "-o", tmp, _SRC, "-lm"]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, _LIB_PATH)
-    return _LIB_PATH
+    os.replace(tmp, path)
+    return path
 
 
 class _Cfg(ctypes.Structure):
@@ -59,35 +65,54 @@ class _Cfg(ctypes.Structure):
                 ("sm_scale", ctypes.c_double), ("causal", ctypes.c_int)]
 
 
+def _configure(lib):
+    P = ctypes.c_void_p
+    lib.oracle_e4m3_from_f32.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_from_f32.restype = ctypes.c_uint8
+    lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_to_f64.restype = ctypes.c_double
+    lib.oracle_int8_code.argtypes = [ctypes.c_float, ctypes.c_float]
+    lib.oracle_int8_code.restype = ctypes.c_int8
+    lib.oracle_int8_scale.argtypes = [ctypes.c_float]
+    lib.oracle_int8_scale.restype = ctypes.c_float
+    lib.oracle_f16_round.argtypes = [ctypes.c_float]
+    lib.oracle_f16_round.restype = ctypes.c_double
+    lib.oracle_prepass.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 17
+    lib.oracle_e2m1_from_f32.argtypes = [ctypes.c_float]
+    lib.oracle_e2m1_from_f32.restype = ctypes.c_uint8
+    lib.oracle_e2m1_to_f64.argtypes = [ctypes.c_uint8]
+    lib.oracle_e2m1_to_f64.restype = ctypes.c_double
+    lib.oracle_prepass.restype = ctypes.c_int
+    lib.oracle_attn.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 9 + [ctypes.c_int, P, P, P]
+    lib.oracle_attn.restype = ctypes.c_int
+    lib.oracle_ref_attn.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double, ctypes.c_int, P, P, P, P]
+    lib.oracle_ref_attn.restype = ctypes.c_int
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
-            P = ctypes.c_void_p
-            lib.oracle_e4m3_from_f32.argtypes = [ctypes.c_float]
-            lib.oracle_e4m3_from_f32.restype = ctypes.c_uint8
-            lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
-            lib.oracle_e4m3_to_f64.restype = ctypes.c_double
-            lib.oracle_int8_code.argtypes = [ctypes.c_float, ctypes.c_float]
-            lib.oracle_int8_code.restype = ctypes.c_int8
-            lib.oracle_int8_scale.argtypes = [ctypes.c_float]
-            lib.oracle_int8_scale.restype = ctypes.c_float
-            lib.oracle_f16_round.argtypes = [ctypes.c_float]
-            lib.oracle_f16_round.restype = ctypes.c_double
-            lib.oracle_prepass.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 17
-            lib.oracle_e2m1_from_f32.argtypes = [ctypes.c_float]
-            lib.oracle_e2m1_from_f32.restype = ctypes.c_uint8
-            lib.oracle_e2m1_to_f64.argtypes = [ctypes.c_uint8]
-            lib.oracle_e2m1_to_f64.restype = ctypes.c_double
-            lib.oracle_prepass.restype = ctypes.c_int
-            lib.oracle_attn.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 9 + [ctypes.c_int, P, P, P]
-            lib.oracle_attn.restype = ctypes.c_int
-            lib.oracle_ref_attn.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double, ctypes.c_int, P, P, P, P]
-            lib.oracle_ref_attn.restype = ctypes.c_int
-            lib.oracle_num_threads.restype = ctypes.c_int
-            _lib = lib
+            # SAGE_ORACLE_MUTATION selects a planted mistake, for the pins' own tests
+            _lib = _configure(ctypes.CDLL(build(mutation=int(os.environ.get("SAGE_ORACLE_MUTATION", "0")))))
     return _lib
+
+
+@contextlib.contextmanager
+def mutant(mutation: int):
+    """Run the oracle with planted mistake `mutation` inside the block (tests of the
+    pins only)."""
+    global _lib
+    lib = _configure(ctypes.CDLL(build(mutation=mutation)))
+    with _lock:
+        saved, _lib = _lib, lib
+    try:
+        yield
+    finally:
+        with _lock:
+            _lib = saved
 
 
 def _ptr(a: np.ndarray):

@@ -56,6 +56,14 @@
 
 #define ORACLE_TILE 128 /* Q block rows and KV tile keys; part of the numerics */
 
+/* Planted mistakes for the pins' own tests (tests/test_oracle_mutations.py): a build
+ * with ORACLE_MUTATION = k > 0 computes the method with mistake k, which at least one
+ * pin must then reject.  The default build (0) compiles every mutation away. */
+#ifndef ORACLE_MUTATION
+#define ORACLE_MUTATION 0
+#endif
+#define MUT(k) (ORACLE_MUTATION == (k))
+
 typedef struct {
     int n_q, n_kv, d;
     int g_q, g_k;         /* INT8 group sizes (rows of a Q block, keys of a KV tile) */
@@ -95,7 +103,7 @@ uint8_t oracle_e4m3_from_f32(float xf)
         double fr = frexp(a, &e);     /* a = fr * 2^e, fr in [0.5, 1) */
         int ex = e - 1;               /* a = (2 fr) * 2^ex, 2 fr in [1, 2) */
         double mant = (2.0 * fr - 1.0) * 8.0;  /* exact */
-        double q = nearbyint(mant);
+        double q = MUT(1) ? floor(mant + 0.5) : nearbyint(mant);   /* 1: E4M3 ties away from 0 */
         if (q >= 8.0) { q = 0.0; ex += 1; }
         int be = ex + 7;
         if (be > 15 || (be == 15 && q >= 7.0)) return (uint8_t)(sign | 0x7E);
@@ -130,7 +138,7 @@ double oracle_f16_round(float xf)
     int q = e - 11;               /* spacing of 11 significant bits */
     if (q < -24) q = -24;         /* subnormal spacing */
     double step = ldexp(1.0, q);
-    return copysign(nearbyint(a / step) * step, x);
+    return copysign((MUT(2) ? trunc(a / step) : nearbyint(a / step)) * step, x);   /* 2: fp16 truncates */
 }
 
 /* E2M1 (4-bit: 1 sign, 2 exponent bits with bias 1, 1 mantissa bit; magnitudes
@@ -153,7 +161,7 @@ uint8_t oracle_e2m1_from_f32(float xf)
     int best = 0;
     for (int i = 1; i < 8; ++i) {
         double di = fabs(a - oracle_e2m1_mag[i]), db = fabs(a - oracle_e2m1_mag[best]);
-        if (di < db || (di == db && (i & 1) == 0)) best = i;  /* ties: even mantissa */
+        if (di < db || (di == db && (MUT(3) || (i & 1) == 0))) best = i;  /* ties: even mantissa (3: upward) */
     }
     return (uint8_t)(sign | best);
 }
@@ -206,7 +214,7 @@ static float oracle_fp4_tile(const float *xs, int d, int8_t *code, double *hat, 
 int8_t oracle_int8_code(float xs, float delta)
 {
     float r = xs / delta;
-    float n = nearbyintf(r);
+    float n = MUT(4) ? truncf(r) : nearbyintf(r);   /* 4: INT8 codes truncate */
     if (n > 127.0f) n = 127.0f;
     if (n < -127.0f) n = -127.0f;
     return (int8_t)n;
@@ -254,7 +262,7 @@ int oracle_prepass(const oracle_cfg_t *cfg, const double *q, const double *k, co
             double s = 0.0;
             if (cfg->smooth_q) {
                 for (int i = r0; i < r1; ++i) s += q[(size_t)i * d + c];
-                s /= (double)(r1 - r0);
+                s /= (double)(MUT(5) ? ORACLE_TILE : r1 - r0);   /* 5: ragged block mean over 128 rows */
             }
             qbar[(size_t)t * d + c] = (float)s;
         }
@@ -313,7 +321,7 @@ int oracle_prepass(const oracle_cfg_t *cfg, const double *q, const double *k, co
     }
     for (int j = 0; j < nk; ++j)
         for (int c = 0; c < d; ++c)
-            k_s[(size_t)j * d + c] = k[(size_t)j * d + c] - (double)kbar[c];
+            k_s[(size_t)j * d + c] = k[(size_t)j * d + c] + (MUT(6) ? 1.0 : -1.0) * (double)kbar[c];   /* 6: sign */
     /* --- K: FP4 codes with two-level scales per 128-key tile --- */
     if (cfg->quant_qk == 2) {
         float *ks = (float *)malloc(sizeof(float) * (size_t)ORACLE_TILE * d);
@@ -364,7 +372,7 @@ int oracle_prepass(const oracle_cfg_t *cfg, const double *q, const double *k, co
             float a = fabsf((float)v[(size_t)j * d + c]);
             if (a > amax) amax = a;
         }
-        dv[c] = (amax == 0.0f || cfg->quant_v == 2) ? 1.0f : amax / vr;
+        dv[c] = (amax == 0.0f || cfg->quant_v == 2) ? 1.0f : (MUT(7) ? amax * vr : amax / vr);   /* 7 */
     }
     for (int j = 0; j < nk; ++j)
         for (int c = 0; c < d; ++c) {
@@ -423,7 +431,7 @@ int oracle_attn(const oracle_cfg_t *cfg, const float *qbar, const double *q_hat,
         for (int j = 0; j < nk; ++j) {
             double s = 0.0;
             for (int c = 0; c < d; ++c) s += (double)qbar[(size_t)t * d + c] * k_s[(size_t)j * d + c];
-            ds[j] = s;
+            ds[j] = MUT(8) ? -s : s;   /* 8: dS sign */
         }
         #pragma omp parallel for schedule(dynamic, 4)
         for (int i = r0; i < r1; ++i) {
@@ -436,14 +444,14 @@ int oracle_attn(const oracle_cfg_t *cfg, const float *qbar, const double *q_hat,
                 double tmax = -INFINITY;
                 int any = 0;
                 for (int j = j0; j < j1; ++j) {
-                    int visible = !cfg->causal || (long)j <= (long)i + off;
+                    int visible = !cfg->causal || (MUT(9) ? (long)j < (long)i + off : (long)j <= (long)i + off);
                     vis[j - j0] = (char)visible;
                     if (!visible) continue;
                     double dot = 0.0;
                     for (int c = 0; c < d; ++c) dot += q_hat[(size_t)i * d + c] * k_hat[(size_t)j * d + c];
                     double s = (double)dq_row[i] * (double)dk_key[j] * dot + ds[j];
                     x[j - j0] = s * cfg->sm_scale;
-                    if (x[j - j0] > tmax) tmax = x[j - j0];
+                    if (x[j - j0] > tmax && !(MUT(10) && j == j1 - 1)) tmax = x[j - j0];   /* 10: last key missed */
                     any = 1;
                 }
                 if (!any) continue; /* tile fully masked for this row: skipped */
@@ -463,7 +471,7 @@ int oracle_attn(const oracle_cfg_t *cfg, const float *qbar, const double *q_hat,
                 m = mn;
             }
             for (int c = 0; c < d; ++c)
-                o[(size_t)i * d + c] = (l > 0.0) ? acc[c] / pr * (double)dv[c] / l : 0.0;
+                o[(size_t)i * d + c] = (l > 0.0) ? acc[c] / (MUT(11) ? 1.0 : pr) * (double)dv[c] / l : 0.0;   /* 11 */
             if (row_l) row_l[i] = l;
             if (row_m) row_m[i] = m;
             free(acc); free(x); free(vis);

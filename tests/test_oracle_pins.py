@@ -668,3 +668,13 @@ def test_fp4_qk_accuracy_and_smoothing():
 def cos_np(a, b):
     a, b = np.ravel(a), np.ravel(b)
     return float(a @ b / math.sqrt((a @ a) * (b @ b)))
+
+
+def test_q_block_means_of_ragged_blocks():
+    """q̄ of each 128-row block is the fp64 mean of its valid rows (numpy), rounded once
+    to fp32: the ragged last block averages its 72 rows, not 128."""
+    q, k, v = _rand_head(200, 130, 64, seed=88, qbias=2.0)
+    pre = oracle.prepass_head(q, k, v)
+    for t, (r0, r1) in enumerate(((0, 128), (128, 200))):
+        assert np.array_equal(pre["qbar"][t], q[r0:r1].mean(axis=0).astype(np.float32))
+    assert np.array_equal(pre["kbar"], k.mean(axis=0).astype(np.float32))
