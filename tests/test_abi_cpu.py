@@ -164,3 +164,31 @@ def test_python_binding_has_no_fallback(monkeypatch, tmp_path):
     monkeypatch.setattr(sage, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         sage.load_library()
+
+
+def test_varlen_and_mode_argument_errors_return_synchronously(lib):
+    """Argument checks of the packed-batch entry point and of the quantization mode:
+    each returns before any CUDA call (so they run here, without a GPU)."""
+    P, I = ctypes.c_void_p, ctypes.c_int
+    fake = P(1 << 20)
+    assert lib.sage_workspace_bytes_varlen(3, 8, 2, 700, 900, 128) == lib.sage_workspace_bytes_gqa(3, 8, 2, 700, 900,
+                                                                                                   128)
+    f = lib.sage_attn_fwd_varlen
+    args = lambda **kw: [kw.get("q", fake), fake, fake, fake, kw.get("dtype", 1), kw.get("cu_q", fake),
+                         kw.get("cu_kv", fake), kw.get("B", 2), 8, kw.get("Hk", 2), kw.get("tq", 100),
+                         kw.get("tk", 100), 64, 64, kw.get("d", 64), 1, 0.0, kw.get("mode", None), fake, 1 << 30,
+                         None]
+    assert f(*args(cu_q=None)) == 1                     # offsets are required
+    assert f(*args(cu_kv=None)) == 1
+    assert f(*args(tq=-1)) == 1                         # negative totals
+    assert f(*args(Hk=3)) == 1                          # 3 does not divide 8
+    assert f(*args(d=96)) == 2                          # head dim
+    assert f(*args(dtype=5)) == 1                       # dtype
+    assert f(*args(q=P((1 << 20) + 4))) == 2            # misaligned
+    assert f(*args(B=0)) == 0 and f(*args(tq=0)) == 0   # nothing to do
+    bad = sage.QuantMode.make()
+    bad.pv_fp16 = 3
+    assert f(*args(mode=ctypes.byref(bad))) == 1
+    bad = sage.QuantMode.make()
+    bad.p_range = 500.0                                 # beyond the E4M3 range
+    assert f(*args(mode=ctypes.byref(bad))) == 1
