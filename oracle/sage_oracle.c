@@ -183,7 +183,7 @@ static float oracle_fp4_tile(const float *xs, int d, int8_t *code, double *hat, 
         float a = fabsf(xs[i]);
         if (a > amax) amax = a;
     }
-    const float g = (amax == 0.0f) ? 1.0f : amax / 2688.0f;
+    const float g = (amax == 0.0f) ? 1.0f : amax / (MUT(12) ? 6.0f : 2688.0f);   /* 12: no E4M3 headroom */
     for (int r = 0; r < ORACLE_TILE; ++r)
         for (int b0 = 0; b0 < d; b0 += 16) {
             float am = 0.0f;
@@ -194,7 +194,7 @@ static float oracle_fp4_tile(const float *xs, int d, int8_t *code, double *hat, 
             uint8_t sc = 0x38;  /* 1.0 */
             if (am != 0.0f) {
                 sc = oracle_e4m3_from_f32((am / g) / 6.0f);
-                if ((sc & 0x7F) == 0) sc = 0x01;
+                if ((sc & 0x7F) == 0 && !MUT(13)) sc = 0x01;   /* 13: an underflowing scale stays 0 */
             }
             sf_code[(size_t)r * (d / 16) + b0 / 16] = sc;
             const double sfv = oracle_e4m3_to_f64(sc);

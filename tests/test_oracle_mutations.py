@@ -25,6 +25,8 @@ MUTATIONS = {
     9: "causal mask off by one",
     10: "the last key of a tile is missed by the running max",
     11: "the 1 / Pr of the output dropped",
+    12: "FP4 tile scale g = amax / 6 (no E4M3 headroom for the block scales)",
+    13: "an FP4 block scale that underflows E4M3 stays 0",
 }
 
 

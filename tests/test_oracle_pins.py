@@ -622,6 +622,54 @@ def test_fp4_block_scales_reconstruct_within_half_a_code_step():
     assert np.all((blk_max >= 4) | (xs_max == 0))
 
 
+def test_fp4_tile_scale_puts_the_largest_block_at_the_top_of_e4m3():
+    """The per-tile fp32 scale g exists to keep the E4M3 block scales in range while
+    using all of it (the microscaling form of 4-bit operands, "SageAttention3:
+    Microscaling FP4 Attention" in the notes' related-papers table; the 4-bit QK of the
+    SageAttention2 abstract): in every 128-row tile with a nonzero entry, the 16-channel
+    block that holds the tile's largest magnitude gets the largest finite E4M3 scale,
+    448 (code 0x7E), and its largest element codes to E2M1 6, so that g = amax / 2688
+    follows from 6 * 448 * g = amax.  Checked on Q (three tiles, one ragged) and K."""
+    q, k, v = _rand_head(300, 270, 128, seed=57, kbias=3.0, qbias=1.0)
+    pre = oracle.prepass_head(q, k, v, quant=oracle.QK_FP4_PV_FP8)
+    for x, bar, sf_all, code_all, n in (
+            (q, np.repeat(pre["qbar"].astype(np.float64), 128, axis=0), pre["q_sf"], pre["q_code"], 300),
+            (k, pre["kbar"].astype(np.float64)[None, :], pre["k_sf"], pre["k_code"], 270)):
+        xs = np.zeros((-(-n // 128) * 128, 128), np.float32)
+        xs[:n] = (x - bar[:n] if bar.shape[0] > 1 else x - bar).astype(np.float32)
+        for t in range(xs.shape[0] // 128):
+            tile = np.abs(xs[128 * t:128 * (t + 1)])
+            r, c = np.unravel_index(np.argmax(tile), tile.shape)
+            assert tile[r, c] > 0
+            assert sf_all[128 * t + r, c // 16] == 0x7E
+            assert oracle.e2m1_decode(code_all[128 * t + r, c]) in (6.0, -6.0)
+            # no block scale exceeds the top one
+            assert np.all(np.array([[oracle.e4m3_decode(s) for s in row]
+                                    for row in sf_all[128 * t:128 * (t + 1)]]) <= 448.0)
+
+
+def test_fp4_block_scale_that_underflows_e4m3_is_the_smallest_subnormal():
+    """A 16-channel block far below the tile maximum has amax / g / 6 below half of
+    E4M3's smallest subnormal 2^-9, which rounds to 0; a zero scale would divide by 0,
+    so the block takes the smallest positive scale 2^-9 (code 0x01) and its elements
+    code to 0.  Crafted tile: one entry 1000, one block with entries of 1e-6, the rest 0
+    (an all-zero block keeps the scale 1.0, code 0x38)."""
+    nq, d = 128, 64
+    q = np.zeros((nq, d))
+    q[3, 5] = 1000.0
+    q[70, 16:32] = 1e-6
+    k = np.eye(128, d)
+    v = np.ones((128, d))
+    pre = oracle.prepass_head(q, k, v, quant=oracle.QK_FP4_PV_FP8, smooth_q=False)
+    g = 1000.0 / 2688.0
+    assert (1e-6 / g) / 6 < 2.0 ** -10          # rounds to E4M3 zero
+    assert pre["q_sf"][70, 1] == 0x01
+    assert oracle.e4m3_decode(0x01) == 2.0 ** -9
+    assert np.all(oracle.e2m1_decode(pre["q_code"][70, 16:32]) == 0.0)
+    assert pre["q_sf"][3, 0] == 0x7E
+    assert pre["q_sf"][70, 0] == 0x38 and pre["q_sf"][0, 2] == 0x38
+
+
 def test_fp4_scores_equal_attention_on_dequantized_q_k():
     """With FP4 Q / K and exact P / V, the oracle is textbook attention on the
     dequantized smoothed operands plus the Q-smoothing bias (numpy, from the pre-pass
