@@ -200,21 +200,34 @@ SAGE_API sage_status_t sage_attn_fwd_varlen(const void *q, const void *k, const 
  * allocation, or a serving loop where a cudaMalloc, which can synchronize the
  * device, is not acceptable) and so cannot provide a workspace.  The pages have no
  * counterpart of this entry point.
- *   - Scratch: one 64 MiB device array inside the library, reserved on every GPU
- *     the library is loaded on and held until the process exits.  Problems whose
+ *   - Scratch: one 64 MiB device array inside the library, held on every GPU where
+ *     the library's device code is loaded, until the process exits.  Problems whose
  *     sage_workspace_bytes_mode(B, H, H, n_q, n_kv, d, mode) exceeds 64 MiB - 1 KiB
  *     are refused with SAGE_ERR_WORKSPACE before anything is enqueued.
- *   - Allocates nothing: no cudaMalloc / cudaFree or allocating library call.
- *   - The first call on a device looks up the array's device address; make that
- *     first call before any stream capture.
+ *   - Allocates nothing itself: no cudaMalloc / cudaFree or allocating library call.
+ *     Under CUDA's default lazy module loading, though, the array is reserved when
+ *     the library's device code is first used on a device, and that first use may
+ *     allocate and synchronize inside the CUDA runtime.  So make one call on each
+ *     device at initialisation, before any stream capture: a call with B = 0 (all
+ *     other arguments valid, pointers may be NULL) reserves the array and looks up
+ *     its address without enqueueing any work.
  *   - All calls on a device share the array, which keeps the previous call's
  *     contents (the status block is cleared at the start of each call).  Calls
  *     that overlap on the GPU (other streams, other host threads) race with each
  *     other: serialize them.
- *   - Arguments, layouts and errors otherwise as sage_attn_fwd. */
+ *   - A device-side wait that runs out is recorded in the array's status block:
+ *     read it with sage_noalloc_get_device_status.
+ *   - Arguments, layouts and errors otherwise as sage_attn_fwd; argument errors are
+ *     returned before anything is enqueued. */
 SAGE_API sage_status_t sage_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *o, int dtype,
                                              int layout, int B, int H, int n_q, int n_kv, int d, int causal,
                                              float sm_scale, const sage_quant_mode_t *mode, void *stream);
+
+/* sage_get_device_status for the scratch array of sage_attn_fwd_noalloc on the
+ * current device: synchronizes `stream`, reads and clears the status block of the
+ * array.  *code: SAGE_OK or the first device-side error (SAGE_ERR_TIMEOUT) of the
+ * calls since the last read; *site: the id of the wait that ran out (0 if none). */
+SAGE_API sage_status_t sage_noalloc_get_device_status(void *stream, int *code, int *site);
 
 /* Synchronizes `stream`, copies the workspace status block to the host and clears
  * it.  *code receives SAGE_OK or the first device-side error (SAGE_ERR_TIMEOUT);
@@ -316,7 +329,10 @@ SAGE_API sage_status_t sage_debug_quant_fp4(const float *xs, int n_rows, int d, 
 
 /* Runs the attention kernel with one deliberately missing producer signal so that
  * the consumer's bounded wait must run out; the kernel records SAGE_ERR_TIMEOUT in
- * the status block and exits without hanging.  Arguments as sage_attn_fwd_prequant. */
+ * the status block and exits without hanging.  Arguments as sage_attn_fwd_prequant;
+ * workspace NULL runs it on the scratch array of sage_attn_fwd_noalloc (as the last
+ * call on the current device left it), whose status block
+ * sage_noalloc_get_device_status reads. */
 SAGE_API sage_status_t sage_debug_attn_fault_inject(void *o, int dtype, int layout, int B, int H,
                                                     int n_q, int n_kv, int d, int causal,
                                                     const void *workspace, size_t workspace_bytes,

@@ -301,6 +301,33 @@ sage_status_t check_common(int dtype, int layout) {
 
 }  // namespace
 
+namespace sage {
+
+sage_status_t check_fwd_args(const void *q, const void *k, const void *v, const void *o, int dtype, int layout,
+                             int B, int H, int H_kv, int n_q, int n_kv, int d, const sage_quant_mode_t *mode,
+                             int *plan, size_t *ws_need) {
+    Shape s;
+    Mode m;
+    *plan = kFwdNoop;
+    *ws_need = 0;
+    SAGE_TRY(check_common(dtype, layout));
+    SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
+    SAGE_TRY(read_mode(mode, &m));
+    s.pv16 = m.pv16;
+    if (s.BH == 0 || n_q == 0) return SAGE_OK;
+    if (!q || !o || (n_kv > 0 && (!k || !v))) return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(o) || (k && !aligned16(k)) || (v && !aligned16(v))) return SAGE_ERR_UNSUPPORTED;
+    if (n_kv == 0) {
+        *plan = kFwdZeroOut;
+        return SAGE_OK;
+    }
+    *plan = kFwdRun;
+    *ws_need = ws_layout(s).total;
+    return SAGE_OK;
+}
+
+}  // namespace sage
+
 extern "C" {
 
 size_t sage_workspace_bytes_gqa(int B, int H, int H_kv, int n_q, int n_kv, int d) {
@@ -429,17 +456,17 @@ sage_status_t sage_attn_fwd_gqa(const void *q, const void *k, const void *v, voi
                                 int H, int H_kv, int n_q, int n_kv, int d, int causal, float sm_scale,
                                 const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes,
                                 void *stream) {
+    int plan = kFwdNoop;
+    size_t need = 0;
+    SAGE_TRY(check_fwd_args(q, k, v, o, dtype, layout, B, H, H_kv, n_q, n_kv, d, mode, &plan, &need));
+    if (plan == kFwdNoop) return SAGE_OK;
     Shape s;
     Mode m;
-    SAGE_TRY(check_common(dtype, layout));
-    SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
-    SAGE_TRY(read_mode(mode, &m));
+    check_sizes(B, H, H_kv, n_q, n_kv, d, &s);   // both validated by check_fwd_args
+    read_mode(mode, &m);
     s.pv16 = m.pv16;
-    if (s.BH == 0 || n_q == 0) return SAGE_OK;
-    if (!q || !o || (n_kv > 0 && (!k || !v))) return SAGE_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(o) || (k && !aligned16(k)) || (v && !aligned16(v))) return SAGE_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (n_kv == 0)
+    if (plan == kFwdZeroOut)
         return cudaMemsetAsync(o, 0, (size_t)s.BH * n_q * d * 2, st) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
     SAGE_TRY(check_ws(s, workspace, workspace_bytes));
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -568,6 +595,11 @@ sage_status_t sage_debug_attn_fault_inject(void *o, int dtype, int layout, int B
     SAGE_TRY(check_sizes(B, H, H, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(nullptr, &m));
     if (!o || s.BH == 0 || n_q == 0 || n_kv == 0) return SAGE_ERR_INVALID_ARG;
+    if (!workspace) {  // the scratch array of sage_attn_fwd_noalloc, as its last call left it
+        uint8_t *ws = nullptr;
+        SAGE_TRY(noalloc_workspace(&ws, &workspace_bytes));
+        workspace = ws;
+    }
     SAGE_TRY(check_ws(s, workspace, workspace_bytes));
     return run_attention(o, dtype, layout, s, causal, 0.f, m, static_cast<const uint8_t *>(workspace), 1, nullptr,
                          nullptr, static_cast<cudaStream_t>(stream));

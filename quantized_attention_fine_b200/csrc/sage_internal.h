@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/sage.h"
+
 namespace sage {
 
 constexpr int kTile = 128;        // Q block rows = KV tile keys (part of the numerics)
@@ -160,5 +162,18 @@ cudaError_t launch_debug_mma_rate(int kind, int n_iter, int n_ctas, int *status,
 cudaError_t launch_debug_quant_fp4(const float *xs, int n_rows, int d, uint8_t *codes, uint8_t *sf, float *g,
                                    cudaStream_t stream);
 cudaError_t launch_zero_output(void *o, size_t bytes, cudaStream_t stream);
+
+// How a whole-forward call (sage_attn_fwd_gqa's arguments) proceeds once its
+// arguments are valid: nothing to do (B * H == 0 or n_q == 0), O = 0 without a
+// workspace (n_kv == 0), or the full path with a workspace of *ws_need bytes.
+enum FwdPlan { kFwdNoop = 0, kFwdZeroOut = 1, kFwdRun = 2 };
+// Every check sage_attn_fwd_gqa makes before it enqueues anything, in the same order
+// and with the same status; on SAGE_OK also the plan and the workspace size.
+sage_status_t check_fwd_args(const void *q, const void *k, const void *v, const void *o, int dtype, int layout,
+                             int B, int H, int H_kv, int n_q, int n_kv, int d, const sage_quant_mode_t *mode,
+                             int *plan, size_t *ws_need);
+// The scratch array of sage_attn_fwd_noalloc on the current device, 1024-byte
+// aligned, and its usable bytes (the first call on a device looks its address up).
+sage_status_t noalloc_workspace(uint8_t **ws, size_t *bytes);
 
 }  // namespace sage

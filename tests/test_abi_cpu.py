@@ -159,6 +159,27 @@ def test_argument_errors_return_synchronously(lib):
     assert lib.sage_debug_pv_accumulate(fake, fake, 0, 64, fake, None) == 1
 
 
+def test_noalloc_argument_errors_come_before_any_cuda_call(lib):
+    """sage_attn_fwd_noalloc checks its arguments as sage_attn_fwd does before it
+    touches CUDA: with no GPU here, any CUDA call would turn the result into
+    SAGE_ERR_CUDA, so the exact statuses show that nothing was enqueued."""
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fn = lib.sage_attn_fwd_noalloc
+    fn.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, F, ctypes.POINTER(sage.QuantMode), P]
+    fn.restype = I
+    fake = P(1 << 20)
+    assert fn(fake, fake, fake, fake, 7, 0, 1, 1, 128, 128, 64, 0, 0.0, None, None) == 1      # dtype
+    assert fn(fake, fake, fake, fake, 1, 3, 1, 1, 128, 128, 64, 0, 0.0, None, None) == 1      # layout
+    assert fn(fake, fake, fake, fake, 1, 0, 1, 1, 128, 128, 80, 0, 0.0, None, None) == 2      # d
+    assert fn(None, fake, fake, fake, 1, 0, 1, 1, 128, 128, 64, 0, 0.0, None, None) == 1      # null q
+    assert fn(P((1 << 20) + 2), fake, fake, fake, 1, 0, 1, 1, 128, 128, 64, 0, 0.0, None, None) == 2
+    bad = sage.QuantMode(9, 1, 1, 448.0, 448.0)
+    assert fn(fake, fake, fake, fake, 1, 0, 1, 1, 128, 128, 64, 0, 0.0, ctypes.byref(bad), None) == 1
+    # beyond 32-bit TMA coordinates: the unsupported-size status of sage_attn_fwd
+    assert fn(fake, fake, fake, fake, 1, 0, 1 << 16, 1 << 10, 1 << 12, 128, 64, 0, 0.0, None, None) == 2
+    assert lib.sage_noalloc_get_device_status(None, None, None) == 1
+
+
 def test_python_binding_has_no_fallback(monkeypatch, tmp_path):
     monkeypatch.setattr(sage, "_LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(sage, "_lib", None)
