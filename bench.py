@@ -9,9 +9,12 @@ already resident in HBM, through the public C-ABI call sage_attn_fwd: the
 smoothing/quantization pre-pass of Q, K and V, the dS product, and the fused
 attention kernel.  A second timed loop runs the attention kernel alone
 (sage_attn_fwd_prequant on the same workspace) for its roofline figure.  Metric: attention TOPS
-= 4 B H N_q N_kv d / t (halved when causal), summed over all ranks.  With N > 1
-every rank runs the full workload on its own seeded inputs (heads are independent,
-so the path shards with no collective): weak scaling.  Rank 0 prints one JSON line.
+= 4 B H N_q N_kv d / t (halved when causal), summed over all ranks.  With N > 1 the
+ranks compute disjoint slices of one seeded global problem, split by heads (each head's
+K mean, delta_V, dS and O depend on that head alone, so no data-path collective is
+needed): by default the global problem holds N batch blocks of the workload and rank r
+computes block r (weak scaling); --scaling strong splits the workload's own heads into
+N contiguous ranges.  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -56,6 +59,10 @@ def parse_args():
                     help="PV precision: fp8 (the method's default) or fp16 (the qk_int8_pv_fp16 mode)")
     ap.add_argument("--graph", action="store_true",
                     help="time the step as a replay of a CUDA graph that captured one sage_attn_fwd call")
+    ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
+                    help="N > 1: weak = N batch blocks of the workload, one per rank; strong = the workload's "
+                         "heads split across the ranks")
+    ap.add_argument("--no-probe", action="store_true", help="skip the tcgen05.mma rate probe (second denominator)")
     ap.add_argument("--mma-rates", action="store_true",
                     help="print the tensor-core rate of each tcgen05.mma form (diagnostic) and exit")
     return ap.parse_args()
@@ -66,14 +73,71 @@ def dist_env():
 
 
 # ---------------------------------------------------------------------------
-# Multi-rank host logic (weak scaling: every rank runs the whole workload on its own
-# seeded inputs; no data-path collective).  Tested with gloo ranks on the CPU.
+# Multi-rank host logic: every rank computes a disjoint slice of one seeded global
+# problem, split by heads; no data-path collective.  Tested with gloo ranks on the CPU.
+#
+# The unit of work is one key/value head group: key/value head (b, h_kv) with its
+# H / H_kv query heads (one head under multi-head attention).  Units are independent:
+# a head's K mean, delta_V, Q blocks, dS and O use no other head.
+#   weak   the global problem is `world` batch blocks of the workload (B_g = world * B);
+#          block r is drawn from seed + 7919 r, and rank r computes block r.
+#   strong the global problem is the workload; its B * H_kv units are split into
+#          `world` contiguous ranges (world must divide B * H_kv).
 # ---------------------------------------------------------------------------
 def rank_workload(w, rank: int):
-    """The workload with rank's own seed (the inputs differ per rank, the shapes do not)."""
+    """Batch block `rank` of the weak-scaling global problem: the workload drawn from
+    the block's own seed (block 0 is the workload itself)."""
     from quantized_attention_fine_b200 import workloads as wl
     return wl.Workload(w.name, w.B, w.H, w.N_q, w.N_kv, w.d, w.causal, w.dtype, w.seed + 7919 * rank, w.recipe,
                        H_kv=w.H_kv)
+
+
+def unit_range(n_units: int, world: int, rank: int):
+    """Contiguous share [u0, u1) of n_units units for rank of world (world divides n_units)."""
+    if world < 1 or n_units % world:
+        raise ValueError("%d ranks cannot split %d key/value head groups evenly" % (world, n_units))
+    per = n_units // world
+    return rank * per, (rank + 1) * per
+
+
+def global_inputs(w, world: int, scaling: str):
+    """The seeded global problem (q, k, v) of a world-rank run, as one [B_g, H, N, d] batch."""
+    from quantized_attention_fine_b200 import workloads as wl
+    import torch
+    if scaling == "strong":
+        return wl.generate(w)
+    blocks = [wl.generate(rank_workload(w, r)) for r in range(world)]
+    return tuple(torch.cat([b[i] for b in blocks], dim=0) for i in range(3))
+
+
+def rank_inputs(w, world: int, rank: int, scaling: str):
+    """(sub-workload, q, k, v) of rank: its slice of the global problem, drawn without
+    drawing the rest under weak scaling.  Under strong scaling the slice is units
+    [u0, u1) of the workload, returned as one batch of (u1 - u0) * group query heads
+    over (u1 - u0) key/value heads (HND tensors, contiguous)."""
+    from quantized_attention_fine_b200 import workloads as wl
+    if scaling == "weak":
+        wr = rank_workload(w, rank)
+        return (wr,) + tuple(wl.generate(wr))
+    q, k, v = wl.generate(w)
+    group = w.H // w.Hk
+    u0, u1 = unit_range(w.B * w.Hk, world, rank)
+    qs = q.reshape(w.B * w.Hk, group, w.N_q, w.d)[u0:u1].reshape(1, (u1 - u0) * group, w.N_q, w.d).contiguous()
+    ks = k.reshape(w.B * w.Hk, w.N_kv, w.d)[u0:u1].unsqueeze(0).contiguous()
+    vs = v.reshape(w.B * w.Hk, w.N_kv, w.d)[u0:u1].unsqueeze(0).contiguous()
+    sub = wl.Workload(w.name, 1, (u1 - u0) * group, w.N_q, w.N_kv, w.d, w.causal, w.dtype, w.seed, w.recipe,
+                      H_kv=(u1 - u0) if group > 1 else 0)
+    return sub, qs, ks, vs
+
+
+def parallelism_label(w, world: int, scaling: str) -> str:
+    if world == 1:
+        return "one GPU: the whole workload (%d heads)" % (w.B * w.H)
+    if scaling == "weak":
+        return ("heads split, weak: global problem of %d batch blocks (%d heads); rank r computes block r "
+                "(%d heads); no data-path collective" % (world, world * w.B * w.H, w.B * w.H))
+    return ("heads split, strong: the workload's %d heads in %d contiguous ranges of %d; no data-path collective"
+            % (w.B * w.H, world, w.B * w.H // world))
 
 
 def max_over_ranks(values, device="cpu"):
@@ -276,13 +340,12 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     sage.load_library()
 
-    # seeded inputs: each rank draws its own batch (weak scaling)
-    wr = rank_workload(w, rank)
-    q_cpu, k_cpu, v_cpu = wl.generate(wr)
+    # this rank's slice of the seeded global problem
+    wr, q_cpu, k_cpu, v_cpu = rank_inputs(w, world, rank, args.scaling)
     q, k, v = q_cpu.to(dev), k_cpu.to(dev), v_cpu.to(dev)
-    B, H, nq, nk, d = w.B, w.H, w.N_q, w.N_kv, w.d
+    B, H, nq, nk, d = wr.B, wr.H, wr.N_q, wr.N_kv, wr.d
     pv16 = args.pv == "fp16"
-    ws = sage.make_workspace(B, H, nq, nk, d, device=dev, H_kv=w.Hk, pv_fp16=pv16)
+    ws = sage.make_workspace(B, H, nq, nk, d, device=dev, H_kv=wr.Hk, pv_fp16=pv16)
     out = torch.empty_like(q)
     mode = sage.QuantMode.make(pv=args.pv)
     stream = torch.cuda.current_stream(dev)
@@ -341,7 +404,7 @@ def main():
     total_ms, attn_avg_ms = max_over_ranks([total_ms, statistics.mean(attn_ms)], device=dev)
     ms_per_step = total_ms / args.steps
     pre_avg_ms = ms_per_step - attn_avg_ms
-    ops_step = w.ops()
+    ops_step = wr.ops()     # this rank's slice; every rank's slice has the same size
     value = whole_job_tops(world, ops_step, ms_per_step)
     attn_tops = ops_step / (attn_avg_ms * 1e-3) / 1e12
 
@@ -416,15 +479,24 @@ def main():
         peak = 2.0 / (1.0 / (2.0 * bf16_burst) + 1.0 / bf16_burst)
         peak_note = ("%s bf16 burst %.1f: INT8 QK at 2x, FP16 PV at 1x, equal work: harmonic mean"
                      % (peak_src, bf16_burst))
+    # the tensor cores' own rate on this GPU (tcgen05.mma probe, one CTA per SM), the
+    # second denominator: QK^T at the S8 rate and PV at the E4M3 (or BF16) rate, equal
+    # work, so their harmonic mean
+    probe = None
+    if not args.no_probe:
+        r_qk = sage.debug_mma_rate("s8_s32")
+        r_pv = sage.debug_mma_rate("bf16_f32" if pv16 else "e4m3_f32")
+        probe = 2.0 / (1.0 / r_qk + 1.0 / r_pv)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         ops_s, secs, desc, threads = oracle_sample(w, args.cpu_seconds)
         cpu = {"value": ops_s / secs / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": args.scaling if world > 1 else "weak",
         "vs_baseline": None, "dtype": "int8+fp16" if pv16 else "int8+e4m3", "data": "synthetic",
-        "config": dict(w.describe(), parallelism="heads sharded: each of %d rank(s) runs the full workload" % world,
+        "config": dict(w.describe(), parallelism=parallelism_label(w, world, args.scaling),
                        l2="inputs (%.0f MiB) larger than L2 (126 MB); no flush" % ((2 * q.numel() + 2 * k.numel()) * 2 / 2 ** 20),
                        granularity="per_threadgroup (g_q=32, g_k=16)",
                        **({"pv": "fp16 (qk_int8_pv_fp16)"} if pv16 else {"pv": "fp8", "pr": 448, "vr": 448})),
@@ -434,6 +506,8 @@ def main():
         "attn_frac_of_spec_4500": attn_tops / SPEC_INT8_TOPS,
         "roofline": {"bound": "tensor", "achieved": attn_tops, "peak": peak, "unit": "TFLOP/s",
                      "frac": attn_tops / peak, "traffic": None if pv16 else recorded_traffic(w.name),
+                     "frac_of_tcgen05_probe": (attn_tops / probe) if probe else None,
+                     "tcgen05_probe_peak": probe,
                      "peak_source": peak_note,
                      "kernel": "attn_fwd_kernel<%d>" % d},
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,

@@ -327,6 +327,20 @@ SAGE_API sage_status_t sage_debug_mma_rate(int kind, int n_iter, int n_ctas, voi
 SAGE_API sage_status_t sage_debug_quant_fp4(const float *xs, int n_rows, int d, uint8_t *codes, uint8_t *sf,
                                             float *g, void *stream);
 
+/* One 128 x 128 QK^T tile of the 4-bit mode on the block-scaled tensor core
+ * (tcgen05.mma kind::mxf4nvf4, one E4M3 scale per 16 channels, scale factors copied
+ * into tensor memory by tcgen05.cp):
+ *   s_out[i][j] = sum over 16-channel blocks b of sfq[i][b] * sfk[j][b] *
+ *                 (sum over the block's channels c of e2m1(q4[i][c]) * e2m1(k4[j][c]))
+ * accumulated in FP32.  q4, k4: device uint8 [128][d/2] E2M1 codes, channel 2c in the
+ * low nibble of byte c (16-byte aligned); sfq, sfk: device uint8 [128][d/16] E4M3 scale
+ * codes; s_out: device fp32 [128][128] (row = query, column = key).  status_block:
+ * device buffer of at least 256 zeroed bytes (read with sage_get_device_status).  The
+ * per-tile fp32 scales g of the 4-bit mode multiply the result outside the tensor core. */
+SAGE_API sage_status_t sage_debug_qk_tile_fp4(const uint8_t *q4, const uint8_t *k4, const uint8_t *sfq,
+                                              const uint8_t *sfk, int d, float *s_out, void *status_block,
+                                              void *stream);
+
 /* Runs the attention kernel with one deliberately missing producer signal so that
  * the consumer's bounded wait must run out; the kernel records SAGE_ERR_TIMEOUT in
  * the status block and exits without hanging.  Arguments as sage_attn_fwd_prequant;

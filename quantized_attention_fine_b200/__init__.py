@@ -117,6 +117,7 @@ def load_library():
         lib.sage_debug_pv_accumulate_f16acc.argtypes = [P, P, I, I, P, P]
         lib.sage_debug_mma_rate.argtypes = [I, I, I, P, P]
         lib.sage_debug_quant_fp4.argtypes = [P, I, I, P, P, P, P]
+        lib.sage_debug_qk_tile_fp4.argtypes = [P, P, P, P, I, P, P, P]
         lib.sage_debug_attn_fault_inject.argtypes = [P, I, I, I, I, I, I, I, I, P, S, P]
         lib.sage_version.restype = ctypes.c_char_p
         for fn in ("sage_quant_qk", "sage_quant_v", "sage_attn_fwd_prequant", "sage_attn_fwd",
@@ -124,6 +125,7 @@ def load_library():
                    "sage_attn_fwd_varlen",
                    "sage_get_device_status", "sage_debug_qk_tile", "sage_debug_pv_accumulate",
                    "sage_debug_pv_accumulate_f16acc", "sage_debug_mma_rate", "sage_debug_quant_fp4",
+                   "sage_debug_qk_tile_fp4",
                    "sage_debug_attn_fault_inject"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
@@ -522,6 +524,25 @@ def debug_quant_fp4(xs, stream=None):
     _check(load_library().sage_debug_quant_fp4(_ptr(xs), n, d, _ptr(codes), _ptr(sf), _ptr(g),
                                                _stream_handle(stream)), "sage_debug_quant_fp4")
     return codes, sf, g
+
+
+def debug_qk_tile_fp4(q4, k4, sfq, sfk, stream=None):
+    """One 128 x 128 QK^T tile of the 4-bit mode on the block-scaled tensor core
+    (diagnostic).  q4, k4: uint8 [128, d/2] E2M1 codes (channel 2c in the low nibble of
+    byte c); sfq, sfk: uint8 [128, d/16] E4M3 scale codes.  Returns fp32 [128, 128]."""
+    torch = _torch()
+    d = int(q4.shape[1]) * 2
+    out = torch.empty((128, 128), dtype=torch.float32, device=q4.device)
+    status = torch.zeros(64, dtype=torch.int32, device=q4.device)
+    lib = load_library()
+    _check(lib.sage_debug_qk_tile_fp4(_ptr(q4), _ptr(k4), _ptr(sfq), _ptr(sfk), d, _ptr(out), _ptr(status),
+                                      _stream_handle(stream)), "sage_debug_qk_tile_fp4")
+    code, site = ctypes.c_int(), ctypes.c_int()
+    _check(lib.sage_get_device_status(_ptr(status), _stream_handle(stream), ctypes.byref(code), ctypes.byref(site)),
+           "sage_get_device_status")
+    if code.value != SAGE_OK:
+        raise SageError(code.value, "sage_debug_qk_tile_fp4 (device site %d)" % site.value)
+    return out
 
 
 def debug_fault_inject(workspace: Workspace, out, *, layout="HND", causal=False, stream=None):

@@ -266,6 +266,125 @@ cudaError_t launch_debug_qk_tile(const CUtensorMap &tq, const CUtensorMap &tk, i
 }
 
 // ---------------------------------------------------------------------------
+// Diagnostic: one FP4 QK^T tile on the block-scaled tensor core (tcgen05.mma
+// kind::mxf4nvf4, scale_vec::4X): S = sum over 16-channel blocks b of sfq[i][b] sfk[j][b]
+// (Q4[i] . K4[j] over the block), FP32 in tensor memory.  Rows of E2M1 codes (two per
+// byte, channel 2c in the low nibble) are staged K-major with the 32-byte (d = 64) or
+// 64-byte (d = 128) swizzle; the E4M3 scales of each 64-channel chunk as a 512-byte atom
+// (row m, block b at byte 16 (m mod 32) + 4 (m / 32) + b), copied into tensor memory by
+// tcgen05.cp.  The smoothed Q / K tiles of the 4-bit mode take exactly this form
+// ("SageAttention2" abstract: 4-bit QK^T; "SageAttention3: Microscaling FP4 Attention",
+// listed among the notes' related papers).
+// ---------------------------------------------------------------------------
+template <int D>
+struct Fp4Layout {
+    static constexpr uint32_t row_bytes = D / 2;
+    static constexpr uint32_t layout = (D == 64) ? 6u : 4u;   // UMMA 32-byte / 64-byte swizzle
+    static constexpr uint32_t sbo = 8 * row_bytes;            // 8-row groups
+    static constexpr int chunks = D / 64;                     // K = 64 per MMA
+};
+// Byte offset of 16-byte chunk c of row r in a swizzled K-major FP4 tile.
+template <int D>
+__device__ __forceinline__ uint32_t fp4_row_offset(uint32_t r, uint32_t c) {
+    if constexpr (D == 64) return r * 32u + ((c ^ ((r >> 2) & 1u)) << 4);
+    return r * 64u + ((c ^ ((r >> 1) & 3u)) << 4);
+}
+
+template <int D>
+struct __align__(1024) Fp4QkSmem {
+    uint8_t q[kTile * D / 2];
+    uint8_t k[kTile * D / 2];
+    uint8_t sfq[D / 64][512];
+    uint8_t sfk[D / 64][512];
+    uint64_t bar_mma;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+    debug_qk_fp4_kernel(const uint8_t *q4, const uint8_t *k4, const uint8_t *sfq, const uint8_t *sfk, float *out,
+                        int *status) {
+    using L = Fp4Layout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    Fp4QkSmem<D> &sm = *reinterpret_cast<Fp4QkSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = threadIdx.x;
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.bar_mma, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) { tmem_alloc(&sm.tmem_base, 256); tmem_relinquish(); }
+    // row r of Q and K into the swizzled tiles; its scales into the atoms
+#pragma unroll
+    for (uint32_t c = 0; c < L::row_bytes / 16; ++c) {
+        *reinterpret_cast<uint4 *>(sm.q + fp4_row_offset<D>(r, c)) = reinterpret_cast<const uint4 *>(q4 + (size_t)r * L::row_bytes)[c];
+        *reinterpret_cast<uint4 *>(sm.k + fp4_row_offset<D>(r, c)) = reinterpret_cast<const uint4 *>(k4 + (size_t)r * L::row_bytes)[c];
+    }
+#pragma unroll
+    for (int b = 0; b < D / 16; ++b) {
+        const int at = 16 * (r & 31) + 4 * (r >> 5) + (b & 3);
+        sm.sfq[b >> 2][at] = sfq[(size_t)r * (D / 16) + b];
+        sm.sfk[b >> 2][at] = sfk[(size_t)r * (D / 16) + b];
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t t_sfq = tmem + 128u, t_sfk = tmem + 144u;   // 4 columns per 64-channel chunk
+    volatile int *abort_flag = &sm.abort_flag;
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int kc = 0; kc < L::chunks; ++kc) {
+            tmem_cp_sf_atom(t_sfq + 4u * kc, sf_atom_desc(smem_u32(sm.sfq[kc])));
+            tmem_cp_sf_atom(t_sfk + 4u * kc, sf_atom_desc(smem_u32(sm.sfk[kc])));
+        }
+        constexpr uint32_t idesc = idesc_mxf4_e4m3sf(128, 128);
+#pragma unroll
+        for (int kc = 0; kc < L::chunks; ++kc)
+            mma_mxf4_ss(tmem, smem_desc(smem_u32(sm.q) + 32u * kc, L::sbo, L::layout),
+                        smem_desc(smem_u32(sm.k) + 32u * kc, L::sbo, L::layout), idesc, t_sfq + 4u * kc,
+                        t_sfk + 4u * kc, kc > 0 ? 1u : 0u);
+        mma_commit(&sm.bar_mma);
+    }
+    __syncwarp();
+    mbar_wait(&sm.bar_mma, 0, abort_flag, status, kSiteDebug);
+    tc_fence_after();
+    __syncthreads();
+    if (*abort_flag == 0) {
+#pragma unroll
+        for (int c0 = 0; c0 < kTile; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
+            tmem_wait_ld_regs(v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) out[(size_t)(warp * 32 + lane) * kTile + c0 + i] = __uint_as_float(v[i]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) { __syncwarp(); tc_fence_after(); tmem_dealloc(tmem, 256); }
+}
+
+cudaError_t launch_debug_qk_fp4(const uint8_t *q4, const uint8_t *k4, const uint8_t *sfq, const uint8_t *sfk, int d,
+                                float *out, int *status, cudaStream_t stream) {
+    if (d == 128) {
+        const size_t smem = sizeof(Fp4QkSmem<128>) + 1024;
+        cudaError_t e = cudaFuncSetAttribute(debug_qk_fp4_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        debug_qk_fp4_kernel<128><<<1, 128, smem, stream>>>(q4, k4, sfq, sfk, out, status);
+    } else {
+        const size_t smem = sizeof(Fp4QkSmem<64>) + 1024;
+        cudaError_t e = cudaFuncSetAttribute(debug_qk_fp4_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        debug_qk_fp4_kernel<64><<<1, 128, smem, stream>>>(q4, k4, sfq, sfk, out, status);
+    }
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Diagnostic: sum over tiles of P . V on the FP8 path, one FP32 accumulator
 // (ACC16: an FP16 accumulator instead, the SageAttention2++ variant; the raw
 // 32-bit tensor-memory words are written out).  P and V^T tiles are copied row by

@@ -586,6 +586,17 @@ sage_status_t sage_debug_quant_fp4(const float *xs, int n_rows, int d, uint8_t *
                : SAGE_ERR_CUDA;
 }
 
+sage_status_t sage_debug_qk_tile_fp4(const uint8_t *q4, const uint8_t *k4, const uint8_t *sfq, const uint8_t *sfk,
+                                     int d, float *s_out, void *status_block, void *stream) {
+    if (!q4 || !k4 || !sfq || !sfk || !s_out || !status_block) return SAGE_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
+    if (!aligned16(q4) || !aligned16(k4) || !aligned16(s_out)) return SAGE_ERR_UNSUPPORTED;
+    return launch_debug_qk_fp4(q4, k4, sfq, sfk, d, s_out, static_cast<int *>(status_block),
+                               static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SAGE_OK
+               : SAGE_ERR_CUDA;
+}
+
 sage_status_t sage_debug_attn_fault_inject(void *o, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
                                            int causal, const void *workspace, size_t workspace_bytes,
                                            void *stream) {

@@ -314,6 +314,39 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// Block-scaled FP4 (kind::mxf4nvf4): E2M1 A and B (K-major, two codes per byte), one
+// unsigned E4M3 scale per 16 elements of K (scale_vec::4X, K = 64 per instruction), FP32
+// D.  Fields as above, plus [4,6) B scale-factor id and [29,31) A scale-factor id (the
+// byte offset of the scales inside their tensor-memory word: 0 here), [23] scale format
+// (0 = E4M3), [31] K size (0 = 64); A and B format 1 = E2M1.
+__host__ __device__ constexpr uint32_t idesc_mxf4_e4m3sf(int M, int N) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void mma_mxf4_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+// Shared-memory descriptor of a 512-byte scale-factor atom: 32 rows of 16 bytes, no
+// swizzle, 8-row core matrices 128 bytes apart (the K-major interleaved layout).
+__device__ __forceinline__ uint64_t sf_atom_desc(uint32_t saddr) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)(128u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    return d;
+}
+// Copy a scale-factor atom (32 rows of 16 bytes) into 4 tensor-memory columns at
+// `taddr`, every lane quadrant receiving the same 32 rows: lane 32 q + l holds atom row
+// l.  Row m's four scales are then found in lane m, column taddr + m / 32, which is
+// where kind::mxf4nvf4 with scale_vec::4X reads them.
+__device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive once on `bar` when all previously issued tcgen05.mma of this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

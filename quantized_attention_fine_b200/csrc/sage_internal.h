@@ -162,6 +162,9 @@ cudaError_t launch_debug_mma_rate(int kind, int n_iter, int n_ctas, int *status,
 cudaError_t launch_debug_quant_fp4(const float *xs, int n_rows, int d, uint8_t *codes, uint8_t *sf, float *g,
                                    cudaStream_t stream);
 cudaError_t launch_zero_output(void *o, size_t bytes, cudaStream_t stream);
+// One FP4 QK^T tile on the block-scaled tensor core; see sage_debug_qk_tile_fp4.
+cudaError_t launch_debug_qk_fp4(const uint8_t *q4, const uint8_t *k4, const uint8_t *sfq, const uint8_t *sfk, int d,
+                                float *out, int *status, cudaStream_t stream);
 
 // How a whole-forward call (sage_attn_fwd_gqa's arguments) proceeds once its
 // arguments are valid: nothing to do (B * H == 0 or n_q == 0), O = 0 without a

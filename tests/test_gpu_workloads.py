@@ -40,9 +40,12 @@ def _full_precision_rows(qh, kh, vh, rows, causal):
     return (p @ vh) / p.sum(1, keepdims=True)
 
 
-@pytest.mark.parametrize("name", ["image_dit", "llm_prefill", "video_dit", "llm_prefill_gqa"])
+@pytest.mark.parametrize("name", ["image_dit", "llm_prefill", "video_dit", "llm_prefill_gqa",
+                                  "sweep_n65536_d128_causal", "sweep_n65536_d64_full"])
 def test_full_size_workload_sampled(name):
-    w = wl.WORKLOADS[name]
+    """Also the longest sweep points, N = 65,536 (the sweep recipe names N up to 64K):
+    the first, middle and last Q blocks of two heads over all 65,536 keys."""
+    w = wl.by_name(name)
     q, k, v = wl.generate(w)
     dev = torch.device("cuda", 0)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)

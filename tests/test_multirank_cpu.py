@@ -1,8 +1,12 @@
 """The N > 1 host path of bench.py, as two gloo ranks on the CPU.
 
-Each rank runs the whole workload on its own seeded inputs (weak scaling), the
-timings are reduced to the slowest rank, and the value is all ranks' work over that
-time.  The reference arm runs on rank 0 only.  No GPU is involved.
+Each rank computes a disjoint slice of one seeded global problem, split by heads
+(weak: one batch block per rank; strong: the workload's key/value head groups split
+into contiguous ranges).  The oracle run on each rank's slice, put back together,
+equals the oracle run on the whole global problem bit for bit, with every head
+computed exactly once.  The timings are reduced to the slowest rank, and the value is
+all ranks' work over that time.  The reference arm runs on rank 0 only.  No GPU is
+involved.
 """
 import os
 import socket
@@ -22,6 +26,12 @@ def _free_port():
         return s.getsockname()[1]
 
 
+def _strong_workload():
+    from quantized_attention_fine_b200 import workloads as wl
+    # 4 query heads over 2 key/value heads: a rank takes one key/value head group
+    return wl.custom("mr_gqa", 1, 4, 150, 200, 64, True, recipe="llm", H_kv=2, seed=777)
+
+
 def _rank_main(rank, world, port, out_dir):
     sys.path.insert(0, ROOT)
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
@@ -29,6 +39,8 @@ def _rank_main(rank, world, port, out_dir):
     import bench
     from quantized_attention_fine_b200 import workloads as wl
     from datetime import timedelta
+    global _STRONG
+    _STRONG = _strong_workload()
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
     try:
         # per-rank inputs: same shapes, different seeds
@@ -41,8 +53,15 @@ def _rank_main(rank, world, port, out_dir):
         class _A:
             steps, warmup, cpu_seconds = 1, 0, 0.01
         ref_rc = bench.reference_arm(_A(), w) if rank != 0 else 0
-        torch.save({"seed": wr.seed, "q_sum": float(q.float().sum()), "max": got, "ref_rc": ref_rc},
-                   os.path.join(out_dir, "rank%d.pt" % rank))
+        # this rank's slice of the global problem, through the oracle
+        import oracle
+        slices = {}
+        for scaling, wg in (("weak", w), ("strong", _STRONG)):
+            sub, qs, ks, vs = bench.rank_inputs(wg, world, rank, scaling)
+            o = oracle.sage_attention(*(x.double().numpy() for x in (qs, ks, vs)), causal=wg.causal)
+            slices[scaling] = (sub.B, sub.H, sub.Hk, torch.from_numpy(o))
+        torch.save({"seed": wr.seed, "q_sum": float(q.float().sum()), "max": got, "ref_rc": ref_rc,
+                    "slices": slices}, os.path.join(out_dir, "rank%d.pt" % rank))
         dist.barrier()
     finally:
         dist.destroy_process_group()
@@ -57,6 +76,36 @@ def test_two_gloo_ranks(tmp_path):
     for x in r:
         assert x["max"] == [11.0, 3.0]
     assert r[1]["ref_rc"] == 0
+    # the slices tile the global problem: concatenated, they equal the oracle on the
+    # whole global problem, and together they cover each head once
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    import oracle
+    from quantized_attention_fine_b200 import workloads as wl
+    w = wl.custom("mr", 1, 2, 160, 160, 64, True, recipe="llm")
+    gq, gk, gv = bench.global_inputs(w, world, "weak")
+    assert gq.shape[0] == world * w.B
+    full = oracle.sage_attention(*(x.double().numpy() for x in (gq, gk, gv)), causal=True)
+    got = np.concatenate([x["slices"]["weak"][3].numpy() for x in r], axis=0)
+    assert np.array_equal(got, full)
+    ws_ = _strong_workload()
+    gq, gk, gv = bench.global_inputs(ws_, world, "strong")
+    full = oracle.sage_attention(*(x.double().numpy() for x in (gq, gk, gv)), causal=True)
+    heads = [x["slices"]["strong"] for x in r]
+    assert [(b, h, hk) for b, h, hk, _ in heads] == [(1, 2, 1)] * world   # 2 query heads over 1 kv head each
+    got = np.concatenate([o.numpy() for _, _, _, o in heads], axis=1)
+    assert got.shape == full.shape and np.array_equal(got, full)
+
+
+def test_unit_range_covers_every_unit_once():
+    sys.path.insert(0, ROOT)
+    import bench
+    for n, world in ((32, 1), (32, 2), (32, 8), (96, 4), (8, 8)):
+        seen = [u for r in range(world) for u in range(*bench.unit_range(n, world, r))]
+        assert seen == list(range(n))
+    with pytest.raises(ValueError):
+        bench.unit_range(32, 3, 0)
 
 
 def test_whole_job_value_is_all_ranks_work_over_slowest_time():
