@@ -57,6 +57,9 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--pv", default="fp8", choices=["fp8", "fp16"],
                     help="PV precision: fp8 (the method's default) or fp16 (the qk_int8_pv_fp16 mode)")
+    ap.add_argument("--qk", default="int8", choices=["int8", "fp4"],
+                    help="Q / K precision: int8 (grouped INT8, the default) or fp4 (the 4-bit mode: block-scaled "
+                         "E2M1 on tcgen05.mma kind::mxf4nvf4; d = 64 workloads)")
     ap.add_argument("--graph", action="store_true",
                     help="time the step as a replay of a CUDA graph that captured one sage_attn_fwd call")
     ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
@@ -161,10 +164,11 @@ def whole_job_tops(world: int, ops_per_rank_step: float, ms_per_step: float) -> 
 _HEAD_CACHE = {}
 
 
-def oracle_sample(w, seconds: float):
+def oracle_sample(w, seconds: float, quant=(1, 1, 1)):
     """Time the fp64 oracle on a bounded sample of workload w: head (0, 0) of the seeded
     inputs, its pre-pass, then Q blocks in a seeded order until `seconds` have passed.
-    Returns (ops_done, time_s, description, threads)."""
+    quant: the oracle's (QK, P, V) mode of the run.  Returns (ops_done, time_s,
+    description, threads)."""
     import numpy as np
     import oracle
     from quantized_attention_fine_b200 import workloads as wl
@@ -174,7 +178,7 @@ def oracle_sample(w, seconds: float):
         del q, k, v
     qh, kh, vh = _HEAD_CACHE[w.name]
     t0 = time.perf_counter()
-    pre = oracle.prepass_head(qh, kh, vh)
+    pre = oracle.prepass_head(qh, kh, vh, quant=quant)
     t_pre = time.perf_counter() - t0
     tq = -(-w.N_q // 128)
     order = np.random.default_rng(w.seed).permutation(tq)
@@ -345,13 +349,15 @@ def main():
     q, k, v = q_cpu.to(dev), k_cpu.to(dev), v_cpu.to(dev)
     B, H, nq, nk, d = wr.B, wr.H, wr.N_q, wr.N_kv, wr.d
     pv16 = args.pv == "fp16"
-    ws = sage.make_workspace(B, H, nq, nk, d, device=dev, H_kv=wr.Hk, pv_fp16=pv16)
+    fp4 = args.qk == "fp4"
+    gran = "fp4" if fp4 else "per_threadgroup"
+    ws = sage.make_workspace(B, H, nq, nk, d, device=dev, H_kv=wr.Hk, pv_fp16=pv16, qk_fp4=fp4)
     out = torch.empty_like(q)
-    mode = sage.QuantMode.make(pv=args.pv)
+    mode = sage.QuantMode.make(gran, pv=args.pv)
     stream = torch.cuda.current_stream(dev)
 
     def step_eager():
-        sage.attn_fwd(q, k, v, causal=w.causal, out=out, workspace=ws, pv=args.pv)
+        sage.attn_fwd(q, k, v, causal=w.causal, out=out, workspace=ws, pv=args.pv, granularity=gran)
 
     step = step_eager
     graph = None
@@ -440,7 +446,8 @@ def main():
                 stream.wait_event(ev_in[i])
                 if i >= 2:
                     stream.wait_event(ev_out[i - 2])     # and its output has been copied out
-                sage.attn_fwd(qd, kd, vd, causal=w.causal, out=od, workspace=ws, stream=stream, pv=args.pv)
+                sage.attn_fwd(qd, kd, vd, causal=w.causal, out=od, workspace=ws, stream=stream, pv=args.pv,
+                              granularity=gran)
                 ev_comp[i].record(stream)
                 s_out.wait_event(ev_comp[i])
                 with torch.cuda.stream(s_out):
@@ -475,6 +482,10 @@ def main():
     bf16_burst, bf16_sust, peak_src = measured_peaks()
     peak = 2.0 * bf16_burst   # dense INT8 / FP8 = 2x dense BF16 (nominal 4.5 vs 2.25 PFLOP/s)
     peak_note = "%s bf16 burst %.1f x 2 (dense int8/fp8 = 2x bf16)" % (peak_src, bf16_burst)
+    if fp4:   # QK^T at the FP4 rate (nominal 2x FP8), PV at the FP8 rate, equal work: the harmonic mean
+        peak = 2.0 / (1.0 / (4.0 * bf16_burst) + 1.0 / (2.0 * bf16_burst))
+        peak_note = ("%s bf16 burst %.1f: FP4 QK at 4x (nominal 2x FP8), FP8 PV at 2x, equal work: harmonic mean"
+                     % (peak_src, bf16_burst))
     if pv16:  # half the work at the INT8 rate, half at the FP16 rate: the harmonic mean
         peak = 2.0 / (1.0 / (2.0 * bf16_burst) + 1.0 / bf16_burst)
         peak_note = ("%s bf16 burst %.1f: INT8 QK at 2x, FP16 PV at 1x, equal work: harmonic mean"
@@ -484,32 +495,36 @@ def main():
     # work, so their harmonic mean
     probe = None
     if not args.no_probe:
-        r_qk = sage.debug_mma_rate("s8_s32")
+        # the 4-bit QK^T rate is taken as twice the probe's E4M3 rate (the nominal ratio)
+        r_qk = 2.0 * sage.debug_mma_rate("e4m3_f32") if fp4 else sage.debug_mma_rate("s8_s32")
         r_pv = sage.debug_mma_rate("bf16_f32" if pv16 else "e4m3_f32")
         probe = 2.0 / (1.0 / r_qk + 1.0 / r_pv)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        ops_s, secs, desc, threads = oracle_sample(w, args.cpu_seconds)
+        ops_s, secs, desc, threads = oracle_sample(w, args.cpu_seconds,
+                                                   quant=(2 if fp4 else 1, 2 if pv16 else 1, 2 if pv16 else 1))
         cpu = {"value": ops_s / secs / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": args.scaling if world > 1 else "weak",
-        "vs_baseline": None, "dtype": "int8+fp16" if pv16 else "int8+e4m3", "data": "synthetic",
+        "vs_baseline": None, "dtype": ("e2m1" if fp4 else "int8") + ("+fp16" if pv16 else "+e4m3"),
+        "data": "synthetic",
         "config": dict(w.describe(), parallelism=parallelism_label(w, world, args.scaling),
                        l2="inputs (%.0f MiB) larger than L2 (126 MB); no flush" % ((2 * q.numel() + 2 * k.numel()) * 2 / 2 ** 20),
-                       granularity="per_threadgroup (g_q=32, g_k=16)",
+                       granularity=("fp4 (E2M1, E4M3 scale per 16 channels, fp32 scale per 128-row tile)" if fp4
+                                    else "per_threadgroup (g_q=32, g_k=16)"),
                        **({"pv": "fp16 (qk_int8_pv_fp16)"} if pv16 else {"pv": "fp8", "pr": 448, "vr": 448})),
         "attn_kernel_tops": attn_tops, "attn_kernel_ms": attn_avg_ms, "prepass_ms": pre_avg_ms,
         "step_call": ("sage_attn_fwd (pre-pass + dS + attention)" + (", replayed from a CUDA graph" if args.graph else "")
                       + "; prepass_ms = ms_per_step - attn_kernel_ms"),
         "attn_frac_of_spec_4500": attn_tops / SPEC_INT8_TOPS,
         "roofline": {"bound": "tensor", "achieved": attn_tops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": attn_tops / peak, "traffic": None if pv16 else recorded_traffic(w.name),
+                     "frac": attn_tops / peak, "traffic": None if (pv16 or fp4) else recorded_traffic(w.name),
                      "frac_of_tcgen05_probe": (attn_tops / probe) if probe else None,
                      "tcgen05_probe_peak": probe,
                      "peak_source": peak_note,
-                     "kernel": "attn_fwd_kernel<%d>" % d},
+                     "kernel": "attn_fwd_kernel<%d>%s" % (d, " (4-bit QK)" if fp4 else "")},
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         "gpu_launches": args.steps * LAUNCHES_PER_STEP,
     }

@@ -93,7 +93,20 @@ typedef enum { SAGE_DTYPE_F16 = 0, SAGE_DTYPE_BF16 = 1 } sage_dtype_t;
 typedef enum {
     SAGE_QK_PER_BLOCK = 0,        /* g_q = 128, g_k = 128 */
     SAGE_QK_PER_WARP = 1,         /* g_q = 32,  g_k = 128 */
-    SAGE_QK_PER_THREADGROUP = 2   /* g_q = 32,  g_k = 16  (default) */
+    SAGE_QK_PER_THREADGROUP = 2,  /* g_q = 32,  g_k = 16  (default) */
+    SAGE_QK_FP4 = 3               /* 4-bit Q and K instead of INT8 (the pages' "4+8"
+                                   * variant), in the block-scaled form B200's tensor
+                                   * cores take: per 128-row tile an fp32 scale
+                                   * g = amax / 2688 (1 if amax = 0); per row and 16
+                                   * channels an E4M3 scale sf = E4M3(amax / g / 6) (1 if
+                                   * that amax is 0, 2^-9 if it rounds to 0); per element
+                                   * the E2M1 code of x / (g sf) (round to nearest even,
+                                   * saturating at 6).  QK^T runs on tcgen05.mma
+                                   * kind::mxf4nvf4.  The quantization calls take d = 64 or
+                                   * 128; attention in this mode takes d = 64 (at d = 128
+                                   * the four FP32 tensor-memory accumulators of the two Q
+                                   * tiles fill all 512 columns and leave none for the
+                                   * scales: SAGE_ERR_UNSUPPORTED).  FP8 P / V only. */
 } sage_qk_gran_t;
 
 typedef struct {
@@ -109,7 +122,14 @@ typedef struct {
                         *    are unused.  The workspace of this mode is larger
                         *    (sage_workspace_bytes_mode). */
 } sage_quant_mode_t;
-/* A NULL mode pointer means {SAGE_QK_PER_THREADGROUP, 1, 1, 448, 448, 0}. */
+/* A NULL mode pointer means {SAGE_QK_PER_THREADGROUP, 1, 1, 448, 448, 0}.
+ * In the SAGE_QK_FP4 mode the workspace views change as follows: SAGE_WS_Q8 / SAGE_WS_K8
+ * hold the E2M1 codes, [rows][d/2] bytes (channel 2c in the low nibble of byte c) in the
+ * same regions; SAGE_WS_DQ holds each row's tile scale g, SAGE_WS_DK each 16-key run's
+ * tile scale g; SAGE_WS_SFQ / SAGE_WS_SFK hold the E4M3 scales per 128-row tile and
+ * 64-channel chunk as 512-byte atoms (the scale of tile row m and block b at byte
+ * 16 (m mod 32) + 4 (m / 32) + (b mod 4) of atom b / 4): [BH][Tq][d/64][512] and
+ * [BHk][Tk][d/64][512]. */
 
 /* Bytes of workspace for one problem size (any dtype/layout).  0 on bad sizes. */
 SAGE_API size_t sage_workspace_bytes(int B, int H, int n_q, int n_kv, int d);
@@ -252,6 +272,8 @@ SAGE_API sage_status_t sage_get_device_status(void *workspace, void *stream, int
  *                                                invisible entries left unwritten)
  *   SAGE_WS_QS_KBAR fp32 [BH][nq_pad]            (q_i - qbar_t) . kbar per row: the
  *                                                shift K smoothing gives the row's logits
+ *   SAGE_WS_SFQ, SAGE_WS_SFK                     E4M3 scale atoms of the SAGE_QK_FP4 mode
+ *                                                (zero bytes in the other modes)
  *   SAGE_WS_LSE   fp32  [BH][nq_pad]             per row, written by the attention
  *                                                step: log-sum-exp (natural log) of the
  *                                                row's logits sm_scale q_i . k_j over its
@@ -269,7 +291,7 @@ SAGE_API sage_status_t sage_get_device_status(void *workspace, void *stream, int
 enum {
     SAGE_WS_Q8 = 0, SAGE_WS_K8 = 1, SAGE_WS_VT8 = 2, SAGE_WS_DQ = 3, SAGE_WS_DK = 4,
     SAGE_WS_DV = 5, SAGE_WS_QBAR = 6, SAGE_WS_KBAR = 7, SAGE_WS_DS = 8, SAGE_WS_QS_KBAR = 9,
-    SAGE_WS_LSE = 10, SAGE_WS_NUM_VIEWS = 11
+    SAGE_WS_LSE = 10, SAGE_WS_SFQ = 11, SAGE_WS_SFK = 12, SAGE_WS_NUM_VIEWS = 13
 };
 /* Byte offset of view `which` inside the workspace, or -1 for bad arguments. */
 SAGE_API int64_t sage_workspace_offset(int B, int H, int n_q, int n_kv, int d, int which);

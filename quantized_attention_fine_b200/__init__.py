@@ -43,10 +43,11 @@ _lib = None
 SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_WORKSPACE, SAGE_ERR_CUDA, SAGE_ERR_TIMEOUT = range(6)
 _ERR_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED", 3: "SAGE_ERR_WORKSPACE",
               4: "SAGE_ERR_CUDA", 5: "SAGE_ERR_TIMEOUT"}
-GRANULARITIES = {"per_block": 0, "per_warp": 1, "per_threadgroup": 2}
+GRANULARITIES = {"per_block": 0, "per_warp": 1, "per_threadgroup": 2, "fp4": 3}
+QK_FP4 = 3   # granularity code of the 4-bit Q / K mode (SAGE_QK_FP4)
 _LAYOUTS = {"HND": 0, "NHD": 1}
 WS_VIEWS = {"q8": 0, "k8": 1, "vt8": 2, "dq": 3, "dk": 4, "dv": 5, "qbar": 6, "kbar": 7, "ds": 8, "qs_kbar": 9,
-            "lse": 10}
+            "lse": 10, "sfq": 11, "sfk": 12}
 WS_ALIGN = 1024
 
 
@@ -184,9 +185,14 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def workspace_bytes(B, H, n_q, n_kv, d, H_kv=None, pv_fp16=False) -> int:
+def _layout_mode(pv_fp16=False, qk_fp4=False):
+    """A mode with the workspace layout of these flags (the other fields do not change it)."""
+    return QuantMode.make("fp4" if qk_fp4 else "per_threadgroup", pv="fp16" if pv_fp16 else "fp8")
+
+
+def workspace_bytes(B, H, n_q, n_kv, d, H_kv=None, pv_fp16=False, qk_fp4=False) -> int:
     H_kv = H if H_kv is None else H_kv
-    mode = QuantMode.make(pv="fp16" if pv_fp16 else "fp8")
+    mode = _layout_mode(pv_fp16, qk_fp4)
     return int(load_library().sage_workspace_bytes_mode(B, H, H_kv, n_q, n_kv, d, ctypes.byref(mode)))
 
 
@@ -194,14 +200,16 @@ class Workspace:
     """Caller-owned device workspace: a zeroed uint8 tensor with a 1024-byte aligned window.
 
     dims = (B, H, n_q, n_kv, d) with H query heads; H_kv key/value heads (H_kv = H
-    for multi-head attention); pv_fp16: laid out for the FP16 P / V mode."""
+    for multi-head attention); pv_fp16: laid out for the FP16 P / V mode; qk_fp4: for
+    the 4-bit Q / K mode."""
 
-    def __init__(self, B, H, n_q, n_kv, d, device=None, H_kv=None, pv_fp16=False):
+    def __init__(self, B, H, n_q, n_kv, d, device=None, H_kv=None, pv_fp16=False, qk_fp4=False):
         torch = _torch()
         self.dims = (int(B), int(H), int(n_q), int(n_kv), int(d))
         self.H_kv = int(H if H_kv is None else H_kv)
         self.pv_fp16 = bool(pv_fp16)
-        self.nbytes = workspace_bytes(*self.dims, H_kv=self.H_kv, pv_fp16=self.pv_fp16)
+        self.qk_fp4 = bool(qk_fp4)
+        self.nbytes = workspace_bytes(*self.dims, H_kv=self.H_kv, pv_fp16=self.pv_fp16, qk_fp4=self.qk_fp4)
         if self.nbytes == 0:
             raise SageError(SAGE_ERR_UNSUPPORTED, "sage_workspace_bytes")
         self.tensor = torch.zeros(self.nbytes + WS_ALIGN, dtype=torch.uint8, device=device or "cuda")
@@ -209,10 +217,10 @@ class Workspace:
         self.offset = (-base) % WS_ALIGN
         self.ptr = base + self.offset
 
-    def fits(self, B, H, n_q, n_kv, d, H_kv=None, pv_fp16=False) -> bool:
+    def fits(self, B, H, n_q, n_kv, d, H_kv=None, pv_fp16=False, qk_fp4=False) -> bool:
         H_kv = H if H_kv is None else H_kv
         return (self.dims == (int(B), int(H), int(n_q), int(n_kv), int(d)) and self.H_kv == int(H_kv)
-                and self.pv_fp16 == bool(pv_fp16))
+                and self.pv_fp16 == bool(pv_fp16) and self.qk_fp4 == bool(qk_fp4))
 
     def lse(self):
         """Row log-sum-exp [B, H, n_q] (fp32, natural log) of the last attention call on
@@ -225,12 +233,17 @@ class Workspace:
         head for q8, dq, qbar, ds; per key/value head for k8, vt8, dk, dv, kbar."""
         torch = _torch()
         B, H, n_q, n_kv, d = self.dims
-        mode = QuantMode.make(pv="fp16" if self.pv_fp16 else "fp8")
+        mode = _layout_mode(self.pv_fp16, self.qk_fp4)
         off = int(load_library().sage_workspace_offset_mode(B, H, self.H_kv, n_q, n_kv, d, ctypes.byref(mode),
                                                             WS_VIEWS[which]))
-        BH, BHk, Tq = B * H, B * self.H_kv, -(-n_q // 128)
-        nq_pad, nk_pad = Tq * 128, -(-n_kv // 128) * 128
-        shapes = {"q8": ((BH, nq_pad, d), torch.int8), "k8": ((BHk, nk_pad, d), torch.int8),
+        BH, BHk, Tq, Tk = B * H, B * self.H_kv, -(-n_q // 128), -(-n_kv // 128)
+        nq_pad, nk_pad = Tq * 128, Tk * 128
+        qk = ((BH, nq_pad, d // 2), torch.uint8) if self.qk_fp4 else ((BH, nq_pad, d), torch.int8)
+        kk = ((BHk, nk_pad, d // 2), torch.uint8) if self.qk_fp4 else ((BHk, nk_pad, d), torch.int8)
+        shapes = {"q8": qk, "k8": kk,
+                  # E4M3 scale atoms: regions of the 4-bit mode only (empty otherwise)
+                  "sfq": ((BH, Tq, d // 64 if self.qk_fp4 else 0, 512), torch.uint8),
+                  "sfk": ((BHk, Tk, d // 64 if self.qk_fp4 else 0, 512), torch.uint8),
                   "vt8": ((BHk, d, nk_pad), torch.float16 if self.pv_fp16 else torch.uint8), "dq": ((BH, nq_pad), torch.float32),
                   "dk": ((BHk, nk_pad // 16), torch.float32), "dv": ((BHk, d), torch.float32),
                   "qbar": ((BH, Tq, d), torch.float32), "kbar": ((BHk, d), torch.float32),
@@ -242,23 +255,24 @@ class Workspace:
         return self.tensor[start:start + n].view(dt).view(shp)
 
 
-def make_workspace(B, H, n_q, n_kv, d, device=None, H_kv=None, pv_fp16=False) -> Workspace:
-    return Workspace(B, H, n_q, n_kv, d, device, H_kv=H_kv, pv_fp16=pv_fp16)
+def make_workspace(B, H, n_q, n_kv, d, device=None, H_kv=None, pv_fp16=False, qk_fp4=False) -> Workspace:
+    return Workspace(B, H, n_q, n_kv, d, device, H_kv=H_kv, pv_fp16=pv_fp16, qk_fp4=qk_fp4)
 
 
-def _ws_for(ws, B, H, H_kv, n_q, n_kv, d, device, pv_fp16=False):
+def _ws_for(ws, B, H, H_kv, n_q, n_kv, d, device, pv_fp16=False, qk_fp4=False):
     if ws is None:
-        return Workspace(B, H, n_q, n_kv, d, device, H_kv=H_kv, pv_fp16=pv_fp16)
-    if not ws.fits(B, H, n_q, n_kv, d, H_kv, pv_fp16):
-        raise ValueError("workspace was made for %s (H_kv %d, pv_fp16 %s), not %s (H_kv %d, pv_fp16 %s)"
-                         % (ws.dims, ws.H_kv, ws.pv_fp16, (B, H, n_q, n_kv, d), H_kv, bool(pv_fp16)))
+        return Workspace(B, H, n_q, n_kv, d, device, H_kv=H_kv, pv_fp16=pv_fp16, qk_fp4=qk_fp4)
+    if not ws.fits(B, H, n_q, n_kv, d, H_kv, pv_fp16, qk_fp4):
+        raise ValueError("workspace was made for %s (H_kv %d, pv_fp16 %s, qk_fp4 %s), not %s (H_kv %d, pv_fp16 %s, "
+                         "qk_fp4 %s)" % (ws.dims, ws.H_kv, ws.pv_fp16, ws.qk_fp4, (B, H, n_q, n_kv, d), H_kv,
+                                         bool(pv_fp16), bool(qk_fp4)))
     return ws
 
 
 def quant_qk(q, k, *, layout="HND", mode=None, workspace=None, stream=None) -> Workspace:
     B, H, H_kv, n_q, n_kv, d = _shape(q, k, layout)
     mode = mode or QuantMode.make()
-    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, q.device, mode.pv_fp16)
+    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, q.device, mode.pv_fp16, mode.gran == QK_FP4)
     _check(load_library().sage_quant_qk_gqa(_ptr(q), _ptr(k), _dtype_code(q), _LAYOUTS[layout], B, H, H_kv, n_q,
                                             n_kv, d, ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
                                             _stream_handle(stream)), "sage_quant_qk_gqa")
@@ -276,7 +290,7 @@ def quant_v(v, *, n_q, H=None, layout="HND", mode=None, workspace=None, stream=N
         H = workspace.dims[1] if workspace is not None else H_kv
     B, H, H_kv, n_kv, d = int(B), int(H), int(H_kv), int(n_kv), int(d)
     mode = mode or QuantMode.make()
-    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, v.device, mode.pv_fp16)
+    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, v.device, mode.pv_fp16, mode.gran == QK_FP4)
     _check(load_library().sage_quant_v_gqa(_ptr(v), _dtype_code(v), _LAYOUTS[layout], B, H, H_kv, n_q, n_kv, d,
                                            ctypes.byref(mode), ctypes.c_void_p(ws.ptr), ws.nbytes,
                                            _stream_handle(stream)), "sage_quant_v_gqa")
@@ -293,8 +307,8 @@ def attn_fwd_prequant(workspace: Workspace, *, dtype, layout="HND", causal=False
         shape = (B, H, n_q, d) if layout == "HND" else (B, n_q, H, d)
         out = torch.empty(shape, dtype=dtype, device=workspace.tensor.device)
     mode = mode or QuantMode.make()
-    if bool(mode.pv_fp16) != workspace.pv_fp16:
-        raise ValueError("the mode's pv setting does not match the workspace")
+    if bool(mode.pv_fp16) != workspace.pv_fp16 or (mode.gran == QK_FP4) != workspace.qk_fp4:
+        raise ValueError("the mode's pv / qk setting does not match the workspace")
     _check(load_library().sage_attn_fwd_prequant_gqa(_ptr(out), _dtype_code(out), _LAYOUTS[layout], B, H,
                                                      workspace.H_kv, n_q, n_kv, d, int(bool(causal)),
                                                      float(sm_scale or 0.0), ctypes.byref(mode),
@@ -318,7 +332,7 @@ def attn_fwd(q, k, v, *, causal=False, sm_scale=None, layout="HND", granularity=
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share a dtype")
     mode = QuantMode.make(granularity, smooth_q, smooth_k, p_range, v_range, pv)
-    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, q.device, mode.pv_fp16)
+    ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, q.device, mode.pv_fp16, mode.gran == QK_FP4)
     if out is None:
         out = torch.empty_like(q)
     _check(load_library().sage_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q),
@@ -358,7 +372,7 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, max_seqlen_q=None, 
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share a dtype")
     mode = QuantMode.make(granularity, smooth_q, smooth_k, p_range, v_range, pv)
-    ws = _ws_for(workspace, B, H, H_kv, max_seqlen_q, max_seqlen_kv, d, q.device, mode.pv_fp16)
+    ws = _ws_for(workspace, B, H, H_kv, max_seqlen_q, max_seqlen_kv, d, q.device, mode.pv_fp16, mode.gran == QK_FP4)
     if out is None:
         out = torch.empty_like(q)
     _check(load_library().sage_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q),
@@ -406,9 +420,10 @@ class SageAttention:
             raise ValueError("head dim %d, configured %d" % (int(q.shape[-1]), self.head_dim))
         B, H, H_kv, n_q, n_kv, d = _shape(q, k, self.tensor_layout)
         pv = QUANT_MODES[self.quant_mode]
-        if self._ws is None or not self._ws.fits(B, H, n_q, n_kv, d, H_kv, pv == "fp16") or \
+        fp4 = self.granularity == "fp4"
+        if self._ws is None or not self._ws.fits(B, H, n_q, n_kv, d, H_kv, pv == "fp16", fp4) or \
                 self._ws.tensor.device != q.device:
-            self._ws = Workspace(B, H, n_q, n_kv, d, q.device, H_kv=H_kv, pv_fp16=(pv == "fp16"))
+            self._ws = Workspace(B, H, n_q, n_kv, d, q.device, H_kv=H_kv, pv_fp16=(pv == "fp16"), qk_fp4=fp4)
         return attn_fwd(q, k, v, causal=self.is_causal, sm_scale=self.sm_scale, layout=self.tensor_layout,
                         granularity=self.granularity, smooth_q=self.smooth_q, smooth_k=self.smooth_k, pv=pv,
                         workspace=self._ws, return_lse=return_lse)

@@ -30,6 +30,9 @@
 // tile i), so QK^T of tile i + 2 runs on the tensor core during the softmax of
 // tile i + 1; the MMA issuer serves the tiles in turn with the pair (QK^T of tile
 // i + 2, PV of tile i).  P is double-buffered per tile.
+// In the 4-bit mode (QK4, d = 64) Q and K are E2M1 codes with E4M3 scales per 16
+// channels: each QK^T is one tcgen05.mma kind::mxf4nvf4 (K = 64) whose scale atoms
+// tcgen05.cp copies into tensor-memory columns 384-407, and S arrives in fp32.
 // Every wait is bounded: a wait that runs out records SAGE_ERR_TIMEOUT in the
 // status block, raises a CTA-wide abort flag that makes every role leave its loop,
 // drains the copies in flight, frees tensor memory and exits.
@@ -47,6 +50,8 @@ constexpr int kSoftmaxWarps = 16;
 constexpr int kWarpK = 16, kWarpMma = 17, kWarpV = 18;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;
+// 4-bit mode (d = 64): scale atoms of Q tiles A, B at 384 / 388, of K stage s at 392 + 4 s
+constexpr uint32_t kTmemSfQ = 384, kTmemSfK = 392;
 constexpr uint64_t kDrainNs = 50ull * 1000ull * 1000ull;
 // K codes + V^T codes of the heads whose CTAs run together stay within this many
 // bytes, a part of the 126 MB L2 (the rest holds the streaming Q codes, dS and O).
@@ -86,6 +91,9 @@ struct __align__(1024) AttnSmem {
     uint8_t p[2][AttnCfg<D, PV16>::kPBufs][AttnCfg<D, PV16>::kPBytes];
     float ds[KS][2][kTile];          // keys in storage order
     float dk[KS][kTile / kKeyRun];
+    // 4-bit mode: E4M3 scale atoms of the Q tiles and of each K stage (d = 64 only)
+    alignas(128) uint8_t sfq[2][D == 64 ? 512 : 16];
+    alignas(128) uint8_t sfk[KS][D == 64 ? 512 : 16];
     uint64_t bar_q, bar_kfull[KS], bar_kempty[KS], bar_vfull[VS], bar_vempty[VS];
     uint64_t bar_s[2], bar_sfree[2], bar_p[2], bar_o[2], bar_drain;
     uint32_t tmem_base;
@@ -150,14 +158,24 @@ __device__ __forceinline__ float4 lds_f32x4(const float *ptr) {
 // chunk), in place (S int32 -> fp32 bits); ds holds their dS contiguously (storage
 // order); a_lo / a_hi scale the keys of the chunk's first / second 16-key run
 // (k < 8 / k >= 8).  Returns the maximum.
+// QK4: S is already fp32 (the block-scaled FP4 product), a_lo / a_hi the tile scales.
+template <bool QK4>
 __device__ __forceinline__ float dequant16(uint32_t (&w)[16], float a_lo, float a_hi, const float *ds) {
 #pragma unroll
     for (int j = 0; j < 16; j += 4) {
         const float a = j < 8 ? a_lo : a_hi;
         const float2 a2 = make_float2(a, a);
         const float4 d4 = lds_f32x4(ds + j);
-        const float2 y01 = __ffma2_rn(make_float2((float)(int)w[j], (float)(int)w[j + 1]), a2, make_float2(d4.x, d4.y));
-        const float2 y23 = __ffma2_rn(make_float2((float)(int)w[j + 2], (float)(int)w[j + 3]), a2, make_float2(d4.z, d4.w));
+        float2 s01, s23;
+        if constexpr (QK4) {
+            s01 = make_float2(__uint_as_float(w[j]), __uint_as_float(w[j + 1]));
+            s23 = make_float2(__uint_as_float(w[j + 2]), __uint_as_float(w[j + 3]));
+        } else {
+            s01 = make_float2((float)(int)w[j], (float)(int)w[j + 1]);
+            s23 = make_float2((float)(int)w[j + 2], (float)(int)w[j + 3]);
+        }
+        const float2 y01 = __ffma2_rn(s01, a2, make_float2(d4.x, d4.y));
+        const float2 y23 = __ffma2_rn(s23, a2, make_float2(d4.z, d4.w));
         w[j] = __float_as_uint(y01.x);
         w[j + 1] = __float_as_uint(y01.y);
         w[j + 2] = __float_as_uint(y23.x);
@@ -240,7 +258,7 @@ __device__ __forceinline__ uint32_t pack16x2(float lo, float hi, int out_bf16) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-template <int D, bool PV16>
+template <int D, bool PV16, bool QK4>
 __device__ __forceinline__ void softmax_role(AttnSmem<D, PV16> &sm, const AttnParams &p, uint32_t tmem, int X, int t,
                                              int n_tiles, int bh, int64_t o_base, int n_q, int n_kv,
                                              volatile int *abort_flag) {
@@ -285,7 +303,7 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D, PV16> &sm, const AttnPa
         for (int q = 0; q < 4; ++q) {
             tmem_ld16x64b_x16(s_tmem + q * 32, sv[q]);
             tmem_wait_ld_regs16(sv[q]);
-            mx[q] = dequant16(sv[q], dq * sm.dk[0][2 * q], dq * sm.dk[0][2 * q + 1], sm.ds[0][X] + pos0 + 16 * q);
+            mx[q] = dequant16<QK4>(sv[q], dq * sm.dk[0][2 * q], dq * sm.dk[0][2 * q + 1], sm.ds[0][X] + pos0 + 16 * q);
         }
         // S may take the next QK^T, and K slot 0 may be refilled: both are read now (the
         // arrival must follow the dS / delta_K reads above, since it also frees the slot)
@@ -335,7 +353,7 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D, PV16> &sm, const AttnPa
             }
             tmem_ld16x64b_x16(s_tmem + q * 32, sv[q]);
             tmem_wait_ld_regs16(sv[q]);
-            mx[q] = dequant16(sv[q], dq * dkn[2 * q], dq * dkn[2 * q + 1], dsn + 16 * q);
+            mx[q] = dequant16<QK4>(sv[q], dq * dkn[2 * q], dq * dkn[2 * q + 1], dsn + 16 * q);
         }
         if (has_next) {  // tile it + 1's scores are in registers: its S buffer may take the next QK^T
             tc_fence_before();
@@ -431,12 +449,14 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D, PV16> &sm, const AttnPa
 // the dense lengths); without RT the kernel serves dense batches only and reads the
 // lengths straight from the parameters.  The two compile to different register
 // allocations: d = 128 dense runs faster without RT, d = 64 dense with it (measured).
-template <int D, bool RT, bool PV16>
+template <int D, bool RT, bool PV16, bool QK4>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
     constexpr int KS = AttnCfg<D, PV16>::kKStages, VS = AttnCfg<D, PV16>::kVStages;
     constexpr int kPBufs = AttnCfg<D, PV16>::kPBufs, kPBytes = AttnCfg<D, PV16>::kPBytes;
+    static_assert(!QK4 || (D == 64 && !PV16), "the 4-bit mode runs at d = 64 with FP8 P / V");
+    constexpr int kQkRowBytes = QK4 ? D / 2 : D;   // bytes of one Q / K row in shared memory
     extern __shared__ uint8_t smem_raw[];
     AttnSmem<D, PV16> &sm =
         *reinterpret_cast<AttnSmem<D, PV16> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -510,9 +530,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // ---------------- TMA producer: Q tiles, then the K / dS / delta_K ring ----------------
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
-            mbar_arrive_expect_tx(&sm.bar_q, (hasB ? 2 : 1) * kTile * D);
+            mbar_arrive_expect_tx(&sm.bar_q, (hasB ? 2 : 1) * (kTile * kQkRowBytes + (QK4 ? 512 : 0)));
             tma_load_2d(sm.q[0], &tm_q, &sm.bar_q, 0, bh * p.nq_pad + tA * kTile);
             if (hasB) tma_load_2d(sm.q[1], &tm_q, &sm.bar_q, 0, bh * p.nq_pad + tB * kTile);
+            if constexpr (QK4) {
+                bulk_load(sm.sfq[0], p.sfq + ((size_t)bh * p.Tq + tA) * 512, 512, &sm.bar_q);
+                if (hasB) bulk_load(sm.sfq[1], p.sfq + ((size_t)bh * p.Tq + tB) * 512, 512, &sm.bar_q);
+            }
             const float *ds_a = p.ds + ((size_t)bh * p.Tq + tA) * p.nk_pad;
             const float *ds_b = p.ds + ((size_t)bh * p.Tq + tB) * p.nk_pad;
             const float *dk_row = p.dk + (size_t)bh_kv * (p.nk_pad / kKeyRun);
@@ -524,9 +548,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 issued = it + 1;
                 if (p.fault_inject && it == 0) continue;  // diagnostic: leave slot 0 unsignalled
                 const bool dsA = p.use_ds && it < nA, dsB = p.use_ds && it < nB;
-                const uint32_t bytes = kTile * D + (dsA ? kTile * 4 : 0) + (dsB ? kTile * 4 : 0) + (kTile / kKeyRun) * 4;
+                const uint32_t bytes = kTile * kQkRowBytes + (dsA ? kTile * 4 : 0) + (dsB ? kTile * 4 : 0) +
+                                       (kTile / kKeyRun) * 4 + (QK4 ? 512 : 0);
                 mbar_arrive_expect_tx(&sm.bar_kfull[s], bytes);
                 tma_load_2d(sm.k[s], &tm_k, &sm.bar_kfull[s], 0, bh_kv * p.nk_pad + it * kTile);
+                if constexpr (QK4) bulk_load(sm.sfk[s], p.sfk + ((size_t)bh_kv * p.Tk + it) * 512, 512, &sm.bar_kfull[s]);
                 if (dsA) bulk_load(sm.ds[s][0], ds_a + it * kTile, kTile * 4, &sm.bar_kfull[s]);
                 if (dsB) bulk_load(sm.ds[s][1], ds_b + it * kTile, kTile * 4, &sm.bar_kfull[s]);
                 bulk_load(sm.dk[s], dk_row + it * (kTile / kKeyRun), (kTile / kKeyRun) * 4, &sm.bar_kfull[s]);
@@ -562,26 +588,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // ------------------------------ MMA issuer ------------------------------
             // Q tile x at q_s + x * kTile * D; P buffer (x, b) at p_s + (x * kPBufs + b) * kPBytes
             const uint32_t q_s = smem_u32(sm.q[0]), p_s = smem_u32(sm.p[0][0]);
+            // QK^T of Q tile x against K stage ks (the 4-bit mode: one block-scaled MMA whose
+            // scale atoms were copied to tensor memory beforehand)
+            auto qk = [&](int x, int ks) {
+                if constexpr (QK4) {
+                    mma_mxf4_ss(tmem + (uint32_t)x * 128u, smem_desc(q_s + (uint32_t)x * (kTile * D), 256u, 6u),
+                                smem_desc(smem_u32(sm.k[ks]), 256u, 6u), idesc_mxf4_e4m3sf(128, 128),
+                                tmem + kTmemSfQ + 4u * x, tmem + kTmemSfK + 4u * ks, 0u);
+                } else {
+                    issue_qk<D>(tmem + (uint32_t)x * 128u, q_s + (uint32_t)x * (kTile * D), smem_u32(sm.k[ks]));
+                }
+            };
+            // 4-bit mode: the scale atom of K stage ks into tensor memory (before its QK^T)
+            auto sf_k = [&](int ks) {
+                if constexpr (QK4) tmem_cp_sf_atom(tmem + kTmemSfK + 4u * ks, sf_atom_desc(smem_u32(sm.sfk[ks])));
+            };
             bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, p.status, kSiteQ);
             if (ok) ok = mbar_wait(&sm.bar_kfull[0], 0, abort_flag, p.status, kSiteFull);
             if (ok) {
                 tc_fence_after();
+                if constexpr (QK4) {
+                    for (int x = 0; x < 2; ++x)
+                        if ((x ? nB : nA) > 0) tmem_cp_sf_atom(tmem + kTmemSfQ + 4u * x, sf_atom_desc(smem_u32(sm.sfq[x])));
+                }
+                sf_k(0);
                 for (int x = 0; x < 2; ++x)
                     if ((x ? nB : nA) > 0) {
-                        issue_qk<D>(tmem + (uint32_t)x * 128u, q_s + (uint32_t)x * (kTile * D), smem_u32(sm.k[0]));
+                        qk(x, 0);
                         mma_commit(&sm.bar_s[x]);
                     }
             }
             // QK^T of key tile 1 as soon as a warpgroup holds tile 0's scores; K slot 0
             // is released once both warpgroups have dequantized tile 0
             if (ok && n_tiles > 1) ok = mbar_wait(&sm.bar_kfull[1 % KS], (1 / KS) & 1, abort_flag, p.status, kSiteFull);
+            if (ok && n_tiles > 1) {
+                tc_fence_after();
+                sf_k(1 % KS);
+            }
             for (int x = 0; ok && x < 2; ++x) {
                 const int nx = x ? nB : nA;
                 if (nx <= 0) continue;
                 ok = mbar_wait(&sm.bar_sfree[x], 0, abort_flag, p.status, kSiteSfree);
                 if (ok && nx > 1) {
                     tc_fence_after();
-                    issue_qk<D>(tmem + (uint32_t)x * 128u, q_s + (uint32_t)x * (kTile * D), smem_u32(sm.k[1 % KS]));
+                    qk(x, 1 % KS);
                     mma_commit(&sm.bar_s[x]);
                 }
             }
@@ -591,8 +641,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // shared memory (a warpgroup releases the two close together).
             for (int it = 0; ok && it < n_tiles; ++it) {
                 const int k1 = (it + 1) % KS, k2 = (it + 2) % KS, sv = it % VS;
-                if (it + 2 < n_tiles && !mbar_wait(&sm.bar_kfull[k2], ((it + 2) / KS) & 1, abort_flag, p.status, kSiteFull))
-                    break;
+                if (it + 2 < n_tiles) {
+                    if (!mbar_wait(&sm.bar_kfull[k2], ((it + 2) / KS) & 1, abort_flag, p.status, kSiteFull)) break;
+                    tc_fence_after();
+                    sf_k(k2);
+                }
                 bool brk = false, v_ready = false;
                 for (int x = 0; x < 2; ++x) {
                     const int nx = x ? nB : nA;
@@ -600,7 +653,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         if (!mbar_wait(&sm.bar_sfree[x], (it + 1) & 1, abort_flag, p.status, kSiteSfree)) { brk = true; break; }
                         if (it + 2 < nx) {
                             tc_fence_after();
-                            issue_qk<D>(tmem + (uint32_t)x * 128u, q_s + (uint32_t)x * (kTile * D), smem_u32(sm.k[k2]));
+                            qk(x, k2);
                             mma_commit(&sm.bar_s[x]);
                         }
                     }
@@ -638,34 +691,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // one copy of the softmax code serves both tiles (instruction-cache footprint)
     const int X = warp >> 3;
     if (X == 0 || hasB)
-        softmax_role<D, PV16>(sm, p, tmem, X, X ? tB : tA, X ? nB : nA, bh, o_base, n_q, n_kv, abort_flag);
+        softmax_role<D, PV16, QK4>(sm, p, tmem, X, X ? tB : tA, X ? nB : nA, bh, o_base, n_q, n_kv, abort_flag);
     tc_fence_before();
     __syncthreads();
 }
 
-template <int D, bool RT, bool PV16>
+template <int D, bool RT, bool PV16, bool QK4 = false>
 static cudaError_t launch_attention_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                       const AttnParams &p, cudaStream_t stream) {
     const size_t smem = sizeof(AttnSmem<D, PV16>) + 1024;
     static_assert(sizeof(AttnSmem<D, PV16>) + 1024 <= 227 * 1024, "shared memory of one CTA");
     cudaError_t e =
-        cudaFuncSetAttribute(attn_fwd_kernel<D, RT, PV16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(attn_fwd_kernel<D, RT, PV16, QK4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((p.Tq + 1) / 2) * (unsigned)p.BH;
     // Heads per block of the CTA order: as many key/value heads as fit kKvL2Budget
     // bytes of K codes + V^T codes, times the query heads that share each.
     AttnParams pp = p;
-    const size_t kv_head_bytes = (PV16 ? 3ull : 2ull) * (size_t)p.nk_pad * D;
+    const size_t kv_head_bytes = (size_t)p.nk_pad * D * ((PV16 ? 2 : 1) + (QK4 ? 0.5 : 1.0));
     const size_t kv_heads = kv_head_bytes ? kKvL2Budget / kv_head_bytes : 0;
     const size_t hb = (kv_heads < 1 ? 1 : kv_heads) * (size_t)p.group;
     pp.head_block = (int)(hb < (size_t)p.BH ? hb : (size_t)p.BH);
     if (pp.head_block < 1) pp.head_block = 1;
-    attn_fwd_kernel<D, RT, PV16><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, pp);
+    attn_fwd_kernel<D, RT, PV16, QK4><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, pp);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                              const AttnParams &p, int d, cudaStream_t stream) {
+    if (p.fp4) {   // the 4-bit mode: d = 64, FP8 P / V (checked by the callers)
+        if (d != 64 || p.pv16) return cudaErrorInvalidValue;
+        return launch_attention_d<64, true, false, true>(tq, tk, tv, p, stream);
+    }
     if (p.pv16) {
         if (d == 128) return launch_attention_d<128, true, true>(tq, tk, tv, p, stream);
         return launch_attention_d<64, true, true>(tq, tk, tv, p, stream);

@@ -53,18 +53,6 @@ constexpr size_t kRateSmem = 160u * 1024u;
 // block spans 16 / VEC lanes.  Output: codes packed two per byte (channel 2i in the
 // low nibble), [n_pad][d / 2]; E4M3 scale codes [n_pad][d / 16]; g per tile.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float e4m3_value(uint8_t code) {
-    uint32_t h2;
-    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h2) : "r"((uint32_t)code));
-    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-}
-
-__device__ __forceinline__ uint32_t e2m1x2(float hi, float lo) {
-    uint32_t r;
-    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\tcvt.u32.u8 %0, b;\n\t}" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
 template <int D>
 __global__ void __launch_bounds__(256) debug_quant_fp4_kernel(const float *__restrict__ xs, int n_rows,
                                                               uint8_t *__restrict__ codes, uint8_t *__restrict__ sf,

@@ -213,6 +213,47 @@ __device__ __forceinline__ RingCtl<D> ring_setup(const CUtensorMap *tm, int nhd,
     return rc;
 }
 
+// FP4 (block-scaled E2M1) codes of this warp's 16 rows of a 128-row tile with tile
+// scale g (the microscaling form of the 4-bit Q / K of "SageAttention2", abstract;
+// "SageAttention3: Microscaling FP4 Attention" among the notes' related papers): per
+// row and 16 channels the E4M3 scale sf = E4M3(fp32(fp32(amax / g) / 6)) (1.0 for an
+// all-zero block, 2^-9 where it rounds to zero), per element the E2M1 code of the IEEE
+// quotient x / fp32(g sf).  Codes go to codes_tile ([128][D/2], channel 2c in the low
+// nibble of byte c); the scales into the tile's 512-byte atoms (row m, block b at byte
+// 16 (m mod 32) + 4 (m / 32) + (b mod 4) of atom b / 4), the layout tcgen05.cp moves into
+// tensor memory for kind::mxf4nvf4.
+template <int D>
+__device__ __forceinline__ void fp4_rows(const float (&x)[kRowsPerWarp][D / 32], float g, uint8_t *codes_tile,
+                                         uint8_t *atoms_tile, int warp, int lane) {
+    constexpr int VEC = D / 32, LPB = 16 / VEC;   // lanes per 16-channel block
+#pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+        const int r = warp * kRowsPerWarp + i;
+        float bm = 0.f;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) bm = fmaxf(bm, fabsf(x[i][v]));
+#pragma unroll
+        for (int o = 1; o < LPB; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, o));
+        uint8_t sc = 0x38;
+        if (bm != 0.f) {
+            sc = (uint8_t)(pack_e4m3x4(__fdiv_rn(__fdiv_rn(bm, g), 6.f), 0.f, 0.f, 0.f) & 0xFFu);
+            if ((sc & 0x7F) == 0) sc = 0x01;
+        }
+        const float delta = __fmul_rn(g, e4m3_value(sc));
+        if (lane % LPB == 0) {
+            const int b = lane / LPB;
+            atoms_tile[(b >> 2) * 512 + 16 * (r & 31) + 4 * (r >> 5) + (b & 3)] = sc;
+        }
+        uint32_t packed = 0;   // VEC codes, 4 bits each, channel lane * VEC + v at bits 4 v
+#pragma unroll
+        for (int v = 0; v < VEC; v += 2)
+            packed |= e2m1x2(__fdiv_rn(x[i][v + 1], delta), __fdiv_rn(x[i][v], delta)) << (4 * v);
+        uint8_t *dst = codes_tile + (size_t)r * (D / 2) + lane * (VEC / 2);
+        if constexpr (VEC == 4) *reinterpret_cast<uint16_t *>(dst) = (uint16_t)packed;
+        else *dst = (uint8_t)packed;
+    }
+}
+
 // Largest |x| over the 16-row groups of warps [w0, w0 + n) of this tile.
 __device__ __forceinline__ float group_amax(const float *wmax, int w0, int n) {
     float am = 0.f;
@@ -376,6 +417,13 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
         __syncthreads();
         const int gw = a.g_q / RPW;  // warps per quantization group (g_q = 32 or 128)
         const float gam = group_amax(s_wmax, (warp / gw) * gw, gw);
+        if (a.fp4) {   // 4-bit Q: the tile scale takes delta_Q's place
+            const float g = (gam == 0.f) ? 1.f : __fdiv_rn(gam, 2688.f);
+            if (lane < RPW) reinterpret_cast<float *>(a.ws + a.L.dq)[(size_t)bh * S.nq_pad + r0 + warp * RPW + lane] = g;
+            fp4_rows<D>(x, g, a.ws + a.L.q8 + ((size_t)bh * S.nq_pad + r0) * (D / 2),
+                        a.ws + a.L.sfq + ((size_t)bh * S.Tq + t) * (D / 64) * 512, warp, lane);
+            continue;
+        }
         const float dl = (gam == 0.f) ? 1.f : __fdiv_rn(gam, 127.f);
         if (lane < RPW) reinterpret_cast<float *>(a.ws + a.L.dq)[(size_t)bh * S.nq_pad + r0 + warp * RPW + lane] = dl;
         const float inv = 1.0f / dl;
@@ -433,6 +481,14 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_
         if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
         const int gw = a.g_k / RPW;  // warps per quantization group (g_k = 16 or 128)
         const float gam = group_amax(s_wmax[k & 1], (warp / gw) * gw, gw);
+        if (a.fp4) {   // 4-bit K: the tile scale takes delta_K's place in every 16-key run
+            const float g = (gam == 0.f) ? 1.f : __fdiv_rn(gam, 2688.f);
+            if (lane == 0)
+                reinterpret_cast<float *>(a.ws + a.L.dk)[(size_t)bh * (S.nk_pad / kKeyRun) + (j0 + warp * RPW) / kKeyRun] = g;
+            fp4_rows<D>(x, g, a.ws + a.L.k8 + ((size_t)bh * S.nk_pad + j0) * (D / 2),
+                        a.ws + a.L.sfk + ((size_t)bh * S.Tk + jt) * (D / 64) * 512, warp, lane);
+            continue;
+        }
         const float dl = (gam == 0.f) ? 1.f : __fdiv_rn(gam, 127.f);
         if (lane == 0)  // one delta_K per 16-key run = this warp's rows
             reinterpret_cast<float *>(a.ws + a.L.dk)[(size_t)bh * (S.nk_pad / kKeyRun) + (j0 + warp * RPW) / kKeyRun] = dl;

@@ -33,6 +33,7 @@ struct Mode {
     int g_q, g_k, smooth_q, smooth_k;
     float p_range, v_range;
     int pv16;
+    int fp4;   // 4-bit Q / K (SAGE_QK_FP4)
 };
 
 sage_status_t read_mode(const sage_quant_mode_t *m, Mode *out) {
@@ -42,8 +43,10 @@ sage_status_t read_mode(const sage_quant_mode_t *m, Mode *out) {
         case SAGE_QK_PER_BLOCK: out->g_q = 128; out->g_k = 128; break;
         case SAGE_QK_PER_WARP: out->g_q = 32; out->g_k = 128; break;
         case SAGE_QK_PER_THREADGROUP: out->g_q = 32; out->g_k = 16; break;
+        case SAGE_QK_FP4: out->g_q = 128; out->g_k = 128; break;   // the tile scale spans the tile
         default: return SAGE_ERR_INVALID_ARG;
     }
+    out->fp4 = (d.gran == SAGE_QK_FP4) ? 1 : 0;
     if (!(d.p_range > 0.f && d.p_range <= 448.f) || !(d.v_range > 0.f && d.v_range <= 448.f))
         return SAGE_ERR_INVALID_ARG;
     out->smooth_q = d.smooth_q ? 1 : 0;
@@ -52,6 +55,7 @@ sage_status_t read_mode(const sage_quant_mode_t *m, Mode *out) {
     out->v_range = d.v_range;
     if (d.pv_fp16 != 0 && d.pv_fp16 != 1) return SAGE_ERR_INVALID_ARG;
     out->pv16 = d.pv_fp16;
+    if (out->fp4 && out->pv16) return SAGE_ERR_UNSUPPORTED;   // the 4-bit mode pairs with FP8 P / V
     return SAGE_OK;
 }
 
@@ -113,10 +117,13 @@ bool encode_2d16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
 // transposed V codes ([BH*d][nk_pad] bytes, d x 128 boxes).
 bool make_maps(const Shape &s, const uint8_t *ws, CUtensorMap *tq, CUtensorMap *tk, CUtensorMap *tv) {
     const WsLayout L = ws_layout(s);
-    const CUtensorMapSwizzle swz_qk = (s.d == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     const uint64_t d = (uint64_t)s.d;
-    if (tq && !encode_2d(tq, ws + L.q8, d, (uint64_t)s.BH * s.nq_pad, d, (uint32_t)d, kTile, swz_qk)) return false;
-    if (tk && !encode_2d(tk, ws + L.k8, d, (uint64_t)s.BH_kv * s.nk_pad, d, (uint32_t)d, kTile, swz_qk)) return false;
+    // INT8 rows of d bytes (128- / 64-byte swizzle); FP4 rows of d / 2 bytes (64- / 32-byte swizzle)
+    const uint64_t rb = s.fp4 ? d / 2 : d;
+    const CUtensorMapSwizzle swz_qk = (rb == 128) ? CU_TENSOR_MAP_SWIZZLE_128B
+                                      : (rb == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+    if (tq && !encode_2d(tq, ws + L.q8, rb, (uint64_t)s.BH * s.nq_pad, rb, (uint32_t)rb, kTile, swz_qk)) return false;
+    if (tk && !encode_2d(tk, ws + L.k8, rb, (uint64_t)s.BH_kv * s.nk_pad, rb, (uint32_t)rb, kTile, swz_qk)) return false;
     if (tv && !s.pv16 &&
         !encode_2d(tv, ws + L.vt8, (uint64_t)s.nk_pad, (uint64_t)s.BH_kv * d, (uint64_t)s.nk_pad, kTile, (uint32_t)d,
                    CU_TENSOR_MAP_SWIZZLE_128B))
@@ -228,6 +235,7 @@ sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype
     a.smooth_k = m.smooth_k;
     a.v_range = m.v_range;
     a.pv16 = m.pv16;
+    a.fp4 = m.fp4;
     a.ws = ws;
     a.L = ws_layout(s);
     if (launch_prepass(a, stream) != cudaSuccess) return SAGE_ERR_CUDA;
@@ -281,6 +289,9 @@ sage_status_t run_attention(void *o, int dtype, int layout, const Shape &s, int 
     const float scale = (sm_scale > 0.f) ? sm_scale : 1.0f / sqrtf((float)s.d);
     p.scale_log2 = scale * 1.4426950408889634f;
     p.pv16 = m.pv16;
+    p.fp4 = m.fp4;
+    p.sfq = ws + L.sfq;
+    p.sfk = ws + L.sfk;
     p.log2_pr = m.pv16 ? 0.f : log2f(m.p_range);  // FP16 P~ is not scaled (Pr = 1)
     p.status = reinterpret_cast<int *>(const_cast<uint8_t *>(ws) + L.status);
     p.fault_inject = fault_inject;
@@ -314,6 +325,8 @@ sage_status_t check_fwd_args(const void *q, const void *k, const void *v, const 
     SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
     s.pv16 = m.pv16;
+    s.fp4 = m.fp4;
+    if (m.fp4 && d != 64) return SAGE_ERR_UNSUPPORTED;   // FP4 attention: d = 64 (tensor-memory budget)
     if (s.BH == 0 || n_q == 0) return SAGE_OK;
     if (!q || !o || (n_kv > 0 && (!k || !v))) return SAGE_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(o) || (k && !aligned16(k)) || (v && !aligned16(v))) return SAGE_ERR_UNSUPPORTED;
@@ -341,6 +354,7 @@ size_t sage_workspace_bytes_mode(int B, int H, int H_kv, int n_q, int n_kv, int 
     Mode m;
     if (check_sizes(B, H, H_kv, n_q, n_kv, d, &s) != SAGE_OK || read_mode(mode, &m) != SAGE_OK) return 0;
     s.pv16 = m.pv16;
+    s.fp4 = m.fp4;
     return ws_layout(s).total;
 }
 
@@ -354,6 +368,7 @@ int64_t sage_workspace_offset_mode(int B, int H, int H_kv, int n_q, int n_kv, in
     Mode m;
     if (check_sizes(B, H, H_kv, n_q, n_kv, d, &s) != SAGE_OK || read_mode(mode, &m) != SAGE_OK) return -1;
     s.pv16 = m.pv16;
+    s.fp4 = m.fp4;
     const WsLayout L = ws_layout(s);
     switch (which) {
         case SAGE_WS_Q8: return (int64_t)L.q8;
@@ -367,6 +382,8 @@ int64_t sage_workspace_offset_mode(int B, int H, int H_kv, int n_q, int n_kv, in
         case SAGE_WS_DS: return (int64_t)L.ds;
         case SAGE_WS_QS_KBAR: return (int64_t)L.qs_kbar;
         case SAGE_WS_LSE: return (int64_t)L.lse;
+        case SAGE_WS_SFQ: return (int64_t)L.sfq;
+        case SAGE_WS_SFK: return (int64_t)L.sfk;
         default: return -1;
     }
 }
@@ -388,6 +405,7 @@ sage_status_t sage_quant_qk_gqa(const void *q, const void *k, int dtype, int lay
     SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
     s.pv16 = m.pv16;
+    s.fp4 = m.fp4;
     if (s.BH == 0 || (n_q == 0 && n_kv == 0)) return SAGE_OK;
     if ((n_q > 0 && !q) || (n_kv > 0 && !k)) return SAGE_ERR_INVALID_ARG;
     if ((q && !aligned16(q)) || (k && !aligned16(k))) return SAGE_ERR_UNSUPPORTED;
@@ -411,6 +429,7 @@ sage_status_t sage_quant_v_gqa(const void *v, int dtype, int layout, int B, int 
     SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
     s.pv16 = m.pv16;
+    s.fp4 = m.fp4;
     if (s.BH == 0 || n_kv == 0) return SAGE_OK;
     if (!v) return SAGE_ERR_INVALID_ARG;
     if (!aligned16(v)) return SAGE_ERR_UNSUPPORTED;
@@ -434,6 +453,8 @@ sage_status_t sage_attn_fwd_prequant_gqa(void *o, int dtype, int layout, int B, 
     SAGE_TRY(check_sizes(B, H, H_kv, n_q, n_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
     s.pv16 = m.pv16;
+    s.fp4 = m.fp4;
+    if (m.fp4 && d != 64) return SAGE_ERR_UNSUPPORTED;   // FP4 attention: d = 64 (tensor-memory budget)
     if (s.BH == 0 || n_q == 0) return SAGE_OK;
     if (!o) return SAGE_ERR_INVALID_ARG;
     if (!aligned16(o)) return SAGE_ERR_UNSUPPORTED;
@@ -465,6 +486,7 @@ sage_status_t sage_attn_fwd_gqa(const void *q, const void *k, const void *v, voi
     check_sizes(B, H, H_kv, n_q, n_kv, d, &s);   // both validated by check_fwd_args
     read_mode(mode, &m);
     s.pv16 = m.pv16;
+    s.fp4 = m.fp4;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (plan == kFwdZeroOut)
         return cudaMemsetAsync(o, 0, (size_t)s.BH * n_q * d * 2, st) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
@@ -497,6 +519,8 @@ sage_status_t sage_attn_fwd_varlen(const void *q, const void *k, const void *v, 
     SAGE_TRY(check_sizes(B, H, H_kv, max_seqlen_q, max_seqlen_kv, d, &s));
     SAGE_TRY(read_mode(mode, &m));
     s.pv16 = m.pv16;
+    s.fp4 = m.fp4;
+    if (m.fp4 && d != 64) return SAGE_ERR_UNSUPPORTED;   // FP4 attention: d = 64 (tensor-memory budget)
     s.varlen = 1;
     s.total_q = total_q;
     s.total_kv = total_kv;

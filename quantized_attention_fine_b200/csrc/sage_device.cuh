@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -371,6 +372,19 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, fl
         "mov.b32 %0, {lo, hi};\n\t}"
         : "=r"(r)
         : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+    return r;
+}
+
+// Value of an E4M3 code (exact, via the hardware E4M3 -> f16 conversion).
+__device__ __forceinline__ float e4m3_value(uint8_t code) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h2) : "r"((uint32_t)code));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+// Two E2M1 codes (round to nearest even, saturating): `lo` in bits 0-3, `hi` in 4-7.
+__device__ __forceinline__ uint32_t e2m1x2(float hi, float lo) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\tcvt.u32.u8 %0, b;\n\t}" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
 

@@ -26,12 +26,13 @@ struct Shape {
     int BH, BH_kv, Tq, Tk, nq_pad, nk_pad, n_chunks;
     int varlen, total_q, total_kv;
     int pv16;   // FP16 P / V mode: the transposed V holds 2 bytes per element
+    int fp4;    // FP4 Q / K mode: E2M1 codes and E4M3 scale atoms (sfq, sfk regions)
 };
 
 inline Shape make_shape(int B, int H, int H_kv, int n_q, int n_kv, int d) {
     Shape s;
     s.B = B; s.H = H; s.H_kv = H_kv; s.n_q = n_q; s.n_kv = n_kv; s.d = d;
-    s.varlen = 0; s.total_q = 0; s.total_kv = 0; s.pv16 = 0;
+    s.varlen = 0; s.total_q = 0; s.total_kv = 0; s.pv16 = 0; s.fp4 = 0;
     s.BH = B * H;
     s.BH_kv = B * H_kv;
     s.Tq = (n_q + kTile - 1) / kTile;
@@ -45,7 +46,7 @@ inline Shape make_shape(int B, int H, int H_kv, int n_q, int n_kv, int d) {
 
 // Byte offsets of every workspace region.
 struct WsLayout {
-    size_t status, q8, k8, vt8, dq, dk, dv, qbar, kbar, ds, qs_kbar, lse, ksum_part, vmax_part, total;
+    size_t status, q8, k8, vt8, dq, dk, dv, qbar, kbar, ds, qs_kbar, lse, ksum_part, vmax_part, sfq, sfk, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -69,6 +70,9 @@ inline WsLayout ws_layout(const Shape &s) {
     w.lse = take(BH * s.nq_pad * 4);
     w.ksum_part = take(BHk * s.n_chunks * d * 8);
     w.vmax_part = take(BHk * s.n_chunks * d * 4);
+    // FP4 scale atoms: 512 bytes per 128-row tile and 64-channel chunk
+    w.sfq = take(s.fp4 ? BH * s.Tq * (d / 64) * 512 : 0);
+    w.sfk = take(s.fp4 ? BHk * s.Tk * (d / 64) * 512 : 0);
     w.total = off;
     return w;
 }
@@ -111,6 +115,7 @@ struct PrepassArgs {
     int g_q, g_k, smooth_q, smooth_k;
     float v_range;
     int pv16;   // FP16 V (no per-channel scale: delta_V = 1) instead of E4M3 codes
+    int fp4;    // FP4 Q / K (E2M1 codes, E4M3 block scales, per-tile fp32 scales)
     uint8_t *ws;
     WsLayout L;
 };
@@ -130,6 +135,8 @@ struct AttnParams {
     int causal;
     int use_ds;         // 0: Q smoothing off, dS not read
     int pv16;           // FP16 P~ and V, kind::f16 PV (log2_pr is then 0)
+    int fp4;            // FP4 Q / K, QK^T on kind::mxf4nvf4 (d = 64)
+    const uint8_t *sfq, *sfk;   // FP4 scale atoms
     int out_bf16;
     float scale_log2;   // sm_scale * log2(e)
     float log2_pr;      // log2(Pr)

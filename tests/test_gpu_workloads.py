@@ -105,3 +105,29 @@ def test_full_size_fp16_pv_mode_sampled():
         og = to_np64(o[0, h].cpu())[rows]
         assert_close_to_oracle(og, oo[rows], "pv16 head %d" % h)
         assert cos(og, _full_precision_rows(qh, kh, vh, rows, True)) >= O_COS_FULL
+
+
+def test_full_size_fp4_video_dit_sampled():
+    """The 4-bit mode at the video_dit size (B2 H48 N17776 d64, the d = 64 workload it
+    runs on), in the launch configuration of `bench.py --qk fp4`: sampled heads and Q
+    blocks against the oracle's FP4 mode, and against full precision."""
+    w = wl.VIDEO_DIT
+    q, k, v = wl.generate(w)
+    dev = torch.device("cuda", 0)
+    mode = sage.QuantMode.make("fp4")
+    ws = sage.make_workspace(w.B, w.H, w.N_q, w.N_kv, w.d, device=dev, qk_fp4=True)
+    sage.quant_qk(q.to(dev), k.to(dev), mode=mode, workspace=ws)
+    sage.quant_v(v.to(dev), n_q=w.N_q, mode=mode, workspace=ws)
+    o = sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode)
+    assert sage.get_device_status(ws) == (0, 0)
+    tq = -(-w.N_q // 128)
+    blocks = [0, tq // 2, tq - 1]
+    rows = rows_of_blocks(w.N_q, blocks)
+    for b, h in ((0, 0), (w.B - 1, w.H - 1)):
+        qh, kh, vh = to_np64(q[b, h]), to_np64(k[b, h]), to_np64(v[b, h])
+        pre = oracle.prepass_head(qh, kh, vh, quant=oracle.QK_FP4_PV_FP8)
+        oo = oracle.attn_head(pre, causal=False, qblocks=blocks)
+        og = to_np64(o[b, h].cpu())[rows]
+        assert_close_to_oracle(og, oo[rows], "fp4 video_dit head (%d,%d)" % (b, h))
+        # FP4 is the lossier mode: the oracle's own FP4 cosine on this workload is 0.9896
+        assert cos(og, _full_precision_rows(qh, kh, vh, rows, False)) >= 0.98
