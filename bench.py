@@ -8,7 +8,10 @@ One step = one pass of the whole hot path over one batch of synthetic input
 already resident in HBM, through the public C-ABI call sage_attn_fwd: the
 smoothing/quantization pre-pass of Q, K and V, the dS product, and the fused
 attention kernel.  A second timed loop runs the attention kernel alone
-(sage_attn_fwd_prequant on the same workspace) for its roofline figure.  Metric: attention TOPS
+(sage_attn_fwd_prequant on the same workspace) for its roofline figure.  With
+--fuse-q the step is sage_attn_fwd_qfused_gqa instead (K / V pre-pass, then the
+attention kernel that quantizes its own Q tiles and forms dS itself), and the second
+loop times that kernel (the same entry without v).  Metric: attention TOPS
 = 4 B H N_q N_kv d / t (halved when causal), summed over all ranks.  With N > 1 the
 ranks compute disjoint slices of one seeded global problem, split by heads (each head's
 K mean, delta_V, dS and O depend on that head alone, so no data-path collective is
@@ -37,8 +40,10 @@ UNIT = "TOPS"
 SPEC_INT8_TOPS = 4500.0          # B200 dense INT8 / FP8 datasheet figure
 FALLBACK_BF16_TFLOPS = 1590.0    # pool measurement used when MEASURED_PEAKS.json is absent
 # library kernels per step of sage_attn_fwd: kv_stats, kv_finalize, quant_q, quant_k,
-# quant_v, ds_gemm, attn_fwd_kernel
+# quant_v, ds_gemm, attn_fwd_kernel; with --fuse-q: kv_stats, kv_finalize, quant_k,
+# quant_v, attn_fwd_kernel
 LAUNCHES_PER_STEP = 7
+LAUNCHES_PER_STEP_FUSE_Q = 5
 KERNEL_SOURCES = ["quantized_attention_fine_b200/csrc/attn_fwd.cu", "quantized_attention_fine_b200/csrc/attn_mma.cuh",
                   "quantized_attention_fine_b200/csrc/sage_device.cuh"]
 
@@ -57,6 +62,8 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--pv", default="fp8", choices=["fp8", "fp16"],
                     help="PV precision: fp8 (the method's default) or fp16 (the qk_int8_pv_fp16 mode)")
+    ap.add_argument("--fuse-q", action="store_true",
+                    help="quantize Q inside the attention kernel (sage_attn_fwd_qfused_gqa) instead of the pre-pass")
     ap.add_argument("--qk", default="int8", choices=["int8", "fp4"],
                     help="Q / K precision: int8 (grouped INT8, the default) or fp4 (the 4-bit mode: block-scaled "
                          "E2M1 on tcgen05.mma kind::mxf4nvf4; d = 64 workloads)")
@@ -356,8 +363,10 @@ def main():
     mode = sage.QuantMode.make(gran, pv=args.pv)
     stream = torch.cuda.current_stream(dev)
 
+    fuse_q = bool(args.fuse_q) and not fp4
+
     def step_eager():
-        sage.attn_fwd(q, k, v, causal=w.causal, out=out, workspace=ws, pv=args.pv, granularity=gran)
+        sage.attn_fwd(q, k, v, causal=w.causal, out=out, workspace=ws, pv=args.pv, granularity=gran, fuse_q=fuse_q)
 
     step = step_eager
     graph = None
@@ -369,8 +378,11 @@ def main():
             step_eager()
         step = graph.replay
 
-    def attn_only():
-        sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode, out=out)
+    def attn_only():   # the attention kernel of the step, on the workspace the step filled
+        if fuse_q:
+            sage.attn_fwd_qfused(q, k, ws, causal=w.causal, mode=mode, out=out)
+        else:
+            sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode, out=out)
 
     for _ in range(args.warmup):
         step()
@@ -447,7 +459,7 @@ def main():
                 if i >= 2:
                     stream.wait_event(ev_out[i - 2])     # and its output has been copied out
                 sage.attn_fwd(qd, kd, vd, causal=w.causal, out=od, workspace=ws, stream=stream, pv=args.pv,
-                              granularity=gran)
+                              granularity=gran, fuse_q=fuse_q)
                 ev_comp[i].record(stream)
                 s_out.wait_event(ev_comp[i])
                 with torch.cuda.stream(s_out):
@@ -516,17 +528,20 @@ def main():
                                     else "per_threadgroup (g_q=32, g_k=16)"),
                        **({"pv": "fp16 (qk_int8_pv_fp16)"} if pv16 else {"pv": "fp8", "pr": 448, "vr": 448})),
         "attn_kernel_tops": attn_tops, "attn_kernel_ms": attn_avg_ms, "prepass_ms": pre_avg_ms,
-        "step_call": ("sage_attn_fwd (pre-pass + dS + attention)" + (", replayed from a CUDA graph" if args.graph else "")
+        "step_call": (("sage_attn_fwd_qfused_gqa (K / V pre-pass + attention with Q quantization and dS in the kernel)"
+                       if fuse_q else "sage_attn_fwd (pre-pass + dS + attention)")
+                      + (", replayed from a CUDA graph" if args.graph else "")
                       + "; prepass_ms = ms_per_step - attn_kernel_ms"),
         "attn_frac_of_spec_4500": attn_tops / SPEC_INT8_TOPS,
         "roofline": {"bound": "tensor", "achieved": attn_tops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": attn_tops / peak, "traffic": None if (pv16 or fp4) else recorded_traffic(w.name),
+                     "frac": attn_tops / peak, "traffic": None if (pv16 or fp4 or fuse_q) else recorded_traffic(w.name),
                      "frac_of_tcgen05_probe": (attn_tops / probe) if probe else None,
                      "tcgen05_probe_peak": probe,
                      "peak_source": peak_note,
-                     "kernel": "attn_fwd_kernel<%d>%s" % (d, " (4-bit QK)" if fp4 else "")},
+                     "kernel": "attn_fwd_kernel<%d>%s" % (d, " (4-bit QK)" if fp4 else
+                                                          (" (Q quantized in the kernel)" if fuse_q else ""))},
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-        "gpu_launches": args.steps * LAUNCHES_PER_STEP,
+        "gpu_launches": args.steps * (LAUNCHES_PER_STEP_FUSE_Q if fuse_q else LAUNCHES_PER_STEP),
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -189,6 +189,35 @@ SAGE_API sage_status_t sage_attn_fwd_gqa(const void *q, const void *k, const voi
                                          const sage_quant_mode_t *mode,
                                          void *workspace, size_t workspace_bytes, void *stream);
 
+/* The whole forward with Q quantized inside the attention kernel ("SageAttention2"
+ * abstract: Q is smoothed per 128-row block, so a block's mean, delta_Q and codes need
+ * only that block):
+ *   K / V pre-pass (K mean, K codes, delta_V, V codes)  ->  attention
+ * where the attention kernel reads the caller's 16-bit Q tiles, smooths and quantizes
+ * them (codes, delta_Q and qbar bit-identical to sage_quant_qk's), and forms the dS
+ * bias qbar . K of every key tile from the caller's K on one of its warps.  The
+ * results equal sage_attn_fwd_gqa's up to the rounding of dS (its products are summed
+ * in another order).  On B200 this path is slower than sage_attn_fwd_gqa (the dS
+ * warp reads every key tile's 16-bit K again and its products run on the warp-level
+ * tensor-core path); it is kept as an alternative, not the default.
+ * With v == NULL only the attention runs, on a workspace whose K / V parts were
+ * filled for the same sizes and mode (by sage_quant_qk + sage_quant_v, or by an
+ * earlier call).  The workspace then holds qbar (SAGE_WS_QBAR) and delta_Q
+ * (SAGE_WS_DQ) of the call; SAGE_WS_Q8, SAGE_WS_DS and SAGE_WS_QS_KBAR are not
+ * written (the Q codes are, under sage_debug_set_q_code_dump).  Arguments and errors
+ * as sage_attn_fwd_gqa; SAGE_ERR_UNSUPPORTED for the 4-bit mode (SAGE_QK_FP4), whose
+ * Q is quantized in the pre-pass. */
+SAGE_API sage_status_t sage_attn_fwd_qfused_gqa(const void *q, const void *k, const void *v, void *o, int dtype,
+                                                int layout, int B, int H, int H_kv, int n_q, int n_kv, int d,
+                                                int causal, float sm_scale, const sage_quant_mode_t *mode,
+                                                void *workspace, size_t workspace_bytes, void *stream);
+
+/* Diagnostic switch (process-wide, not for concurrent use): while enabled (1), forward
+ * calls that quantize Q inside the attention kernel also write the Q codes to the
+ * workspace's SAGE_WS_Q8 view, so that they can be compared with sage_quant_qk's.
+ * 0 disables (the default).  SAGE_ERR_INVALID_ARG for other values. */
+SAGE_API sage_status_t sage_debug_set_q_code_dump(int enable);
+
 /* ---- variable-length (packed) batches -------------------------------------------
  * B sequences of different lengths packed token-major, as in the pages' varlen
  * kernels (the deployment guide's "dynamic sequence length" tip: a per-block causal
@@ -214,6 +243,13 @@ SAGE_API sage_status_t sage_attn_fwd_varlen(const void *q, const void *k, const 
                                             int max_seqlen_q, int max_seqlen_kv, int d, int causal,
                                             float sm_scale, const sage_quant_mode_t *mode,
                                             void *workspace, size_t workspace_bytes, void *stream);
+/* The same with Q quantized inside the attention kernel (as sage_attn_fwd_qfused_gqa). */
+SAGE_API sage_status_t sage_attn_fwd_varlen_qfused(const void *q, const void *k, const void *v, void *o, int dtype,
+                                                   const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_kv,
+                                                   int B, int H, int H_kv, int total_q, int total_kv,
+                                                   int max_seqlen_q, int max_seqlen_kv, int d, int causal,
+                                                   float sm_scale, const sage_quant_mode_t *mode,
+                                                   void *workspace, size_t workspace_bytes, void *stream);
 
 /* The whole forward, exactly as sage_attn_fwd, for callers that must not allocate
  * device memory (for example a plugin whose host application owns every device

@@ -120,6 +120,9 @@ def load_library():
         lib.sage_debug_quant_fp4.argtypes = [P, I, I, P, P, P, P]
         lib.sage_debug_qk_tile_fp4.argtypes = [P, P, P, P, I, P, P, P]
         lib.sage_debug_attn_fault_inject.argtypes = [P, I, I, I, I, I, I, I, I, P, S, P]
+        lib.sage_attn_fwd_qfused_gqa.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, F, QM, P, S, P]
+        lib.sage_attn_fwd_varlen_qfused.argtypes = [P, P, P, P, I, P, P] + [I] * 9 + [F, QM, P, S, P]
+        lib.sage_debug_set_q_code_dump.argtypes = [I]
         lib.sage_version.restype = ctypes.c_char_p
         for fn in ("sage_quant_qk", "sage_quant_v", "sage_attn_fwd_prequant", "sage_attn_fwd",
                    "sage_quant_qk_gqa", "sage_quant_v_gqa", "sage_attn_fwd_prequant_gqa", "sage_attn_fwd_gqa",
@@ -127,7 +130,8 @@ def load_library():
                    "sage_get_device_status", "sage_debug_qk_tile", "sage_debug_pv_accumulate",
                    "sage_debug_pv_accumulate_f16acc", "sage_debug_mma_rate", "sage_debug_quant_fp4",
                    "sage_debug_qk_tile_fp4",
-                   "sage_debug_attn_fault_inject"):
+                   "sage_debug_attn_fault_inject", "sage_attn_fwd_qfused_gqa", "sage_attn_fwd_varlen_qfused",
+                   "sage_debug_set_q_code_dump"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -317,10 +321,41 @@ def attn_fwd_prequant(workspace: Workspace, *, dtype, layout="HND", causal=False
     return (out, workspace.lse()) if return_lse else out
 
 
+def attn_fwd_qfused(q, k, workspace: Workspace, *, causal=False, sm_scale=None, layout="HND", mode=None, out=None,
+                    stream=None, return_lse=False):
+    """The attention half of ``attn_fwd(..., fuse_q=True)``: Q quantized and the dS bias
+    formed inside the attention kernel, from q, k and a workspace whose K / V parts hold
+    the pre-pass of k and v (quant_qk + quant_v, or an earlier attn_fwd call, with the
+    same sizes and mode)."""
+    torch = _torch()
+    B, H, H_kv, n_q, n_kv, d = _shape(q, k, layout)
+    if (B, H, n_q, n_kv, d) != tuple(workspace.dims) or H_kv != workspace.H_kv:
+        raise ValueError("q, k do not match the workspace sizes")
+    mode = mode or QuantMode.make()
+    if bool(mode.pv_fp16) != workspace.pv_fp16 or (mode.gran == QK_FP4) != workspace.qk_fp4:
+        raise ValueError("the mode's pv / qk setting does not match the workspace")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(load_library().sage_attn_fwd_qfused_gqa(_ptr(q), _ptr(k), None, _ptr(out), _dtype_code(q), _LAYOUTS[layout],
+                                                   B, H, H_kv, n_q, n_kv, d, int(bool(causal)),
+                                                   float(sm_scale or 0.0), ctypes.byref(mode),
+                                                   ctypes.c_void_p(workspace.ptr), workspace.nbytes,
+                                                   _stream_handle(stream)), "sage_attn_fwd_qfused_gqa")
+    return (out, workspace.lse()) if return_lse else out
+
+
+def debug_set_q_code_dump(enable: bool):
+    """While enabled, forward calls that quantize Q inside the attention kernel also
+    write the Q codes to the workspace's q8 view (process-wide diagnostic switch)."""
+    _check(load_library().sage_debug_set_q_code_dump(int(bool(enable))), "sage_debug_set_q_code_dump")
+
+
 def attn_fwd(q, k, v, *, causal=False, sm_scale=None, layout="HND", granularity="per_threadgroup",
              smooth_q=True, smooth_k=True, p_range=448.0, v_range=448.0, pv="fp8", out=None, workspace=None,
-             stream=None, return_lse=False):
-    """O = quantized attention of q, k, v (pre-pass + fused kernel, enqueued on the current stream).
+             stream=None, return_lse=False, fuse_q=False):
+    """O = quantized attention of q, k, v (pre-pass + fused kernel, enqueued on the current
+    stream).  fuse_q: quantize Q inside the attention kernel instead of the pre-pass
+    (sage_attn_fwd_qfused_gqa; slower on B200, kept as an alternative).
 
     k and v may have fewer heads than q (grouped-query attention): query head h
     reads key/value head h // (H // H_kv).  With return_lse, returns (O, LSE), LSE the
@@ -335,17 +370,19 @@ def attn_fwd(q, k, v, *, causal=False, sm_scale=None, layout="HND", granularity=
     ws = _ws_for(workspace, B, H, H_kv, n_q, n_kv, d, q.device, mode.pv_fp16, mode.gran == QK_FP4)
     if out is None:
         out = torch.empty_like(q)
-    _check(load_library().sage_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q),
-                                            _LAYOUTS[layout], B, H, H_kv, n_q, n_kv, d, int(bool(causal)),
-                                            float(sm_scale or 0.0), ctypes.byref(mode), ctypes.c_void_p(ws.ptr),
-                                            ws.nbytes, _stream_handle(stream)), "sage_attn_fwd_gqa")
+    fn = "sage_attn_fwd_qfused_gqa" if fuse_q else "sage_attn_fwd_gqa"
+    _check(getattr(load_library(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q),
+                                       _LAYOUTS[layout], B, H, H_kv, n_q, n_kv, d, int(bool(causal)),
+                                       float(sm_scale or 0.0), ctypes.byref(mode), ctypes.c_void_p(ws.ptr),
+                                       ws.nbytes, _stream_handle(stream)), fn)
     return (out, ws.lse()) if return_lse else out
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, max_seqlen_q=None, max_seqlen_kv=None, causal=False,
                     sm_scale=None, granularity="per_threadgroup", smooth_q=True, smooth_k=True, p_range=448.0,
-                    v_range=448.0, pv="fp8", out=None, workspace=None, stream=None, return_lse=False):
-    """Quantized attention of a packed batch of variable-length sequences.
+                    v_range=448.0, pv="fp8", out=None, workspace=None, stream=None, return_lse=False, fuse_q=False):
+    """Quantized attention of a packed batch of variable-length sequences (fuse_q: Q
+    quantized inside the attention kernel, as in ``attn_fwd``).
 
     q: [total_q, H, d]; k, v: [total_kv, H_kv, d] (H_kv divides H); cu_seqlens_q,
     cu_seqlens_kv: int32 CUDA tensors of B + 1 offsets.  Sequence b is attended on its
@@ -375,11 +412,12 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_kv, *, max_seqlen_q=None, 
     ws = _ws_for(workspace, B, H, H_kv, max_seqlen_q, max_seqlen_kv, d, q.device, mode.pv_fp16, mode.gran == QK_FP4)
     if out is None:
         out = torch.empty_like(q)
-    _check(load_library().sage_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q),
-                                               _ptr(cu_seqlens_q), _ptr(cu_seqlens_kv), B, H, H_kv, total_q, total_kv,
-                                               int(max_seqlen_q), int(max_seqlen_kv), d, int(bool(causal)),
-                                               float(sm_scale or 0.0), ctypes.byref(mode), ctypes.c_void_p(ws.ptr),
-                                               ws.nbytes, _stream_handle(stream)), "sage_attn_fwd_varlen")
+    fn = "sage_attn_fwd_varlen_qfused" if fuse_q else "sage_attn_fwd_varlen"
+    _check(getattr(load_library(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q),
+                                       _ptr(cu_seqlens_q), _ptr(cu_seqlens_kv), B, H, H_kv, total_q, total_kv,
+                                       int(max_seqlen_q), int(max_seqlen_kv), d, int(bool(causal)),
+                                       float(sm_scale or 0.0), ctypes.byref(mode), ctypes.c_void_p(ws.ptr),
+                                       ws.nbytes, _stream_handle(stream)), fn)
     if return_lse:
         return out, ws.view("lse").view(B, H, -1)[:, :, :max_seqlen_q]
     return out

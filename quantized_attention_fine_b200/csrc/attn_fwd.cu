@@ -47,7 +47,7 @@ namespace sage {
 
 constexpr int kAttnThreads = 640;
 constexpr int kSoftmaxWarps = 16;
-constexpr int kWarpK = 16, kWarpMma = 17, kWarpV = 18;
+constexpr int kWarpK = 16, kWarpMma = 17, kWarpV = 18, kWarpDs = 19;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;
 // 4-bit mode (d = 64): scale atoms of Q tiles A, B at 384 / 388, of K stage s at 392 + 4 s
@@ -72,23 +72,45 @@ enum { kSiteQ = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteS = 4, kSiteP = 5, kSiteO
 // PV16 (the FP16 P / V mode): P~ and V^T are fp16, two 64-key 128-byte swizzle spans
 // per row; the larger tiles leave room for one P buffer per Q tile (a tile's
 // warpgroup writes P(i) once PV(i - 1) has read it) and shorter rings at d = 128.
-template <int D, bool PV16>
+// FQ (Q quantized in the kernel): the raw-K chunk ring of the dS warp takes the
+// room of one K stage at d = 128.
+template <int D, bool PV16, bool FQ = false>
 struct AttnCfg {
-    static constexpr int kKStages = (PV16 && D == 128) ? 3 : 4;
+    static constexpr int kKStages = ((PV16 || FQ) && D == 128) ? 3 : 4;
+    static constexpr int kRawChunks = (D == 128 && PV16) ? 2 : 4;   // FQ: 16-key raw K chunks in flight
     static constexpr int kVStages = PV16 ? (D == 128 ? 2 : 3) : (D == 128 ? 3 : 4);
     static constexpr int kPBufs = PV16 ? 1 : 2;                     // P buffers per Q tile
     static constexpr int kPBytes = kTile * kTile * (PV16 ? 2 : 1);  // one P tile
     static constexpr int kVBytes = D * kTile * (PV16 ? 2 : 1);      // one V^T tile
 };
 
-template <int D, bool PV16>
+// Shared memory of the in-kernel Q quantization and the dS warp (FQ only).
+template <bool FQ, int D, int KS, int RC>
+struct FqSmem {};
+template <int D, int KS, int RC>
+struct __align__(1024) FqSmem<true, D, KS, RC> {
+    // raw K chunks: 16 keys x d of the caller's 16-bit K, as d / 64 boxes of 16 rows x
+    // 128 bytes (128-byte swizzle, 2 KB each)
+    uint8_t kr[RC][D / 64][16 * 128];
+    // qbar of Q tiles A, B as hi / lo 16-bit numbers (rows 2x, 2x + 1), each row in
+    // the order the mma.sync B operand takes it: channel 16 s + w at 16 s + 4 q + e
+    // (w = 2 q + e for w < 8, w = 2 q + 8 + e - 2 for w >= 8)
+    uint16_t qhl[4][D];
+    float qbar[2][D];
+    float wmax[2][8];
+    int kr_coord[3];   // raw K coordinates: row offset, head (or head-major index), batch (-1: head-major)
+    uint64_t bar_kr[RC], bar_dsfull[KS], bar_qraw, bar_qready[2];
+};
+
+template <int D, bool PV16, bool FQ = false>
 struct __align__(1024) AttnSmem {
-    static constexpr int KS = AttnCfg<D, PV16>::kKStages, VS = AttnCfg<D, PV16>::kVStages;
+    static constexpr int KS = AttnCfg<D, PV16, FQ>::kKStages, VS = AttnCfg<D, PV16, FQ>::kVStages;
+    static constexpr int RC = AttnCfg<D, PV16, FQ>::kRawChunks;
     uint8_t q[2][kTile * D];
     uint8_t k[KS][kTile * D];
-    uint8_t v[VS][AttnCfg<D, PV16>::kVBytes];
+    uint8_t v[VS][AttnCfg<D, PV16, FQ>::kVBytes];
     // [Q tile][key tile parity (FP8) or 0 (FP16)], keys in storage order
-    uint8_t p[2][AttnCfg<D, PV16>::kPBufs][AttnCfg<D, PV16>::kPBytes];
+    uint8_t p[2][AttnCfg<D, PV16, FQ>::kPBufs][AttnCfg<D, PV16, FQ>::kPBytes];
     float ds[KS][2][kTile];          // keys in storage order
     float dk[KS][kTile / kKeyRun];
     // 4-bit mode: E4M3 scale atoms of the Q tiles and of each K stage (d = 64 only)
@@ -99,6 +121,7 @@ struct __align__(1024) AttnSmem {
     uint32_t tmem_base;
     int abort_flag;
     int bh_kv;  // key/value head of this CTA's query head (read by the epilogue)
+    FqSmem<FQ, D, KS, RC> fq;
 };
 
 // A bounded wait whose outcome is the same for all 32 lanes (so that the warp
@@ -258,11 +281,222 @@ __device__ __forceinline__ uint32_t pack16x2(float lo, float hi, int out_bf16) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-template <int D, bool PV16, bool QK4>
-__device__ __forceinline__ void softmax_role(AttnSmem<D, PV16> &sm, const AttnParams &p, uint32_t tmem, int X, int t,
-                                             int n_tiles, int bh, int64_t o_base, int n_q, int n_kv,
+// ---------------------------------------------------------------------------
+// Q quantization of one Q tile inside the kernel (FQ), by the tile's 8 softmax warps
+// ("SageAttention2", arXiv 2411.10958, abstract: Q smoothed per block, then quantized
+// per group).  The caller's 16-bit tile sits in the tile's P buffers (TMA, 128-byte
+// swizzle, d / 64 boxes of [128 rows][128 B]), which PV does not use before the
+// tile's first scores exist; the codes go to the tile's Q operand.  The arithmetic
+// is the pre-pass quantizer's, so the codes, delta_Q and qbar are the same bits:
+//   qbar[c] = fp32(fp64 sum of the valid rows / rows)  (0 without Q smoothing),
+//   x = fp32(q) - qbar (0 on rows past n_q), delta = amax_group / 127 (1 if 0),
+//   code = round-half-even(x / delta).
+// Also returns the row's x . kbar (the logit shift of K smoothing, for the LSE).
+// Every thread of the 8 warps reaches both warpgroup barriers, whatever the outcome
+// of its wait, so a failed wait cannot leave the others waiting.
+// ---------------------------------------------------------------------------
+template <int D, bool PV16>
+__device__ __forceinline__ bool quantize_q_tile(AttnSmem<D, PV16, true> &sm, const AttnParams &p, int X, int t,
+                                                int n_q, int bh, int r, int par, float &dq_out, float &shift_out,
+                                                volatile int *abort_flag) {
+    constexpr int kBox = kTile * 128;   // one 64-channel box of the raw tile
+    const int j = threadIdx.x & 255, w8 = j >> 5, lane = j & 31;
+    const int bf16 = p.out_bf16;
+    const uint8_t *raw = &sm.p[X][0][0];
+    const int nvalid = min(kTile, n_q - t * kTile);
+    const bool ok = warp_wait(&sm.fq.bar_qraw, 0, abort_flag, p.status, kSiteQ);
+
+    // column sums: warp w8 owns D / 8 columns, lane = column + (D / 8) * row segment
+    {
+        constexpr int CPW = D / 8, SEG = 32 / CPW, RPS = kTile / SEG;
+        const int c = w8 * CPW + lane % CPW, seg = lane / CPW;
+        const uint8_t *col = raw + (c / 64) * kBox + ((c % 64) & 7) * 2;
+        const uint32_t chunk = (uint32_t)((c % 64) >> 3);
+        double s0 = 0.0, s1 = 0.0;
+        if (ok) {
+#pragma unroll 4
+            for (int i = 0; i < RPS; i += 2) {
+                const int r0 = seg * RPS + i;
+                const float x0 = h16_to_f32(*reinterpret_cast<const uint16_t *>(col + sw128_offset(r0, chunk)), bf16);
+                const float x1 = h16_to_f32(*reinterpret_cast<const uint16_t *>(col + sw128_offset(r0 + 1, chunk)), bf16);
+                s0 = __dadd_rn(s0, r0 < nvalid ? (double)x0 : 0.0);
+                s1 = __dadd_rn(s1, r0 + 1 < nvalid ? (double)x1 : 0.0);
+            }
+        }
+        double sum = __dadd_rn(s0, s1);
+#pragma unroll
+        for (int o = CPW; o < 32; o <<= 1) sum = __dadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, o));
+        if (seg == 0) {
+            const float qb = (p.use_ds && nvalid > 0) ? (float)__ddiv_rn(sum, (double)nvalid) : 0.f;
+            sm.fq.qbar[X][c] = qb;
+            // hi / lo 16-bit split for the dS product, in the mma.sync operand order
+            const float hi = bf16 ? __bfloat162float(__float2bfloat16_rn(qb)) : __half2float(__float2half_rn(qb));
+            const float lo = qb - hi;
+            const uint16_t hb = bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(hi)) : __half_as_ushort(__float2half_rn(hi));
+            const uint16_t lb = bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(lo)) : __half_as_ushort(__float2half_rn(lo));
+            const int w = c & 15, pos = (c & ~15) + ((w & 7) >> 1) * 4 + (w >= 8 ? 2 : 0) + (w & 1);
+            sm.fq.qhl[2 * X][pos] = hb;
+            sm.fq.qhl[2 * X + 1][pos] = lb;
+            if (ok) p.qbar_w[((size_t)bh * p.Tq + t) * D + c] = qb;
+        }
+    }
+    named_bar_sync(1 + X, 256);
+
+    // this thread's half row: channels [par D / 2, par D / 2 + D / 2), 8 per 16-byte chunk
+    const bool valid = r < nvalid;
+    const float *kbar = p.kbar + (size_t)sm.bh_kv * D + par * (D / 2);
+    const float *qbar = sm.fq.qbar[X] + par * (D / 2);
+    auto load8 = [&](int cc, float (&x)[8]) {   // x = Q_s of 8 channels (0 past n_q)
+        const int c0 = par * (D / 2) + 8 * cc;
+        const uint4 u = *reinterpret_cast<const uint4 *>(raw + (c0 / 64) * kBox + sw128_offset(r, (c0 % 64) >> 3));
+        const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float q = h16_to_f32((e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu), bf16);
+            x[e] = valid ? __fsub_rn(q, qbar[8 * cc + e]) : 0.f;
+        }
+    };
+    float am = 0.f, shift = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < D / 16; ++cc) {
+        float x[8];
+        load8(cc, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            am = fmaxf(am, fabsf(x[e]));
+            shift = fmaf(x[e], __ldg(kbar + 8 * cc + e), shift);
+        }
+    }
+    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 16));
+    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 8));
+    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 4));
+    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
+    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+    if (lane == 0) sm.fq.wmax[X][w8] = am;
+    named_bar_sync(1 + X, 256);
+    // group amax: 32 rows are the two warps of one lane quadrant, 128 rows all eight
+    float gam;
+    if (p.g_q == kTile) {
+        gam = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) gam = fmaxf(gam, sm.fq.wmax[X][i]);
+    } else {
+        gam = fmaxf(sm.fq.wmax[X][w8 & 3], sm.fq.wmax[X][(w8 & 3) + 4]);
+    }
+    const float dl = (gam == 0.f) ? 1.f : __fdiv_rn(gam, 127.f);
+    const float inv = 1.0f / dl;
+    // codes: 16 channels per 16-byte chunk of the operand row (d bytes, 128- / 64-byte swizzle)
+    uint8_t *qrow = sm.q[X];
+    int8_t *dump = p.q8_dump ? p.q8_dump + ((size_t)bh * p.nq_pad + (size_t)t * kTile + r) * D + par * (D / 2) : nullptr;
+#pragma unroll
+    for (int cc = 0; cc < D / 16; cc += 2) {
+        float x0[8], x1[8];
+        load8(cc, x0);
+        load8(cc + 1, x1);
+        const float a0[4] = {x0[0], x0[1], x0[2], x0[3]}, a1[4] = {x0[4], x0[5], x0[6], x0[7]};
+        const float a2[4] = {x1[0], x1[1], x1[2], x1[3]}, a3[4] = {x1[4], x1[5], x1[6], x1[7]};
+        const uint4 code = make_uint4(int8_codes<4>(a0, dl, inv), int8_codes<4>(a1, dl, inv),
+                                      int8_codes<4>(a2, dl, inv), int8_codes<4>(a3, dl, inv));
+        const uint32_t ch = (uint32_t)((par * (D / 2) + 8 * cc) >> 4);   // 16-byte chunk of the code row
+        const uint32_t off = (D == 128) ? sw128_offset((uint32_t)r, ch)
+                                        : (uint32_t)r * 64u + ((ch ^ (((uint32_t)r >> 1) & 3u)) << 4);
+        *reinterpret_cast<uint4 *>(qrow + off) = code;
+        if (dump && ok) *reinterpret_cast<uint4 *>(dump + 8 * cc) = code;
+    }
+    shift += __shfl_xor_sync(0xFFFFFFFFu, shift, 2);
+    if (ok && par == 0) p.dq_w[(size_t)bh * p.nq_pad + (size_t)t * kTile + r] = dl;
+    dq_out = dl;
+    shift_out = shift;
+    // the codes are read by the tensor core: make them visible to the async proxy
+    fence_proxy_async_smem();
+    mbar_arrive(&sm.fq.bar_qready[X]);
+    return ok;
+}
+
+// Storage position of key k of a 128-key tile: keys 32 q + 2 i + par sit at
+// par * 64 + 16 q + i (the half-row order of the scores).
+__device__ __forceinline__ int key_position(int k) { return (k & 1) * 64 + (k >> 5) * 16 + ((k & 31) >> 1); }
+
+// ---------------------------------------------------------------------------
+// dS warp (FQ): dS[t, j] = qbar_t . K[j] for both Q tiles and every key tile, on
+// mma.sync from 16-key chunks of the caller's 16-bit K (raw-K ring, its own TMA
+// loads), qbar split into hi + lo 16-bit numbers as in the pre-pass product:
+// D[key][n] = sum_c K[key][c] B[c][n], B's columns (hi_A, lo_A, hi_B, lo_B, 0...),
+// dS_x = D[.][2x] + D[.][2x + 1].  K enters unsmoothed: qbar_t . kbar is the same for
+// every key of a row, so softmax does not see it and the LSE adds back only x . kbar.
+// Results go to the dS slot of the key tile's K stage, which the stage's
+// empty barrier frees; bar_dsfull[s] tells the softmax warps they are there.
+// ---------------------------------------------------------------------------
+template <int D, bool PV16>
+__device__ __forceinline__ void ds_role(AttnSmem<D, PV16, true> &sm, const AttnParams &p, const CUtensorMap *tm_kr,
+                                        int n_tiles, bool hasB, volatile int *abort_flag) {
+    constexpr int KS = AttnCfg<D, PV16, true>::kKStages, RC = AttnCfg<D, PV16, true>::kRawChunks;
+    constexpr int CH = kTile / 16;          // chunks per key tile
+    constexpr int kChunkBytes = (D / 64) * 16 * 128;
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const bool bf16 = p.out_bf16 != 0;
+    const int total = n_tiles * CH;
+    // lane 0: chunk c into ring slot c % RC (coordinates from shared memory, written by
+    // the kernel's set-up, so that they take no registers of this 32-register warp)
+    auto issue = [&](int c) {
+        const int slot = c % RC, key = (c / CH) * kTile + (c % CH) * 16 + sm.fq.kr_coord[0];
+        const int hd = sm.fq.kr_coord[1], bt = sm.fq.kr_coord[2];
+        mbar_arrive_expect_tx(&sm.fq.bar_kr[slot], kChunkBytes);
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx) {
+            if (bt >= 0) tma_load_4d(sm.fq.kr[slot][bx], tm_kr, &sm.fq.bar_kr[slot], bx * 64, hd, key, bt);
+            else tma_load_3d(sm.fq.kr[slot][bx], tm_kr, &sm.fq.bar_kr[slot], bx * 64, key, hd);
+        }
+    };
+    if (lane == 0) {
+        prefetch_tmap(tm_kr);
+        for (int c = 0; c < RC && c < total; ++c) issue(c);
+    }
+    bool ok = warp_wait(&sm.fq.bar_qready[0], 0, abort_flag, p.status, kSiteQ);
+    if (ok && hasB) ok = warp_wait(&sm.fq.bar_qready[1], 0, abort_flag, p.status, kSiteQ);
+    // this lane's ldmatrix row: key (lane & 7) + 8 ((lane >> 3) & 1), 8-channel half lane >> 4
+    const uint32_t lr = (uint32_t)((lane & 7) + 8 * ((lane >> 3) & 1));
+    const uint32_t a_lane = smem_u32(sm.fq.kr[0][0]) + lr * 128u, a_x = lr & 7u, a_h = (uint32_t)(lane >> 4);
+    const uint32_t b_lane = smem_u32(sm.fq.qhl[g < 4 ? g : 0]) + 8u * (uint32_t)q;
+    int c = 0;   // chunks consumed
+    for (; ok && c < total; ++c) {
+        const int it = c / CH, ch = c % CH, s = it % KS, slot = c % RC;
+        if (ch == 0 && it >= KS &&   // the dS slot of this key tile's K stage is free
+            !warp_wait(&sm.bar_kempty[s], ((it / KS) & 1) ^ 1, abort_flag, p.status, kSiteEmpty)) {
+            ok = false;
+            break;
+        }
+        if (!warp_wait(&sm.fq.bar_kr[slot], (c / RC) & 1, abort_flag, p.status, kSiteFull)) { ok = false; break; }
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t a_slot = a_lane + (uint32_t)slot * kChunkBytes;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t c8 = 2u * (uint32_t)ks + a_h;   // 8-channel chunk over d
+            uint32_t a0, a1, a2, a3, b0, b1;
+            ldmatrix_x4(a_slot + (c8 >> 3) * 2048u + (((c8 & 7u) ^ a_x) << 4), a0, a1, a2, a3);
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(b_lane + 32u * ks));
+            if (g >= 4) b0 = b1 = 0u;
+            mma_16816(acc, a0, a1, a2, a3, b0, b1, bf16);
+        }
+        __syncwarp();   // every lane's reads of the slot are complete: it may be refilled
+        if (lane == 0 && c + RC < total) issue(c + RC);
+        if (q < 2) {    // lane q = x holds tile x's hi / lo columns for keys g, g + 8
+            float *ds = sm.ds[s][q];
+            ds[key_position(ch * 16 + g)] = acc[0] + acc[1];
+            ds[key_position(ch * 16 + g + 8)] = acc[2] + acc[3];
+        }
+        if (ch == CH - 1) mbar_arrive(&sm.fq.bar_dsfull[s]);
+    }
+    if (!ok && lane == 0)   // let the chunk loads in flight land before the CTA exits
+        for (int k = c; k < total && k < c + RC; ++k) mbar_wait_quiet(&sm.fq.bar_kr[k % RC], (k / RC) & 1, kDrainNs);
+    __syncwarp();
+}
+
+template <int D, bool PV16, bool QK4, bool FQ>
+__device__ __forceinline__ void softmax_role(AttnSmem<D, PV16, FQ> &sm, const AttnParams &p, uint32_t tmem, int X, int t,
+                                             int n_tiles, int bh, int64_t o_base, int n_q, int n_kv, bool q_loaded,
                                              volatile int *abort_flag) {
-    constexpr int KS = AttnCfg<D, PV16>::kKStages;
+    constexpr int KS = AttnCfg<D, PV16, FQ>::kKStages;
     const int w8 = (threadIdx.x >> 5) & 7;  // warp within the tile's eight
     const int quad = w8 & 3, half = w8 >> 2;
     const int lane = threadIdx.x & 31;
@@ -277,6 +511,14 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D, PV16> &sm, const AttnPa
     // this thread writes output columns [par * D / 2, par * D / 2 + D / 2) of its row
     uint16_t *orow = static_cast<uint16_t *>(p.o) + o_base + (int64_t)row * p.so_n + par * (D / 2);
 
+    // FQ: this warpgroup quantizes its own Q tile first (when the CTA loaded Q at all)
+    float dq_fq = 1.f, shift_fq = 0.f;
+    bool q_ok = true;
+    if constexpr (FQ) {
+        if (q_loaded) q_ok = quantize_q_tile<D, PV16>(sm, p, X, t, n_q, bh, r, par, dq_fq, shift_fq, abort_flag);
+    }
+    const bool wait_ds = FQ && p.use_ds;
+
     if (n_tiles == 0) {  // this tile's rows see no key: O = 0, LSE = -inf
         if (row < n_q) {
             uint4 *dst = reinterpret_cast<uint4 *>(orow);
@@ -287,15 +529,18 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D, PV16> &sm, const AttnPa
         return;
     }
 
-    const float dq = p.dq[(size_t)bh * p.nq_pad + row];
+    const float dq = FQ ? dq_fq : p.dq[(size_t)bh * p.nq_pad + row];
     const float c = p.scale_log2;
     const float2 c2 = make_float2(c, c);
     float m, l = 0.f, alpha = 1.f, bias;
     uint32_t sv[4][16];  // 32-key chunks of the tile, 16 of this thread's keys each
 
     // prologue: scores of key tile 0
-    bool ok = warp_wait(&sm.bar_s[X], 0, abort_flag, p.status, kSiteS) &&
+    bool ok = q_ok && warp_wait(&sm.bar_s[X], 0, abort_flag, p.status, kSiteS) &&
               warp_wait(&sm.bar_kfull[0], 0, abort_flag, p.status, kSiteFull);
+    if constexpr (FQ) {
+        if (ok && wait_ds) ok = warp_wait(&sm.fq.bar_dsfull[0], 0, abort_flag, p.status, kSiteFull);
+    }
     if (ok) {
         tc_fence_after();
         float mx[4];
@@ -321,6 +566,12 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D, PV16> &sm, const AttnPa
         if (has_next) {
             if (!warp_wait(&sm.bar_s[X], (it + 1) & 1, abort_flag, p.status, kSiteS)) { ok = false; break; }
             if (!warp_wait(&sm.bar_kfull[sn], ((it + 1) / KS) & 1, abort_flag, p.status, kSiteFull)) { ok = false; break; }
+            if constexpr (FQ) {
+                if (wait_ds && !warp_wait(&sm.fq.bar_dsfull[sn], ((it + 1) / KS) & 1, abort_flag, p.status, kSiteFull)) {
+                    ok = false;
+                    break;
+                }
+            }
             tc_fence_after();
         }
         // exponentials of tile it, interleaved with the scores of tile it + 1 (on the
@@ -413,7 +664,8 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D, PV16> &sm, const AttnPa
             // ln 2 (c (m + Q_s . kbar) + log2(l / Pr)), the Q_s . kbar term undoing the
             // shift that K smoothing applied to the whole row
             const size_t ri = (size_t)bh * p.nq_pad + row;
-            p.lse[ri] = (l_row > 0.f) ? 0.6931471805599453f * (c * (m + p.qs_kbar[ri]) + log2f(l_row) - p.log2_pr)
+            const float shift = FQ ? shift_fq : p.qs_kbar[ri];
+            p.lse[ri] = (l_row > 0.f) ? 0.6931471805599453f * (c * (m + shift) + log2f(l_row) - p.log2_pr)
                                       : -INFINITY;
         }
         const float *dv = p.dv + (size_t)sm.bh_kv * D;
@@ -449,17 +701,22 @@ __device__ __forceinline__ void softmax_role(AttnSmem<D, PV16> &sm, const AttnPa
 // the dense lengths); without RT the kernel serves dense batches only and reads the
 // lengths straight from the parameters.  The two compile to different register
 // allocations: d = 128 dense runs faster without RT, d = 64 dense with it (measured).
-template <int D, bool RT, bool PV16, bool QK4>
+// FQ: Q quantized in the kernel from the caller's 16-bit Q (tm_q), dS formed in the
+// kernel from the caller's 16-bit K (tm_kr) by warp 19; without FQ tm_kr is unused.
+template <int D, bool RT, bool PV16, bool QK4, bool FQ>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
-    constexpr int KS = AttnCfg<D, PV16>::kKStages, VS = AttnCfg<D, PV16>::kVStages;
-    constexpr int kPBufs = AttnCfg<D, PV16>::kPBufs, kPBytes = AttnCfg<D, PV16>::kPBytes;
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kr,
+                    const __grid_constant__ AttnParams p) {
+    constexpr int KS = AttnCfg<D, PV16, FQ>::kKStages, VS = AttnCfg<D, PV16, FQ>::kVStages;
+    constexpr int kPBufs = AttnCfg<D, PV16, FQ>::kPBufs, kPBytes = AttnCfg<D, PV16, FQ>::kPBytes;
     static_assert(!QK4 || (D == 64 && !PV16), "the 4-bit mode runs at d = 64 with FP8 P / V");
+    static_assert(!(QK4 && FQ), "the 4-bit mode quantizes Q in the pre-pass");
+    static_assert(!FQ || (size_t)kPBufs * kPBytes >= (size_t)kTile * D * 2, "a raw 16-bit Q tile fits its P buffers");
     constexpr int kQkRowBytes = QK4 ? D / 2 : D;   // bytes of one Q / K row in shared memory
     extern __shared__ uint8_t smem_raw[];
-    AttnSmem<D, PV16> &sm =
-        *reinterpret_cast<AttnSmem<D, PV16> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    AttnSmem<D, PV16, FQ> &sm =
+        *reinterpret_cast<AttnSmem<D, PV16, FQ> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // Work item: a pair of Q tiles of one head.  The CTAs are ordered in blocks of
@@ -481,12 +738,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // workspace rows stay padded to the longest, p.n_q / p.n_kv)
     int n_q = p.n_q, n_kv = p.n_kv;
     int64_t o_base = (int64_t)b * p.so_b + (int64_t)h * p.so_h;
+    int q_off = 0, kv_off = 0;   // first row of the sequence in a packed batch
     if (RT && p.cu_q) {
         const SeqRange sq = seq_range(p.cu_q, b, p.n_q, p.total_q), sk = seq_range(p.cu_kv, b, p.n_kv, p.total_kv);
         n_q = sq.n;
         n_kv = sk.n;
         o_base = (int64_t)sq.off * p.so_n + (int64_t)h * p.so_h;
+        q_off = sq.off;
+        kv_off = sk.off;
     }
+    // raw-tensor coordinates (FQ): token-major maps are [batch][row][head][d] (a packed
+    // batch is one batch), head-major maps [head][row][d]
+    const bool tok = p.nhd || (RT && p.cu_q);
+    const int b_coord = (RT && p.cu_q) ? 0 : b;
     const int Tq = (n_q + kTile - 1) / kTile, Tk = (n_kv + kTile - 1) / kTile;
     if (tA >= Tq) return;  // a pair past the end of a shorter packed sequence (the whole CTA)
     const int off = n_kv - n_q;
@@ -506,9 +770,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(&sm.bar_o[x], 1);
         }
         mbar_init(&sm.bar_drain, 1);
+        if constexpr (FQ) {
+            mbar_init(&sm.fq.bar_qraw, 1);
+            mbar_init(&sm.fq.bar_qready[0], 256);
+            mbar_init(&sm.fq.bar_qready[1], 256);
+            for (int i = 0; i < AttnCfg<D, PV16, FQ>::kRawChunks; ++i) mbar_init(&sm.fq.bar_kr[i], 1);
+            for (int i = 0; i < KS; ++i) mbar_init(&sm.fq.bar_dsfull[i], 32);
+            sm.fq.kr_coord[0] = kv_off;
+            sm.fq.kr_coord[1] = tok ? h / p.group : bh_kv;
+            sm.fq.kr_coord[2] = tok ? b_coord : -1;
+        }
         sm.abort_flag = 0;
         sm.bh_kv = bh_kv;
         fence_mbar_init();
+    }
+    if constexpr (FQ) {   // qbar digits of a missing tile B stay zero
+        uint32_t *z = reinterpret_cast<uint32_t *>(&sm.fq.qhl[0][0]);
+        for (int i = threadIdx.x; i < 4 * D / 2; i += kAttnThreads) z[i] = 0u;
     }
     if (!p.use_ds) {  // without Q smoothing the dS rows stay zero
         float *z = &sm.ds[0][0][0];
@@ -530,9 +808,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // ---------------- TMA producer: Q tiles, then the K / dS / delta_K ring ----------------
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
-            mbar_arrive_expect_tx(&sm.bar_q, (hasB ? 2 : 1) * (kTile * kQkRowBytes + (QK4 ? 512 : 0)));
-            tma_load_2d(sm.q[0], &tm_q, &sm.bar_q, 0, bh * p.nq_pad + tA * kTile);
-            if (hasB) tma_load_2d(sm.q[1], &tm_q, &sm.bar_q, 0, bh * p.nq_pad + tB * kTile);
+            if constexpr (FQ) {   // the caller's 16-bit Q tiles into the tiles' P buffers
+                mbar_arrive_expect_tx(&sm.fq.bar_qraw, (hasB ? 2 : 1) * kTile * D * 2);
+                for (int x = 0; x < (hasB ? 2 : 1); ++x) {
+                    const int row = (x ? tB : tA) * kTile + q_off;
+#pragma unroll
+                    for (int bx = 0; bx < D / 64; ++bx) {
+                        uint8_t *dst = &sm.p[x][0][0] + bx * (kTile * 128);
+                        if (tok) tma_load_4d(dst, &tm_q, &sm.fq.bar_qraw, bx * 64, h, row, b_coord);
+                        else tma_load_3d(dst, &tm_q, &sm.fq.bar_qraw, bx * 64, row, bh);
+                    }
+                }
+            } else {
+                mbar_arrive_expect_tx(&sm.bar_q, (hasB ? 2 : 1) * (kTile * kQkRowBytes + (QK4 ? 512 : 0)));
+                tma_load_2d(sm.q[0], &tm_q, &sm.bar_q, 0, bh * p.nq_pad + tA * kTile);
+                if (hasB) tma_load_2d(sm.q[1], &tm_q, &sm.bar_q, 0, bh * p.nq_pad + tB * kTile);
+            }
             if constexpr (QK4) {
                 bulk_load(sm.sfq[0], p.sfq + ((size_t)bh * p.Tq + tA) * 512, 512, &sm.bar_q);
                 if (hasB) bulk_load(sm.sfq[1], p.sfq + ((size_t)bh * p.Tq + tB) * 512, 512, &sm.bar_q);
@@ -547,7 +838,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     break;
                 issued = it + 1;
                 if (p.fault_inject && it == 0) continue;  // diagnostic: leave slot 0 unsignalled
-                const bool dsA = p.use_ds && it < nA, dsB = p.use_ds && it < nB;
+                const bool dsA = !FQ && p.use_ds && it < nA, dsB = !FQ && p.use_ds && it < nB;
                 const uint32_t bytes = kTile * kQkRowBytes + (dsA ? kTile * 4 : 0) + (dsB ? kTile * 4 : 0) +
                                        (kTile / kKeyRun) * 4 + (QK4 ? 512 : 0);
                 mbar_arrive_expect_tx(&sm.bar_kfull[s], bytes);
@@ -558,7 +849,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 bulk_load(sm.dk[s], dk_row + it * (kTile / kKeyRun), (kTile / kKeyRun) * 4, &sm.bar_kfull[s]);
             }
             if (*abort_flag) {  // let the copies in flight land before the CTA exits
-                mbar_wait_quiet(&sm.bar_q, 0, kDrainNs);
+                if constexpr (FQ) mbar_wait_quiet(&sm.fq.bar_qraw, 0, kDrainNs);
+                else mbar_wait_quiet(&sm.bar_q, 0, kDrainNs);
                 for (int it = max(0, issued - KS); it < issued; ++it) {
                     if (p.fault_inject && it == 0) continue;
                     mbar_wait_quiet(&sm.bar_kfull[it % KS], (it / KS) & 1, kDrainNs);
@@ -603,7 +895,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             auto sf_k = [&](int ks) {
                 if constexpr (QK4) tmem_cp_sf_atom(tmem + kTmemSfK + 4u * ks, sf_atom_desc(smem_u32(sm.sfk[ks])));
             };
-            bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, p.status, kSiteQ);
+            bool ok = FQ || mbar_wait(&sm.bar_q, 0, abort_flag, p.status, kSiteQ);
             if (ok) ok = mbar_wait(&sm.bar_kfull[0], 0, abort_flag, p.status, kSiteFull);
             if (ok) {
                 tc_fence_after();
@@ -612,8 +904,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         if ((x ? nB : nA) > 0) tmem_cp_sf_atom(tmem + kTmemSfQ + 4u * x, sf_atom_desc(smem_u32(sm.sfq[x])));
                 }
                 sf_k(0);
-                for (int x = 0; x < 2; ++x)
+                for (int x = 0; ok && x < 2; ++x)
                     if ((x ? nB : nA) > 0) {
+                        if constexpr (FQ) {   // the warpgroup has written this tile's codes
+                            ok = mbar_wait(&sm.fq.bar_qready[x], 0, abort_flag, p.status, kSiteQ);
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
                         qk(x, 0);
                         mma_commit(&sm.bar_s[x]);
                     }
@@ -676,6 +973,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             mma_commit(&sm.bar_drain);
             mbar_wait_quiet(&sm.bar_drain, 0, kDrainNs);
+        } else if (FQ && warp == kWarpDs && n_tiles > 0 && p.use_ds) {
+            // ------------------------------ dS warp ------------------------------
+            if constexpr (FQ)
+                ds_role<D, PV16>(sm, p, &tm_kr, n_tiles, hasB, abort_flag);
         }
         // all roles meet here before tensor memory is released
         tc_fence_before();
@@ -691,47 +992,61 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // one copy of the softmax code serves both tiles (instruction-cache footprint)
     const int X = warp >> 3;
     if (X == 0 || hasB)
-        softmax_role<D, PV16, QK4>(sm, p, tmem, X, X ? tB : tA, X ? nB : nA, bh, o_base, n_q, n_kv, abort_flag);
+        softmax_role<D, PV16, QK4, FQ>(sm, p, tmem, X, X ? tB : tA, X ? nB : nA, bh, o_base, n_q, n_kv, n_tiles > 0,
+                                       abort_flag);
     tc_fence_before();
     __syncthreads();
 }
 
-template <int D, bool RT, bool PV16, bool QK4 = false>
+template <int D, bool RT, bool PV16, bool QK4 = false, bool FQ = false>
 static cudaError_t launch_attention_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                      const AttnParams &p, cudaStream_t stream) {
-    const size_t smem = sizeof(AttnSmem<D, PV16>) + 1024;
-    static_assert(sizeof(AttnSmem<D, PV16>) + 1024 <= 227 * 1024, "shared memory of one CTA");
-    cudaError_t e =
-        cudaFuncSetAttribute(attn_fwd_kernel<D, RT, PV16, QK4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                                      const CUtensorMap &tkr, const AttnParams &p, cudaStream_t stream) {
+    const size_t smem = sizeof(AttnSmem<D, PV16, FQ>) + 1024;
+    static_assert(sizeof(AttnSmem<D, PV16, FQ>) + 1024 <= 227 * 1024, "shared memory of one CTA");
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, RT, PV16, QK4, FQ>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((p.Tq + 1) / 2) * (unsigned)p.BH;
     // Heads per block of the CTA order: as many key/value heads as fit kKvL2Budget
-    // bytes of K codes + V^T codes, times the query heads that share each.
+    // bytes of K codes + V^T codes (+ the caller's 16-bit K that the dS warp reads),
+    // times the query heads that share each.
     AttnParams pp = p;
-    const size_t kv_head_bytes = (size_t)p.nk_pad * D * ((PV16 ? 2 : 1) + (QK4 ? 0.5 : 1.0));
+    const size_t kv_head_bytes =
+        (size_t)p.nk_pad * D * ((PV16 ? 2 : 1) + (QK4 ? 0.5 : 1.0) + ((FQ && p.use_ds) ? 2.0 : 0.0));
     const size_t kv_heads = kv_head_bytes ? kKvL2Budget / kv_head_bytes : 0;
     const size_t hb = (kv_heads < 1 ? 1 : kv_heads) * (size_t)p.group;
     pp.head_block = (int)(hb < (size_t)p.BH ? hb : (size_t)p.BH);
     if (pp.head_block < 1) pp.head_block = 1;
-    attn_fwd_kernel<D, RT, PV16, QK4><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, pp);
+    attn_fwd_kernel<D, RT, PV16, QK4, FQ><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, tkr, pp);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                             const AttnParams &p, int d, cudaStream_t stream) {
+                             const CUtensorMap &tkr, const AttnParams &p, int d, cudaStream_t stream) {
     if (p.fp4) {   // the 4-bit mode: d = 64, FP8 P / V (checked by the callers)
-        if (d != 64 || p.pv16) return cudaErrorInvalidValue;
-        return launch_attention_d<64, true, false, true>(tq, tk, tv, p, stream);
+        if (d != 64 || p.pv16 || p.fused_q) return cudaErrorInvalidValue;
+        return launch_attention_d<64, true, false, true>(tq, tk, tv, tkr, p, stream);
+    }
+    if (p.fused_q) {   // Q quantized in the kernel
+        if (p.pv16) {
+            if (d == 128) return launch_attention_d<128, true, true, false, true>(tq, tk, tv, tkr, p, stream);
+            return launch_attention_d<64, true, true, false, true>(tq, tk, tv, tkr, p, stream);
+        }
+        if (d == 128) {
+            if (p.cu_q) return launch_attention_d<128, true, false, false, true>(tq, tk, tv, tkr, p, stream);
+            return launch_attention_d<128, false, false, false, true>(tq, tk, tv, tkr, p, stream);
+        }
+        return launch_attention_d<64, true, false, false, true>(tq, tk, tv, tkr, p, stream);
     }
     if (p.pv16) {
-        if (d == 128) return launch_attention_d<128, true, true>(tq, tk, tv, p, stream);
-        return launch_attention_d<64, true, true>(tq, tk, tv, p, stream);
+        if (d == 128) return launch_attention_d<128, true, true>(tq, tk, tv, tkr, p, stream);
+        return launch_attention_d<64, true, true>(tq, tk, tv, tkr, p, stream);
     }
     if (d == 128) {
-        if (p.cu_q) return launch_attention_d<128, true, false>(tq, tk, tv, p, stream);
-        return launch_attention_d<128, false, false>(tq, tk, tv, p, stream);
+        if (p.cu_q) return launch_attention_d<128, true, false>(tq, tk, tv, tkr, p, stream);
+        return launch_attention_d<128, false, false>(tq, tk, tv, tkr, p, stream);
     }
-    return launch_attention_d<64, true, false>(tq, tk, tv, p, stream);
+    return launch_attention_d<64, true, false>(tq, tk, tv, tkr, p, stream);
 }
 
 }  // namespace sage

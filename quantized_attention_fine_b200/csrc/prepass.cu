@@ -30,10 +30,6 @@ namespace sage {
 
 namespace {
 
-__device__ __forceinline__ float h16_to_f32(uint32_t bits, int bf16) {
-    return bf16 ? __uint_as_float(bits << 16) : __half2float(__ushort_as_half((unsigned short)bits));
-}
-
 template <int VEC>
 __device__ __forceinline__ void load_row_slice(const uint16_t *p, int bf16, float (&x)[VEC]) {
     if constexpr (VEC == 4) {
@@ -71,38 +67,6 @@ __device__ __forceinline__ float warp_sum16_scatter(float (&v)[16]) {
         }
     }
     return v[0] + __shfl_xor_sync(0xFFFFFFFFu, v[0], 1);
-}
-
-// INT8 codes of VEC values, round-half-even of the IEEE fp32 quotient xs / delta,
-// packed little-endian.
-// - For |xs / delta| <= 128, t = RN(xs * RN(1 / delta)) lies within 2.3e-5 of the
-//   correctly rounded quotient, so when t is at least 2^-15 (3.05e-5) away from a
-//   half-integer both round to the same integer; only the rare near-tie takes the
-//   IEEE division.
-// - Rounding is done on the FMA pipe: m = RN(t + 1.5 * 2^23) holds round-half-even(t)
-//   in its low mantissa bits, so its low byte is the two's-complement code, and
-//   m - 1.5 * 2^23 is that integer exactly.
-// - delta = amax / 127 bounds |t| by 127 (1 + 3 * 2^-24) < 127.5, so the codes never
-//   leave [-127, 127] and the clamp of the definition never binds.
-template <int VEC>
-__device__ __forceinline__ uint32_t int8_codes(const float (&xs)[VEC], float delta, float inv_delta) {
-    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-    uint32_t m[4] = {0, 0, 0, 0};
-    bool near_tie = false;
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) {
-        const float t = xs[v] * inv_delta;
-        const float tm = t + kMagic;
-        near_tie |= fabsf(t - (tm - kMagic)) > 0.5f - 0x1p-15f;
-        m[v] = __float_as_uint(tm);
-    }
-    if (near_tie) {
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) m[v] = __float_as_uint(__fdiv_rn(xs[v], delta) + kMagic);
-    }
-    const uint32_t lo = __byte_perm(m[0], m[1], 0x0040);
-    if constexpr (VEC == 4) return __byte_perm(lo, __byte_perm(m[2], m[3], 0x0040), 0x5410);
-    return lo & 0xFFFFu;
 }
 
 // The IEEE fp32 quotient x / delta as far as its E4M3 rounding is concerned.

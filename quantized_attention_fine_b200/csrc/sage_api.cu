@@ -5,6 +5,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/sage.h"
@@ -16,6 +17,9 @@ namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
+// sage_debug_set_q_code_dump: forward calls that quantize Q in the attention kernel
+// also write the Q codes to the workspace.
+std::atomic<int> g_q_code_dump{0};
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     std::call_once(g_encode_once, [] {
@@ -136,10 +140,12 @@ bool make_maps(const Shape &s, const uint8_t *ws, CUtensorMap *tq, CUtensorMap *
     return true;
 }
 
-// Tensor map of the caller's 16-bit K for the dS product: [BH][n_kv][d] (head-major)
-// or [B][n_kv][H][d] (token-major), 64-element x 128-key boxes, 128-byte swizzle.
-// Keys past n_kv read as zero.
-bool make_k16_map(CUtensorMap *map, const void *k, int dtype, int layout, const Shape &s) {
+// Tensor map of a caller's 16-bit Q or K (`heads` heads of `n` rows per sequence, or
+// a packed batch of s.total_* rows): [BH][n][d] (head-major) or [B][n][heads][d]
+// (token-major; a packed batch is one batch), 64-element x `box_rows` boxes, 128-byte
+// swizzle.  Rows past the end read as zero.
+bool make_raw16_map(CUtensorMap *map, const void *x, int dtype, int layout, const Shape &s, int n, int total,
+                    int heads, uint32_t box_rows) {
     auto enc = get_encode();
     if (!enc) return false;
     const CUtensorMapDataType dt =
@@ -147,24 +153,28 @@ bool make_k16_map(CUtensorMap *map, const void *k, int dtype, int layout, const 
     const uint64_t d = (uint64_t)s.d;
     CUresult r;
     if (layout == SAGE_LAYOUT_HND && !s.varlen) {
-        cuuint64_t dims[3] = {d, (uint64_t)s.n_kv, (uint64_t)s.BH_kv};
-        cuuint64_t strides[2] = {d * 2, (uint64_t)s.n_kv * d * 2};
-        cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+        cuuint64_t dims[3] = {d, (uint64_t)n, (uint64_t)s.B * heads};
+        cuuint64_t strides[2] = {d * 2, (uint64_t)n * d * 2};
+        cuuint32_t box[3] = {64, box_rows, 1};
         cuuint32_t estr[3] = {1, 1, 1};
-        r = enc(map, dt, 3, const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+        r = enc(map, dt, 3, const_cast<void *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     } else {
-        // token-major; a packed batch is one "batch" of total_kv tokens
-        const uint64_t n = s.varlen ? (uint64_t)s.total_kv : (uint64_t)s.n_kv;
+        const uint64_t rows = s.varlen ? (uint64_t)total : (uint64_t)n;
         const uint64_t nb = s.varlen ? 1 : (uint64_t)s.B;
-        cuuint64_t dims[4] = {d, (uint64_t)s.H_kv, n, nb};
-        cuuint64_t strides[3] = {d * 2, (uint64_t)s.H_kv * d * 2, n * s.H_kv * d * 2};
-        cuuint32_t box[4] = {64, 1, (cuuint32_t)kTile, 1};
+        cuuint64_t dims[4] = {d, (uint64_t)heads, rows, nb};
+        cuuint64_t strides[3] = {d * 2, (uint64_t)heads * d * 2, rows * heads * d * 2};
+        cuuint32_t box[4] = {64, 1, box_rows, 1};
         cuuint32_t estr[4] = {1, 1, 1, 1};
-        r = enc(map, dt, 4, const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+        r = enc(map, dt, 4, const_cast<void *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     }
     return r == CUDA_SUCCESS;
+}
+
+// The caller's K for the dS product of the pre-pass: 128-key boxes.
+bool make_k16_map(CUtensorMap *map, const void *k, int dtype, int layout, const Shape &s) {
+    return make_raw16_map(map, k, dtype, layout, s, s.n_kv, s.total_kv, s.H_kv, (uint32_t)kTile);
 }
 
 // Load map of a caller's 16-bit Q, K or V (n rows per head, `batches` batches): d x
@@ -212,7 +222,7 @@ bool make_ds_map(CUtensorMap *map, float *ds, const Shape &s) {
 // [total][heads][d] tensors, per-sequence offsets cu_q, cu_kv on the device).
 sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype, int layout, const Shape &s,
                           const Mode &m, uint8_t *ws, int ds_t_skip, int causal_off, const int *cu_q,
-                          const int *cu_kv, cudaStream_t stream) {
+                          const int *cu_kv, cudaStream_t stream, bool ds_product = true) {
     PrepassArgs a;
     a.q = q;
     a.k = k;
@@ -239,7 +249,7 @@ sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype
     a.ws = ws;
     a.L = ws_layout(s);
     if (launch_prepass(a, stream) != cudaSuccess) return SAGE_ERR_CUDA;
-    if (k && m.smooth_q) {
+    if (k && m.smooth_q && ds_product) {
         CUtensorMap tmk, tmds;
         if (!make_k16_map(&tmk, k, dtype, layout, s)) return SAGE_ERR_CUDA;
         if (!make_ds_map(&tmds, reinterpret_cast<float *>(ws + a.L.ds), s)) return SAGE_ERR_CUDA;
@@ -251,11 +261,20 @@ sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype
     return SAGE_OK;
 }
 
+// q_raw, k_raw (both or neither): the caller's 16-bit Q and K; the kernel then
+// quantizes Q itself and forms dS from K (the workspace needs only the K / V pre-pass).
 sage_status_t run_attention(void *o, int dtype, int layout, const Shape &s, int causal, float sm_scale,
                             const Mode &m, const uint8_t *ws, int fault_inject, const int *cu_q, const int *cu_kv,
-                            cudaStream_t stream) {
-    CUtensorMap tq, tk, tv;
-    if (!make_maps(s, ws, &tq, &tk, &tv)) return SAGE_ERR_CUDA;
+                            cudaStream_t stream, const void *q_raw = nullptr, const void *k_raw = nullptr) {
+    CUtensorMap tq, tk, tv, tkr;
+    const bool fused = q_raw != nullptr && k_raw != nullptr;
+    if (!make_maps(s, ws, fused ? nullptr : &tq, &tk, &tv)) return SAGE_ERR_CUDA;
+    if (fused) {
+        if (!make_raw16_map(&tq, q_raw, dtype, layout, s, s.n_q, s.total_q, s.H, (uint32_t)kTile)) return SAGE_ERR_CUDA;
+        if (!make_raw16_map(&tkr, k_raw, dtype, layout, s, s.n_kv, s.total_kv, s.H_kv, 16u)) return SAGE_ERR_CUDA;
+    } else {
+        tkr = tq;   // not read
+    }
     const WsLayout L = ws_layout(s);
     const Strides so = make_strides(layout, s.H, s.varlen ? s.total_q : s.n_q, s.d);
     AttnParams p;
@@ -295,7 +314,14 @@ sage_status_t run_attention(void *o, int dtype, int layout, const Shape &s, int 
     p.log2_pr = m.pv16 ? 0.f : log2f(m.p_range);  // FP16 P~ is not scaled (Pr = 1)
     p.status = reinterpret_cast<int *>(const_cast<uint8_t *>(ws) + L.status);
     p.fault_inject = fault_inject;
-    return launch_attention(tq, tk, tv, p, s.d, stream) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+    p.fused_q = fused ? 1 : 0;
+    p.g_q = m.g_q;
+    p.nhd = (layout == SAGE_LAYOUT_NHD);
+    p.kbar = reinterpret_cast<const float *>(ws + L.kbar);
+    p.qbar_w = reinterpret_cast<float *>(const_cast<uint8_t *>(ws) + L.qbar);
+    p.dq_w = reinterpret_cast<float *>(const_cast<uint8_t *>(ws) + L.dq);
+    p.q8_dump = (fused && g_q_code_dump.load()) ? reinterpret_cast<int8_t *>(const_cast<uint8_t *>(ws) + L.q8) : nullptr;
+    return launch_attention(tq, tk, tv, tkr, p, s.d, stream) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
 sage_status_t check_common(int dtype, int layout) {
@@ -496,6 +522,38 @@ sage_status_t sage_attn_fwd_gqa(const void *q, const void *k, const void *v, voi
     return run_attention(o, dtype, layout, s, causal, sm_scale, m, ws, 0, nullptr, nullptr, st);
 }
 
+sage_status_t sage_attn_fwd_qfused_gqa(const void *q, const void *k, const void *v, void *o, int dtype, int layout,
+                                       int B, int H, int H_kv, int n_q, int n_kv, int d, int causal, float sm_scale,
+                                       const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes,
+                                       void *stream) {
+    int plan = kFwdNoop;
+    size_t need = 0;
+    // the whole forward's checks (without v, k stands in for it: only the attention runs)
+    SAGE_TRY(check_fwd_args(q, k, v ? v : k, o, dtype, layout, B, H, H_kv, n_q, n_kv, d, mode, &plan, &need));
+    Shape s;
+    Mode m;
+    check_sizes(B, H, H_kv, n_q, n_kv, d, &s);
+    read_mode(mode, &m);
+    if (m.fp4) return SAGE_ERR_UNSUPPORTED;   // the 4-bit mode quantizes Q in the pre-pass
+    if (plan == kFwdNoop) return SAGE_OK;
+    s.pv16 = m.pv16;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (plan == kFwdZeroOut)
+        return cudaMemsetAsync(o, 0, (size_t)s.BH * n_q * d * 2, st) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+    SAGE_TRY(check_ws(s, workspace, workspace_bytes));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    // K / V pre-pass (no Q quantization, no dS product), then attention with Q quantized
+    // and dS formed in the kernel
+    if (v) SAGE_TRY(run_prepass(nullptr, k, v, dtype, layout, s, m, ws, 0, 0, nullptr, nullptr, st, false));
+    return run_attention(o, dtype, layout, s, causal, sm_scale, m, ws, 0, nullptr, nullptr, st, q, k);
+}
+
+sage_status_t sage_debug_set_q_code_dump(int enable) {
+    if (enable != 0 && enable != 1) return SAGE_ERR_INVALID_ARG;
+    g_q_code_dump.store(enable);
+    return SAGE_OK;
+}
+
 sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *o, int dtype, int layout, int B,
                             int H, int n_q, int n_kv, int d, int causal, float sm_scale,
                             const sage_quant_mode_t *mode, void *workspace, size_t workspace_bytes, void *stream) {
@@ -507,11 +565,11 @@ size_t sage_workspace_bytes_varlen(int B, int H, int H_kv, int max_seqlen_q, int
     return sage_workspace_bytes_gqa(B, H, H_kv, max_seqlen_q, max_seqlen_kv, d);
 }
 
-sage_status_t sage_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, int dtype,
-                                   const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_kv, int B, int H, int H_kv,
-                                   int total_q, int total_kv, int max_seqlen_q, int max_seqlen_kv, int d, int causal,
-                                   float sm_scale, const sage_quant_mode_t *mode, void *workspace,
-                                   size_t workspace_bytes, void *stream) {
+static sage_status_t attn_fwd_varlen_impl(const void *q, const void *k, const void *v, void *o, int dtype,
+                                          const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_kv, int B, int H,
+                                          int H_kv, int total_q, int total_kv, int max_seqlen_q, int max_seqlen_kv,
+                                          int d, int causal, float sm_scale, const sage_quant_mode_t *mode,
+                                          void *workspace, size_t workspace_bytes, void *stream, bool fuse_q) {
     Shape s;
     Mode m;
     SAGE_TRY(check_common(dtype, SAGE_LAYOUT_NHD));
@@ -534,9 +592,38 @@ sage_status_t sage_attn_fwd_varlen(const void *q, const void *k, const void *v, 
     if (!aligned16(k) || !aligned16(v)) return SAGE_ERR_UNSUPPORTED;
     SAGE_TRY(check_ws(s, workspace, workspace_bytes));
     uint8_t *ws = static_cast<uint8_t *>(workspace);
+    if (fuse_q && !m.fp4) {   // K / V pre-pass, then attention with Q quantized in the kernel
+        SAGE_TRY(run_prepass(nullptr, k, v, dtype, SAGE_LAYOUT_NHD, s, m, ws, 0, 0, cu_seqlens_q, cu_seqlens_kv, st,
+                             false));
+        return run_attention(o, dtype, SAGE_LAYOUT_NHD, s, causal, sm_scale, m, ws, 0, cu_seqlens_q, cu_seqlens_kv, st,
+                             q, k);
+    }
     SAGE_TRY(run_prepass(q, k, v, dtype, SAGE_LAYOUT_NHD, s, m, ws, causal ? 1 : 0, 0, cu_seqlens_q, cu_seqlens_kv,
                          st));
     return run_attention(o, dtype, SAGE_LAYOUT_NHD, s, causal, sm_scale, m, ws, 0, cu_seqlens_q, cu_seqlens_kv, st);
+}
+
+sage_status_t sage_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, int dtype,
+                                   const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_kv, int B, int H, int H_kv,
+                                   int total_q, int total_kv, int max_seqlen_q, int max_seqlen_kv, int d, int causal,
+                                   float sm_scale, const sage_quant_mode_t *mode, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    return attn_fwd_varlen_impl(q, k, v, o, dtype, cu_seqlens_q, cu_seqlens_kv, B, H, H_kv, total_q, total_kv,
+                                max_seqlen_q, max_seqlen_kv, d, causal, sm_scale, mode, workspace, workspace_bytes,
+                                stream, false);
+}
+
+sage_status_t sage_attn_fwd_varlen_qfused(const void *q, const void *k, const void *v, void *o, int dtype,
+                                          const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_kv, int B, int H,
+                                          int H_kv, int total_q, int total_kv, int max_seqlen_q, int max_seqlen_kv,
+                                          int d, int causal, float sm_scale, const sage_quant_mode_t *mode,
+                                          void *workspace, size_t workspace_bytes, void *stream) {
+    sage_quant_mode_t md = {SAGE_QK_PER_THREADGROUP, 1, 1, 448.f, 448.f, 0};
+    if (mode) md = *mode;
+    if (md.gran == SAGE_QK_FP4) return SAGE_ERR_UNSUPPORTED;   // the 4-bit mode quantizes Q in the pre-pass
+    return attn_fwd_varlen_impl(q, k, v, o, dtype, cu_seqlens_q, cu_seqlens_kv, B, H, H_kv, total_q, total_kv,
+                                max_seqlen_q, max_seqlen_kv, d, causal, sm_scale, mode, workspace, workspace_bytes,
+                                stream, true);
 }
 
 sage_status_t sage_get_device_status(void *workspace, void *stream, int *code, int *site) {

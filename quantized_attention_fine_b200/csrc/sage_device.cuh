@@ -1,6 +1,7 @@
 // sage_device.cuh -- sm_100a device building blocks written as inline PTX:
 // mbarriers with bounded waits, TMA (tensor and bulk) loads, tensor-memory
-// allocation / load / store, tcgen05.mma issue, shared-memory matrix descriptors.
+// allocation / load / store, tcgen05.mma issue, shared-memory matrix descriptors,
+// and the INT8 quantizer shared by the pre-pass and the attention prologue.
 #pragma once
 
 #include <cuda.h>
@@ -386,6 +387,75 @@ __device__ __forceinline__ uint32_t e2m1x2(float hi, float lo) {
     uint32_t r;
     asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\tcvt.u32.u8 %0, b;\n\t}" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// One 16-bit element (bf16 when `bf16`, else fp16) as fp32, exactly.
+__device__ __forceinline__ float h16_to_f32(uint32_t bits, int bf16) {
+    return bf16 ? __uint_as_float(bits << 16) : __half2float(__ushort_as_half((unsigned short)bits));
+}
+
+// INT8 codes of VEC values, round-half-even of the IEEE fp32 quotient xs / delta,
+// packed little-endian.
+// - For |xs / delta| <= 128, t = RN(xs * RN(1 / delta)) lies within 2.3e-5 of the
+//   correctly rounded quotient, so when t is at least 2^-15 (3.05e-5) away from a
+//   half-integer both round to the same integer; only the rare near-tie takes the
+//   IEEE division.
+// - Rounding is done on the FMA pipe: m = RN(t + 1.5 * 2^23) holds round-half-even(t)
+//   in its low mantissa bits, so its low byte is the two's-complement code, and
+//   m - 1.5 * 2^23 is that integer exactly.
+// - delta = amax / 127 bounds |t| by 127 (1 + 3 * 2^-24) < 127.5, so the codes never
+//   leave [-127, 127] and the clamp of the definition never binds.
+template <int VEC>
+__device__ __forceinline__ uint32_t int8_codes(const float (&xs)[VEC], float delta, float inv_delta) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    uint32_t m[4] = {0, 0, 0, 0};
+    bool near_tie = false;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+        const float t = xs[v] * inv_delta;
+        const float tm = t + kMagic;
+        near_tie |= fabsf(t - (tm - kMagic)) > 0.5f - 0x1p-15f;
+        m[v] = __float_as_uint(tm);
+    }
+    if (near_tie) {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) m[v] = __float_as_uint(__fdiv_rn(xs[v], delta) + kMagic);
+    }
+    const uint32_t lo = __byte_perm(m[0], m[1], 0x0040);
+    if constexpr (VEC == 4) return __byte_perm(lo, __byte_perm(m[2], m[3], 0x0040), 0x5410);
+    return lo & 0xFFFFu;
+}
+
+// ---------------------------------------------------------------------------
+// Warp-level matrix multiply (mma.sync) for small side products
+// ---------------------------------------------------------------------------
+// Four 8 x 8 matrices of 16-bit elements from shared memory: lane l gives the row
+// address of row l % 8 of matrix l / 8; register i of every lane receives its part of
+// matrix i (lane t: row t / 4, elements 2 (t % 4), 2 (t % 4) + 1).
+__device__ __forceinline__ void ldmatrix_x4(uint32_t saddr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(saddr)
+                 : "memory");
+}
+// D (16 x 8, fp32) += A (16 x 16, row-major) . B (16 x 8, column-major), 16-bit A and B
+// of the same type (bf16 when `bf16`, else fp16).  Lane t = 4 g + q holds
+// a = {A[g][2q..], A[g + 8][2q..], A[g][2q + 8..], A[g + 8][2q + 8..]},
+// b = {B[2q..][g], B[2q + 8..][g]}, d = {D[g][2q], D[g][2q + 1], D[g + 8][2q], D[g + 8][2q + 1]}.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1, bool bf16) {
+    if (bf16)
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    else
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // 128-byte swizzle of a tile with 128-byte rows: byte offset of 16-byte chunk `c`

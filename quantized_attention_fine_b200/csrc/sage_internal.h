@@ -142,6 +142,17 @@ struct AttnParams {
     float log2_pr;      // log2(Pr)
     int *status;
     int fault_inject;
+    // Q quantized inside the attention kernel (fused_q): the kernel reads the caller's
+    // 16-bit Q through its Q tensor map and 16-bit K through the raw-K map, forms
+    // qbar, delta_Q and the INT8 codes of its own Q tiles and the dS rows of every key
+    // tile; dq / ds / qs_kbar above are then unused.
+    int fused_q;
+    int g_q;                 // rows per delta_Q group (32 or 128)
+    int nhd;                 // token-major caller tensors (coordinates of the raw maps)
+    const float *kbar;       // [BH_kv][d] K channel means
+    float *qbar_w;           // [BH][Tq][d] written: qbar of every Q tile
+    float *dq_w;             // [BH][nq_pad] written: delta_Q of every row
+    int8_t *q8_dump;         // [BH][nq_pad][d] written when not null: the Q codes
 };
 
 cudaError_t launch_prepass(const PrepassArgs &a, cudaStream_t stream);
@@ -155,8 +166,11 @@ cudaError_t launch_prepass(const PrepassArgs &a, cudaStream_t stream);
 cudaError_t launch_ds_gemm(const CUtensorMap &tm_k, const CUtensorMap &tm_ds, const float *qbar, const Shape &s,
                            int nhd, int bf16, int causal_skip, int causal_off, const int *cu_q, const int *cu_kv,
                            int *status, cudaStream_t stream);
+// tq: Q codes, or with p.fused_q the caller's 16-bit Q (64-element x 128-row boxes,
+// 128-byte swizzle); tkr: with p.fused_q the caller's 16-bit K (64-element x 16-key
+// boxes, 128-byte swizzle), else unused.
 cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                             const AttnParams &p, int d, cudaStream_t stream);
+                             const CUtensorMap &tkr, const AttnParams &p, int d, cudaStream_t stream);
 cudaError_t launch_debug_qk_tile(const CUtensorMap &tq, const CUtensorMap &tk, int d, int q_row0, int k_row0,
                                  int32_t *s_out, int *status, cudaStream_t stream);
 cudaError_t launch_debug_pv(const uint8_t *p, const uint8_t *vt, int n_tiles, int d, float *o, int *status,

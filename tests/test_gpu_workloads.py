@@ -1,5 +1,8 @@
 """Parity at the full workload sizes, in the launch configuration bench.py times
-(sage_quant_qk + sage_quant_v + sage_attn_fwd_prequant on one workspace).
+(sage_quant_qk + sage_quant_v + sage_attn_fwd_prequant on one workspace), and for
+llm_prefill also through the path with Q quantized inside the attention kernel
+(sage_attn_fwd_qfused_gqa, `bench.py --fuse-q`; its Q codes read back through the
+code-dump switch).
 
 The oracle cannot redo a whole 32K-token workload, so it recomputes sampled heads
 completely (pre-pass, bit-exact) and sampled Q blocks of them over the full KV range
@@ -40,9 +43,11 @@ def _full_precision_rows(qh, kh, vh, rows, causal):
     return (p @ vh) / p.sum(1, keepdims=True)
 
 
-@pytest.mark.parametrize("name", ["image_dit", "llm_prefill", "video_dit", "llm_prefill_gqa",
-                                  "sweep_n65536_d128_causal", "sweep_n65536_d64_full"])
-def test_full_size_workload_sampled(name):
+@pytest.mark.parametrize("name,path", [("image_dit", "prequant"), ("llm_prefill", "prequant"),
+                                       ("video_dit", "prequant"), ("llm_prefill_gqa", "prequant"),
+                                       ("sweep_n65536_d128_causal", "prequant"), ("sweep_n65536_d64_full", "prequant"),
+                                       ("llm_prefill", "fuse_q")])
+def test_full_size_workload_sampled(name, path):
     """Also the longest sweep points, N = 65,536 (the sweep recipe names N up to 64K):
     the first, middle and last Q blocks of two heads over all 65,536 keys."""
     w = wl.by_name(name)
@@ -51,9 +56,17 @@ def test_full_size_workload_sampled(name):
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     mode = sage.QuantMode.make()
     ws = sage.make_workspace(w.B, w.H, w.N_q, w.N_kv, w.d, device=dev, H_kv=w.Hk)
-    sage.quant_qk(qd, kd, mode=mode, workspace=ws)
-    sage.quant_v(vd, n_q=w.N_q, mode=mode, workspace=ws)
-    o = sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode)
+    if path == "fuse_q":
+        sage.debug_set_q_code_dump(True)
+        try:
+            o = sage.attn_fwd(qd, kd, vd, causal=w.causal, workspace=ws, fuse_q=True)
+            torch.cuda.synchronize()
+        finally:
+            sage.debug_set_q_code_dump(False)
+    else:
+        sage.quant_qk(qd, kd, mode=mode, workspace=ws)
+        sage.quant_v(vd, n_q=w.N_q, mode=mode, workspace=ws)
+        o = sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode)
     assert sage.get_device_status(ws) == (0, 0)
     tq = -(-w.N_q // 128)
     heads = [(0, 0), (w.B - 1, w.H - 1)]
