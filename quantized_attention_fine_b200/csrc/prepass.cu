@@ -149,12 +149,16 @@ struct RingCtl {
     }
 };
 
+// ring_base: where the ring starts (128-byte aligned); null = the start of dynamic
+// shared memory, rounded up.
 template <int D>
 __device__ __forceinline__ RingCtl<D> ring_setup(const CUtensorMap *tm, int nhd, int H, int T, int BH, uint64_t *full,
-                                                 volatile int *abort_flag, const int *cu, int n_max, int total) {
+                                                 volatile int *abort_flag, const int *cu, int n_max, int total,
+                                                 uint8_t *ring_base = nullptr) {
     extern __shared__ uint8_t smem_raw[];
     RingCtl<D> rc;
-    rc.ring = reinterpret_cast<uint16_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    rc.ring = ring_base ? reinterpret_cast<uint16_t *>(ring_base)
+                        : reinterpret_cast<uint16_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     rc.full = full;
     rc.n_units = BH * T;
     rc.T = T;
@@ -313,9 +317,18 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
     for (;; ++k) {
         const int u = blockIdx.x + k * gridDim.x;
         if (u >= rc.n_units) break;
-        if (!rc.wait(k, &s_abort, status)) break;
         const int bh = u / S.Tq, t = u % S.Tq;
+        // kbar of this query head's key/value head (0 without K, i.e. no keys), loaded
+        // before the tile is waited for
+        float kb[VEC];
+        {
+            const int bh_kv = (bh / S.H) * S.H_kv + (bh % S.H) / (S.H / S.H_kv);
+            const float *kbar = reinterpret_cast<const float *>(a.ws + a.L.kbar) + (size_t)bh_kv * D + lane * VEC;
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) kb[v] = a.k ? kbar[v] : 0.f;
+        }
         const int r0 = t * kTile, nvalid = min(kTile, seq_range(a.cu_q, bh / S.H, S.n_q, S.total_q).n - r0);
+        if (!rc.wait(k, &s_abort, status)) break;
         if (nvalid <= 0) {  // a tile past the end of a shorter packed sequence: nothing to do
             __syncthreads();
             if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
@@ -349,15 +362,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
             reinterpret_cast<float *>(a.ws + a.L.qbar)[((size_t)bh * S.Tq + t) * D + c] = qb;
         }
         __syncthreads();
-        float qb[VEC], kb[VEC];
-        // kbar of this query head's key/value head (0 without K, i.e. no keys)
-        const int bh_kv = (bh / S.H) * S.H_kv + (bh % S.H) / (S.H / S.H_kv);
-        const float *kbar = reinterpret_cast<const float *>(a.ws + a.L.kbar) + (size_t)bh_kv * D + lane * VEC;
+        float qb[VEC];
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) {
-            qb[v] = s_qbar[lane * VEC + v];
-            kb[v] = a.k ? kbar[v] : 0.f;
-        }
+        for (int v = 0; v < VEC; ++v) qb[v] = s_qbar[lane * VEC + v];
         float am = 0.f;
         float shift[RPW];  // this lane's part of Q_s . kbar for each of the warp's rows
 #pragma unroll
@@ -414,18 +421,18 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_
     for (;; ++k) {
         const int u = blockIdx.x + k * gridDim.x;
         if (u >= rc.n_units) break;
-        if (!rc.wait(k, &s_abort, status)) break;
         const int bh = u / S.Tk, jt = u % S.Tk;
+        float kb[VEC];   // this unit's K mean, loaded before the tile is waited for
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) kb[v] = reinterpret_cast<const float *>(a.ws + a.L.kbar)[(size_t)bh * D + lane * VEC + v];
         const int j0 = jt * kTile, nvalid = min(kTile, seq_range(a.cu_kv, bh / S.H_kv, S.n_kv, S.total_kv).n - j0);
+        if (!rc.wait(k, &s_abort, status)) break;
         if (nvalid <= 0) {  // a tile past the end of a shorter packed sequence
             __syncthreads();
             if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
             continue;
         }
         const uint16_t *tile = rc.stage(k) + lane * VEC;
-        float kb[VEC];
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) kb[v] = reinterpret_cast<const float *>(a.ws + a.L.kbar)[(size_t)bh * D + lane * VEC + v];
         float x[RPW][VEC];
         float am = 0.f;
 #pragma unroll
@@ -469,24 +476,47 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_
 // first, then odd keys), the order in which the attention kernel's threads hold P.
 // Lane l holds the 16 keys of its warp for channels l*VEC ..; their 8 even and 8 odd
 // codes per channel are two 8-byte pieces of that channel's row of V^T.
+// The E4M3 V^T tile is built in shared memory ([d channels][128 positions], the
+// 128-byte swizzle TMA uses) and written with one tensor store, rather than as 8-byte
+// pieces scattered over d rows of the workspace.
+// Dynamic shared memory (the kernel has no static part, so it starts on the shared
+// window's own boundary): the V^T tile, the ring, the ring's barriers and abort flag.
+// Should the start not fall on a 1024-byte boundary (the swizzle's period), the tile
+// is written with plain stores instead (same bytes).
+template <int D>
+struct QuantVSmem {
+    static constexpr size_t kStageBytes = (size_t)D * kTile;
+    static constexpr size_t kRingBytes = (size_t)QuantRing<D>::kStages * QuantRing<D>::kTileBytes;
+    static constexpr size_t kBytes = kStageBytes + kRingBytes + 8 * QuantRing<D>::kStages + 16;
+};
+
 template <int D>
 __global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_constant__ PrepassArgs a) {
     constexpr int VEC = D / 32, RPW = kRowsPerWarp;
     static_assert(RPW == 16, "a lane stores 16 keys of a channel as one 16-byte piece");
-    __shared__ uint64_t s_full[QuantRing<D>::kStages];
-    __shared__ int s_abort;
     const Shape &S = a.shape;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *status = reinterpret_cast<int *>(a.ws + a.L.status);
-    const RingCtl<D> rc =
-        ring_setup<D>(&a.tm_v, a.nhd, S.H_kv, S.Tk, S.BH_kv, s_full, &s_abort, a.cu_kv, S.n_kv, S.total_kv);
+    extern __shared__ uint8_t smem_raw[];   // (no alignment claimed: checked below)
+    uint8_t *vts = smem_raw;
+    uint64_t *s_full = reinterpret_cast<uint64_t *>(smem_raw + QuantVSmem<D>::kStageBytes + QuantVSmem<D>::kRingBytes);
+    int *s_abort = reinterpret_cast<int *>(s_full + QuantRing<D>::kStages);
+    const RingCtl<D> rc = ring_setup<D>(&a.tm_v, a.nhd, S.H_kv, S.Tk, S.BH_kv, s_full, s_abort, a.cu_kv, S.n_kv,
+                                        S.total_kv, smem_raw + QuantVSmem<D>::kStageBytes);
+    const bool staged = !a.pv16 && (smem_u32(smem_raw) & 1023u) == 0;
+    if (threadIdx.x == 0 && staged) prefetch_tmap(&a.tm_vt);
     int k = 0;
     for (;; ++k) {
         const int u = blockIdx.x + k * gridDim.x;
         if (u >= rc.n_units) break;
-        if (!rc.wait(k, &s_abort, status)) break;
         const int bh = u / S.Tk, jt = u % S.Tk;
+        // this unit's per-channel scales, loaded before the tile is waited for
+        float dv[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v)
+            dv[v] = a.pv16 ? 1.f : reinterpret_cast<const float *>(a.ws + a.L.dv)[(size_t)bh * D + lane * VEC + v];
         const int j0 = jt * kTile, nvalid = min(kTile, seq_range(a.cu_kv, bh / S.H_kv, S.n_kv, S.total_kv).n - j0);
+        if (!rc.wait(k, s_abort, status)) break;
         if (nvalid <= 0) {  // a tile past the end of a shorter packed sequence
             __syncthreads();
             if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
@@ -503,6 +533,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_
                 for (int v = 0; v < VEC; ++v) x[i][v] = 0.f;
             }
         }
+        // the previous tile's store has read the staging tile before it is rewritten
+        if (threadIdx.x == 0 && staged) bulk_wait_group_read<0>();
         __syncthreads();  // the stage is in registers: refill it
         if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
         if (a.pv16) {
@@ -525,26 +557,43 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_
                 }
             continue;
         }
-        // keys j0 + 16w + i: even i at position 8w + i/2, odd i at 64 + 8w + i/2
+        // keys j0 + 16w + i: even i at position 8w + i/2, odd i at 64 + 8w + i/2; channel c's
+        // row of the staging tile holds the 128 positions, 16-byte chunk h at (h ^ (c & 7))
         uint8_t *vt8 = a.ws + a.L.vt8 + ((size_t)bh * D + lane * VEC) * S.nk_pad + j0 + warp * (RPW / 2);
 #pragma unroll
         for (int v = 0; v < VEC; ++v) {
-            const float dv = reinterpret_cast<const float *>(a.ws + a.L.dv)[(size_t)bh * D + lane * VEC + v];
-            const float inv = 1.0f / dv;
+            const float inv = 1.0f / dv[v];
             uint32_t w[2][2];
 #pragma unroll
             for (int par = 0; par < 2; ++par)
 #pragma unroll
                 for (int q = 0; q < 2; ++q)
-                    w[par][q] = pack_e4m3x4(e4m3_quotient(x[8 * q + par][v], dv, inv),
-                                            e4m3_quotient(x[8 * q + 2 + par][v], dv, inv),
-                                            e4m3_quotient(x[8 * q + 4 + par][v], dv, inv),
-                                            e4m3_quotient(x[8 * q + 6 + par][v], dv, inv));
-            *reinterpret_cast<uint2 *>(vt8 + (size_t)v * S.nk_pad) = make_uint2(w[0][0], w[0][1]);
-            *reinterpret_cast<uint2 *>(vt8 + (size_t)v * S.nk_pad + kTile / 2) = make_uint2(w[1][0], w[1][1]);
+                    w[par][q] = pack_e4m3x4(e4m3_quotient(x[8 * q + par][v], dv[v], inv),
+                                            e4m3_quotient(x[8 * q + 2 + par][v], dv[v], inv),
+                                            e4m3_quotient(x[8 * q + 4 + par][v], dv[v], inv),
+                                            e4m3_quotient(x[8 * q + 6 + par][v], dv[v], inv));
+            if (staged) {
+                const uint32_t c = (uint32_t)(lane * VEC + v), half8 = 8u * (uint32_t)(warp & 1);
+                *reinterpret_cast<uint2 *>(vts + sw128_offset(c, (uint32_t)(warp >> 1)) + half8) =
+                    make_uint2(w[0][0], w[0][1]);
+                *reinterpret_cast<uint2 *>(vts + sw128_offset(c, 4u + (uint32_t)(warp >> 1)) + half8) =
+                    make_uint2(w[1][0], w[1][1]);
+            } else {
+                *reinterpret_cast<uint2 *>(vt8 + (size_t)v * S.nk_pad) = make_uint2(w[0][0], w[0][1]);
+                *reinterpret_cast<uint2 *>(vt8 + (size_t)v * S.nk_pad + kTile / 2) = make_uint2(w[1][0], w[1][1]);
+            }
+        }
+        if (staged) {
+            fence_proxy_async_smem();   // the tile is read by the tensor store (async proxy)
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                tma_store_2d(&a.tm_vt, vts, j0, bh * D);
+                bulk_commit_group();
+            }
         }
     }
-    if (s_abort && threadIdx.x == 0) rc.drain(k);
+    if (threadIdx.x == 0 && staged) bulk_wait_group<0>();   // the last stores are done
+    if (*s_abort && threadIdx.x == 0) rc.drain(k);
 }
 
 // ---------------------------------------------------------------------------
@@ -569,8 +618,9 @@ static cudaError_t launch_prepass_d(const PrepassArgs &a, cudaStream_t stream) {
         quant_k_kernel<D><<<grid_of(S.BH_kv * S.Tk), kQuantThreads, smem, stream>>>(a);
     }
     if (a.v) {
-        cudaFuncSetAttribute(quant_v_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        quant_v_kernel<D><<<grid_of(S.BH_kv * S.Tk), kQuantThreads, smem, stream>>>(a);
+        const size_t smem_v = QuantVSmem<D>::kBytes;
+        cudaFuncSetAttribute(quant_v_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_v);
+        quant_v_kernel<D><<<grid_of(S.BH_kv * S.Tk), kQuantThreads, smem_v, stream>>>(a);
     }
     return cudaGetLastError();
 }

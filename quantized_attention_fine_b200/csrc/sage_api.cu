@@ -236,6 +236,7 @@ sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype
     if (q && !make_rows16_map(&a.tm_q, q, dtype, layout, s, nq_rows, s.H, batches)) return SAGE_ERR_CUDA;
     if (k && !make_rows16_map(&a.tm_k, k, dtype, layout, s, nkv_rows, s.H_kv, batches)) return SAGE_ERR_CUDA;
     if (v && !make_rows16_map(&a.tm_v, v, dtype, layout, s, nkv_rows, s.H_kv, batches)) return SAGE_ERR_CUDA;
+    if (v && !m.pv16 && !make_maps(s, ws, nullptr, nullptr, &a.tm_vt)) return SAGE_ERR_CUDA;
     a.sq = make_strides(layout, s.H, nq_rows, s.d);
     a.skv = make_strides(layout, s.H_kv, nkv_rows, s.d);
     a.shape = s;

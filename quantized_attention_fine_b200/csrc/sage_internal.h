@@ -107,6 +107,9 @@ struct PrepassArgs {
     // tensor maps of the caller's 16-bit Q, K, V ([BH][n][d] or [B][n][H][d]; d x 128-row
     // boxes, no swizzle), valid where the pointer below is not null
     CUtensorMap tm_q, tm_k, tm_v;
+    // store map of the V^T codes (the workspace's [BH_kv * d][nk_pad] bytes, 128-key x
+    // d boxes, 128-byte swizzle), valid where v is not null and V is quantized to E4M3
+    CUtensorMap tm_vt;
     const void *q, *k, *v;   // any may be null: that part is skipped
     int bf16, nhd;
     const int *cu_q, *cu_kv;  // packed batch offsets (device), or null for a dense batch
