@@ -301,7 +301,9 @@ __global__ void kv_finalize_kernel(const PrepassArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-template <int D>
+// FP4: the 4-bit mode (a separate instantiation, so that the INT8 kernel carries
+// none of its code).
+template <int D, bool FP4>
 __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_constant__ PrepassArgs a) {
     constexpr int VEC = D / 32, RPW = kRowsPerWarp;
     __shared__ uint64_t s_full[QuantRing<D>::kStages];
@@ -388,7 +390,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
         __syncthreads();
         const int gw = a.g_q / RPW;  // warps per quantization group (g_q = 32 or 128)
         const float gam = group_amax(s_wmax, (warp / gw) * gw, gw);
-        if (a.fp4) {   // 4-bit Q: the tile scale takes delta_Q's place
+        if constexpr (FP4) {   // 4-bit Q: the tile scale takes delta_Q's place
             const float g = (gam == 0.f) ? 1.f : __fdiv_rn(gam, 2688.f);
             if (lane < RPW) reinterpret_cast<float *>(a.ws + a.L.dq)[(size_t)bh * S.nq_pad + r0 + warp * RPW + lane] = g;
             fp4_rows<D>(x, g, a.ws + a.L.q8 + ((size_t)bh * S.nq_pad + r0) * (D / 2),
@@ -406,7 +408,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
 }
 
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool FP4>
 __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_constant__ PrepassArgs a) {
     constexpr int VEC = D / 32, RPW = kRowsPerWarp;
     __shared__ uint64_t s_full[QuantRing<D>::kStages];
@@ -452,7 +454,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_
         if (threadIdx.x == 0) rc.issue(k + QuantRing<D>::kStages);
         const int gw = a.g_k / RPW;  // warps per quantization group (g_k = 16 or 128)
         const float gam = group_amax(s_wmax[k & 1], (warp / gw) * gw, gw);
-        if (a.fp4) {   // 4-bit K: the tile scale takes delta_K's place in every 16-key run
+        if constexpr (FP4) {   // 4-bit K: the tile scale takes delta_K's place in every 16-key run
             const float g = (gam == 0.f) ? 1.f : __fdiv_rn(gam, 2688.f);
             if (lane == 0)
                 reinterpret_cast<float *>(a.ws + a.L.dk)[(size_t)bh * (S.nk_pad / kKeyRun) + (j0 + warp * RPW) / kKeyRun] = g;
@@ -610,12 +612,14 @@ static cudaError_t launch_prepass_d(const PrepassArgs &a, cudaStream_t stream) {
     const size_t smem = QuantRing<D>::kSmemBytes;
     auto grid_of = [&](int units) { return (unsigned)(units < 2 * sms ? units : 2 * sms); };
     if (a.q) {
-        cudaFuncSetAttribute(quant_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        quant_q_kernel<D><<<grid_of(S.BH * S.Tq), kQuantThreads, smem, stream>>>(a);
+        auto kq = a.fp4 ? quant_q_kernel<D, true> : quant_q_kernel<D, false>;
+        cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kq<<<grid_of(S.BH * S.Tq), kQuantThreads, smem, stream>>>(a);
     }
     if (a.k) {
-        cudaFuncSetAttribute(quant_k_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        quant_k_kernel<D><<<grid_of(S.BH_kv * S.Tk), kQuantThreads, smem, stream>>>(a);
+        auto kk = a.fp4 ? quant_k_kernel<D, true> : quant_k_kernel<D, false>;
+        cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kk<<<grid_of(S.BH_kv * S.Tk), kQuantThreads, smem, stream>>>(a);
     }
     if (a.v) {
         const size_t smem_v = QuantVSmem<D>::kBytes;
