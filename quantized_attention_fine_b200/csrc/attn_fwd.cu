@@ -17,7 +17,7 @@
 //               delta_K runs through one shared-memory ring
 //   warp 17     tensor-memory allocation and single-thread tcgen05.mma issue
 //   warp 18     TMA producer of the V^T ring
-//   warp 19     idle (it only completes the producer warpgroup)
+//   warp 19     idle (it completes the producer warpgroup), except in the FQ form
 // Half rows: each row of a tile is held by two threads of one warp, one with its
 // even and one with its odd keys (the tcgen05.ld 16x64b shape), so each scheduler
 // runs four softmax warps.  Keys are stored in every 128-key tile in the order
@@ -33,6 +33,10 @@
 // In the 4-bit mode (QK4, d = 64) Q and K are E2M1 codes with E4M3 scales per 16
 // channels: each QK^T is one tcgen05.mma kind::mxf4nvf4 (K = 64) whose scale atoms
 // tcgen05.cp copies into tensor-memory columns 384-407, and S arrives in fp32.
+// In the FQ form (opt-in: Q quantized in the kernel) warp 16 loads the caller's 16-bit
+// Q tiles into the tiles' P buffers, each softmax warpgroup smooths and quantizes its
+// own tile before its first scores (quantize_q_tile), and warp 19 forms the dS rows
+// of every key tile from the caller's 16-bit K (ds_role).
 // Every wait is bounded: a wait that runs out records SAGE_ERR_TIMEOUT in the
 // status block, raises a CTA-wide abort flag that makes every role leave its loop,
 // drains the copies in flight, frees tensor memory and exits.
