@@ -410,6 +410,16 @@ SAGE_API sage_status_t sage_debug_attn_fault_inject(void *o, int dtype, int layo
                                                     const void *workspace, size_t workspace_bytes,
                                                     void *stream);
 
+/* The same for the attention kernel that quantizes Q itself (sage_attn_fwd_qfused_gqa
+ * with v = NULL): q, k are the caller's 16-bit tensors and the workspace holds their K / V
+ * pre-pass.  Every role of that kernel (its Q quantization, its dS warp) leaves through
+ * its bounded waits.  Arguments otherwise as sage_debug_attn_fault_inject (no NULL
+ * workspace). */
+SAGE_API sage_status_t sage_debug_attn_fault_inject_qfused(const void *q, const void *k, void *o, int dtype,
+                                                          int layout, int B, int H, int n_q, int n_kv, int d,
+                                                          int causal, const void *workspace, size_t workspace_bytes,
+                                                          void *stream);
+
 /* Library build identification string (static storage). */
 SAGE_API const char *sage_version(void);
 

@@ -123,6 +123,7 @@ def load_library():
         lib.sage_attn_fwd_qfused_gqa.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, F, QM, P, S, P]
         lib.sage_attn_fwd_varlen_qfused.argtypes = [P, P, P, P, I, P, P] + [I] * 9 + [F, QM, P, S, P]
         lib.sage_debug_set_q_code_dump.argtypes = [I]
+        lib.sage_debug_attn_fault_inject_qfused.argtypes = [P, P, P, I, I, I, I, I, I, I, I, P, S, P]
         lib.sage_version.restype = ctypes.c_char_p
         for fn in ("sage_quant_qk", "sage_quant_v", "sage_attn_fwd_prequant", "sage_attn_fwd",
                    "sage_quant_qk_gqa", "sage_quant_v_gqa", "sage_attn_fwd_prequant_gqa", "sage_attn_fwd_gqa",
@@ -131,7 +132,7 @@ def load_library():
                    "sage_debug_pv_accumulate_f16acc", "sage_debug_mma_rate", "sage_debug_quant_fp4",
                    "sage_debug_qk_tile_fp4",
                    "sage_debug_attn_fault_inject", "sage_attn_fwd_qfused_gqa", "sage_attn_fwd_varlen_qfused",
-                   "sage_debug_set_q_code_dump"):
+                   "sage_debug_set_q_code_dump", "sage_debug_attn_fault_inject_qfused"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -596,6 +597,18 @@ def debug_qk_tile_fp4(q4, k4, sfq, sfk, stream=None):
     if code.value != SAGE_OK:
         raise SageError(code.value, "sage_debug_qk_tile_fp4 (device site %d)" % site.value)
     return out
+
+
+def debug_fault_inject_qfused(q, k, workspace: Workspace, out, *, layout="HND", causal=False, stream=None):
+    """The same for the attention kernel that quantizes Q itself (q, k: the caller's tensors)."""
+    B, H, n_q, n_kv, d = workspace.dims
+    if workspace.H_kv != H:
+        raise ValueError("debug_fault_inject_qfused takes a multi-head workspace")
+    _check(load_library().sage_debug_attn_fault_inject_qfused(_ptr(q), _ptr(k), _ptr(out), _dtype_code(out),
+                                                              _LAYOUTS[layout], B, H, n_q, n_kv, d, int(bool(causal)),
+                                                              ctypes.c_void_p(workspace.ptr), workspace.nbytes,
+                                                              _stream_handle(stream)),
+           "sage_debug_attn_fault_inject_qfused")
 
 
 def debug_fault_inject(workspace: Workspace, out, *, layout="HND", causal=False, stream=None):

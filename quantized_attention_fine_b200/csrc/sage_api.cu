@@ -709,6 +709,21 @@ sage_status_t sage_debug_qk_tile_fp4(const uint8_t *q4, const uint8_t *k4, const
                : SAGE_ERR_CUDA;
 }
 
+sage_status_t sage_debug_attn_fault_inject_qfused(const void *q, const void *k, void *o, int dtype, int layout, int B,
+                                                  int H, int n_q, int n_kv, int d, int causal, const void *workspace,
+                                                  size_t workspace_bytes, void *stream) {
+    Shape s;
+    Mode m;
+    SAGE_TRY(check_common(dtype, layout));
+    SAGE_TRY(check_sizes(B, H, H, n_q, n_kv, d, &s));
+    SAGE_TRY(read_mode(nullptr, &m));
+    if (!q || !k || !o || !workspace || s.BH == 0 || n_q == 0 || n_kv == 0) return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(o)) return SAGE_ERR_UNSUPPORTED;
+    SAGE_TRY(check_ws(s, workspace, workspace_bytes));
+    return run_attention(o, dtype, layout, s, causal, 0.f, m, static_cast<const uint8_t *>(workspace), 1, nullptr,
+                         nullptr, static_cast<cudaStream_t>(stream), q, k);
+}
+
 sage_status_t sage_debug_attn_fault_inject(void *o, int dtype, int layout, int B, int H, int n_q, int n_kv, int d,
                                            int causal, const void *workspace, size_t workspace_bytes,
                                            void *stream) {

@@ -198,3 +198,25 @@ def test_four_bit_mode_is_refused():
     q, k, v = (x.cuda() for x in _inputs(1, 1, 1, 128, 128, 64, seed=6))
     with pytest.raises(sage.SageError):
         sage.attn_fwd(q, k, v, granularity="fp4", fuse_q=True)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_bounded_waits_report_timeout_and_context_survives(d):
+    """One K slot's signal withheld: the kernel that quantizes Q itself leaves through its
+    bounded waits (Q quantization, dS warp, producers, MMA issuer), records the timeout,
+    and the context stays usable.  Eight key tiles, so that the dS warp also meets a
+    K-stage wait that never completes."""
+    q, k, v = (x.cuda() for x in _inputs(1, 1, 1, 256, 1024, d, seed=7))
+    ws = sage.quant_qk(q, k)
+    sage.quant_v(v, n_q=256, workspace=ws)
+    assert sage.get_device_status(ws) == (0, 0)
+    out = torch.zeros_like(q)
+    sage.debug_fault_inject_qfused(q, k, ws, out)
+    code, site = sage.get_device_status(ws)
+    assert code == sage.SAGE_ERR_TIMEOUT and site != 0
+    assert sage.get_device_status(ws) == (0, 0)
+    o = sage.attn_fwd_qfused(q, k, ws).cpu()
+    torch.cuda.synchronize()
+    assert sage.get_device_status(ws) == (0, 0)
+    _, oo = oracle_head(q[0, 0].cpu(), k[0, 0].cpu(), v[0, 0].cpu(), causal=False)
+    assert_close_to_oracle(to_np64(o[0, 0]), oo, "after timeout")
