@@ -341,7 +341,7 @@ int oracle_prepass(const oracle_cfg_t *cfg, const double *q, const double *k, co
     /* --- K: INT8 codes per group of g_k keys inside each 128-key tile --- */
     for (int g0 = 0; cfg->quant_qk != 2 && g0 < nk_pad; g0 += cfg->g_k) {
         float amax = 0.0f;
-        for (int j = g0; j < g0 + cfg->g_k && j < nk; ++j)
+        for (int j = g0; j < g0 + cfg->g_k - (MUT(17) ? 1 : 0) && j < nk; ++j)   /* 17: group amax misses a key */
             for (int c = 0; c < d; ++c) {
                 float a = fabsf((float)k[(size_t)j * d + c] - kbar[c]);
                 if (a > amax) amax = a;
@@ -416,7 +416,7 @@ int oracle_attn(const oracle_cfg_t *cfg, const float *qbar, const double *q_hat,
 {
     const int nq = cfg->n_q, nk = cfg->n_kv, d = cfg->d;
     const int tq = ceil_div(nq, ORACLE_TILE), tk = ceil_div(nk, ORACLE_TILE);
-    const long off = (long)nk - (long)nq;
+    const long off = MUT(15) ? 0 : (long)nk - (long)nq;   /* 15: causal aligned top-left */
     const double pr = (cfg->quant_p == 2) ? 1.0 : cfg->p_range;  /* FP16 P~ is not scaled */
     for (int b = 0; b < n_qblocks; ++b)
         if (qblocks[b] < 0 || qblocks[b] >= tq) return 1;
@@ -430,7 +430,9 @@ int oracle_attn(const oracle_cfg_t *cfg, const float *qbar, const double *q_hat,
         if (!ds) return 3;
         for (int j = 0; j < nk; ++j) {
             double s = 0.0;
-            for (int c = 0; c < d; ++c) s += (double)qbar[(size_t)t * d + c] * k_s[(size_t)j * d + c];
+            for (int c = 0; c < d; ++c)   /* 16: dS from the dequantized K instead of K_s */
+                s += (double)qbar[(size_t)t * d + c] *
+                     (MUT(16) ? k_hat[(size_t)j * d + c] * (double)dk_key[j] : k_s[(size_t)j * d + c]);
             ds[j] = MUT(8) ? -s : s;   /* 8: dS sign */
         }
         #pragma omp parallel for schedule(dynamic, 4)
@@ -456,7 +458,7 @@ int oracle_attn(const oracle_cfg_t *cfg, const float *qbar, const double *q_hat,
                 }
                 if (!any) continue; /* tile fully masked for this row: skipped */
                 double mn = m > tmax ? m : tmax;
-                double alpha = (m == -INFINITY) ? 0.0 : exp(m - mn);
+                double alpha = (m == -INFINITY) ? 0.0 : exp(MUT(14) ? mn - m : m - mn);   /* 14: inverted */
                 l *= alpha;
                 for (int c = 0; c < d; ++c) acc[c] *= alpha;
                 for (int j = j0; j < j1; ++j) {

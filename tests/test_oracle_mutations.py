@@ -27,6 +27,10 @@ MUTATIONS = {
     11: "the 1 / Pr of the output dropped",
     12: "FP4 tile scale g = amax / 6 (no E4M3 headroom for the block scales)",
     13: "an FP4 block scale that underflows E4M3 stays 0",
+    14: "the online-softmax rescale factor inverted",
+    15: "the causal mask aligned top-left when N_q != N_kv",
+    16: "dS formed from the dequantized K instead of the smoothed K",
+    17: "a K group's amax misses its last key",
 }
 
 

@@ -457,13 +457,15 @@ def test_lse_unquantized_equals_torch_logsumexp(smooth_q, smooth_k, causal, nq, 
         assert np.all(lse[:nq - nk] == -np.inf)
 
 
-@pytest.mark.parametrize("gran", ["per_block", "per_threadgroup"])
-def test_lse_quantized_within_logit_error_bound(gran):
+@pytest.mark.parametrize("gran,qbias", [("per_block", 0.0), ("per_threadgroup", 0.0), ("per_threadgroup", 20.0)])
+def test_lse_quantized_within_logit_error_bound(gran, qbias):
     """Log-sum-exp is 1-Lipschitz in the largest logit change, and the row sum uses the
     unquantized P~, so each row's LSE lies within sm_scale times its largest INT8 score
-    error bound, sum_c (dQ/2 |K_s| + dK/2 |Q_s| + dQ dK/4), of the exact value."""
+    error bound, sum_c (dQ/2 |K_s| + dK/2 |Q_s| + dQ dK/4), of the exact value.  The
+    bound holds whatever the Q channel offset, because the offset's part of the scores
+    (qbar . K_s, the dS bias) is exact: the case with a large offset pins that."""
     nq, nk, d = 300, 400, 128
-    q, k, v = _rand_head(nq, nk, d, seed=77, kbias=3.0)
+    q, k, v = _rand_head(nq, nk, d, seed=77, kbias=3.0, qbias=qbias)
     g_q, g_k = oracle.GRANULARITY[gran]
     pre = oracle.prepass_head(q, k, v, g_q=g_q, g_k=g_k)
     lse = oracle.lse_head(pre, causal=True)
