@@ -81,3 +81,53 @@ def test_random_configuration(seed):
             assert np.array_equal(np.isfinite(got), fin), what + ": LSE finite pattern"
             if fin.any():
                 assert np.max(np.abs(got[fin] - ll[fin])) <= 1e-3, what + ": LSE"
+
+
+N_VARLEN = 8
+
+
+@pytest.mark.parametrize("seed", range(N_VARLEN))
+def test_random_packed_batch(seed):
+    """Packed variable-length batches (empty sequences, one-token sequences, q shorter or
+    longer than kv), drawn like the dense cases, against the oracle's packed forward."""
+    r = np.random.default_rng(7000 + seed)
+    nb = int(r.integers(1, 5))
+    H_kv = int(r.choice([1, 2]))
+    H = H_kv * int(r.choice([1, 2, 3]))
+    d = int(r.choice([64, 128]))
+    dtype = [torch.float16, torch.bfloat16][int(r.integers(0, 2))]
+    causal = bool(r.integers(0, 2))
+    gran = ["per_threadgroup", "per_warp", "per_block"][int(r.integers(0, 3))]
+    pv = "fp16" if r.random() < 0.25 else "fp8"
+    fuse_q = bool(seed % 2)
+    lq = [int(x) for x in r.choice([0, 1, 90, 128, 200, 333], size=nb)]
+    lk = [int(x) for x in r.choice([1, 64, 128, 250, 400], size=nb)]
+    g = torch.Generator().manual_seed(8000 + seed)
+    q = torch.randn(sum(lq), H, d, generator=g) + 3.0 * torch.randn(1, H, d, generator=g)
+    k = torch.randn(sum(lk), H_kv, d, generator=g) + 3.0 * torch.randn(1, H_kv, d, generator=g)
+    v = torch.randn(sum(lk), H_kv, d, generator=g)
+    q, k, v = (x.to(dtype) for x in (q, k, v))
+    cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    o, lse = sage.attn_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(cu_q).cuda(),
+                                  torch.from_numpy(cu_k).cuda(), causal=causal, granularity=gran, pv=pv,
+                                  return_lse=True, fuse_q=fuse_q)
+    torch.cuda.synchronize()
+    o = o.cpu()
+    lse = lse.cpu().double().numpy()
+    oo, ll = oracle.sage_attention_varlen(to_np64(q), to_np64(k), to_np64(v), cu_q, cu_k, causal=causal,
+                                          return_lse=True, granularity=gran,
+                                          quant=oracle.PV_FP16 if pv == "fp16" else (1, 1, 1))
+    what = "seed %d: lq %s lk %s H %d/%d d %d causal %s %s pv %s fuse_q %s" % (seed, lq, lk, H, H_kv, d, causal,
+                                                                             gran, pv, fuse_q)
+    for b in range(nb):
+        q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
+        for h in range(H):
+            if q1 > q0:
+                assert_close_to_oracle(to_np64(o[q0:q1, h]), oo[q0:q1, h], what + " seq %d head %d" % (b, h))
+                ref = ll[q0:q1, h]
+                got = lse[b, h, :q1 - q0]
+                fin = np.isfinite(ref)
+                assert np.array_equal(np.isfinite(got), fin), what + ": LSE finite pattern"
+                if fin.any():
+                    assert np.max(np.abs(got[fin] - ref[fin])) <= 1e-3, what + ": LSE"
