@@ -213,3 +213,34 @@ def test_varlen_and_mode_argument_errors_return_synchronously(lib):
     bad = sage.QuantMode.make()
     bad.p_range = 500.0                                 # beyond the E4M3 range
     assert f(*args(mode=ctypes.byref(bad))) == 1
+
+
+def test_in_kernel_q_entry_points_check_arguments_before_any_cuda_call(lib):
+    """The entry points that quantize Q inside the attention kernel check their arguments
+    as sage_attn_fwd does, before any CUDA call (with no GPU here a CUDA call would turn
+    the result into SAGE_ERR_CUDA), and refuse the 4-bit mode, whose Q is quantized in
+    the pre-pass."""
+    P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    fn = lib.sage_attn_fwd_qfused_gqa
+    fn.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, F, ctypes.POINTER(sage.QuantMode), P, S, P]
+    fn.restype = I
+    fake = P(1 << 20)
+    assert fn(fake, fake, fake, fake, 7, 0, 1, 2, 2, 128, 128, 64, 0, 0.0, None, fake, 1 << 30, None) == 1   # dtype
+    assert fn(fake, fake, fake, fake, 1, 0, 1, 3, 2, 128, 128, 64, 0, 0.0, None, fake, 1 << 30, None) == 1   # heads
+    assert fn(None, fake, fake, fake, 1, 0, 1, 2, 2, 128, 128, 64, 0, 0.0, None, fake, 1 << 30, None) == 1   # null q
+    assert fn(fake, fake, fake, fake, 1, 0, 1, 2, 2, 128, 128, 80, 0, 0.0, None, fake, 1 << 30, None) == 2   # d
+    fp4 = sage.QuantMode.make("fp4")
+    assert fn(fake, fake, fake, fake, 1, 0, 1, 2, 2, 128, 128, 64, 0, 0.0, ctypes.byref(fp4), fake, 1 << 30,
+              None) == 2
+    # v = NULL (the attention only) passes the same checks; a workspace too small is refused
+    assert fn(fake, fake, None, fake, 1, 0, 1, 2, 2, 128, 128, 64, 0, 0.0, None, fake, 16, None) == 3
+    vfn = lib.sage_attn_fwd_varlen_qfused
+    vfn.argtypes = [P, P, P, P, I, P, P] + [I] * 9 + [F, ctypes.POINTER(sage.QuantMode), P, S, P]
+    vfn.restype = I
+    assert vfn(fake, fake, fake, fake, 1, fake, fake, 1, 2, 2, 128, 128, 128, 128, 64, 0, 0.0, ctypes.byref(fp4),
+               fake, 1 << 30, None) == 2
+    dump = lib.sage_debug_set_q_code_dump
+    dump.argtypes = [I]
+    dump.restype = I
+    assert dump(2) == 1 and dump(-1) == 1
+    assert dump(0) == 0
