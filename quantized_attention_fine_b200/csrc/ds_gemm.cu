@@ -64,12 +64,14 @@ __global__ void __launch_bounds__(kDsThreads, 1)
     ds_gemm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ds,
                    const float *__restrict__ qbar, int H, int H_kv, int Tq, int Tk, int nhd, int bf16, int causal_skip,
                    int causal_off, const int *__restrict__ cu_q, const int *__restrict__ cu_kv, int n_q_max,
-                   int n_kv_max, int total_q, int total_kv, int tiles_per_cta, int *status) {
+                   int n_kv_max, int total_q, int total_kv, int tiles_per_cta, int ctas_per_head, int *status) {
     constexpr int KA = D / 64;
     extern __shared__ uint8_t smem_raw[];
     DsSmem<D> &sm = *reinterpret_cast<DsSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.y;  // query head
+    // one-dimensional grid (head-major), so any head count fits: block = bh * ctas_per_head + x
+    const int bh = (int)(blockIdx.x / (unsigned)ctas_per_head);   // query head
+    const int bx = (int)(blockIdx.x % (unsigned)ctas_per_head);
     // key/value head read by query head bh: h_kv = h / (H / H_kv)
     const int b = bh / H, h_kv = (bh % H) / (H / H_kv), bh_kv = b * H_kv + h_kv;
     // Q blocks and key tiles of this sequence (a packed batch has its own per sequence;
@@ -78,7 +80,7 @@ __global__ void __launch_bounds__(kDsThreads, 1)
     const int Tq_s = cu_q ? (sq.n + kTile - 1) / kTile : Tq;
     const int Tk_s = cu_kv ? (sk.n + kTile - 1) / kTile : Tk;
     if (cu_q) causal_off = sk.n - sq.n;
-    const int jt0 = blockIdx.x * tiles_per_cta;
+    const int jt0 = bx * tiles_per_cta;
     const int n_kt = min(tiles_per_cta, Tk_s - jt0);
     if (n_kt <= 0 || Tq_s <= 0) return;  // past the end of a shorter packed sequence
     const bool is_bf16 = bf16 != 0;
@@ -255,21 +257,22 @@ cudaError_t launch_ds_gemm(const CUtensorMap &tm_k, const CUtensorMap &tm_ds, co
     const long long units = (long long)s.BH * s.Tk;
     int tpc = (int)((units + 2LL * sms - 1) / (2LL * sms));
     tpc = tpc < 1 ? 1 : (tpc > kDsTilesPerCta ? kDsTilesPerCta : tpc);
-    dim3 grid((s.Tk + tpc - 1) / tpc, s.BH);
+    const int ctas_per_head = (s.Tk + tpc - 1) / tpc;
+    const unsigned grid = (unsigned)((size_t)ctas_per_head * s.BH);
     if (s.d == 128) {
         const size_t smem = sizeof(DsSmem<128>) + 1024;
         cudaError_t e = cudaFuncSetAttribute(ds_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         ds_gemm_kernel<128><<<grid, kDsThreads, smem, stream>>>(tm_k, tm_ds, qbar, s.H, s.H_kv, s.Tq, s.Tk, nhd, bf16,
                                                                  causal_skip, causal_off, cu_q, cu_kv, s.n_q, s.n_kv,
-                                                                 s.total_q, s.total_kv, tpc, status);
+                                                                 s.total_q, s.total_kv, tpc, ctas_per_head, status);
     } else {
         const size_t smem = sizeof(DsSmem<64>) + 1024;
         cudaError_t e = cudaFuncSetAttribute(ds_gemm_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         ds_gemm_kernel<64><<<grid, kDsThreads, smem, stream>>>(tm_k, tm_ds, qbar, s.H, s.H_kv, s.Tq, s.Tk, nhd, bf16,
                                                                 causal_skip, causal_off, cu_q, cu_kv, s.n_q, s.n_kv,
-                                                                s.total_q, s.total_kv, tpc, status);
+                                                                s.total_q, s.total_kv, tpc, ctas_per_head, status);
     }
     return cudaGetLastError();
 }

@@ -235,7 +235,8 @@ __global__ void __launch_bounds__(256) kv_stats_kernel(const PrepassArgs a) {
     constexpr int VEC = D / 32;
     __shared__ double s_sum[8][D];
     __shared__ float s_max[8][D];
-    const int chunk = blockIdx.x, bh = blockIdx.y;
+    // one-dimensional grid (head-major), so any head count fits: block = bh * n_chunks + chunk
+    const int chunk = (int)(blockIdx.x % (unsigned)a.shape.n_chunks), bh = (int)(blockIdx.x / (unsigned)a.shape.n_chunks);
     const int b = bh / a.shape.H_kv, h = bh % a.shape.H_kv;  // key/value head
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const SeqRange sr = seq_range(a.cu_kv, b, a.shape.n_kv, a.shape.total_kv);
@@ -603,7 +604,7 @@ template <int D>
 static cudaError_t launch_prepass_d(const PrepassArgs &a, cudaStream_t stream) {
     const Shape &S = a.shape;
     if (a.k || a.v) {
-        kv_stats_kernel<D><<<dim3(S.n_chunks, S.BH_kv), 256, 0, stream>>>(a);
+        kv_stats_kernel<D><<<(unsigned)((size_t)S.n_chunks * S.BH_kv), 256, 0, stream>>>(a);
         kv_finalize_kernel<D><<<S.BH_kv, D, 0, stream>>>(a);
     }
     // persistent grids: two CTAs per SM, or one per work unit if fewer

@@ -334,3 +334,22 @@ def test_head_blocks_with_a_partial_last_block():
         oo = oracle.attn_head(pre, causal=True, qblocks=blocks)
         rows = np.concatenate([np.arange(t * 128, t * 128 + 128) for t in blocks])
         assert_close_to_oracle(to_np64(o[0, h])[rows], oo[rows], "head %d" % h)
+
+
+def test_more_heads_than_a_grid_dimension_holds():
+    """B * H above 65,535 (the limit of a grid's y dimension): every pre-pass kernel and
+    the attention kernel spread the heads along x, so the call runs; sampled heads match
+    the oracle, on both paths."""
+    B, H, n, d = 550, 128, 16, 64   # 70,400 heads of 16 tokens
+    g = torch.Generator().manual_seed(4242)
+    q = torch.randn(B, H, n, d, generator=g).bfloat16()
+    k = (torch.randn(B, H, n, d, generator=g) + 2.0 * torch.randn(B, H, 1, d, generator=g)).bfloat16()
+    v = torch.randn(B, H, n, d, generator=g).bfloat16()
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    for fuse_q in (False, True):
+        o = sage.attn_fwd(qd, kd, vd, causal=True, fuse_q=fuse_q)
+        torch.cuda.synchronize()
+        for b, h in ((0, 0), (311, 77), (B - 1, H - 1)):
+            _, oo = oracle_head(q[b, h], k[b, h], v[b, h], causal=True)
+            assert_close_to_oracle(to_np64(o[b, h].cpu()), oo, "fuse_q=%s head (%d,%d)" % (fuse_q, b, h))
+        del o
