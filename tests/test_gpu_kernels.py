@@ -353,3 +353,31 @@ def test_more_heads_than_a_grid_dimension_holds():
             _, oo = oracle_head(q[b, h], k[b, h], v[b, h], causal=True)
             assert_close_to_oracle(to_np64(o[b, h].cpu()), oo, "fuse_q=%s head (%d,%d)" % (fuse_q, b, h))
         del o
+
+
+def test_concurrent_calls_on_two_streams():
+    """Two forward calls with their own workspaces, enqueued on two streams so that they
+    overlap on the GPU, give the bits of the same calls run one after the other: the
+    library keeps no state between calls outside the workspace."""
+    _, q1, k1, v1 = _inputs("conc1", 1, 8, 2048, 2048, 128, True, recipe="llm")
+    _, q2, k2, v2 = _inputs("conc2", 2, 4, 1500, 1800, 64, False, recipe="video_dit")
+    a = [x.cuda() for x in (q1, k1, v1)]
+    b = [x.cuda() for x in (q2, k2, v2)]
+    ref1 = sage.attn_fwd(*a, causal=True).clone()
+    ref2 = sage.attn_fwd(*b, causal=False).clone()
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    ws1 = sage.make_workspace(1, 8, 2048, 2048, 128)
+    ws2 = sage.make_workspace(2, 4, 1500, 1800, 64)
+    torch.cuda.synchronize()
+    outs = []
+    for _ in range(3):
+        with torch.cuda.stream(s1):
+            o1 = sage.attn_fwd(*a, causal=True, workspace=ws1, stream=s1)
+        with torch.cuda.stream(s2):
+            o2 = sage.attn_fwd(*b, causal=False, workspace=ws2, stream=s2)
+        outs.append((o1, o2))
+    torch.cuda.synchronize()
+    for o1, o2 in outs:
+        assert torch.equal(o1, ref1) and torch.equal(o2, ref2)
+    assert sage.get_device_status(ws1) == (0, 0) and sage.get_device_status(ws2) == (0, 0)
