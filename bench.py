@@ -75,7 +75,10 @@ def parse_args():
     ap.add_argument("--no-probe", action="store_true", help="skip the tcgen05.mma rate probe (second denominator)")
     ap.add_argument("--mma-rates", action="store_true",
                     help="print the tensor-core rate of each tcgen05.mma form (diagnostic) and exit")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.fuse_q and args.qk == "fp4":
+        ap.error("--fuse-q: the 4-bit mode quantizes Q in the pre-pass (no in-kernel form)")
+    return args
 
 
 def dist_env():
@@ -363,7 +366,7 @@ def main():
     mode = sage.QuantMode.make(gran, pv=args.pv)
     stream = torch.cuda.current_stream(dev)
 
-    fuse_q = bool(args.fuse_q) and not fp4
+    fuse_q = bool(args.fuse_q)
 
     def step_eager():
         sage.attn_fwd(q, k, v, causal=w.causal, out=out, workspace=ws, pv=args.pv, granularity=gran, fuse_q=fuse_q)
