@@ -230,7 +230,8 @@ def reference_arm(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": dict(w.describe(), parallelism="oracle on host cores, rank 0 only"),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+                             "host": host_cpu()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -303,6 +304,20 @@ def measured_peaks():
         d = json.load(open(path))
         return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
     return FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def host_cpu() -> dict:
+    """The host the CPU baseline ran on: its processor model and logical core count."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu": model, "nproc": os.cpu_count()}
 
 
 def kernel_source_hash() -> str:
@@ -518,7 +533,8 @@ def main():
     if world == 1 and not args.no_cpu_baseline:
         ops_s, secs, desc, threads = oracle_sample(w, args.cpu_seconds,
                                                    quant=(2 if fp4 else 1, 2 if pv16 else 1, 2 if pv16 else 1))
-        cpu = {"value": ops_s / secs / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+        cpu = {"value": ops_s / secs / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+               "host": host_cpu()}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
