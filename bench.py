@@ -73,6 +73,9 @@ def parse_args():
                     help="N > 1: weak = N batch blocks of the workload, one per rank; strong = the workload's "
                          "heads split across the ranks")
     ap.add_argument("--no-probe", action="store_true", help="skip the tcgen05.mma rate probe (second denominator)")
+    ap.add_argument("--lib-peaks", action="store_true",
+                    help="diagnostic: library INT8 / FP8 / BF16 GEMM rates (torch._int_mm, torch._scaled_mm, "
+                         "torch.matmul; 8192^3, best of 10 and a sustained loop)")
     ap.add_argument("--mma-rates", action="store_true",
                     help="print the tensor-core rate of each tcgen05.mma form (diagnostic) and exit")
     args = ap.parse_args()
@@ -231,7 +234,8 @@ def reference_arm(args, w):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": dict(w.describe(), parallelism="oracle on host cores, rank 0 only"),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
-                             "host": host_cpu()},
+                             "host": host_cpu(), "pair_updates_per_s": ops / secs / (4.0 * w.d),
+                             "extrapolated_step_s": w.ops() / (ops / secs)},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -306,6 +310,51 @@ def measured_peaks():
     return FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
+def library_gemm_peaks(n: int = 8192, sustained_s: float = 4.0) -> dict:
+    """Dense GEMM rates of the vendor library on this GPU (context for the roofline's
+    denominator): INT8 (torch._int_mm, int32 out), FP8 E4M3 (torch._scaled_mm, bf16 out)
+    and BF16 (torch.matmul), n^3 each; the best of 10 single launches and the mean over a
+    loop of about sustained_s seconds, with the SM clock sampled during the loops."""
+    import torch
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(1)
+    a8 = torch.randint(-127, 128, (n, n), generator=g, device=dev, dtype=torch.int8)
+    b8 = torch.randint(-127, 128, (n, n), generator=g, device=dev, dtype=torch.int8)
+    af = torch.randn(n, n, generator=g, device=dev).to(torch.float8_e4m3fn)
+    bf = torch.randn(n, n, generator=g, device=dev).to(torch.float8_e4m3fn).t()   # column-major operand
+    one = torch.ones((), device=dev)
+    ab = torch.randn(n, n, generator=g, device=dev, dtype=torch.bfloat16)
+    bb = torch.randn(n, n, generator=g, device=dev, dtype=torch.bfloat16)
+    ops = {"int8": lambda: torch._int_mm(a8, b8),
+           "fp8": lambda: torch._scaled_mm(af, bf, scale_a=one, scale_b=one, out_dtype=torch.bfloat16),
+           "bf16": lambda: torch.matmul(ab, bb)}
+    work = 2.0 * n ** 3
+    clocks = ClockSampler(0, enabled=True)
+    out = {}
+    for name, fn in ops.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            best = min(best, e0.elapsed_time(e1) * 1e-3)
+        reps = max(10, int(sustained_s / best))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        mean = e0.elapsed_time(e1) * 1e-3 / reps
+        out[name] = {"burst": work / best / 1e12, "sustained": work / mean / 1e12}
+    return {"lib_gemm_peaks": out, "unit": "TOPS (int8) / TFLOP/s", "shape": "%d^3" % n, "clocks": clocks.stop()}
+
+
 def host_cpu() -> dict:
     """The host the CPU baseline ran on: its processor model and logical core count."""
     model = None
@@ -350,6 +399,9 @@ def main():
         raise SystemExit("%s (choices: %s, or sweep_n<N>_d<64|128>_<causal|full>)" % (e, ", ".join(wl.WORKLOADS)))
     if args.impl == "reference":
         return reference_arm(args, w)
+    if args.lib_peaks:
+        print(json.dumps(library_gemm_peaks()), flush=True)
+        return 0
     if args.mma_rates:
         import quantized_attention_fine_b200 as sage
         rates = {k: sage.debug_mma_rate(k) for k in sage.MMA_KINDS}
@@ -534,7 +586,8 @@ def main():
         ops_s, secs, desc, threads = oracle_sample(w, args.cpu_seconds,
                                                    quant=(2 if fp4 else 1, 2 if pv16 else 1, 2 if pv16 else 1))
         cpu = {"value": ops_s / secs / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
-               "host": host_cpu()}
+               "host": host_cpu(), "pair_updates_per_s": ops_s / secs / (4.0 * w.d),
+               "extrapolated_step_s": ops_step / (ops_s / secs)}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
