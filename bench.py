@@ -489,7 +489,8 @@ def main():
 
     total_ms = t_start.elapsed_time(t_end)
     attn_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    total_ms, attn_avg_ms = max_over_ranks([total_ms, statistics.mean(attn_ms)], device=dev)
+    total_ms, attn_avg_ms, attn_med_ms = max_over_ranks([total_ms, statistics.mean(attn_ms), statistics.median(attn_ms)],
+                                                        device=dev)
     ms_per_step = total_ms / args.steps
     pre_avg_ms = ms_per_step - attn_avg_ms
     ops_step = wr.ops()     # this rank's slice; every rank's slice has the same size
@@ -599,7 +600,8 @@ def main():
                        granularity=("fp4 (E2M1, E4M3 scale per 16 channels, fp32 scale per 128-row tile)" if fp4
                                     else "per_threadgroup (g_q=32, g_k=16)"),
                        **({"pv": "fp16 (qk_int8_pv_fp16)"} if pv16 else {"pv": "fp8", "pr": 448, "vr": 448})),
-        "attn_kernel_tops": attn_tops, "attn_kernel_ms": attn_avg_ms, "prepass_ms": pre_avg_ms,
+        "attn_kernel_tops": attn_tops, "attn_kernel_ms": attn_avg_ms, "attn_kernel_ms_median": attn_med_ms,
+        "prepass_ms": pre_avg_ms,
         "step_call": (("sage_attn_fwd_qfused_gqa (K / V pre-pass + attention with Q quantization and dS in the kernel)"
                        if fuse_q else "sage_attn_fwd (pre-pass + dS + attention)")
                       + (", replayed from a CUDA graph" if args.graph else "")
