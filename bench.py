@@ -454,9 +454,15 @@ def main():
         else:
             sage.attn_fwd_prequant(ws, dtype=q.dtype, causal=w.causal, mode=mode, out=out)
 
+    def prepass_only():   # the step's pre-pass launches alone (the Q-fused form has no separate entry)
+        sage.quant_qk(q, k, mode=mode, workspace=ws)
+        sage.quant_v(v, n_q=nq, H=H, mode=mode, workspace=ws)
+
     for _ in range(args.warmup):
         step()
         attn_only()
+        if not fuse_q:
+            prepass_only()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -485,14 +491,26 @@ def main():
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
+    # the pre-pass alone, the same way (it refills the workspace with the same codes)
+    evp = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    if not fuse_q:
+        for i in range(args.steps):
+            evp[i][0].record(stream)
+            prepass_only()
+            evp[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
     clk = clocks.stop()
 
     total_ms = t_start.elapsed_time(t_end)
     attn_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    total_ms, attn_avg_ms, attn_med_ms = max_over_ranks([total_ms, statistics.mean(attn_ms), statistics.median(attn_ms)],
-                                                        device=dev)
+    pre_ms = [evp[i][0].elapsed_time(evp[i][1]) for i in range(args.steps)] if not fuse_q else [0.0]
+    total_ms, attn_avg_ms, attn_med_ms, pre_meas_ms = max_over_ranks(
+        [total_ms, statistics.mean(attn_ms), statistics.median(attn_ms), statistics.mean(pre_ms)], device=dev)
     ms_per_step = total_ms / args.steps
-    pre_avg_ms = ms_per_step - attn_avg_ms
+    # with Q quantized in the attention kernel there is no pre-pass call of its own to time
+    pre_avg_ms = (ms_per_step - attn_avg_ms) if fuse_q else pre_meas_ms
     ops_step = wr.ops()     # this rank's slice; every rank's slice has the same size
     value = whole_job_tops(world, ops_step, ms_per_step)
     attn_tops = ops_step / (attn_avg_ms * 1e-3) / 1e12
@@ -601,11 +619,12 @@ def main():
                                     else "per_threadgroup (g_q=32, g_k=16)"),
                        **({"pv": "fp16 (qk_int8_pv_fp16)"} if pv16 else {"pv": "fp8", "pr": 448, "vr": 448})),
         "attn_kernel_tops": attn_tops, "attn_kernel_ms": attn_avg_ms, "attn_kernel_ms_median": attn_med_ms,
-        "prepass_ms": pre_avg_ms,
+        "prepass_ms": pre_avg_ms, "step_minus_attn_ms": ms_per_step - attn_avg_ms,
         "step_call": (("sage_attn_fwd_qfused_gqa (K / V pre-pass + attention with Q quantization and dS in the kernel)"
                        if fuse_q else "sage_attn_fwd (pre-pass + dS + attention)")
                       + (", replayed from a CUDA graph" if args.graph else "")
-                      + "; prepass_ms = ms_per_step - attn_kernel_ms"),
+                      + ("; prepass_ms = ms_per_step - attn_kernel_ms" if fuse_q else
+                         "; prepass_ms: sage_quant_qk_gqa + sage_quant_v_gqa timed alone with CUDA events")),
         "attn_frac_of_spec_4500": attn_tops / SPEC_INT8_TOPS,
         "roofline": {"bound": "tensor", "achieved": attn_tops, "peak": peak, "unit": "TFLOP/s",
                      "frac": attn_tops / peak, "traffic": None if (pv16 or fp4 or fuse_q) else recorded_traffic(w.name),
