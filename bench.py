@@ -624,7 +624,8 @@ def main():
                        if fuse_q else "sage_attn_fwd (pre-pass + dS + attention)")
                       + (", replayed from a CUDA graph" if args.graph else "")
                       + ("; prepass_ms = ms_per_step - attn_kernel_ms" if fuse_q else
-                         "; prepass_ms: sage_quant_qk_gqa + sage_quant_v_gqa timed alone with CUDA events")),
+                         "; prepass_ms: sage_quant_qk_gqa + sage_quant_v_gqa timed alone with CUDA events (the "
+                         "step's pre-pass kernels, with the K and the V statistics in two launches instead of one)")),
         "attn_frac_of_spec_4500": attn_tops / SPEC_INT8_TOPS,
         "roofline": {"bound": "tensor", "achieved": attn_tops, "peak": peak, "unit": "TFLOP/s",
                      "frac": attn_tops / peak, "traffic": None if (pv16 or fp4 or fuse_q) else recorded_traffic(w.name),

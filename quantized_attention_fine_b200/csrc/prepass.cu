@@ -30,8 +30,33 @@ namespace sage {
 
 namespace {
 
+// VEC consecutive 16-bit elements (bf16 when BF16, else fp16) as fp32, exactly.
+template <int VEC, bool BF16>
+__device__ __forceinline__ void load_row_slice(const uint16_t *p, float (&x)[VEC]) {
+    uint32_t u[VEC / 2];
+    if constexpr (VEC == 4) {
+        const uint2 w = *reinterpret_cast<const uint2 *>(p);
+        u[0] = w.x;
+        u[1] = w.y;
+    } else {
+        u[0] = *reinterpret_cast<const uint32_t *>(p);
+    }
+#pragma unroll
+    for (int j = 0; j < VEC / 2; ++j) {
+        if constexpr (BF16) {
+            x[2 * j] = __uint_as_float(u[j] << 16);
+            x[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+        } else {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&u[j]));
+            x[2 * j] = f.x;
+            x[2 * j + 1] = f.y;
+        }
+    }
+}
+
+// The same with the type chosen at run time (bf16 when `bf16`, else fp16).
 template <int VEC>
-__device__ __forceinline__ void load_row_slice(const uint16_t *p, int bf16, float (&x)[VEC]) {
+__device__ __forceinline__ void load_row_slice_rt(const uint16_t *p, int bf16, float (&x)[VEC]) {
     if constexpr (VEC == 4) {
         const uint2 u = *reinterpret_cast<const uint2 *>(p);
         x[0] = h16_to_f32(u.x & 0xFFFFu, bf16);
@@ -230,7 +255,7 @@ __device__ __forceinline__ float group_amax(const float *wmax, int w0, int n) {
 }
 
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool BF16>
 __global__ void __launch_bounds__(256) kv_stats_kernel(const PrepassArgs a) {
     constexpr int VEC = D / 32;
     __shared__ double s_sum[8][D];
@@ -249,15 +274,36 @@ __global__ void __launch_bounds__(256) kv_stats_kernel(const PrepassArgs a) {
     for (int v = 0; v < VEC; ++v) { ks[v] = 0.0; vm[v] = 0.f; }
     const uint16_t *kp = a.k ? static_cast<const uint16_t *>(a.k) + base + lane * VEC : nullptr;
     const uint16_t *vp = a.v ? static_cast<const uint16_t *>(a.v) + base + lane * VEC : nullptr;
-    for (int j = j0 + warp; j < j1; j += 8) {
+    constexpr int U = 4;   // rows whose loads are issued before the first is used
+    int j = j0 + warp;
+    for (; j + 8 * (U - 1) < j1; j += 8 * U) {
+        float xk[U][VEC], xv[U][VEC];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (kp) load_row_slice<VEC, BF16>(kp + (int64_t)(j + 8 * u) * a.skv.n, xk[u]);
+            if (vp) load_row_slice<VEC, BF16>(vp + (int64_t)(j + 8 * u) * a.skv.n, xv[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (kp) {
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) ks[v] = __dadd_rn(ks[v], (double)xk[u][v]);
+            }
+            if (vp) {
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) vm[v] = fmaxf(vm[v], fabsf(xv[u][v]));
+            }
+        }
+    }
+    for (; j < j1; j += 8) {
         float x[VEC];
         if (kp) {
-            load_row_slice<VEC>(kp + (int64_t)j * a.skv.n, a.bf16, x);
+            load_row_slice<VEC, BF16>(kp + (int64_t)j * a.skv.n, x);
 #pragma unroll
             for (int v = 0; v < VEC; ++v) ks[v] = __dadd_rn(ks[v], (double)x[v]);
         }
         if (vp) {
-            load_row_slice<VEC>(vp + (int64_t)j * a.skv.n, a.bf16, x);
+            load_row_slice<VEC, BF16>(vp + (int64_t)j * a.skv.n, x);
 #pragma unroll
             for (int v = 0; v < VEC; ++v) vm[v] = fmaxf(vm[v], fabsf(x[v]));
         }
@@ -304,7 +350,7 @@ __global__ void kv_finalize_kernel(const PrepassArgs a) {
 // ---------------------------------------------------------------------------
 // FP4: the 4-bit mode (a separate instantiation, so that the INT8 kernel carries
 // none of its code).
-template <int D, bool FP4>
+template <int D, bool FP4, bool BF16>
 __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_constant__ PrepassArgs a) {
     constexpr int VEC = D / 32, RPW = kRowsPerWarp;
     __shared__ uint64_t s_full[QuantRing<D>::kStages];
@@ -345,7 +391,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
             const int r = warp * RPW + i;
-            load_row_slice<VEC>(tile + r * D, a.bf16, x[i]);
+            load_row_slice<VEC, BF16>(tile + r * D, x[i]);
             if (r < nvalid) {
 #pragma unroll
                 for (int v = 0; v < VEC; ++v) ps[v] = __dadd_rn(ps[v], (double)x[i][v]);
@@ -365,22 +411,35 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
             reinterpret_cast<float *>(a.ws + a.L.qbar)[((size_t)bh * S.Tq + t) * D + c] = qb;
         }
         __syncthreads();
-        float qb[VEC];
+        float2 nqb[VEC / 2];   // -qbar of this lane's channels: x + (-qbar) is x - qbar exactly
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) qb[v] = s_qbar[lane * VEC + v];
+        for (int v = 0; v < VEC; v += 2) nqb[v / 2] = make_float2(-s_qbar[lane * VEC + v], -s_qbar[lane * VEC + v + 1]);
         float am = 0.f;
-        float shift[RPW];  // this lane's part of Q_s . kbar for each of the warp's rows
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
-            const int r = warp * RPW + i;
-            shift[i] = 0.f;
 #pragma unroll
-            for (int v = 0; v < VEC; ++v) {
-                const float xs = (r < nvalid) ? __fsub_rn(x[i][v], qb[v]) : 0.f;
-                x[i][v] = xs;
-                am = fmaxf(am, fabsf(xs));
-                shift[i] = fmaf(xs, kb[v], shift[i]);
+            for (int v = 0; v < VEC; v += 2) {
+                const float2 xs = __fadd2_rn(make_float2(x[i][v], x[i][v + 1]), nqb[v / 2]);
+                x[i][v] = xs.x;
+                x[i][v + 1] = xs.y;
             }
+            if (warp * RPW + i >= nvalid) {   // rows past the sequence (warp-uniform)
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) x[i][v] = 0.f;
+            }
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) am = fmaxf(am, fabsf(x[i][v]));
+        }
+        // this lane's part of Q_s . kbar for each of the warp's rows, channel by channel
+        // (rows taken in pairs by the packed fma)
+        float shift[RPW];
+#pragma unroll
+        for (int i = 0; i < RPW; i += 2) {
+            float2 sh = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) sh = __ffma2_rn(make_float2(x[i][v], x[i + 1][v]), make_float2(kb[v], kb[v]), sh);
+            shift[i] = sh.x;
+            shift[i + 1] = sh.y;
         }
         static_assert(RPW == 16, "one shift value per row of the warp's 16");
         const float row_shift = warp_sum16_scatter(shift);  // row warp * RPW + (lane >> 1)
@@ -409,7 +468,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
 }
 
 // ---------------------------------------------------------------------------
-template <int D, bool FP4>
+template <int D, bool FP4, bool BF16>
 __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_constant__ PrepassArgs a) {
     constexpr int VEC = D / 32, RPW = kRowsPerWarp;
     __shared__ uint64_t s_full[QuantRing<D>::kStages];
@@ -425,9 +484,14 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_
         const int u = blockIdx.x + k * gridDim.x;
         if (u >= rc.n_units) break;
         const int bh = u / S.Tk, jt = u % S.Tk;
-        float kb[VEC];   // this unit's K mean, loaded before the tile is waited for
+        // minus this unit's K mean (x + (-kbar) is x - kbar exactly), loaded before the
+        // tile is waited for
+        float2 nkb[VEC / 2];
+        {
+            const float *kbar = reinterpret_cast<const float *>(a.ws + a.L.kbar) + (size_t)bh * D + lane * VEC;
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) kb[v] = reinterpret_cast<const float *>(a.ws + a.L.kbar)[(size_t)bh * D + lane * VEC + v];
+            for (int v = 0; v < VEC; v += 2) nkb[v / 2] = make_float2(-kbar[v], -kbar[v + 1]);
+        }
         const int j0 = jt * kTile, nvalid = min(kTile, seq_range(a.cu_kv, bh / S.H_kv, S.n_kv, S.total_kv).n - j0);
         if (!rc.wait(k, &s_abort, status)) break;
         if (nvalid <= 0) {  // a tile past the end of a shorter packed sequence
@@ -441,13 +505,19 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
             const int r = warp * RPW + i;
-            load_row_slice<VEC>(tile + r * D, a.bf16, x[i]);
+            load_row_slice<VEC, BF16>(tile + r * D, x[i]);
 #pragma unroll
-            for (int v = 0; v < VEC; ++v) {
-                const float xs = (r < nvalid) ? __fsub_rn(x[i][v], kb[v]) : 0.f;
-                x[i][v] = xs;
-                am = fmaxf(am, fabsf(xs));
+            for (int v = 0; v < VEC; v += 2) {
+                const float2 xs = __fadd2_rn(make_float2(x[i][v], x[i][v + 1]), nkb[v / 2]);
+                x[i][v] = xs.x;
+                x[i][v + 1] = xs.y;
             }
+            if (r >= nvalid) {   // keys past the sequence (warp-uniform)
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) x[i][v] = 0.f;
+            }
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) am = fmaxf(am, fabsf(x[i][v]));
         }
         am = warp_max(am);
         if (lane == 0) s_wmax[k & 1][warp] = am;
@@ -530,7 +600,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
             const int r = warp * RPW + i;
-            load_row_slice<VEC>(tile + r * D, a.bf16, x[i]);
+            load_row_slice_rt<VEC>(tile + r * D, a.bf16, x[i]);
             if (r >= nvalid) {
 #pragma unroll
                 for (int v = 0; v < VEC; ++v) x[i][v] = 0.f;
@@ -600,11 +670,11 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_
 }
 
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool BF16>
 static cudaError_t launch_prepass_d(const PrepassArgs &a, cudaStream_t stream) {
     const Shape &S = a.shape;
     if (a.k || a.v) {
-        kv_stats_kernel<D><<<(unsigned)((size_t)S.n_chunks * S.BH_kv), 256, 0, stream>>>(a);
+        kv_stats_kernel<D, BF16><<<(unsigned)((size_t)S.n_chunks * S.BH_kv), 256, 0, stream>>>(a);
         kv_finalize_kernel<D><<<S.BH_kv, D, 0, stream>>>(a);
     }
     // persistent grids: two CTAs per SM, or one per work unit if fewer
@@ -613,12 +683,12 @@ static cudaError_t launch_prepass_d(const PrepassArgs &a, cudaStream_t stream) {
     const size_t smem = QuantRing<D>::kSmemBytes;
     auto grid_of = [&](int units) { return (unsigned)(units < 2 * sms ? units : 2 * sms); };
     if (a.q) {
-        auto kq = a.fp4 ? quant_q_kernel<D, true> : quant_q_kernel<D, false>;
+        auto kq = a.fp4 ? quant_q_kernel<D, true, BF16> : quant_q_kernel<D, false, BF16>;
         cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         kq<<<grid_of(S.BH * S.Tq), kQuantThreads, smem, stream>>>(a);
     }
     if (a.k) {
-        auto kk = a.fp4 ? quant_k_kernel<D, true> : quant_k_kernel<D, false>;
+        auto kk = a.fp4 ? quant_k_kernel<D, true, BF16> : quant_k_kernel<D, false, BF16>;
         cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         kk<<<grid_of(S.BH_kv * S.Tk), kQuantThreads, smem, stream>>>(a);
     }
@@ -631,8 +701,8 @@ static cudaError_t launch_prepass_d(const PrepassArgs &a, cudaStream_t stream) {
 }
 
 cudaError_t launch_prepass(const PrepassArgs &a, cudaStream_t stream) {
-    if (a.shape.d == 128) return launch_prepass_d<128>(a, stream);
-    return launch_prepass_d<64>(a, stream);
+    if (a.shape.d == 128) return a.bf16 ? launch_prepass_d<128, true>(a, stream) : launch_prepass_d<128, false>(a, stream);
+    return a.bf16 ? launch_prepass_d<64, true>(a, stream) : launch_prepass_d<64, false>(a, stream);
 }
 
 }  // namespace sage

@@ -366,6 +366,18 @@ __device__ __forceinline__ float h16_to_f32(uint32_t bits, int bf16) {
     return bf16 ? __uint_as_float(bits << 16) : __half2float(__ushort_as_half((unsigned short)bits));
 }
 
+// INT8 codes of four values by IEEE division (round-half-even of x / delta), packed
+// little-endian: the near-tie path of int8_codes, kept out of line so that the common
+// path carries none of the division code.
+static __device__ __noinline__ uint32_t int8_codes4_div(float x0, float x1, float x2, float x3, float delta) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    const uint32_t m0 = __float_as_uint(__fdiv_rn(x0, delta) + kMagic);
+    const uint32_t m1 = __float_as_uint(__fdiv_rn(x1, delta) + kMagic);
+    const uint32_t m2 = __float_as_uint(__fdiv_rn(x2, delta) + kMagic);
+    const uint32_t m3 = __float_as_uint(__fdiv_rn(x3, delta) + kMagic);
+    return __byte_perm(__byte_perm(m0, m1, 0x0040), __byte_perm(m2, m3, 0x0040), 0x5410);
+}
+
 // INT8 codes of VEC values, round-half-even of the IEEE fp32 quotient xs / delta,
 // packed little-endian.
 // - For |xs / delta| <= 128, t = RN(xs * RN(1 / delta)) lies within 2.3e-5 of the
@@ -374,24 +386,32 @@ __device__ __forceinline__ float h16_to_f32(uint32_t bits, int bf16) {
 //   IEEE division.
 // - Rounding is done on the FMA pipe: m = RN(t + 1.5 * 2^23) holds round-half-even(t)
 //   in its low mantissa bits, so its low byte is the two's-complement code, and
-//   m - 1.5 * 2^23 is that integer exactly.
+//   m - 1.5 * 2^23 is that integer exactly (so t - it is exact too).
 // - delta = amax / 127 bounds |t| by 127 (1 + 3 * 2^-24) < 127.5, so the codes never
 //   leave [-127, 127] and the clamp of the definition never binds.
+// Pairs of values go through the packed fp32x2 operations (each lane rounds as the
+// scalar operation does).
 template <int VEC>
 __device__ __forceinline__ uint32_t int8_codes(const float (&xs)[VEC], float delta, float inv_delta) {
+    static_assert(VEC == 2 || VEC == 4, "two or four values");
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    const float2 inv2 = make_float2(inv_delta, inv_delta);
+    const float2 mg = make_float2(kMagic, kMagic), nmg = make_float2(-kMagic, -kMagic);
+    const float2 neg1 = make_float2(-1.f, -1.f);
     uint32_t m[4] = {0, 0, 0, 0};
-    bool near_tie = false;
+    float dev = 0.f;   // largest |t - round(t)|
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) {
-        const float t = xs[v] * inv_delta;
-        const float tm = t + kMagic;
-        near_tie |= fabsf(t - (tm - kMagic)) > 0.5f - 0x1p-15f;
-        m[v] = __float_as_uint(tm);
+    for (int v = 0; v < VEC; v += 2) {
+        const float2 t = __fmul2_rn(make_float2(xs[v], xs[v + 1]), inv2);
+        const float2 tm = __fadd2_rn(t, mg);
+        const float2 e = __ffma2_rn(__fadd2_rn(tm, nmg), neg1, t);
+        dev = fmaxf(dev, fmaxf(fabsf(e.x), fabsf(e.y)));
+        m[v] = __float_as_uint(tm.x);
+        m[v + 1] = __float_as_uint(tm.y);
     }
-    if (near_tie) {
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) m[v] = __float_as_uint(__fdiv_rn(xs[v], delta) + kMagic);
+    if (dev > 0.5f - 0x1p-15f) {
+        if constexpr (VEC == 4) return int8_codes4_div(xs[0], xs[1], xs[2], xs[3], delta);
+        return int8_codes4_div(xs[0], xs[1], 0.f, 0.f, delta) & 0xFFFFu;
     }
     const uint32_t lo = __byte_perm(m[0], m[1], 0x0040);
     if constexpr (VEC == 4) return __byte_perm(lo, __byte_perm(m[2], m[3], 0x0040), 0x5410);
