@@ -204,20 +204,6 @@ bool make_rows16_map(CUtensorMap *map, const void *x, int dtype, int layout, con
            CUDA_SUCCESS;
 }
 
-// Store map of the dS array [BH][Tq][nk_pad] fp32: 128-key x 32-block boxes, no
-// swizzle; rows past Tq are clipped by the copy engine.
-bool make_ds_map(CUtensorMap *map, float *ds, const Shape &s) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[3] = {(uint64_t)s.nk_pad, (uint64_t)s.Tq, (uint64_t)s.BH};
-    cuuint64_t strides[2] = {(uint64_t)s.nk_pad * 4, (uint64_t)s.Tq * s.nk_pad * 4};
-    cuuint32_t box[3] = {(cuuint32_t)kTile, 32, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ds, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
-}
-
 // Pre-pass of a dense batch (cu_q = cu_kv = null) or of a packed one (token-major
 // [total][heads][d] tensors, per-sequence offsets cu_q, cu_kv on the device).
 sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype, int layout, const Shape &s,
@@ -251,10 +237,10 @@ sage_status_t run_prepass(const void *q, const void *k, const void *v, int dtype
     a.L = ws_layout(s);
     if (launch_prepass(a, stream) != cudaSuccess) return SAGE_ERR_CUDA;
     if (k && m.smooth_q && ds_product) {
-        CUtensorMap tmk, tmds;
+        CUtensorMap tmk;
         if (!make_k16_map(&tmk, k, dtype, layout, s)) return SAGE_ERR_CUDA;
-        if (!make_ds_map(&tmds, reinterpret_cast<float *>(ws + a.L.ds), s)) return SAGE_ERR_CUDA;
-        if (launch_ds_gemm(tmk, tmds, reinterpret_cast<const float *>(ws + a.L.qbar), s, layout == SAGE_LAYOUT_NHD,
+        if (launch_ds_gemm(tmk, reinterpret_cast<float *>(ws + a.L.ds), reinterpret_cast<const float *>(ws + a.L.qbar), s,
+                           layout == SAGE_LAYOUT_NHD,
                            dtype == SAGE_DTYPE_BF16, ds_t_skip, causal_off, cu_q, cu_kv,
                            reinterpret_cast<int *>(ws + a.L.status), stream) != cudaSuccess)
             return SAGE_ERR_CUDA;

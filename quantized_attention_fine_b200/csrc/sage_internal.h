@@ -166,7 +166,7 @@ cudaError_t launch_prepass(const PrepassArgs &a, cudaStream_t stream);
 // j visible to query i iff j <= i + causal_off; for a packed batch the offset is each
 // sequence's n_kv - n_q and causal_off is unused).  cu_q, cu_kv: packed batch offsets
 // or null.
-cudaError_t launch_ds_gemm(const CUtensorMap &tm_k, const CUtensorMap &tm_ds, const float *qbar, const Shape &s,
+cudaError_t launch_ds_gemm(const CUtensorMap &tm_k, float *ds_out, const float *qbar, const Shape &s,
                            int nhd, int bf16, int causal_skip, int causal_off, const int *cu_q, const int *cu_kv,
                            int *status, cudaStream_t stream);
 // tq: Q codes, or with p.fused_q the caller's 16-bit Q (64-element x 128-row boxes,
