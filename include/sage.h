@@ -385,6 +385,23 @@ SAGE_API sage_status_t sage_debug_mma_rate(int kind, int n_iter, int n_ctas, voi
 SAGE_API sage_status_t sage_debug_quant_fp4(const float *xs, int n_rows, int d, uint8_t *codes, uint8_t *sf,
                                             float *g, void *stream);
 
+/* Check of the quotient routine of the quantizers (Markstein's correction of x * RN(1/delta),
+ * "Computation of elementary functions on the IBM RISC System/6000 processor", 1990),
+ * which stands for the IEEE fp32 division x / delta that the INT8 and E4M3 codes are
+ * defined on: for every finite 16-bit pattern x of dtype (SAGE_DTYPE_BF16 or
+ * SAGE_DTYPE_F16) and every deltas[j] >= 2^-60 (below that the quantizers divide)
+ * with |x| <= 448 deltas[j], the routine's results for x and for -x are compared with
+ * the division: bit for bit where the quotient is at least 2^-20; for every x as the
+ * E4M3 codes the V
+ * quantizer forms; and, where |x / deltas[j]| <= 127, as the INT8 codes the Q and K
+ * quantizers form.
+ *   deltas : device fp32 [n_delta], 1 <= n_delta <= 65535
+ *   count  : device uint64, incremented by the number of mismatches (zero it first)
+ *   first  : device uint32 [3], zeroed; on a mismatch {pattern, delta index, 1}
+ * Asynchronous on `stream`; SAGE_ERR_INVALID_ARG for null pointers or a bad count or dtype. */
+SAGE_API sage_status_t sage_debug_quotient_check(const float *deltas, int n_delta, int dtype, unsigned long long *count,
+                                                 unsigned int *first, void *stream);
+
 /* One 128 x 128 QK^T tile of the 4-bit mode on the block-scaled tensor core
  * (tcgen05.mma kind::mxf4nvf4, one E4M3 scale per 16 channels, scale factors copied
  * into tensor memory by tcgen05.cp):

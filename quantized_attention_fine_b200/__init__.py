@@ -32,7 +32,7 @@ import threading
 __all__ = [
     "QuantMode", "Workspace", "workspace_bytes", "make_workspace", "quant_qk", "quant_v", "attn_fwd_prequant",
     "attn_fwd", "attn_fwd_varlen", "SageAttention", "scaled_dot_product_attention", "QUANT_MODES", "get_device_status", "workspace_view", "debug_qk_tile", "debug_pv_accumulate",
-    "debug_fault_inject", "debug_pv_accumulate_f16acc", "debug_mma_rate", "debug_quant_fp4", "library_path", "load_library", "SageError", "GRANULARITIES",
+    "debug_fault_inject", "debug_pv_accumulate_f16acc", "debug_mma_rate", "debug_quant_fp4", "debug_quotient_check", "library_path", "load_library", "SageError", "GRANULARITIES",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -118,6 +118,7 @@ def load_library():
         lib.sage_debug_pv_accumulate_f16acc.argtypes = [P, P, I, I, P, P]
         lib.sage_debug_mma_rate.argtypes = [I, I, I, P, P]
         lib.sage_debug_quant_fp4.argtypes = [P, I, I, P, P, P, P]
+        lib.sage_debug_quotient_check.argtypes = [P, I, I, P, P, P]
         lib.sage_debug_qk_tile_fp4.argtypes = [P, P, P, P, I, P, P, P]
         lib.sage_debug_attn_fault_inject.argtypes = [P, I, I, I, I, I, I, I, I, P, S, P]
         lib.sage_attn_fwd_qfused_gqa.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, F, QM, P, S, P]
@@ -129,7 +130,7 @@ def load_library():
                    "sage_quant_qk_gqa", "sage_quant_v_gqa", "sage_attn_fwd_prequant_gqa", "sage_attn_fwd_gqa",
                    "sage_attn_fwd_varlen",
                    "sage_get_device_status", "sage_debug_qk_tile", "sage_debug_pv_accumulate",
-                   "sage_debug_pv_accumulate_f16acc", "sage_debug_mma_rate", "sage_debug_quant_fp4",
+                   "sage_debug_pv_accumulate_f16acc", "sage_debug_mma_rate", "sage_debug_quant_fp4", "sage_debug_quotient_check",
                    "sage_debug_qk_tile_fp4",
                    "sage_debug_attn_fault_inject", "sage_attn_fwd_qfused_gqa", "sage_attn_fwd_varlen_qfused",
                    "sage_debug_set_q_code_dump", "sage_debug_attn_fault_inject_qfused"):
@@ -578,6 +579,22 @@ def debug_quant_fp4(xs, stream=None):
     _check(load_library().sage_debug_quant_fp4(_ptr(xs), n, d, _ptr(codes), _ptr(sf), _ptr(g),
                                                _stream_handle(stream)), "sage_debug_quant_fp4")
     return codes, sf, g
+
+
+def debug_quotient_check(deltas, dtype, stream=None):
+    """Mismatches between the quantizers' quotient routine and the IEEE division over
+    every finite 16-bit pattern of `dtype` (torch.bfloat16 or torch.float16) and every
+    scale in `deltas` (device fp32).  Returns (count, first) with first = (pattern,
+    delta index) of one mismatch, or None."""
+    torch = _torch()
+    count = torch.zeros(1, dtype=torch.int64, device=deltas.device)
+    first = torch.zeros(3, dtype=torch.int32, device=deltas.device)
+    deltas = deltas.contiguous()
+    _check(load_library().sage_debug_quotient_check(_ptr(deltas), int(deltas.numel()), _dtype_code(torch.empty(0, dtype=dtype)),
+                                                    _ptr(count), _ptr(first), _stream_handle(stream)),
+           "sage_debug_quotient_check")
+    c, f = int(count.item()), first.tolist()
+    return c, ((f[0] & 0xFFFF, f[1]) if f[2] else None)
 
 
 def debug_qk_tile_fp4(q4, k4, sfq, sfk, stream=None):

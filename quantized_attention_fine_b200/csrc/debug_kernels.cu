@@ -106,6 +106,60 @@ __global__ void __launch_bounds__(256) debug_quant_fp4_kernel(const float *__res
     }
 }
 
+// The pre-pass quotient routines against the IEEE division: for every finite 16-bit
+// input pattern x (bf16 when `bf16`, else fp16) and every delta of the list with
+// |x| <= 448 delta (the range a quantization group presents: its amax over 448 or
+// 127), where the quantizers use the routines (delta >= kQuotientMinDelta):
+// - quotient2_rn(x), quotient2_rn(-x) against __fdiv_rn bit for bit where the quotient
+//   is at least 2^-20 (below, the quotient or the remainder may be subnormal);
+// - e4m3x4_codes_rn (the V codes) against the E4M3 codes of the divisions, for every x;
+// - int8_codes_rn (the Q and K codes) against round-half-even of the divisions, where
+//   |x / delta| <= 127.
+// Mismatches are counted in *count; the first one found is written to first[0..2]
+// (pattern, delta index, 1).
+__global__ void __launch_bounds__(256) debug_quotient_check_kernel(const float *__restrict__ deltas, int n_delta,
+                                                                   int bf16, unsigned long long *count,
+                                                                   unsigned int *first) {
+    const int j = blockIdx.y;   // delta index
+    const float delta = deltas[j];
+    if (!(delta >= kQuotientMinDelta) || !(delta < 0x1p+120f)) return;
+    const float y = 1.0f / delta;
+    unsigned long long bad = 0;
+    unsigned int bad_pat = 0;
+    for (uint32_t p = blockIdx.x * blockDim.x + threadIdx.x; p < 65536u; p += gridDim.x * blockDim.x) {
+        const float x = h16_to_f32(p, bf16);
+        if (!isfinite(x) || fabsf(x) > 448.0f * delta) continue;
+        const float2 y2 = make_float2(y, y), nd2 = make_float2(-delta, -delta);
+        const float2 q = quotient2_rn(make_float2(x, -x), y2, nd2);
+        const float ref = __fdiv_rn(x, delta), nref = __fdiv_rn(-x, delta);
+        bool same = e4m3x4_codes_rn(x, -x, -x, x, y2, nd2) == pack_e4m3x4(ref, nref, nref, ref);
+        if (fabsf(ref) >= 0x1p-20f)
+            same = same && __float_as_uint(q.x) == __float_as_uint(ref) && __float_as_uint(q.y) == __float_as_uint(nref);
+        if (fabsf(ref) <= 127.0f) {
+            const float xs[2] = {x, -x};
+            const uint32_t want = (uint32_t)(uint8_t)(int)rintf(ref) | ((uint32_t)(uint8_t)(int)rintf(nref) << 8);
+            same = same && int8_codes_rn<2>(xs, y2, nd2) == want;
+        }
+        if (!same) {
+            ++bad;
+            bad_pat = p;
+        }
+    }
+    if (bad) {
+        atomicAdd(count, bad);
+        if (atomicCAS(&first[2], 0u, 1u) == 0u) {
+            first[0] = bad_pat;
+            first[1] = (unsigned int)j;
+        }
+    }
+}
+
+cudaError_t launch_debug_quotient_check(const float *deltas, int n_delta, int bf16, unsigned long long *count,
+                                        unsigned int *first, cudaStream_t stream) {
+    debug_quotient_check_kernel<<<dim3(64, (unsigned)n_delta), 256, 0, stream>>>(deltas, n_delta, bf16, count, first);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_debug_quant_fp4(const float *xs, int n_rows, int d, uint8_t *codes, uint8_t *sf, float *g,
                                    cudaStream_t stream) {
     const int tiles = (n_rows + kTile - 1) / kTile;

@@ -18,8 +18,9 @@
 //                in the FP16 P / V mode V -> fp16 (round to nearest even), same layout.
 // Every code decision (INT8 rounding, E4M3 rounding) is made on the IEEE fp32
 // quotient x / delta, rounded to nearest even, so that it is reproducible on the
-// host.  The quotient is formed as x * (1 / delta) when that product provably
-// rounds to the same code, and by IEEE division otherwise (see fast_quotient_*).
+// host.  The quotient is formed without a division per element (quotient2_rn, by
+// Markstein's correction of x * RN(1 / delta)), and by IEEE division for groups whose
+// scale is below 2^-60.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -92,18 +93,6 @@ __device__ __forceinline__ float warp_sum16_scatter(float (&v)[16]) {
         }
     }
     return v[0] + __shfl_xor_sync(0xFFFFFFFFu, v[0], 1);
-}
-
-// The IEEE fp32 quotient x / delta as far as its E4M3 rounding is concerned.
-// t = RN(x * RN(1 / delta)) is within about 1.5 fp32 ulp of the correctly rounded
-// quotient; E4M3 rounds at bit 19 of the fp32 mantissa (normal range), so unless the
-// 20 low bits of t are within 4 of the tie pattern 0x80000 both round alike.  The
-// subnormal E4M3 range (|t| < 2^-6) and near-ties use the IEEE division.
-__device__ __forceinline__ float e4m3_quotient(float x, float delta, float inv_delta) {
-    const float t = x * inv_delta;
-    const int dist = (int)(__float_as_uint(t) & 0xFFFFFu) - 0x80000;
-    if (fabsf(t) < 0x1p-6f || (dist >= -4 && dist <= 4)) return __fdiv_rn(x, delta);
-    return t;
 }
 
 template <int VEC>
@@ -459,10 +448,18 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
         }
         const float dl = (gam == 0.f) ? 1.f : __fdiv_rn(gam, 127.f);
         if (lane < RPW) reinterpret_cast<float *>(a.ws + a.L.dq)[(size_t)bh * S.nq_pad + r0 + warp * RPW + lane] = dl;
-        const float inv = 1.0f / dl;
         int8_t *q8 = reinterpret_cast<int8_t *>(a.ws + a.L.q8) + ((size_t)bh * S.nq_pad + r0 + warp * RPW) * D + lane * VEC;
+        if (dl >= kQuotientMinDelta) {
+            const float y = 1.0f / dl;
+            const float2 y2 = make_float2(y, y), nd2 = make_float2(-dl, -dl);
 #pragma unroll
-        for (int i = 0; i < RPW; ++i) store_codes<VEC>(q8 + (size_t)i * D, int8_codes<VEC>(x[i], dl, inv));
+            for (int i = 0; i < RPW; ++i) store_codes<VEC>(q8 + (size_t)i * D, int8_codes_rn<VEC>(x[i], y2, nd2));
+        } else {   // a group of tiny values: IEEE divisions
+#pragma unroll
+            for (int i = 0; i < RPW; ++i)
+                store_codes<VEC>(q8 + (size_t)i * D, int8_codes4_div(x[i][0], x[i][1], VEC == 4 ? x[i][VEC - 2] : 0.f,
+                                                                     VEC == 4 ? x[i][VEC - 1] : 0.f, dl));
+        }
     }
     if (s_abort && threadIdx.x == 0) rc.drain(k);
 }
@@ -536,10 +533,18 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_k_kernel(const __grid_
         const float dl = (gam == 0.f) ? 1.f : __fdiv_rn(gam, 127.f);
         if (lane == 0)  // one delta_K per 16-key run = this warp's rows
             reinterpret_cast<float *>(a.ws + a.L.dk)[(size_t)bh * (S.nk_pad / kKeyRun) + (j0 + warp * RPW) / kKeyRun] = dl;
-        const float inv = 1.0f / dl;
         int8_t *k8 = reinterpret_cast<int8_t *>(a.ws + a.L.k8) + ((size_t)bh * S.nk_pad + j0 + warp * RPW) * D + lane * VEC;
+        if (dl >= kQuotientMinDelta) {
+            const float y = 1.0f / dl;
+            const float2 y2 = make_float2(y, y), nd2 = make_float2(-dl, -dl);
 #pragma unroll
-        for (int i = 0; i < RPW; ++i) store_codes<VEC>(k8 + (size_t)i * D, int8_codes<VEC>(x[i], dl, inv));
+            for (int i = 0; i < RPW; ++i) store_codes<VEC>(k8 + (size_t)i * D, int8_codes_rn<VEC>(x[i], y2, nd2));
+        } else {   // a group of tiny values: IEEE divisions
+#pragma unroll
+            for (int i = 0; i < RPW; ++i)
+                store_codes<VEC>(k8 + (size_t)i * D, int8_codes4_div(x[i][0], x[i][1], VEC == 4 ? x[i][VEC - 2] : 0.f,
+                                                                     VEC == 4 ? x[i][VEC - 1] : 0.f, dl));
+        }
     }
     if (s_abort && threadIdx.x == 0) rc.drain(k);
 }
@@ -635,16 +640,25 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_v_kernel(const __grid_
         uint8_t *vt8 = a.ws + a.L.vt8 + ((size_t)bh * D + lane * VEC) * S.nk_pad + j0 + warp * (RPW / 2);
 #pragma unroll
         for (int v = 0; v < VEC; ++v) {
-            const float inv = 1.0f / dv[v];
             uint32_t w[2][2];
+            if (dv[v] >= kQuotientMinDelta) {   // the E4M3 codes of the correctly rounded quotients
+                const float y = 1.0f / dv[v];
+                const float2 y2 = make_float2(y, y), nd2 = make_float2(-dv[v], -dv[v]);
 #pragma unroll
-            for (int par = 0; par < 2; ++par)
+                for (int par = 0; par < 2; ++par)
 #pragma unroll
-                for (int q = 0; q < 2; ++q)
-                    w[par][q] = pack_e4m3x4(e4m3_quotient(x[8 * q + par][v], dv[v], inv),
-                                            e4m3_quotient(x[8 * q + 2 + par][v], dv[v], inv),
-                                            e4m3_quotient(x[8 * q + 4 + par][v], dv[v], inv),
-                                            e4m3_quotient(x[8 * q + 6 + par][v], dv[v], inv));
+                    for (int q = 0; q < 2; ++q)
+                        w[par][q] = e4m3x4_codes_rn(x[8 * q + par][v], x[8 * q + 2 + par][v], x[8 * q + 4 + par][v],
+                                                    x[8 * q + 6 + par][v], y2, nd2);
+            } else {   // a channel of tiny values: IEEE divisions
+#pragma unroll
+                for (int par = 0; par < 2; ++par)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q)
+                        w[par][q] = pack_e4m3x4(__fdiv_rn(x[8 * q + par][v], dv[v]), __fdiv_rn(x[8 * q + 2 + par][v], dv[v]),
+                                                __fdiv_rn(x[8 * q + 4 + par][v], dv[v]),
+                                                __fdiv_rn(x[8 * q + 6 + par][v], dv[v]));
+            }
             if (staged) {
                 const uint32_t c = (uint32_t)(lane * VEC + v), half8 = 8u * (uint32_t)(warp & 1);
                 *reinterpret_cast<uint2 *>(vts + sw128_offset(c, (uint32_t)(warp >> 1)) + half8) =

@@ -674,6 +674,16 @@ sage_status_t sage_debug_mma_rate(int kind, int n_iter, int n_ctas, void *status
                : SAGE_ERR_CUDA;
 }
 
+sage_status_t sage_debug_quotient_check(const float *deltas, int n_delta, int dtype, unsigned long long *count,
+                                       unsigned int *first, void *stream) {
+    if (!deltas || !count || !first || n_delta < 1 || n_delta > 65535) return SAGE_ERR_INVALID_ARG;
+    if (dtype != SAGE_DTYPE_BF16 && dtype != SAGE_DTYPE_F16) return SAGE_ERR_INVALID_ARG;
+    return launch_debug_quotient_check(deltas, n_delta, dtype == SAGE_DTYPE_BF16 ? 1 : 0, count, first,
+                                       static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SAGE_OK
+               : SAGE_ERR_CUDA;
+}
+
 sage_status_t sage_debug_quant_fp4(const float *xs, int n_rows, int d, uint8_t *codes, uint8_t *sf, float *g,
                                    void *stream) {
     if (!xs || !codes || !sf || !g || n_rows < 1 || n_rows > (1 << 24)) return SAGE_ERR_INVALID_ARG;

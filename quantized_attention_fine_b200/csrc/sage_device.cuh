@@ -366,6 +366,61 @@ __device__ __forceinline__ float h16_to_f32(uint32_t bits, int bf16) {
     return bf16 ? __uint_as_float(bits << 16) : __half2float(__ushort_as_half((unsigned short)bits));
 }
 
+// Correctly rounded fp32 quotients x / delta of a pair of values, without a division
+// per value, by Markstein's theorem (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Develop. 34, 1990):
+// with y = RN(1 / delta) and q = RN(x y), which lies within an ulp of x / delta, the
+// remainder x - q delta is exact in one fma, and RN(q + (x - q delta) y) = RN(x / delta)
+// as long as nothing underflows.  Callers take this path only when delta >=
+// kQuotientMinDelta = 2^-60.  Then a quotient of at least 2^-20 has |x| >= 2^-80, so
+// that it and the remainder (about 2^-24 |x|) are normal numbers and the theorem
+// applies; a smaller quotient rounds to the code 0 (INT8 or E4M3) whether exact or as
+// computed here.  (x comes from the group whose amax sets delta, so x y cannot
+// overflow.)
+constexpr float kQuotientMinDelta = 0x1p-60f;
+__device__ __forceinline__ float2 quotient2_rn(float2 x, float2 y, float2 neg_delta) {
+    const float2 q = __fmul2_rn(x, y);
+    const float2 r = __ffma2_rn(q, neg_delta, x);
+    return __ffma2_rn(r, y, q);
+}
+
+// x's magnitude with s's sign bit.
+__device__ __forceinline__ float with_sign_of(float x, float s) {
+    return __uint_as_float((__float_as_uint(x) & 0x7FFFFFFFu) | (__float_as_uint(s) & 0x80000000u));
+}
+
+// Four E4M3 codes (byte i = value i; round to nearest even, saturating) of the
+// correctly rounded quotients x_i / delta for delta >= kQuotientMinDelta; y =
+// RN(1 / delta).  A quotient takes its dividend's sign: that changes nothing but the
+// quotient of -0, which the correction step turns into +0 (+0 + -0 rounds to +0),
+// while -0 / delta is -0, whose code is 0x80.
+__device__ __forceinline__ uint32_t e4m3x4_codes_rn(float x0, float x1, float x2, float x3, float2 y,
+                                                    float2 neg_delta) {
+    const float2 a = quotient2_rn(make_float2(x0, x1), y, neg_delta);
+    const float2 b = quotient2_rn(make_float2(x2, x3), y, neg_delta);
+    return pack_e4m3x4(with_sign_of(a.x, x0), with_sign_of(a.y, x1), with_sign_of(b.x, x2), with_sign_of(b.y, x3));
+}
+
+// INT8 codes (packed little-endian) of round-half-even(RN(x_v / delta)) for delta >=
+// kQuotientMinDelta: the quotients by quotient2_rn, rounded on the FMA pipe (RN(t +
+// 1.5 * 2^23) holds round-half-even(t) in its low mantissa byte, as a two's-complement
+// code).  y = RN(1 / delta); delta = amax / 127 keeps |t| below 127.5.
+template <int VEC>
+__device__ __forceinline__ uint32_t int8_codes_rn(const float (&xs)[VEC], float2 y, float2 neg_delta) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    const float2 mg = make_float2(kMagic, kMagic);
+    uint32_t m[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int v = 0; v < VEC; v += 2) {
+        const float2 t = __fadd2_rn(quotient2_rn(make_float2(xs[v], xs[v + 1]), y, neg_delta), mg);
+        m[v] = __float_as_uint(t.x);
+        m[v + 1] = __float_as_uint(t.y);
+    }
+    const uint32_t lo = __byte_perm(m[0], m[1], 0x0040);
+    if constexpr (VEC == 4) return __byte_perm(lo, __byte_perm(m[2], m[3], 0x0040), 0x5410);
+    return lo & 0xFFFFu;
+}
+
 // INT8 codes of four values by IEEE division (round-half-even of x / delta), packed
 // little-endian: the near-tie path of int8_codes, kept out of line so that the common
 // path carries none of the division code.

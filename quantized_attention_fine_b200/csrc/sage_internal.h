@@ -183,6 +183,8 @@ cudaError_t launch_debug_pv(const uint8_t *p, const uint8_t *vt, int n_tiles, in
 cudaError_t launch_debug_mma_rate(int kind, int n_iter, int n_ctas, int *status, cudaStream_t stream);
 // FP4 (E2M1) quantization of fp32 rows [n_rows][d] with two-level scales, per 128-row
 // tile; see sage_debug_quant_fp4.
+cudaError_t launch_debug_quotient_check(const float *deltas, int n_delta, int bf16, unsigned long long *count,
+                                        unsigned int *first, cudaStream_t stream);
 cudaError_t launch_debug_quant_fp4(const float *xs, int n_rows, int d, uint8_t *codes, uint8_t *sf, float *g,
                                    cudaStream_t stream);
 cudaError_t launch_zero_output(void *o, size_t bytes, cudaStream_t stream);

@@ -157,6 +157,9 @@ def test_argument_errors_return_synchronously(lib):
     # diagnostics validate their indices
     assert lib.sage_debug_qk_tile(fake, 1, 1, 128, 128, 64, 1, 0, 0, fake, None) == 1
     assert lib.sage_debug_pv_accumulate(fake, fake, 0, 64, fake, None) == 1
+    assert lib.sage_debug_quotient_check(fake, 0, 1, fake, fake, None) == 1
+    assert lib.sage_debug_quotient_check(fake, 4, 7, fake, fake, None) == 1
+    assert lib.sage_debug_quotient_check(None, 4, 1, fake, fake, None) == 1
 
 
 def test_noalloc_argument_errors_come_before_any_cuda_call(lib):

@@ -87,6 +87,38 @@ def test_prepass_bit_exact(B, H, nq, nk, d, dtype, layout, gran):
             assert np.max(np.abs(diff - diff[:, :1])) < 1e-9
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_prepass_bit_exact_signed_zeros_and_tiny_scales(d):
+    """Negative zeros in V (E4M3 code 0x80, as -0 / delta is -0) and groups and channels
+    whose scale is below 2^-60, where the quantizers divide instead of correcting the
+    product with the reciprocal: codes and scales still bit-exact against the oracle."""
+    g = torch.Generator().manual_seed(77 + d)
+    nq, nk = 130, 200
+    q = torch.randn(1, 1, nq, d, generator=g)
+    k = torch.randn(1, 1, nk, d, generator=g)
+    v = torch.randn(1, 1, nk, d, generator=g)
+    v[0, 0, ::3, 5] = -0.0                                         # negative zeros among ordinary values
+    v[0, 0, :, 7] = torch.randn(nk, generator=g) * 2.0 ** -75     # a channel of tiny values (delta_V < 2^-60)
+    v[0, 0, :, 9] = -0.0                                           # a channel of negative zeros only
+    q[0, 0, :128] *= 2.0 ** -70                                    # a 128-row block of tiny rows (delta_Q < 2^-60)
+    k *= 2.0 ** -70                                                # tiny keys: every K group below 2^-60
+    q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
+    assert (v[0, 0, :, 9].view(torch.int16) == -32768).all()
+    ws = sage.quant_qk(q.cuda(), k.cuda())
+    sage.quant_v(v.cuda(), n_q=nq, workspace=ws)
+    torch.cuda.synchronize()
+    pre = oracle.prepass_head(to_np64(q[0, 0]), to_np64(k[0, 0]), to_np64(v[0, 0]))
+    assert (pre["v_code"][:, 9] == 0x80).all() and (pre["v_code"][::3, 5] == 0x80).all()
+    assert pre["dv"][7] < 2.0 ** -60 and pre["dv"][9] == 1.0
+    assert pre["dq_row"][:128].max() < 2.0 ** -60 < pre["dq_row"][128:nq].min() and pre["dk_key"][:nk].max() < 2.0 ** -60
+    for name, ref in (("dq", pre["dq_row"]), ("dk", pre["dk_key"][::16]), ("dv", pre["dv"]), ("q8", pre["q_code"]),
+                      ("k8", pre["k_code"])):
+        got = ws.view(name)[0].cpu().numpy()
+        assert np.array_equal(got[:len(ref)] if name in ("dq", "q8", "k8") else got, ref), name
+    vt = natural_key_order(ws.view("vt8")[0].cpu().numpy())
+    assert np.array_equal(vt[:, :nk].T, pre["v_code"]), "V codes"
+
+
 # ---------------------------------------------------------------------------
 # Tensor-core stages
 # ---------------------------------------------------------------------------
