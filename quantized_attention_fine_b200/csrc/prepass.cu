@@ -395,7 +395,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_q_kernel(const __grid_
             double sum = 0.0;
 #pragma unroll
             for (int w = 0; w < kQuantWarps; ++w) sum = __dadd_rn(sum, s_sum[w][c]);
-            const float qb = a.smooth_q ? (float)__ddiv_rn(sum, (double)nvalid) : 0.f;
+            // a full tile divides by 128, which the product with 2^-7 does exactly
+            const double mean = (nvalid == kTile) ? sum * (1.0 / kTile) : __ddiv_rn(sum, (double)nvalid);
+            const float qb = a.smooth_q ? (float)mean : 0.f;
             s_qbar[c] = qb;
             reinterpret_cast<float *>(a.ws + a.L.qbar)[((size_t)bh * S.Tq + t) * D + c] = qb;
         }
